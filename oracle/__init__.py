@@ -1,0 +1,197 @@
+"""fp64 CPU oracle for DiffQKV attention -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product path (the CUDA library and
+its Python binding in ``asymmetric_head_kv_b200``) never imports, links or
+executes anything here, and this package imports nothing from it.
+
+The arithmetic lives in ``oracle.c`` (plain C, fp64) and follows "Sigma:
+Differential Rescaling of Query, Key and Value for Efficient Language Models"
+(structured summary page), section 3.4 "DiffQKV Attention: Generalized
+Formulation" Steps 2-5, "Selective V Cache Fetching", and "FlexHeadFA Kernel
+and Deployment Infrastructure".  This module only marshals arrays.
+
+Inputs are bf16 tensors (torch) or uint16 arrays holding bf16 bit patterns.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from fractions import Fraction
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.c into liboracle.so with gcc (no CUDA)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-pthread", "-o", tmp, _SRC, "-lm"]
+        )
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    lib = ctypes.CDLL(build())
+    c_i, c_d, c_p, c_i64 = ctypes.c_int, ctypes.c_double, ctypes.c_void_p, ctypes.c_int64
+    lib.oracle_head_map.argtypes = [c_i, c_i, c_i]
+    lib.oracle_head_map.restype = c_i
+    lib.oracle_decode.argtypes = [c_i] * 6 + [c_d] + [c_p] * 4 + [c_i, c_i, c_p, c_i64, c_p, c_i]
+    lib.oracle_decode.restype = c_i
+    lib.oracle_prefill_causal.argtypes = [c_i] * 7 + [c_d] + [c_p] * 4 + [c_i64, c_p, c_i]
+    lib.oracle_prefill_causal.restype = c_i
+    lib.oracle_exact_dot.argtypes = [c_p, c_p, c_i, c_p, ctypes.POINTER(c_i)]
+    lib.oracle_exact_dot.restype = c_i
+    lib.oracle_decode_topv.argtypes = (
+        [c_i] * 6 + [c_d] + [c_p] * 4 + [c_i, c_i, c_p, c_i64, c_p, c_p, c_i]
+    )
+    lib.oracle_decode_topv.restype = c_i
+    _lib = lib
+    return lib
+
+
+def _bits(x) -> np.ndarray:
+    """bf16 tensor / uint16 array -> C-contiguous uint16 numpy view of the bits."""
+    try:
+        import torch
+
+        if isinstance(x, torch.Tensor):
+            if x.dtype != torch.bfloat16:
+                raise TypeError(f"expected bfloat16, got {x.dtype}")
+            x = x.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+    except ImportError:  # pragma: no cover
+        pass
+    x = np.ascontiguousarray(x)
+    if x.dtype != np.uint16:
+        raise TypeError(f"expected bf16 bit patterns (uint16), got {x.dtype}")
+    return x
+
+
+def _i32(x) -> np.ndarray:
+    try:
+        import torch
+
+        if isinstance(x, torch.Tensor):
+            x = x.detach().cpu().numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    return np.ascontiguousarray(np.asarray(x, dtype=np.int32))
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _check(rc: int, what: str):
+    if rc < 0:
+        raise RuntimeError(f"oracle {what} failed with status {rc}")
+
+
+def head_map(n_q: int, n_kv: int, h: int) -> int:
+    """GroupSharing: query head h reads K/V head floor(h * n_kv / n_q)."""
+    r = _load().oracle_head_map(n_q, n_kv, h)
+    if r < 0:
+        raise ValueError("bad head-map arguments")
+    return r
+
+
+def decode(q, k_cache, v_cache, seq_lens, scale: float, *, num_splits: int = 0,
+           rows=None, threads: int = 0) -> np.ndarray:
+    """fp64 decode attention.
+
+    q [B, n_q, d_k], k_cache [B, t_max, n_k, d_k], v_cache [B, t_max, n_v, d_v]
+    (bf16), seq_lens [B].  ``num_splits`` > 0 runs the split/combine form.
+    Returns [B, n_q, d_v] float64, or [len(rows), d_v] for ``rows`` = (b, h) pairs.
+    """
+    qb, kb, vb = _bits(q), _bits(k_cache), _bits(v_cache)
+    B, n_q, d_k = qb.shape
+    _, t_max, n_k, d_k2 = kb.shape
+    _, t_max2, n_v, d_v = vb.shape
+    assert d_k == d_k2 and t_max == t_max2 and kb.shape[0] == B and vb.shape[0] == B
+    sl = _i32(seq_lens)
+    assert sl.shape == (B,)
+    if rows is None:
+        out = np.empty((B * n_q, d_v), np.float64)
+        rp, nr = None, B * n_q
+    else:
+        rr = _i32(rows).reshape(-1, 2)
+        out = np.empty((rr.shape[0], d_v), np.float64)
+        rp, nr = _ptr(rr), rr.shape[0]
+    rc = _load().oracle_decode(B, n_q, n_k, n_v, d_k, d_v, float(scale), _ptr(qb), _ptr(kb), _ptr(vb),
+                               _ptr(sl), t_max, num_splits, rp, nr, _ptr(out), threads)
+    _check(rc, "decode")
+    return out.reshape(B, n_q, d_v) if rows is None else out
+
+
+def prefill_causal(q, k, v, scale: float, *, rows=None, threads: int = 0) -> np.ndarray:
+    """fp64 causal prefill.
+
+    q [B, S, n_q, d_k], k [B, S, n_k, d_k], v [B, S, n_v, d_v] (bf16).
+    Returns [B, S, n_q, d_v] float64, or [len(rows), d_v] for ``rows`` = (b, i, h).
+    """
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    B, S, n_q, d_k = qb.shape
+    n_k, n_v, d_v = kb.shape[2], vb.shape[2], vb.shape[3]
+    assert kb.shape == (B, S, n_k, d_k) and vb.shape[:2] == (B, S)
+    if rows is None:
+        out = np.empty((B * S * n_q, d_v), np.float64)
+        rp, nr = None, B * S * n_q
+    else:
+        rr = _i32(rows).reshape(-1, 3)
+        out = np.empty((rr.shape[0], d_v), np.float64)
+        rp, nr = _ptr(rr), rr.shape[0]
+    rc = _load().oracle_prefill_causal(B, S, n_q, n_k, n_v, d_k, d_v, float(scale), _ptr(qb), _ptr(kb),
+                                       _ptr(vb), rp, nr, _ptr(out), threads)
+    _check(rc, "prefill_causal")
+    return out.reshape(B, S, n_q, d_v) if rows is None else out
+
+
+def exact_dot(a, b) -> Fraction:
+    """Exact value of sum_i a_i * b_i for bf16 vectors, as a Fraction."""
+    ab, bb = _bits(a).reshape(-1), _bits(b).reshape(-1)
+    assert ab.shape == bb.shape
+    digits = np.zeros(32, np.int64)
+    lsb = ctypes.c_int(0)
+    nd = _load().oracle_exact_dot(_ptr(ab), _ptr(bb), ab.shape[0], _ptr(digits), ctypes.byref(lsb))
+    _check(nd, "exact_dot")
+    total = sum(int(digits[i]) << (32 * i) for i in range(nd))
+    return Fraction(total, 1) * Fraction(2) ** lsb.value
+
+
+def decode_topv(q, k_cache, v_cache, seq_lens, topk: int, scale: float, *, rows=None,
+                threads: int = 0):
+    """fp64 selective-V decode over the top-k exact-scoring positions per query head.
+
+    Returns (out float64 [B, n_q, d_v], idx int32 [B, n_q, topk]) -- idx ascending,
+    padded with -1 when topk exceeds the context -- or row-major [len(rows), ...].
+    """
+    qb, kb, vb = _bits(q), _bits(k_cache), _bits(v_cache)
+    B, n_q, d_k = qb.shape
+    _, t_max, n_k, _ = kb.shape
+    _, _, n_v, d_v = vb.shape
+    sl = _i32(seq_lens)
+    if rows is None:
+        nr, rp = B * n_q, None
+    else:
+        rr = _i32(rows).reshape(-1, 2)
+        nr, rp = rr.shape[0], _ptr(rr)
+    out = np.empty((nr, d_v), np.float64)
+    idx = np.empty((nr, max(topk, 0)), np.int32)
+    rc = _load().oracle_decode_topv(B, n_q, n_k, n_v, d_k, d_v, float(scale), _ptr(qb), _ptr(kb),
+                                    _ptr(vb), _ptr(sl), t_max, topk, rp, nr, _ptr(out), _ptr(idx),
+                                    threads)
+    _check(rc, "decode_topv")
+    if rows is None:
+        return out.reshape(B, n_q, d_v), idx.reshape(B, n_q, max(topk, 0))
+    return out, idx

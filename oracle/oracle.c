@@ -1,0 +1,489 @@
+/*
+ * oracle.c -- plain, slow, fp64 CPU oracle for DiffQKV attention.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may call, link or
+ * load this file; only tests/, the smoke check and the CPU-baseline leg of
+ * the benchmark do.  It shares no code, header, table or helper with the
+ * CUDA library under asymmetric_head_kv_b200/.
+ *
+ * What it computes (source: "Sigma: Differential Rescaling of Query, Key and
+ * Value for Efficient Language Models", structured summary page, section 3.4
+ * "DiffQKV Attention: Generalized Formulation", Steps 2-5; "Selective V Cache
+ * Fetching"; "FlexHeadFA Kernel and Deployment Infrastructure"):
+ *
+ *   head map     idx_i = floor(idx_q * n_i / n_q), i in {k, v}     (Step 3)
+ *   scores       s_j   = scale * <q_h, K[j, idx_k]>                 (Step 4)
+ *   weights      alpha = softmax_j(s)                               (Step 4)
+ *   output       o_h   = sum_j alpha_j V[j, idx_v]                  (Step 5)
+ *   split/combine   per KV chunk: (max, sum of exp, unnormalised o); the
+ *                combine pass rescales each chunk by exp(m_c - M)   (FlexHeadFA)
+ *   selective V  o_h  ~= sum over the top-k positions of the weights,
+ *                renormalised over that set                         (Selective V)
+ *
+ * All arithmetic is fp64.  bf16 inputs arrive as raw 16-bit patterns and are
+ * widened exactly.  The top-k selection ranks positions by the EXACT dot
+ * product (a fixed-point superaccumulator, every bf16 x bf16 product is an
+ * integer times a power of two), ties broken toward the lower position.
+ *
+ * Status codes: 0 ok, -1 bad argument, -2 non-finite bf16 input where an
+ * exact key is needed, -3 out of memory.
+ *
+ * Parity pins: every function here is pinned by tests in tests/test_oracle_*.py
+ * (closed forms, library SDPA in fp64, brute force, Fraction arithmetic).
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#include <unistd.h>
+
+/* ------------------------------------------------------------------ */
+/* bf16 widening                                                       */
+/* ------------------------------------------------------------------ */
+
+/* bf16 is the upper half of an IEEE binary32 pattern: widening is exact. */
+static double bf16_to_f64(uint16_t bits) {
+    uint32_t u = ((uint32_t)bits) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* ------------------------------------------------------------------ */
+/* GroupSharing head map (section 3.4, Step 3; FlexHeadFA address calc) */
+/* ------------------------------------------------------------------ */
+
+/* Query head h reads K (or V) head floor(h * n_kv / n_q). */
+int oracle_head_map(int n_q, int n_kv, int h) {
+    if (n_q <= 0 || n_kv <= 0 || h < 0 || h >= n_q) return -1;
+    return (int)(((int64_t)h * n_kv) / n_q);
+}
+
+/* ------------------------------------------------------------------ */
+/* simple pthread fan-out over independent rows                        */
+/* ------------------------------------------------------------------ */
+
+typedef void (*row_fn)(void *ctx, int64_t row);
+
+typedef struct {
+    row_fn fn;
+    void *ctx;
+    int64_t n_rows;
+    int64_t next;
+    pthread_mutex_t lock;
+} pool_t;
+
+static void *pool_worker(void *arg) {
+    pool_t *p = (pool_t *)arg;
+    for (;;) {
+        pthread_mutex_lock(&p->lock);
+        int64_t r = p->next++;
+        pthread_mutex_unlock(&p->lock);
+        if (r >= p->n_rows) break;
+        p->fn(p->ctx, r);
+    }
+    return NULL;
+}
+
+static void run_rows(row_fn fn, void *ctx, int64_t n_rows, int n_threads) {
+    if (n_threads <= 0) n_threads = (int)sysconf(_SC_NPROCESSORS_ONLN);
+    if (n_threads < 1) n_threads = 1;
+    if (n_threads > 256) n_threads = 256;
+    if ((int64_t)n_threads > n_rows) n_threads = (int)(n_rows > 0 ? n_rows : 1);
+    pool_t p;
+    p.fn = fn;
+    p.ctx = ctx;
+    p.n_rows = n_rows;
+    p.next = 0;
+    pthread_mutex_init(&p.lock, NULL);
+    if (n_threads == 1) {
+        pool_worker(&p);
+    } else {
+        pthread_t th[256];
+        int started = 0;
+        for (int i = 0; i < n_threads; ++i) {
+            if (pthread_create(&th[i], NULL, pool_worker, &p) != 0) break;
+            ++started;
+        }
+        if (started == 0) pool_worker(&p);
+        for (int i = 0; i < started; ++i) pthread_join(th[i], NULL);
+    }
+    pthread_mutex_destroy(&p.lock);
+}
+
+/* ------------------------------------------------------------------ */
+/* Decode over a KV cache (section 3.4, Steps 2-5)                     */
+/* ------------------------------------------------------------------ */
+
+typedef struct {
+    int batch, n_q, n_k, n_v, d_k, d_v, t_max;
+    double scale;
+    int num_splits;            /* 0: plain two-pass softmax; >0: split/combine */
+    const uint16_t *q;         /* [B, n_q, d_k]        */
+    const uint16_t *k;         /* [B, t_max, n_k, d_k] */
+    const uint16_t *v;         /* [B, t_max, n_v, d_v] */
+    const int32_t *seq_lens;   /* [B]                  */
+    const int32_t *rows;       /* n_rows pairs (b, h), or NULL for all */
+    double *out;               /* [n_rows, d_v]        */
+    int status;
+} decode_ctx;
+
+/* s_j = scale * sum_c q[c] * K[b, j, kh, c], for 0 <= j < T */
+static void decode_scores(const decode_ctx *c, int b, int h, int T, double *s) {
+    const int kh = oracle_head_map(c->n_q, c->n_k, h);
+    const uint16_t *q = c->q + ((int64_t)b * c->n_q + h) * c->d_k;
+    for (int j = 0; j < T; ++j) {
+        const uint16_t *kr = c->k + (((int64_t)b * c->t_max + j) * c->n_k + kh) * c->d_k;
+        double acc = 0.0;
+        for (int e = 0; e < c->d_k; ++e) acc += bf16_to_f64(q[e]) * bf16_to_f64(kr[e]);
+        s[j] = c->scale * acc;
+    }
+}
+
+static const uint16_t *v_row(const decode_ctx *c, int b, int j, int vh) {
+    return c->v + (((int64_t)b * c->t_max + j) * c->n_v + vh) * c->d_v;
+}
+
+static void decode_row(void *vctx, int64_t r) {
+    decode_ctx *c = (decode_ctx *)vctx;
+    int b, h;
+    if (c->rows) { b = c->rows[2 * r]; h = c->rows[2 * r + 1]; }
+    else { b = (int)(r / c->n_q); h = (int)(r % c->n_q); }
+    double *o = c->out + r * c->d_v;
+    for (int e = 0; e < c->d_v; ++e) o[e] = 0.0;
+    int T = c->seq_lens[b];
+    if (T > c->t_max) T = c->t_max;
+    if (T <= 0) return; /* empty context: the output row is zero */
+    const int vh = oracle_head_map(c->n_q, c->n_v, h);
+    double *s = (double *)malloc(sizeof(double) * (size_t)T);
+    if (!s) { c->status = -3; return; }
+    decode_scores(c, b, h, T, s);
+
+    if (c->num_splits <= 0) {
+        /* two-pass full softmax: m = max s; w = exp(s - m); o = sum w V / sum w */
+        double m = -INFINITY;
+        for (int j = 0; j < T; ++j) if (s[j] > m) m = s[j];
+        double den = 0.0;
+        for (int j = 0; j < T; ++j) {
+            const double w = exp(s[j] - m);
+            den += w;
+            const uint16_t *vr = v_row(c, b, j, vh);
+            for (int e = 0; e < c->d_v; ++e) o[e] += w * bf16_to_f64(vr[e]);
+        }
+        for (int e = 0; e < c->d_v; ++e) o[e] /= den;
+    } else {
+        /* split/combine: chunk i covers [i*L, min(T, (i+1)*L)), L = ceil(T/splits).
+         * Each chunk keeps (m_i, l_i, o_i) with o_i unnormalised; the combine
+         * pass merges them with weights exp(m_i - M), M = max_i m_i. */
+        const int ns = c->num_splits;
+        const int L = (T + ns - 1) / ns;
+        double *mi = (double *)malloc(sizeof(double) * (size_t)ns);
+        double *li = (double *)malloc(sizeof(double) * (size_t)ns);
+        double *oi = (double *)calloc((size_t)ns * (size_t)c->d_v, sizeof(double));
+        int *used = (int *)calloc((size_t)ns, sizeof(int));
+        if (!mi || !li || !oi || !used) { c->status = -3; free(mi); free(li); free(oi); free(used); free(s); return; }
+        for (int i = 0; i < ns; ++i) {
+            const int j0 = i * L, j1 = (j0 + L < T) ? j0 + L : T;
+            if (j0 >= j1) continue;
+            used[i] = 1;
+            double m = -INFINITY;
+            for (int j = j0; j < j1; ++j) if (s[j] > m) m = s[j];
+            double l = 0.0;
+            for (int j = j0; j < j1; ++j) {
+                const double w = exp(s[j] - m);
+                l += w;
+                const uint16_t *vr = v_row(c, b, j, vh);
+                for (int e = 0; e < c->d_v; ++e) oi[(int64_t)i * c->d_v + e] += w * bf16_to_f64(vr[e]);
+            }
+            mi[i] = m;
+            li[i] = l;
+        }
+        double M = -INFINITY;
+        for (int i = 0; i < ns; ++i) if (used[i] && mi[i] > M) M = mi[i];
+        double den = 0.0;
+        for (int i = 0; i < ns; ++i) {
+            if (!used[i]) continue;
+            const double f = exp(mi[i] - M);
+            den += f * li[i];
+            for (int e = 0; e < c->d_v; ++e) o[e] += f * oi[(int64_t)i * c->d_v + e];
+        }
+        for (int e = 0; e < c->d_v; ++e) o[e] /= den;
+        free(mi); free(li); free(oi); free(used);
+    }
+    free(s);
+}
+
+static int check_dims(int batch, int n_q, int n_k, int n_v, int d_k, int d_v) {
+    if (batch < 0 || n_q <= 0 || n_k <= 0 || n_v <= 0 || d_k <= 0 || d_v <= 0) return -1;
+    if (n_k > n_q || n_v > n_q) return -1;
+    return 0;
+}
+
+/* Decode for n_rows (b, h) pairs (rows == NULL: all B*n_q rows in order).
+ * out: fp64 [n_rows, d_v]. */
+int oracle_decode(int batch, int n_q, int n_k, int n_v, int d_k, int d_v, double scale,
+                  const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
+                  const int32_t *seq_lens, int t_max, int num_splits,
+                  const int32_t *rows, int64_t n_rows, double *out, int n_threads) {
+    if (check_dims(batch, n_q, n_k, n_v, d_k, d_v) || t_max < 0 || !q || !k_cache || !v_cache ||
+        !seq_lens || !out)
+        return -1;
+    if (!rows) n_rows = (int64_t)batch * n_q;
+    for (int64_t r = 0; rows && r < n_rows; ++r)
+        if (rows[2 * r] < 0 || rows[2 * r] >= batch || rows[2 * r + 1] < 0 || rows[2 * r + 1] >= n_q)
+            return -1;
+    decode_ctx c = {batch, n_q, n_k, n_v, d_k, d_v, t_max, scale, num_splits,
+                    q, k_cache, v_cache, seq_lens, rows, out, 0};
+    run_rows(decode_row, &c, n_rows, n_threads);
+    return c.status;
+}
+
+/* ------------------------------------------------------------------ */
+/* Causal prefill: row i attends to positions j <= i (same arithmetic) */
+/* ------------------------------------------------------------------ */
+
+typedef struct {
+    int batch, seq, n_q, n_k, n_v, d_k, d_v;
+    double scale;
+    const uint16_t *q;   /* [B, S, n_q, d_k] */
+    const uint16_t *k;   /* [B, S, n_k, d_k] */
+    const uint16_t *v;   /* [B, S, n_v, d_v] */
+    const int32_t *rows; /* n_rows triples (b, i, h), or NULL for all */
+    double *out;         /* [n_rows, d_v] */
+    int status;
+} prefill_ctx;
+
+static void prefill_row(void *vctx, int64_t r) {
+    prefill_ctx *c = (prefill_ctx *)vctx;
+    int b, i, h;
+    if (c->rows) { b = c->rows[3 * r]; i = c->rows[3 * r + 1]; h = c->rows[3 * r + 2]; }
+    else {
+        b = (int)(r / ((int64_t)c->seq * c->n_q));
+        const int64_t rem = r % ((int64_t)c->seq * c->n_q);
+        i = (int)(rem / c->n_q);
+        h = (int)(rem % c->n_q);
+    }
+    const int kh = oracle_head_map(c->n_q, c->n_k, h);
+    const int vh = oracle_head_map(c->n_q, c->n_v, h);
+    const int T = i + 1;
+    double *o = c->out + r * c->d_v;
+    for (int e = 0; e < c->d_v; ++e) o[e] = 0.0;
+    double *s = (double *)malloc(sizeof(double) * (size_t)T);
+    if (!s) { c->status = -3; return; }
+    const uint16_t *qr = c->q + (((int64_t)b * c->seq + i) * c->n_q + h) * c->d_k;
+    double m = -INFINITY;
+    for (int j = 0; j < T; ++j) {
+        const uint16_t *kr = c->k + (((int64_t)b * c->seq + j) * c->n_k + kh) * c->d_k;
+        double acc = 0.0;
+        for (int e = 0; e < c->d_k; ++e) acc += bf16_to_f64(qr[e]) * bf16_to_f64(kr[e]);
+        s[j] = c->scale * acc;
+        if (s[j] > m) m = s[j];
+    }
+    double den = 0.0;
+    for (int j = 0; j < T; ++j) {
+        const double w = exp(s[j] - m);
+        den += w;
+        const uint16_t *vr = c->v + (((int64_t)b * c->seq + j) * c->n_v + vh) * c->d_v;
+        for (int e = 0; e < c->d_v; ++e) o[e] += w * bf16_to_f64(vr[e]);
+    }
+    for (int e = 0; e < c->d_v; ++e) o[e] /= den;
+    free(s);
+}
+
+int oracle_prefill_causal(int batch, int seq, int n_q, int n_k, int n_v, int d_k, int d_v,
+                          double scale, const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                          const int32_t *rows, int64_t n_rows, double *out, int n_threads) {
+    if (check_dims(batch, n_q, n_k, n_v, d_k, d_v) || seq < 0 || !q || !k || !v || !out) return -1;
+    if (!rows) n_rows = (int64_t)batch * seq * n_q;
+    for (int64_t r = 0; rows && r < n_rows; ++r)
+        if (rows[3 * r] < 0 || rows[3 * r] >= batch || rows[3 * r + 1] < 0 || rows[3 * r + 1] >= seq ||
+            rows[3 * r + 2] < 0 || rows[3 * r + 2] >= n_q)
+            return -1;
+    prefill_ctx c = {batch, seq, n_q, n_k, n_v, d_k, d_v, scale, q, k, v, rows, out, 0};
+    run_rows(prefill_row, &c, n_rows, n_threads);
+    return c.status;
+}
+
+/* ------------------------------------------------------------------ */
+/* Exact dot products of bf16 vectors (fixed-point superaccumulator)   */
+/* ------------------------------------------------------------------ */
+/*
+ * A finite bf16 value is M * 2^x with integer 0 <= M < 256:
+ *   exponent field E = 0  (zero/subnormal): M = mantissa,       x = -133
+ *   1 <= E <= 254         (normal):         M = 128 + mantissa, x = E - 134
+ * so a product is P * 2^(xa + xb) with 0 <= P < 2^16 and xa + xb >= -266.
+ * The accumulator is an integer in units of 2^-266, held as SA_DIGITS
+ * base-2^32 digits in int64 slots (room for carries while summing).
+ * After normalisation digits 0..SA_DIGITS-2 lie in [0, 2^32) and the top
+ * digit is signed: the value is sum_i d_i * 2^(32 i - 266).
+ */
+#define SA_DIGITS 18
+#define SA_LSB_EXP 266
+
+typedef struct { int64_t d[SA_DIGITS]; } sacc_t;
+
+static int bf16_decompose(uint16_t bits, int *neg, int *mant, int *expo) {
+    const int E = (bits >> 7) & 0xff;
+    const int m = bits & 0x7f;
+    if (E == 0xff) return -2; /* inf / nan */
+    *neg = (bits >> 15) & 1;
+    if (E == 0) { *mant = m; *expo = -133; }
+    else { *mant = 128 + m; *expo = E - 134; }
+    return 0;
+}
+
+static int sa_add_product(sacc_t *a, uint16_t x, uint16_t y) {
+    int nx, mx, ex, ny, my, ey;
+    if (bf16_decompose(x, &nx, &mx, &ex) || bf16_decompose(y, &ny, &my, &ey)) return -2;
+    const int64_t P = (int64_t)mx * my;
+    if (P == 0) return 0;
+    const int off = ex + ey + SA_LSB_EXP; /* >= 0 */
+    const int64_t v = P * ((int64_t)1 << (off % 32)); /* < 2^47 */
+    a->d[off / 32] += (nx ^ ny) ? -v : v;
+    return 0;
+}
+
+static void sa_normalize(sacc_t *a) {
+    for (int i = 0; i + 1 < SA_DIGITS; ++i) {
+        /* floor division by 2^32 (works for negative digits too) */
+        int64_t c = a->d[i] / 4294967296LL;
+        if (a->d[i] - c * 4294967296LL < 0) c -= 1;
+        a->d[i] -= c * 4294967296LL;
+        a->d[i + 1] += c;
+    }
+}
+
+/* Compare two normalised accumulators: -1, 0, +1. */
+static int sa_compare(const sacc_t *a, const sacc_t *b) {
+    for (int i = SA_DIGITS - 1; i >= 0; --i) {
+        if (a->d[i] < b->d[i]) return -1;
+        if (a->d[i] > b->d[i]) return 1;
+    }
+    return 0;
+}
+
+static int sa_dot(const uint16_t *a, const uint16_t *b, int n, sacc_t *out) {
+    memset(out, 0, sizeof *out);
+    for (int i = 0; i < n; ++i)
+        if (sa_add_product(out, a[i], b[i])) return -2;
+    sa_normalize(out);
+    return 0;
+}
+
+/* Exact dot product; digits_out[SA_DIGITS] receives the normalised digits.
+ * Returns the number of digits (SA_DIGITS) and writes the weight exponent of
+ * digit 0 (-266) to *lsb_exp, or a negative status. */
+int oracle_exact_dot(const uint16_t *a, const uint16_t *b, int n, int64_t *digits_out, int *lsb_exp) {
+    if (!a || !b || !digits_out || n < 0) return -1;
+    sacc_t s;
+    if (sa_dot(a, b, n, &s)) return -2;
+    memcpy(digits_out, s.d, sizeof s.d);
+    if (lsb_exp) *lsb_exp = -SA_LSB_EXP;
+    return SA_DIGITS;
+}
+
+/* ------------------------------------------------------------------ */
+/* Selective V fetch (top-k positions per query head), renormalised    */
+/* ------------------------------------------------------------------ */
+
+typedef struct {
+    decode_ctx base;
+    int topk;
+    int32_t *idx_out; /* [n_rows, topk], ascending, -1 padded */
+} topv_ctx;
+
+typedef struct { sacc_t key; int j; } keyed_pos;
+
+/* order: larger exact key first; equal keys -> lower position first */
+static int keyed_cmp(const void *pa, const void *pb) {
+    const keyed_pos *a = (const keyed_pos *)pa, *b = (const keyed_pos *)pb;
+    const int c = sa_compare(&a->key, &b->key);
+    if (c != 0) return -c;
+    return (a->j > b->j) - (a->j < b->j);
+}
+
+static int int_cmp(const void *pa, const void *pb) {
+    const int a = *(const int *)pa, b = *(const int *)pb;
+    return (a > b) - (a < b);
+}
+
+static void topv_row(void *vctx, int64_t r) {
+    topv_ctx *tc = (topv_ctx *)vctx;
+    decode_ctx *c = &tc->base;
+    int b, h;
+    if (c->rows) { b = c->rows[2 * r]; h = c->rows[2 * r + 1]; }
+    else { b = (int)(r / c->n_q); h = (int)(r % c->n_q); }
+    double *o = c->out + r * c->d_v;
+    int32_t *idx = tc->idx_out + r * tc->topk;
+    for (int e = 0; e < c->d_v; ++e) o[e] = 0.0;
+    for (int e = 0; e < tc->topk; ++e) idx[e] = -1;
+    int T = c->seq_lens[b];
+    if (T > c->t_max) T = c->t_max;
+    if (T <= 0 || tc->topk <= 0) return;
+    const int kh = oracle_head_map(c->n_q, c->n_k, h);
+    const int vh = oracle_head_map(c->n_q, c->n_v, h);
+    const uint16_t *q = c->q + ((int64_t)b * c->n_q + h) * c->d_k;
+
+    /* 1. exact key e_j = <q, K_j> for every cached position */
+    keyed_pos *kp = (keyed_pos *)malloc(sizeof(keyed_pos) * (size_t)T);
+    if (!kp) { c->status = -3; return; }
+    for (int j = 0; j < T; ++j) {
+        const uint16_t *kr = c->k + (((int64_t)b * c->t_max + j) * c->n_k + kh) * c->d_k;
+        if (sa_dot(q, kr, c->d_k, &kp[j].key)) { c->status = -2; free(kp); return; }
+        kp[j].j = j;
+    }
+    /* 2. the k largest, ties toward the lower position */
+    qsort(kp, (size_t)T, sizeof(keyed_pos), keyed_cmp);
+    const int ksel = tc->topk < T ? tc->topk : T;
+    int *sel = (int *)malloc(sizeof(int) * (size_t)ksel);
+    if (!sel) { c->status = -3; free(kp); return; }
+    for (int e = 0; e < ksel; ++e) sel[e] = kp[e].j;
+    free(kp);
+    qsort(sel, (size_t)ksel, sizeof(int), int_cmp);
+    for (int e = 0; e < ksel; ++e) idx[e] = sel[e];
+
+    /* 3. softmax renormalised over the selected set, weighted V rows */
+    double *s = (double *)malloc(sizeof(double) * (size_t)ksel);
+    if (!s) { c->status = -3; free(sel); return; }
+    double m = -INFINITY;
+    for (int e = 0; e < ksel; ++e) {
+        const uint16_t *kr = c->k + (((int64_t)b * c->t_max + sel[e]) * c->n_k + kh) * c->d_k;
+        double acc = 0.0;
+        for (int d = 0; d < c->d_k; ++d) acc += bf16_to_f64(q[d]) * bf16_to_f64(kr[d]);
+        s[e] = c->scale * acc;
+        if (s[e] > m) m = s[e];
+    }
+    double den = 0.0;
+    for (int e = 0; e < ksel; ++e) {
+        const double w = exp(s[e] - m);
+        den += w;
+        const uint16_t *vr = v_row(c, b, sel[e], vh);
+        for (int d = 0; d < c->d_v; ++d) o[d] += w * bf16_to_f64(vr[d]);
+    }
+    for (int d = 0; d < c->d_v; ++d) o[d] /= den;
+    free(s);
+    free(sel);
+}
+
+int oracle_decode_topv(int batch, int n_q, int n_k, int n_v, int d_k, int d_v, double scale,
+                       const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
+                       const int32_t *seq_lens, int t_max, int topk,
+                       const int32_t *rows, int64_t n_rows, double *out, int32_t *idx_out,
+                       int n_threads) {
+    if (check_dims(batch, n_q, n_k, n_v, d_k, d_v) || t_max < 0 || topk < 0 || !q || !k_cache ||
+        !v_cache || !seq_lens || !out || !idx_out)
+        return -1;
+    if (!rows) n_rows = (int64_t)batch * n_q;
+    for (int64_t r = 0; rows && r < n_rows; ++r)
+        if (rows[2 * r] < 0 || rows[2 * r] >= batch || rows[2 * r + 1] < 0 || rows[2 * r + 1] >= n_q)
+            return -1;
+    topv_ctx c;
+    decode_ctx base = {batch, n_q, n_k, n_v, d_k, d_v, t_max, scale, 0,
+                       q, k_cache, v_cache, seq_lens, rows, out, 0};
+    c.base = base;
+    c.topk = topk;
+    c.idx_out = idx_out;
+    run_rows(topv_row, &c, n_rows, n_threads);
+    return c.base.status;
+}
