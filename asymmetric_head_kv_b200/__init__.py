@@ -1,0 +1,194 @@
+"""DiffQKV attention on NVIDIA B200 (sm_100a): Python binding of libdiffqkv.so.
+
+DiffQKV attention (Sigma paper, structured summary page, section 3.4) lets the
+K and V caches have different head counts and head dims; query head h reads K
+head h/(n_q/n_k) and V head h/(n_q/n_v).  Every function below only marshals
+torch tensors into the C ABI declared in include/diffqkv.h: shapes become a
+``diffqkv_dims_t``, tensors become device pointers, and the current torch CUDA
+stream is passed through.  All arithmetic runs in the library's CUDA kernels;
+torch provides device memory and streams.
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import Optional
+
+import torch
+
+from . import _capi
+from ._capi import DiffqkvError, Dims, DecodePlan, DecodeTuning, check, lib
+
+__all__ = [
+    "decode", "decode_workspace", "decode_plan", "decode_from_host", "decode_topv", "decode_topv_workspace",
+    "prefill_causal", "device_status", "selftest_wait_timeout", "DiffqkvError", "Dims", "library_path",
+]
+
+library_path = _capi.LIB_PATH
+
+
+def _stream_ptr(stream: Optional[torch.cuda.Stream]) -> ctypes.c_void_p:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> ctypes.c_void_p:
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _bf16_dev(t: torch.Tensor, name: str, ndim: int):
+    if t.dtype != torch.bfloat16:
+        raise TypeError(f"{name} must be bfloat16, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dim() != ndim or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous {ndim}-D tensor, got shape {tuple(t.shape)}")
+
+
+def make_dims(batch, n_q, n_k, n_v, d_k, d_v, scale) -> Dims:
+    return Dims(batch, n_q, n_k, n_v, d_k, d_v, float(scale))
+
+
+def _decode_dims(q, k_cache, v_cache, scale):
+    B, n_q, d_k = q.shape
+    Bk, t_max, n_k, d_k2 = k_cache.shape
+    Bv, t_max2, n_v, d_v = v_cache.shape
+    if B != Bk or B != Bv or d_k != d_k2 or t_max != t_max2:
+        raise ValueError("q / k_cache / v_cache shapes disagree")
+    if scale is None:
+        scale = d_k ** -0.5
+    return make_dims(B, n_q, n_k, n_v, d_k, d_v, scale), t_max
+
+
+def decode_workspace(q_or_dims, k_cache=None, v_cache=None, device=None) -> torch.Tensor:
+    """Zero-filled workspace for :func:`decode` (reusable across calls of one shape)."""
+    dims = q_or_dims if isinstance(q_or_dims, Dims) else _decode_dims(q_or_dims, k_cache, v_cache, 1.0)[0]
+    n = lib().diffqkv_decode_workspace_size(ctypes.byref(dims))
+    if n == 0:
+        raise DiffqkvError(_capi.INVALID_ARG, "decode_workspace_size")
+    dev = device if device is not None else (q_or_dims.device if isinstance(q_or_dims, torch.Tensor) else "cuda")
+    return torch.zeros(n, dtype=torch.uint8, device=dev)
+
+
+def decode_plan(dims: Dims, t_max: int, max_seq_len: int, num_sms: int, tuning: Optional[dict] = None) -> dict:
+    """Host-side launch plan of :func:`decode` (no GPU needed)."""
+    plan = DecodePlan()
+    tun = DecodeTuning(**tuning) if tuning else None
+    st = lib().diffqkv_decode_plan(ctypes.byref(dims), t_max, max_seq_len, num_sms,
+                                   ctypes.byref(tun) if tun else None, ctypes.byref(plan))
+    check(st, "decode_plan")
+    return {f: getattr(plan, f) for f, _ in DecodePlan._fields_}
+
+
+def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, seq_lens: torch.Tensor, *,
+           scale: Optional[float] = None, max_seq_len: Optional[int] = None, out: Optional[torch.Tensor] = None,
+           workspace: Optional[torch.Tensor] = None, tuning: Optional[dict] = None,
+           stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Split/combine DiffQKV decode: out[b, h] = softmax(scale q.K^T) V over seq_lens[b] positions.
+
+    q [B, n_q, d_k], k_cache [B, t_max, n_k, d_k], v_cache [B, t_max, n_v, d_v] (bf16, CUDA),
+    seq_lens int32 [B] (CUDA).  Returns bf16 [B, n_q, d_v].
+    """
+    _bf16_dev(q, "q", 3)
+    _bf16_dev(k_cache, "k_cache", 4)
+    _bf16_dev(v_cache, "v_cache", 4)
+    if seq_lens.dtype != torch.int32 or not seq_lens.is_cuda:
+        raise TypeError("seq_lens must be an int32 CUDA tensor")
+    dims, t_max = _decode_dims(q, k_cache, v_cache, scale)
+    if out is None:
+        out = torch.empty((dims.batch, dims.n_q, dims.d_v), dtype=torch.bfloat16, device=q.device)
+    if workspace is None:
+        workspace = decode_workspace(dims, device=q.device)
+    msl = t_max if max_seq_len is None else int(max_seq_len)
+    if tuning:
+        tun = DecodeTuning(**tuning)
+        st = lib().diffqkv_decode_ex(ctypes.byref(dims), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seq_lens),
+                                     t_max, msl, _ptr(out), _ptr(workspace), workspace.numel(), ctypes.byref(tun),
+                                     _stream_ptr(stream))
+    else:
+        st = lib().diffqkv_decode(ctypes.byref(dims), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seq_lens), t_max,
+                                  msl, _ptr(out), _ptr(workspace), workspace.numel(), _stream_ptr(stream))
+    check(st, "diffqkv_decode")
+    return out
+
+
+def decode_from_host(q_host, k_host, v_host, seq_lens_host, out_host, dev_buffers: dict, *,
+                     scale: Optional[float] = None, max_seq_len: Optional[int] = None,
+                     stream: Optional[torch.cuda.Stream] = None) -> None:
+    """End-to-end decode from (pinned) host tensors through one C-ABI call.
+
+    ``dev_buffers`` holds preallocated CUDA tensors q, k_cache, v_cache, seq_lens, out, workspace
+    of the same shapes.  Host->device copies, the decode and the device->host copy of the
+    output are all enqueued on the stream; synchronise before reading ``out_host``.
+    """
+    dims, t_max = _decode_dims(q_host, k_host, v_host, scale)
+    d = dev_buffers
+    msl = t_max if max_seq_len is None else int(max_seq_len)
+    st = lib().diffqkv_decode_from_host(
+        ctypes.byref(dims), _ptr(q_host), _ptr(k_host), _ptr(v_host), _ptr(seq_lens_host), t_max, msl,
+        _ptr(out_host), _ptr(d["q"]), _ptr(d["k_cache"]), _ptr(d["v_cache"]), _ptr(d["seq_lens"]), _ptr(d["out"]),
+        _ptr(d["workspace"]), d["workspace"].numel(), _stream_ptr(stream))
+    check(st, "diffqkv_decode_from_host")
+
+
+def decode_topv_workspace(dims: Dims, t_max: int, topk: int, device="cuda") -> torch.Tensor:
+    n = lib().diffqkv_decode_topv_workspace_size(ctypes.byref(dims), t_max, topk)
+    if n == 0:
+        raise DiffqkvError(_capi.INVALID_ARG, "decode_topv_workspace_size")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def decode_topv(q, k_cache, v_cache, seq_lens, topk: int, *, scale: Optional[float] = None,
+                max_seq_len: Optional[int] = None, out=None, idx_out=None, workspace=None,
+                stream: Optional[torch.cuda.Stream] = None):
+    """Selective-V decode over the top-k exact-scoring positions of each query head.
+
+    Returns (out bf16 [B, n_q, d_v], idx int32 [B, n_q, topk] ascending, -1 padded).
+    """
+    _bf16_dev(q, "q", 3)
+    _bf16_dev(k_cache, "k_cache", 4)
+    _bf16_dev(v_cache, "v_cache", 4)
+    if seq_lens.dtype != torch.int32 or not seq_lens.is_cuda:
+        raise TypeError("seq_lens must be an int32 CUDA tensor")
+    dims, t_max = _decode_dims(q, k_cache, v_cache, scale)
+    if out is None:
+        out = torch.empty((dims.batch, dims.n_q, dims.d_v), dtype=torch.bfloat16, device=q.device)
+    if idx_out is None:
+        idx_out = torch.empty((dims.batch, dims.n_q, topk), dtype=torch.int32, device=q.device)
+    if workspace is None:
+        workspace = decode_topv_workspace(dims, t_max, topk, q.device)
+    msl = t_max if max_seq_len is None else int(max_seq_len)
+    st = lib().diffqkv_decode_topv(ctypes.byref(dims), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seq_lens),
+                                   t_max, msl, topk, _ptr(out), _ptr(idx_out), _ptr(workspace), workspace.numel(),
+                                   _stream_ptr(stream))
+    check(st, "diffqkv_decode_topv")
+    return out, idx_out
+
+
+def prefill_causal(q, k, v, *, scale: Optional[float] = None, out=None,
+                   stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Causal prefill: q [B,S,n_q,d_k], k [B,S,n_k,d_k], v [B,S,n_v,d_v] -> out [B,S,n_q,d_v] (bf16)."""
+    _bf16_dev(q, "q", 4)
+    _bf16_dev(k, "k", 4)
+    _bf16_dev(v, "v", 4)
+    B, S, n_q, d_k = q.shape
+    n_k, n_v, d_v = k.shape[2], v.shape[2], v.shape[3]
+    if k.shape != (B, S, n_k, d_k) or v.shape[:2] != (B, S):
+        raise ValueError("q / k / v shapes disagree")
+    dims = make_dims(B, n_q, n_k, n_v, d_k, d_v, d_k ** -0.5 if scale is None else scale)
+    if out is None:
+        out = torch.empty((B, S, n_q, d_v), dtype=torch.bfloat16, device=q.device)
+    st = lib().diffqkv_prefill_causal(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), S, _ptr(out),
+                                      _stream_ptr(stream))
+    check(st, "diffqkv_prefill_causal")
+    return out
+
+
+def device_status(stream: Optional[torch.cuda.Stream] = None) -> int:
+    """Synchronises the stream and returns (and clears) the device error word."""
+    v = ctypes.c_int32(0)
+    check(lib().diffqkv_get_device_status(_stream_ptr(stream), ctypes.byref(v)), "diffqkv_get_device_status")
+    return v.value
+
+
+def selftest_wait_timeout(timeout_ns: int, stream: Optional[torch.cuda.Stream] = None) -> None:
+    check(lib().diffqkv_selftest_wait_timeout(int(timeout_ns), _stream_ptr(stream)), "diffqkv_selftest_wait_timeout")

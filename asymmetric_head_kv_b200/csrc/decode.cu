@@ -1,0 +1,626 @@
+// decode.cu -- split/combine DiffQKV decode attention for sm_100a.
+//
+// Follows the split kernel + combine kernel structure of FlexHeadFA ("Sigma:
+// Differential Rescaling of Query, Key and Value for Efficient Language
+// Models", structured summary page, "FlexHeadFA Kernel and Deployment
+// Infrastructure"): every KV chunk yields (running max, sum of exp,
+// unnormalised output) and a combine step merges the chunks.  The K and V
+// head of a query head are addressed separately (GroupSharing, section 3.4
+// Step 3): K head h/(n_q/n_k), V head h/(n_q/n_v).
+//
+// B200 design (one launch, memory-bound):
+//  * Work unit = (batch b, K-head group g): the n_q/n_k query heads that
+//    share K head g.  One K tile in shared memory serves all of them; each
+//    query head reads its own V head.
+//  * The K/V token range of all units is concatenated into one tile list and
+//    cut into equal contiguous ranges, one per CTA (grid = SMs x resident
+//    CTAs), so ragged batches and short contexts keep every SM equally busy.
+//    A CTA range may start or end inside a unit: each (unit, CTA) piece is one
+//    split.
+//  * One producer warp streams K and V tiles with TMA (cp.async.bulk.tensor,
+//    no multicast) into a multi-stage shared-memory ring guarded by
+//    mbarriers; consumer warps compute scores with 16-byte shared loads and
+//    warp-shuffle reductions, keep the online softmax in the log2 domain and
+//    accumulate P.V in fp32 registers.
+//  * The combine is fused: the last CTA to finish a unit (atomic counter in
+//    the workspace, reset afterwards) merges that unit's split partials and
+//    writes bf16 output.  No CTA ever waits on another.
+#include <math.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace diffqkv {
+
+namespace {
+
+constexpr int kGridMax = 2048;        // upper bound of split-kernel CTAs (sizes the workspace)
+constexpr int kWorkspaceHeader = 256; // reserved
+constexpr int kPartialPad = 4;        // per-head partial record: o[d_v], m, l, pad, pad
+
+struct DecodeArgs {
+    const __nv_bfloat16 *q;
+    const int32_t *seq_lens;
+    __nv_bfloat16 *out;
+    float *partials;
+    uint32_t *counters;
+    int32_t *status;
+    int32_t batch, n_q, n_k, n_v, t_max;
+    int32_t vpg;      // V heads carried by one tile
+    int32_t q_per_v;  // n_q / n_v
+    int32_t stages;
+    int32_t grid;
+    uint32_t stage_bytes;   // bytes TMA lands per stage (K box + V box)
+    uint32_t k_tile_bytes;  // offset of the V box inside a stage
+    uint32_t stage_stride;  // bytes between stages
+    float scale_log2;       // scale * log2(e)
+    uint64_t wait_limit_ns;
+};
+
+// Position of the tile walk: unit (b, g), tile i of nt, first global tile P.
+struct Walker {
+    int b, g, i, nt, T;
+    long long P;
+};
+
+__device__ __forceinline__ int clamp_len(int v, int t_max) { return v < 0 ? 0 : (v > t_max ? t_max : v); }
+
+template <int TT>
+__device__ __forceinline__ void walker_advance(Walker &w, const DecodeArgs &a) {
+    if (++w.i < w.nt) return;
+    w.P += w.nt;
+    w.i = 0;
+    if (++w.g < a.n_k) return;
+    w.g = 0;
+    for (;;) {
+        if (++w.b >= a.batch) { w.nt = 0; return; }
+        w.T = clamp_len(__ldg(a.seq_lens + w.b), a.t_max);
+        w.nt = (w.T + TT - 1) / TT;
+        if (w.nt > 0) return;
+    }
+}
+
+// CTA that owns global tile t when N tiles are cut into G equal ranges
+// [floor(c N / G), floor((c+1) N / G)).
+__device__ __forceinline__ long long cta_of_tile(long long t, long long N, long long G) {
+    return ((t + 1) * G - 1) / N;
+}
+
+template <int DK, int DV, int QPK, int TT, int NCW>
+__global__ void __launch_bounds__((NCW + 1) * 32, 1)
+    decode_split_combine_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                                const DecodeArgs a) {
+    constexpr int LPT = DK / 8;      // lanes per token in the score pass (8 bf16 per lane)
+    constexpr int TPP = 32 / LPT;    // tokens per score pass
+    constexpr int R = NCW / QPK;     // warps per query head (token split inside a tile)
+    constexpr int TPW = TT / R;      // tokens per warp per tile
+    constexpr int NPASS = TPW / TPP; // score passes per tile
+    constexpr int CPV = DV / 8;      // lanes per V row (8 bf16 per lane)
+    constexpr int NSL = 32 / CPV;    // token slots in the P.V pass
+    static_assert(NCW % QPK == 0 && TT % R == 0, "bad warp split");
+    static_assert(TPW % TPP == 0 && TPW % NSL == 0 && NPASS >= 1, "bad tile split");
+    static_assert(DK % 64 == 0 && DV % 64 == 0, "head dims");
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *full_bar = reinterpret_cast<uint64_t *>(smem + a.stages * a.stage_stride);
+    uint64_t *empty_bar = full_bar + a.stages;
+    float *p_s = reinterpret_cast<float *>(empty_bar + a.stages);  // [NCW][TPW]
+    float *merge_s = p_s + NCW * TPW;                               // [NCW][DV + 4]
+    int *flags = reinterpret_cast<int *>(merge_s + NCW * (DV + kPartialPad));
+    volatile int *abort_flag = flags;      // flags[0]
+    volatile int *last_flag = flags + 1;   // flags[1]
+    long long *scan_s = reinterpret_cast<long long *>(flags + 4);  // [0]=N, [1]=P0, [2]=b0|g0, [3]=i0
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+    const long long G = a.grid;
+    const long long c = blockIdx.x;
+
+    if (tid == 0) {
+        for (int s = 0; s < a.stages; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&empty_bar[s], NCW);
+        }
+        flags[0] = 0;
+        flags[1] = 0;
+        fence_barrier_init();
+    }
+    if (warp == NCW && lane == 0) {
+        prefetch_tensormap(&tm_k);
+        prefetch_tensormap(&tm_v);
+    }
+
+    // ---- prologue (warp 0): total tile count N, then the unit holding this CTA's first tile
+    if (warp == 0) {
+        long long acc = 0;
+        for (int base = 0; base < a.batch; base += 32) {
+            const int b = base + lane;
+            int nt = 0;
+            if (b < a.batch) {
+                const int raw = __ldg(a.seq_lens + b);
+                if (c == 0 && (raw < 0 || raw > a.t_max)) record_error(a.status, DIFFQKV_ERR_DEVICE_SEQLEN);
+                nt = (clamp_len(raw, a.t_max) + TT - 1) / TT;
+            }
+            long long incl = (long long)nt * a.n_k;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const long long y = __shfl_up_sync(0xffffffffu, incl, off);
+                if (lane >= off) incl += y;
+            }
+            acc += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        const long long N = acc;
+        // never more CTAs than tiles: every CTA range is then non-empty
+        const long long Ge = N < G ? N : G;
+        const long long t_begin = (c < Ge) ? (c * N) / Ge : N;
+        long long P0 = 0;
+        int b0 = a.batch, g0 = 0, i0 = 0;
+        acc = 0;
+        bool found = false;
+        for (int base = 0; base < a.batch && !found && N > 0; base += 32) {
+            const int b = base + lane;
+            const int nt = b < a.batch ? (clamp_len(__ldg(a.seq_lens + b), a.t_max) + TT - 1) / TT : 0;
+            const long long w = (long long)nt * a.n_k;
+            long long incl = w;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const long long y = __shfl_up_sync(0xffffffffu, incl, off);
+                if (lane >= off) incl += y;
+            }
+            const long long excl = incl - w;
+            const bool hit = b < a.batch && nt > 0 && acc + excl <= t_begin && t_begin < acc + incl;
+            const unsigned m = __ballot_sync(0xffffffffu, hit);
+            if (m) {
+                const int L = __ffs(m) - 1;
+                const long long start = __shfl_sync(0xffffffffu, acc + excl, L);
+                const int ntL = __shfl_sync(0xffffffffu, nt, L);
+                const long long within = t_begin - start;
+                b0 = base + L;
+                g0 = (int)(within / ntL);
+                i0 = (int)(within % ntL);
+                P0 = start + (long long)g0 * ntL;
+                found = true;
+            }
+            acc += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) {
+            scan_s[0] = N;
+            scan_s[1] = P0;
+            scan_s[2] = ((long long)b0 << 32) | (unsigned)g0;
+            scan_s[3] = i0;
+        }
+    }
+    __syncthreads();
+
+    const long long N = scan_s[0];
+    // sequences with no cached positions produce zero rows (distributed over CTAs)
+    for (int b = (int)c; b < a.batch; b += (int)G) {
+        if (clamp_len(__ldg(a.seq_lens + b), a.t_max) == 0) {
+            __nv_bfloat16 *o = a.out + (size_t)b * a.n_q * DV;
+            for (int e = tid; e < a.n_q * DV; e += blockDim.x) o[e] = __float2bfloat16(0.f);
+        }
+    }
+    const long long Ge = N < G ? N : G;  // CTAs that own tiles
+    if (c >= Ge) return;
+    const long long t_begin = (c * N) / Ge;
+    const long long t_end = ((c + 1) * N) / Ge;
+
+    Walker w0;
+    w0.b = (int)(scan_s[2] >> 32);
+    w0.g = (int)(scan_s[2] & 0xffffffff);
+    w0.i = (int)scan_s[3];
+    w0.P = scan_s[1];
+    w0.T = clamp_len(__ldg(a.seq_lens + w0.b), a.t_max);
+    w0.nt = (w0.T + TT - 1) / TT;
+
+    if (warp == NCW) {
+        // ================= producer: one elected lane issues all TMA loads
+        if (lane == 0) {
+            Walker w = w0;
+            long long k = 0;
+            for (long long t = t_begin; t < t_end; ++t, ++k) {
+                const int stage = (int)(k % a.stages);
+                if (k >= a.stages) {
+                    const uint32_t parity = (uint32_t)(((k / a.stages) - 1) & 1);
+                    mbar_wait_bounded(&empty_bar[stage], parity, a.wait_limit_ns, abort_flag, a.status);
+                }
+                if (*abort_flag) break;
+                uint8_t *sb = smem + (size_t)stage * a.stage_stride;
+                mbar_arrive_expect_tx(&full_bar[stage], a.stage_bytes);
+                const int v0 = (w.g * QPK) / a.q_per_v;
+                tma_load_4d(sb, &tm_k, &full_bar[stage], 0, w.g, w.i * TT, w.b);
+                tma_load_4d(sb + a.k_tile_bytes, &tm_v, &full_bar[stage], 0, v0, w.i * TT, w.b);
+                walker_advance<TT>(w, a);
+            }
+            // drain: never leave the CTA with copies still landing in its shared memory
+            const long long issued = k;
+            for (long long j = (issued > a.stages ? issued - a.stages : 0); j < issued; ++j) {
+                const int stage = (int)(j % a.stages);
+                mbar_wait_bounded(&full_bar[stage], (uint32_t)((j / a.stages) & 1), a.wait_limit_ns, nullptr,
+                                  a.status);
+            }
+        }
+        return;
+    }
+
+    // ================= consumers: warp = (head slot hs, token slice r)
+    const int hs = warp / R;
+    const int r = warp % R;
+    float *my_p = p_s + warp * TPW;
+    float *my_merge = merge_s + warp * (DV + kPartialPad);
+    const int kc = lane % LPT;   // K chunk (8 dims)
+    const int kt = lane / LPT;   // token within a score pass
+    const int vc = lane % CPV;   // V chunk (8 dims)
+    const int vs = lane / CPV;   // token slot in the P.V pass
+
+    float qf[8];
+    float o[8];
+    float m_run = -INFINITY, l_run = 0.f;
+    int v_local = 0;
+
+    Walker w = w0;
+    long long k = 0;
+    for (long long t = t_begin; t < t_end; ++t, ++k) {
+        const int h = w.g * QPK + hs;
+        if (t == t_begin || w.i == 0) {
+            // new split: this warp's query chunk, pre-scaled into the log2 domain
+            const uint4 qv = __ldg(reinterpret_cast<const uint4 *>(a.q + ((size_t)w.b * a.n_q + h) * DK) + kc);
+            unpack8(qv, qf);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) qf[e] *= a.scale_log2;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) o[e] = 0.f;
+            m_run = -INFINITY;
+            l_run = 0.f;
+            v_local = h / a.q_per_v - (w.g * QPK) / a.q_per_v;
+        }
+        const int stage = (int)(k % a.stages);
+        mbar_wait_bounded(&full_bar[stage], (uint32_t)((k / a.stages) & 1), a.wait_limit_ns, abort_flag, a.status);
+        const uint8_t *sb = smem + (size_t)stage * a.stage_stride;
+        const __nv_bfloat16 *Ks = reinterpret_cast<const __nv_bfloat16 *>(sb);
+        const __nv_bfloat16 *Vs = reinterpret_cast<const __nv_bfloat16 *>(sb + a.k_tile_bytes);
+
+        const int valid = min(TT, w.T - w.i * TT);
+        const int my_valid = max(0, min(TPW, valid - r * TPW));
+
+        // ---- scores s = (q . k) * scale * log2(e) for this warp's TPW tokens
+        float s[NPASS];
+#pragma unroll
+        for (int ps = 0; ps < NPASS; ++ps) {
+            const int tw = ps * TPP + kt;
+            const uint4 kv = lds128(Ks + (size_t)(r * TPW + tw) * DK + kc * 8);
+            float kf[8];
+            unpack8(kv, kf);
+            float acc = 0.f;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc = fmaf(qf[e], kf[e], acc);
+#pragma unroll
+            for (int off = LPT / 2; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+            s[ps] = tw < my_valid ? acc : -INFINITY;
+        }
+        // ---- online softmax update (log2 domain)
+        float mx = s[0];
+#pragma unroll
+        for (int ps = 1; ps < NPASS; ++ps) mx = fmaxf(mx, s[ps]);
+#pragma unroll
+        for (int off = LPT; off < 32; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        const float m_new = fmaxf(m_run, mx);
+        const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+        const float alpha = fast_exp2(m_run - m_use);
+        float psum = 0.f;
+#pragma unroll
+        for (int ps = 0; ps < NPASS; ++ps) {
+            s[ps] = fast_exp2(s[ps] - m_use);
+            psum += s[ps];
+        }
+#pragma unroll
+        for (int off = LPT; off < 32; off <<= 1) psum += __shfl_xor_sync(0xffffffffu, psum, off);
+        l_run = l_run * alpha + psum;
+        m_run = m_new;
+        if (kc == 0) {
+#pragma unroll
+            for (int ps = 0; ps < NPASS; ++ps) my_p[ps * TPP + kt] = s[ps];
+        }
+        __syncwarp();
+
+        // ---- o = o * alpha + sum_j p_j V[j, vh]
+#pragma unroll
+        for (int e = 0; e < 8; ++e) o[e] *= alpha;
+        const __nv_bfloat16 *vrow = Vs + ((size_t)(r * TPW) * a.vpg + v_local) * DV + vc * 8;
+        const size_t vstride = (size_t)a.vpg * DV;
+        if (my_valid == TPW) {
+#pragma unroll
+            for (int tt = vs; tt < TPW; tt += NSL) {
+                const float pv = my_p[tt];
+                const uint4 vv = lds128(vrow + tt * vstride);
+                float vf[8];
+                unpack8(vv, vf);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) o[e] = fmaf(pv, vf[e], o[e]);
+            }
+        } else {
+            for (int tt = vs; tt < my_valid; tt += NSL) {
+                const float pv = my_p[tt];
+                const uint4 vv = lds128(vrow + tt * vstride);
+                float vf[8];
+                unpack8(vv, vf);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) o[e] = fmaf(pv, vf[e], o[e]);
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty_bar[stage]);
+
+        // ---- end of this CTA's piece of the unit: write the split partial, maybe combine
+        if (w.i == w.nt - 1 || t == t_end - 1) {
+#pragma unroll
+            for (int off = CPV; off < 32; off <<= 1) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) o[e] += __shfl_xor_sync(0xffffffffu, o[e], off);
+            }
+            if (R > 1) {
+                if (vs == 0) {
+                    *reinterpret_cast<float4 *>(my_merge + vc * 8) = make_float4(o[0], o[1], o[2], o[3]);
+                    *reinterpret_cast<float4 *>(my_merge + vc * 8 + 4) = make_float4(o[4], o[5], o[6], o[7]);
+                }
+                if (lane == 0) {
+                    my_merge[DV] = m_run;
+                    my_merge[DV + 1] = l_run;
+                }
+            }
+            named_barrier(1, NCW * 32);
+            const long long u = (long long)w.b * a.n_k + w.g;
+            const long long first = cta_of_tile(w.P, N, Ge);
+            const long long last = cta_of_tile(w.P + w.nt - 1, N, Ge);
+            if (r == 0) {
+                float M = m_run, L = l_run;
+                float O[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) O[e] = o[e];
+                if (R > 1) {
+                    M = -INFINITY;
+#pragma unroll
+                    for (int rr = 0; rr < R; ++rr) M = fmaxf(M, merge_s[(warp + rr) * (DV + kPartialPad) + DV]);
+                    const float Mu = (M == -INFINITY) ? 0.f : M;
+                    L = 0.f;
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) O[e] = 0.f;
+#pragma unroll
+                    for (int rr = 0; rr < R; ++rr) {
+                        const float *src = merge_s + (warp + rr) * (DV + kPartialPad);
+                        const float f = fast_exp2(src[DV] - Mu);
+                        L += f * src[DV + 1];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) O[e] = fmaf(f, src[vc * 8 + e], O[e]);
+                    }
+                }
+                float *dst = a.partials + ((size_t)(u + c) * QPK + hs) * (DV + kPartialPad);
+                if (vs == 0) {
+                    __stcg(reinterpret_cast<float4 *>(dst + vc * 8), make_float4(O[0], O[1], O[2], O[3]));
+                    __stcg(reinterpret_cast<float4 *>(dst + vc * 8 + 4), make_float4(O[4], O[5], O[6], O[7]));
+                }
+                if (lane == 0) {
+                    __stcg(dst + DV, M);
+                    __stcg(dst + DV + 1, L);
+                }
+            }
+            __threadfence();
+            named_barrier(1, NCW * 32);
+            if (tid == 0) {
+                const unsigned old = atomicAdd(a.counters + u, 1u);
+                *last_flag = (old == (unsigned)(last - first)) ? 1 : 0;
+            }
+            named_barrier(1, NCW * 32);
+            if (*last_flag) {
+                __threadfence();
+                constexpr int ITEMS = QPK * (DV / 4);
+                for (int it = tid; it < ITEMS; it += NCW * 32) {
+                    const int h2 = it / (DV / 4);
+                    const int d4 = it % (DV / 4);
+                    float M = -INFINITY;
+                    for (long long cc = first; cc <= last; ++cc)
+                        M = fmaxf(M, __ldcg(a.partials + ((size_t)(u + cc) * QPK + h2) * (DV + kPartialPad) + DV));
+                    const float Mu = (M == -INFINITY) ? 0.f : M;
+                    float L = 0.f;
+                    float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+                    for (long long cc = first; cc <= last; ++cc) {
+                        const float *src = a.partials + ((size_t)(u + cc) * QPK + h2) * (DV + kPartialPad);
+                        const float f = fast_exp2(__ldcg(src + DV) - Mu);
+                        L = fmaf(f, __ldcg(src + DV + 1), L);
+                        const float4 x = __ldcg(reinterpret_cast<const float4 *>(src) + d4);
+                        O.x = fmaf(f, x.x, O.x);
+                        O.y = fmaf(f, x.y, O.y);
+                        O.z = fmaf(f, x.z, O.z);
+                        O.w = fmaf(f, x.w, O.w);
+                    }
+                    const float inv = L > 0.f ? 1.f / L : 0.f;
+                    __nv_bfloat162 lo = __floats2bfloat162_rn(O.x * inv, O.y * inv);
+                    __nv_bfloat162 hi = __floats2bfloat162_rn(O.z * inv, O.w * inv);
+                    uint2 packed;
+                    packed.x = *reinterpret_cast<uint32_t *>(&lo);
+                    packed.y = *reinterpret_cast<uint32_t *>(&hi);
+                    *reinterpret_cast<uint2 *>(a.out + ((size_t)w.b * a.n_q + w.g * QPK + h2) * DV + d4 * 4) = packed;
+                }
+                if (tid == 0) a.counters[u] = 0u;
+            }
+            named_barrier(1, NCW * 32);
+        }
+        walker_advance<TT>(w, a);
+    }
+}
+
+// ------------------------------------------------------------------ host side
+
+constexpr int ncw_for(int qpk) { return qpk > 8 ? qpk : 8; }
+
+// Tile height: about 32-40 KiB of K+V per stage (V side sized for the widest group).
+constexpr int tt_for(int dk, int dv, int qpk) {
+    const int bytes_per_token = 2 * dk + 2 * qpk * dv;
+    int tt = 16;
+    while (tt < 128 && (tt * 2) * bytes_per_token <= 40 * 1024) tt *= 2;
+    return tt;
+}
+
+int v_heads_per_tile(const diffqkv_dims_t *d) {
+    const int qpk = d->n_q / d->n_k;
+    const int qpv = d->n_q / d->n_v;
+    int span = 1;
+    for (int g = 0; g < d->n_k; ++g) {
+        const int v0 = (g * qpk) / qpv;
+        const int v1 = ((g + 1) * qpk - 1) / qpv;
+        span = std::max(span, v1 - v0 + 1);
+    }
+    return span;
+}
+
+bool supported_qpk(int qpk) { return qpk == 1 || qpk == 2 || qpk == 4 || qpk == 8 || qpk == 16; }
+
+using KernelFn = void (*)(CUtensorMap, CUtensorMap, DecodeArgs);
+
+template <int DK, int DV, int QPK>
+KernelFn kernel_for() {
+    return decode_split_combine_kernel<DK, DV, QPK, tt_for(DK, DV, QPK), ncw_for(QPK)>;
+}
+
+template <int DK, int DV>
+KernelFn pick_kernel_qpk(int qpk) {
+    switch (qpk) {
+        case 1: return kernel_for<DK, DV, 1>();
+        case 2: return kernel_for<DK, DV, 2>();
+        case 4: return kernel_for<DK, DV, 4>();
+        case 8: return kernel_for<DK, DV, 8>();
+        case 16: return kernel_for<DK, DV, 16>();
+        default: return nullptr;
+    }
+}
+
+KernelFn pick_kernel(int dk, int dv, int qpk) {
+    if (dk == 64 && dv == 64) return pick_kernel_qpk<64, 64>(qpk);
+    if (dk == 64 && dv == 128) return pick_kernel_qpk<64, 128>(qpk);
+    if (dk == 128 && dv == 64) return pick_kernel_qpk<128, 64>(qpk);
+    if (dk == 128 && dv == 128) return pick_kernel_qpk<128, 128>(qpk);
+    return nullptr;
+}
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+}  // namespace
+
+size_t decode_workspace_size(const diffqkv_dims_t *d) {
+    if (validate_dims(d) != DIFFQKV_OK) return 0;
+    const size_t units = (size_t)d->batch * d->n_k;
+    const size_t qpk = d->n_q / d->n_k;
+    const size_t counters = align_up(units * sizeof(uint32_t), 256);
+    const size_t partials = (units + kGridMax) * qpk * (d->d_v + kPartialPad) * sizeof(float);
+    return kWorkspaceHeader + counters + partials;
+}
+
+diffqkv_status_t decode_plan(const diffqkv_dims_t *d, int32_t t_max, int32_t max_seq_len, int32_t num_sms,
+                             const diffqkv_decode_tuning_t *tuning, diffqkv_decode_plan_t *plan) {
+    if (!plan) return DIFFQKV_ERR_INVALID_ARG;
+    diffqkv_status_t st = validate_dims(d);
+    if (st != DIFFQKV_OK) return st;
+    if (t_max < 1 || num_sms < 1) return DIFFQKV_ERR_INVALID_ARG;
+    const int qpk = d->n_q / d->n_k;
+    if (!supported_qpk(qpk) || (d->d_k != 64 && d->d_k != 128) || (d->d_v != 64 && d->d_v != 128))
+        return DIFFQKV_ERR_UNSUPPORTED;
+    struct { int tt, ncw; } ks = {tt_for(d->d_k, d->d_v, qpk), ncw_for(qpk)};
+    const int vpg = v_heads_per_tile(d);
+    const size_t k_tile = (size_t)ks.tt * d->d_k * 2;
+    const size_t v_tile = (size_t)ks.tt * vpg * d->d_v * 2;
+    const size_t stage_stride = align_up(k_tile + v_tile, 1024);
+    const size_t extra = 16 * 8 /*barriers*/ + (size_t)ks.ncw * (ks.tt / (ks.ncw / qpk)) * 4 +
+                         (size_t)ks.ncw * (d->d_v + kPartialPad) * 4 + 64 + 1024 /*alignment slack*/;
+    const size_t smem_cap = 227 * 1024;
+    int stages = (tuning && tuning->stages) ? tuning->stages : 0;
+    if (stages == 0) {
+        stages = 2;
+        while (stages < 8 && (stages + 1) * stage_stride + extra <= std::min<size_t>(smem_cap, 200 * 1024)) ++stages;
+    }
+    if (stages < 2 || stages > 8 || stages * stage_stride + extra > smem_cap) return DIFFQKV_ERR_UNSUPPORTED;
+    int cps = (tuning && tuning->ctas_per_sm) ? tuning->ctas_per_sm : 1;
+    if (cps < 1 || cps > 4) return DIFFQKV_ERR_INVALID_ARG;
+    const int msl = (max_seq_len >= 1 && max_seq_len <= t_max) ? max_seq_len : t_max;
+    const long long n_est = (long long)d->batch * d->n_k * ((msl + ks.tt - 1) / ks.tt);
+    long long grid = (long long)num_sms * cps;
+    if (grid > n_est) grid = n_est;
+    if (tuning && tuning->grid_ctas) grid = tuning->grid_ctas;
+    if (grid < 1 || grid > kGridMax) return DIFFQKV_ERR_INVALID_ARG;
+    plan->tile_tokens = ks.tt;
+    plan->stages = stages;
+    plan->grid_ctas = (int32_t)grid;
+    plan->threads = (ks.ncw + 1) * 32;
+    plan->v_heads_per_tile = vpg;
+    plan->smem_bytes = (int64_t)(stages * stage_stride + extra);
+    plan->workspace_bytes = (int64_t)decode_workspace_size(d);
+    return DIFFQKV_OK;
+}
+
+diffqkv_status_t decode_launch(const diffqkv_dims_t *d, const void *q, const void *k_cache, const void *v_cache,
+                               const int32_t *seq_lens, int32_t t_max, int32_t max_seq_len, void *out,
+                               void *workspace, size_t workspace_bytes, const diffqkv_decode_tuning_t *tuning,
+                               cudaStream_t stream) {
+    diffqkv_status_t st = validate_dims(d);
+    if (st != DIFFQKV_OK) return st;
+    if (!q || !k_cache || !v_cache || !seq_lens || !out || t_max < 1) return DIFFQKV_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
+        (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
+        return DIFFQKV_ERR_MISALIGNED;
+    const size_t need = decode_workspace_size(d);
+    if (!workspace || workspace_bytes < need) return DIFFQKV_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return DIFFQKV_ERR_MISALIGNED;
+
+    DeviceInfo dev;
+    st = current_device_info(&dev);
+    if (st != DIFFQKV_OK) return st;
+    diffqkv_decode_plan_t plan;
+    st = decode_plan(d, t_max, max_seq_len, dev.num_sms, tuning, &plan);
+    if (st != DIFFQKV_OK) return st;
+    const int qpk = d->n_q / d->n_k;
+    KernelFn fn = pick_kernel(d->d_k, d->d_v, qpk);
+    if (!fn) return DIFFQKV_ERR_UNSUPPORTED;
+
+    CUtensorMap tm_k, tm_v;
+    st = make_tensor_map_4d(&tm_k, k_cache, d->d_k, d->n_k, t_max, d->batch, d->d_k, 1, plan.tile_tokens, 1,
+                            CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (st != DIFFQKV_OK) return st;
+    st = make_tensor_map_4d(&tm_v, v_cache, d->d_v, d->n_v, t_max, d->batch, d->d_v, plan.v_heads_per_tile,
+                            plan.tile_tokens, 1, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (st != DIFFQKV_OK) return st;
+
+    DecodeArgs a;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    const size_t units = (size_t)d->batch * d->n_k;
+    a.q = static_cast<const __nv_bfloat16 *>(q);
+    a.seq_lens = seq_lens;
+    a.out = static_cast<__nv_bfloat16 *>(out);
+    a.counters = reinterpret_cast<uint32_t *>(ws + kWorkspaceHeader);
+    a.partials = reinterpret_cast<float *>(ws + kWorkspaceHeader + align_up(units * sizeof(uint32_t), 256));
+    a.status = dev.status_word;
+    a.batch = d->batch;
+    a.n_q = d->n_q;
+    a.n_k = d->n_k;
+    a.n_v = d->n_v;
+    a.t_max = t_max;
+    a.vpg = plan.v_heads_per_tile;
+    a.q_per_v = d->n_q / d->n_v;
+    a.stages = plan.stages;
+    a.grid = plan.grid_ctas;
+    a.k_tile_bytes = (uint32_t)plan.tile_tokens * d->d_k * 2;
+    a.stage_bytes = a.k_tile_bytes + (uint32_t)plan.tile_tokens * plan.v_heads_per_tile * d->d_v * 2;
+    a.stage_stride = (uint32_t)align_up(a.stage_bytes, 1024);
+    a.scale_log2 = (float)((double)d->scale * 1.4426950408889634);
+    a.wait_limit_ns = kWaitLimitNs;
+
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)plan.smem_bytes) != cudaSuccess)
+        return DIFFQKV_ERR_CUDA;
+    fn<<<plan.grid_ctas, plan.threads, plan.smem_bytes, stream>>>(tm_k, tm_v, a);
+    if (cudaGetLastError() != cudaSuccess) return DIFFQKV_ERR_CUDA;
+    return DIFFQKV_OK;
+}
+
+}  // namespace diffqkv

@@ -1,0 +1,64 @@
+// internal.h -- host-side helpers shared by the libdiffqkv translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/diffqkv.h"
+
+namespace diffqkv {
+
+// Per-device cached attributes and the device address of the error word.
+struct DeviceInfo {
+    int device = -1;
+    int num_sms = 0;
+    int max_smem_optin = 0;
+    int32_t *status_word = nullptr;  // device address of the error word
+};
+
+// Fills `info` for the current device.  Returns DIFFQKV_OK or an error.
+diffqkv_status_t current_device_info(DeviceInfo *info);
+
+// Encodes a rank-4 tiled tensor map over a bf16 tensor laid out as
+// [dim3][dim2][dim1][dim0] (dim0 innermost, contiguous), box {b0,b1,b2,b3}.
+diffqkv_status_t make_tensor_map_4d(CUtensorMap *map, const void *base, uint64_t dim0, uint64_t dim1,
+                                    uint64_t dim2, uint64_t dim3, uint32_t box0, uint32_t box1,
+                                    uint32_t box2, uint32_t box3, CUtensorMapSwizzle swizzle);
+
+// Encodes a rank-3 tiled tensor map ([dim2][dim1][dim0], dim0 contiguous).
+diffqkv_status_t make_tensor_map_3d(CUtensorMap *map, const void *base, uint64_t dim0, uint64_t dim1,
+                                    uint64_t dim2, uint64_t stride1_bytes, uint64_t stride2_bytes,
+                                    uint32_t box0, uint32_t box1, uint32_t box2,
+                                    CUtensorMapSwizzle swizzle);
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Shape checks common to every entry point.
+diffqkv_status_t validate_dims(const diffqkv_dims_t *d);
+
+// decode.cu
+diffqkv_status_t decode_plan(const diffqkv_dims_t *d, int32_t t_max, int32_t max_seq_len, int32_t num_sms,
+                             const diffqkv_decode_tuning_t *tuning, diffqkv_decode_plan_t *plan);
+size_t decode_workspace_size(const diffqkv_dims_t *d);
+diffqkv_status_t decode_launch(const diffqkv_dims_t *d, const void *q, const void *k_cache,
+                               const void *v_cache, const int32_t *seq_lens, int32_t t_max,
+                               int32_t max_seq_len, void *out, void *workspace, size_t workspace_bytes,
+                               const diffqkv_decode_tuning_t *tuning, cudaStream_t stream);
+
+// topv.cu
+size_t topv_workspace_size(const diffqkv_dims_t *d, int32_t t_max, int32_t topk);
+diffqkv_status_t topv_launch(const diffqkv_dims_t *d, const void *q, const void *k_cache, const void *v_cache,
+                             const int32_t *seq_lens, int32_t t_max, int32_t max_seq_len, int32_t topk,
+                             void *out, int32_t *idx_out, void *workspace, size_t workspace_bytes,
+                             cudaStream_t stream);
+
+// prefill.cu
+diffqkv_status_t prefill_launch(const diffqkv_dims_t *d, const void *q, const void *k, const void *v,
+                                int32_t seq_len, void *out, cudaStream_t stream);
+
+// api.cu
+diffqkv_status_t wait_timeout_selftest_launch(int64_t timeout_ns, cudaStream_t stream);
+
+}  // namespace diffqkv

@@ -1,0 +1,363 @@
+#!/usr/bin/env python
+"""Benchmark: DiffQKV decode attention KV-cache bandwidth at 32k context vs GQA.
+
+One step = one diffqkv_decode call over the whole batch of the Sigma-1.5B-shaped
+decode workload (B=16, n_q=16, n_k=4, n_v=16, d_k=64, d_v=128, 32768 cached
+positions per sequence, bf16 N(0,1) inputs, seed 1): head mapping, split
+scores, online-softmax partials, split P.V, combine -- one kernel launch.
+The symmetric GQA control (n_k=n_v=16, d_k=d_v=128, same seed) is timed the
+same way and reported beside it.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs under torchrun, one process per GPU; every rank decodes its own
+full batch (independent sequences: weak scaling, no collective on the data
+path); the time is the max over ranks.  ``--impl reference`` times the fp64
+CPU oracle on a bounded sample of the same workload (rank 0 only).
+Prints ONE JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as wl  # noqa: E402
+
+METRIC = "decode attn KV-cache GB/s (% of HBM peak) and us/step at 32k ctx vs GQA"
+UNIT = "GB/s"
+WORKLOAD = wl.DECODE_32K
+CONTROL = wl.DECODE_32K_GQA
+PROFILE = os.path.join(ROOT, "profiles", "decode_split_combine_b16_t32768.md")
+KERNEL_SOURCES = ["asymmetric_head_kv_b200/csrc/decode.cu", "asymmetric_head_kv_b200/csrc/common.cuh"]
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=1000)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--e2e-steps", type=int, default=5)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on this kernel source."""
+    if not os.path.exists(PROFILE):
+        return None
+    text = open(PROFILE).read()
+    m_hash = re.search(r"kernel_source_sha256:\s*([0-9a-f]+)", text)
+    m_tr = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    if not m_hash or not m_tr or m_hash.group(1) != kernel_source_hash():
+        return None
+    return float(m_tr.group(1))
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while the timed region runs (read-only)."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4, "hw_slowdown": 0x8,
+        "sync_boost": 0x10, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+        "hw_power_brake_slowdown": 0x80, "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, device_index: int):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # no NVML: report no samples
+            self.nv = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                mask = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for name, bit in self.REASONS.items():
+                    if mask & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.02)
+
+    def __enter__(self):
+        if self.nv:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self.nv:
+            self.t.join()
+
+    def summary(self):
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def time_decode(ak, w: wl.DecodeWorkload, steps: int, warmup: int, world: int, sampler=None):
+    """Times `steps` decode calls; returns dict with region time, per-launch times, bytes."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    d = wl.make_decode_inputs(w, dev)
+    out = torch.empty((w.batch, w.shape.n_q, w.shape.d_v), dtype=torch.bfloat16, device=dev)
+    ws = ak.decode_workspace(d["q"], d["k_cache"], d["v_cache"])
+    msl = int(d["seq_lens"].max())
+    stream = torch.cuda.current_stream()
+
+    def step():
+        ak.decode(d["q"], d["k_cache"], d["v_cache"], d["seq_lens"], scale=d["scale"], max_seq_len=msl,
+                  out=out, workspace=ws, stream=stream)
+
+    for _ in range(max(warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    assert ak.device_status() == 0
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    ctx = sampler if sampler is not None else _Null()
+    with ctx:
+        for i in range(steps):
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    region_ms = starts[0].elapsed_time(ends[-1])
+    per_launch = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    nbytes = wl.decode_kv_bytes(w.shape, d["seq_lens"].cpu())
+    res = {"region_ms": region_ms, "launch_ms_mean": statistics.fmean(per_launch),
+           "launch_ms_median": statistics.median(per_launch), "kv_bytes": nbytes, "inputs": d, "out": out}
+    return res
+
+
+class _Null:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *a):
+        return False
+
+
+def time_e2e(ak, w: wl.DecodeWorkload, d_dev: dict, steps: int):
+    """Same step through the host-buffer C-ABI entry point: H2D of all inputs, decode, D2H of the output."""
+    host = {k: d_dev[k].cpu().pin_memory() for k in ("q", "k_cache", "v_cache", "seq_lens")}
+    out_host = torch.empty((w.batch, w.shape.n_q, w.shape.d_v), dtype=torch.bfloat16).pin_memory()
+    dev = {k: torch.empty_like(d_dev[k]) for k in ("q", "k_cache", "v_cache", "seq_lens")}
+    dev["out"] = torch.empty((w.batch, w.shape.n_q, w.shape.d_v), dtype=torch.bfloat16, device=d_dev["q"].device)
+    dev["workspace"] = ak.decode_workspace(d_dev["q"], d_dev["k_cache"], d_dev["v_cache"])
+    msl = int(host["seq_lens"].max())
+    stream = torch.cuda.current_stream()
+
+    def step():
+        ak.decode_from_host(host["q"], host["k_cache"], host["v_cache"], host["seq_lens"], out_host, dev,
+                            scale=w.shape.scale, max_seq_len=msl, stream=stream)
+
+    step()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for _ in range(steps):
+        step()
+    e.record(stream)
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e) / steps
+    h2d = sum(host[k].numel() * host[k].element_size() for k in host)
+    d2h = out_host.numel() * out_host.element_size()
+    return ms, h2d, d2h
+
+
+def oracle_sample_rate(w: wl.DecodeWorkload, d_cpu: dict, budget_s: float):
+    """fp64 oracle on a bounded sample of (b, h) rows; GB/s attributed pro rata to the step's KV bytes."""
+    import oracle
+
+    rows_total = w.batch * w.shape.n_q
+    step_bytes = wl.decode_kv_bytes(w.shape, d_cpu["seq_lens"])
+    threads = os.cpu_count() or 1
+    # calibrate on one row per thread, then size the sample to the budget
+    n = min(rows_total, threads)
+    rows = [(i // w.shape.n_q, i % w.shape.n_q) for i in range(n)]
+    t0 = time.perf_counter()
+    oracle.decode(d_cpu["q"], d_cpu["k_cache"], d_cpu["v_cache"], d_cpu["seq_lens"], d_cpu["scale"], rows=rows,
+                  threads=threads)
+    dt = time.perf_counter() - t0
+    n = int(max(1, min(rows_total, n * budget_s / max(dt, 1e-6))))
+    rows = [(i // w.shape.n_q, i % w.shape.n_q) for i in range(n)]
+    t0 = time.perf_counter()
+    oracle.decode(d_cpu["q"], d_cpu["k_cache"], d_cpu["v_cache"], d_cpu["seq_lens"], d_cpu["scale"], rows=rows,
+                  threads=threads)
+    dt = time.perf_counter() - t0
+    nbytes = step_bytes * n / rows_total
+    return {"value": nbytes / dt / 1e9, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{n} of {rows_total} (b, h) rows of one step ({n / rows_total:.0%} of its KV bytes), "
+                      f"fp64 C oracle, {dt:.2f} s", "seconds": dt}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    budget = max(0.5, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    d = wl.make_decode_inputs(WORKLOAD, "cpu")
+    total_bytes, total_s, info = 0.0, 0.0, None
+    for i in range(args.warmup + args.steps):
+        info = oracle_sample_rate(WORKLOAD, d, budget)
+        if i >= args.warmup:
+            total_bytes += info["value"] * 1e9 * info["seconds"]
+            total_s += info["seconds"]
+    value = total_bytes / total_s / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD.name, "batch": WORKLOAD.batch, "context": WORKLOAD.t_max,
+                   "n_q": 16, "n_k": 4, "n_v": 16, "d_k": 64, "d_v": 128},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": info["cores"], "kind": "oracle",
+                         "sample": info["sample"] + " per step"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_setup(args)
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        return
+    import asymmetric_head_kv_b200 as ak
+
+    torch.cuda.set_device(local)
+    peaks, peak_src = load_peaks()
+    sampler = ClockSampler(local)
+    main_res = time_decode(ak, WORKLOAD, args.steps, args.warmup, world, sampler)
+    region_ms = max_over_ranks(main_res["region_ms"], world)
+    ms_per_step = region_ms / args.steps
+    total_bytes = main_res["kv_bytes"] * world
+    value = total_bytes / (region_ms / args.steps * 1e-3) / 1e9
+
+    launch_ms = main_res["launch_ms_mean"]
+    achieved = main_res["kv_bytes"] / (launch_ms * 1e-3) / 1e9
+    peak = float(peaks["hbm_gbs"])
+    traffic = profiled_traffic()
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                "traffic": traffic, "peak_source": f"{peak_src} hbm_gbs (copy bandwidth)",
+                "kernel": "decode_split_combine_kernel", "launch_us_mean": launch_ms * 1e3,
+                "launch_us_median": main_res["launch_ms_median"] * 1e3,
+                "algorithmic_bytes_per_launch": main_res["kv_bytes"]}
+
+    # symmetric GQA control, same seed and context
+    ctrl = time_decode(ak, CONTROL, max(50, args.steps // 4), args.warmup, world)
+    ctrl_ms = max_over_ranks(ctrl["region_ms"], world) / max(50, args.steps // 4)
+    control = {"workload": CONTROL.name, "ms_per_step": ctrl_ms, "us_per_step": ctrl_ms * 1e3,
+               "value": ctrl["kv_bytes"] * world / (ctrl_ms * 1e-3) / 1e9, "unit": UNIT,
+               "kv_bytes_per_gpu": ctrl["kv_bytes"],
+               "frac_of_peak": ctrl["kv_bytes"] / (ctrl["launch_ms_mean"] * 1e-3) / 1e9 / peak,
+               "diffqkv_time_reduction": 1.0 - ms_per_step / ctrl_ms}
+    del ctrl
+
+    e2e_ms, h2d, d2h = time_e2e(ak, WORKLOAD, main_res["inputs"], args.e2e_steps)
+    e2e_ms = max_over_ranks(e2e_ms, world)
+    e2e = {"value": total_bytes / (e2e_ms * 1e-3) / 1e9, "unit": UNIT, "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": args.e2e_steps,
+           "api": "diffqkv_decode_from_host (pinned host buffers)"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        d_cpu = {k: (v.cpu() if isinstance(v, torch.Tensor) else v) for k, v in main_res["inputs"].items()}
+        info = oracle_sample_rate(WORKLOAD, d_cpu, 15.0)
+        cpu = {k: info[k] for k in ("value", "unit", "cores", "kind", "sample")}
+        del d_cpu
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "us_per_step": ms_per_step * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD.name, "batch_per_gpu": WORKLOAD.batch, "context": WORKLOAD.t_max,
+                       "n_q": 16, "n_k": 4, "n_v": 16, "d_k": 64, "d_v": 128, "parallelism": f"replicas x{world}",
+                       "l2": "inputs (2.42 GB) larger than L2 (126 MB); no flush",
+                       "kv_bytes_per_gpu_step": main_res["kv_bytes"]},
+            "pct_of_hbm_peak": 100.0 * achieved / peak,
+            "gqa_control": control,
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": args.steps,
+            "clocks": sampler.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

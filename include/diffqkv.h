@@ -1,0 +1,222 @@
+/*
+ * diffqkv.h -- C ABI of libdiffqkv.so: DiffQKV attention for NVIDIA B200 (sm_100a).
+ *
+ * DiffQKV attention ("Sigma: Differential Rescaling of Query, Key and Value
+ * for Efficient Language Models", structured summary page, section 3.4
+ * "DiffQKV Attention: Generalized Formulation") lets the K and V sides of a
+ * KV cache have different head counts (n_k != n_v) and head dims
+ * (d_k != d_v).  Under GroupSharing (same section, Step 3; and "FlexHeadFA
+ * Kernel and Deployment Infrastructure", address calculation) query head h
+ * reads K head h / (n_q / n_k) and V head h / (n_q / n_v).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Tensors are dense, row-major, bf16 unless stated; pointers are DEVICE
+ *    pointers unless stated and must be 16-byte aligned.
+ *  - The caller owns every buffer.  The library never allocates or frees
+ *    device memory and keeps no per-call state; the only library-wide state is
+ *    a per-device error word (see diffqkv_get_device_status) and cached device
+ *    attributes.
+ *  - Every call is asynchronous on the caller's stream (NULL = legacy default
+ *    stream) and never synchronises, except diffqkv_get_device_status and
+ *    diffqkv_decode_from_host's callers' own syncs.
+ *  - Every call returns a diffqkv_status_t.  Argument errors are detected on
+ *    the host before anything is launched; nothing crosses the ABI as an
+ *    exception.  Conditions only the device can see (a seq_len outside
+ *    [0, t_max], a bounded wait that ran out) are recorded in the device error
+ *    word and reported by diffqkv_get_device_status.
+ *  - Supported shapes: n_q % n_k == 0, n_q % n_v == 0 (else INVALID_ARG);
+ *    n_q / n_k in {1, 2, 4, 8, 16} and d_k, d_v in {64, 128} (else
+ *    UNSUPPORTED).
+ */
+#ifndef DIFFQKV_H_
+#define DIFFQKV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t; NULL selects the legacy default stream. */
+typedef struct CUstream_st *diffqkv_stream_t;
+
+/* Attention shape.  scale multiplies q.k before the softmax (1/sqrt(d_k) in
+ * the paper's Attend step, section 3.4 Step 4). */
+typedef struct {
+    int32_t batch; /* B >= 1 */
+    int32_t n_q;   /* query heads */
+    int32_t n_k;   /* K heads (n_q % n_k == 0) */
+    int32_t n_v;   /* V heads (n_q % n_v == 0) */
+    int32_t d_k;   /* K (and q) head dim */
+    int32_t d_v;   /* V (and output) head dim */
+    float scale;   /* > 0, finite */
+} diffqkv_dims_t;
+
+typedef enum {
+    DIFFQKV_OK = 0,
+    DIFFQKV_ERR_INVALID_ARG = 1,    /* bad dims, null pointer, bad size */
+    DIFFQKV_ERR_UNSUPPORTED = 2,    /* legal shape this build has no kernel for */
+    DIFFQKV_ERR_MISALIGNED = 3,     /* a pointer is not 16-byte aligned */
+    DIFFQKV_ERR_WORKSPACE = 4,      /* workspace null or smaller than required */
+    DIFFQKV_ERR_CUDA = 5,           /* a CUDA runtime call or launch failed */
+    DIFFQKV_ERR_DEVICE_TIMEOUT = 6, /* a bounded device-side wait ran out */
+    DIFFQKV_ERR_DEVICE_SEQLEN = 7,  /* a device seq_len was < 0 or > t_max (clamped) */
+    DIFFQKV_ERR_NO_DEVICE = 8       /* no CUDA device / driver */
+} diffqkv_status_t;
+
+/* Human-readable name of a status code (static storage; never NULL). */
+const char *diffqkv_status_string(int32_t status);
+
+/* Library ABI version: major * 10000 + minor * 100 + patch. */
+int32_t diffqkv_version(void);
+
+/* ------------------------------------------------------------------------ */
+/* Split/combine decode (FlexHeadFA's split kernel + combine kernel, section */
+/* "FlexHeadFA Kernel and Deployment Infrastructure"; Steps 2-5 of 3.4).    */
+/* ------------------------------------------------------------------------ */
+
+/* Bytes of workspace diffqkv_decode needs for this shape (0 if dims are
+ * invalid).  Depends only on the dims, not on the device or the lengths.
+ * The workspace must be zero-filled before its FIRST use (cudaMemset, or
+ * diffqkv_workspace_init); every call that completes leaves it zero-filled
+ * again, so it can be reused without clearing.  Two calls that may run
+ * concurrently must not share a workspace. */
+size_t diffqkv_decode_workspace_size(const diffqkv_dims_t *dims);
+
+/* Zero-fill a workspace on `stream` (cudaMemsetAsync). */
+diffqkv_status_t diffqkv_workspace_init(void *workspace, size_t workspace_bytes,
+                                        diffqkv_stream_t stream);
+
+/*
+ * Decode attention of one query token per sequence over a KV cache.
+ *
+ *   q        [B, n_q, d_k]          query (already projected and rotated)
+ *   k_cache  [B, t_max, n_k, d_k]   K cache, token-major
+ *   v_cache  [B, t_max, n_v, d_v]   V cache, token-major, separate from K
+ *   seq_lens [B] int32 (device)     positions 0..seq_lens[b]-1 are attended
+ *   out      [B, n_q, d_v]          bf16 output (written, never read)
+ *
+ * out[b,h] = sum_j softmax_j(scale * q[b,h].k_cache[b,j,h/(n_q/n_k)])
+ *                   * v_cache[b,j,h/(n_q/n_v)],  j < seq_lens[b].
+ * A row with seq_lens[b] == 0 is written as zeros.  seq_lens[b] < 0 or
+ * > t_max is clamped into [0, t_max] and flagged DIFFQKV_ERR_DEVICE_SEQLEN.
+ * max_seq_len is a host-side upper bound of seq_lens (used only to size the
+ * grid; a wrong hint costs speed, never correctness); pass t_max if unknown.
+ * Each KV chunk produces (running max, sum of exp, unnormalised output)
+ * partials and the combine merges them; both run in ONE kernel launch.
+ */
+diffqkv_status_t diffqkv_decode(const diffqkv_dims_t *dims, const void *q, const void *k_cache,
+                                const void *v_cache, const int32_t *seq_lens, int32_t t_max,
+                                int32_t max_seq_len, void *out, void *workspace,
+                                size_t workspace_bytes, diffqkv_stream_t stream);
+
+/* Optional launch controls for diffqkv_decode_ex (0 = library default). */
+typedef struct {
+    int32_t grid_ctas;   /* CTAs of the split kernel (>= 1); changes the split points */
+    int32_t stages;      /* shared-memory pipeline depth (2..8) */
+    int32_t ctas_per_sm; /* resident CTAs per SM the default grid assumes (1..4) */
+} diffqkv_decode_tuning_t;
+
+/* diffqkv_decode with explicit launch controls (tuning may be NULL).  The
+ * result does not depend on the controls beyond fp32 rounding order. */
+diffqkv_status_t diffqkv_decode_ex(const diffqkv_dims_t *dims, const void *q, const void *k_cache,
+                                   const void *v_cache, const int32_t *seq_lens, int32_t t_max,
+                                   int32_t max_seq_len, void *out, void *workspace,
+                                   size_t workspace_bytes, const diffqkv_decode_tuning_t *tuning,
+                                   diffqkv_stream_t stream);
+
+/* Host-side launch plan of diffqkv_decode (no device needed; num_sms is the
+ * SM count to plan for).  Returns INVALID_ARG / UNSUPPORTED like the call. */
+typedef struct {
+    int32_t tile_tokens;     /* cached positions per pipeline stage */
+    int32_t stages;          /* pipeline depth */
+    int32_t grid_ctas;       /* split-kernel CTAs */
+    int32_t threads;         /* threads per CTA */
+    int32_t v_heads_per_tile;/* V heads one K-head group reads */
+    int64_t smem_bytes;      /* dynamic shared memory per CTA */
+    int64_t workspace_bytes; /* == diffqkv_decode_workspace_size */
+} diffqkv_decode_plan_t;
+
+diffqkv_status_t diffqkv_decode_plan(const diffqkv_dims_t *dims, int32_t t_max, int32_t max_seq_len,
+                                     int32_t num_sms, const diffqkv_decode_tuning_t *tuning,
+                                     diffqkv_decode_plan_t *plan);
+
+/*
+ * End-to-end decode from HOST buffers: copies q, k_cache, v_cache and
+ * seq_lens (host pointers, ideally pinned) into the caller's device buffers
+ * with one cudaMemcpyAsync each, runs diffqkv_decode, and copies the bf16
+ * output back into out_host, all on `stream`.  The caller synchronises the
+ * stream before reading out_host.  Device buffers follow diffqkv_decode's
+ * layouts; host buffers the same layouts.
+ */
+diffqkv_status_t diffqkv_decode_from_host(const diffqkv_dims_t *dims, const void *q_host,
+                                          const void *k_cache_host, const void *v_cache_host,
+                                          const int32_t *seq_lens_host, int32_t t_max,
+                                          int32_t max_seq_len, void *out_host, void *q_dev,
+                                          void *k_cache_dev, void *v_cache_dev,
+                                          int32_t *seq_lens_dev, void *out_dev, void *workspace,
+                                          size_t workspace_bytes, diffqkv_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Selective V fetch decode ("Selective V Cache Fetching": only the V rows  */
+/* of the top-k scoring positions are read; the softmax is renormalised    */
+/* over them).                                                              */
+/* ------------------------------------------------------------------------ */
+
+/* Workspace bytes for diffqkv_decode_topv (0 if invalid).  No zero-fill is
+ * required. */
+size_t diffqkv_decode_topv_workspace_size(const diffqkv_dims_t *dims, int32_t t_max, int32_t topk);
+
+/*
+ * Per (b, h): S = the topk positions j < seq_lens[b] with the largest EXACT
+ * dot product q[b,h].k_cache[b,j,kh] (exact rational value, not a rounded
+ * one), ties broken toward the lower j; all positions if topk >= seq_lens[b].
+ *   out[b,h]     = sum_{j in S} e^{s_j - m} v[b,j,vh] / sum_{j in S} e^{s_j - m},
+ *                  s_j = scale * q.k_j, m = max_{j in S} s_j   (bf16 [B,n_q,d_v])
+ *   idx_out[b,h] = S in ascending order, padded with -1          (int32 [B,n_q,topk])
+ * Only the selected V rows are read from v_cache.  Inputs as diffqkv_decode;
+ * 1 <= topk <= 4096.
+ */
+diffqkv_status_t diffqkv_decode_topv(const diffqkv_dims_t *dims, const void *q, const void *k_cache,
+                                     const void *v_cache, const int32_t *seq_lens, int32_t t_max,
+                                     int32_t max_seq_len, int32_t topk, void *out,
+                                     int32_t *idx_out, void *workspace, size_t workspace_bytes,
+                                     diffqkv_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Causal prefill (the "prefix" phase the paper's efficiency study times)    */
+/* ------------------------------------------------------------------------ */
+
+/*
+ *   q   [B, S, n_q, d_k], k [B, S, n_k, d_k], v [B, S, n_v, d_v]   bf16
+ *   out [B, S, n_q, d_v]                                           bf16
+ * out[b,i,h] = sum_{j<=i} softmax_j(scale * q[b,i,h].k[b,j,kh]) v[b,j,vh].
+ * Runs on the tcgen05 tensor cores (TMEM accumulators, TMA-fed tiles).
+ * Requires S >= 1; d_k = 64 or 128, d_v = 64 or 128.
+ */
+diffqkv_status_t diffqkv_prefill_causal(const diffqkv_dims_t *dims, const void *q, const void *k,
+                                        const void *v, int32_t seq_len, void *out,
+                                        diffqkv_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Device error word                                                        */
+/* ------------------------------------------------------------------------ */
+
+/* Synchronises `stream`, returns (in *device_status) the first device-side
+ * error recorded on the current device since the last read (DIFFQKV_OK if
+ * none), and clears it.  The return value reports failures of the query. */
+diffqkv_status_t diffqkv_get_device_status(diffqkv_stream_t stream, int32_t *device_status);
+
+/* Launches a kernel that waits on a barrier nothing ever signals, with a
+ * bounded wait of `timeout_ns`, so callers can check that a wait that runs
+ * out ends with DIFFQKV_ERR_DEVICE_TIMEOUT in the device error word instead
+ * of a hang.  1e3 <= timeout_ns <= 5e9. */
+diffqkv_status_t diffqkv_selftest_wait_timeout(int64_t timeout_ns, diffqkv_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DIFFQKV_H_ */

@@ -1,0 +1,123 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol the
+header declares, plans launches, and rejects bad arguments before launching."""
+import ctypes
+
+import pytest
+
+import asymmetric_head_kv_b200 as ak
+from asymmetric_head_kv_b200 import _capi
+from asymmetric_head_kv_b200.build import build
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    build()
+
+
+def test_exports_every_declared_symbol():
+    lib = _capi.lib()
+    names = _capi.header_symbols()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(_capi.SIGNATURES), "binding and header disagree"
+
+
+def test_status_strings_and_version():
+    lib = _capi.lib()
+    for code, name in _capi.STATUS.items():
+        assert lib.diffqkv_status_string(code).decode() == name
+    assert lib.diffqkv_status_string(999).decode() == "DIFFQKV_ERR_UNKNOWN"
+    assert lib.diffqkv_version() >= 10000
+
+
+def dims(**kw):
+    base = dict(batch=16, n_q=16, n_k=4, n_v=16, d_k=64, d_v=128, scale=0.125)
+    base.update(kw)
+    return ak.make_dims(**base)
+
+
+def test_workspace_size_depends_only_on_dims():
+    lib = _capi.lib()
+    d = dims()
+    n = lib.diffqkv_decode_workspace_size(ctypes.byref(d))
+    assert n > 0 and n % 16 == 0
+    assert lib.diffqkv_decode_workspace_size(ctypes.byref(dims(batch=32))) > n
+    assert lib.diffqkv_decode_workspace_size(ctypes.byref(dims(n_k=3))) == 0   # 16 % 3 != 0
+    assert lib.diffqkv_decode_workspace_size(None) == 0
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(n_k=3), _capi.INVALID_ARG),
+    (dict(n_v=5), _capi.INVALID_ARG),
+    (dict(batch=0), _capi.INVALID_ARG),
+    (dict(scale=0.0), _capi.INVALID_ARG),
+    (dict(scale=float("nan")), _capi.INVALID_ARG),
+    (dict(d_k=96), _capi.UNSUPPORTED),
+    (dict(n_q=64, n_k=2, n_v=16), _capi.UNSUPPORTED),   # 32 query heads per K head
+])
+def test_plan_rejects_bad_shapes(kw, code):
+    with pytest.raises(ak.DiffqkvError) as e:
+        ak.decode_plan(dims(**kw), 32768, 32768, 148)
+    assert e.value.status == code
+
+
+@pytest.mark.parametrize("shape", [
+    dict(), dict(n_k=16, d_k=128), dict(n_q=32, n_k=4, n_v=16, d_v=64), dict(n_k=16, n_v=16, d_k=64, d_v=64),
+    dict(n_k=1, n_v=1), dict(n_k=8, n_v=2), dict(n_q=24, n_k=12, n_v=8),
+])
+def test_plan_fits_b200(shape):
+    p = ak.decode_plan(dims(**shape), 32768, 32768, 148)
+    assert 2 <= p["stages"] <= 8
+    assert p["smem_bytes"] <= 227 * 1024
+    assert 1 <= p["grid_ctas"] <= 148
+    assert p["tile_tokens"] in (16, 32, 64, 128)
+    assert p["threads"] % 32 == 0 and p["threads"] <= 1024
+
+
+def test_plan_grid_follows_context_and_override():
+    p = ak.decode_plan(dims(batch=1), 512, 512, 148)
+    assert p["grid_ctas"] == 4 * (512 // p["tile_tokens"])    # fewer tiles than SMs
+    p = ak.decode_plan(dims(), 32768, 32768, 148, {"grid_ctas": 7, "stages": 3, "ctas_per_sm": 0})
+    assert p["grid_ctas"] == 7 and p["stages"] == 3
+    with pytest.raises(ak.DiffqkvError):
+        ak.decode_plan(dims(), 32768, 32768, 148, {"grid_ctas": 5000, "stages": 0, "ctas_per_sm": 0})
+
+
+def test_v_heads_per_tile():
+    assert ak.decode_plan(dims(), 1024, 1024, 148)["v_heads_per_tile"] == 4
+    assert ak.decode_plan(dims(n_k=16, d_k=128), 1024, 1024, 148)["v_heads_per_tile"] == 1
+    assert ak.decode_plan(dims(n_k=8, n_v=2), 1024, 1024, 148)["v_heads_per_tile"] == 1
+    # n_q=24, n_k=12 (2 q-heads per K head), n_v=8 (3 per V head): group 1 spans V heads 0 and 1
+    assert ak.decode_plan(dims(n_q=24, n_k=12, n_v=8), 1024, 1024, 148)["v_heads_per_tile"] == 2
+    with pytest.raises(ak.DiffqkvError):   # 3 query heads per K head has no kernel
+        ak.decode_plan(dims(n_q=12, n_k=4, n_v=6), 1024, 1024, 148)
+
+
+def _decode_raw(d, q=0x1000, k=0x2000, v=0x3000, sl=0x4000, t_max=128, out=0x5000, ws=0x6000, ws_bytes=1 << 30):
+    return _capi.lib().diffqkv_decode(ctypes.byref(d), q, k, v, sl, t_max, t_max, out, ws, ws_bytes, None)
+
+
+def test_decode_rejects_before_launch():
+    d = dims()
+    assert _decode_raw(d, q=None) == _capi.INVALID_ARG
+    assert _decode_raw(d, t_max=0) == _capi.INVALID_ARG
+    assert _decode_raw(d, q=0x1008) == _capi.MISALIGNED
+    assert _decode_raw(d, out=0x5004) == _capi.MISALIGNED
+    assert _decode_raw(d, ws=None) == _capi.WORKSPACE
+    assert _decode_raw(d, ws_bytes=16) == _capi.WORKSPACE
+    assert _decode_raw(dims(n_k=3)) == _capi.INVALID_ARG
+
+
+def test_prefill_and_topv_reject_null():
+    lib = _capi.lib()
+    d = dims()
+    assert lib.diffqkv_prefill_causal(ctypes.byref(d), None, None, None, 16, None, None) != _capi.OK
+    assert lib.diffqkv_decode_topv(ctypes.byref(d), None, None, None, None, 16, 16, 4, None, None, None, 0,
+                                   None) != _capi.OK
+
+
+def test_selftest_and_status_reject_bad_args():
+    lib = _capi.lib()
+    assert lib.diffqkv_selftest_wait_timeout(10, None) == _capi.INVALID_ARG
+    assert lib.diffqkv_get_device_status(None, None) == _capi.INVALID_ARG
