@@ -21,6 +21,7 @@ from ._capi import DiffqkvError, Dims, DecodePlan, DecodeTuning, check, lib
 __all__ = [
     "decode", "decode_workspace", "decode_plan", "decode_from_host", "decode_topv", "decode_topv_workspace",
     "prefill_causal", "device_status", "selftest_wait_timeout", "DiffqkvError", "Dims", "library_path",
+    "decode_noalloc",
 ]
 
 library_path = _capi.LIB_PATH
@@ -192,3 +193,29 @@ def device_status(stream: Optional[torch.cuda.Stream] = None) -> int:
 
 def selftest_wait_timeout(timeout_ns: int, stream: Optional[torch.cuda.Stream] = None) -> None:
     check(lib().diffqkv_selftest_wait_timeout(int(timeout_ns), _stream_ptr(stream)), "diffqkv_selftest_wait_timeout")
+
+
+def decode_noalloc(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, seq_lens: torch.Tensor, *,
+                   scale: Optional[float] = None, max_seq_len: Optional[int] = None,
+                   out: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """:func:`decode` through ``diffqkv_decode_noalloc``: no workspace argument.
+
+    For callers that cannot hand the library device memory (plugin interfaces
+    that only pass inputs and outputs, servers that forbid device allocation
+    after start-up).  The library's built-in scratch array is shared by every
+    call: calls that can overlap on the GPU must be serialised.  Pass ``out``
+    to make the call itself allocate nothing on the Python side either.
+    """
+    _bf16_dev(q, "q", 3)
+    _bf16_dev(k_cache, "k_cache", 4)
+    _bf16_dev(v_cache, "v_cache", 4)
+    if seq_lens.dtype != torch.int32 or not seq_lens.is_cuda:
+        raise TypeError("seq_lens must be an int32 CUDA tensor")
+    dims, t_max = _decode_dims(q, k_cache, v_cache, scale)
+    if out is None:
+        out = torch.empty((dims.batch, dims.n_q, dims.d_v), dtype=torch.bfloat16, device=q.device)
+    msl = t_max if max_seq_len is None else int(max_seq_len)
+    st = lib().diffqkv_decode_noalloc(ctypes.byref(dims), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seq_lens),
+                                      t_max, msl, _ptr(out), _stream_ptr(stream))
+    check(st, "diffqkv_decode_noalloc")
+    return out

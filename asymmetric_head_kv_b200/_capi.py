@@ -23,8 +23,10 @@ STATUS = {
     6: "DIFFQKV_ERR_DEVICE_TIMEOUT",
     7: "DIFFQKV_ERR_DEVICE_SEQLEN",
     8: "DIFFQKV_ERR_NO_DEVICE",
+    9: "DIFFQKV_ERR_SCRATCH_LIMIT",
 }
-OK, INVALID_ARG, UNSUPPORTED, MISALIGNED, WORKSPACE, CUDA_ERR, DEVICE_TIMEOUT, DEVICE_SEQLEN, NO_DEVICE = range(9)
+(OK, INVALID_ARG, UNSUPPORTED, MISALIGNED, WORKSPACE, CUDA_ERR, DEVICE_TIMEOUT, DEVICE_SEQLEN, NO_DEVICE,
+ SCRATCH_LIMIT) = range(10)
 
 
 class Dims(ctypes.Structure):
@@ -84,6 +86,7 @@ SIGNATURES = {
     "diffqkv_prefill_causal": ([_DIMS, _P, _P, _P, _I32, _P, _P], _I32),
     "diffqkv_get_device_status": ([_P, ctypes.POINTER(_I32)], _I32),
     "diffqkv_selftest_wait_timeout": ([_I64, _P], _I32),
+    "diffqkv_decode_noalloc": ([_DIMS, _P, _P, _P, _P, _I32, _I32, _P, _P], _I32),
 }
 
 

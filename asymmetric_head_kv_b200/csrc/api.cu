@@ -148,6 +148,7 @@ const char *diffqkv_status_string(int32_t status) {
         case DIFFQKV_ERR_DEVICE_TIMEOUT: return "DIFFQKV_ERR_DEVICE_TIMEOUT";
         case DIFFQKV_ERR_DEVICE_SEQLEN: return "DIFFQKV_ERR_DEVICE_SEQLEN";
         case DIFFQKV_ERR_NO_DEVICE: return "DIFFQKV_ERR_NO_DEVICE";
+        case DIFFQKV_ERR_SCRATCH_LIMIT: return "DIFFQKV_ERR_SCRATCH_LIMIT";
         default: return "DIFFQKV_ERR_UNKNOWN";
     }
 }
@@ -257,6 +258,13 @@ diffqkv_status_t diffqkv_get_device_status(diffqkv_stream_t stream, int32_t *dev
 
 diffqkv_status_t diffqkv_selftest_wait_timeout(int64_t timeout_ns, diffqkv_stream_t stream) {
     return diffqkv::wait_timeout_selftest_launch(timeout_ns, (cudaStream_t)stream);
+}
+
+diffqkv_status_t diffqkv_decode_noalloc(const diffqkv_dims_t *dims, const void *q, const void *k_cache,
+                                        const void *v_cache, const int32_t *seq_lens, int32_t t_max,
+                                        int32_t max_seq_len, void *out, diffqkv_stream_t stream) {
+    return diffqkv::decode_noalloc_launch(dims, q, k_cache, v_cache, seq_lens, t_max, max_seq_len, out,
+                                          (cudaStream_t)stream);
 }
 
 }  // extern "C"

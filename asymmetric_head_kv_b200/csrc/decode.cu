@@ -28,6 +28,7 @@
 #include <math.h>
 
 #include <algorithm>
+#include <mutex>
 
 #include "common.cuh"
 #include "internal.h"
@@ -616,6 +617,109 @@ diffqkv_status_t decode_launch(const diffqkv_dims_t *d, const void *q, const voi
     a.scale_log2 = (float)((double)d->scale * 1.4426950408889634);
     a.wait_limit_ns = kWaitLimitNs;
 
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)plan.smem_bytes) != cudaSuccess)
+        return DIFFQKV_ERR_CUDA;
+    fn<<<plan.grid_ctas, plan.threads, plan.smem_bytes, stream>>>(tm_k, tm_v, a);
+    if (cudaGetLastError() != cudaSuccess) return DIFFQKV_ERR_CUDA;
+    return DIFFQKV_OK;
+}
+
+// ------------------------------------------------------------------ allocation-free variant
+//
+// The same split/combine kernel, with its scratch (split partials and per-unit
+// counters) in a file-scope device array instead of a caller workspace.
+
+static __device__ __align__(256) uint8_t g_decode_noalloc_scratch[DIFFQKV_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kNoAllocMaxDevices = 64;
+void *g_noalloc_scratch_ptr[kNoAllocMaxDevices];
+std::mutex g_noalloc_mutex;
+
+// Device address of the scratch array on the current device (looked up once per device).
+diffqkv_status_t noalloc_scratch(int device, uint8_t **ptr) {
+    if (device < 0 || device >= kNoAllocMaxDevices) return DIFFQKV_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_scratch_ptr[device]) {
+        void *p = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress((void **)&p, g_decode_noalloc_scratch);
+        if (e != cudaSuccess || !p) {
+            cudaGetLastError();
+            return DIFFQKV_ERR_CUDA;
+        }
+        g_noalloc_scratch_ptr[device] = p;
+    }
+    *ptr = static_cast<uint8_t *>(g_noalloc_scratch_ptr[device]);
+    return DIFFQKV_OK;
+}
+
+}  // namespace
+
+diffqkv_status_t decode_noalloc_launch(const diffqkv_dims_t *d, const void *q, const void *k_cache,
+                                       const void *v_cache, const int32_t *seq_lens, int32_t t_max,
+                                       int32_t max_seq_len, void *out, cudaStream_t stream) {
+    diffqkv_status_t st = validate_dims(d);
+    if (st != DIFFQKV_OK) return st;
+    if (!q || !k_cache || !v_cache || !seq_lens || !out || t_max < 1) return DIFFQKV_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
+        (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
+        return DIFFQKV_ERR_MISALIGNED;
+    DeviceInfo dev;
+    st = current_device_info(&dev);
+    if (st != DIFFQKV_OK) return st;
+    diffqkv_decode_plan_t plan;
+    st = decode_plan(d, t_max, max_seq_len, dev.num_sms, nullptr, &plan);
+    if (st != DIFFQKV_OK) return st;
+    const int qpk = d->n_q / d->n_k;
+    KernelFn fn = pick_kernel(d->d_k, d->d_v, qpk);
+    if (!fn) return DIFFQKV_ERR_UNSUPPORTED;
+
+    // scratch: header, one counter per unit, then partial slots u + c < units + grid
+    const size_t units = (size_t)d->batch * d->n_k;
+    const size_t counter_bytes = align_up(units * sizeof(uint32_t), 256);
+    const size_t need = kWorkspaceHeader + counter_bytes +
+                        (units + (size_t)plan.grid_ctas) * qpk * (d->d_v + kPartialPad) * sizeof(float);
+    if (need > (size_t)DIFFQKV_NOALLOC_SCRATCH_BYTES) return DIFFQKV_ERR_SCRATCH_LIMIT;
+    uint8_t *scratch = nullptr;
+    st = noalloc_scratch(dev.device, &scratch);
+    if (st != DIFFQKV_OK) return st;
+
+    CUtensorMap tm_k, tm_v;
+    st = make_tensor_map_4d(&tm_k, k_cache, d->d_k, d->n_k, t_max, d->batch, d->d_k, 1, plan.tile_tokens, 1,
+                            CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (st != DIFFQKV_OK) return st;
+    st = make_tensor_map_4d(&tm_v, v_cache, d->d_v, d->n_v, t_max, d->batch, d->d_v, plan.v_heads_per_tile,
+                            plan.tile_tokens, 1, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (st != DIFFQKV_OK) return st;
+
+    DecodeArgs a;
+    a.q = static_cast<const __nv_bfloat16 *>(q);
+    a.seq_lens = seq_lens;
+    a.out = static_cast<__nv_bfloat16 *>(out);
+    a.counters = reinterpret_cast<uint32_t *>(scratch + kWorkspaceHeader);
+    a.partials = reinterpret_cast<float *>(scratch + kWorkspaceHeader + counter_bytes);
+    a.status = dev.status_word;
+    a.batch = d->batch;
+    a.n_q = d->n_q;
+    a.n_k = d->n_k;
+    a.n_v = d->n_v;
+    a.t_max = t_max;
+    a.vpg = plan.v_heads_per_tile;
+    a.q_per_v = d->n_q / d->n_v;
+    a.stages = plan.stages;
+    a.grid = plan.grid_ctas;
+    a.k_tile_bytes = (uint32_t)plan.tile_tokens * d->d_k * 2;
+    a.stage_bytes = a.k_tile_bytes + (uint32_t)plan.tile_tokens * plan.v_heads_per_tile * d->d_v * 2;
+    a.stage_stride = (uint32_t)align_up(a.stage_bytes, 1024);
+    a.scale_log2 = (float)((double)d->scale * 1.4426950408889634);
+    a.wait_limit_ns = kWaitLimitNs;
+
+    // the counters must start at zero whatever an earlier call left behind
+    if (cudaMemsetAsync(a.counters, 0, units * sizeof(uint32_t), stream) != cudaSuccess) {
+        cudaGetLastError();
+        return DIFFQKV_ERR_CUDA;
+    }
     if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)plan.smem_bytes) != cudaSuccess)
         return DIFFQKV_ERR_CUDA;
     fn<<<plan.grid_ctas, plan.threads, plan.smem_bytes, stream>>>(tm_k, tm_v, a);

@@ -47,6 +47,10 @@ diffqkv_status_t decode_launch(const diffqkv_dims_t *d, const void *q, const voi
                                int32_t max_seq_len, void *out, void *workspace, size_t workspace_bytes,
                                const diffqkv_decode_tuning_t *tuning, cudaStream_t stream);
 
+diffqkv_status_t decode_noalloc_launch(const diffqkv_dims_t *d, const void *q, const void *k_cache,
+                                       const void *v_cache, const int32_t *seq_lens, int32_t t_max,
+                                       int32_t max_seq_len, void *out, cudaStream_t stream);
+
 // topv.cu
 size_t topv_workspace_size(const diffqkv_dims_t *d, int32_t t_max, int32_t topk);
 diffqkv_status_t topv_launch(const diffqkv_dims_t *d, const void *q, const void *k_cache, const void *v_cache,

@@ -63,7 +63,8 @@ typedef enum {
     DIFFQKV_ERR_CUDA = 5,           /* a CUDA runtime call or launch failed */
     DIFFQKV_ERR_DEVICE_TIMEOUT = 6, /* a bounded device-side wait ran out */
     DIFFQKV_ERR_DEVICE_SEQLEN = 7,  /* a device seq_len was < 0 or > t_max (clamped) */
-    DIFFQKV_ERR_NO_DEVICE = 8       /* no CUDA device / driver */
+    DIFFQKV_ERR_NO_DEVICE = 8,      /* no CUDA device / driver */
+    DIFFQKV_ERR_SCRATCH_LIMIT = 9   /* shape needs more than the built-in scratch of diffqkv_decode_noalloc */
 } diffqkv_status_t;
 
 /* Human-readable name of a status code (static storage; never NULL). */
@@ -214,6 +215,43 @@ diffqkv_status_t diffqkv_get_device_status(diffqkv_stream_t stream, int32_t *dev
  * out ends with DIFFQKV_ERR_DEVICE_TIMEOUT in the device error word instead
  * of a hang.  1e3 <= timeout_ns <= 5e9. */
 diffqkv_status_t diffqkv_selftest_wait_timeout(int64_t timeout_ns, diffqkv_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Allocation-free decode (no counterpart in the paper)                      */
+/* ------------------------------------------------------------------------ */
+
+/* Size of the scratch buffer built into the library for diffqkv_decode_noalloc.
+ * Every GPU that loads the library holds this much device memory until the
+ * process exits. */
+#define DIFFQKV_NOALLOC_SCRATCH_BYTES (8u << 20) /* 8 MiB */
+
+/*
+ * diffqkv_decode without a workspace argument, for callers that cannot hand
+ * the library device memory: plugin interfaces whose enqueue step receives
+ * only input and output buffers, and servers that forbid device allocation
+ * after start-up (cudaMalloc synchronises the device and carves up a pool the
+ * caller has already reserved).  The split partials and per-unit counters live
+ * in a static device array of DIFFQKV_NOALLOC_SCRATCH_BYTES inside the
+ * library instead; the call allocates and frees nothing.
+ *
+ * Arguments, layouts and results are those of diffqkv_decode.
+ * - A shape whose scratch (split partials for batch * n_k units plus one
+ *   per CTA, and batch * n_k counters) exceeds the array returns
+ *   DIFFQKV_ERR_SCRATCH_LIMIT before anything is launched.  With the paper's
+ *   decode shape (n_q 16, n_k 4, n_v 16, d_v 128) on a 148-SM B200 that
+ *   allows batch <= 954.
+ * - The first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress, with that device current) and caches it; make that
+ *   first call before any stream capture on the device.
+ * - Every call uses the same array, which keeps whatever the last call left
+ *   there; each call clears the counters on `stream` before its kernel.
+ *   Calls whose execution can overlap on the GPU (different streams, or
+ *   concurrent host threads) race on the array and give wrong results:
+ *   serialise them.
+ */
+diffqkv_status_t diffqkv_decode_noalloc(const diffqkv_dims_t *dims, const void *q, const void *k_cache,
+                                        const void *v_cache, const int32_t *seq_lens, int32_t t_max,
+                                        int32_t max_seq_len, void *out, diffqkv_stream_t stream);
 
 #ifdef __cplusplus
 }

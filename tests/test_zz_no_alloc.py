@@ -1,0 +1,56 @@
+"""diffqkv_decode_noalloc: decode for callers that cannot allocate device memory.
+
+Some callers cannot hand the library a workspace: plugin interfaces whose
+enqueue step receives only input and output buffers, and servers that forbid
+cudaMalloc after start-up (it synchronises the device and carves up a pool
+that is already reserved).  This entry point keeps its scratch in a static
+device array inside the library.  Its results must equal those of
+diffqkv_decode, the workspace-based entry point, call after call, because the
+shared array keeps the previous call's contents.
+
+This file is named to be collected last, so a run that stops at the first
+failure has already run every other test; it also passes on its own in a fresh
+process (the first call on the device performs the array's address lookup).
+"""
+import ctypes
+
+import pytest
+import torch
+
+import asymmetric_head_kv_b200 as ak
+import workloads as wl
+from asymmetric_head_kv_b200 import _capi
+from parity import assert_parity
+
+pytestmark = pytest.mark.gpu
+
+
+def _inputs(batch, t_max, lens, seed, dev):
+    d = wl.random_decode_inputs(batch, t_max, wl.DIFFQKV, seed=seed, seq_lens=lens)
+    return {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
+
+
+def test_noalloc_matches_workspace_decode_on_consecutive_calls(cuda_device):
+    cases = [
+        (4, 3000, [3000, 1, 1777, 64], 201),              # call 1
+        (8, 5000, [5000, 4999, 0, 17, 2048, 333, 1, 4096], 202),  # call 2, different shape and lengths
+    ]
+    for call, (B, T, lens, seed) in enumerate(cases):
+        d = _inputs(B, T, lens, seed, cuda_device)
+        got = ak.decode_noalloc(d["q"], d["k_cache"], d["v_cache"], d["seq_lens"], scale=d["scale"])
+        torch.cuda.synchronize()
+        assert ak.device_status() == 0
+        ref = ak.decode(d["q"], d["k_cache"], d["v_cache"], d["seq_lens"], scale=d["scale"])
+        torch.cuda.synchronize()
+        assert_parity(got, ref.double().cpu().numpy(), f"noalloc call {call + 1}")
+
+
+def test_noalloc_rejects_shapes_beyond_its_scratch(cuda_device):
+    # batch 955 of the paper's decode shape needs more than the 8 MiB array on a 148-SM B200
+    sms = torch.cuda.get_device_properties(cuda_device).multi_processor_count
+    B = 955 if sms == 148 else 4096
+    dims = ak.make_dims(B, 16, 4, 16, 64, 128, 0.125)
+    fake = 1 << 20   # aligned, never dereferenced: the size check runs before any launch
+    st = _capi.lib().diffqkv_decode_noalloc(ctypes.byref(dims), fake, fake, fake, fake, 32768, 32768, fake, None)
+    assert st == _capi.SCRATCH_LIMIT
+    assert _capi.lib().diffqkv_status_string(st).decode() == "DIFFQKV_ERR_SCRATCH_LIMIT"
