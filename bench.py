@@ -40,8 +40,15 @@ UNIT = "GB/s"
 WORKLOAD = wl.DECODE_32K
 CONTROL = wl.DECODE_32K_GQA
 PROFILE = os.path.join(ROOT, "profiles", "decode_split_combine_b16_t32768.md")
-KERNEL_SOURCES = ["asymmetric_head_kv_b200/csrc/decode.cu", "asymmetric_head_kv_b200/csrc/common.cuh"]
+KERNEL_SOURCES = ["asymmetric_head_kv_b200/csrc/decode.cu", "asymmetric_head_kv_b200/csrc/common.cuh",
+                  "asymmetric_head_kv_b200/csrc/api.cu"]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+
+# Reduced cases for ncu captures: inputs larger than L2 (126 MB), a few GB at most.
+PROFILE_CASES = {
+    "decode_b4_t32768": wl.DecodeWorkload("decode_b4_t32768", wl.DIFFQKV, 4, 32768, seed=1),
+    "decode_gqa_b4_t32768": wl.DecodeWorkload("decode_gqa_b4_t32768", wl.GQA_CONTROL, 4, 32768, seed=1),
+}
 
 
 def parse():
@@ -52,6 +59,8 @@ def parse():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--e2e-steps", type=int, default=5)
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--profile-case", choices=sorted(PROFILE_CASES), default=None,
+                   help="run a few launches of one kernel on a reduced case for ncu; prints no bench line")
     return p.parse_args()
 
 
@@ -285,8 +294,24 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
+def run_profile_case(name: str, launches: int = 4):
+    import asymmetric_head_kv_b200 as ak
+
+    w = PROFILE_CASES[name]
+    d = wl.make_decode_inputs(w, torch.device("cuda", 0))
+    ws = ak.decode_workspace(d["q"], d["k_cache"], d["v_cache"])
+    for _ in range(launches):
+        ak.decode(d["q"], d["k_cache"], d["v_cache"], d["seq_lens"], scale=d["scale"], workspace=ws)
+    torch.cuda.synchronize()
+    assert ak.device_status() == 0
+    print(f"profile case {name}: {launches} launches, kv bytes/launch {wl.decode_kv_bytes(w.shape, d['seq_lens'])}")
+
+
 def main():
     args = parse()
+    if args.profile_case:
+        run_profile_case(args.profile_case)
+        return
     world, rank, local = dist_setup(args)
     if args.impl == "reference":
         run_reference(args, world, rank)
