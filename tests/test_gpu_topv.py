@@ -1,0 +1,121 @@
+"""GPU parity of selective-V decode (through the C ABI) against the fp64 oracle.
+
+Index sets must match bit-exactly (exact dot products, ties toward the lower
+position); outputs within the bf16 parity tolerance."""
+import numpy as np
+import pytest
+import torch
+
+import asymmetric_head_kv_b200 as ak
+import oracle
+import workloads as wl
+from workloads import Shape
+from parity import assert_parity
+
+pytestmark = pytest.mark.gpu
+
+
+def _gpu(d, topk, dev, **kw):
+    g = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
+    out, idx = ak.decode_topv(g["q"], g["k_cache"], g["v_cache"], g["seq_lens"], topk, scale=d["scale"], **kw)
+    torch.cuda.synchronize()
+    assert ak.device_status() == 0
+    return out, idx
+
+
+def _check(d, topk, dev, what, **kw):
+    out, idx = _gpu(d, topk, dev, **kw)
+    r_out, r_idx = oracle.decode_topv(d["q"], d["k_cache"], d["v_cache"], d["seq_lens"], topk, d["scale"])
+    got = idx.cpu().numpy()
+    bad = np.argwhere((got != r_idx).any(axis=-1))
+    assert bad.size == 0, f"{what}: index sets differ for (b, h) {bad[:5].tolist()}"
+    assert_parity(out, r_out, what)
+    return out, idx
+
+
+@pytest.mark.parametrize("name,shape", [("diffqkv", wl.DIFFQKV), ("gqa", wl.GQA_CONTROL),
+                                        ("paper", wl.SIGMA_1P5B_PAPER), ("mha64", Shape(8, 8, 8, 64, 64)),
+                                        ("k_more_than_v", Shape(16, 8, 2, 64, 128))])
+def test_ragged_shapes(cuda_device, name, shape):
+    lens = [3000, 1, 100, 101, 2500]
+    d = wl.random_decode_inputs(len(lens), 3000, shape, seed=301, seq_lens=lens)
+    _check(d, 100, cuda_device, name)
+
+
+@pytest.mark.parametrize("topk", [1, 2, 7, 64, 1024, 2999, 3000, 5000])
+def test_topk_sizes(cuda_device, topk):
+    d = wl.random_decode_inputs(2, 3000, wl.DIFFQKV, seed=302, seq_lens=[3000, 1500])
+    out, idx = _check(d, topk, cuda_device, f"k={topk}")
+    if topk >= 3000:   # every position kept: plain decode, indices 0..T-1 then -1
+        full = oracle.decode(d["q"], d["k_cache"], d["v_cache"], d["seq_lens"], d["scale"])
+        assert_parity(out, full, "k >= T")
+        assert idx[0, 0, :3000].tolist() == list(range(3000))
+        assert torch.all(idx[1, :, 1500:] == -1)
+
+
+def test_empty_rows(cuda_device):
+    d = wl.random_decode_inputs(3, 200, wl.DIFFQKV, seed=303, seq_lens=[0, 200, 0])
+    out, idx = _check(d, 16, cuda_device, "empty rows")
+    assert torch.all(idx[0] == -1) and torch.all(out[0] == 0)
+
+
+def test_exact_ties_choose_lower_positions(cuda_device):
+    """Every cached key identical: all scores tie exactly; the kept set is 0..k-1
+    (thousands of ambiguous positions: the radix path of the exact select)."""
+    d = wl.random_decode_inputs(1, 5000, wl.DIFFQKV, seed=304)
+    d["k_cache"][:] = d["k_cache"][:, :1]
+    _, idx = _check(d, 1000, cuda_device, "all ties")
+    assert torch.all(idx[0, :, :] == torch.arange(1000, dtype=torch.int32, device=idx.device))
+
+
+def test_duplicate_rows_at_the_boundary(cuda_device):
+    d = wl.random_decode_inputs(1, 4000, wl.DIFFQKV, seed=305)
+    # copy a few rows many times so exact ties straddle the k-th position (pairwise path)
+    for src, dsts in ((11, range(100, 4000, 400)), (500, range(7, 4000, 333)), (1234, range(2, 4000, 97))):
+        for j in dsts:
+            d["k_cache"][0, j] = d["k_cache"][0, src]
+    for k in (5, 33, 40, 200):
+        _check(d, k, cuda_device, f"dup k={k}")
+
+
+def _near_tie_inputs(n_rows, seed):
+    """Keys whose exact dots differ by ~2^-30 relative: fp32 scores tie, exact order does not."""
+    s = wl.DIFFQKV
+    d = wl.random_decode_inputs(1, n_rows, s, seed=seed)
+    g = torch.Generator().manual_seed(seed)
+    q = d["q"][0].float()
+    q[:, 1] = 2.0 ** -30                    # tiny weight on component 1 for every head
+    d["q"][0] = q.to(torch.bfloat16)
+    base = d["k_cache"][0, 0].clone()
+    k = base.repeat(n_rows, 1, 1)
+    # component 1 takes small integer values: differences of 2^-30 .. 2^-27 in the dot
+    k[:, :, 1] = torch.randint(-8, 9, (n_rows, s.n_k), generator=g).to(torch.bfloat16)
+    d["k_cache"][0] = k
+    return d
+
+
+@pytest.mark.parametrize("n_rows,topk", [(50, 10), (3000, 700)])
+def test_near_ties_ordered_by_exact_value(cuda_device, n_rows, topk):
+    d = _near_tie_inputs(n_rows, 306)
+    _check(d, topk, cuda_device, f"near ties {n_rows}")
+
+
+def test_workspace_too_small_is_rejected(cuda_device):
+    d = wl.random_decode_inputs(1, 100, wl.DIFFQKV, seed=307)
+    g = {k: (v.to(cuda_device) if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
+    ws = torch.empty(64, dtype=torch.uint8, device=cuda_device)
+    with pytest.raises(ak.DiffqkvError) as e:
+        ak.decode_topv(g["q"], g["k_cache"], g["v_cache"], g["seq_lens"], 8, workspace=ws)
+    assert e.value.status == ak._capi.WORKSPACE
+
+
+def test_full_topv_workload(cuda_device):
+    w = wl.TOPV_64K
+    d = wl.make_decode_inputs(w, cuda_device)
+    out, idx = ak.decode_topv(d["q"], d["k_cache"], d["v_cache"], d["seq_lens"], w.topk, scale=d["scale"])
+    torch.cuda.synchronize()
+    assert ak.device_status() == 0
+    cpu = {k: (v.cpu() if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
+    r_out, r_idx = oracle.decode_topv(cpu["q"], cpu["k_cache"], cpu["v_cache"], cpu["seq_lens"], w.topk, d["scale"])
+    assert np.array_equal(idx.cpu().numpy(), r_idx)
+    assert_parity(out, r_out, w.name)
