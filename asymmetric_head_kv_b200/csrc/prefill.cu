@@ -1,10 +1,381 @@
-// prefill.cu -- causal prefill (placeholder until the kernels land).
+// prefill.cu -- causal DiffQKV prefill on the sm_100a tensor cores.
+//
+// out[b,i,h] = sum_{j<=i} softmax_j(scale q[b,i,h].k[b,j,kh]) v[b,j,vh],
+// kh = h/(n_q/n_k), vh = h/(n_q/n_v)  (Sigma paper, structured summary page,
+// section 3.4 Steps 3-5, with the causal lower-triangular mask of the prefix
+// phase).  Unlike decode this is a dense contraction, so it runs on tcgen05.
+//
+// One CTA = one 128-row query tile of one (batch, head); 64-position K/V tiles.
+//   warp 4      TMA producer: Q once, K/V tiles into a shared-memory ring
+//               (128-byte swizzle, the layout the MMA descriptors describe)
+//   warp 5      allocates 256 TMEM columns; lane 0 issues every tcgen05.mma:
+//               S = Q K^T (M128 N64, fp32 in TMEM, two S buffers) and
+//               O += P V (M128 N=d_v, fp32 in TMEM)
+//   warps 0-3   softmax: thread t owns query row t = TMEM lane t, so row max and
+//               row sum need no shuffles; P is written to shared memory as bf16
+//               in the K-major swizzled layout the PV MMA reads.  O is rescaled
+//               in TMEM only when a row maximum grows by more than 2^8 (the
+//               stale maximum is used consistently for O and the row sum, so
+//               the result is exact up to rounding).
+// Every mbarrier wait is bounded; CTAs are ordered heaviest (most K/V tiles)
+// first.  Two CTAs fit on one SM (104 KB smem, 256 TMEM columns each).
+#include <math.h>
+
 #include "common.cuh"
 #include "internal.h"
 
 namespace diffqkv {
-diffqkv_status_t prefill_launch(const diffqkv_dims_t *, const void *, const void *, const void *, int32_t, void *,
-                                cudaStream_t) {
-    return DIFFQKV_ERR_UNSUPPORTED;
+
+namespace {
+
+constexpr int BM = 128;             // query rows per CTA
+constexpr int BN = 64;              // K/V positions per tile
+constexpr int kThreads = 192;       // 4 softmax warps, producer, MMA
+constexpr int kTmemCols = 256;      // S0 | S1 | O
+constexpr float kRescaleLog2 = 8.f; // lazy O rescale threshold (log2 domain)
+
+template <int DK, int DV>
+struct Cfg {
+    static constexpr int KB = DK / 64;                 // 64-wide swizzle blocks along d_k
+    static constexpr int VB = DV / 64;                 // ... along d_v
+    static constexpr int Q_BYTES = BM * DK * 2;
+    static constexpr int K_BYTES = BN * DK * 2;
+    static constexpr int V_BYTES = BN * DV * 2;
+    static constexpr int P_BYTES = BM * BN * 2;
+    static constexpr int STAGES = DK == 64 ? 3 : 2;
+    static constexpr int STAGE_BYTES = K_BYTES + V_BYTES;
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_KV = Q_BYTES;
+    static constexpr int OFF_P = OFF_KV + STAGES * STAGE_BYTES;
+    static constexpr int OFF_BAR = OFF_P + P_BYTES;
+    static constexpr int SMEM = OFF_BAR + 256 + 1024;  // barriers/flags + alignment slack
+};
+
+struct PrefillArgs {
+    __nv_bfloat16 *out;
+    int32_t *status;
+    int32_t batch, seq, n_q, n_k, n_v, q_per_k, q_per_v, n_qtiles;
+    float scale_log2;
+    uint64_t wait_limit_ns;
+};
+
+template <int DK, int DV>
+__global__ void __launch_bounds__(kThreads, 2)
+    prefill_causal_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                          const __grid_constant__ CUtensorMap tm_v, const PrefillArgs a) {
+    using C = Cfg<DK, DV>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
+    uint64_t *kv_full = bars;                 // [STAGES]
+    uint64_t *kv_empty = bars + 4;            // [STAGES]
+    uint64_t *q_full = bars + 8;
+    uint64_t *s_full = bars + 9;              // [2]
+    uint64_t *s_free = bars + 11;             // [2]
+    uint64_t *p_full = bars + 13;
+    uint64_t *pv_done = bars + 14;
+    uint64_t *mma_done = bars + 15;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 16);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 17);
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+
+    // heaviest tiles first: query tile index descends with blockIdx
+    const int bh_count = a.batch * a.n_q;
+    const int qt = a.n_qtiles - 1 - (int)(blockIdx.x / bh_count);
+    const int bh = (int)(blockIdx.x % bh_count);
+    const int b = bh / a.n_q;
+    const int h = bh % a.n_q;
+    const int kh = h / a.q_per_k;
+    const int vh = h / a.q_per_v;
+    const int row0 = qt * BM;
+    const int kv_tiles_total = (a.seq + BN - 1) / BN;
+    const int n_kv = min(kv_tiles_total, (row0 + BM + BN - 1) / BN);
+
+    if (tid == 0) {
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(&kv_full[s], 1);
+            mbar_init(&kv_empty[s], 1);
+        }
+        mbar_init(q_full, 1);
+        mbar_init(&s_full[0], 1);
+        mbar_init(&s_full[1], 1);
+        mbar_init(&s_free[0], 4);
+        mbar_init(&s_free[1], 4);
+        mbar_init(p_full, 4);
+        mbar_init(pv_done, 1);
+        mbar_init(mma_done, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 5) {
+        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t t_s[2] = {tmem, tmem + BN};
+    const uint32_t t_o = tmem + 2 * BN;
+
+    if (warp == 4) {
+        // ======================= TMA producer
+        if (lane == 0) {
+            prefetch_tensormap(&tm_q);
+            prefetch_tensormap(&tm_k);
+            prefetch_tensormap(&tm_v);
+            mbar_arrive_expect_tx(q_full, C::Q_BYTES);
+#pragma unroll
+            for (int kb = 0; kb < C::KB; ++kb)
+                tma_load_4d(smem + C::OFF_Q + kb * (BM * 128), &tm_q, q_full, kb * 64, h, row0, b);
+            for (int n = 0; n < n_kv; ++n) {
+                const int st = n % C::STAGES;
+                if (n >= C::STAGES)
+                    mbar_wait_bounded(&kv_empty[st], (uint32_t)(((n / C::STAGES) - 1) & 1), a.wait_limit_ns,
+                                      abort_flag, a.status);
+                if (*abort_flag) break;
+                uint8_t *kdst = smem + C::OFF_KV + st * C::STAGE_BYTES;
+                uint8_t *vdst = kdst + C::K_BYTES;
+                mbar_arrive_expect_tx(&kv_full[st], C::STAGE_BYTES);
+#pragma unroll
+                for (int kb = 0; kb < C::KB; ++kb)
+                    tma_load_4d(kdst + kb * (BN * 128), &tm_k, &kv_full[st], kb * 64, kh, n * BN, b);
+#pragma unroll
+                for (int vb = 0; vb < C::VB; ++vb)
+                    tma_load_4d(vdst + vb * (BN * 128), &tm_v, &kv_full[st], vb * 64, vh, n * BN, b);
+            }
+            // drain: no copy may still be landing when the CTA exits
+            mbar_wait_bounded(q_full, 0, a.wait_limit_ns, nullptr, a.status);
+            for (int n = (n_kv > C::STAGES ? n_kv - C::STAGES : 0); n < n_kv; ++n)
+                mbar_wait_bounded(&kv_full[n % C::STAGES], (uint32_t)((n / C::STAGES) & 1), a.wait_limit_ns,
+                                  nullptr, a.status);
+        }
+    } else if (warp == 5) {
+        // ======================= MMA issuer (one thread)
+        if (lane == 0) {
+            constexpr uint32_t idesc_qk = umma_idesc_bf16(BM, BN, false, false);
+            constexpr uint32_t idesc_pv = umma_idesc_bf16(BM, DV, false, true);
+            const uint32_t q_addr = smem_addr(smem + C::OFF_Q);
+            const uint32_t p_addr = smem_addr(smem + C::OFF_P);
+            mbar_wait_bounded(q_full, 0, a.wait_limit_ns, abort_flag, a.status);
+            for (int n = 0; n <= n_kv; ++n) {
+                if (n < n_kv) {
+                    // S[n%2] = Q K_n^T
+                    const int st = n % C::STAGES;
+                    const int sb = n & 1;
+                    mbar_wait_bounded(&kv_full[st], (uint32_t)((n / C::STAGES) & 1), a.wait_limit_ns, abort_flag,
+                                      a.status);
+                    if (n >= 2)
+                        mbar_wait_bounded(&s_free[sb], (uint32_t)(((n >> 1) - 1) & 1), a.wait_limit_ns, abort_flag,
+                                          a.status);
+                    tc_fence_after();
+                    const uint32_t k_addr = smem_addr(smem + C::OFF_KV + st * C::STAGE_BYTES);
+#pragma unroll
+                    for (int ks = 0; ks < DK / 16; ++ks) {
+                        const uint32_t blk = (uint32_t)(ks >> 2), sub = (uint32_t)(ks & 3) * 32u;
+                        const uint64_t da = smem_desc_sw128(q_addr + blk * (BM * 128) + sub, 16, 1024);
+                        const uint64_t db = smem_desc_sw128(k_addr + blk * (BN * 128) + sub, 16, 1024);
+                        umma_bf16(t_s[sb], da, db, idesc_qk, ks > 0 ? 1u : 0u);
+                    }
+                    umma_commit(&s_full[sb]);
+                }
+                if (n >= 1) {
+                    // O += P_{n-1} V_{n-1}
+                    const int m = n - 1;
+                    const int st = m % C::STAGES;
+                    mbar_wait_bounded(p_full, (uint32_t)(m & 1), a.wait_limit_ns, abort_flag, a.status);
+                    tc_fence_after();
+                    const uint32_t v_addr = smem_addr(smem + C::OFF_KV + st * C::STAGE_BYTES + C::K_BYTES);
+#pragma unroll
+                    for (int ks = 0; ks < BN / 16; ++ks) {
+                        const uint64_t da = smem_desc_sw128(p_addr + (uint32_t)ks * 32u, 16, 1024);
+                        const uint64_t db = smem_desc_sw128(v_addr + (uint32_t)ks * (16 * 128), BN * 128, 1024);
+                        umma_bf16(t_o, da, db, idesc_pv, (m > 0 || ks > 0) ? 1u : 0u);
+                    }
+                    umma_commit(pv_done);
+                    umma_commit(&kv_empty[st]);
+                }
+            }
+            umma_commit(mma_done);
+            mbar_wait_bounded(mma_done, 0, a.wait_limit_ns, nullptr, a.status);
+        }
+    } else {
+        // ======================= softmax warps 0-3: thread tid owns query row row0 + tid
+        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        const int i = row0 + tid;  // query position of this thread's row
+        float m_used = -INFINITY;  // log2-domain maximum the stored O and l are relative to
+        float l = 0.f;
+        uint8_t *p_row = smem + C::OFF_P + (tid >> 3) * 1024 + (tid & 7) * 128;
+        for (int n = 0; n < n_kv; ++n) {
+            const int sb = n & 1;
+            mbar_wait_bounded(&s_full[sb], (uint32_t)((n >> 1) & 1), a.wait_limit_ns, abort_flag, a.status);
+            tc_fence_after();
+            float s[BN];
+            {
+                uint32_t r[32];
+                tmem_ld32(t_s[sb] + lane_base, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 32; ++c) s[c] = __uint_as_float(r[c]);
+                tmem_ld32(t_s[sb] + lane_base + 32, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 32; ++c) s[32 + c] = __uint_as_float(r[c]);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s_free[sb]);
+
+            // causal mask on tiles that reach past this row
+            const int j0 = n * BN;
+            if (j0 + BN - 1 > row0) {
+#pragma unroll
+                for (int c = 0; c < BN; ++c)
+                    if (j0 + c > i) s[c] = -INFINITY;
+            }
+            float mx = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < BN; ++c) mx = fmaxf(mx, s[c]);
+            const float m_new = mx * a.scale_log2;
+            bool waited_pv = false;
+            if (n == 0) {
+                m_used = m_new;
+            } else {
+                const bool need = m_new > m_used + kRescaleLog2;
+                if (__any_sync(0xffffffffu, need)) {
+                    // O must be final for tile n-1 before it is rescaled in TMEM
+                    mbar_wait_bounded(pv_done, (uint32_t)((n - 1) & 1), a.wait_limit_ns, abort_flag, a.status);
+                    waited_pv = true;
+                    tc_fence_after();
+                    const float alpha = need ? fast_exp2(m_used - m_new) : 1.f;
+#pragma unroll 1
+                    for (int c = 0; c < DV; c += 32) {
+                        uint32_t r[32];
+                        tmem_ld32(t_o + lane_base + c, r);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+                        tmem_st32(t_o + lane_base + c, r);
+                    }
+                    tmem_wait_st();
+                    if (need) {
+                        l *= alpha;
+                        m_used = m_new;
+                    }
+                }
+            }
+            // p = 2^(s * scale * log2 e - m_used), row sum, bf16 pack
+            const float neg_m = -m_used;
+            uint32_t pk[BN / 2];
+#pragma unroll
+            for (int c = 0; c < BN; c += 2) {
+                const float p0 = fast_exp2(fmaf(s[c], a.scale_log2, neg_m));
+                const float p1 = fast_exp2(fmaf(s[c + 1], a.scale_log2, neg_m));
+                l += p0 + p1;
+                pk[c >> 1] = pack_bf16x2(p0, p1);
+            }
+            if (n >= 1 && !waited_pv) {
+                // the previous P.V must have consumed the P buffer
+                mbar_wait_bounded(pv_done, (uint32_t)((n - 1) & 1), a.wait_limit_ns, abort_flag, a.status);
+            }
+            // row of P: 8 chunks of 16 bytes, 128-byte swizzle (chunk ^ row%8)
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                uint8_t *dst = p_row + ((c ^ (tid & 7)) << 4);
+                sts128(dst, pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(p_full);
+        }
+        // epilogue: O / l -> bf16
+        mbar_wait_bounded(pv_done, (uint32_t)((n_kv - 1) & 1), a.wait_limit_ns, abort_flag, a.status);
+        tc_fence_after();
+        const float inv_l = l > 0.f ? 1.f / l : 0.f;
+        __nv_bfloat16 *orow = a.out + (((size_t)b * a.seq + i) * a.n_q + h) * DV;
+#pragma unroll 1
+        for (int c = 0; c < DV; c += 32) {
+            uint32_t r[32];
+            tmem_ld32(t_o + lane_base + c, r);
+            tmem_wait_ld();
+            if (i < a.seq) {
+#pragma unroll
+                for (int e = 0; e < 32; e += 8) {
+                    uint4 v;
+                    v.x = pack_bf16x2(__uint_as_float(r[e]) * inv_l, __uint_as_float(r[e + 1]) * inv_l);
+                    v.y = pack_bf16x2(__uint_as_float(r[e + 2]) * inv_l, __uint_as_float(r[e + 3]) * inv_l);
+                    v.z = pack_bf16x2(__uint_as_float(r[e + 4]) * inv_l, __uint_as_float(r[e + 5]) * inv_l);
+                    v.w = pack_bf16x2(__uint_as_float(r[e + 6]) * inv_l, __uint_as_float(r[e + 7]) * inv_l);
+                    *reinterpret_cast<uint4 *>(orow + c + e) = v;
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 5) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
 }
+
+using PrefillFn = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, PrefillArgs);
+
+PrefillFn pick(int dk, int dv, int *smem) {
+    if (dk == 64 && dv == 64) { *smem = Cfg<64, 64>::SMEM; return prefill_causal_kernel<64, 64>; }
+    if (dk == 64 && dv == 128) { *smem = Cfg<64, 128>::SMEM; return prefill_causal_kernel<64, 128>; }
+    if (dk == 128 && dv == 64) { *smem = Cfg<128, 64>::SMEM; return prefill_causal_kernel<128, 64>; }
+    if (dk == 128 && dv == 128) { *smem = Cfg<128, 128>::SMEM; return prefill_causal_kernel<128, 128>; }
+    return nullptr;
+}
+
+}  // namespace
+
+diffqkv_status_t prefill_launch(const diffqkv_dims_t *d, const void *q, const void *k, const void *v, int32_t seq_len,
+                                void *out, cudaStream_t stream) {
+    diffqkv_status_t st = validate_dims(d);
+    if (st != DIFFQKV_OK) return st;
+    if (!q || !k || !v || !out || seq_len < 1) return DIFFQKV_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return DIFFQKV_ERR_MISALIGNED;
+    int smem = 0;
+    PrefillFn fn = pick(d->d_k, d->d_v, &smem);
+    if (!fn) return DIFFQKV_ERR_UNSUPPORTED;
+    DeviceInfo dev;
+    st = current_device_info(&dev);
+    if (st != DIFFQKV_OK) return st;
+
+    CUtensorMap tm_q, tm_k, tm_v;
+    st = make_tensor_map_4d(&tm_q, q, d->d_k, d->n_q, seq_len, d->batch, 64, 1, BM, 1, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != DIFFQKV_OK) return st;
+    st = make_tensor_map_4d(&tm_k, k, d->d_k, d->n_k, seq_len, d->batch, 64, 1, BN, 1, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != DIFFQKV_OK) return st;
+    st = make_tensor_map_4d(&tm_v, v, d->d_v, d->n_v, seq_len, d->batch, 64, 1, BN, 1, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != DIFFQKV_OK) return st;
+
+    PrefillArgs a;
+    a.out = static_cast<__nv_bfloat16 *>(out);
+    a.status = dev.status_word;
+    a.batch = d->batch;
+    a.seq = seq_len;
+    a.n_q = d->n_q;
+    a.n_k = d->n_k;
+    a.n_v = d->n_v;
+    a.q_per_k = d->n_q / d->n_k;
+    a.q_per_v = d->n_q / d->n_v;
+    a.n_qtiles = (seq_len + BM - 1) / BM;
+    a.scale_log2 = (float)((double)d->scale * 1.4426950408889634);
+    a.wait_limit_ns = kWaitLimitNs;
+    const long long grid = (long long)a.n_qtiles * d->batch * d->n_q;
+    if (grid > 0x7fffffffLL) return DIFFQKV_ERR_UNSUPPORTED;
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return DIFFQKV_ERR_CUDA;
+    fn<<<(unsigned)grid, kThreads, smem, stream>>>(tm_q, tm_k, tm_v, a);
+    if (cudaGetLastError() != cudaSuccess) return DIFFQKV_ERR_CUDA;
+    return DIFFQKV_OK;
+}
+
 }  // namespace diffqkv
