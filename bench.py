@@ -48,7 +48,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 PROFILE_CASES = {
     "decode_b4_t32768": wl.DecodeWorkload("decode_b4_t32768", wl.DIFFQKV, 4, 32768, seed=1),
     "decode_gqa_b4_t32768": wl.DecodeWorkload("decode_gqa_b4_t32768", wl.GQA_CONTROL, 4, 32768, seed=1),
+    "prefill_b2_s8192": wl.PREFILL_8K,
+    "topv_b4_t65536": wl.TOPV_64K,
 }
+L2_FLUSH_BYTES = 256 << 20  # written between timed calls whose inputs fit in the 126 MB L2
 
 
 def parse():
@@ -58,7 +61,6 @@ def parse():
     p.add_argument("--warmup", type=int, default=20)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--e2e-steps", type=int, default=5)
-    p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--profile-case", choices=sorted(PROFILE_CASES), default=None,
                    help="run a few launches of one kernel on a reduced case for ncu; prints no bench line")
     return p.parse_args()
@@ -298,13 +300,86 @@ def run_profile_case(name: str, launches: int = 4):
     import asymmetric_head_kv_b200 as ak
 
     w = PROFILE_CASES[name]
-    d = wl.make_decode_inputs(w, torch.device("cuda", 0))
-    ws = ak.decode_workspace(d["q"], d["k_cache"], d["v_cache"])
-    for _ in range(launches):
-        ak.decode(d["q"], d["k_cache"], d["v_cache"], d["seq_lens"], scale=d["scale"], workspace=ws)
+    dev = torch.device("cuda", 0)
+    if isinstance(w, wl.PrefillWorkload):
+        d = wl.make_prefill_inputs(w, dev)
+        out = torch.empty((w.batch, w.seq, w.shape.n_q, w.shape.d_v), dtype=torch.bfloat16, device=dev)
+        for _ in range(launches):
+            ak.prefill_causal(d["q"], d["k"], d["v"], scale=d["scale"], out=out)
+        what = f"causal flops/launch {wl.prefill_causal_flops(w.shape, w.batch, w.seq)}"
+    elif w.topk:
+        d = wl.make_decode_inputs(w, dev)
+        for _ in range(launches):
+            ak.decode_topv(d["q"], d["k_cache"], d["v_cache"], d["seq_lens"], w.topk, scale=d["scale"])
+        what = f"algorithmic bytes/launch {topv_bytes(w, d['seq_lens'])}"
+    else:
+        d = wl.make_decode_inputs(w, dev)
+        ws = ak.decode_workspace(d["q"], d["k_cache"], d["v_cache"])
+        for _ in range(launches):
+            ak.decode(d["q"], d["k_cache"], d["v_cache"], d["seq_lens"], scale=d["scale"], workspace=ws)
+        what = f"kv bytes/launch {wl.decode_kv_bytes(w.shape, d['seq_lens'])}"
     torch.cuda.synchronize()
     assert ak.device_status() == 0
-    print(f"profile case {name}: {launches} launches, kv bytes/launch {wl.decode_kv_bytes(w.shape, d['seq_lens'])}")
+    print(f"profile case {name}: {launches} launches, {what}")
+
+
+def topv_bytes(w: wl.DecodeWorkload, seq_lens) -> int:
+    """Selective-V algorithmic bytes: every cached K row once, plus the selected V rows."""
+    lens = torch.as_tensor(seq_lens, dtype=torch.int64).clamp(min=0)
+    k_bytes = int(lens.sum()) * w.shape.n_k * w.shape.d_k * 2
+    v_rows = int(lens.clamp(max=w.topk).sum()) * w.shape.n_q
+    return k_bytes + v_rows * w.shape.d_v * 2
+
+
+def _timed_calls(fn, steps: int, flush: torch.Tensor):
+    """Per-call CUDA-event times (ms) on the current stream, L2 flushed before every call."""
+    stream = torch.cuda.current_stream()
+    times = []
+    for _ in range(steps):
+        flush.add_(1)
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        fn()
+        e.record(stream)
+        times.append((s, e))
+    torch.cuda.synchronize()
+    return [s.elapsed_time(e) for s, e in times]
+
+
+def time_paths(ak, peaks, steps: int, warmup: int):
+    """Causal prefill (tensor cores) and selective-V decode, one call = one step of each."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    flush = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    res = {}
+    bf16_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    for w in (wl.PREFILL_8K, wl.PREFILL_8K_GQA):
+        d = wl.make_prefill_inputs(w, dev)
+        out = torch.empty((w.batch, w.seq, w.shape.n_q, w.shape.d_v), dtype=torch.bfloat16, device=dev)
+        fn = lambda: ak.prefill_causal(d["q"], d["k"], d["v"], scale=d["scale"], out=out)  # noqa: E731
+        for _ in range(max(3, warmup)):
+            fn()
+        ms = statistics.median(_timed_calls(fn, steps, flush))
+        flops = wl.prefill_causal_flops(w.shape, w.batch, w.seq)
+        tf = flops / (ms * 1e-3) / 1e12
+        res[w.name] = {"ms": ms, "causal_flops": flops, "tflops": tf, "bound": "tensor", "peak_tflops": bf16_peak,
+                       "frac": tf / bf16_peak, "peak_source": "bf16_tflops (burst, cuBLAS bf16 GEMM)"}
+        del d, out
+    w = wl.TOPV_64K
+    d = wl.make_decode_inputs(w, dev)
+    ws = ak.decode_topv_workspace(ak.make_dims(w.batch, w.shape.n_q, w.shape.n_k, w.shape.n_v, w.shape.d_k,
+                                               w.shape.d_v, w.shape.scale), w.t_max, w.topk, dev)
+    fn = lambda: ak.decode_topv(d["q"], d["k_cache"], d["v_cache"], d["seq_lens"], w.topk,  # noqa: E731
+                                scale=d["scale"], workspace=ws)
+    for _ in range(max(3, warmup)):
+        fn()
+    ms = statistics.median(_timed_calls(fn, steps, flush))
+    nbytes = topv_bytes(w, d["seq_lens"].cpu())
+    hbm = float(peaks["hbm_gbs"])
+    res[w.name] = {"us": ms * 1e3, "algorithmic_bytes": nbytes, "gbs": nbytes / (ms * 1e-3) / 1e9,
+                   "bound": "hbm", "peak_gbs": hbm, "frac": nbytes / (ms * 1e-3) / 1e9 / hbm,
+                   "launches_per_call": 2}
+    assert ak.device_status() == 0
+    return res
 
 
 def main():
@@ -353,8 +428,10 @@ def main():
            "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": args.e2e_steps,
            "api": "diffqkv_decode_from_host (pinned host buffers)"}
 
+    paths = time_paths(ak, peaks, max(10, min(50, args.steps // 10)), args.warmup)
+
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1:
         d_cpu = {k: (v.cpu() if isinstance(v, torch.Tensor) else v) for k, v in main_res["inputs"].items()}
         info = oracle_sample_rate(WORKLOAD, d_cpu, 15.0)
         cpu = {k: info[k] for k in ("value", "unit", "cores", "kind", "sample")}
@@ -372,6 +449,7 @@ def main():
                        "kv_bytes_per_gpu_step": main_res["kv_bytes"]},
             "pct_of_hbm_peak": 100.0 * achieved / peak,
             "gqa_control": control,
+            "paths": paths,
             "roofline": roofline,
             "cpu_baseline": cpu,
             "e2e": e2e,
