@@ -158,12 +158,19 @@ def dist_setup(args):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """Max of a per-rank scalar (device time) over all ranks."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def weak_scaling_value(bytes_per_rank: int, world: int, region_ms_max: float, steps: int) -> float:
+    """Whole-job GB/s: bytes every rank moved in one step, over the slowest rank's time per step."""
+    return bytes_per_rank * world / (region_ms_max / steps * 1e-3) / 1e9
 
 
 def barrier(world: int):
@@ -400,7 +407,7 @@ def main():
     region_ms = max_over_ranks(main_res["region_ms"], world)
     ms_per_step = region_ms / args.steps
     total_bytes = main_res["kv_bytes"] * world
-    value = total_bytes / (region_ms / args.steps * 1e-3) / 1e9
+    value = weak_scaling_value(main_res["kv_bytes"], world, region_ms, args.steps)
 
     launch_ms = main_res["launch_ms_mean"]
     achieved = main_res["kv_bytes"] / (launch_ms * 1e-3) / 1e9
