@@ -113,6 +113,38 @@ diffqkv_status_t make_tensor_map_3d(CUtensorMap *map, const void *base, uint64_t
     return r == CUDA_SUCCESS ? DIFFQKV_OK : DIFFQKV_ERR_INVALID_ARG;
 }
 
+diffqkv_status_t ensure_dynamic_smem(const void *kernel, int bytes) {
+    // cudaFuncSetAttribute costs host time on every call; remember what each
+    // (kernel, device) pair has already been given
+    struct Entry {
+        const void *fn;
+        int device;
+        int bytes;
+    };
+    static Entry cache[256];
+    static int used = 0;
+    static std::mutex m;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return DIFFQKV_ERR_NO_DEVICE;
+    }
+    std::lock_guard<std::mutex> lock(m);
+    for (int i = 0; i < used; ++i)
+        if (cache[i].fn == kernel && cache[i].device == dev && cache[i].bytes >= bytes) return DIFFQKV_OK;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) {
+        cudaGetLastError();
+        return DIFFQKV_ERR_CUDA;
+    }
+    for (int i = 0; i < used; ++i)
+        if (cache[i].fn == kernel && cache[i].device == dev) {
+            cache[i].bytes = bytes;
+            return DIFFQKV_OK;
+        }
+    if (used < 256) cache[used++] = Entry{kernel, dev, bytes};
+    return DIFFQKV_OK;
+}
+
 diffqkv_status_t validate_dims(const diffqkv_dims_t *d) {
     if (!d) return DIFFQKV_ERR_INVALID_ARG;
     if (d->batch < 1 || d->n_q < 1 || d->n_k < 1 || d->n_v < 1 || d->d_k < 1 || d->d_v < 1)

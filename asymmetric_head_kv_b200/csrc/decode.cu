@@ -617,8 +617,7 @@ diffqkv_status_t decode_launch(const diffqkv_dims_t *d, const void *q, const voi
     a.scale_log2 = (float)((double)d->scale * 1.4426950408889634);
     a.wait_limit_ns = kWaitLimitNs;
 
-    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)plan.smem_bytes) != cudaSuccess)
-        return DIFFQKV_ERR_CUDA;
+    if (ensure_dynamic_smem((const void *)fn, (int)plan.smem_bytes) != DIFFQKV_OK) return DIFFQKV_ERR_CUDA;
     fn<<<plan.grid_ctas, plan.threads, plan.smem_bytes, stream>>>(tm_k, tm_v, a);
     if (cudaGetLastError() != cudaSuccess) return DIFFQKV_ERR_CUDA;
     return DIFFQKV_OK;
@@ -720,8 +719,7 @@ diffqkv_status_t decode_noalloc_launch(const diffqkv_dims_t *d, const void *q, c
         cudaGetLastError();
         return DIFFQKV_ERR_CUDA;
     }
-    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)plan.smem_bytes) != cudaSuccess)
-        return DIFFQKV_ERR_CUDA;
+    if (ensure_dynamic_smem((const void *)fn, (int)plan.smem_bytes) != DIFFQKV_OK) return DIFFQKV_ERR_CUDA;
     fn<<<plan.grid_ctas, plan.threads, plan.smem_bytes, stream>>>(tm_k, tm_v, a);
     if (cudaGetLastError() != cudaSuccess) return DIFFQKV_ERR_CUDA;
     return DIFFQKV_OK;

@@ -35,6 +35,9 @@ diffqkv_status_t make_tensor_map_3d(CUtensorMap *map, const void *base, uint64_t
 
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Sets a kernel's dynamic shared-memory limit once per (kernel, device).
+diffqkv_status_t ensure_dynamic_smem(const void *kernel, int bytes);
+
 // Shape checks common to every entry point.
 diffqkv_status_t validate_dims(const diffqkv_dims_t *d);
 

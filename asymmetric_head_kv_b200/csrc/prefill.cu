@@ -371,8 +371,7 @@ diffqkv_status_t prefill_launch(const diffqkv_dims_t *d, const void *q, const vo
     a.wait_limit_ns = kWaitLimitNs;
     const long long grid = (long long)a.n_qtiles * d->batch * d->n_q;
     if (grid > 0x7fffffffLL) return DIFFQKV_ERR_UNSUPPORTED;
-    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-        return DIFFQKV_ERR_CUDA;
+    if (ensure_dynamic_smem((const void *)fn, smem) != DIFFQKV_OK) return DIFFQKV_ERR_CUDA;
     fn<<<(unsigned)grid, kThreads, smem, stream>>>(tm_q, tm_k, tm_v, a);
     if (cudaGetLastError() != cudaSuccess) return DIFFQKV_ERR_CUDA;
     return DIFFQKV_OK;

@@ -7,23 +7,26 @@
 // ranked by the EXACT dot product q.k (ties toward the lower position) so the
 // selected set is unique and reproducible.
 //
-// Two launches:
-//  1. topv_score_kernel: streams K once (16-byte loads, one K row serves all
-//     n_q/n_k query heads of its group) and writes fp32 scores s_j = q.k_j
-//     (unscaled, fp32 FMA chain: every bf16 x bf16 product is exact) plus, per
-//     (batch, K head), the largest |k| element for the rounding bound.
-//  2. topv_select_kernel, one CTA per (batch, query head):
-//     a. tau = k-th largest fp32 score (3-pass radix select over the
-//        order-preserving integer image of the floats);
-//     b. rigorous bound d >= |s_j - e_j| for every j (e_j the exact dot):
-//        d = gamma_n * ||q||_1 * max|k| (gamma_n = n u / (1 - n u), u = 2^-24)
-//        plus n * 2^-149 for subnormal roundings;
-//     c. s_j > tau + 2d: certainly selected; s_j < tau - 2d: certainly not;
-//        the rest (usually a handful) get exact keys -- an integer
-//        superaccumulator of the products -- and the remaining slots go to the
-//        largest exact keys, lower position first on ties;
-//     d. selected positions are compacted in ascending order, and the
-//        renormalised softmax-weighted sum of exactly those V rows is written.
+// Three launches:
+//  1. topv_score_kernel -- streams K once with TMA (one K row serves all
+//     n_q/n_k query heads of its group; one position per thread) and writes
+//     fp32 scores s_j = q.k_j (unscaled fp32 FMA chain: every bf16 x bf16
+//     product is exact), a 2048-bucket histogram of the top 11 bits of each
+//     score's order key per row, and per (batch, K head) the largest |k|.
+//  2. topv_filter_kernel -- all SMs: per row, the histogram gives the bucket
+//     holding the k-th largest score; every position whose score is at least
+//     that bucket's lower end minus 2d (d the rounding bound below) is
+//     appended to the row's candidate list.  Everything else is certainly out.
+//  3. topv_select_kernel, one CTA per row, on the candidates in shared memory:
+//     a. tau = k-th largest fp32 score (radix select, byte by byte);
+//     b. d >= |s_j - e_j| for every j, e_j the exact dot product:
+//        d = 1.01 gamma_n ||q||_1 max|k| + n 2^-149, gamma_n = n u / (1 - n u), u = 2^-24;
+//     c. s_j > tau + 2d: certainly kept; s_j < tau - 2d: certainly not; the
+//        rest (usually a handful) get exact keys -- an integer superaccumulator
+//        of the products -- and the remaining slots go to the largest exact
+//        keys, the lower position first on ties;
+//     d. kept positions are marked in a bitmap and written in ascending order;
+//     e. the renormalised softmax-weighted sum of exactly those V rows is written.
 #include <math.h>
 
 #include <algorithm>
@@ -35,13 +38,20 @@ namespace diffqkv {
 
 namespace {
 
-constexpr int kScoreThreads = 256;
-constexpr int kScoreChunk = 2048;     // positions per score CTA iteration
-constexpr int kSelThreads = 1024;
+constexpr int kScoreThreads = 128;      // consumer threads of the score kernel (+1 producer warp)
+constexpr int kScoreTile = 128;         // positions per TMA tile (one per consumer thread)
+constexpr int kHistBuckets = 2048;      // first radix digit: top 11 bits of the order key
+constexpr int kRadixBuckets = 256;      // later radix digits: one byte
+constexpr int kFilterThreads = 256;
+constexpr int kFilterChunk = 4096;      // positions per filter CTA
+constexpr int kSelThreads = 512;
 constexpr int kSelWarps = kSelThreads / 32;
-constexpr int kPairwiseMax = 64;      // ambiguous sets up to this size are ranked pairwise
-constexpr int kKeyWords = 19;         // 18 superaccumulator digits + inverted position
+constexpr int kPairwiseMax = 64;        // ambiguous sets up to this size are ranked pairwise
+constexpr int kKeyWords = 19;           // 18 superaccumulator digits + inverted position
 constexpr int kTopvHeader = 256;
+constexpr int kCandCap = 12288;         // candidates held in shared memory by the select kernel
+constexpr int kSelCap = 4096;           // kept (position, score) pairs held in shared memory
+constexpr int kTopvMaxContext = 131072; // bitmap of kept positions: 16 KB of shared memory
 
 struct TopvArgs {
     const __nv_bfloat16 *q;
@@ -50,89 +60,23 @@ struct TopvArgs {
     const int32_t *seq_lens;
     __nv_bfloat16 *out;
     int32_t *idx_out;
-    float *scores;     // [B*n_q][t_max]
-    int32_t *alist;    // [B*n_q][t_max] ambiguous positions
-    uint8_t *flags;    // [B*n_q][t_max] 1 = selected
-    uint8_t *astate;   // [B*n_q][t_max] exact-select state of ambiguous entries
-    uint8_t *adigit;   // [B*n_q][t_max] current radix digit of ambiguous entries
-    uint32_t *kmax;    // [B*n_k] bf16 bit pattern of max |k|
+    float *scores;     // [B*n_q][t_pad]
+    int32_t *cand_j;   // [B*n_q][t_pad] candidate positions (filter -> select)
+    float *cand_s;     // [B*n_q][t_pad] their scores
+    int32_t *alist;    // [B*n_q][t_pad] ambiguous positions
+    uint8_t *astate;   // [B*n_q][t_pad] exact-select state of ambiguous entries
+    uint8_t *adigit;   // [B*n_q][t_pad] current radix digit of ambiguous entries
+    uint32_t *kmax;    // [B*n_k] bf16 bit pattern of max |k| (zeroed per call)
+    uint32_t *ghist;   // [B*n_q][2048] histogram of the top 11 bits of the score keys (zeroed per call)
+    uint32_t *ncand;   // [B*n_q] candidate counts (zeroed per call)
     int32_t *status;
-    int32_t batch, n_q, n_k, n_v, t_max, topk, q_per_k, q_per_v;
+    int32_t batch, n_q, n_k, n_v, t_max, t_pad, topk, q_per_k, q_per_v;
+    int32_t score_stages;
     float scale_log2;
+    uint64_t wait_limit_ns;
 };
 
 __device__ __forceinline__ int clamp_len(int v, int t_max) { return v < 0 ? 0 : (v > t_max ? t_max : v); }
-
-// ------------------------------------------------------------------ scores
-
-template <int DK, int QPK>
-__global__ void __launch_bounds__(kScoreThreads) topv_score_kernel(const TopvArgs a) {
-    constexpr int LPT = DK / 8;           // lanes per K row (16 bytes each)
-    constexpr int TPW = 32 / LPT;         // rows per warp per step
-    constexpr int NW = kScoreThreads / 32;
-    constexpr int UNROLL = 4;
-    const int unit = blockIdx.x;
-    const int b = unit / a.n_k;
-    const int g = unit % a.n_k;
-    const int T = clamp_len(__ldg(a.seq_lens + b), a.t_max);
-    const int lane = threadIdx.x & 31;
-    const int warp = threadIdx.x >> 5;
-    const int kc = lane % LPT;
-    const int kt = lane / LPT;
-
-    float qf[QPK][8];
-#pragma unroll
-    for (int h = 0; h < QPK; ++h) {
-        const uint4 qv = __ldg(reinterpret_cast<const uint4 *>(a.q + ((size_t)b * a.n_q + g * QPK + h) * DK) + kc);
-        unpack8(qv, qf[h]);
-    }
-    uint32_t kmx = 0;
-    const __nv_bfloat16 *kbase = a.k + (size_t)b * a.t_max * a.n_k * DK + (size_t)g * DK + kc * 8;
-    const size_t krow = (size_t)a.n_k * DK;
-    float *sbase = a.scores + ((size_t)b * a.n_q + g * QPK) * a.t_max;
-
-    for (int c0 = blockIdx.y * kScoreChunk; c0 < T; c0 += gridDim.y * kScoreChunk) {
-        const int c1 = min(T, c0 + kScoreChunk);
-        for (int base = c0 + warp * TPW; base < c1; base += NW * TPW * UNROLL) {
-            uint4 kv[UNROLL];
-#pragma unroll
-            for (int u = 0; u < UNROLL; ++u) {
-                const int j = base + u * NW * TPW + kt;
-                kv[u] = j < c1 ? __ldg(reinterpret_cast<const uint4 *>(kbase + (size_t)j * krow))
-                               : make_uint4(0, 0, 0, 0);
-            }
-#pragma unroll
-            for (int u = 0; u < UNROLL; ++u) {
-                const int j = base + u * NW * TPW + kt;
-                const uint32_t w[4] = {kv[u].x, kv[u].y, kv[u].z, kv[u].w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) kmx = max(kmx, max(w[e] & 0x7fffu, (w[e] >> 16) & 0x7fffu));
-                float kf[8];
-                unpack8(kv[u], kf);
-                float acc[QPK];
-#pragma unroll
-                for (int h = 0; h < QPK; ++h) {
-                    float s = 0.f;
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) s = fmaf(qf[h][e], kf[e], s);
-#pragma unroll
-                    for (int off = LPT / 2; off >= 1; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-                    acc[h] = s;
-                }
-                if (j < c1) {
-#pragma unroll
-                    for (int h = 0; h < QPK; ++h)
-                        if (h % LPT == kc) sbase[(size_t)h * a.t_max + j] = acc[h];
-                }
-            }
-        }
-    }
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) kmx = max(kmx, __shfl_xor_sync(0xffffffffu, kmx, off));
-    if (lane == 0) atomicMax(a.kmax + unit, kmx);
-}
-
-// ------------------------------------------------------------------ selection helpers
 
 // Order-preserving map of finite floats onto uint32 (larger float -> larger key).
 __device__ __forceinline__ uint32_t float_key(float f) {
@@ -143,6 +87,150 @@ __device__ __forceinline__ float key_float(uint32_t k) {
     return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
 }
 
+// Rigorous bound of |fp32 FMA-chain score - exact dot| for a row: every product
+// is exact, every one of the (at most n = d_k) additions a score sees rounds by
+// at most u relative (u = 2^-24) or, in the subnormal range, by 2^-150 absolute;
+// sum_c |q_c k_c| <= ||q||_1 max|k|.  1.01 covers the rounding of this formula.
+template <int DK>
+__device__ __forceinline__ float score_error_bound(float q_l1, float kmax) {
+    const double nu = (double)DK * 5.9604644775390625e-08;  // n * 2^-24
+    const float gamma = (float)(nu / (1.0 - nu));
+    return __fmul_ru(__fmul_ru(__fmul_ru(1.01f, gamma), q_l1), kmax) + (float)DK * 1.4012984643e-45f;
+}
+
+// ------------------------------------------------------------------ 1. scores
+
+// One CTA streams K tiles of one (batch, K head) over an equal share of its
+// positions: a producer thread issues TMA loads (128-byte swizzle, so a thread
+// reading "its" 128-byte row hits eight distinct 16-byte bank groups) into a
+// ring of tiles; each of the 128 consumer threads owns one position of the tile
+// and accumulates the dot products of all n_q/n_k query heads of the group,
+// with q read from shared memory by broadcast.
+template <int DK, int QPK>
+__global__ void __launch_bounds__(kScoreThreads + 32) topv_score_kernel(const __grid_constant__ CUtensorMap tm_k,
+                                                                         const TopvArgs a) {
+    constexpr int KB = DK / 64;  // 64-wide swizzle blocks per row
+    constexpr int TILE_BYTES = kScoreTile * DK * 2;
+    extern __shared__ uint8_t dsm_raw[];
+    uint8_t *dsm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *tiles = dsm;                                                                 // [stages][TILE_BYTES]
+    uint32_t *hist_s = reinterpret_cast<uint32_t *>(dsm + a.score_stages * TILE_BYTES);  // [QPK][2048]
+    float *q_s = reinterpret_cast<float *>(hist_s + QPK * kHistBuckets);                 // [QPK][DK]
+    uint64_t *full_bar = reinterpret_cast<uint64_t *>(q_s + QPK * DK);
+    uint64_t *empty_bar = full_bar + a.score_stages;
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(empty_bar + a.score_stages);
+
+    const int unit = blockIdx.x;
+    const int b = unit / a.n_k;
+    const int g = unit % a.n_k;
+    const int T = clamp_len(__ldg(a.seq_lens + b), a.t_max);
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    const int ntiles = (T + kScoreTile - 1) / kScoreTile;
+    const int tb = (int)(((long long)ntiles * blockIdx.y) / gridDim.y);
+    const int te = (int)(((long long)ntiles * (blockIdx.y + 1)) / gridDim.y);
+
+    if (tid == 0) {
+        for (int s = 0; s < a.score_stages; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&empty_bar[s], kScoreThreads / 32);
+        }
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    for (int i = tid; i < QPK * kHistBuckets; i += blockDim.x) hist_s[i] = 0;
+    for (int i = tid; i < QPK * DK; i += blockDim.x) {
+        const int hh = i / DK, c = i % DK;
+        q_s[i] = __bfloat162float(a.q[((size_t)b * a.n_q + g * QPK + hh) * DK + c]);
+    }
+    __syncthreads();
+
+    if (warp == kScoreThreads / 32) {
+        // ---- producer
+        if (lane == 0 && te > tb) {
+            prefetch_tensormap(&tm_k);
+            for (int t = tb, k = 0; t < te; ++t, ++k) {
+                const int st = k % a.score_stages;
+                if (k >= a.score_stages)
+                    mbar_wait_bounded(&empty_bar[st], (uint32_t)(((k / a.score_stages) - 1) & 1), a.wait_limit_ns,
+                                      abort_flag, a.status);
+                if (*abort_flag) break;
+                uint8_t *dst = tiles + st * TILE_BYTES;
+                mbar_arrive_expect_tx(&full_bar[st], TILE_BYTES);
+#pragma unroll
+                for (int kb = 0; kb < KB; ++kb)
+                    tma_load_4d(dst + kb * (kScoreTile * 128), &tm_k, &full_bar[st], kb * 64, g, t * kScoreTile, b);
+            }
+            const int issued = te - tb;
+            for (int k = (issued > a.score_stages ? issued - a.score_stages : 0); k < issued; ++k)
+                mbar_wait_bounded(&full_bar[k % a.score_stages], (uint32_t)((k / a.score_stages) & 1),
+                                  a.wait_limit_ns, nullptr, a.status);
+        }
+    } else {
+        // ---- consumers: thread tid owns position tile * kScoreTile + tid
+        uint32_t kmx2 = 0;  // two packed |bf16| maxima
+        float *sbase = a.scores + ((size_t)b * a.n_q + g * QPK) * a.t_pad;
+        for (int t = tb, k = 0; t < te; ++t, ++k) {
+            const int st = k % a.score_stages;
+            mbar_wait_bounded(&full_bar[st], (uint32_t)((k / a.score_stages) & 1), a.wait_limit_ns, abort_flag,
+                              a.status);
+            const uint8_t *row = tiles + st * TILE_BYTES + tid * 128;
+            const int j = t * kScoreTile + tid;
+            const uint32_t live = j < T ? 0x7fff7fffu : 0u;  // the |k| bound covers cached positions only
+            float acc[QPK];
+#pragma unroll
+            for (int hh = 0; hh < QPK; ++hh) acc[hh] = 0.f;
+#pragma unroll
+            for (int kb = 0; kb < KB; ++kb) {
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const uint4 kv = lds128(row + kb * (kScoreTile * 128) + ((c ^ (tid & 7)) << 4));
+                    kmx2 = __vmaxu2(kmx2, kv.x & live);
+                    kmx2 = __vmaxu2(kmx2, kv.y & live);
+                    kmx2 = __vmaxu2(kmx2, kv.z & live);
+                    kmx2 = __vmaxu2(kmx2, kv.w & live);
+                    float kf[8];
+                    unpack8(kv, kf);
+#pragma unroll
+                    for (int hh = 0; hh < QPK; ++hh) {
+                        const float4 qa = *reinterpret_cast<const float4 *>(q_s + hh * DK + kb * 64 + c * 8);
+                        const float4 qb = *reinterpret_cast<const float4 *>(q_s + hh * DK + kb * 64 + c * 8 + 4);
+                        float x = acc[hh];
+                        x = fmaf(qa.x, kf[0], x);
+                        x = fmaf(qa.y, kf[1], x);
+                        x = fmaf(qa.z, kf[2], x);
+                        x = fmaf(qa.w, kf[3], x);
+                        x = fmaf(qb.x, kf[4], x);
+                        x = fmaf(qb.y, kf[5], x);
+                        x = fmaf(qb.z, kf[6], x);
+                        x = fmaf(qb.w, kf[7], x);
+                        acc[hh] = x;
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty_bar[st]);
+            if (j < T) {
+#pragma unroll
+                for (int hh = 0; hh < QPK; ++hh) {
+                    sbase[(size_t)hh * a.t_pad + j] = acc[hh];
+                    atomicAdd(hist_s + hh * kHistBuckets + (float_key(acc[hh]) >> 21), 1u);
+                }
+            }
+        }
+        uint32_t kmx = max(kmx2 & 0xffffu, kmx2 >> 16);
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) kmx = max(kmx, __shfl_xor_sync(0xffffffffu, kmx, off));
+        if (lane == 0) atomicMax(a.kmax + unit, kmx);
+    }
+    __syncthreads();
+    uint32_t *gh = a.ghist + ((size_t)b * a.n_q + g * QPK) * kHistBuckets;
+    for (int i = tid; i < QPK * kHistBuckets; i += blockDim.x)
+        if (hist_s[i]) atomicAdd(gh + i, hist_s[i]);
+}
+
+// ------------------------------------------------------------------ helpers
+
 // Warp-aggregated shared-memory histogram increment; `bucket` < 0 skips.
 __device__ __forceinline__ void hist_add(uint32_t *hist, int bucket) {
     const unsigned peers = __match_any_sync(0xffffffffu, bucket);
@@ -150,20 +238,12 @@ __device__ __forceinline__ void hist_add(uint32_t *hist, int bucket) {
     if (bucket >= 0 && (threadIdx.x & 31) == leader) atomicAdd(hist + bucket, (uint32_t)__popc(peers));
 }
 
-// Block-wide: find the bucket d (counting from the highest bucket down) that
-// holds the kk-th largest element (kk >= 1), and the count strictly above it.
-// nb <= 2 * kSelThreads.  Results in *d_out / *above_out (shared).
-__device__ void find_bucket_from_top(const uint32_t *hist, int nb, uint32_t kk, int *d_out, uint32_t *above_out,
-                                     uint32_t *warp_sums) {
-    const int t = threadIdx.x;
-    const int hi = nb - 1 - 2 * t;
-    const int lo = hi - 1;
-    const uint32_t chi = hi >= 0 ? hist[hi] : 0u;
-    const uint32_t clo = lo >= 0 ? hist[lo] : 0u;
-    const uint32_t mine = chi + clo;
-    // exclusive scan over threads (thread 0 owns the top buckets)
-    uint32_t incl = mine;
-    const int lane = t & 31, warp = t >> 5;
+// Block-wide exclusive prefix sum of one value per thread (thread order).
+// warp_sums needs 33 entries; returns the exclusive prefix and writes the
+// block total to *total.
+__device__ uint32_t block_exclusive_scan(uint32_t v, uint32_t *warp_sums, uint32_t *total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    uint32_t incl = v;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
         const uint32_t y = __shfl_up_sync(0xffffffffu, incl, off);
@@ -172,24 +252,46 @@ __device__ void find_bucket_from_top(const uint32_t *hist, int nb, uint32_t kk, 
     if (lane == 31) warp_sums[warp] = incl;
     __syncthreads();
     if (warp == 0) {
-        uint32_t ws = warp_sums[lane];
+        const uint32_t ws = lane < nw ? warp_sums[lane] : 0u;
         uint32_t wi = ws;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
             const uint32_t y = __shfl_up_sync(0xffffffffu, wi, off);
             if (lane >= off) wi += y;
         }
-        warp_sums[lane] = wi - ws;  // exclusive prefix of warps
+        if (lane < nw) warp_sums[lane] = wi - ws;
+        if (lane == 31) warp_sums[32] = wi;
     }
     __syncthreads();
-    const uint32_t excl = warp_sums[warp] + incl - mine;
+    const uint32_t r = warp_sums[warp] + incl - v;
+    *total = warp_sums[32];
+    __syncthreads();
+    return r;
+}
+
+// Block-wide: the bucket d (counting from the top bucket down) that holds the
+// kk-th largest element (kk >= 1) of a histogram of nb buckets, and the count
+// strictly above it, into *d_out / *above_out (shared).  Thread t scans the
+// buckets [nb - (t+1)*span, nb - t*span) from the top down.
+__device__ void find_bucket_from_top(const uint32_t *hist, int nb, uint32_t kk, int *d_out, uint32_t *above_out,
+                                     uint32_t *warp_sums) {
+    const int span = (nb + blockDim.x - 1) / blockDim.x;
+    const int top = nb - 1 - (int)threadIdx.x * span;  // first (highest) bucket of this thread
+    uint32_t mine = 0;
+    for (int i = 0; i < span; ++i)
+        if (top - i >= 0) mine += hist[top - i];
+    uint32_t total;
+    const uint32_t excl = block_exclusive_scan(mine, warp_sums, &total);
     if (mine > 0 && excl < kk && kk <= excl + mine) {
-        if (excl + chi >= kk) {
-            *d_out = hi;
-            *above_out = excl;
-        } else {
-            *d_out = lo;
-            *above_out = excl + chi;
+        uint32_t above = excl;
+        for (int i = 0; i < span && top - i >= 0; ++i) {
+            const uint32_t c = hist[top - i];
+            if (above + c >= kk) {
+                *d_out = top - i;
+                *above_out = above;
+                break;
+            }
+            above += c;
         }
     }
     __syncthreads();
@@ -203,19 +305,28 @@ __device__ void find_bucket_from_top(const uint32_t *hist, int nb, uint32_t kk, 
 //   base-2^32 digits held in int64 slots, then carry-normalised.
 template <int DK>
 __device__ void exact_key(const uint16_t *qbits, const uint16_t *kbits, int j, uint32_t *out) {
+    // digit slots stay in registers: each product is added to its slot by a
+    // predicated add over the 16 slots a product can start in (offsets <= 506)
     long long acc[18];
 #pragma unroll
     for (int i = 0; i < 18; ++i) acc[i] = 0;
-    for (int c = 0; c < DK; ++c) {
-        const uint32_t qb = qbits[c], kb = kbits[c];
-        const int eq = (qb >> 7) & 0xff, ek = (kb >> 7) & 0xff;
-        const int mq = (qb & 0x7f) | (eq ? 0x80 : 0), mk = (kb & 0x7f) | (ek ? 0x80 : 0);
-        const long long P = (long long)(mq * mk);
-        if (P == 0) continue;
-        const int off = (eq ? eq - 134 : -133) + (ek ? ek - 134 : -133) + 266;
-        const long long v = P << (off & 31);
-        if ((qb ^ kb) & 0x8000u) acc[off >> 5] -= v;
-        else acc[off >> 5] += v;
+#pragma unroll 1
+    for (int c8 = 0; c8 < DK / 8; ++c8) {
+        const uint4 kw = *reinterpret_cast<const uint4 *>(kbits + 8 * c8);
+        const uint32_t words[4] = {kw.x, kw.y, kw.z, kw.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const uint32_t kb = (e & 1) ? (words[e >> 1] >> 16) : (words[e >> 1] & 0xffffu);
+            const uint32_t qb = qbits[8 * c8 + e];
+            const int eq = (qb >> 7) & 0xff, ek = (kb >> 7) & 0xff;
+            const int mq = (qb & 0x7f) | (eq ? 0x80 : 0), mk = (kb & 0x7f) | (ek ? 0x80 : 0);
+            const int off = (eq ? eq - 134 : -133) + (ek ? ek - 134 : -133) + 266;
+            long long v = (long long)(mq * mk) << (off & 31);
+            if ((qb ^ kb) & 0x8000u) v = -v;
+            const int slot = off >> 5;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) acc[i] += (slot == i) ? v : 0ll;
+        }
     }
 #pragma unroll
     for (int i = 0; i < 17; ++i) {
@@ -235,12 +346,108 @@ __device__ __forceinline__ bool key_greater(const uint32_t *x, const uint32_t *y
     return false;
 }
 
-// ------------------------------------------------------------------ select + gather
+// ||q||_1 of this row's query (every thread gets it; same summation order in all).
+template <int DK>
+__device__ float row_q_l1(const __nv_bfloat16 *q, float *red) {
+    float v = 0.f;
+    for (int c = threadIdx.x; c < DK; c += blockDim.x) v += fabsf(__bfloat162float(q[c]));
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+    __syncthreads();
+    float t = 0.f;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t += red[w];
+    __syncthreads();
+    return t;
+}
+
+// ------------------------------------------------------------------ 2. filter
+
+template <int DK>
+__global__ void __launch_bounds__(kFilterThreads) topv_filter_kernel(const TopvArgs a) {
+    __shared__ uint32_t warp_sums[33];
+    __shared__ float red[kFilterThreads / 32];
+    __shared__ __align__(16) uint32_t hist_s[kHistBuckets];  // filled with 16-byte stores
+    __shared__ int sh_d;
+    __shared__ uint32_t sh_above;
+    const int row = blockIdx.x;
+    const int b = row / a.n_q, h = row % a.n_q, g = h / a.q_per_k;
+    const int T = clamp_len(__ldg(a.seq_lens + b), a.t_max);
+    const int j_begin = blockIdx.y * kFilterChunk;
+    if (T <= a.topk || j_begin >= T) return;  // every position kept / nothing here (uniform per CTA)
+    const int tid = threadIdx.x, lane = tid & 31;
+
+    // bucket of the k-th largest score, and the lower end of the range that can be kept
+    {
+        const uint4 *src = reinterpret_cast<const uint4 *>(a.ghist + (size_t)row * kHistBuckets);
+        uint4 hv[kHistBuckets / 4 / kFilterThreads];
+#pragma unroll
+        for (int u = 0; u < kHistBuckets / 4 / kFilterThreads; ++u) hv[u] = __ldcg(src + u * kFilterThreads + tid);
+#pragma unroll
+        for (int u = 0; u < kHistBuckets / 4 / kFilterThreads; ++u)
+            reinterpret_cast<uint4 *>(hist_s)[u * kFilterThreads + tid] = hv[u];
+    }
+    __syncthreads();
+    find_bucket_from_top(hist_s, kHistBuckets, (uint32_t)a.topk, &sh_d, &sh_above, warp_sums);
+    const float q1 = row_q_l1<DK>(a.q + (size_t)row * DK, red);
+    const float kmax = __uint_as_float(__ldcg(a.kmax + b * a.n_k + g) << 16);
+    const float two_d = __fmul_ru(2.f, score_error_bound<DK>(q1, kmax));
+    // (bucket 0 starts at the NaN patterns: everything in it and above is a candidate)
+    const float lower = sh_d == 0 ? -INFINITY : __fsub_rd(key_float((uint32_t)sh_d << 21), two_d);
+
+    const float *s = a.scores + (size_t)row * a.t_pad;
+    int32_t *cj = a.cand_j + (size_t)row * a.t_pad;
+    float *cs = a.cand_s + (size_t)row * a.t_pad;
+    const int j_end = min(T, j_begin + kFilterChunk);
+    // lane-interleaved 16-byte loads: each warp load covers 512 contiguous bytes.
+    // A thread's hits form a 16-bit mask; one block scan gives every thread its
+    // slots and one global atomic per CTA reserves them.
+    static_assert(kFilterChunk == kFilterThreads * 16, "one pass of 16 positions per thread");
+    float4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int p = j_begin + (u * kFilterThreads + tid) * 4;
+        v[u] = p < j_end ? __ldcg(reinterpret_cast<const float4 *>(s + p)) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    uint32_t hits = 0;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int p = j_begin + (u * kFilterThreads + tid) * 4;
+        const float x[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            if (p + e < j_end && x[e] >= lower) hits |= 1u << (4 * u + e);
+    }
+    uint32_t total;
+    uint32_t slot = block_exclusive_scan((uint32_t)__popc(hits), warp_sums, &total);
+    __shared__ uint32_t sh_base;
+    if (tid == 0 && total) sh_base = atomicAdd(a.ncand + row, total);
+    __syncthreads();
+    if (hits) {
+        slot += sh_base;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int p = j_begin + (u * kFilterThreads + tid) * 4;
+            const float x[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                if ((hits >> (4 * u + e)) & 1u) {
+                    cj[slot] = p + e;
+                    cs[slot] = x[e];
+                    ++slot;
+                }
+            }
+        }
+    }
+    (void)lane;
+}
+
+// ------------------------------------------------------------------ 3. select + gather
 
 template <int DK, int DV>
 __global__ void __launch_bounds__(kSelThreads, 1) topv_select_kernel(const TopvArgs a) {
-    __shared__ uint32_t hist[2048];
-    __shared__ uint32_t warp_sums[32];
+    __shared__ uint32_t hist[kRadixBuckets];
+    __shared__ uint32_t warp_sums[33];
     __shared__ uint16_t q_s[DK];
     __shared__ uint32_t keys_s[kPairwiseMax][kKeyWords];
     __shared__ float red_s[kSelWarps];
@@ -248,6 +455,13 @@ __global__ void __launch_bounds__(kSelThreads, 1) topv_select_kernel(const TopvA
     __shared__ int sh_d;
     __shared__ uint32_t sh_above;
     __shared__ int sh_cnt_in, sh_na, sh_done;
+    extern __shared__ __align__(16) uint8_t sel_dyn[];
+    int32_t *c_j = reinterpret_cast<int32_t *>(sel_dyn);           // [kCandCap]
+    float *c_s = reinterpret_cast<float *>(c_j + kCandCap);           // [kCandCap]
+    uint32_t *bitmap = reinterpret_cast<uint32_t *>(c_s + kCandCap);  // [kTopvMaxContext / 32]
+    uint32_t *wprefix = bitmap + kTopvMaxContext / 32;                               // [kTopvMaxContext / 32]
+    int32_t *sel_j = reinterpret_cast<int32_t *>(wprefix + kTopvMaxContext / 32);   // [kSelCap]
+    float *sel_s = reinterpret_cast<float *>(sel_j + kSelCap);                       // [kSelCap]
 
     const int row = blockIdx.x;
     const int b = row / a.n_q;
@@ -257,11 +471,10 @@ __global__ void __launch_bounds__(kSelThreads, 1) topv_select_kernel(const TopvA
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int T = clamp_len(__ldg(a.seq_lens + b), a.t_max);
     const int K = a.topk;
-    const float *s = a.scores + (size_t)row * a.t_max;
-    uint8_t *fl = a.flags + (size_t)row * a.t_max;
-    int32_t *alist = a.alist + (size_t)row * a.t_max;
-    uint8_t *ast = a.astate + (size_t)row * a.t_max;
-    uint8_t *adg = a.adigit + (size_t)row * a.t_max;
+    const float *s = a.scores + (size_t)row * a.t_pad;
+    int32_t *alist = a.alist + (size_t)row * a.t_pad;
+    uint8_t *ast = a.astate + (size_t)row * a.t_pad;
+    uint8_t *adg = a.adigit + (size_t)row * a.t_pad;
     int32_t *idx = a.idx_out + (size_t)row * K;
     __nv_bfloat16 *outp = a.out + (size_t)row * DV;
 
@@ -271,96 +484,134 @@ __global__ void __launch_bounds__(kSelThreads, 1) topv_select_kernel(const TopvA
         for (int i = tid; i < DV; i += kSelThreads) outp[i] = __float2bfloat16(0.f);
         return;
     }
+    const int nwords = (T + 31) / 32;
+    int nsel;
 
     if (T <= K) {
-        for (int j = tid; j < T; j += kSelThreads) fl[j] = 1;
+        // every cached position is kept: positions 0..T-1, then -1
+        for (int i = tid; i < K; i += kSelThreads) idx[i] = i < T ? i : -1;
+        float mx = -INFINITY;
+        for (int i = tid; i < T; i += kSelThreads) {
+            const float x = s[i];
+            if (i < kSelCap) {
+                sel_j[i] = i;
+                sel_s[i] = x;
+            }
+            mx = fmaxf(mx, x);
+        }
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        if (lane == 0) red_s[warp] = mx;
+        nsel = T;
     } else {
-        // ---- a. tau: the K-th largest fp32 score (radix digits 11, 11, 10 bits)
+        // ---- candidates from the filter (every position that can be kept)
+        const uint32_t nc = __ldcg(a.ncand + row);
+        const bool in_smem = nc <= (uint32_t)kCandCap;
+        const int32_t *cj = in_smem ? c_j : a.cand_j + (size_t)row * a.t_pad;
+        const float *cs = in_smem ? c_s : a.cand_s + (size_t)row * a.t_pad;
+        if (in_smem) {
+            const int32_t *gj = a.cand_j + (size_t)row * a.t_pad;
+            const float *gs = a.cand_s + (size_t)row * a.t_pad;
+            for (uint32_t base = 0; base < nc; base += 4 * kSelThreads) {
+                int32_t jj[4];
+                float xx[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const uint32_t i = base + u * kSelThreads + tid;
+                    jj[u] = i < nc ? __ldcg(gj + i) : 0;
+                    xx[u] = i < nc ? __ldcg(gs + i) : 0.f;
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const uint32_t i = base + u * kSelThreads + tid;
+                    if (i < nc) {
+                        c_j[i] = jj[u];
+                        c_s[i] = xx[u];
+                    }
+                }
+            }
+        }
+        for (int i = tid; i < nwords; i += kSelThreads) bitmap[i] = 0u;
+        __syncthreads();
+
+        // ---- a. tau = the K-th largest score: radix select over the candidates, a byte per pass
         uint32_t prefix = 0, pmask = 0, kk = (uint32_t)K;
-        const int shifts[3] = {21, 10, 0};
-        const int widths[3] = {11, 11, 10};
-        for (int pass = 0; pass < 3; ++pass) {
-            const int nb = 1 << widths[pass];
-            for (int i = tid; i < nb; i += kSelThreads) hist[i] = 0;
+        for (int pass = 0; pass < 4; ++pass) {
+            const int shift = 24 - 8 * pass;
+            for (int i = tid; i < kRadixBuckets; i += kSelThreads) hist[i] = 0;
             __syncthreads();
-            for (int base = 0; base < T; base += kSelThreads) {
-                const int j = base + tid;
+            for (uint32_t base = 0; base < nc; base += kSelThreads) {
+                const uint32_t i = base + tid;
                 int bucket = -1;
-                if (j < T) {
-                    const uint32_t key = float_key(s[j]);
-                    if ((key & pmask) == prefix) bucket = (int)((key >> shifts[pass]) & (uint32_t)(nb - 1));
+                if (i < nc) {
+                    const uint32_t key = float_key(cs[i]);
+                    if ((key & pmask) == prefix) bucket = (int)((key >> shift) & 0xffu);
                 }
                 hist_add(hist, bucket);
             }
             __syncthreads();
-            find_bucket_from_top(hist, nb, kk, &sh_d, &sh_above, warp_sums);
-            prefix |= (uint32_t)sh_d << shifts[pass];
-            pmask |= (uint32_t)(nb - 1) << shifts[pass];
+            find_bucket_from_top(hist, kRadixBuckets, kk, &sh_d, &sh_above, warp_sums);
+            prefix |= (uint32_t)sh_d << shift;
+            pmask |= 0xffu << shift;
             kk -= sh_above;
-            __syncthreads();
         }
         const float tau = key_float(prefix);
 
-        // ---- b. rounding bound of every fp32 score
-        float q1 = 0.f;
-        if (warp == 0) {
-            for (int c = lane; c < DK; c += 32) q1 += fabsf(__uint_as_float((uint32_t)q_s[c] << 16));
-#pragma unroll
-            for (int off = 16; off >= 1; off >>= 1) q1 += __shfl_xor_sync(0xffffffffu, q1, off);
-            if (lane == 0) red_s[0] = q1;
-        }
+        // ---- b. rounding bound of every score of this row
+        const float q1 = row_q_l1<DK>(a.q + (size_t)row * DK, red_s);
+        const float kmax = __uint_as_float(__ldcg(a.kmax + b * a.n_k + g) << 16);
+        const float two_d = __fmul_ru(2.f, score_error_bound<DK>(q1, kmax));
+        const float hi_edge = __fadd_ru(tau, two_d);
+        const float lo_edge = __fsub_rd(tau, two_d);
         if (tid == 0) {
             sh_cnt_in = 0;
             sh_na = 0;
         }
         __syncthreads();
-        q1 = red_s[0];
-        const float kmax = __uint_as_float(__ldcg(a.kmax + b * a.n_k + g) << 16);
-        const double nu = (double)DK * 5.9604644775390625e-08;  // n * 2^-24
-        const float gamma = (float)(nu / (1.0 - nu));
-        const float delta = __fmul_ru(__fmul_ru(__fmul_ru(1.01f, gamma), q1), kmax) + (float)DK * 1.4012984643e-45f;
-        const float two_d = __fmul_ru(2.f, delta);
-        const float hi_edge = __fadd_ru(tau, two_d);
-        const float lo_edge = __fsub_rd(tau, two_d);
 
-        // ---- c. certain / ambiguous classification
+        // ---- c. certain / ambiguous classification of the candidates
         int my_in = 0;
-        for (int j = tid; j < T; j += kSelThreads) {
-            const float x = s[j];
-            uint8_t f = 0;
+        for (uint32_t i = tid; i < nc; i += kSelThreads) {
+            const float x = cs[i];
             if (x > hi_edge) {
-                f = 1;
+                const int j = cj[i];
+                atomicOr(bitmap + (j >> 5), 1u << (j & 31));
                 ++my_in;
             } else if (x >= lo_edge) {
-                const int slot = atomicAdd(&sh_na, 1);
-                alist[slot] = j;
+                alist[atomicAdd(&sh_na, 1)] = cj[i];
             }
-            fl[j] = f;
         }
 #pragma unroll
         for (int off = 16; off >= 1; off >>= 1) my_in += __shfl_xor_sync(0xffffffffu, my_in, off);
         if (lane == 0 && my_in) atomicAdd(&sh_cnt_in, my_in);
         __syncthreads();
         const int na = sh_na;
-        const int need = K - sh_cnt_in;  // 1 <= need <= na
+        const int need = K - sh_cnt_in;  // 1 <= need <= na when the bound holds
         const __nv_bfloat16 *krow0 = a.k + ((size_t)b * a.t_max * a.n_k + g) * DK;
         const size_t kstride = (size_t)a.n_k * DK;
+        auto keep = [&](int j) { atomicOr(bitmap + (j >> 5), 1u << (j & 31)); };
 
         if (need <= 0) {
             // nothing left to choose (cannot happen when the bound holds)
         } else if (need >= na) {
-            for (int i = tid; i < na; i += kSelThreads) fl[alist[i]] = 1;
+            for (int i = tid; i < na; i += kSelThreads) keep(alist[i]);
         } else if (na <= kPairwiseMax) {
-            // rank the few ambiguous positions pairwise by exact key
-            if (tid < na) {
-                const int j = alist[tid];
-                exact_key<DK>(q_s, reinterpret_cast<const uint16_t *>(krow0 + (size_t)j * kstride), j, keys_s[tid]);
+            // rank the few ambiguous positions pairwise by exact key; their K rows are
+            // staged in shared memory first (in the kept-pairs buffer, free until compaction)
+            uint4 *krows = reinterpret_cast<uint4 *>(sel_j);  // [na][DK / 8]
+            for (int i = tid; i < na * (DK / 8); i += kSelThreads) {
+                const int r = i / (DK / 8), c = i % (DK / 8);
+                krows[i] = __ldg(reinterpret_cast<const uint4 *>(krow0 + (size_t)alist[r] * kstride) + c);
             }
+            __syncthreads();
+            if (tid < na)
+                exact_key<DK>(q_s, reinterpret_cast<const uint16_t *>(krows + tid * (DK / 8)), alist[tid],
+                              keys_s[tid]);
             __syncthreads();
             if (tid < na) {
                 int better = 0;
                 for (int u = 0; u < na; ++u) better += key_greater(keys_s[u], keys_s[tid]) ? 1 : 0;
-                if (better < need) fl[alist[tid]] = 1;
+                if (better < need) keep(alist[tid]);
             }
         } else {
             // radix select over the exact keys, one byte per pass (keys are unique)
@@ -369,7 +620,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) topv_select_kernel(const TopvA
             uint32_t kk2 = (uint32_t)need;
             __syncthreads();
             for (int p = 0; p < kKeyWords * 4 && !sh_done; ++p) {
-                for (int i = tid; i < 256; i += kSelThreads) hist[i] = 0;
+                for (int i = tid; i < kRadixBuckets; i += kSelThreads) hist[i] = 0;
                 __syncthreads();
                 for (int base = 0; base < na; base += kSelThreads) {
                     const int i = base + tid;
@@ -384,7 +635,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) topv_select_kernel(const TopvA
                     hist_add(hist, bucket);
                 }
                 __syncthreads();
-                find_bucket_from_top(hist, 256, kk2, &sh_d, &sh_above, warp_sums);
+                find_bucket_from_top(hist, kRadixBuckets, kk2, &sh_d, &sh_above, warp_sums);
                 const int d = sh_d;
                 kk2 -= sh_above;
                 const bool finish = hist[d] == kk2;
@@ -398,58 +649,55 @@ __global__ void __launch_bounds__(kSelThreads, 1) topv_select_kernel(const TopvA
                 __syncthreads();
             }
             for (int i = tid; i < na; i += kSelThreads)
-                if (ast[i] == 1) fl[alist[i]] = 1;
+                if (ast[i] == 1) keep(alist[i]);
         }
-    }
-    __syncthreads();
+        __syncthreads();
 
-    // ---- d. compaction in ascending position order
-    const int per = (T + kSelThreads - 1) / kSelThreads;
-    const int j0 = min(T, tid * per), j1 = min(T, j0 + per);
-    int cnt = 0;
-    for (int j = j0; j < j1; ++j) cnt += fl[j];
-    int incl = cnt;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += y;
-    }
-    if (lane == 31) warp_sums[warp] = (uint32_t)incl;
-    __syncthreads();
-    if (warp == 0) {
-        const uint32_t ws = warp_sums[lane];
-        uint32_t wi = ws;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const uint32_t y = __shfl_up_sync(0xffffffffu, wi, off);
-            if (lane >= off) wi += y;
+        // ---- d. ascending order: a kept position's slot is the number of kept
+        //         positions before it, from per-word prefix counts of the bitmap
+        const int wper = (nwords + kSelThreads - 1) / kSelThreads;
+        const int w0 = min(nwords, tid * wper), w1 = min(nwords, w0 + wper);
+        uint32_t cnt = 0;
+        for (int w = w0; w < w1; ++w) cnt += __popc(bitmap[w]);
+        uint32_t total;
+        uint32_t run = block_exclusive_scan(cnt, warp_sums, &total);
+        for (int w = w0; w < w1; ++w) {
+            wprefix[w] = run;
+            run += __popc(bitmap[w]);
         }
-        warp_sums[lane] = wi - ws;
-        if (lane == 31) sh_cnt_in = (int)wi;  // total selected
+        nsel = (int)total;
+        __syncthreads();
+        float mx = -INFINITY;
+        for (uint32_t i = tid; i < nc; i += kSelThreads) {
+            const int j = cj[i];
+            const uint32_t word = bitmap[j >> 5];
+            if ((word >> (j & 31)) & 1u) {
+                const uint32_t slot = wprefix[j >> 5] + __popc(word & ((1u << (j & 31)) - 1u));
+                const float x = cs[i];
+                idx[slot] = j;
+                if (slot < (uint32_t)kSelCap) {
+                    sel_j[slot] = j;
+                    sel_s[slot] = x;
+                }
+                mx = fmaxf(mx, x);
+            }
+        }
+        if (tid == 0 && nsel != K) record_error(a.status, DIFFQKV_ERR_INVALID_ARG);
+        for (int i = nsel + tid; i < K; i += kSelThreads) idx[i] = -1;
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        if (lane == 0) red_s[warp] = mx;
     }
     __syncthreads();
-    int pos = (int)warp_sums[warp] + incl - cnt;
-    for (int j = j0; j < j1; ++j)
-        if (fl[j]) idx[pos++] = j;
-    const int nsel = sh_cnt_in;
-    if (tid == 0 && nsel != min(K, T)) record_error(a.status, DIFFQKV_ERR_INVALID_ARG);
-    for (int i = nsel + tid; i < K; i += kSelThreads) idx[i] = -1;
-    __syncthreads();
-
-    // ---- e. renormalised softmax over the selected rows; only their V rows are read
-    float m = -INFINITY;
-    for (int i = tid; i < nsel; i += kSelThreads) m = fmaxf(m, s[idx[i]]);
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-    if (lane == 0) red_s[warp] = m;
-    __syncthreads();
-    m = red_s[0];
+    float m = red_s[0];
 #pragma unroll 1
     for (int w = 1; w < kSelWarps; ++w) m = fmaxf(m, red_s[w]);
     __syncthreads();
 
+    // ---- e. renormalised softmax over the kept rows; only their V rows are read
     constexpr int CPV = DV / 8;      // lanes per V row
     constexpr int RPW = 32 / CPV;    // V rows per warp step
+    constexpr int GU = 8;            // V rows in flight per lane
     const int vc = lane % CPV, vs = lane / CPV;
     float o[8];
 #pragma unroll
@@ -457,15 +705,16 @@ __global__ void __launch_bounds__(kSelThreads, 1) topv_select_kernel(const TopvA
     float l = 0.f;
     const __nv_bfloat16 *vbase = a.v + ((size_t)b * a.t_max * a.n_v + vh) * DV + vc * 8;
     const size_t vstride = (size_t)a.n_v * DV;
-    for (int i0 = warp * RPW; i0 < nsel; i0 += kSelWarps * RPW * 2) {
-        uint4 vv[2];
-        float w[2];
+    for (int i0 = warp * RPW; i0 < nsel; i0 += kSelWarps * RPW * GU) {
+        uint4 vv[GU];
+        float w[GU];
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
+        for (int u = 0; u < GU; ++u) {
             const int i = i0 + u * kSelWarps * RPW + vs;
             if (i < nsel) {
-                const int j = idx[i];
-                w[u] = fast_exp2((s[j] - m) * a.scale_log2);
+                const int j = i < kSelCap ? sel_j[i] : __ldcg(idx + i);
+                const float x = i < kSelCap ? sel_s[i] : s[j];
+                w[u] = fast_exp2((x - m) * a.scale_log2);
                 vv[u] = __ldg(reinterpret_cast<const uint4 *>(vbase + (size_t)j * vstride));
             } else {
                 w[u] = 0.f;
@@ -473,7 +722,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) topv_select_kernel(const TopvA
             }
         }
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
+        for (int u = 0; u < GU; ++u) {
             float vf[8];
             unpack8(vv[u], vf);
             l += w[u];
@@ -507,8 +756,8 @@ __global__ void __launch_bounds__(kSelThreads, 1) topv_select_kernel(const TopvA
 
 size_t align_up(size_t x, size_t al) { return (x + al - 1) / al * al; }
 
-using ScoreFn = void (*)(TopvArgs);
-using SelectFn = void (*)(TopvArgs);
+using ScoreFn = void (*)(CUtensorMap, TopvArgs);
+using RowFn = void (*)(TopvArgs);
 
 template <int DK>
 ScoreFn pick_score_qpk(int qpk) {
@@ -528,7 +777,13 @@ ScoreFn pick_score(int dk, int qpk) {
     return nullptr;
 }
 
-SelectFn pick_select(int dk, int dv) {
+RowFn pick_filter(int dk) {
+    if (dk == 64) return topv_filter_kernel<64>;
+    if (dk == 128) return topv_filter_kernel<128>;
+    return nullptr;
+}
+
+RowFn pick_select(int dk, int dv) {
     if (dk == 64 && dv == 64) return topv_select_kernel<64, 64>;
     if (dk == 64 && dv == 128) return topv_select_kernel<64, 128>;
     if (dk == 128 && dv == 64) return topv_select_kernel<128, 64>;
@@ -536,14 +791,25 @@ SelectFn pick_select(int dk, int dv) {
     return nullptr;
 }
 
+size_t padded_len(int32_t t_max) { return align_up((size_t)t_max, 64); }
+
+// kmax entries, rounded up so the histograms after them start 16-byte aligned.
+size_t kmax_slots(const diffqkv_dims_t *d) { return align_up((size_t)d->batch * d->n_k, 4); }
+
+// Zero-filled per call: kmax [B*n_k, padded], histograms [rows][2048], candidate counts [rows].
+size_t zeroed_bytes(const diffqkv_dims_t *d) {
+    const size_t rows = (size_t)d->batch * d->n_q;
+    return kmax_slots(d) * 4 + rows * kHistBuckets * 4 + rows * 4;
+}
+
 }  // namespace
 
 size_t topv_workspace_size(const diffqkv_dims_t *d, int32_t t_max, int32_t topk) {
     if (validate_dims(d) != DIFFQKV_OK || t_max < 1 || topk < 1) return 0;
     const size_t rows = (size_t)d->batch * d->n_q;
-    const size_t per = (size_t)t_max;
-    return kTopvHeader + align_up((size_t)d->batch * d->n_k * 4, 256) + align_up(rows * per * 4, 256) * 2 +
-           align_up(rows * per, 256) * 3;
+    const size_t per = padded_len(t_max);
+    return kTopvHeader + align_up(zeroed_bytes(d), 256) + align_up(rows * per * 4, 256) * 4 +
+           align_up(rows * per, 256) * 2;
 }
 
 diffqkv_status_t topv_launch(const diffqkv_dims_t *d, const void *q, const void *k_cache, const void *v_cache,
@@ -553,10 +819,12 @@ diffqkv_status_t topv_launch(const diffqkv_dims_t *d, const void *q, const void 
     if (st != DIFFQKV_OK) return st;
     if (!q || !k_cache || !v_cache || !seq_lens || !out || !idx_out || t_max < 1 || topk < 1)
         return DIFFQKV_ERR_INVALID_ARG;
+    if (t_max > kTopvMaxContext) return DIFFQKV_ERR_UNSUPPORTED;
     const int qpk = d->n_q / d->n_k;
     ScoreFn score = pick_score(d->d_k, qpk);
-    SelectFn select = pick_select(d->d_k, d->d_v);
-    if (!score || !select) return DIFFQKV_ERR_UNSUPPORTED;
+    RowFn filter = pick_filter(d->d_k);
+    RowFn select = pick_select(d->d_k, d->d_v);
+    if (!score || !filter || !select) return DIFFQKV_ERR_UNSUPPORTED;
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
         (reinterpret_cast<uintptr_t>(idx_out) & 3u) || (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
         return DIFFQKV_ERR_MISALIGNED;
@@ -568,18 +836,23 @@ diffqkv_status_t topv_launch(const diffqkv_dims_t *d, const void *q, const void 
     if (st != DIFFQKV_OK) return st;
 
     const size_t rows = (size_t)d->batch * d->n_q;
+    const size_t t_pad = padded_len(t_max);
     uint8_t *ws = static_cast<uint8_t *>(workspace) + kTopvHeader;
     TopvArgs a;
     a.kmax = reinterpret_cast<uint32_t *>(ws);
-    ws += align_up((size_t)d->batch * d->n_k * 4, 256);
+    a.ghist = a.kmax + kmax_slots(d);  // 16-byte aligned (read with 16-byte loads)
+    a.ncand = a.ghist + rows * kHistBuckets;
+    ws += align_up(zeroed_bytes(d), 256);
     a.scores = reinterpret_cast<float *>(ws);
-    ws += align_up(rows * t_max * 4, 256);
+    ws += align_up(rows * t_pad * 4, 256);
+    a.cand_j = reinterpret_cast<int32_t *>(ws);
+    ws += align_up(rows * t_pad * 4, 256);
+    a.cand_s = reinterpret_cast<float *>(ws);
+    ws += align_up(rows * t_pad * 4, 256);
     a.alist = reinterpret_cast<int32_t *>(ws);
-    ws += align_up(rows * t_max * 4, 256);
-    a.flags = ws;
-    ws += align_up(rows * t_max, 256);
+    ws += align_up(rows * t_pad * 4, 256);
     a.astate = ws;
-    ws += align_up(rows * t_max, 256);
+    ws += align_up(rows * t_pad, 256);
     a.adigit = ws;
     a.q = static_cast<const __nv_bfloat16 *>(q);
     a.k = static_cast<const __nv_bfloat16 *>(k_cache);
@@ -593,24 +866,43 @@ diffqkv_status_t topv_launch(const diffqkv_dims_t *d, const void *q, const void 
     a.n_k = d->n_k;
     a.n_v = d->n_v;
     a.t_max = t_max;
+    a.t_pad = (int32_t)t_pad;
     a.topk = topk;
     a.q_per_k = qpk;
     a.q_per_v = d->n_q / d->n_v;
     a.scale_log2 = (float)((double)d->scale * 1.4426950408889634);
+    a.wait_limit_ns = kWaitLimitNs;
+    (void)max_seq_len;  // every grid adapts to the device lengths by itself
 
-    if (cudaMemsetAsync(a.kmax, 0, (size_t)d->batch * d->n_k * 4, stream) != cudaSuccess) {
+    if (cudaMemsetAsync(a.kmax, 0, zeroed_bytes(d), stream) != cudaSuccess) {
         cudaGetLastError();
         return DIFFQKV_ERR_CUDA;
     }
-    const int msl = (max_seq_len >= 1 && max_seq_len <= t_max) ? max_seq_len : t_max;
+    // 1. scores: TMA tiles of K {d_k, n_k, t_max, B}, box {64, 1, 128, 1}, 128-byte swizzle
+    CUtensorMap tm_k;
+    st = make_tensor_map_4d(&tm_k, k_cache, d->d_k, d->n_k, t_max, d->batch, 64, 1, kScoreTile, 1,
+                            CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != DIFFQKV_OK) return st;
+    const int tile_bytes = kScoreTile * d->d_k * 2;
+    const int fixed = qpk * kHistBuckets * 4 + qpk * d->d_k * 4 + 16 * 8 + 16 + 1024;
+    int stages = 4;
+    while (stages > 2 && stages * tile_bytes + fixed > 100 * 1024) --stages;
+    a.score_stages = stages;
+    const int score_smem = stages * tile_bytes + fixed;
+    const int per_sm = std::max(1, std::min(3, (227 * 1024) / (score_smem + 1024)));
     const int units = d->batch * d->n_k;
-    int chunks = (msl + kScoreChunk - 1) / kScoreChunk;
-    const int want = dev.num_sms * 8;  // resident score CTAs
-    chunks = std::max(1, std::min(chunks, (want + units - 1) / units));
-    dim3 grid_s(units, chunks);
-    score<<<grid_s, kScoreThreads, 0, stream>>>(a);
+    const int ygrid = std::max(1, (dev.num_sms * per_sm) / units);
+    const int select_smem = kCandCap * 8 + 2 * (kTopvMaxContext / 8) + kSelCap * 8;
+    if (ensure_dynamic_smem((const void *)score, score_smem) != DIFFQKV_OK ||
+        ensure_dynamic_smem((const void *)select, select_smem) != DIFFQKV_OK)
+        return DIFFQKV_ERR_CUDA;
+    score<<<dim3(units, ygrid), kScoreThreads + 32, score_smem, stream>>>(tm_k, a);
     if (cudaGetLastError() != cudaSuccess) return DIFFQKV_ERR_CUDA;
-    select<<<(unsigned)rows, kSelThreads, 0, stream>>>(a);
+    // 2. filter: every row, in chunks of kFilterChunk positions (chunks past a row's length return at once)
+    filter<<<dim3((unsigned)rows, (t_max + kFilterChunk - 1) / kFilterChunk), kFilterThreads, 0, stream>>>(a);
+    if (cudaGetLastError() != cudaSuccess) return DIFFQKV_ERR_CUDA;
+    // 3. select + gather
+    select<<<(unsigned)rows, kSelThreads, select_smem, stream>>>(a);
     if (cudaGetLastError() != cudaSuccess) return DIFFQKV_ERR_CUDA;
     return DIFFQKV_OK;
 }
