@@ -85,7 +85,7 @@ diffqkv_status_t current_device_info(DeviceInfo *info) {
 
 diffqkv_status_t make_tensor_map_4d(CUtensorMap *map, const void *base, uint64_t dim0, uint64_t dim1,
                                     uint64_t dim2, uint64_t dim3, uint32_t box0, uint32_t box1, uint32_t box2,
-                                    uint32_t box3, CUtensorMapSwizzle swizzle) {
+                                    uint32_t box3, CUtensorMapSwizzle swizzle, CUtensorMapL2promotion promotion) {
     auto fn = encode_fn();
     if (!fn) return DIFFQKV_ERR_CUDA;
     const cuuint64_t dims[4] = {dim0, dim1, dim2, dim3};
@@ -93,8 +93,7 @@ diffqkv_status_t make_tensor_map_4d(CUtensorMap *map, const void *base, uint64_t
     const cuuint32_t box[4] = {box0, box1, box2, box3};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, promotion, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? DIFFQKV_OK : DIFFQKV_ERR_INVALID_ARG;
 }
 

@@ -23,9 +23,12 @@ diffqkv_status_t current_device_info(DeviceInfo *info);
 
 // Encodes a rank-4 tiled tensor map over a bf16 tensor laid out as
 // [dim3][dim2][dim1][dim0] (dim0 innermost, contiguous), box {b0,b1,b2,b3}.
+// `promotion`: L2 sector promotion of the loads (256 B by default; 128 B when
+// the box rows are 128-byte slices whose neighbours belong to other CTAs).
 diffqkv_status_t make_tensor_map_4d(CUtensorMap *map, const void *base, uint64_t dim0, uint64_t dim1,
                                     uint64_t dim2, uint64_t dim3, uint32_t box0, uint32_t box1,
-                                    uint32_t box2, uint32_t box3, CUtensorMapSwizzle swizzle);
+                                    uint32_t box2, uint32_t box3, CUtensorMapSwizzle swizzle,
+                                    CUtensorMapL2promotion promotion = CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
 
 // Encodes a rank-3 tiled tensor map ([dim2][dim1][dim0], dim0 contiguous).
 diffqkv_status_t make_tensor_map_3d(CUtensorMap *map, const void *base, uint64_t dim0, uint64_t dim1,

@@ -236,9 +236,14 @@ __global__ void __launch_bounds__(kThreads, 2)
                 for (int c = 0; c < BN; ++c)
                     if (j0 + c > i) s[c] = -INFINITY;
             }
-            float mx = -INFINITY;
+            // row max as 8 independent chains (a single 64-long chain is latency-bound)
+            float mx8[8];
 #pragma unroll
-            for (int c = 0; c < BN; ++c) mx = fmaxf(mx, s[c]);
+            for (int e = 0; e < 8; ++e) mx8[e] = s[e];
+#pragma unroll
+            for (int c = 8; c < BN; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
+            const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                   fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
             const float m_new = mx * a.scale_log2;
             bool waited_pv = false;
             if (n == 0) {
@@ -267,16 +272,25 @@ __global__ void __launch_bounds__(kThreads, 2)
                     }
                 }
             }
-            // p = 2^(s * scale * log2 e - m_used), row sum, bf16 pack
-            const float neg_m = -m_used;
+            // p = 2^(s * scale * log2 e - m): packed fp32 pairs, row sum as 4 pair-chains
+            const f32x2_t sc2 = f2_pack(a.scale_log2, a.scale_log2);
+            const f32x2_t nm2 = f2_pack(-m_used, -m_used);
             uint32_t pk[BN / 2];
+            f32x2_t l2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
             for (int c = 0; c < BN; c += 2) {
-                const float p0 = fast_exp2(fmaf(s[c], a.scale_log2, neg_m));
-                const float p1 = fast_exp2(fmaf(s[c + 1], a.scale_log2, neg_m));
-                l += p0 + p1;
+                float t0, t1;
+                f2_unpack(f2_fma(f2_pack(s[c], s[c + 1]), sc2, nm2), t0, t1);
+                const float p0 = fast_exp2(t0);
+                const float p1 = fast_exp2(t1);
+                l2[(c >> 1) & 3] = f2_add(l2[(c >> 1) & 3], f2_pack(p0, p1));
                 pk[c >> 1] = pack_bf16x2(p0, p1);
             }
+            float la, lb, lc, ld;
+            f2_unpack(f2_add(f2_add(l2[0], l2[1]), f2_add(l2[2], l2[3])), la, lb);
+            (void)lc;
+            (void)ld;
+            l += la + lb;
             if (n >= 1 && !waited_pv) {
                 // the previous P.V must have consumed the P buffer
                 mbar_wait_bounded(pv_done, (uint32_t)((n - 1) & 1), a.wait_limit_ns, abort_flag, a.status);
