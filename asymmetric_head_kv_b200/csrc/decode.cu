@@ -468,11 +468,25 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
 
 constexpr int ncw_for(int qpk) { return qpk > 8 ? qpk : 8; }
 
-// Tile height: about 32-40 KiB of K+V per stage (V side sized for the widest group).
+// Smallest legal tile height: the R warps of a head split the tile, and each
+// warp's share must be whole score passes and whole P.V slot rounds.
+constexpr int tile_granule(int dk, int dv, int qpk) {
+    const int r = ncw_for(qpk) / qpk;
+    const int tpp = 32 / (dk / 8), nsl = 32 / (dv / 8);
+    return r * (tpp > nsl ? tpp : nsl);
+}
+
+// Tile height: about 56 KiB of K+V per stage (V side sized for the widest group),
+// at most 128 positions.  Measured on B200 at 32k context: per-tile overheads
+// (barrier, softmax reductions, rescale) make small tiles slow, while more than
+// ~170 KiB in flight per SM reads more slowly (16 x 32768 DiffQKV: 32-position
+// tiles 6074 GB/s, 48 x 3 stages 6836, 64 x 3 stages 6487).
 constexpr int tt_for(int dk, int dv, int qpk) {
+    const int g = tile_granule(dk, dv, qpk);
     const int bytes_per_token = 2 * dk + 2 * qpk * dv;
-    int tt = 16;
-    while (tt < 128 && (tt * 2) * bytes_per_token <= 40 * 1024) tt *= 2;
+    int tt = (56 * 1024 / bytes_per_token) / g * g;
+    if (tt < g) tt = g;
+    if (tt > 128) tt = 128 / g * g;
     return tt;
 }
 
@@ -556,8 +570,7 @@ diffqkv_status_t decode_plan(const diffqkv_dims_t *d, int32_t t_max, int32_t max
     const size_t smem_cap = 227 * 1024;
     int stages = (tuning && tuning->stages) ? tuning->stages : 0;
     if (stages == 0) {
-        // three stages: measured on B200 at 32k context, deeper rings read more slowly
-        // (5892 GB/s at 3 stages, 5856 at 4, 5715 at 5 for 16 x 32768 positions)
+        // three ~56 KiB stages (see tt_for): deeper rings read more slowly on B200
         stages = 3;
         while (stages > 2 && stages * stage_stride + extra > smem_cap) --stages;
     }

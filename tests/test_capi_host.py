@@ -71,13 +71,13 @@ def test_plan_fits_b200(shape):
     assert 2 <= p["stages"] <= 8
     assert p["smem_bytes"] <= 227 * 1024
     assert 1 <= p["grid_ctas"] <= 148
-    assert p["tile_tokens"] in (16, 32, 64, 128)
+    assert 4 <= p["tile_tokens"] <= 128
     assert p["threads"] % 32 == 0 and p["threads"] <= 1024
 
 
 def test_plan_grid_follows_context_and_override():
     p = ak.decode_plan(dims(batch=1), 512, 512, 148)
-    assert p["grid_ctas"] == 4 * (512 // p["tile_tokens"])    # fewer tiles than SMs
+    assert p["grid_ctas"] == 4 * -(-512 // p["tile_tokens"])    # fewer tiles than SMs
     p = ak.decode_plan(dims(), 32768, 32768, 148, {"grid_ctas": 7, "stages": 3, "ctas_per_sm": 0})
     assert p["grid_ctas"] == 7 and p["stages"] == 3
     with pytest.raises(ak.DiffqkvError):

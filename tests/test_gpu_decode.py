@@ -63,10 +63,16 @@ def test_split_points_do_not_change_result(cuda_device, grid):
 def test_pipeline_depth(cuda_device, stages):
     d = wl.random_decode_inputs(2, 3000, wl.DIFFQKV, seed=103, seq_lens=[3000, 1777])
     tuning = {"grid_ctas": 0, "stages": stages, "ctas_per_sm": 0}
-    if stages == 8:   # 8 stages of 36 KiB do not fit in 227 KiB of shared memory: rejected up front
-        with pytest.raises(ak.DiffqkvError) as e:
+    dims = ak.make_dims(2, 16, 4, 16, 64, 128, 0.125)
+    sms = torch.cuda.get_device_properties(cuda_device).multi_processor_count
+    try:
+        ak.decode_plan(dims, 3000, 3000, sms, tuning)
+    except ak.DiffqkvError as e:
+        # a ring that does not fit in 227 KiB of shared memory is rejected before launch
+        assert e.status == ak._capi.UNSUPPORTED
+        with pytest.raises(ak.DiffqkvError) as e2:
             _run(d, cuda_device, tuning=tuning)
-        assert e.value.status == ak._capi.UNSUPPORTED
+        assert e2.value.status == ak._capi.UNSUPPORTED
         return
     out = _run(d, cuda_device, tuning=tuning)
     assert_parity(out, _oracle(d), f"stages={stages}")
