@@ -177,8 +177,16 @@ size_t diffqkv_decode_topv_workspace_size(const diffqkv_dims_t *dims, int32_t t_
  *   out[b,h]     = sum_{j in S} e^{s_j - m} v[b,j,vh] / sum_{j in S} e^{s_j - m},
  *                  s_j = scale * q.k_j, m = max_{j in S} s_j   (bf16 [B,n_q,d_v])
  *   idx_out[b,h] = S in ascending order, padded with -1          (int32 [B,n_q,topk])
- * Only the selected V rows are read from v_cache.  Inputs as diffqkv_decode;
- * 1 <= topk <= 4096.
+ * Only the selected V rows are read from v_cache.  Inputs and layouts as
+ * diffqkv_decode.  topk >= 1 (any size; topk >= seq_lens[b] keeps every
+ * position).  1 <= t_max <= 131072, else DIFFQKV_ERR_UNSUPPORTED (t_max >
+ * 131072) or DIFFQKV_ERR_INVALID_ARG.  idx_out must be 4-byte aligned, the
+ * other buffers and the workspace 16-byte aligned (DIFFQKV_ERR_MISALIGNED).
+ * max_seq_len is accepted for symmetry with diffqkv_decode and ignored: the
+ * kernels read the lengths from seq_lens on the device.  Lengths outside
+ * [0, t_max] are clamped to that range.  A row with length 0 gets a zero
+ * output and an all -1 index row.  Launches three kernels on `stream`;
+ * returns once they are queued.
  */
 diffqkv_status_t diffqkv_decode_topv(const diffqkv_dims_t *dims, const void *q, const void *k_cache,
                                      const void *v_cache, const int32_t *seq_lens, int32_t t_max,

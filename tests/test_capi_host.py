@@ -121,3 +121,23 @@ def test_selftest_and_status_reject_bad_args():
     lib = _capi.lib()
     assert lib.diffqkv_selftest_wait_timeout(10, None) == _capi.INVALID_ARG
     assert lib.diffqkv_get_device_status(None, None) == _capi.INVALID_ARG
+
+
+def _topv_raw(d, t_max=128, topk=4, q=0x1000, idx=0x7000, ws=0x6000, ws_bytes=1 << 34):
+    return _capi.lib().diffqkv_decode_topv(ctypes.byref(d), q, 0x2000, 0x3000, 0x4000, t_max, t_max, topk, 0x5000,
+                                           idx, ws, ws_bytes, None)
+
+
+def test_topv_rejects_before_launch():
+    d = dims()
+    assert _topv_raw(d, topk=0) == _capi.INVALID_ARG
+    assert _topv_raw(d, t_max=0) == _capi.INVALID_ARG
+    assert _topv_raw(d, t_max=131073) == _capi.UNSUPPORTED  # kept-position bitmap holds 131072 positions
+    assert _topv_raw(d, q=0x1008) == _capi.MISALIGNED
+    assert _topv_raw(d, idx=0x7002) == _capi.MISALIGNED
+    assert _topv_raw(d, ws_bytes=16) == _capi.WORKSPACE
+    assert _capi.lib().diffqkv_decode_topv_workspace_size(ctypes.byref(d), 131072, 1024) > 0
+    # 18 bytes per (row, position) plus the zeroed histograms
+    small = _capi.lib().diffqkv_decode_topv_workspace_size(ctypes.byref(d), 1024, 8)
+    large = _capi.lib().diffqkv_decode_topv_workspace_size(ctypes.byref(d), 2048, 8)
+    assert large - small == d.batch * d.n_q * 1024 * 18
