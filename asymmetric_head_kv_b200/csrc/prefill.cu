@@ -10,15 +10,19 @@
 //               (128-byte swizzle, the layout the MMA descriptors describe)
 //   warp 5      allocates 256 TMEM columns; lane 0 issues every tcgen05.mma:
 //               S = Q K^T (M128 N64, fp32 in TMEM, two S buffers) and
-//               O += P V (M128 N=d_v, fp32 in TMEM)
+//               O += P V (M128 N=d_v, fp32 in TMEM, P read from TMEM)
 //   warps 0-3   softmax: thread t owns query row t = TMEM lane t, so row max and
-//               row sum need no shuffles; P is written to shared memory as bf16
-//               in the K-major swizzled layout the PV MMA reads.  O is rescaled
-//               in TMEM only when a row maximum grows by more than 2^8 (the
-//               stale maximum is used consistently for O and the row sum, so
-//               the result is exact up to rounding).
+//               row sum need no shuffles; P is written back as bf16 pairs over
+//               the first 32 columns of its own S buffer, where the PV MMA
+//               reads it as the A operand.  O is rescaled in TMEM only when a
+//               row maximum grows by more than 2^8 (the stale maximum is used
+//               consistently for O and the row sum, so the result is exact up
+//               to rounding).
+// The MMA thread issues S(n+2) into a buffer only after P(n) V(n), which reads
+// P(n) from that buffer; tcgen05.mma operations from one thread run in issue
+// order, so no other hand-back of the S buffers is needed.
 // Every mbarrier wait is bounded; CTAs are ordered heaviest (most K/V tiles)
-// first.  Two CTAs fit on one SM (104 KB smem, 256 TMEM columns each).
+// first.  Two CTAs fit on one SM (at most 98 KB smem and 256 TMEM columns each).
 #include <math.h>
 
 #include "common.cuh"
@@ -30,10 +34,12 @@ namespace {
 
 constexpr int BM = 128;             // query rows per CTA
 constexpr int BN = 64;              // K/V positions per tile
+constexpr int kSoftmaxWarps = 4;
+constexpr int kProducerWarp = 4;
+constexpr int kMmaWarp = 5;
 constexpr int kThreads = 192;       // 4 softmax warps, producer, MMA
 constexpr int kTmemCols = 256;      // S0 | S1 | O
 constexpr float kRescaleLog2 = 8.f; // lazy O rescale threshold (log2 domain)
-
 template <int DK, int DV>
 struct Cfg {
     static constexpr int KB = DK / 64;                 // 64-wide swizzle blocks along d_k
@@ -41,13 +47,11 @@ struct Cfg {
     static constexpr int Q_BYTES = BM * DK * 2;
     static constexpr int K_BYTES = BN * DK * 2;
     static constexpr int V_BYTES = BN * DV * 2;
-    static constexpr int P_BYTES = BM * BN * 2;
     static constexpr int STAGES = DK == 64 ? 3 : 2;
     static constexpr int STAGE_BYTES = K_BYTES + V_BYTES;
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_KV = Q_BYTES;
-    static constexpr int OFF_P = OFF_KV + STAGES * STAGE_BYTES;
-    static constexpr int OFF_BAR = OFF_P + P_BYTES;
+    static constexpr int OFF_BAR = OFF_KV + STAGES * STAGE_BYTES;
     static constexpr int SMEM = OFF_BAR + 256 + 1024;  // barriers/flags + alignment slack
 };
 
@@ -71,7 +75,6 @@ __global__ void __launch_bounds__(kThreads, 2)
     uint64_t *kv_empty = bars + 4;            // [STAGES]
     uint64_t *q_full = bars + 8;
     uint64_t *s_full = bars + 9;              // [2]
-    uint64_t *s_free = bars + 11;             // [2]
     uint64_t *p_full = bars + 13;
     uint64_t *pv_done = bars + 14;
     uint64_t *mma_done = bars + 15;
@@ -102,15 +105,13 @@ __global__ void __launch_bounds__(kThreads, 2)
         mbar_init(q_full, 1);
         mbar_init(&s_full[0], 1);
         mbar_init(&s_full[1], 1);
-        mbar_init(&s_free[0], 4);
-        mbar_init(&s_free[1], 4);
-        mbar_init(p_full, 4);
+        mbar_init(p_full, kSoftmaxWarps);
         mbar_init(pv_done, 1);
         mbar_init(mma_done, 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
-    if (warp == 5) {
+    if (warp == kMmaWarp) {
         tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();
     }
@@ -118,10 +119,9 @@ __global__ void __launch_bounds__(kThreads, 2)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t t_s[2] = {tmem, tmem + BN};
-    const uint32_t t_o = tmem + 2 * BN;
+    const uint32_t t_o = tmem + 2 * BN;  // S buffer sb (and P over its first BN/2 columns) at tmem + sb * BN
 
-    if (warp == 4) {
+    if (warp == kProducerWarp) {
         // ======================= TMA producer
         if (lane == 0) {
             prefetch_tensormap(&tm_q);
@@ -153,24 +153,22 @@ __global__ void __launch_bounds__(kThreads, 2)
                 mbar_wait_bounded(&kv_full[n % C::STAGES], (uint32_t)((n / C::STAGES) & 1), a.wait_limit_ns,
                                   nullptr, a.status);
         }
-    } else if (warp == 5) {
+    } else if (warp == kMmaWarp) {
         // ======================= MMA issuer (one thread)
         if (lane == 0) {
             constexpr uint32_t idesc_qk = umma_idesc_bf16(BM, BN, false, false);
             constexpr uint32_t idesc_pv = umma_idesc_bf16(BM, DV, false, true);
             const uint32_t q_addr = smem_addr(smem + C::OFF_Q);
-            const uint32_t p_addr = smem_addr(smem + C::OFF_P);
             mbar_wait_bounded(q_full, 0, a.wait_limit_ns, abort_flag, a.status);
             for (int n = 0; n <= n_kv; ++n) {
                 if (n < n_kv) {
                     // S[n%2] = Q K_n^T
                     const int st = n % C::STAGES;
                     const int sb = n & 1;
+                    // S buffer sb last held S(n-2) and P(n-2): the softmax was done with it before
+                    // p_full(n-2), and P(n-2) V(n-2) was issued ahead of this MMA
                     mbar_wait_bounded(&kv_full[st], (uint32_t)((n / C::STAGES) & 1), a.wait_limit_ns, abort_flag,
                                       a.status);
-                    if (n >= 2)
-                        mbar_wait_bounded(&s_free[sb], (uint32_t)(((n >> 1) - 1) & 1), a.wait_limit_ns, abort_flag,
-                                          a.status);
                     tc_fence_after();
                     const uint32_t k_addr = smem_addr(smem + C::OFF_KV + st * C::STAGE_BYTES);
 #pragma unroll
@@ -178,7 +176,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                         const uint32_t blk = (uint32_t)(ks >> 2), sub = (uint32_t)(ks & 3) * 32u;
                         const uint64_t da = smem_desc_sw128(q_addr + blk * (BM * 128) + sub, 16, 1024);
                         const uint64_t db = smem_desc_sw128(k_addr + blk * (BN * 128) + sub, 16, 1024);
-                        umma_bf16(t_s[sb], da, db, idesc_qk, ks > 0 ? 1u : 0u);
+                        umma_bf16(tmem + (uint32_t)(sb * BN), da, db, idesc_qk, ks > 0 ? 1u : 0u);
                     }
                     umma_commit(&s_full[sb]);
                 }
@@ -189,11 +187,12 @@ __global__ void __launch_bounds__(kThreads, 2)
                     mbar_wait_bounded(p_full, (uint32_t)(m & 1), a.wait_limit_ns, abort_flag, a.status);
                     tc_fence_after();
                     const uint32_t v_addr = smem_addr(smem + C::OFF_KV + st * C::STAGE_BYTES + C::K_BYTES);
+                    const uint32_t p_tmem = tmem + (uint32_t)((m & 1) * BN);
 #pragma unroll
                     for (int ks = 0; ks < BN / 16; ++ks) {
-                        const uint64_t da = smem_desc_sw128(p_addr + (uint32_t)ks * 32u, 16, 1024);
+                        // A = P(m) columns [8 ks, 8 ks + 8): 16 bf16 keys per row
                         const uint64_t db = smem_desc_sw128(v_addr + (uint32_t)ks * (16 * 128), BN * 128, 1024);
-                        umma_bf16(t_o, da, db, idesc_pv, (m > 0 || ks > 0) ? 1u : 0u);
+                        umma_bf16_tmem_a(t_o, p_tmem + (uint32_t)ks * 8u, db, idesc_pv, (m > 0 || ks > 0) ? 1u : 0u);
                     }
                     umma_commit(pv_done);
                     umma_commit(&kv_empty[st]);
@@ -208,26 +207,23 @@ __global__ void __launch_bounds__(kThreads, 2)
         const int i = row0 + tid;  // query position of this thread's row
         float m_used = -INFINITY;  // log2-domain maximum the stored O and l are relative to
         float l = 0.f;
-        uint8_t *p_row = smem + C::OFF_P + (tid >> 3) * 1024 + (tid & 7) * 128;
         for (int n = 0; n < n_kv; ++n) {
             const int sb = n & 1;
+            const uint32_t t_sb = tmem + (uint32_t)(sb * BN) + lane_base;
             mbar_wait_bounded(&s_full[sb], (uint32_t)((n >> 1) & 1), a.wait_limit_ns, abort_flag, a.status);
             tc_fence_after();
             float s[BN];
             {
-                uint32_t r[32];
-                tmem_ld32(t_s[sb] + lane_base, r);
+                uint32_t r0[32], r1[32];
+                tmem_ld32(t_sb, r0);
+                tmem_ld32(t_sb + 32, r1);
                 tmem_wait_ld();
 #pragma unroll
-                for (int c = 0; c < 32; ++c) s[c] = __uint_as_float(r[c]);
-                tmem_ld32(t_s[sb] + lane_base + 32, r);
-                tmem_wait_ld();
-#pragma unroll
-                for (int c = 0; c < 32; ++c) s[32 + c] = __uint_as_float(r[c]);
+                for (int c = 0; c < 32; ++c) {
+                    s[c] = __uint_as_float(r0[c]);
+                    s[32 + c] = __uint_as_float(r1[c]);
+                }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&s_free[sb]);
 
             // causal mask on tiles that reach past this row
             const int j0 = n * BN;
@@ -286,22 +282,16 @@ __global__ void __launch_bounds__(kThreads, 2)
                 l2[(c >> 1) & 3] = f2_add(l2[(c >> 1) & 3], f2_pack(p0, p1));
                 pk[c >> 1] = pack_bf16x2(p0, p1);
             }
-            float la, lb, lc, ld;
+            float la, lb;
             f2_unpack(f2_add(f2_add(l2[0], l2[1]), f2_add(l2[2], l2[3])), la, lb);
-            (void)lc;
-            (void)ld;
             l += la + lb;
+            // P(n) over the first 32 columns of S(n): key 2c in the low half of column c
+            tmem_st32(t_sb, pk);
+            tmem_wait_st();
             if (n >= 1 && !waited_pv) {
-                // the previous P.V must have consumed the P buffer
+                // keeps this warp at most one P.V behind, so every pv_done phase is waited in turn
                 mbar_wait_bounded(pv_done, (uint32_t)((n - 1) & 1), a.wait_limit_ns, abort_flag, a.status);
             }
-            // row of P: 8 chunks of 16 bytes, 128-byte swizzle (chunk ^ row%8)
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                uint8_t *dst = p_row + ((c ^ (tid & 7)) << 4);
-                sts128(dst, pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-            }
-            fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(p_full);
@@ -331,7 +321,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == kMmaWarp) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }

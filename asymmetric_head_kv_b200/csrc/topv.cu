@@ -10,23 +10,28 @@
 // Three launches:
 //  1. topv_score_kernel -- streams K once with TMA (one K row serves all
 //     n_q/n_k query heads of its group; one position per thread) and writes
-//     fp32 scores s_j = q.k_j (unscaled fp32 FMA chain: every bf16 x bf16
-//     product is exact), a 2048-bucket histogram of the top 11 bits of each
+//     fp32 scores s_j = q.k_j (unscaled fp32 FMAs, two per packed f32x2
+//     instruction; every bf16 x bf16 product is exact), a 2048-bucket histogram of the top 11 bits of each
 //     score's order key per row, and per (batch, K head) the largest |k|.
 //  2. topv_filter_kernel -- all SMs: per row, the histogram gives the bucket
 //     holding the k-th largest score; every position whose score is at least
 //     that bucket's lower end minus 2d (d the rounding bound below) is
 //     appended to the row's candidate list.  Everything else is certainly out.
 //  3. topv_select_kernel, one CTA per row, on the candidates in shared memory:
-//     a. tau = k-th largest fp32 score (radix select, byte by byte);
+//     a. tau = k-th largest fp32 score (radix select on the 21 key bits below
+//        the bucket the filter found: 11 bits, then 10);
 //     b. d >= |s_j - e_j| for every j, e_j the exact dot product:
 //        d = 1.01 gamma_n ||q||_1 max|k| + n 2^-149, gamma_n = n u / (1 - n u), u = 2^-24;
 //     c. s_j > tau + 2d: certainly kept; s_j < tau - 2d: certainly not; the
 //        rest (usually a handful) get exact keys -- an integer superaccumulator
 //        of the products -- and the remaining slots go to the largest exact
 //        keys, the lower position first on ties;
-//     d. kept positions are marked in a bitmap and written in ascending order;
-//     e. the renormalised softmax-weighted sum of exactly those V rows is written.
+//     d. kept positions are marked in a bitmap and written in ascending order.
+//  4. topv_gather_kernel, several CTAs per row: the renormalised softmax-weighted
+//     sum of exactly the kept V rows; the last CTA of a row adds the parts up.
+// Launches 2-4 use programmatic dependent launch: each kernel lets the next one
+// be scheduled early and waits (griddepcontrol.wait) before it reads anything
+// the previous one wrote.
 #include <math.h>
 
 #include <algorithm>
@@ -50,8 +55,11 @@ constexpr int kPairwiseMax = 64;        // ambiguous sets up to this size are ra
 constexpr int kKeyWords = 19;           // 18 superaccumulator digits + inverted position
 constexpr int kTopvHeader = 256;
 constexpr int kCandCap = 12288;         // candidates held in shared memory by the select kernel
-constexpr int kSelCap = 4096;           // kept (position, score) pairs held in shared memory
 constexpr int kTopvMaxContext = 131072; // bitmap of kept positions: 16 KB of shared memory
+constexpr int kGatherThreads = 256;
+constexpr int kGatherWarps = kGatherThreads / 32;
+constexpr int kGatherRows = 128;        // kept V rows per gather CTA (target)
+constexpr int kGatherMaxSplit = 64;
 
 struct TopvArgs {
     const __nv_bfloat16 *q;
@@ -69,14 +77,26 @@ struct TopvArgs {
     uint32_t *kmax;    // [B*n_k] bf16 bit pattern of max |k| (zeroed per call)
     uint32_t *ghist;   // [B*n_q][2048] histogram of the top 11 bits of the score keys (zeroed per call)
     uint32_t *ncand;   // [B*n_q] candidate counts (zeroed per call)
+    uint32_t *gcount;  // [B*n_q] gather CTAs finished per row (zeroed per call)
+    uint32_t *rowinfo; // [B*n_q][4]: threshold bucket, count above it (filter); kept max score, kept count (select)
+    float *gpart;      // [B*n_q][gather_split][d_v + 1] partial sums of the gather
     int32_t *status;
     int32_t batch, n_q, n_k, n_v, t_max, t_pad, topk, q_per_k, q_per_v;
     int32_t score_stages;
+    int32_t gather_split;
     float scale_log2;
     uint64_t wait_limit_ns;
 };
 
 __device__ __forceinline__ int clamp_len(int v, int t_max) { return v < 0 ? 0 : (v > t_max ? t_max : v); }
+
+// Programmatic dependent launch: let the next kernel in the stream be scheduled
+// now / wait until the previous kernel has finished and its writes are visible.
+// Both are no-ops for a kernel launched without the attribute.  Every chained
+// kernel waits before it can exit, so each one finishing implies that all the
+// kernels before it have finished too.
+__device__ __forceinline__ void pdl_launch_next() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait_prev() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 // Order-preserving map of finite floats onto uint32 (larger float -> larger key).
 __device__ __forceinline__ uint32_t float_key(float f) {
@@ -138,6 +158,7 @@ __global__ void __launch_bounds__(kScoreThreads + 32) topv_score_kernel(const __
         *abort_flag = 0;
         fence_barrier_init();
     }
+    pdl_launch_next();
     for (int i = tid; i < QPK * kHistBuckets; i += blockDim.x) hist_s[i] = 0;
     for (int i = tid; i < QPK * DK; i += blockDim.x) {
         const int hh = i / DK, c = i % DK;
@@ -177,9 +198,12 @@ __global__ void __launch_bounds__(kScoreThreads + 32) topv_score_kernel(const __
             const uint8_t *row = tiles + st * TILE_BYTES + tid * 128;
             const int j = t * kScoreTile + tid;
             const uint32_t live = j < T ? 0x7fff7fffu : 0u;  // the |k| bound covers cached positions only
-            float acc[QPK];
+            // even/odd keys of each head in packed fp32 pairs, split over two chains per head:
+            // every lane of fma.rn.f32x2 is an IEEE fp32 FMA, and each product meets at most
+            // d_k/4 + 2 roundings on its way into the score
+            f32x2_t acc_a[QPK], acc_b[QPK];
 #pragma unroll
-            for (int hh = 0; hh < QPK; ++hh) acc[hh] = 0.f;
+            for (int hh = 0; hh < QPK; ++hh) acc_a[hh] = acc_b[hh] = 0ull;
 #pragma unroll
             for (int kb = 0; kb < KB; ++kb) {
 #pragma unroll
@@ -189,24 +213,26 @@ __global__ void __launch_bounds__(kScoreThreads + 32) topv_score_kernel(const __
                     kmx2 = __vmaxu2(kmx2, kv.y & live);
                     kmx2 = __vmaxu2(kmx2, kv.z & live);
                     kmx2 = __vmaxu2(kmx2, kv.w & live);
-                    float kf[8];
-                    unpack8(kv, kf);
+                    const f32x2_t k01 = bf16x2_to_f2(kv.x), k23 = bf16x2_to_f2(kv.y);
+                    const f32x2_t k45 = bf16x2_to_f2(kv.z), k67 = bf16x2_to_f2(kv.w);
 #pragma unroll
                     for (int hh = 0; hh < QPK; ++hh) {
                         const float4 qa = *reinterpret_cast<const float4 *>(q_s + hh * DK + kb * 64 + c * 8);
                         const float4 qb = *reinterpret_cast<const float4 *>(q_s + hh * DK + kb * 64 + c * 8 + 4);
-                        float x = acc[hh];
-                        x = fmaf(qa.x, kf[0], x);
-                        x = fmaf(qa.y, kf[1], x);
-                        x = fmaf(qa.z, kf[2], x);
-                        x = fmaf(qa.w, kf[3], x);
-                        x = fmaf(qb.x, kf[4], x);
-                        x = fmaf(qb.y, kf[5], x);
-                        x = fmaf(qb.z, kf[6], x);
-                        x = fmaf(qb.w, kf[7], x);
-                        acc[hh] = x;
+                        acc_a[hh] = f2_fma(f2_pack(qa.x, qa.y), k01, acc_a[hh]);
+                        acc_b[hh] = f2_fma(f2_pack(qb.x, qb.y), k45, acc_b[hh]);
+                        acc_a[hh] = f2_fma(f2_pack(qa.z, qa.w), k23, acc_a[hh]);
+                        acc_b[hh] = f2_fma(f2_pack(qb.z, qb.w), k67, acc_b[hh]);
                     }
                 }
+            }
+            float acc[QPK];
+#pragma unroll
+            for (int hh = 0; hh < QPK; ++hh) {
+                float a0, a1, b0, b1;
+                f2_unpack(acc_a[hh], a0, a1);
+                f2_unpack(acc_b[hh], b0, b1);
+                acc[hh] = (a0 + a1) + (b0 + b1);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty_bar[st]);
@@ -340,6 +366,46 @@ __device__ void exact_key(const uint16_t *qbits, const uint16_t *kbits, int j, u
     out[18] = ~(uint32_t)j;
 }
 
+// exact_key computed by a whole warp: lane l takes products l, l + 32, ...; the
+// per-lane digit slots are integers, so summing them across the warp is exact
+// in any order (|slot| < d_k 2^47 <= 2^54); lane 0 normalises and writes.
+template <int DK>
+__device__ void exact_key_warp(const uint16_t *qbits, const uint16_t *kbits, int j, uint32_t *out, int lane) {
+    long long acc[18];
+#pragma unroll
+    for (int i = 0; i < 18; ++i) acc[i] = 0;
+#pragma unroll
+    for (int u = 0; u < DK / 32; ++u) {
+        const int c = lane + 32 * u;
+        const uint32_t qb = qbits[c], kb = kbits[c];
+        const int eq = (qb >> 7) & 0xff, ek = (kb >> 7) & 0xff;
+        const int mq = (qb & 0x7f) | (eq ? 0x80 : 0), mk = (kb & 0x7f) | (ek ? 0x80 : 0);
+        const int off = (eq ? eq - 134 : -133) + (ek ? ek - 134 : -133) + 266;
+        long long v = (long long)(mq * mk) << (off & 31);
+        if ((qb ^ kb) & 0x8000u) v = -v;
+        const int slot = off >> 5;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) acc[i] += (slot == i) ? v : 0ll;
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
+    }
+    if (lane == 0) {
+#pragma unroll
+        for (int i = 0; i < 17; ++i) {
+            const long long c = acc[i] >> 32;  // floor division by 2^32
+            acc[i] -= c * 4294967296LL;
+            acc[i + 1] += c;
+        }
+        out[0] = (uint32_t)acc[17] ^ 0x80000000u;
+#pragma unroll
+        for (int i = 1; i < 18; ++i) out[i] = (uint32_t)acc[17 - i];
+        out[18] = ~(uint32_t)j;
+    }
+}
+
 __device__ __forceinline__ bool key_greater(const uint32_t *x, const uint32_t *y) {
     for (int i = 0; i < kKeyWords; ++i)
         if (x[i] != y[i]) return x[i] > y[i];
@@ -374,6 +440,8 @@ __global__ void __launch_bounds__(kFilterThreads) topv_filter_kernel(const TopvA
     const int b = row / a.n_q, h = row % a.n_q, g = h / a.q_per_k;
     const int T = clamp_len(__ldg(a.seq_lens + b), a.t_max);
     const int j_begin = blockIdx.y * kFilterChunk;
+    pdl_launch_next();
+    pdl_wait_prev();  // scores, histograms and max |k| of the score kernel
     if (T <= a.topk || j_begin >= T) return;  // every position kept / nothing here (uniform per CTA)
     const int tid = threadIdx.x, lane = tid & 31;
 
@@ -389,6 +457,10 @@ __global__ void __launch_bounds__(kFilterThreads) topv_filter_kernel(const TopvA
     }
     __syncthreads();
     find_bucket_from_top(hist_s, kHistBuckets, (uint32_t)a.topk, &sh_d, &sh_above, warp_sums);
+    if (blockIdx.y == 0 && tid == 0) {
+        a.rowinfo[4 * row + 0] = (uint32_t)sh_d;
+        a.rowinfo[4 * row + 1] = sh_above;
+    }
     const float q1 = row_q_l1<DK>(a.q + (size_t)row * DK, red);
     const float kmax = __uint_as_float(__ldcg(a.kmax + b * a.n_k + g) << 16);
     const float two_d = __fmul_ru(2.f, score_error_bound<DK>(q1, kmax));
@@ -446,12 +518,11 @@ __global__ void __launch_bounds__(kFilterThreads) topv_filter_kernel(const TopvA
 
 template <int DK, int DV>
 __global__ void __launch_bounds__(kSelThreads, 1) topv_select_kernel(const TopvArgs a) {
-    __shared__ uint32_t hist[kRadixBuckets];
+    __shared__ uint32_t hist[kHistBuckets];
     __shared__ uint32_t warp_sums[33];
     __shared__ uint16_t q_s[DK];
     __shared__ uint32_t keys_s[kPairwiseMax][kKeyWords];
     __shared__ float red_s[kSelWarps];
-    __shared__ float o_s[kSelWarps][DV];
     __shared__ int sh_d;
     __shared__ uint32_t sh_above;
     __shared__ int sh_cnt_in, sh_na, sh_done;
@@ -460,14 +531,12 @@ __global__ void __launch_bounds__(kSelThreads, 1) topv_select_kernel(const TopvA
     float *c_s = reinterpret_cast<float *>(c_j + kCandCap);           // [kCandCap]
     uint32_t *bitmap = reinterpret_cast<uint32_t *>(c_s + kCandCap);  // [kTopvMaxContext / 32]
     uint32_t *wprefix = bitmap + kTopvMaxContext / 32;                               // [kTopvMaxContext / 32]
-    int32_t *sel_j = reinterpret_cast<int32_t *>(wprefix + kTopvMaxContext / 32);   // [kSelCap]
-    float *sel_s = reinterpret_cast<float *>(sel_j + kSelCap);                       // [kSelCap]
+    uint4 *krows = reinterpret_cast<uint4 *>(wprefix + kTopvMaxContext / 32);  // [kPairwiseMax][DK / 8]
 
     const int row = blockIdx.x;
     const int b = row / a.n_q;
     const int h = row % a.n_q;
     const int g = h / a.q_per_k;
-    const int vh = h / a.q_per_v;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int T = clamp_len(__ldg(a.seq_lens + b), a.t_max);
     const int K = a.topk;
@@ -476,12 +545,16 @@ __global__ void __launch_bounds__(kSelThreads, 1) topv_select_kernel(const TopvA
     uint8_t *ast = a.astate + (size_t)row * a.t_pad;
     uint8_t *adg = a.adigit + (size_t)row * a.t_pad;
     int32_t *idx = a.idx_out + (size_t)row * K;
-    __nv_bfloat16 *outp = a.out + (size_t)row * DV;
 
+    pdl_launch_next();
     if (tid < DK) q_s[tid] = reinterpret_cast<const uint16_t *>(a.q)[(size_t)row * DK + tid];
+    pdl_wait_prev();  // candidates, bucket and max |k| of the filter and score kernels
     if (T == 0) {
         for (int i = tid; i < K; i += kSelThreads) idx[i] = -1;
-        for (int i = tid; i < DV; i += kSelThreads) outp[i] = __float2bfloat16(0.f);
+        if (tid == 0) {
+            a.rowinfo[4 * row + 2] = __float_as_uint(0.f);
+            a.rowinfo[4 * row + 3] = 0u;
+        }
         return;
     }
     const int nwords = (T + 31) / 32;
@@ -491,14 +564,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) topv_select_kernel(const TopvA
         // every cached position is kept: positions 0..T-1, then -1
         for (int i = tid; i < K; i += kSelThreads) idx[i] = i < T ? i : -1;
         float mx = -INFINITY;
-        for (int i = tid; i < T; i += kSelThreads) {
-            const float x = s[i];
-            if (i < kSelCap) {
-                sel_j[i] = i;
-                sel_s[i] = x;
-            }
-            mx = fmaxf(mx, x);
-        }
+        for (int i = tid; i < T; i += kSelThreads) mx = fmaxf(mx, s[i]);
 #pragma unroll
         for (int off = 16; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
         if (lane == 0) red_s[warp] = mx;
@@ -534,25 +600,29 @@ __global__ void __launch_bounds__(kSelThreads, 1) topv_select_kernel(const TopvA
         for (int i = tid; i < nwords; i += kSelThreads) bitmap[i] = 0u;
         __syncthreads();
 
-        // ---- a. tau = the K-th largest score: radix select over the candidates, a byte per pass
-        uint32_t prefix = 0, pmask = 0, kk = (uint32_t)K;
-        for (int pass = 0; pass < 4; ++pass) {
-            const int shift = 24 - 8 * pass;
-            for (int i = tid; i < kRadixBuckets; i += kSelThreads) hist[i] = 0;
+        // ---- a. tau = the K-th largest score.  Its top 11 key bits are the filter's bucket,
+        //         and `above` positions lie in higher buckets (all of them candidates); a radix
+        //         select over the candidates finds the other 21 bits, 11 and then 10 at a time
+        uint32_t prefix = __ldcg(a.rowinfo + 4 * row) << 21, pmask = 0xffe00000u;
+        uint32_t kk = (uint32_t)K - __ldcg(a.rowinfo + 4 * row + 1);
+        for (int pass = 0; pass < 2; ++pass) {
+            const int shift = pass == 0 ? 10 : 0;
+            const int nb = pass == 0 ? 2048 : 1024;
+            for (int i = tid; i < nb; i += kSelThreads) hist[i] = 0;
             __syncthreads();
             for (uint32_t base = 0; base < nc; base += kSelThreads) {
                 const uint32_t i = base + tid;
                 int bucket = -1;
                 if (i < nc) {
                     const uint32_t key = float_key(cs[i]);
-                    if ((key & pmask) == prefix) bucket = (int)((key >> shift) & 0xffu);
+                    if ((key & pmask) == prefix) bucket = (int)((key >> shift) & (uint32_t)(nb - 1));
                 }
                 hist_add(hist, bucket);
             }
             __syncthreads();
-            find_bucket_from_top(hist, kRadixBuckets, kk, &sh_d, &sh_above, warp_sums);
+            find_bucket_from_top(hist, nb, kk, &sh_d, &sh_above, warp_sums);
             prefix |= (uint32_t)sh_d << shift;
-            pmask |= 0xffu << shift;
+            pmask |= (uint32_t)(nb - 1) << shift;
             kk -= sh_above;
         }
         const float tau = key_float(prefix);
@@ -597,16 +667,15 @@ __global__ void __launch_bounds__(kSelThreads, 1) topv_select_kernel(const TopvA
             for (int i = tid; i < na; i += kSelThreads) keep(alist[i]);
         } else if (na <= kPairwiseMax) {
             // rank the few ambiguous positions pairwise by exact key; their K rows are
-            // staged in shared memory first (in the kept-pairs buffer, free until compaction)
-            uint4 *krows = reinterpret_cast<uint4 *>(sel_j);  // [na][DK / 8]
+            // staged in shared memory first
             for (int i = tid; i < na * (DK / 8); i += kSelThreads) {
                 const int r = i / (DK / 8), c = i % (DK / 8);
                 krows[i] = __ldg(reinterpret_cast<const uint4 *>(krow0 + (size_t)alist[r] * kstride) + c);
             }
             __syncthreads();
-            if (tid < na)
-                exact_key<DK>(q_s, reinterpret_cast<const uint16_t *>(krows + tid * (DK / 8)), alist[tid],
-                              keys_s[tid]);
+            for (int r = warp; r < na; r += kSelWarps)
+                exact_key_warp<DK>(q_s, reinterpret_cast<const uint16_t *>(krows + r * (DK / 8)), alist[r],
+                                   keys_s[r], lane);
             __syncthreads();
             if (tid < na) {
                 int better = 0;
@@ -673,13 +742,8 @@ __global__ void __launch_bounds__(kSelThreads, 1) topv_select_kernel(const TopvA
             const uint32_t word = bitmap[j >> 5];
             if ((word >> (j & 31)) & 1u) {
                 const uint32_t slot = wprefix[j >> 5] + __popc(word & ((1u << (j & 31)) - 1u));
-                const float x = cs[i];
                 idx[slot] = j;
-                if (slot < (uint32_t)kSelCap) {
-                    sel_j[slot] = j;
-                    sel_s[slot] = x;
-                }
-                mx = fmaxf(mx, x);
+                mx = fmaxf(mx, cs[i]);
             }
         }
         if (tid == 0 && nsel != K) record_error(a.status, DIFFQKV_ERR_INVALID_ARG);
@@ -689,15 +753,39 @@ __global__ void __launch_bounds__(kSelThreads, 1) topv_select_kernel(const TopvA
         if (lane == 0) red_s[warp] = mx;
     }
     __syncthreads();
-    float m = red_s[0];
-#pragma unroll 1
-    for (int w = 1; w < kSelWarps; ++w) m = fmaxf(m, red_s[w]);
-    __syncthreads();
+    if (tid == 0) {
+        float m = red_s[0];
+        for (int w = 1; w < kSelWarps; ++w) m = fmaxf(m, red_s[w]);
+        a.rowinfo[4 * row + 2] = __float_as_uint(m);
+        a.rowinfo[4 * row + 3] = (uint32_t)nsel;
+    }
+}
 
-    // ---- e. renormalised softmax over the kept rows; only their V rows are read
+// ------------------------------------------------------------------ 4. gather
+
+// CTA (row, part) sums its share of the kept positions (in ascending order):
+// sum_j 2^((s_j - m) scale log2 e) v_j and the weight sum, with m the largest
+// kept score; the last CTA of the row to finish adds the parts in a fixed order
+// and writes the normalised output.
+template <int DV>
+__global__ void __launch_bounds__(kGatherThreads) topv_gather_kernel(const TopvArgs a) {
+    __shared__ float o_s[kGatherWarps][DV];
+    __shared__ float l_s[kGatherWarps];
+    __shared__ bool sh_last;
+    const int row = blockIdx.x, part = blockIdx.y, nparts = gridDim.y;
+    const int b = row / a.n_q, h = row % a.n_q, vh = h / a.q_per_v;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    pdl_wait_prev();  // kept positions and their maximum from the select kernel
+    const float m = __uint_as_float(__ldcg(a.rowinfo + 4 * row + 2));
+    const int nsel = (int)__ldcg(a.rowinfo + 4 * row + 3);
+    const int i_begin = (int)(((long long)nsel * part) / nparts);
+    const int i_end = (int)(((long long)nsel * (part + 1)) / nparts);
+    const int32_t *idx = a.idx_out + (size_t)row * a.topk;
+    const float *s = a.scores + (size_t)row * a.t_pad;
+
     constexpr int CPV = DV / 8;      // lanes per V row
     constexpr int RPW = 32 / CPV;    // V rows per warp step
-    constexpr int GU = 8;            // V rows in flight per lane
+    constexpr int GU = 4;            // V rows in flight per lane
     const int vc = lane % CPV, vs = lane / CPV;
     float o[8];
 #pragma unroll
@@ -705,16 +793,15 @@ __global__ void __launch_bounds__(kSelThreads, 1) topv_select_kernel(const TopvA
     float l = 0.f;
     const __nv_bfloat16 *vbase = a.v + ((size_t)b * a.t_max * a.n_v + vh) * DV + vc * 8;
     const size_t vstride = (size_t)a.n_v * DV;
-    for (int i0 = warp * RPW; i0 < nsel; i0 += kSelWarps * RPW * GU) {
+    for (int i0 = i_begin + warp * RPW; i0 < i_end; i0 += kGatherWarps * RPW * GU) {
         uint4 vv[GU];
         float w[GU];
 #pragma unroll
         for (int u = 0; u < GU; ++u) {
-            const int i = i0 + u * kSelWarps * RPW + vs;
-            if (i < nsel) {
-                const int j = i < kSelCap ? sel_j[i] : __ldcg(idx + i);
-                const float x = i < kSelCap ? sel_s[i] : s[j];
-                w[u] = fast_exp2((x - m) * a.scale_log2);
+            const int i = i0 + u * kGatherWarps * RPW + vs;
+            const int j = i < i_end ? __ldcg(idx + i) : -1;
+            if (j >= 0) {
+                w[u] = fast_exp2((__ldcg(s + j) - m) * a.scale_log2);
                 vv[u] = __ldg(reinterpret_cast<const uint4 *>(vbase + (size_t)j * vstride));
             } else {
                 w[u] = 0.f;
@@ -741,17 +828,29 @@ __global__ void __launch_bounds__(kSelThreads, 1) topv_select_kernel(const TopvA
 #pragma unroll
         for (int e = 0; e < 8; ++e) o_s[warp][vc * 8 + e] = o[e];
     }
-    if (lane == 0) red_s[warp] = l;
+    if (lane == 0) l_s[warp] = l;
     __syncthreads();
-    if (tid < DV) {
-        float acc = 0.f, lt = 0.f;
-#pragma unroll 1
-        for (int w = 0; w < kSelWarps; ++w) {
-            acc += o_s[w][tid];
-            lt += red_s[w];
-        }
-        outp[tid] = __float2bfloat16(lt > 0.f ? acc / lt : 0.f);
+    float *mine = a.gpart + ((size_t)row * a.gather_split + part) * (DV + 1);
+    for (int c = tid; c <= DV; c += kGatherThreads) {
+        float acc = 0.f;
+        for (int w = 0; w < kGatherWarps; ++w) acc += c < DV ? o_s[w][c] : l_s[w];
+        mine[c] = acc;
     }
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) sh_last = atomicAdd(a.gcount + row, 1u) == (uint32_t)(nparts - 1);
+    __syncthreads();
+    if (!sh_last) return;
+    __threadfence();
+    const float *parts = a.gpart + (size_t)row * a.gather_split * (DV + 1);
+    float lt = 0.f;
+    for (int p = 0; p < nparts; ++p) lt += __ldcg(parts + (size_t)p * (DV + 1) + DV);
+    for (int c = tid; c < DV; c += kGatherThreads) {
+        float acc = 0.f;
+        for (int p = 0; p < nparts; ++p) acc += __ldcg(parts + (size_t)p * (DV + 1) + c);
+        a.out[(size_t)row * DV + c] = __float2bfloat16(lt > 0.f ? acc / lt : 0.f);
+    }
+    if (tid == 0) a.gcount[row] = 0u;
 }
 
 size_t align_up(size_t x, size_t al) { return (x + al - 1) / al * al; }
@@ -791,15 +890,46 @@ RowFn pick_select(int dk, int dv) {
     return nullptr;
 }
 
+RowFn pick_gather(int dv) {
+    if (dv == 64) return topv_gather_kernel<64>;
+    if (dv == 128) return topv_gather_kernel<128>;
+    return nullptr;
+}
+
 size_t padded_len(int32_t t_max) { return align_up((size_t)t_max, 64); }
 
 // kmax entries, rounded up so the histograms after them start 16-byte aligned.
 size_t kmax_slots(const diffqkv_dims_t *d) { return align_up((size_t)d->batch * d->n_k, 4); }
 
-// Zero-filled per call: kmax [B*n_k, padded], histograms [rows][2048], candidate counts [rows].
+// Zero-filled per call: kmax [B*n_k, padded], histograms [rows][2048], candidate counts [rows],
+// gather counters [rows].
 size_t zeroed_bytes(const diffqkv_dims_t *d) {
     const size_t rows = (size_t)d->batch * d->n_q;
-    return kmax_slots(d) * 4 + rows * kHistBuckets * 4 + rows * 4;
+    return kmax_slots(d) * 4 + rows * kHistBuckets * 4 + rows * 4 * 2;
+}
+
+int gather_split(int32_t topk) { return std::max(1, std::min(kGatherMaxSplit, (topk + kGatherRows - 1) / kGatherRows)); }
+
+// rowinfo [rows][4] and the gather partials [rows][split][d_v + 1]
+size_t row_bytes(const diffqkv_dims_t *d, int32_t topk) {
+    const size_t rows = (size_t)d->batch * d->n_q;
+    return align_up(rows * 16, 256) + align_up(rows * (size_t)gather_split(topk) * (d->d_v + 1) * 4, 256);
+}
+
+template <typename... P, typename... A>
+cudaError_t launch_after_prev(void (*kernel)(P...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                              A... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
 }  // namespace
@@ -808,7 +938,7 @@ size_t topv_workspace_size(const diffqkv_dims_t *d, int32_t t_max, int32_t topk)
     if (validate_dims(d) != DIFFQKV_OK || t_max < 1 || topk < 1) return 0;
     const size_t rows = (size_t)d->batch * d->n_q;
     const size_t per = padded_len(t_max);
-    return kTopvHeader + align_up(zeroed_bytes(d), 256) + align_up(rows * per * 4, 256) * 4 +
+    return kTopvHeader + align_up(zeroed_bytes(d), 256) + row_bytes(d, topk) + align_up(rows * per * 4, 256) * 4 +
            align_up(rows * per, 256) * 2;
 }
 
@@ -824,7 +954,8 @@ diffqkv_status_t topv_launch(const diffqkv_dims_t *d, const void *q, const void 
     ScoreFn score = pick_score(d->d_k, qpk);
     RowFn filter = pick_filter(d->d_k);
     RowFn select = pick_select(d->d_k, d->d_v);
-    if (!score || !filter || !select) return DIFFQKV_ERR_UNSUPPORTED;
+    RowFn gather = pick_gather(d->d_v);
+    if (!score || !filter || !select || !gather) return DIFFQKV_ERR_UNSUPPORTED;
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
         (reinterpret_cast<uintptr_t>(idx_out) & 3u) || (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
         return DIFFQKV_ERR_MISALIGNED;
@@ -842,7 +973,12 @@ diffqkv_status_t topv_launch(const diffqkv_dims_t *d, const void *q, const void 
     a.kmax = reinterpret_cast<uint32_t *>(ws);
     a.ghist = a.kmax + kmax_slots(d);  // 16-byte aligned (read with 16-byte loads)
     a.ncand = a.ghist + rows * kHistBuckets;
+    a.gcount = a.ncand + rows;
     ws += align_up(zeroed_bytes(d), 256);
+    a.rowinfo = reinterpret_cast<uint32_t *>(ws);
+    a.gpart = reinterpret_cast<float *>(ws + align_up(rows * 16, 256));
+    a.gather_split = gather_split(topk);
+    ws += row_bytes(d, topk);
     a.scores = reinterpret_cast<float *>(ws);
     ws += align_up(rows * t_pad * 4, 256);
     a.cand_j = reinterpret_cast<int32_t *>(ws);
@@ -892,18 +1028,29 @@ diffqkv_status_t topv_launch(const diffqkv_dims_t *d, const void *q, const void 
     const int per_sm = std::max(1, std::min(3, (227 * 1024) / (score_smem + 1024)));
     const int units = d->batch * d->n_k;
     const int ygrid = std::max(1, (dev.num_sms * per_sm) / units);
-    const int select_smem = kCandCap * 8 + 2 * (kTopvMaxContext / 8) + kSelCap * 8;
+    const int select_smem = kCandCap * 8 + 2 * (kTopvMaxContext / 8) + kPairwiseMax * d->d_k * 2;
     if (ensure_dynamic_smem((const void *)score, score_smem) != DIFFQKV_OK ||
         ensure_dynamic_smem((const void *)select, select_smem) != DIFFQKV_OK)
         return DIFFQKV_ERR_CUDA;
     score<<<dim3(units, ygrid), kScoreThreads + 32, score_smem, stream>>>(tm_k, a);
     if (cudaGetLastError() != cudaSuccess) return DIFFQKV_ERR_CUDA;
     // 2. filter: every row, in chunks of kFilterChunk positions (chunks past a row's length return at once)
-    filter<<<dim3((unsigned)rows, (t_max + kFilterChunk - 1) / kFilterChunk), kFilterThreads, 0, stream>>>(a);
-    if (cudaGetLastError() != cudaSuccess) return DIFFQKV_ERR_CUDA;
-    // 3. select + gather
-    select<<<(unsigned)rows, kSelThreads, select_smem, stream>>>(a);
-    if (cudaGetLastError() != cudaSuccess) return DIFFQKV_ERR_CUDA;
+    if (launch_after_prev(filter, dim3((unsigned)rows, (t_max + kFilterChunk - 1) / kFilterChunk),
+                          dim3(kFilterThreads), 0, stream, a) != cudaSuccess) {
+        cudaGetLastError();
+        return DIFFQKV_ERR_CUDA;
+    }
+    // 3. select: one CTA per row
+    if (launch_after_prev(select, dim3((unsigned)rows), dim3(kSelThreads), select_smem, stream, a) != cudaSuccess) {
+        cudaGetLastError();
+        return DIFFQKV_ERR_CUDA;
+    }
+    // 4. gather: gather_split CTAs per row
+    if (launch_after_prev(gather, dim3((unsigned)rows, (unsigned)a.gather_split), dim3(kGatherThreads), 0, stream,
+                          a) != cudaSuccess) {
+        cudaGetLastError();
+        return DIFFQKV_ERR_CUDA;
+    }
     return DIFFQKV_OK;
 }
 

@@ -384,7 +384,7 @@ def time_paths(ak, peaks, steps: int, warmup: int):
     hbm = float(peaks["hbm_gbs"])
     res[w.name] = {"us": ms * 1e3, "algorithmic_bytes": nbytes, "gbs": nbytes / (ms * 1e-3) / 1e9,
                    "bound": "hbm", "peak_gbs": hbm, "frac": nbytes / (ms * 1e-3) / 1e9 / hbm,
-                   "launches_per_call": 2}
+                   "launches_per_call": 3}
     assert ak.device_status() == 0
     return res
 
@@ -429,6 +429,17 @@ def main():
                "diffqkv_time_reduction": 1.0 - ms_per_step / ctrl_ms}
     del ctrl
 
+    # long-context ragged decode (lengths 16384..131072) and its GQA control: the same kernel, per-launch events
+    long_ctx = {}
+    for w in (wl.DECODE_RAGGED, wl.DECODE_RAGGED_GQA):
+        r = time_decode(ak, w, 50, args.warmup, world)
+        gbs = r["kv_bytes"] / (r["launch_ms_mean"] * 1e-3) / 1e9
+        long_ctx[w.name] = {"us_per_step": r["launch_ms_mean"] * 1e3, "kv_bytes": r["kv_bytes"], "gbs": gbs,
+                            "frac_of_peak": gbs / peak, "steps": 50}
+        del r
+    rag, rag_gqa = long_ctx[wl.DECODE_RAGGED.name], long_ctx[wl.DECODE_RAGGED_GQA.name]
+    long_ctx["diffqkv_time_reduction"] = 1.0 - rag["us_per_step"] / rag_gqa["us_per_step"]
+
     e2e_ms, h2d, d2h = time_e2e(ak, WORKLOAD, main_res["inputs"], args.e2e_steps)
     e2e_ms = max_over_ranks(e2e_ms, world)
     e2e = {"value": total_bytes / (e2e_ms * 1e-3) / 1e9, "unit": UNIT, "h2d_bytes_per_step": h2d,
@@ -456,6 +467,7 @@ def main():
                        "kv_bytes_per_gpu_step": main_res["kv_bytes"]},
             "pct_of_hbm_peak": 100.0 * achieved / peak,
             "gqa_control": control,
+            "long_context": long_ctx,
             "paths": paths,
             "roofline": roofline,
             "cpu_baseline": cpu,

@@ -119,3 +119,24 @@ def test_full_topv_workload(cuda_device):
     r_out, r_idx = oracle.decode_topv(cpu["q"], cpu["k_cache"], cpu["v_cache"], cpu["seq_lens"], w.topk, d["scale"])
     assert np.array_equal(idx.cpu().numpy(), r_idx)
     assert_parity(out, r_out, w.name)
+
+
+@pytest.mark.parametrize("topk", [64, 1024, 4000])
+def test_workspace_reuse_is_bitwise_stable(cuda_device, topk):
+    """Two calls on one workspace (the gather's per-row counters must come back to
+    zero) give identical bits: the parts of a row are added in a fixed order."""
+    d = wl.random_decode_inputs(3, 6000, wl.DIFFQKV, seed=308, seq_lens=[6000, 2500, 4100])
+    g = {k: (v.to(cuda_device) if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
+    dims = ak.make_dims(3, 16, 4, 16, 64, 128, d["scale"])
+    ws = ak.decode_topv_workspace(dims, 6000, topk, cuda_device)
+    runs = []
+    for _ in range(2):
+        out, idx = ak.decode_topv(g["q"], g["k_cache"], g["v_cache"], g["seq_lens"], topk, scale=d["scale"],
+                                  workspace=ws)
+        torch.cuda.synchronize()
+        assert ak.device_status() == 0
+        runs.append((out.clone(), idx.clone()))
+    assert torch.equal(runs[0][0], runs[1][0]) and torch.equal(runs[0][1], runs[1][1])
+    r_out, r_idx = oracle.decode_topv(d["q"], d["k_cache"], d["v_cache"], d["seq_lens"], topk, d["scale"])
+    assert np.array_equal(runs[0][1].cpu().numpy(), r_idx)
+    assert_parity(runs[0][0], r_out, f"reuse k={topk}")
