@@ -46,6 +46,8 @@ namespace {
 constexpr int kScoreThreads = 128;      // consumer threads of the score kernel (+1 producer warp)
 constexpr int kScoreTile = 128;         // positions per TMA tile (one per consumer thread)
 constexpr int kHistBuckets = 2048;      // first radix digit: top 11 bits of the order key
+constexpr int kHistWords = kHistBuckets / 2;  // score-kernel histogram: two 16-bit counters per word
+constexpr int kScoreMaxTilesPerCta = 511;     // keeps a CTA's positions (and any counter) below 2^16
 constexpr int kRadixBuckets = 256;      // later radix digits: one byte
 constexpr int kFilterThreads = 256;
 constexpr int kFilterChunk = 4096;      // positions per filter CTA
@@ -120,12 +122,38 @@ __device__ __forceinline__ float score_error_bound(float q_l1, float kmax) {
 
 // ------------------------------------------------------------------ 1. scores
 
+// Sum over the 4 lanes of a position group of HG per-lane partials, one per
+// head; returns the total of head `head_of_lane(r)` to lane r (r = lane % 4).
+// For HG = 4 a butterfly leaves head r's total in lane r (3 shuffles).
+template <int HG>
+__device__ __forceinline__ float reduce_heads(const float (&v)[HG], int r) {
+    if constexpr (HG == 4) {
+        const bool hi2 = (r & 2) != 0;
+        const float a0 = (hi2 ? v[2] : v[0]) + __shfl_xor_sync(0xffffffffu, hi2 ? v[0] : v[2], 2);
+        const float a1 = (hi2 ? v[3] : v[1]) + __shfl_xor_sync(0xffffffffu, hi2 ? v[1] : v[3], 2);
+        const bool hi1 = (r & 1) != 0;
+        return (hi1 ? a1 : a0) + __shfl_xor_sync(0xffffffffu, hi1 ? a0 : a1, 1);
+    } else if constexpr (HG == 2) {
+        const bool hi2 = (r & 2) != 0;
+        float x = (hi2 ? v[1] : v[0]) + __shfl_xor_sync(0xffffffffu, hi2 ? v[0] : v[1], 2);
+        return x + __shfl_xor_sync(0xffffffffu, x, 1);
+    } else {
+        float x = v[0] + __shfl_xor_sync(0xffffffffu, v[0], 2);
+        return x + __shfl_xor_sync(0xffffffffu, x, 1);
+    }
+}
+template <int HG>
+__device__ __forceinline__ bool lane_writes(int r) { return HG == 4 ? true : (HG == 2 ? (r & 1) == 0 : r == 0); }
+template <int HG>
+__device__ __forceinline__ int head_of_lane(int r) { return HG == 4 ? r : (HG == 2 ? r >> 1 : 0); }
+
 // One CTA streams K tiles of one (batch, K head) over an equal share of its
-// positions: a producer thread issues TMA loads (128-byte swizzle, so a thread
-// reading "its" 128-byte row hits eight distinct 16-byte bank groups) into a
-// ring of tiles; each of the 128 consumer threads owns one position of the tile
-// and accumulates the dot products of all n_q/n_k query heads of the group,
-// with q read from shared memory by broadcast.
+// positions: a producer thread issues TMA loads (128-byte swizzle) into a ring
+// of tiles.  Four lanes share a position: lane r reads 16-byte chunks
+// (u / 2) * 8 + 2 r + u % 2 of the row, so a quarter warp (two positions, one
+// even and one odd) touches eight distinct bank groups, and holds the matching
+// elements of q for up to four query heads in registers.  The four partial dot
+// products of each head are added across the group, and lane r writes head r.
 template <int DK, int QPK>
 __global__ void __launch_bounds__(kScoreThreads + 32) topv_score_kernel(const __grid_constant__ CUtensorMap tm_k,
                                                                          const TopvArgs a) {
@@ -134,8 +162,8 @@ __global__ void __launch_bounds__(kScoreThreads + 32) topv_score_kernel(const __
     extern __shared__ uint8_t dsm_raw[];
     uint8_t *dsm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *tiles = dsm;                                                                 // [stages][TILE_BYTES]
-    uint32_t *hist_s = reinterpret_cast<uint32_t *>(dsm + a.score_stages * TILE_BYTES);  // [QPK][2048]
-    float *q_s = reinterpret_cast<float *>(hist_s + QPK * kHistBuckets);                 // [QPK][DK]
+    uint32_t *hist_s = reinterpret_cast<uint32_t *>(dsm + a.score_stages * TILE_BYTES);  // [QPK][1024]
+    float *q_s = reinterpret_cast<float *>(hist_s + QPK * kHistWords);                   // [QPK][DK]
     uint64_t *full_bar = reinterpret_cast<uint64_t *>(q_s + QPK * DK);
     uint64_t *empty_bar = full_bar + a.score_stages;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(empty_bar + a.score_stages);
@@ -159,7 +187,7 @@ __global__ void __launch_bounds__(kScoreThreads + 32) topv_score_kernel(const __
         fence_barrier_init();
     }
     pdl_launch_next();
-    for (int i = tid; i < QPK * kHistBuckets; i += blockDim.x) hist_s[i] = 0;
+    for (int i = tid; i < QPK * kHistWords; i += blockDim.x) hist_s[i] = 0;
     for (int i = tid; i < QPK * DK; i += blockDim.x) {
         const int hh = i / DK, c = i % DK;
         q_s[i] = __bfloat162float(a.q[((size_t)b * a.n_q + g * QPK + hh) * DK + c]);
@@ -188,61 +216,85 @@ __global__ void __launch_bounds__(kScoreThreads + 32) topv_score_kernel(const __
                                   a.wait_limit_ns, nullptr, a.status);
         }
     } else {
-        // ---- consumers: thread tid owns position tile * kScoreTile + tid
+        // ---- consumers: warp w takes positions 32 w .. 32 w + 31 of each tile, 8 at a time
+        constexpr int HG = QPK < 4 ? QPK : 4;  // heads per pass (their q in registers)
+        constexpr int NPASS = QPK / HG;
+        constexpr int CPL = DK / 32;           // 16-byte chunks of a K row per lane
+        const int r = lane & 3, pg = lane >> 2;
         uint32_t kmx2 = 0;  // two packed |bf16| maxima
         float *sbase = a.scores + ((size_t)b * a.n_q + g * QPK) * a.t_pad;
+        f32x2_t qp[HG][CPL][4];  // q[head][chunk elements 2i, 2i + 1]
+        auto load_q = [&](int pass) {
+#pragma unroll
+            for (int hh = 0; hh < HG; ++hh)
+#pragma unroll
+                for (int u = 0; u < CPL; ++u) {
+                    const int chunk = (u >> 1) * 8 + 2 * r + (u & 1);
+                    const float *qs = q_s + (pass * HG + hh) * DK + chunk * 8;
+                    const float4 x = *reinterpret_cast<const float4 *>(qs);
+                    const float4 y = *reinterpret_cast<const float4 *>(qs + 4);
+                    qp[hh][u][0] = f2_pack(x.x, x.y);
+                    qp[hh][u][1] = f2_pack(x.z, x.w);
+                    qp[hh][u][2] = f2_pack(y.x, y.y);
+                    qp[hh][u][3] = f2_pack(y.z, y.w);
+                }
+        };
+        if (NPASS == 1) load_q(0);
         for (int t = tb, k = 0; t < te; ++t, ++k) {
             const int st = k % a.score_stages;
             mbar_wait_bounded(&full_bar[st], (uint32_t)((k / a.score_stages) & 1), a.wait_limit_ns, abort_flag,
                               a.status);
-            const uint8_t *row = tiles + st * TILE_BYTES + tid * 128;
-            const int j = t * kScoreTile + tid;
-            const uint32_t live = j < T ? 0x7fff7fffu : 0u;  // the |k| bound covers cached positions only
-            // even/odd keys of each head in packed fp32 pairs, split over two chains per head:
-            // every lane of fma.rn.f32x2 is an IEEE fp32 FMA, and each product meets at most
-            // d_k/4 + 2 roundings on its way into the score
-            f32x2_t acc_a[QPK], acc_b[QPK];
+            const uint8_t *tile = tiles + st * TILE_BYTES;
+#pragma unroll 1
+            for (int pass = 0; pass < NPASS; ++pass) {
+                if (NPASS > 1) load_q(pass);
+#pragma unroll 2
+                for (int step = 0; step < 4; ++step) {
+                    const int pos = warp * 32 + step * 8 + pg;  // row of the tile
+                    const int j = t * kScoreTile + pos;
+                    const uint32_t live = (pass == 0 && j < T) ? 0x7fff7fffu : 0u;  // |k| of cached positions
+                    // even/odd elements in packed fp32 pairs: every lane of fma.rn.f32x2 is an IEEE
+                    // fp32 FMA; a product meets at most 4 CPL + 3 (<= d_k) roundings on its way into the score
+                    f32x2_t acc[HG];
 #pragma unroll
-            for (int hh = 0; hh < QPK; ++hh) acc_a[hh] = acc_b[hh] = 0ull;
+                    for (int hh = 0; hh < HG; ++hh) acc[hh] = 0ull;
 #pragma unroll
-            for (int kb = 0; kb < KB; ++kb) {
+                    for (int u = 0; u < CPL; ++u) {
+                        const int chunk = (u >> 1) * 8 + 2 * r + (u & 1);
+                        const uint4 kv = lds128(tile + (chunk >> 3) * (kScoreTile * 128) + pos * 128 +
+                                                (((chunk & 7) ^ (pos & 7)) << 4));
+                        kmx2 = __vmaxu2(kmx2, kv.x & live);
+                        kmx2 = __vmaxu2(kmx2, kv.y & live);
+                        kmx2 = __vmaxu2(kmx2, kv.z & live);
+                        kmx2 = __vmaxu2(kmx2, kv.w & live);
+                        const f32x2_t k01 = bf16x2_to_f2(kv.x), k23 = bf16x2_to_f2(kv.y);
+                        const f32x2_t k45 = bf16x2_to_f2(kv.z), k67 = bf16x2_to_f2(kv.w);
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const uint4 kv = lds128(row + kb * (kScoreTile * 128) + ((c ^ (tid & 7)) << 4));
-                    kmx2 = __vmaxu2(kmx2, kv.x & live);
-                    kmx2 = __vmaxu2(kmx2, kv.y & live);
-                    kmx2 = __vmaxu2(kmx2, kv.z & live);
-                    kmx2 = __vmaxu2(kmx2, kv.w & live);
-                    const f32x2_t k01 = bf16x2_to_f2(kv.x), k23 = bf16x2_to_f2(kv.y);
-                    const f32x2_t k45 = bf16x2_to_f2(kv.z), k67 = bf16x2_to_f2(kv.w);
+                        for (int hh = 0; hh < HG; ++hh) {
+                            acc[hh] = f2_fma(qp[hh][u][0], k01, acc[hh]);
+                            acc[hh] = f2_fma(qp[hh][u][1], k23, acc[hh]);
+                            acc[hh] = f2_fma(qp[hh][u][2], k45, acc[hh]);
+                            acc[hh] = f2_fma(qp[hh][u][3], k67, acc[hh]);
+                        }
+                    }
+                    float part[HG];
 #pragma unroll
-                    for (int hh = 0; hh < QPK; ++hh) {
-                        const float4 qa = *reinterpret_cast<const float4 *>(q_s + hh * DK + kb * 64 + c * 8);
-                        const float4 qb = *reinterpret_cast<const float4 *>(q_s + hh * DK + kb * 64 + c * 8 + 4);
-                        acc_a[hh] = f2_fma(f2_pack(qa.x, qa.y), k01, acc_a[hh]);
-                        acc_b[hh] = f2_fma(f2_pack(qb.x, qb.y), k45, acc_b[hh]);
-                        acc_a[hh] = f2_fma(f2_pack(qa.z, qa.w), k23, acc_a[hh]);
-                        acc_b[hh] = f2_fma(f2_pack(qb.z, qb.w), k67, acc_b[hh]);
+                    for (int hh = 0; hh < HG; ++hh) {
+                        float x0, x1;
+                        f2_unpack(acc[hh], x0, x1);
+                        part[hh] = x0 + x1;
+                    }
+                    const float score = reduce_heads<HG>(part, r);
+                    if (lane_writes<HG>(r) && j < T) {
+                        const int hh = pass * HG + head_of_lane<HG>(r);
+                        sbase[(size_t)hh * a.t_pad + j] = score;
+                        const uint32_t bk = float_key(score) >> 21;
+                        atomicAdd(hist_s + hh * kHistWords + (bk >> 1), 1u << ((bk & 1u) << 4));
                     }
                 }
             }
-            float acc[QPK];
-#pragma unroll
-            for (int hh = 0; hh < QPK; ++hh) {
-                float a0, a1, b0, b1;
-                f2_unpack(acc_a[hh], a0, a1);
-                f2_unpack(acc_b[hh], b0, b1);
-                acc[hh] = (a0 + a1) + (b0 + b1);
-            }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty_bar[st]);
-            if (j < T) {
-#pragma unroll
-                for (int hh = 0; hh < QPK; ++hh) {
-                    sbase[(size_t)hh * a.t_pad + j] = acc[hh];
-                    atomicAdd(hist_s + hh * kHistBuckets + (float_key(acc[hh]) >> 21), 1u);
-                }
-            }
         }
         uint32_t kmx = max(kmx2 & 0xffffu, kmx2 >> 16);
 #pragma unroll
@@ -250,9 +302,13 @@ __global__ void __launch_bounds__(kScoreThreads + 32) topv_score_kernel(const __
         if (lane == 0) atomicMax(a.kmax + unit, kmx);
     }
     __syncthreads();
+    // word i holds buckets 2i (low half) and 2i + 1 of the group's [QPK][2048] histograms
     uint32_t *gh = a.ghist + ((size_t)b * a.n_q + g * QPK) * kHistBuckets;
-    for (int i = tid; i < QPK * kHistBuckets; i += blockDim.x)
-        if (hist_s[i]) atomicAdd(gh + i, hist_s[i]);
+    for (int i = tid; i < QPK * kHistWords; i += blockDim.x) {
+        const uint32_t w = hist_s[i];
+        if (w & 0xffffu) atomicAdd(gh + 2 * i, w & 0xffffu);
+        if (w >> 16) atomicAdd(gh + 2 * i + 1, w >> 16);
+    }
 }
 
 // ------------------------------------------------------------------ helpers
@@ -445,6 +501,21 @@ __global__ void __launch_bounds__(kFilterThreads) topv_filter_kernel(const TopvA
     if (T <= a.topk || j_begin >= T) return;  // every position kept / nothing here (uniform per CTA)
     const int tid = threadIdx.x, lane = tid & 31;
 
+    // this CTA's scores first (they do not depend on the threshold): lane-interleaved
+    // 16-byte loads, each warp load covering 512 contiguous bytes
+    const float *s = a.scores + (size_t)row * a.t_pad;
+    int32_t *cj = a.cand_j + (size_t)row * a.t_pad;
+    float *cs = a.cand_s + (size_t)row * a.t_pad;
+    const int j_end = min(T, j_begin + kFilterChunk);
+    static_assert(kFilterChunk == kFilterThreads * 16, "one pass of 16 positions per thread");
+    float4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int p = j_begin + (u * kFilterThreads + tid) * 4;
+        v[u] = p < j_end ? __ldcg(reinterpret_cast<const float4 *>(s + p)) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    const uint32_t kmax_bits = __ldcg(a.kmax + b * a.n_k + g);
+
     // bucket of the k-th largest score, and the lower end of the range that can be kept
     {
         const uint4 *src = reinterpret_cast<const uint4 *>(a.ghist + (size_t)row * kHistBuckets);
@@ -462,25 +533,11 @@ __global__ void __launch_bounds__(kFilterThreads) topv_filter_kernel(const TopvA
         a.rowinfo[4 * row + 1] = sh_above;
     }
     const float q1 = row_q_l1<DK>(a.q + (size_t)row * DK, red);
-    const float kmax = __uint_as_float(__ldcg(a.kmax + b * a.n_k + g) << 16);
-    const float two_d = __fmul_ru(2.f, score_error_bound<DK>(q1, kmax));
+    const float two_d = __fmul_ru(2.f, score_error_bound<DK>(q1, __uint_as_float(kmax_bits << 16)));
     // (bucket 0 starts at the NaN patterns: everything in it and above is a candidate)
     const float lower = sh_d == 0 ? -INFINITY : __fsub_rd(key_float((uint32_t)sh_d << 21), two_d);
-
-    const float *s = a.scores + (size_t)row * a.t_pad;
-    int32_t *cj = a.cand_j + (size_t)row * a.t_pad;
-    float *cs = a.cand_s + (size_t)row * a.t_pad;
-    const int j_end = min(T, j_begin + kFilterChunk);
-    // lane-interleaved 16-byte loads: each warp load covers 512 contiguous bytes.
-    // A thread's hits form a 16-bit mask; one block scan gives every thread its
-    // slots and one global atomic per CTA reserves them.
-    static_assert(kFilterChunk == kFilterThreads * 16, "one pass of 16 positions per thread");
-    float4 v[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-        const int p = j_begin + (u * kFilterThreads + tid) * 4;
-        v[u] = p < j_end ? __ldcg(reinterpret_cast<const float4 *>(s + p)) : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
+    // a thread's hits form a 16-bit mask; one block scan gives every thread its slots and
+    // one global atomic per CTA reserves them
     uint32_t hits = 0;
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
@@ -785,7 +842,7 @@ __global__ void __launch_bounds__(kGatherThreads) topv_gather_kernel(const TopvA
 
     constexpr int CPV = DV / 8;      // lanes per V row
     constexpr int RPW = 32 / CPV;    // V rows per warp step
-    constexpr int GU = 4;            // V rows in flight per lane
+    constexpr int GU = 8;            // V rows in flight per lane: a CTA's 128 rows in one round
     const int vc = lane % CPV, vs = lane / CPV;
     float o[8];
 #pragma unroll
@@ -794,27 +851,33 @@ __global__ void __launch_bounds__(kGatherThreads) topv_gather_kernel(const TopvA
     const __nv_bfloat16 *vbase = a.v + ((size_t)b * a.t_max * a.n_v + vh) * DV + vc * 8;
     const size_t vstride = (size_t)a.n_v * DV;
     for (int i0 = i_begin + warp * RPW; i0 < i_end; i0 += kGatherWarps * RPW * GU) {
-        uint4 vv[GU];
-        float w[GU];
+        // every position first, then every score and V row: two dependent rounds of loads
+        int jj[GU];
 #pragma unroll
         for (int u = 0; u < GU; ++u) {
             const int i = i0 + u * kGatherWarps * RPW + vs;
-            const int j = i < i_end ? __ldcg(idx + i) : -1;
-            if (j >= 0) {
-                w[u] = fast_exp2((__ldcg(s + j) - m) * a.scale_log2);
-                vv[u] = __ldg(reinterpret_cast<const uint4 *>(vbase + (size_t)j * vstride));
+            jj[u] = i < i_end ? __ldcg(idx + i) : -1;
+        }
+        uint4 vv[GU];
+        float sx[GU];
+#pragma unroll
+        for (int u = 0; u < GU; ++u) {
+            if (jj[u] >= 0) {
+                sx[u] = __ldcg(s + jj[u]);
+                vv[u] = __ldg(reinterpret_cast<const uint4 *>(vbase + (size_t)jj[u] * vstride));
             } else {
-                w[u] = 0.f;
+                sx[u] = -INFINITY;
                 vv[u] = make_uint4(0, 0, 0, 0);
             }
         }
 #pragma unroll
         for (int u = 0; u < GU; ++u) {
+            const float w = jj[u] >= 0 ? fast_exp2((sx[u] - m) * a.scale_log2) : 0.f;
             float vf[8];
             unpack8(vv[u], vf);
-            l += w[u];
+            l += w;
 #pragma unroll
-            for (int e = 0; e < 8; ++e) o[e] = fmaf(w[u], vf[e], o[e]);
+            for (int e = 0; e < 8; ++e) o[e] = fmaf(w, vf[e], o[e]);
         }
     }
     // reduce over the RPW row slots of the warp, then over warps
@@ -1020,14 +1083,17 @@ diffqkv_status_t topv_launch(const diffqkv_dims_t *d, const void *q, const void 
                             CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != DIFFQKV_OK) return st;
     const int tile_bytes = kScoreTile * d->d_k * 2;
-    const int fixed = qpk * kHistBuckets * 4 + qpk * d->d_k * 4 + 16 * 8 + 16 + 1024;
-    int stages = 4;
-    while (stages > 2 && stages * tile_bytes + fixed > 100 * 1024) --stages;
+    const int fixed = qpk * kHistWords * 4 + qpk * d->d_k * 4 + 16 * 8 + 16 + 1024;
+    // the deepest ring (2..8 tiles) that still lets two CTAs share an SM (228 KB, 1 KB reserved per CTA)
+    int stages = 8;
+    while (stages > 2 && 2 * (stages * tile_bytes + fixed + 1024) > 228 * 1024) --stages;
     a.score_stages = stages;
     const int score_smem = stages * tile_bytes + fixed;
-    const int per_sm = std::max(1, std::min(3, (227 * 1024) / (score_smem + 1024)));
+    const int per_sm = std::max(1, std::min(3, (228 * 1024) / (score_smem + 1024)));
     const int units = d->batch * d->n_k;
-    const int ygrid = std::max(1, (dev.num_sms * per_sm) / units);
+    const int ntiles = (t_max + kScoreTile - 1) / kScoreTile;
+    const int ygrid = std::max({1, (dev.num_sms * per_sm) / units,
+                                (ntiles + kScoreMaxTilesPerCta - 1) / kScoreMaxTilesPerCta});
     const int select_smem = kCandCap * 8 + 2 * (kTopvMaxContext / 8) + kPairwiseMax * d->d_k * 2;
     if (ensure_dynamic_smem((const void *)score, score_smem) != DIFFQKV_OK ||
         ensure_dynamic_smem((const void *)select, select_smem) != DIFFQKV_OK)
