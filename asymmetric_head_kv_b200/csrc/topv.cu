@@ -50,7 +50,7 @@ constexpr int kHistWords = kHistBuckets / 2;  // score-kernel histogram: two 16-
 constexpr int kScoreMaxTilesPerCta = 511;     // keeps a CTA's positions (and any counter) below 2^16
 constexpr int kRadixBuckets = 256;      // later radix digits: one byte
 constexpr int kFilterThreads = 256;
-constexpr int kFilterChunk = 4096;      // positions per filter CTA
+constexpr int kFilterChunk = 8192;      // positions per filter CTA (32 per thread)
 constexpr int kSelThreads = 512;
 constexpr int kSelWarps = kSelThreads / 32;
 constexpr int kPairwiseMax = 64;        // ambiguous sets up to this size are ranked pairwise
@@ -58,6 +58,8 @@ constexpr int kKeyWords = 19;           // 18 superaccumulator digits + inverted
 constexpr int kTopvHeader = 256;
 constexpr int kCandCap = 12288;         // candidates held in shared memory by the select kernel
 constexpr int kTopvMaxContext = 131072; // bitmap of kept positions: 16 KB of shared memory
+constexpr int kRowInfoWords = 8;       // per-row words handed from kernel to kernel
+enum RowInfo { kRiBucket = 0, kRiAbove = 1, kRiTwoDelta = 2, kRiMax = 3, kRiKept = 4 };
 constexpr int kGatherThreads = 256;
 constexpr int kGatherWarps = kGatherThreads / 32;
 constexpr int kGatherRows = 128;        // kept V rows per gather CTA (target)
@@ -80,7 +82,8 @@ struct TopvArgs {
     uint32_t *ghist;   // [B*n_q][2048] histogram of the top 11 bits of the score keys (zeroed per call)
     uint32_t *ncand;   // [B*n_q] candidate counts (zeroed per call)
     uint32_t *gcount;  // [B*n_q] gather CTAs finished per row (zeroed per call)
-    uint32_t *rowinfo; // [B*n_q][4]: threshold bucket, count above it (filter); kept max score, kept count (select)
+    uint32_t *rowinfo; // [B*n_q][kRowInfoWords]: threshold bucket, count above it, 2 x score error bound
+                       // (filter); kept max score, kept count (select)
     float *gpart;      // [B*n_q][gather_split][d_v + 1] partial sums of the gather
     int32_t *status;
     int32_t batch, n_q, n_k, n_v, t_max, t_pad, topk, q_per_k, q_per_v;
@@ -155,7 +158,7 @@ __device__ __forceinline__ int head_of_lane(int r) { return HG == 4 ? r : (HG ==
 // elements of q for up to four query heads in registers.  The four partial dot
 // products of each head are added across the group, and lane r writes head r.
 template <int DK, int QPK>
-__global__ void __launch_bounds__(kScoreThreads + 32) topv_score_kernel(const __grid_constant__ CUtensorMap tm_k,
+__global__ void __launch_bounds__(kScoreThreads + 32, 2) topv_score_kernel(const __grid_constant__ CUtensorMap tm_k,
                                                                          const TopvArgs a) {
     constexpr int KB = DK / 64;  // 64-wide swizzle blocks per row
     constexpr int TILE_BYTES = kScoreTile * DK * 2;
@@ -216,11 +219,20 @@ __global__ void __launch_bounds__(kScoreThreads + 32) topv_score_kernel(const __
                                   a.wait_limit_ns, nullptr, a.status);
         }
     } else {
-        // ---- consumers: warp w takes positions 32 w .. 32 w + 31 of each tile, 8 at a time
+        // ---- consumers: warp w takes positions PPW w .. PPW w + PPW - 1 of each tile, 8 at a time
         constexpr int HG = QPK < 4 ? QPK : 4;  // heads per pass (their q in registers)
         constexpr int NPASS = QPK / HG;
         constexpr int CPL = DK / 32;           // 16-byte chunks of a K row per lane
+        constexpr int PPW = kScoreTile / (kScoreThreads / 32);  // positions per warp and tile
+        static_assert(PPW % 8 == 0, "whole steps of 8 positions");
         const int r = lane & 3, pg = lane >> 2;
+        // byte offset of this lane's u-th chunk in a row, swizzle included (row index mod 8 = pg)
+        uint32_t coff[CPL];
+#pragma unroll
+        for (int u = 0; u < CPL; ++u) {
+            const int chunk = (u >> 1) * 8 + 2 * r + (u & 1);
+            coff[u] = (uint32_t)((chunk >> 3) * (kScoreTile * 128) + (((chunk & 7) ^ pg) << 4));
+        }
         uint32_t kmx2 = 0;  // two packed |bf16| maxima
         float *sbase = a.scores + ((size_t)b * a.n_q + g * QPK) * a.t_pad;
         f32x2_t qp[HG][CPL][4];  // q[head][chunk elements 2i, 2i + 1]
@@ -248,9 +260,9 @@ __global__ void __launch_bounds__(kScoreThreads + 32) topv_score_kernel(const __
 #pragma unroll 1
             for (int pass = 0; pass < NPASS; ++pass) {
                 if (NPASS > 1) load_q(pass);
-#pragma unroll 2
-                for (int step = 0; step < 4; ++step) {
-                    const int pos = warp * 32 + step * 8 + pg;  // row of the tile
+#pragma unroll
+                for (int step = 0; step < PPW / 8; ++step) {
+                    const int pos = warp * PPW + step * 8 + pg;  // row of the tile
                     const int j = t * kScoreTile + pos;
                     const uint32_t live = (pass == 0 && j < T) ? 0x7fff7fffu : 0u;  // |k| of cached positions
                     // even/odd elements in packed fp32 pairs: every lane of fma.rn.f32x2 is an IEEE
@@ -260,13 +272,13 @@ __global__ void __launch_bounds__(kScoreThreads + 32) topv_score_kernel(const __
                     for (int hh = 0; hh < HG; ++hh) acc[hh] = 0ull;
 #pragma unroll
                     for (int u = 0; u < CPL; ++u) {
-                        const int chunk = (u >> 1) * 8 + 2 * r + (u & 1);
-                        const uint4 kv = lds128(tile + (chunk >> 3) * (kScoreTile * 128) + pos * 128 +
-                                                (((chunk & 7) ^ (pos & 7)) << 4));
-                        kmx2 = __vmaxu2(kmx2, kv.x & live);
-                        kmx2 = __vmaxu2(kmx2, kv.y & live);
-                        kmx2 = __vmaxu2(kmx2, kv.z & live);
-                        kmx2 = __vmaxu2(kmx2, kv.w & live);
+                        const uint4 kv = lds128(tile + pos * 128 + coff[u]);
+                        if (pass == 0) {  // magnitudes (sign bit cleared first) of cached positions
+                            kmx2 = __vmaxu2(kmx2, kv.x & live);
+                            kmx2 = __vmaxu2(kmx2, kv.y & live);
+                            kmx2 = __vmaxu2(kmx2, kv.z & live);
+                            kmx2 = __vmaxu2(kmx2, kv.w & live);
+                        }
                         const f32x2_t k01 = bf16x2_to_f2(kv.x), k23 = bf16x2_to_f2(kv.y);
                         const f32x2_t k45 = bf16x2_to_f2(kv.z), k67 = bf16x2_to_f2(kv.w);
 #pragma unroll
@@ -486,7 +498,7 @@ __device__ float row_q_l1(const __nv_bfloat16 *q, float *red) {
 // ------------------------------------------------------------------ 2. filter
 
 template <int DK>
-__global__ void __launch_bounds__(kFilterThreads) topv_filter_kernel(const TopvArgs a) {
+__global__ void __launch_bounds__(kFilterThreads, 4) topv_filter_kernel(const TopvArgs a) {
     __shared__ uint32_t warp_sums[33];
     __shared__ float red[kFilterThreads / 32];
     __shared__ __align__(16) uint32_t hist_s[kHistBuckets];  // filled with 16-byte stores
@@ -507,10 +519,11 @@ __global__ void __launch_bounds__(kFilterThreads) topv_filter_kernel(const TopvA
     int32_t *cj = a.cand_j + (size_t)row * a.t_pad;
     float *cs = a.cand_s + (size_t)row * a.t_pad;
     const int j_end = min(T, j_begin + kFilterChunk);
-    static_assert(kFilterChunk == kFilterThreads * 16, "one pass of 16 positions per thread");
-    float4 v[4];
+    constexpr int kVec = kFilterChunk / kFilterThreads / 4;  // float4 loads per thread
+    static_assert(kVec * 4 <= 32, "a thread's hits fit one 32-bit mask");
+    float4 v[kVec];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < kVec; ++u) {
         const int p = j_begin + (u * kFilterThreads + tid) * 4;
         v[u] = p < j_end ? __ldcg(reinterpret_cast<const float4 *>(s + p)) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
@@ -529,18 +542,19 @@ __global__ void __launch_bounds__(kFilterThreads) topv_filter_kernel(const TopvA
     __syncthreads();
     find_bucket_from_top(hist_s, kHistBuckets, (uint32_t)a.topk, &sh_d, &sh_above, warp_sums);
     if (blockIdx.y == 0 && tid == 0) {
-        a.rowinfo[4 * row + 0] = (uint32_t)sh_d;
-        a.rowinfo[4 * row + 1] = sh_above;
+        a.rowinfo[kRowInfoWords * row + kRiBucket] = (uint32_t)sh_d;
+        a.rowinfo[kRowInfoWords * row + kRiAbove] = sh_above;
     }
     const float q1 = row_q_l1<DK>(a.q + (size_t)row * DK, red);
     const float two_d = __fmul_ru(2.f, score_error_bound<DK>(q1, __uint_as_float(kmax_bits << 16)));
+    if (blockIdx.y == 0 && tid == 0) a.rowinfo[kRowInfoWords * row + kRiTwoDelta] = __float_as_uint(two_d);
     // (bucket 0 starts at the NaN patterns: everything in it and above is a candidate)
     const float lower = sh_d == 0 ? -INFINITY : __fsub_rd(key_float((uint32_t)sh_d << 21), two_d);
-    // a thread's hits form a 16-bit mask; one block scan gives every thread its slots and
+    // a thread's hits form a bit mask; one block scan gives every thread its slots and
     // one global atomic per CTA reserves them
     uint32_t hits = 0;
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < kVec; ++u) {
         const int p = j_begin + (u * kFilterThreads + tid) * 4;
         const float x[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
 #pragma unroll
@@ -555,7 +569,7 @@ __global__ void __launch_bounds__(kFilterThreads) topv_filter_kernel(const TopvA
     if (hits) {
         slot += sh_base;
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < kVec; ++u) {
             const int p = j_begin + (u * kFilterThreads + tid) * 4;
             const float x[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
 #pragma unroll
@@ -609,8 +623,8 @@ __global__ void __launch_bounds__(kSelThreads, 1) topv_select_kernel(const TopvA
     if (T == 0) {
         for (int i = tid; i < K; i += kSelThreads) idx[i] = -1;
         if (tid == 0) {
-            a.rowinfo[4 * row + 2] = __float_as_uint(0.f);
-            a.rowinfo[4 * row + 3] = 0u;
+            a.rowinfo[kRowInfoWords * row + kRiMax] = __float_as_uint(0.f);
+            a.rowinfo[kRowInfoWords * row + kRiKept] = 0u;
         }
         return;
     }
@@ -660,8 +674,8 @@ __global__ void __launch_bounds__(kSelThreads, 1) topv_select_kernel(const TopvA
         // ---- a. tau = the K-th largest score.  Its top 11 key bits are the filter's bucket,
         //         and `above` positions lie in higher buckets (all of them candidates); a radix
         //         select over the candidates finds the other 21 bits, 11 and then 10 at a time
-        uint32_t prefix = __ldcg(a.rowinfo + 4 * row) << 21, pmask = 0xffe00000u;
-        uint32_t kk = (uint32_t)K - __ldcg(a.rowinfo + 4 * row + 1);
+        uint32_t prefix = __ldcg(a.rowinfo + kRowInfoWords * row + kRiBucket) << 21, pmask = 0xffe00000u;
+        uint32_t kk = (uint32_t)K - __ldcg(a.rowinfo + kRowInfoWords * row + kRiAbove);
         for (int pass = 0; pass < 2; ++pass) {
             const int shift = pass == 0 ? 10 : 0;
             const int nb = pass == 0 ? 2048 : 1024;
@@ -684,10 +698,8 @@ __global__ void __launch_bounds__(kSelThreads, 1) topv_select_kernel(const TopvA
         }
         const float tau = key_float(prefix);
 
-        // ---- b. rounding bound of every score of this row
-        const float q1 = row_q_l1<DK>(a.q + (size_t)row * DK, red_s);
-        const float kmax = __uint_as_float(__ldcg(a.kmax + b * a.n_k + g) << 16);
-        const float two_d = __fmul_ru(2.f, score_error_bound<DK>(q1, kmax));
+        // ---- b. rounding bound of every score of this row (the filter's, see score_error_bound)
+        const float two_d = __uint_as_float(__ldcg(a.rowinfo + kRowInfoWords * row + kRiTwoDelta));
         const float hi_edge = __fadd_ru(tau, two_d);
         const float lo_edge = __fsub_rd(tau, two_d);
         if (tid == 0) {
@@ -813,8 +825,8 @@ __global__ void __launch_bounds__(kSelThreads, 1) topv_select_kernel(const TopvA
     if (tid == 0) {
         float m = red_s[0];
         for (int w = 1; w < kSelWarps; ++w) m = fmaxf(m, red_s[w]);
-        a.rowinfo[4 * row + 2] = __float_as_uint(m);
-        a.rowinfo[4 * row + 3] = (uint32_t)nsel;
+        a.rowinfo[kRowInfoWords * row + kRiMax] = __float_as_uint(m);
+        a.rowinfo[kRowInfoWords * row + kRiKept] = (uint32_t)nsel;
     }
 }
 
@@ -833,8 +845,8 @@ __global__ void __launch_bounds__(kGatherThreads) topv_gather_kernel(const TopvA
     const int b = row / a.n_q, h = row % a.n_q, vh = h / a.q_per_v;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     pdl_wait_prev();  // kept positions and their maximum from the select kernel
-    const float m = __uint_as_float(__ldcg(a.rowinfo + 4 * row + 2));
-    const int nsel = (int)__ldcg(a.rowinfo + 4 * row + 3);
+    const float m = __uint_as_float(__ldcg(a.rowinfo + kRowInfoWords * row + kRiMax));
+    const int nsel = (int)__ldcg(a.rowinfo + kRowInfoWords * row + kRiKept);
     const int i_begin = (int)(((long long)nsel * part) / nparts);
     const int i_end = (int)(((long long)nsel * (part + 1)) / nparts);
     const int32_t *idx = a.idx_out + (size_t)row * a.topk;
@@ -973,10 +985,11 @@ size_t zeroed_bytes(const diffqkv_dims_t *d) {
 
 int gather_split(int32_t topk) { return std::max(1, std::min(kGatherMaxSplit, (topk + kGatherRows - 1) / kGatherRows)); }
 
-// rowinfo [rows][4] and the gather partials [rows][split][d_v + 1]
+// rowinfo [rows][kRowInfoWords] and the gather partials [rows][split][d_v + 1]
 size_t row_bytes(const diffqkv_dims_t *d, int32_t topk) {
     const size_t rows = (size_t)d->batch * d->n_q;
-    return align_up(rows * 16, 256) + align_up(rows * (size_t)gather_split(topk) * (d->d_v + 1) * 4, 256);
+    return align_up(rows * kRowInfoWords * 4, 256) +
+           align_up(rows * (size_t)gather_split(topk) * (d->d_v + 1) * 4, 256);
 }
 
 template <typename... P, typename... A>
@@ -1039,7 +1052,7 @@ diffqkv_status_t topv_launch(const diffqkv_dims_t *d, const void *q, const void 
     a.gcount = a.ncand + rows;
     ws += align_up(zeroed_bytes(d), 256);
     a.rowinfo = reinterpret_cast<uint32_t *>(ws);
-    a.gpart = reinterpret_cast<float *>(ws + align_up(rows * 16, 256));
+    a.gpart = reinterpret_cast<float *>(ws + align_up(rows * kRowInfoWords * 4, 256));
     a.gather_split = gather_split(topk);
     ws += row_bytes(d, topk);
     a.scores = reinterpret_cast<float *>(ws);
