@@ -62,8 +62,8 @@ constexpr int kRowInfoWords = 8;       // per-row words handed from kernel to ke
 enum RowInfo { kRiBucket = 0, kRiAbove = 1, kRiTwoDelta = 2, kRiMax = 3, kRiKept = 4 };
 constexpr int kGatherThreads = 256;
 constexpr int kGatherWarps = kGatherThreads / 32;
-constexpr int kGatherRows = 128;        // kept V rows per gather CTA (target)
-constexpr int kGatherMaxSplit = 64;
+constexpr int kGatherRows = 128;        // kept V rows per gather CTA and round
+constexpr int kGatherMaxSplit = 8;      // gather CTAs of a row: one thread-block cluster
 
 struct TopvArgs {
     const __nv_bfloat16 *q;
@@ -81,14 +81,11 @@ struct TopvArgs {
     uint32_t *kmax;    // [B*n_k] bf16 bit pattern of max |k| (zeroed per call)
     uint32_t *ghist;   // [B*n_q][2048] histogram of the top 11 bits of the score keys (zeroed per call)
     uint32_t *ncand;   // [B*n_q] candidate counts (zeroed per call)
-    uint32_t *gcount;  // [B*n_q] gather CTAs finished per row (zeroed per call)
     uint32_t *rowinfo; // [B*n_q][kRowInfoWords]: threshold bucket, count above it, 2 x score error bound
                        // (filter); kept max score, kept count (select)
-    float *gpart;      // [B*n_q][gather_split][d_v + 1] partial sums of the gather
     int32_t *status;
     int32_t batch, n_q, n_k, n_v, t_max, t_pad, topk, q_per_k, q_per_v;
     int32_t score_stages;
-    int32_t gather_split;
     float scale_log2;
     uint64_t wait_limit_ns;
 };
@@ -102,6 +99,19 @@ __device__ __forceinline__ int clamp_len(int v, int t_max) { return v < 0 ? 0 : 
 // kernels before it have finished too.
 __device__ __forceinline__ void pdl_launch_next() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void pdl_wait_prev() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// All threads of all CTAs of the cluster; shared-memory writes before it are visible after it.
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// 32-bit load from the shared memory of cluster CTA `rank`, at this CTA's shared address `addr`.
+__device__ __forceinline__ float ld_dsmem_f32(uint32_t addr, uint32_t rank) {
+    uint32_t remote;
+    float v;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(addr), "r"(rank));
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+    return v;
+}
 
 // Order-preserving map of finite floats onto uint32 (larger float -> larger key).
 __device__ __forceinline__ uint32_t float_key(float f) {
@@ -158,7 +168,7 @@ __device__ __forceinline__ int head_of_lane(int r) { return HG == 4 ? r : (HG ==
 // elements of q for up to four query heads in registers.  The four partial dot
 // products of each head are added across the group, and lane r writes head r.
 template <int DK, int QPK>
-__global__ void __launch_bounds__(kScoreThreads + 32, 2) topv_score_kernel(const __grid_constant__ CUtensorMap tm_k,
+__global__ void __launch_bounds__(kScoreThreads + 32, 3) topv_score_kernel(const __grid_constant__ CUtensorMap tm_k,
                                                                          const TopvArgs a) {
     constexpr int KB = DK / 64;  // 64-wide swizzle blocks per row
     constexpr int TILE_BYTES = kScoreTile * DK * 2;
@@ -436,27 +446,35 @@ __device__ void exact_key(const uint16_t *qbits, const uint16_t *kbits, int j, u
 
 // exact_key computed by a whole warp: lane l takes products l, l + 32, ...; the
 // per-lane digit slots are integers, so summing them across the warp is exact
-// in any order (|slot| < d_k 2^47 <= 2^54); lane 0 normalises and writes.
+// in any order (|slot| < d_k 2^47 <= 2^54).  Only the slots some lane used are
+// summed (the range is warp-uniform); lane 0 normalises and writes.  kbits is
+// the K row in global memory.
 template <int DK>
 __device__ void exact_key_warp(const uint16_t *qbits, const uint16_t *kbits, int j, uint32_t *out, int lane) {
     long long acc[18];
 #pragma unroll
     for (int i = 0; i < 18; ++i) acc[i] = 0;
+    int smin = 15, smax = 0;
 #pragma unroll
     for (int u = 0; u < DK / 32; ++u) {
         const int c = lane + 32 * u;
-        const uint32_t qb = qbits[c], kb = kbits[c];
+        const uint32_t qb = qbits[c], kb = __ldg(kbits + c);
         const int eq = (qb >> 7) & 0xff, ek = (kb >> 7) & 0xff;
         const int mq = (qb & 0x7f) | (eq ? 0x80 : 0), mk = (kb & 0x7f) | (ek ? 0x80 : 0);
         const int off = (eq ? eq - 134 : -133) + (ek ? ek - 134 : -133) + 266;
         long long v = (long long)(mq * mk) << (off & 31);
         if ((qb ^ kb) & 0x8000u) v = -v;
         const int slot = off >> 5;
+        smin = min(smin, slot);
+        smax = max(smax, slot);
 #pragma unroll
         for (int i = 0; i < 16; ++i) acc[i] += (slot == i) ? v : 0ll;
     }
+    smin = __reduce_min_sync(0xffffffffu, smin);
+    smax = __reduce_max_sync(0xffffffffu, smax);
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
+        if (i < smin || i > smax) continue;  // no lane has a product in this slot
 #pragma unroll
         for (int o = 16; o >= 1; o >>= 1) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
     }
@@ -602,7 +620,6 @@ __global__ void __launch_bounds__(kSelThreads, 1) topv_select_kernel(const TopvA
     float *c_s = reinterpret_cast<float *>(c_j + kCandCap);           // [kCandCap]
     uint32_t *bitmap = reinterpret_cast<uint32_t *>(c_s + kCandCap);  // [kTopvMaxContext / 32]
     uint32_t *wprefix = bitmap + kTopvMaxContext / 32;                               // [kTopvMaxContext / 32]
-    uint4 *krows = reinterpret_cast<uint4 *>(wprefix + kTopvMaxContext / 32);  // [kPairwiseMax][DK / 8]
 
     const int row = blockIdx.x;
     const int b = row / a.n_q;
@@ -735,16 +752,12 @@ __global__ void __launch_bounds__(kSelThreads, 1) topv_select_kernel(const TopvA
         } else if (need >= na) {
             for (int i = tid; i < na; i += kSelThreads) keep(alist[i]);
         } else if (na <= kPairwiseMax) {
-            // rank the few ambiguous positions pairwise by exact key; their K rows are
-            // staged in shared memory first
-            for (int i = tid; i < na * (DK / 8); i += kSelThreads) {
-                const int r = i / (DK / 8), c = i % (DK / 8);
-                krows[i] = __ldg(reinterpret_cast<const uint4 *>(krow0 + (size_t)alist[r] * kstride) + c);
-            }
-            __syncthreads();
-            for (int r = warp; r < na; r += kSelWarps)
-                exact_key_warp<DK>(q_s, reinterpret_cast<const uint16_t *>(krows + r * (DK / 8)), alist[r],
+            // rank the few ambiguous positions pairwise by exact key (a warp per key)
+            for (int r = warp; r < na; r += kSelWarps) {
+                const int j = alist[r];
+                exact_key_warp<DK>(q_s, reinterpret_cast<const uint16_t *>(krow0 + (size_t)j * kstride), j,
                                    keys_s[r], lane);
+            }
             __syncthreads();
             if (tid < na) {
                 int better = 0;
@@ -834,13 +847,15 @@ __global__ void __launch_bounds__(kSelThreads, 1) topv_select_kernel(const TopvA
 
 // CTA (row, part) sums its share of the kept positions (in ascending order):
 // sum_j 2^((s_j - m) scale log2 e) v_j and the weight sum, with m the largest
-// kept score; the last CTA of the row to finish adds the parts in a fixed order
-// and writes the normalised output.
+// kept score.  The parts of a row form one thread-block cluster: each leaves its
+// sums in its own shared memory, and rank 0 adds them in rank order through
+// distributed shared memory and writes the normalised output.  No CTA returns
+// early, so every thread reaches both cluster barriers.
 template <int DV>
 __global__ void __launch_bounds__(kGatherThreads) topv_gather_kernel(const TopvArgs a) {
     __shared__ float o_s[kGatherWarps][DV];
     __shared__ float l_s[kGatherWarps];
-    __shared__ bool sh_last;
+    __shared__ float part_s[DV + 1];  // this CTA's sums: o[0..DV-1], then the weight sum
     const int row = blockIdx.x, part = blockIdx.y, nparts = gridDim.y;
     const int b = row / a.n_q, h = row % a.n_q, vh = h / a.q_per_v;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -905,27 +920,23 @@ __global__ void __launch_bounds__(kGatherThreads) topv_gather_kernel(const TopvA
     }
     if (lane == 0) l_s[warp] = l;
     __syncthreads();
-    float *mine = a.gpart + ((size_t)row * a.gather_split + part) * (DV + 1);
     for (int c = tid; c <= DV; c += kGatherThreads) {
         float acc = 0.f;
         for (int w = 0; w < kGatherWarps; ++w) acc += c < DV ? o_s[w][c] : l_s[w];
-        mine[c] = acc;
+        part_s[c] = acc;
     }
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) sh_last = atomicAdd(a.gcount + row, 1u) == (uint32_t)(nparts - 1);
-    __syncthreads();
-    if (!sh_last) return;
-    __threadfence();
-    const float *parts = a.gpart + (size_t)row * a.gather_split * (DV + 1);
-    float lt = 0.f;
-    for (int p = 0; p < nparts; ++p) lt += __ldcg(parts + (size_t)p * (DV + 1) + DV);
-    for (int c = tid; c < DV; c += kGatherThreads) {
-        float acc = 0.f;
-        for (int p = 0; p < nparts; ++p) acc += __ldcg(parts + (size_t)p * (DV + 1) + c);
-        a.out[(size_t)row * DV + c] = __float2bfloat16(lt > 0.f ? acc / lt : 0.f);
+    cluster_sync();  // every part of the row is in its CTA's shared memory
+    if (part == 0) {
+        const uint32_t base = smem_addr(part_s);
+        float lt = 0.f;
+        for (int p = 0; p < nparts; ++p) lt += ld_dsmem_f32(base + DV * 4u, (uint32_t)p);
+        for (int c = tid; c < DV; c += kGatherThreads) {
+            float acc = 0.f;
+            for (int p = 0; p < nparts; ++p) acc += ld_dsmem_f32(base + (uint32_t)c * 4u, (uint32_t)p);
+            a.out[(size_t)row * DV + c] = __float2bfloat16(lt > 0.f ? acc / lt : 0.f);
+        }
     }
-    if (tid == 0) a.gcount[row] = 0u;
+    cluster_sync();  // no CTA leaves while rank 0 still reads its shared memory
 }
 
 size_t align_up(size_t x, size_t al) { return (x + al - 1) / al * al; }
@@ -976,35 +987,40 @@ size_t padded_len(int32_t t_max) { return align_up((size_t)t_max, 64); }
 // kmax entries, rounded up so the histograms after them start 16-byte aligned.
 size_t kmax_slots(const diffqkv_dims_t *d) { return align_up((size_t)d->batch * d->n_k, 4); }
 
-// Zero-filled per call: kmax [B*n_k, padded], histograms [rows][2048], candidate counts [rows],
-// gather counters [rows].
+// Zero-filled per call: kmax [B*n_k, padded], histograms [rows][2048], candidate counts [rows].
 size_t zeroed_bytes(const diffqkv_dims_t *d) {
     const size_t rows = (size_t)d->batch * d->n_q;
-    return kmax_slots(d) * 4 + rows * kHistBuckets * 4 + rows * 4 * 2;
+    return kmax_slots(d) * 4 + rows * kHistBuckets * 4 + rows * 4;
 }
 
+// Gather CTAs per row (one cluster): a round of kGatherRows kept rows each, at most kGatherMaxSplit.
 int gather_split(int32_t topk) { return std::max(1, std::min(kGatherMaxSplit, (topk + kGatherRows - 1) / kGatherRows)); }
 
-// rowinfo [rows][kRowInfoWords] and the gather partials [rows][split][d_v + 1]
-size_t row_bytes(const diffqkv_dims_t *d, int32_t topk) {
-    const size_t rows = (size_t)d->batch * d->n_q;
-    return align_up(rows * kRowInfoWords * 4, 256) +
-           align_up(rows * (size_t)gather_split(topk) * (d->d_v + 1) * 4, 256);
-}
+// rowinfo [rows][kRowInfoWords]
+size_t row_bytes(const diffqkv_dims_t *d) { return align_up((size_t)d->batch * d->n_q * kRowInfoWords * 4, 256); }
 
+// Launch after the previous kernel of the stream with programmatic dependent launch;
+// cluster_y > 1 groups that many consecutive CTAs along y into one cluster.
 template <typename... P, typename... A>
 cudaError_t launch_after_prev(void (*kernel)(P...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
-                              A... args) {
+                              int cluster_y, A... args) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = block;
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
     cfg.numAttrs = 1;
+    if (cluster_y > 1) {
+        attr[1].id = cudaLaunchAttributeClusterDimension;
+        attr[1].val.clusterDim.x = 1;
+        attr[1].val.clusterDim.y = (unsigned)cluster_y;
+        attr[1].val.clusterDim.z = 1;
+        cfg.numAttrs = 2;
+    }
+    cfg.attrs = attr;
     return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
@@ -1014,7 +1030,7 @@ size_t topv_workspace_size(const diffqkv_dims_t *d, int32_t t_max, int32_t topk)
     if (validate_dims(d) != DIFFQKV_OK || t_max < 1 || topk < 1) return 0;
     const size_t rows = (size_t)d->batch * d->n_q;
     const size_t per = padded_len(t_max);
-    return kTopvHeader + align_up(zeroed_bytes(d), 256) + row_bytes(d, topk) + align_up(rows * per * 4, 256) * 4 +
+    return kTopvHeader + align_up(zeroed_bytes(d), 256) + row_bytes(d) + align_up(rows * per * 4, 256) * 4 +
            align_up(rows * per, 256) * 2;
 }
 
@@ -1049,12 +1065,9 @@ diffqkv_status_t topv_launch(const diffqkv_dims_t *d, const void *q, const void 
     a.kmax = reinterpret_cast<uint32_t *>(ws);
     a.ghist = a.kmax + kmax_slots(d);  // 16-byte aligned (read with 16-byte loads)
     a.ncand = a.ghist + rows * kHistBuckets;
-    a.gcount = a.ncand + rows;
     ws += align_up(zeroed_bytes(d), 256);
     a.rowinfo = reinterpret_cast<uint32_t *>(ws);
-    a.gpart = reinterpret_cast<float *>(ws + align_up(rows * kRowInfoWords * 4, 256));
-    a.gather_split = gather_split(topk);
-    ws += row_bytes(d, topk);
+    ws += row_bytes(d);
     a.scores = reinterpret_cast<float *>(ws);
     ws += align_up(rows * t_pad * 4, 256);
     a.cand_j = reinterpret_cast<int32_t *>(ws);
@@ -1097,9 +1110,10 @@ diffqkv_status_t topv_launch(const diffqkv_dims_t *d, const void *q, const void 
     if (st != DIFFQKV_OK) return st;
     const int tile_bytes = kScoreTile * d->d_k * 2;
     const int fixed = qpk * kHistWords * 4 + qpk * d->d_k * 4 + 16 * 8 + 16 + 1024;
-    // the deepest ring (2..8 tiles) that still lets two CTAs share an SM (228 KB, 1 KB reserved per CTA)
+    // the deepest ring (2..8 tiles) that still lets three CTAs share an SM (228 KB, 1 KB reserved per
+    // CTA): occupancy hides more of the consumers' latency than a deeper ring does
     int stages = 8;
-    while (stages > 2 && 2 * (stages * tile_bytes + fixed + 1024) > 228 * 1024) --stages;
+    while (stages > 2 && 3 * (stages * tile_bytes + fixed + 1024) > 228 * 1024) --stages;
     a.score_stages = stages;
     const int score_smem = stages * tile_bytes + fixed;
     const int per_sm = std::max(1, std::min(3, (228 * 1024) / (score_smem + 1024)));
@@ -1107,7 +1121,7 @@ diffqkv_status_t topv_launch(const diffqkv_dims_t *d, const void *q, const void 
     const int ntiles = (t_max + kScoreTile - 1) / kScoreTile;
     const int ygrid = std::max({1, (dev.num_sms * per_sm) / units,
                                 (ntiles + kScoreMaxTilesPerCta - 1) / kScoreMaxTilesPerCta});
-    const int select_smem = kCandCap * 8 + 2 * (kTopvMaxContext / 8) + kPairwiseMax * d->d_k * 2;
+    const int select_smem = kCandCap * 8 + 2 * (kTopvMaxContext / 8);
     if (ensure_dynamic_smem((const void *)score, score_smem) != DIFFQKV_OK ||
         ensure_dynamic_smem((const void *)select, select_smem) != DIFFQKV_OK)
         return DIFFQKV_ERR_CUDA;
@@ -1115,18 +1129,20 @@ diffqkv_status_t topv_launch(const diffqkv_dims_t *d, const void *q, const void 
     if (cudaGetLastError() != cudaSuccess) return DIFFQKV_ERR_CUDA;
     // 2. filter: every row, in chunks of kFilterChunk positions (chunks past a row's length return at once)
     if (launch_after_prev(filter, dim3((unsigned)rows, (t_max + kFilterChunk - 1) / kFilterChunk),
-                          dim3(kFilterThreads), 0, stream, a) != cudaSuccess) {
+                          dim3(kFilterThreads), 0, stream, 1, a) != cudaSuccess) {
         cudaGetLastError();
         return DIFFQKV_ERR_CUDA;
     }
     // 3. select: one CTA per row
-    if (launch_after_prev(select, dim3((unsigned)rows), dim3(kSelThreads), select_smem, stream, a) != cudaSuccess) {
+    if (launch_after_prev(select, dim3((unsigned)rows), dim3(kSelThreads), select_smem, stream, 1, a) !=
+        cudaSuccess) {
         cudaGetLastError();
         return DIFFQKV_ERR_CUDA;
     }
-    // 4. gather: gather_split CTAs per row
-    if (launch_after_prev(gather, dim3((unsigned)rows, (unsigned)a.gather_split), dim3(kGatherThreads), 0, stream,
-                          a) != cudaSuccess) {
+    // 4. gather: one cluster of gather_split CTAs per row
+    const int split = gather_split(topk);
+    if (launch_after_prev(gather, dim3((unsigned)rows, (unsigned)split), dim3(kGatherThreads), 0, stream, split, a) !=
+        cudaSuccess) {
         cudaGetLastError();
         return DIFFQKV_ERR_CUDA;
     }
