@@ -100,6 +100,13 @@ __device__ __forceinline__ int clamp_len(int v, int t_max) { return v < 0 ? 0 : 
 __device__ __forceinline__ void pdl_launch_next() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void pdl_wait_prev() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
+// max(a, b, c) in one instruction (three-input form of max.f32, sm_100).
+__device__ __forceinline__ float fmax3f(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
 // All threads of all CTAs of the cluster; shared-memory writes before it are visible after it.
 __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
@@ -243,7 +250,7 @@ __global__ void __launch_bounds__(kScoreThreads + 32, 3) topv_score_kernel(const
             const int chunk = (u >> 1) * 8 + 2 * r + (u & 1);
             coff[u] = (uint32_t)((chunk >> 3) * (kScoreTile * 128) + (((chunk & 7) ^ pg) << 4));
         }
-        uint32_t kmx2 = 0;  // two packed |bf16| maxima
+        float kmf = 0.f;  // largest |k| seen (a bf16 value, so exact in fp32)
         float *sbase = a.scores + ((size_t)b * a.n_q + g * QPK) * a.t_pad;
         f32x2_t qp[HG][CPL][4];  // q[head][chunk elements 2i, 2i + 1]
         auto load_q = [&](int pass) {
@@ -274,7 +281,7 @@ __global__ void __launch_bounds__(kScoreThreads + 32, 3) topv_score_kernel(const
                 for (int step = 0; step < PPW / 8; ++step) {
                     const int pos = warp * PPW + step * 8 + pg;  // row of the tile
                     const int j = t * kScoreTile + pos;
-                    const uint32_t live = (pass == 0 && j < T) ? 0x7fff7fffu : 0u;  // |k| of cached positions
+                    const bool cached = pass == 0 && j < T;  // |k| counts for cached positions only
                     // even/odd elements in packed fp32 pairs: every lane of fma.rn.f32x2 is an IEEE
                     // fp32 FMA; a product meets at most 4 CPL + 3 (<= d_k) roundings on its way into the score
                     f32x2_t acc[HG];
@@ -283,14 +290,16 @@ __global__ void __launch_bounds__(kScoreThreads + 32, 3) topv_score_kernel(const
 #pragma unroll
                     for (int u = 0; u < CPL; ++u) {
                         const uint4 kv = lds128(tile + pos * 128 + coff[u]);
-                        if (pass == 0) {  // magnitudes (sign bit cleared first) of cached positions
-                            kmx2 = __vmaxu2(kmx2, kv.x & live);
-                            kmx2 = __vmaxu2(kmx2, kv.y & live);
-                            kmx2 = __vmaxu2(kmx2, kv.z & live);
-                            kmx2 = __vmaxu2(kmx2, kv.w & live);
+                        float kf[8];
+                        unpack8(kv, kf);
+                        if (cached) {
+                            kmf = fmax3f(kmf, fabsf(kf[0]), fabsf(kf[1]));
+                            kmf = fmax3f(kmf, fabsf(kf[2]), fabsf(kf[3]));
+                            kmf = fmax3f(kmf, fabsf(kf[4]), fabsf(kf[5]));
+                            kmf = fmax3f(kmf, fabsf(kf[6]), fabsf(kf[7]));
                         }
-                        const f32x2_t k01 = bf16x2_to_f2(kv.x), k23 = bf16x2_to_f2(kv.y);
-                        const f32x2_t k45 = bf16x2_to_f2(kv.z), k67 = bf16x2_to_f2(kv.w);
+                        const f32x2_t k01 = f2_pack(kf[0], kf[1]), k23 = f2_pack(kf[2], kf[3]);
+                        const f32x2_t k45 = f2_pack(kf[4], kf[5]), k67 = f2_pack(kf[6], kf[7]);
 #pragma unroll
                         for (int hh = 0; hh < HG; ++hh) {
                             acc[hh] = f2_fma(qp[hh][u][0], k01, acc[hh]);
@@ -318,7 +327,7 @@ __global__ void __launch_bounds__(kScoreThreads + 32, 3) topv_score_kernel(const
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty_bar[st]);
         }
-        uint32_t kmx = max(kmx2 & 0xffffu, kmx2 >> 16);
+        uint32_t kmx = __float_as_uint(kmf) >> 16;  // its bf16 pattern (kmf >= 0: order-preserving)
 #pragma unroll
         for (int off = 16; off >= 1; off >>= 1) kmx = max(kmx, __shfl_xor_sync(0xffffffffu, kmx, off));
         if (lane == 0) atomicMax(a.kmax + unit, kmx);
