@@ -5,24 +5,24 @@
 // section 3.4 Steps 3-5, with the causal lower-triangular mask of the prefix
 // phase).  Unlike decode this is a dense contraction, so it runs on tcgen05.
 //
-// One CTA = one 128-row query tile of one (batch, head); 64-position K/V tiles.
-//   warp 4      TMA producer: Q once, K/V tiles into a shared-memory ring
-//               (128-byte swizzle, the layout the MMA descriptors describe)
-//   warp 5      allocates 256 TMEM columns; lane 0 issues every tcgen05.mma:
-//               S = Q K^T (M128 N64, fp32 in TMEM, two S buffers) and
-//               O += P V (M128 N=d_v, fp32 in TMEM, P read from TMEM)
-//   warps 0-3   softmax: thread t owns query row t = TMEM lane t, so row max and
-//               row sum need no shuffles; P is written back as bf16 pairs over
-//               the first 32 columns of its own S buffer, where the PV MMA
-//               reads it as the A operand.  O is rescaled in TMEM only when a
-//               row maximum grows by more than 2^8 (the stale maximum is used
-//               consistently for O and the row sum, so the result is exact up
-//               to rounding).
-// The MMA thread issues S(n+2) into a buffer only after P(n) V(n), which reads
-// P(n) from that buffer; tcgen05.mma operations from one thread run in issue
-// order, so no other hand-back of the S buffers is needed.
-// Every mbarrier wait is bounded; CTAs are ordered heaviest (most K/V tiles)
-// first.  Two CTAs fit on one SM (at most 98 KB smem and 256 TMEM columns each).
+// Two tilings, chosen by d_k:
+//  * d_k = 64 (the DiffQKV key width): `tile64` -- one 128-row query tile per
+//    CTA, 64-position K/V tiles, two S buffers in TMEM so that S(n+1) = Q K^T
+//    runs while the softmax works on S(n), two CTAs per SM.  With d_k = 64 the
+//    exponentials (64 per row and tile) outweigh the MMAs, and this overlap
+//    within a tile is what keeps the SFU busy.
+//  * d_k = 128: `pair128` -- two 128-row query tiles per CTA sharing each
+//    128-position K/V tile, one CTA per SM (512 TMEM columns), the MMA thread
+//    alternating between the tiles.  A Q K^T MMA with N = 64 would read its
+//    Q operand from shared memory faster than shared memory delivers it once
+//    d_k = 128 makes that product the larger one; N = 128 halves those reads.
+// In both, P goes back to TMEM (bf16 pairs over the first columns of its S)
+// and the P.V MMA reads it as its A operand; tcgen05.mma operations from one
+// thread run in issue order, so S is overwritten only after the P.V that reads
+// P from the same columns.  O is rescaled in TMEM only when a row maximum grows
+// by more than 2^8 (the stale maximum is used consistently for O and the row
+// sum, so the result is exact up to rounding).  Every mbarrier wait is bounded;
+// CTAs are ordered heaviest (most K/V tiles) first.
 #include <math.h>
 
 #include "common.cuh"
@@ -32,6 +32,22 @@ namespace diffqkv {
 
 namespace {
 
+constexpr float kRescaleLog2 = 8.f;  // lazy O rescale threshold (log2 domain)
+
+struct PrefillArgs {
+    __nv_bfloat16 *out;
+    int32_t *status;
+    int32_t batch, seq, n_q, n_k, n_v, q_per_k, q_per_v, n_ctas_per_head;
+    float scale_log2;
+    uint64_t wait_limit_ns;
+};
+
+// ---------------------------------------------------------------- d_k = 64
+// warps 0-3 softmax (thread t owns query row t = TMEM lane t), warp 4 TMA
+// producer (Q once, K/V ring), warp 5 TMEM allocation and MMA issue.  S(n) goes
+// to one of two 64-column S buffers; P(n) over the first 32 columns of it.
+namespace tile64 {
+
 constexpr int BM = 128;             // query rows per CTA
 constexpr int BN = 64;              // K/V positions per tile
 constexpr int kSoftmaxWarps = 4;
@@ -39,7 +55,6 @@ constexpr int kProducerWarp = 4;
 constexpr int kMmaWarp = 5;
 constexpr int kThreads = 192;       // 4 softmax warps, producer, MMA
 constexpr int kTmemCols = 256;      // S0 | S1 | O
-constexpr float kRescaleLog2 = 8.f; // lazy O rescale threshold (log2 domain)
 template <int DK, int DV>
 struct Cfg {
     static constexpr int KB = DK / 64;                 // 64-wide swizzle blocks along d_k
@@ -53,14 +68,6 @@ struct Cfg {
     static constexpr int OFF_KV = Q_BYTES;
     static constexpr int OFF_BAR = OFF_KV + STAGES * STAGE_BYTES;
     static constexpr int SMEM = OFF_BAR + 256 + 1024;  // barriers/flags + alignment slack
-};
-
-struct PrefillArgs {
-    __nv_bfloat16 *out;
-    int32_t *status;
-    int32_t batch, seq, n_q, n_k, n_v, q_per_k, q_per_v, n_qtiles;
-    float scale_log2;
-    uint64_t wait_limit_ns;
 };
 
 template <int DK, int DV>
@@ -87,7 +94,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 
     // heaviest tiles first: query tile index descends with blockIdx
     const int bh_count = a.batch * a.n_q;
-    const int qt = a.n_qtiles - 1 - (int)(blockIdx.x / bh_count);
+    const int qt = a.n_ctas_per_head - 1 - (int)(blockIdx.x / bh_count);
     const int bh = (int)(blockIdx.x % bh_count);
     const int b = bh / a.n_q;
     const int h = bh % a.n_q;
@@ -327,14 +334,353 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
 }
 
+}  // namespace tile64
+
+// ---------------------------------------------------------------- d_k = 128
+// warps 0-3 softmax of query tile 0 and warps 4-7 of query tile 1 (thread r of a
+// group owns row r = TMEM lane r), warp 8 TMA producer (both Q tiles once, K/V
+// ring), warp 9 TMEM allocation and MMA issue: P_0(n) V(n), Q_0 K(n+1)^T,
+// P_1(n) V(n), Q_1 K(n+1)^T, ... so one tile's softmax overlaps the other's MMAs.
+// S_t is one 128-column buffer per tile; P_t(n) over its first 64 columns.
+namespace pair128 {
+
+constexpr int BM = 128;              // query rows per tile (TMEM lanes)
+constexpr int QT = 2;                // query tiles per CTA
+constexpr int BN = 128;              // K/V positions per tile
+constexpr int kSoftmaxWarps = 4 * QT;
+constexpr int kProducerWarp = kSoftmaxWarps;
+constexpr int kMmaWarp = kSoftmaxWarps + 1;
+constexpr int kThreads = 32 * (kSoftmaxWarps + 2);
+constexpr int kTmemCols = 512;       // S_0 | S_1 | O_0 | O_1
+
+template <int DK, int DV>
+struct Cfg {
+    static constexpr int KB = DK / 64;  // 64-wide swizzle blocks along d_k
+    static constexpr int VB = DV / 64;  // ... along d_v
+    static constexpr int Q_BYTES = BM * DK * 2;  // one query tile
+    static constexpr int K_BYTES = BN * DK * 2;
+    static constexpr int V_BYTES = BN * DV * 2;
+    static constexpr int STAGE_BYTES = K_BYTES + V_BYTES;
+    static constexpr int RING = 220 * 1024 - QT * Q_BYTES;
+    static constexpr int STAGES = RING / STAGE_BYTES > 4 ? 4 : RING / STAGE_BYTES;
+    static_assert(STAGES >= 2, "at least two K/V stages");
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_KV = QT * Q_BYTES;
+    static constexpr int OFF_BAR = OFF_KV + STAGES * STAGE_BYTES;
+    static constexpr int SMEM = OFF_BAR + 256 + 1024;  // barriers/flags + alignment slack
+    static constexpr uint32_t T_O = QT * BN;            // first O column
+};
+
+
+template <int DK, int DV>
+__global__ void __launch_bounds__(kThreads, 1)
+    prefill_causal_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                          const __grid_constant__ CUtensorMap tm_v, const PrefillArgs a) {
+    using C = Cfg<DK, DV>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
+    uint64_t *kv_full = bars;        // [STAGES]
+    uint64_t *kv_empty = bars + 4;   // [STAGES]
+    uint64_t *q_full = bars + 8;
+    uint64_t *s_full = bars + 9;     // [QT]
+    uint64_t *p_full = bars + 11;    // [QT]
+    uint64_t *pv_done = bars + 13;   // [QT]
+    uint64_t *mma_done = bars + 15;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 16);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 17);
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+
+    // heaviest tile pairs first: the pair index descends with blockIdx
+    const int bh_count = a.batch * a.n_q;
+    const int qp = a.n_ctas_per_head - 1 - (int)(blockIdx.x / bh_count);
+    const int bh = (int)(blockIdx.x % bh_count);
+    const int b = bh / a.n_q;
+    const int h = bh % a.n_q;
+    const int kh = h / a.q_per_k;
+    const int vh = h / a.q_per_v;
+    const int row0 = qp * QT * BM;
+    const int kv_tiles_total = (a.seq + BN - 1) / BN;
+    int n_kv[QT];
+#pragma unroll
+    for (int t = 0; t < QT; ++t) n_kv[t] = min(kv_tiles_total, (row0 + (t + 1) * BM + BN - 1) / BN);
+    const int n_kv_all = n_kv[QT - 1];
+
+    if (tid == 0) {
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(&kv_full[s], 1);
+            mbar_init(&kv_empty[s], 1);
+        }
+        mbar_init(q_full, 1);
+        for (int t = 0; t < QT; ++t) {
+            mbar_init(&s_full[t], 1);
+            mbar_init(&p_full[t], 4);
+            mbar_init(&pv_done[t], 1);
+        }
+        mbar_init(mma_done, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == kMmaWarp) {
+        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == kProducerWarp) {
+        // ======================= TMA producer
+        if (lane == 0) {
+            prefetch_tensormap(&tm_q);
+            prefetch_tensormap(&tm_k);
+            prefetch_tensormap(&tm_v);
+            mbar_arrive_expect_tx(q_full, QT * C::Q_BYTES);
+#pragma unroll
+            for (int t = 0; t < QT; ++t)
+#pragma unroll
+                for (int kb = 0; kb < C::KB; ++kb)
+                    tma_load_4d(smem + C::OFF_Q + t * C::Q_BYTES + kb * (BM * 128), &tm_q, q_full, kb * 64, h,
+                                row0 + t * BM, b);
+            for (int n = 0; n < n_kv_all; ++n) {
+                const int st = n % C::STAGES;
+                if (n >= C::STAGES)
+                    mbar_wait_bounded(&kv_empty[st], (uint32_t)(((n / C::STAGES) - 1) & 1), a.wait_limit_ns,
+                                      abort_flag, a.status);
+                if (*abort_flag) break;
+                uint8_t *kdst = smem + C::OFF_KV + st * C::STAGE_BYTES;
+                uint8_t *vdst = kdst + C::K_BYTES;
+                mbar_arrive_expect_tx(&kv_full[st], C::STAGE_BYTES);
+#pragma unroll
+                for (int kb = 0; kb < C::KB; ++kb)
+                    tma_load_4d(kdst + kb * (BN * 128), &tm_k, &kv_full[st], kb * 64, kh, n * BN, b);
+#pragma unroll
+                for (int vb = 0; vb < C::VB; ++vb)
+                    tma_load_4d(vdst + vb * (BN * 128), &tm_v, &kv_full[st], vb * 64, vh, n * BN, b);
+            }
+            // drain: no copy may still be landing when the CTA exits
+            mbar_wait_bounded(q_full, 0, a.wait_limit_ns, nullptr, a.status);
+            for (int n = (n_kv_all > C::STAGES ? n_kv_all - C::STAGES : 0); n < n_kv_all; ++n)
+                mbar_wait_bounded(&kv_full[n % C::STAGES], (uint32_t)((n / C::STAGES) & 1), a.wait_limit_ns,
+                                  nullptr, a.status);
+        }
+    } else if (warp == kMmaWarp) {
+        // ======================= MMA issuer (one thread)
+        if (lane == 0) {
+            constexpr uint32_t idesc_qk = umma_idesc_bf16(BM, BN, false, false);
+            constexpr uint32_t idesc_pv = umma_idesc_bf16(BM, DV, false, true);
+            const uint32_t q_addr = smem_addr(smem + C::OFF_Q);
+            int kv_waited = -1;  // highest K/V stage fill waited for
+            // S_t(n) = Q_t K(n)^T into the tile's S columns
+            auto issue_qk = [&](int t, int n) {
+                if (n > kv_waited) {
+                    mbar_wait_bounded(&kv_full[n % C::STAGES], (uint32_t)((n / C::STAGES) & 1), a.wait_limit_ns,
+                                      abort_flag, a.status);
+                    kv_waited = n;
+                }
+                tc_fence_after();
+                const uint32_t k_addr = smem_addr(smem + C::OFF_KV + (n % C::STAGES) * C::STAGE_BYTES);
+                const uint32_t qa = q_addr + (uint32_t)(t * C::Q_BYTES);
+#pragma unroll
+                for (int ks = 0; ks < DK / 16; ++ks) {
+                    const uint32_t blk = (uint32_t)(ks >> 2), sub = (uint32_t)(ks & 3) * 32u;
+                    const uint64_t da = smem_desc_sw128(qa + blk * (BM * 128) + sub, 16, 1024);
+                    const uint64_t db = smem_desc_sw128(k_addr + blk * (BN * 128) + sub, 16, 1024);
+                    umma_bf16(tmem + (uint32_t)(t * BN), da, db, idesc_qk, ks > 0 ? 1u : 0u);
+                }
+                umma_commit(&s_full[t]);
+            };
+            mbar_wait_bounded(q_full, 0, a.wait_limit_ns, abort_flag, a.status);
+#pragma unroll
+            for (int t = 0; t < QT; ++t)
+                if (n_kv[t] > 0) issue_qk(t, 0);
+            for (int n = 0; n < n_kv_all; ++n) {
+                const uint32_t v_addr =
+                    smem_addr(smem + C::OFF_KV + (n % C::STAGES) * C::STAGE_BYTES + C::K_BYTES);
+#pragma unroll
+                for (int t = 0; t < QT; ++t) {
+                    if (n >= n_kv[t]) continue;
+                    // O_t += P_t(n) V(n), P_t(n) in the first 64 columns of S_t
+                    mbar_wait_bounded(&p_full[t], (uint32_t)(n & 1), a.wait_limit_ns, abort_flag, a.status);
+                    tc_fence_after();
+#pragma unroll
+                    for (int ks = 0; ks < BN / 16; ++ks) {
+                        const uint64_t db = smem_desc_sw128(v_addr + (uint32_t)ks * (16 * 128), BN * 128, 1024);
+                        umma_bf16_tmem_a(tmem + C::T_O + (uint32_t)(t * DV), tmem + (uint32_t)(t * BN + ks * 8), db,
+                                         idesc_pv, (n > 0 || ks > 0) ? 1u : 0u);
+                    }
+                    umma_commit(&pv_done[t]);
+                    if (n + 1 < n_kv[t]) issue_qk(t, n + 1);
+                }
+                umma_commit(&kv_empty[n % C::STAGES]);  // every MMA reading stage n has been issued
+            }
+            umma_commit(mma_done);
+            mbar_wait_bounded(mma_done, 0, a.wait_limit_ns, nullptr, a.status);
+        }
+    } else {
+        // ======================= softmax: warps 4t .. 4t+3 for query tile t, thread r owns row r
+        const int t = warp >> 2;
+        const int r = tid & (BM - 1);
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        const uint32_t t_s = tmem + (uint32_t)(t * BN) + lane_base;
+        const uint32_t t_o = tmem + C::T_O + (uint32_t)(t * DV) + lane_base;
+        const int tile_row0 = row0 + t * BM;
+        const int i = tile_row0 + r;  // query position of this thread's row
+        const int nk = n_kv[t];
+        float m_used = -INFINITY;     // log2-domain maximum the stored O and l are relative to
+        float l = 0.f;
+        for (int n = 0; n < nk; ++n) {
+            mbar_wait_bounded(&s_full[t], (uint32_t)(n & 1), a.wait_limit_ns, abort_flag, a.status);
+            tc_fence_after();
+            float s[BN];
+#pragma unroll
+            for (int c = 0; c < BN; c += 32) {
+                uint32_t rr[32];
+                tmem_ld32(t_s + (uint32_t)c, rr);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) s[c + e] = __uint_as_float(rr[e]);
+            }
+            tmem_wait_ld();
+
+            // causal mask on tiles that reach past this tile's first row
+            const int j0 = n * BN;
+            if (j0 + BN - 1 > tile_row0) {
+#pragma unroll
+                for (int c = 0; c < BN; ++c)
+                    if (j0 + c > i) s[c] = -INFINITY;
+            }
+            // row max as 8 independent chains
+            float mx8[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) mx8[e] = s[e];
+#pragma unroll
+            for (int c = 8; c < BN; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
+            const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                   fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+            const float m_new = mx * a.scale_log2;
+            bool waited_pv = false;
+            if (n == 0) {
+                m_used = m_new;
+            } else {
+                const bool need = m_new > m_used + kRescaleLog2;
+                if (__any_sync(0xffffffffu, need)) {
+                    // O must be final for tile n-1 before it is rescaled in TMEM
+                    mbar_wait_bounded(&pv_done[t], (uint32_t)((n - 1) & 1), a.wait_limit_ns, abort_flag, a.status);
+                    waited_pv = true;
+                    tc_fence_after();
+                    const float alpha = need ? fast_exp2(m_used - m_new) : 1.f;
+#pragma unroll 1
+                    for (int c = 0; c < DV; c += 32) {
+                        uint32_t rr[32];
+                        tmem_ld32(t_o + (uint32_t)c, rr);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) rr[e] = __float_as_uint(__uint_as_float(rr[e]) * alpha);
+                        tmem_st32(t_o + (uint32_t)c, rr);
+                    }
+                    tmem_wait_st();
+                    if (need) {
+                        l *= alpha;
+                        m_used = m_new;
+                    }
+                }
+            }
+            // p = 2^(s * scale * log2 e - m): packed fp32 pairs, row sum as 4 pair-chains;
+            // P in bf16 pairs over the first 64 columns of S (key 2c in the low half of column c)
+            const f32x2_t sc2 = f2_pack(a.scale_log2, a.scale_log2);
+            const f32x2_t nm2 = f2_pack(-m_used, -m_used);
+            f32x2_t l2[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+            for (int c0 = 0; c0 < BN; c0 += 64) {
+                uint32_t pk[32];
+#pragma unroll
+                for (int c = 0; c < 64; c += 2) {
+                    float t0, t1;
+                    f2_unpack(f2_fma(f2_pack(s[c0 + c], s[c0 + c + 1]), sc2, nm2), t0, t1);
+                    const float p0 = fast_exp2(t0);
+                    const float p1 = fast_exp2(t1);
+                    l2[(c >> 1) & 3] = f2_add(l2[(c >> 1) & 3], f2_pack(p0, p1));
+                    pk[c >> 1] = pack_bf16x2(p0, p1);
+                }
+                tmem_st32(t_s + (uint32_t)(c0 / 2), pk);
+            }
+            float la, lb;
+            f2_unpack(f2_add(f2_add(l2[0], l2[1]), f2_add(l2[2], l2[3])), la, lb);
+            l += la + lb;
+            tmem_wait_st();
+            if (n >= 1 && !waited_pv) {
+                // keeps this group at most one P.V behind, so every pv_done phase is waited in turn
+                mbar_wait_bounded(&pv_done[t], (uint32_t)((n - 1) & 1), a.wait_limit_ns, abort_flag, a.status);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&p_full[t]);
+        }
+        // epilogue: O / l -> bf16
+        if (nk > 0) {
+            mbar_wait_bounded(&pv_done[t], (uint32_t)((nk - 1) & 1), a.wait_limit_ns, abort_flag, a.status);
+            tc_fence_after();
+            const float inv_l = l > 0.f ? 1.f / l : 0.f;
+            __nv_bfloat16 *orow = a.out + (((size_t)b * a.seq + i) * a.n_q + h) * DV;
+#pragma unroll 1
+            for (int c = 0; c < DV; c += 32) {
+                uint32_t rr[32];
+                tmem_ld32(t_o + (uint32_t)c, rr);
+                tmem_wait_ld();
+                if (i < a.seq) {
+#pragma unroll
+                    for (int e = 0; e < 32; e += 8) {
+                        uint4 v;
+                        v.x = pack_bf16x2(__uint_as_float(rr[e]) * inv_l, __uint_as_float(rr[e + 1]) * inv_l);
+                        v.y = pack_bf16x2(__uint_as_float(rr[e + 2]) * inv_l, __uint_as_float(rr[e + 3]) * inv_l);
+                        v.z = pack_bf16x2(__uint_as_float(rr[e + 4]) * inv_l, __uint_as_float(rr[e + 5]) * inv_l);
+                        v.w = pack_bf16x2(__uint_as_float(rr[e + 6]) * inv_l, __uint_as_float(rr[e + 7]) * inv_l);
+                        *reinterpret_cast<uint4 *>(orow + c + e) = v;
+                    }
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+}  // namespace pair128
+
 using PrefillFn = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, PrefillArgs);
 
-PrefillFn pick(int dk, int dv, int *smem) {
-    if (dk == 64 && dv == 64) { *smem = Cfg<64, 64>::SMEM; return prefill_causal_kernel<64, 64>; }
-    if (dk == 64 && dv == 128) { *smem = Cfg<64, 128>::SMEM; return prefill_causal_kernel<64, 128>; }
-    if (dk == 128 && dv == 64) { *smem = Cfg<128, 64>::SMEM; return prefill_causal_kernel<128, 64>; }
-    if (dk == 128 && dv == 128) { *smem = Cfg<128, 128>::SMEM; return prefill_causal_kernel<128, 128>; }
-    return nullptr;
+struct Plan {
+    PrefillFn fn;
+    int smem, threads, rows_per_cta, q_box, kv_box;
+};
+
+bool pick(int dk, int dv, Plan *p) {
+    if (dk == 64) {
+        using namespace tile64;
+        p->threads = kThreads;
+        p->rows_per_cta = BM;
+        p->q_box = BM;
+        p->kv_box = BN;
+        if (dv == 64) { p->smem = Cfg<64, 64>::SMEM; p->fn = prefill_causal_kernel<64, 64>; return true; }
+        if (dv == 128) { p->smem = Cfg<64, 128>::SMEM; p->fn = prefill_causal_kernel<64, 128>; return true; }
+    } else if (dk == 128) {
+        using namespace pair128;
+        p->threads = kThreads;
+        p->rows_per_cta = QT * BM;
+        p->q_box = BM;
+        p->kv_box = BN;
+        if (dv == 64) { p->smem = Cfg<128, 64>::SMEM; p->fn = prefill_causal_kernel<128, 64>; return true; }
+        if (dv == 128) { p->smem = Cfg<128, 128>::SMEM; p->fn = prefill_causal_kernel<128, 128>; return true; }
+    }
+    return false;
 }
 
 }  // namespace
@@ -345,19 +691,21 @@ diffqkv_status_t prefill_launch(const diffqkv_dims_t *d, const void *q, const vo
     if (st != DIFFQKV_OK) return st;
     if (!q || !k || !v || !out || seq_len < 1) return DIFFQKV_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return DIFFQKV_ERR_MISALIGNED;
-    int smem = 0;
-    PrefillFn fn = pick(d->d_k, d->d_v, &smem);
-    if (!fn) return DIFFQKV_ERR_UNSUPPORTED;
+    Plan plan;
+    if (!pick(d->d_k, d->d_v, &plan)) return DIFFQKV_ERR_UNSUPPORTED;
     DeviceInfo dev;
     st = current_device_info(&dev);
     if (st != DIFFQKV_OK) return st;
 
     CUtensorMap tm_q, tm_k, tm_v;
-    st = make_tensor_map_4d(&tm_q, q, d->d_k, d->n_q, seq_len, d->batch, 64, 1, BM, 1, CU_TENSOR_MAP_SWIZZLE_128B);
+    st = make_tensor_map_4d(&tm_q, q, d->d_k, d->n_q, seq_len, d->batch, 64, 1, plan.q_box, 1,
+                            CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != DIFFQKV_OK) return st;
-    st = make_tensor_map_4d(&tm_k, k, d->d_k, d->n_k, seq_len, d->batch, 64, 1, BN, 1, CU_TENSOR_MAP_SWIZZLE_128B);
+    st = make_tensor_map_4d(&tm_k, k, d->d_k, d->n_k, seq_len, d->batch, 64, 1, plan.kv_box, 1,
+                            CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != DIFFQKV_OK) return st;
-    st = make_tensor_map_4d(&tm_v, v, d->d_v, d->n_v, seq_len, d->batch, 64, 1, BN, 1, CU_TENSOR_MAP_SWIZZLE_128B);
+    st = make_tensor_map_4d(&tm_v, v, d->d_v, d->n_v, seq_len, d->batch, 64, 1, plan.kv_box, 1,
+                            CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != DIFFQKV_OK) return st;
 
     PrefillArgs a;
@@ -370,13 +718,13 @@ diffqkv_status_t prefill_launch(const diffqkv_dims_t *d, const void *q, const vo
     a.n_v = d->n_v;
     a.q_per_k = d->n_q / d->n_k;
     a.q_per_v = d->n_q / d->n_v;
-    a.n_qtiles = (seq_len + BM - 1) / BM;
+    a.n_ctas_per_head = (seq_len + plan.rows_per_cta - 1) / plan.rows_per_cta;
     a.scale_log2 = (float)((double)d->scale * 1.4426950408889634);
     a.wait_limit_ns = kWaitLimitNs;
-    const long long grid = (long long)a.n_qtiles * d->batch * d->n_q;
+    const long long grid = (long long)a.n_ctas_per_head * d->batch * d->n_q;
     if (grid > 0x7fffffffLL) return DIFFQKV_ERR_UNSUPPORTED;
-    if (ensure_dynamic_smem((const void *)fn, smem) != DIFFQKV_OK) return DIFFQKV_ERR_CUDA;
-    fn<<<(unsigned)grid, kThreads, smem, stream>>>(tm_q, tm_k, tm_v, a);
+    if (ensure_dynamic_smem((const void *)plan.fn, plan.smem) != DIFFQKV_OK) return DIFFQKV_ERR_CUDA;
+    plan.fn<<<(unsigned)grid, plan.threads, plan.smem, stream>>>(tm_q, tm_k, tm_v, a);
     if (cudaGetLastError() != cudaSuccess) return DIFFQKV_ERR_CUDA;
     return DIFFQKV_OK;
 }
