@@ -49,6 +49,7 @@ PROFILE_CASES = {
     "decode_b4_t32768": wl.DecodeWorkload("decode_b4_t32768", wl.DIFFQKV, 4, 32768, seed=1),
     "decode_gqa_b4_t32768": wl.DecodeWorkload("decode_gqa_b4_t32768", wl.GQA_CONTROL, 4, 32768, seed=1),
     "prefill_b2_s8192": wl.PREFILL_8K,
+    "prefill_gqa_b2_s8192": wl.PREFILL_8K_GQA,
     "topv_b4_t65536": wl.TOPV_64K,
 }
 L2_FLUSH_BYTES = 256 << 20  # written between timed calls whose inputs fit in the 126 MB L2
