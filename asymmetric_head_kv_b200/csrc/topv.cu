@@ -620,6 +620,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) topv_select_kernel(const TopvA
     __shared__ uint32_t warp_sums[33];
     __shared__ uint16_t q_s[DK];
     __shared__ uint32_t keys_s[kPairwiseMax][kKeyWords];
+    __shared__ int32_t alist_s[kPairwiseMax];  // the first ambiguous positions (the whole list when pairwise)
     __shared__ float red_s[kSelWarps];
     __shared__ int sh_d;
     __shared__ uint32_t sh_above;
@@ -743,7 +744,9 @@ __global__ void __launch_bounds__(kSelThreads, 1) topv_select_kernel(const TopvA
                 atomicOr(bitmap + (j >> 5), 1u << (j & 31));
                 ++my_in;
             } else if (x >= lo_edge) {
-                alist[atomicAdd(&sh_na, 1)] = cj[i];
+                const int slot = atomicAdd(&sh_na, 1);
+                alist[slot] = cj[i];
+                if (slot < kPairwiseMax) alist_s[slot] = cj[i];
             }
         }
 #pragma unroll
@@ -763,7 +766,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) topv_select_kernel(const TopvA
         } else if (na <= kPairwiseMax) {
             // rank the few ambiguous positions pairwise by exact key (a warp per key)
             for (int r = warp; r < na; r += kSelWarps) {
-                const int j = alist[r];
+                const int j = alist_s[r];
                 exact_key_warp<DK>(q_s, reinterpret_cast<const uint16_t *>(krow0 + (size_t)j * kstride), j,
                                    keys_s[r], lane);
             }

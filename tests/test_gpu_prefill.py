@@ -45,6 +45,18 @@ def test_shapes(cuda_device, name):
     assert_parity(out, oracle.prefill_causal(d["q"], d["k"], d["v"], d["scale"]), name)
 
 
+@pytest.mark.parametrize("seq", [1, 5, 127, 128, 129, 255, 256, 257, 300, 600])
+def test_lengths_dk128(cuda_device, seq):
+    """The d_k = 128 tiling runs two 128-row query tiles per CTA over 128-position K/V tiles:
+    lengths around those boundaries put the second tile partly or wholly past the end and
+    give the two tiles different K/V tile counts."""
+    s = wl.GQA_CONTROL
+    d = wl.random_prefill_inputs(1, seq, s, seed=440 + seq)
+    out = _gpu(d, cuda_device)
+    assert_parity(out, oracle.prefill_causal(d["q"], d["k"], d["v"], d["scale"]), f"d_k 128, S={seq}")
+    assert torch.equal(out[:, 0].cpu(), d["v"][:, 0].repeat_interleave(s.n_q // s.n_v, dim=1))
+
+
 def test_sharp_softmax_rescaling(cuda_device):
     """Large score growth along the sequence forces the in-TMEM output rescaling path."""
     d = wl.random_prefill_inputs(1, 700, wl.DIFFQKV, seed=420)
@@ -52,6 +64,15 @@ def test_sharp_softmax_rescaling(cuda_device):
     d["k"] = (d["k"].float() * ramp[None, :, None, None].float()).to(torch.bfloat16)
     out = _gpu(d, cuda_device)
     assert_parity(out, oracle.prefill_causal(d["q"], d["k"], d["v"], d["scale"]), "rescale")
+
+
+def test_sharp_softmax_rescaling_dk128(cuda_device):
+    """The same ramp on the d_k = 128 tiling (its own rescale path, one per query tile)."""
+    d = wl.random_prefill_inputs(1, 700, wl.GQA_CONTROL, seed=421)
+    ramp = torch.linspace(0.1, 6.0, 700).to(torch.bfloat16)
+    d["k"] = (d["k"].float() * ramp[None, :, None, None].float()).to(torch.bfloat16)
+    out = _gpu(d, cuda_device)
+    assert_parity(out, oracle.prefill_causal(d["q"], d["k"], d["v"], d["scale"]), "rescale d_k 128")
 
 
 def test_prefill_rows_match_gpu_decode(cuda_device):
