@@ -7,12 +7,13 @@
 // ranked by the EXACT dot product q.k (ties toward the lower position) so the
 // selected set is unique and reproducible.
 //
-// Three launches:
+// Four launches:
 //  1. topv_score_kernel -- streams K once with TMA (one K row serves all
-//     n_q/n_k query heads of its group; one position per thread) and writes
-//     fp32 scores s_j = q.k_j (unscaled fp32 FMAs, two per packed f32x2
-//     instruction; every bf16 x bf16 product is exact), a 2048-bucket histogram of the top 11 bits of each
-//     score's order key per row, and per (batch, K head) the largest |k|.
+//     n_q/n_k query heads of its group; four lanes per position, q in
+//     registers) and writes fp32 scores s_j = q.k_j (unscaled fp32 FMAs, two
+//     per packed f32x2 instruction; every bf16 x bf16 product is exact), a
+//     2048-bucket histogram of the top 11 bits of each score's order key per
+//     row, and per (batch, K head) the largest |k|.
 //  2. topv_filter_kernel -- all SMs: per row, the histogram gives the bucket
 //     holding the k-th largest score; every position whose score is at least
 //     that bucket's lower end minus 2d (d the rounding bound below) is

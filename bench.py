@@ -385,7 +385,7 @@ def time_paths(ak, peaks, steps: int, warmup: int):
     hbm = float(peaks["hbm_gbs"])
     res[w.name] = {"us": ms * 1e3, "algorithmic_bytes": nbytes, "gbs": nbytes / (ms * 1e-3) / 1e9,
                    "bound": "hbm", "peak_gbs": hbm, "frac": nbytes / (ms * 1e-3) / 1e9 / hbm,
-                   "launches_per_call": 3}
+                   "launches_per_call": 4}
     assert ak.device_status() == 0
     return res
 

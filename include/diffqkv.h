@@ -185,7 +185,8 @@ size_t diffqkv_decode_topv_workspace_size(const diffqkv_dims_t *dims, int32_t t_
  * max_seq_len is accepted for symmetry with diffqkv_decode and ignored: the
  * kernels read the lengths from seq_lens on the device.  Lengths outside
  * [0, t_max] are clamped to that range.  A row with length 0 gets a zero
- * output and an all -1 index row.  Launches three kernels on `stream`;
+ * output and an all -1 index row.  Launches four kernels on `stream`
+ * (chained with programmatic dependent launch);
  * returns once they are queued.
  */
 diffqkv_status_t diffqkv_decode_topv(const diffqkv_dims_t *dims, const void *q, const void *k_cache,
