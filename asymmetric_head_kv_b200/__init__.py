@@ -112,6 +112,35 @@ def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, seq_le
     return out
 
 
+def decode_append(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor, k_cache: torch.Tensor,
+                  v_cache: torch.Tensor, seq_lens: torch.Tensor, *, scale: Optional[float] = None,
+                  max_seq_len: Optional[int] = None, out: Optional[torch.Tensor] = None,
+                  workspace: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Decode step with the KV-cache append fused in: writes k_new [B, n_k, d_k] and v_new [B, n_v, d_v]
+    into the caches at position seq_lens[b] (the cached count before the step; not modified) and
+    returns attention over positions 0..seq_lens[b] of the updated caches, bf16 [B, n_q, d_v]."""
+    _bf16_dev(q, "q", 3)
+    _bf16_dev(k_new, "k_new", 3)
+    _bf16_dev(v_new, "v_new", 3)
+    _bf16_dev(k_cache, "k_cache", 4)
+    _bf16_dev(v_cache, "v_cache", 4)
+    if seq_lens.dtype != torch.int32 or not seq_lens.is_cuda:
+        raise TypeError("seq_lens must be an int32 CUDA tensor")
+    dims, t_max = _decode_dims(q, k_cache, v_cache, scale)
+    if tuple(k_new.shape) != (dims.batch, dims.n_k, dims.d_k) or tuple(v_new.shape) != (dims.batch, dims.n_v, dims.d_v):
+        raise ValueError("k_new must be [B, n_k, d_k] and v_new [B, n_v, d_v]")
+    if out is None:
+        out = torch.empty((dims.batch, dims.n_q, dims.d_v), dtype=torch.bfloat16, device=q.device)
+    if workspace is None:
+        workspace = decode_workspace(dims, device=q.device)
+    msl = t_max if max_seq_len is None else int(max_seq_len)
+    st = lib().diffqkv_decode_append(ctypes.byref(dims), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache),
+                                     _ptr(v_cache), _ptr(seq_lens), t_max, msl, _ptr(out), _ptr(workspace),
+                                     workspace.numel(), _stream_ptr(stream))
+    check(st, "diffqkv_decode_append")
+    return out
+
+
 def decode_from_host(q_host, k_host, v_host, seq_lens_host, out_host, dev_buffers: dict, *,
                      scale: Optional[float] = None, max_seq_len: Optional[int] = None,
                      stream: Optional[torch.cuda.Stream] = None) -> None:

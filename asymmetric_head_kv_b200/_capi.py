@@ -78,6 +78,7 @@ SIGNATURES = {
     "diffqkv_workspace_init": ([_P, _SZ, _P], _I32),
     "diffqkv_decode": ([_DIMS, _P, _P, _P, _P, _I32, _I32, _P, _P, _SZ, _P], _I32),
     "diffqkv_decode_ex": ([_DIMS, _P, _P, _P, _P, _I32, _I32, _P, _P, _SZ, ctypes.POINTER(DecodeTuning), _P], _I32),
+    "diffqkv_decode_append": ([_DIMS, _P, _P, _P, _P, _P, _P, _I32, _I32, _P, _P, _SZ, _P], _I32),
     "diffqkv_decode_plan": ([_DIMS, _I32, _I32, _I32, ctypes.POINTER(DecodeTuning), ctypes.POINTER(DecodePlan)],
                             _I32),
     "diffqkv_decode_from_host": ([_DIMS, _P, _P, _P, _P, _I32, _I32, _P, _P, _P, _P, _P, _P, _P, _SZ, _P], _I32),

@@ -204,6 +204,16 @@ diffqkv_status_t diffqkv_decode(const diffqkv_dims_t *dims, const void *q, const
                                   workspace_bytes, nullptr, (cudaStream_t)stream);
 }
 
+diffqkv_status_t diffqkv_decode_append(const diffqkv_dims_t *dims, const void *q, const void *k_new,
+                                       const void *v_new, void *k_cache, void *v_cache,
+                                       const int32_t *seq_lens, int32_t t_max, int32_t max_seq_len,
+                                       void *out, void *workspace, size_t workspace_bytes,
+                                       diffqkv_stream_t stream) {
+    if (!k_new || !v_new) return DIFFQKV_ERR_INVALID_ARG;
+    return diffqkv::decode_launch(dims, q, k_cache, v_cache, seq_lens, t_max, max_seq_len, out, workspace,
+                                  workspace_bytes, nullptr, (cudaStream_t)stream, k_new, v_new);
+}
+
 diffqkv_status_t diffqkv_decode_ex(const diffqkv_dims_t *dims, const void *q, const void *k_cache,
                                    const void *v_cache, const int32_t *seq_lens, int32_t t_max, int32_t max_seq_len,
                                    void *out, void *workspace, size_t workspace_bytes,

@@ -25,6 +25,11 @@
 //  * The combine is fused: the last CTA to finish a unit (atomic counter in
 //    the workspace, reset afterwards) merges that unit's split partials and
 //    writes bf16 output.  No CTA ever waits on another.
+//  * Append mode (k_new, v_new given): the step's new token joins the cache at
+//    position p = seq_len and the output attends over positions 0..p.  The
+//    tiles still cover the p cached positions only; the combining CTA adds the
+//    new token as one more partial (m = its score, l = 1, o = v_new) and writes
+//    k_new / v_new into the cache at p, which no CTA of this launch reads.
 #include <math.h>
 
 #include <algorithm>
@@ -43,6 +48,10 @@ constexpr int kPartialPad = 4;        // per-head partial record: o[d_v], m, l, 
 
 struct DecodeArgs {
     const __nv_bfloat16 *q;
+    const __nv_bfloat16 *k_new = nullptr;  // [B, n_k, d_k] (append mode) or null
+    const __nv_bfloat16 *v_new = nullptr;  // [B, n_v, d_v] (append mode) or null
+    __nv_bfloat16 *k_store = nullptr;      // the K cache, written at position seq_len (append mode)
+    __nv_bfloat16 *v_store = nullptr;      // the V cache, likewise
     const int32_t *seq_lens;
     __nv_bfloat16 *out;
     float *partials;
@@ -198,11 +207,23 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
     __syncthreads();
 
     const long long N = scan_s[0];
-    // sequences with no cached positions produce zero rows (distributed over CTAs)
+    // sequences with no cached positions produce zero rows (distributed over CTAs); in
+    // append mode their output is the new token's V row, and the new token fills position 0
     for (int b = (int)c; b < a.batch; b += (int)G) {
         if (clamp_len(__ldg(a.seq_lens + b), a.t_max) == 0) {
             __nv_bfloat16 *o = a.out + (size_t)b * a.n_q * DV;
-            for (int e = tid; e < a.n_q * DV; e += blockDim.x) o[e] = __float2bfloat16(0.f);
+            if (a.k_new) {
+                for (int e = tid; e < a.n_q * DV; e += blockDim.x) {
+                    const int h = e / DV;
+                    o[e] = a.v_new[((size_t)b * a.n_v + h / a.q_per_v) * DV + e % DV];
+                }
+                for (int e = tid; e < a.n_k * DK; e += blockDim.x)
+                    a.k_store[(size_t)b * a.t_max * a.n_k * DK + e] = a.k_new[(size_t)b * a.n_k * DK + e];
+                for (int e = tid; e < a.n_v * DV; e += blockDim.x)
+                    a.v_store[(size_t)b * a.t_max * a.n_v * DV + e] = a.v_new[(size_t)b * a.n_v * DV + e];
+            } else {
+                for (int e = tid; e < a.n_q * DV; e += blockDim.x) o[e] = __float2bfloat16(0.f);
+            }
         }
     }
     const long long Ge = N < G ? N : G;  // CTAs that own tiles
@@ -428,6 +449,38 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
             named_barrier(1, NCW * 32);
             if (*last_flag) {
                 __threadfence();
+                // append mode: the new token's score for each query head of the group (merge_s is
+                // free again here), and its K / V rows into the cache at position p
+                const bool append = a.k_new != nullptr && w.T < a.t_max;
+                if (a.k_new != nullptr && !append && tid == 0) record_error(a.status, DIFFQKV_ERR_DEVICE_SEQLEN);
+                if (append) {
+                    const int p = w.T;
+                    if (warp < QPK) {
+                        const int h = w.g * QPK + warp;
+                        const __nv_bfloat16 *qh = a.q + ((size_t)w.b * a.n_q + h) * DK;
+                        const __nv_bfloat16 *kn = a.k_new + ((size_t)w.b * a.n_k + w.g) * DK;
+                        float dot = 0.f;
+                        for (int e = lane; e < DK; e += 32)
+                            dot = fmaf(__bfloat162float(qh[e]), __bfloat162float(kn[e]), dot);
+#pragma unroll
+                        for (int off = 16; off >= 1; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+                        if (lane == 0) merge_s[warp] = dot * a.scale_log2;
+                    }
+                    const size_t kdst = (((size_t)w.b * a.t_max + p) * a.n_k + w.g) * DK;
+                    const size_t ksrc = ((size_t)w.b * a.n_k + w.g) * DK;
+                    for (int e = tid; e < DK / 8; e += NCW * 32)
+                        reinterpret_cast<uint4 *>(a.k_store + kdst)[e] = reinterpret_cast<const uint4 *>(a.k_new + ksrc)[e];
+                    for (int e = tid; e < QPK * (DV / 8); e += NCW * 32) {
+                        const int h = w.g * QPK + e / (DV / 8);
+                        if (h % a.q_per_v != 0) continue;  // one writer per V head: its first query head
+                        const int vh = h / a.q_per_v;
+                        const size_t vdst = (((size_t)w.b * a.t_max + p) * a.n_v + vh) * DV;
+                        const size_t vsrc = ((size_t)w.b * a.n_v + vh) * DV;
+                        reinterpret_cast<uint4 *>(a.v_store + vdst)[e % (DV / 8)] =
+                            reinterpret_cast<const uint4 *>(a.v_new + vsrc)[e % (DV / 8)];
+                    }
+                    named_barrier(1, NCW * 32);
+                }
                 constexpr int ITEMS = QPK * (DV / 4);
                 for (int it = tid; it < ITEMS; it += NCW * 32) {
                     const int h2 = it / (DV / 4);
@@ -435,6 +488,8 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
                     float M = -INFINITY;
                     for (long long cc = first; cc <= last; ++cc)
                         M = fmaxf(M, __ldcg(a.partials + ((size_t)(u + cc) * QPK + h2) * (DV + kPartialPad) + DV));
+                    const float s_new = append ? merge_s[h2] : -INFINITY;
+                    M = fmaxf(M, s_new);
                     const float Mu = (M == -INFINITY) ? 0.f : M;
                     float L = 0.f;
                     float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -447,6 +502,16 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
                         O.y = fmaf(f, x.y, O.y);
                         O.z = fmaf(f, x.z, O.z);
                         O.w = fmaf(f, x.w, O.w);
+                    }
+                    if (append) {  // the new token: m = s_new, l = 1, o = v_new
+                        const float f = fast_exp2(s_new - Mu);
+                        L += f;
+                        const int vh = (w.g * QPK + h2) / a.q_per_v;
+                        const __nv_bfloat16 *vn = a.v_new + ((size_t)w.b * a.n_v + vh) * DV + d4 * 4;
+                        O.x = fmaf(f, __bfloat162float(vn[0]), O.x);
+                        O.y = fmaf(f, __bfloat162float(vn[1]), O.y);
+                        O.z = fmaf(f, __bfloat162float(vn[2]), O.z);
+                        O.w = fmaf(f, __bfloat162float(vn[3]), O.w);
                     }
                     const float inv = L > 0.f ? 1.f / L : 0.f;
                     __nv_bfloat162 lo = __floats2bfloat162_rn(O.x * inv, O.y * inv);
@@ -596,13 +661,15 @@ diffqkv_status_t decode_plan(const diffqkv_dims_t *d, int32_t t_max, int32_t max
 diffqkv_status_t decode_launch(const diffqkv_dims_t *d, const void *q, const void *k_cache, const void *v_cache,
                                const int32_t *seq_lens, int32_t t_max, int32_t max_seq_len, void *out,
                                void *workspace, size_t workspace_bytes, const diffqkv_decode_tuning_t *tuning,
-                               cudaStream_t stream) {
+                               cudaStream_t stream, const void *k_new, const void *v_new) {
     diffqkv_status_t st = validate_dims(d);
     if (st != DIFFQKV_OK) return st;
     if (!q || !k_cache || !v_cache || !seq_lens || !out || t_max < 1) return DIFFQKV_ERR_INVALID_ARG;
+    if ((k_new == nullptr) != (v_new == nullptr)) return DIFFQKV_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
         (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
         return DIFFQKV_ERR_MISALIGNED;
+    if (k_new && (!aligned16(k_new) || !aligned16(v_new))) return DIFFQKV_ERR_MISALIGNED;
     const size_t need = decode_workspace_size(d);
     if (!workspace || workspace_bytes < need) return DIFFQKV_ERR_WORKSPACE;
     if (!aligned16(workspace)) return DIFFQKV_ERR_MISALIGNED;
@@ -629,6 +696,12 @@ diffqkv_status_t decode_launch(const diffqkv_dims_t *d, const void *q, const voi
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     const size_t units = (size_t)d->batch * d->n_k;
     a.q = static_cast<const __nv_bfloat16 *>(q);
+    if (k_new) {
+        a.k_new = static_cast<const __nv_bfloat16 *>(k_new);
+        a.v_new = static_cast<const __nv_bfloat16 *>(v_new);
+        a.k_store = static_cast<__nv_bfloat16 *>(const_cast<void *>(k_cache));
+        a.v_store = static_cast<__nv_bfloat16 *>(const_cast<void *>(v_cache));
+    }
     a.seq_lens = seq_lens;
     a.out = static_cast<__nv_bfloat16 *>(out);
     a.counters = reinterpret_cast<uint32_t *>(ws + kWorkspaceHeader);

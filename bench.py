@@ -372,6 +372,45 @@ def time_paths(ak, peaks, steps: int, warmup: int):
         res[w.name] = {"ms": ms, "causal_flops": flops, "tflops": tf, "bound": "tensor", "peak_tflops": bf16_peak,
                        "frac": tf / bf16_peak, "peak_source": "bf16_tflops (burst, cuBLAS bf16 GEMM)"}
         del d, out
+    # the small decode case (batch 1, 512 positions: 2.36 MB, launch/latency bound): microseconds
+    # per call with L2 flushed before each call
+    w = wl.DECODE_SMALL
+    d = wl.make_decode_inputs(w, dev)
+    ws_s = ak.decode_workspace(d["q"], d["k_cache"], d["v_cache"])
+    out_s = torch.empty((w.batch, w.shape.n_q, w.shape.d_v), dtype=torch.bfloat16, device=dev)
+    fn = lambda: ak.decode(d["q"], d["k_cache"], d["v_cache"], d["seq_lens"], scale=d["scale"],  # noqa: E731
+                           out=out_s, workspace=ws_s)
+    for _ in range(max(3, warmup)):
+        fn()
+    ms = statistics.median(_timed_calls(fn, max(20, steps), flush))
+    nbytes = wl.decode_kv_bytes(w.shape, d["seq_lens"].cpu())
+    res[w.name] = {"us": ms * 1e3, "kv_bytes": nbytes, "gbs": nbytes / (ms * 1e-3) / 1e9,
+                   "bound": "launch/latency (L2 flushed between calls)", "launches_per_call": 1}
+    del d, ws_s, out_s
+
+    # decode step with the KV-cache append fused in: 16 sequences of 32767 cached positions, the
+    # new token goes to position 32767; bytes = the cached K/V read plus the new rows written
+    w = WORKLOAD
+    d = wl.make_decode_inputs(w, dev)
+    lens = (d["seq_lens"] - 1).contiguous()
+    g = torch.Generator(device=dev).manual_seed(w.seed + 100)
+    k_new = torch.randn(w.batch, w.shape.n_k, w.shape.d_k, generator=g, device=dev).to(torch.bfloat16)
+    v_new = torch.randn(w.batch, w.shape.n_v, w.shape.d_v, generator=g, device=dev).to(torch.bfloat16)
+    ws_d = ak.decode_workspace(d["q"], d["k_cache"], d["v_cache"])
+    out_d = torch.empty((w.batch, w.shape.n_q, w.shape.d_v), dtype=torch.bfloat16, device=dev)
+    fn = lambda: ak.decode_append(d["q"], k_new, v_new, d["k_cache"], d["v_cache"], lens,  # noqa: E731
+                                  scale=d["scale"], out=out_d, workspace=ws_d)
+    for _ in range(max(3, warmup)):
+        fn()
+    ms = statistics.median(_timed_calls(fn, steps, flush))
+    nbytes = wl.decode_kv_bytes(w.shape, lens.cpu()) + w.batch * w.shape.kv_elems_per_token * wl.BF16_BYTES
+    hbm = float(peaks["hbm_gbs"])
+    res["decode_append_b16_t32768"] = {"us": ms * 1e3, "algorithmic_bytes": nbytes,
+                                       "gbs": nbytes / (ms * 1e-3) / 1e9, "bound": "hbm", "peak_gbs": hbm,
+                                       "frac": nbytes / (ms * 1e-3) / 1e9 / hbm, "launches_per_call": 1}
+    assert ak.device_status() == 0
+    del d, ws_d, out_d
+
     w = wl.TOPV_64K
     d = wl.make_decode_inputs(w, dev)
     ws = ak.decode_topv_workspace(ak.make_dims(w.batch, w.shape.n_q, w.shape.n_k, w.shape.n_v, w.shape.d_k,

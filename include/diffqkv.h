@@ -113,6 +113,29 @@ diffqkv_status_t diffqkv_decode(const diffqkv_dims_t *dims, const void *q, const
                                 int32_t max_seq_len, void *out, void *workspace,
                                 size_t workspace_bytes, diffqkv_stream_t stream);
 
+/*
+ * Decode step with the KV-cache append fused in (the KV-cache store step of
+ * the paper's deployment section, "FlexHeadFA Kernel and Deployment
+ * Infrastructure", done inside the decode launch):
+ *
+ *   k_new    [B, n_k, d_k]   the step's new K rows (bf16, device, 16-byte aligned)
+ *   v_new    [B, n_v, d_v]   the step's new V rows
+ *   seq_lens [B] int32       cached positions BEFORE this step (p_b)
+ *
+ * Writes k_new[b] into k_cache[b, p_b] and v_new[b] into v_cache[b, p_b], and
+ * out[b,h] = attention of q[b,h] over positions 0..p_b of the updated caches
+ * (p_b + 1 positions).  seq_lens is not modified: the caller advances it.
+ * Other arguments, layouts and the workspace are those of diffqkv_decode.  A
+ * row with p_b >= t_max (no free slot) or p_b < 0 is flagged
+ * DIFFQKV_ERR_DEVICE_SEQLEN; with p_b >= t_max nothing is written to its
+ * caches and its output covers the t_max cached positions only.
+ */
+diffqkv_status_t diffqkv_decode_append(const diffqkv_dims_t *dims, const void *q, const void *k_new,
+                                       const void *v_new, void *k_cache, void *v_cache,
+                                       const int32_t *seq_lens, int32_t t_max, int32_t max_seq_len,
+                                       void *out, void *workspace, size_t workspace_bytes,
+                                       diffqkv_stream_t stream);
+
 /* Optional launch controls for diffqkv_decode_ex (0 = library default). */
 typedef struct {
     int32_t grid_ctas;   /* CTAs of the split kernel (>= 1); changes the split points */

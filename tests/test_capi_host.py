@@ -141,3 +141,16 @@ def test_topv_rejects_before_launch():
     small = _capi.lib().diffqkv_decode_topv_workspace_size(ctypes.byref(d), 1024, 8)
     large = _capi.lib().diffqkv_decode_topv_workspace_size(ctypes.byref(d), 2048, 8)
     assert large - small == d.batch * d.n_q * 1024 * 18
+
+
+def test_decode_append_rejects_before_launch():
+    lib = _capi.lib()
+    d = dims()
+
+    def call(kn=0x8000, vn=0x9000, q=0x1000):
+        return lib.diffqkv_decode_append(ctypes.byref(d), q, kn, vn, 0x2000, 0x3000, 0x4000, 128, 128, 0x5000,
+                                         0x6000, 1 << 30, None)
+    assert call(kn=None) == _capi.INVALID_ARG
+    assert call(vn=None) == _capi.INVALID_ARG
+    assert call(kn=0x8008) == _capi.MISALIGNED
+    assert call(q=None) == _capi.INVALID_ARG
