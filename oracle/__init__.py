@@ -57,6 +57,10 @@ def _load():
         [c_i] * 6 + [c_d] + [c_p] * 4 + [c_i, c_i, c_p, c_i64, c_p, c_p, c_i]
     )
     lib.oracle_decode_topv.restype = c_i
+    lib.oracle_decode_topv_ex.argtypes = (
+        [c_i] * 6 + [c_d] + [c_p] * 4 + [c_i, c_i, c_i, c_p, c_i64, c_p, c_p, c_i]
+    )
+    lib.oracle_decode_topv_ex.restype = c_i
     _lib = lib
     return lib
 
@@ -170,9 +174,11 @@ def exact_dot(a, b) -> Fraction:
 
 
 def decode_topv(q, k_cache, v_cache, seq_lens, topk: int, scale: float, *, rows=None,
-                threads: int = 0):
+                threads: int = 0, full_weights: bool = False):
     """fp64 selective-V decode over the top-k exact-scoring positions per query head.
 
+    The kept V rows are weighted by the softmax renormalised over the kept set, or with
+    ``full_weights`` by the full-softmax weights alpha_j (the other positions counting as zero).
     Returns (out float64 [B, n_q, d_v], idx int32 [B, n_q, topk]) -- idx ascending,
     padded with -1 when topk exceeds the context -- or row-major [len(rows), ...].
     """
@@ -188,9 +194,9 @@ def decode_topv(q, k_cache, v_cache, seq_lens, topk: int, scale: float, *, rows=
         nr, rp = rr.shape[0], _ptr(rr)
     out = np.empty((nr, d_v), np.float64)
     idx = np.empty((nr, max(topk, 0)), np.int32)
-    rc = _load().oracle_decode_topv(B, n_q, n_k, n_v, d_k, d_v, float(scale), _ptr(qb), _ptr(kb),
-                                    _ptr(vb), _ptr(sl), t_max, topk, rp, nr, _ptr(out), _ptr(idx),
-                                    threads)
+    rc = _load().oracle_decode_topv_ex(B, n_q, n_k, n_v, d_k, d_v, float(scale), _ptr(qb), _ptr(kb),
+                                       _ptr(vb), _ptr(sl), t_max, topk, 1 if full_weights else 0, rp, nr,
+                                       _ptr(out), _ptr(idx), threads)
     _check(rc, "decode_topv")
     if rows is None:
         return out.reshape(B, n_q, d_v), idx.reshape(B, n_q, max(topk, 0))

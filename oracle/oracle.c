@@ -390,6 +390,7 @@ int oracle_exact_dot(const uint16_t *a, const uint16_t *b, int n, int64_t *digit
 typedef struct {
     decode_ctx base;
     int topk;
+    int full_weights; /* 0: renormalise over the kept set; 1: full-softmax weights alpha_j */
     int32_t *idx_out; /* [n_rows, topk], ascending, -1 padded */
 } topv_ctx;
 
@@ -443,7 +444,9 @@ static void topv_row(void *vctx, int64_t r) {
     qsort(sel, (size_t)ksel, sizeof(int), int_cmp);
     for (int e = 0; e < ksel; ++e) idx[e] = sel[e];
 
-    /* 3. softmax renormalised over the selected set, weighted V rows */
+    /* 3. weighted V rows of the selected set: the softmax renormalised over the set
+     *    ("Selective V Cache Fetching" as the workload asks), or the full-softmax
+     *    weights alpha_j of the pages' formula, the other positions counting as zero */
     double *s = (double *)malloc(sizeof(double) * (size_t)ksel);
     if (!s) { c->status = -3; free(sel); return; }
     double m = -INFINITY;
@@ -455,22 +458,40 @@ static void topv_row(void *vctx, int64_t r) {
         if (s[e] > m) m = s[e];
     }
     double den = 0.0;
+    if (tc->full_weights) {
+        /* alpha_j = exp(s_j - M) / sum over every cached position of exp(s_i - M) */
+        double *all = (double *)malloc(sizeof(double) * (size_t)T);
+        if (!all) { c->status = -3; free(s); free(sel); return; }
+        double mall = -INFINITY;
+        for (int j = 0; j < T; ++j) {
+            const uint16_t *kr = c->k + (((int64_t)b * c->t_max + j) * c->n_k + kh) * c->d_k;
+            double acc = 0.0;
+            for (int d = 0; d < c->d_k; ++d) acc += bf16_to_f64(q[d]) * bf16_to_f64(kr[d]);
+            all[j] = c->scale * acc;
+            if (all[j] > mall) mall = all[j];
+        }
+        for (int j = 0; j < T; ++j) den += exp(all[j] - mall);
+        free(all);
+        m = mall;
+    }
+    double kept = 0.0;
     for (int e = 0; e < ksel; ++e) {
         const double w = exp(s[e] - m);
-        den += w;
+        kept += w;
         const uint16_t *vr = v_row(c, b, sel[e], vh);
         for (int d = 0; d < c->d_v; ++d) o[d] += w * bf16_to_f64(vr[d]);
     }
+    if (!tc->full_weights) den = kept;
     for (int d = 0; d < c->d_v; ++d) o[d] /= den;
     free(s);
     free(sel);
 }
 
-int oracle_decode_topv(int batch, int n_q, int n_k, int n_v, int d_k, int d_v, double scale,
-                       const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
-                       const int32_t *seq_lens, int t_max, int topk,
-                       const int32_t *rows, int64_t n_rows, double *out, int32_t *idx_out,
-                       int n_threads) {
+int oracle_decode_topv_ex(int batch, int n_q, int n_k, int n_v, int d_k, int d_v, double scale,
+                          const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
+                          const int32_t *seq_lens, int t_max, int topk, int full_weights,
+                          const int32_t *rows, int64_t n_rows, double *out, int32_t *idx_out,
+                          int n_threads) {
     if (check_dims(batch, n_q, n_k, n_v, d_k, d_v) || t_max < 0 || topk < 0 || !q || !k_cache ||
         !v_cache || !seq_lens || !out || !idx_out)
         return -1;
@@ -483,7 +504,17 @@ int oracle_decode_topv(int batch, int n_q, int n_k, int n_v, int d_k, int d_v, d
                        q, k_cache, v_cache, seq_lens, rows, out, 0};
     c.base = base;
     c.topk = topk;
+    c.full_weights = full_weights ? 1 : 0;
     c.idx_out = idx_out;
     run_rows(topv_row, &c, n_rows, n_threads);
     return c.base.status;
+}
+
+int oracle_decode_topv(int batch, int n_q, int n_k, int n_v, int d_k, int d_v, double scale,
+                       const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
+                       const int32_t *seq_lens, int t_max, int topk,
+                       const int32_t *rows, int64_t n_rows, double *out, int32_t *idx_out,
+                       int n_threads) {
+    return oracle_decode_topv_ex(batch, n_q, n_k, n_v, d_k, d_v, scale, q, k_cache, v_cache, seq_lens, t_max,
+                                 topk, 0, rows, n_rows, out, idx_out, n_threads);
 }

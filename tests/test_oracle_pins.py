@@ -313,3 +313,42 @@ def test_topv_k1_is_argmax_row_and_weights_renormalise():
     d["v_cache"].fill_(1.0)
     out, _ = oracle.decode_topv(d["q"], d["k_cache"], d["v_cache"], d["seq_lens"], 9, d["scale"])
     np.testing.assert_allclose(out, 1.0, rtol=0, atol=1e-12)
+
+
+def _zeroed_v_sdpa(d, b, h, sel, shape):
+    """Full softmax over every cached position, with the V rows outside `sel` set to zero."""
+    kh, vh = h // (shape.n_q // shape.n_k), h // (shape.n_q // shape.n_v)
+    T = int(d["seq_lens"][b])
+    q = d["q"][b, h].double()[None, None, None]
+    k = d["k_cache"][b, :T, kh].double()[None, None]
+    v = d["v_cache"][b, :T, vh].double().clone()
+    keep = torch.zeros(T, dtype=torch.bool)
+    keep[list(sel)] = True
+    v[~keep] = 0.0
+    return F.scaled_dot_product_attention(q, k, v[None, None], scale=d["scale"])[0, 0, 0].numpy()
+
+
+def test_topv_full_weights_equals_full_softmax_with_other_v_rows_zeroed():
+    """The pages' formula: kept rows weighted by the full-softmax alpha_j, the rest counting as zero."""
+    s = wl.DIFFQKV
+    d = wl.random_decode_inputs(2, 90, s, seed=55, seq_lens=[90, 41])
+    k = 12
+    out, idx = oracle.decode_topv(d["q"], d["k_cache"], d["v_cache"], d["seq_lens"], k, d["scale"],
+                                  full_weights=True)
+    _, idx_renorm = oracle.decode_topv(d["q"], d["k_cache"], d["v_cache"], d["seq_lens"], k, d["scale"])
+    assert np.array_equal(idx, idx_renorm)
+    for b in range(2):
+        for h in range(s.n_q):
+            want = _brute_topk(d, b, h, k, s)
+            assert idx[b, h].tolist() == want
+            np.testing.assert_allclose(out[b, h], _zeroed_v_sdpa(d, b, h, want, s), atol=1e-12, rtol=0)
+
+
+def test_topv_full_weights_sum_to_the_kept_mass():
+    s = wl.DIFFQKV
+    d = wl.random_decode_inputs(1, 60, s, seed=56)
+    d["v_cache"].fill_(1.0)
+    out, _ = oracle.decode_topv(d["q"], d["k_cache"], d["v_cache"], d["seq_lens"], 5, d["scale"], full_weights=True)
+    assert np.all(out < 1.0) and np.all(out > 0.0)  # 5 of 60 positions: a strict part of the mass
+    out, _ = oracle.decode_topv(d["q"], d["k_cache"], d["v_cache"], d["seq_lens"], 60, d["scale"], full_weights=True)
+    np.testing.assert_allclose(out, 1.0, rtol=0, atol=1e-12)
