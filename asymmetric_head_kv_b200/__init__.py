@@ -169,9 +169,11 @@ def decode_topv_workspace(dims: Dims, t_max: int, topk: int, device="cuda") -> t
 
 def decode_topv(q, k_cache, v_cache, seq_lens, topk: int, *, scale: Optional[float] = None,
                 max_seq_len: Optional[int] = None, out=None, idx_out=None, workspace=None,
-                stream: Optional[torch.cuda.Stream] = None):
+                full_weights: bool = False, stream: Optional[torch.cuda.Stream] = None):
     """Selective-V decode over the top-k exact-scoring positions of each query head.
 
+    The kept V rows are weighted by the softmax renormalised over them, or with ``full_weights`` by
+    the full-softmax weights of every cached position (the others counting as zero).
     Returns (out bf16 [B, n_q, d_v], idx int32 [B, n_q, topk] ascending, -1 padded).
     """
     _bf16_dev(q, "q", 3)
@@ -187,9 +189,15 @@ def decode_topv(q, k_cache, v_cache, seq_lens, topk: int, *, scale: Optional[flo
     if workspace is None:
         workspace = decode_topv_workspace(dims, t_max, topk, q.device)
     msl = t_max if max_seq_len is None else int(max_seq_len)
-    st = lib().diffqkv_decode_topv(ctypes.byref(dims), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seq_lens),
-                                   t_max, msl, topk, _ptr(out), _ptr(idx_out), _ptr(workspace), workspace.numel(),
-                                   _stream_ptr(stream))
+    if full_weights:
+        st = lib().diffqkv_decode_topv_ex(ctypes.byref(dims), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                          _ptr(seq_lens), t_max, msl, topk, _capi.TOPV_FULL_SOFTMAX_WEIGHTS,
+                                          _ptr(out), _ptr(idx_out), _ptr(workspace), workspace.numel(),
+                                          _stream_ptr(stream))
+    else:
+        st = lib().diffqkv_decode_topv(ctypes.byref(dims), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seq_lens),
+                                       t_max, msl, topk, _ptr(out), _ptr(idx_out), _ptr(workspace),
+                                       workspace.numel(), _stream_ptr(stream))
     check(st, "diffqkv_decode_topv")
     return out, idx_out
 

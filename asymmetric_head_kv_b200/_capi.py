@@ -27,6 +27,7 @@ STATUS = {
 }
 (OK, INVALID_ARG, UNSUPPORTED, MISALIGNED, WORKSPACE, CUDA_ERR, DEVICE_TIMEOUT, DEVICE_SEQLEN, NO_DEVICE,
  SCRATCH_LIMIT) = range(10)
+TOPV_FULL_SOFTMAX_WEIGHTS = 1  # flag of diffqkv_decode_topv_ex (include/diffqkv.h)
 
 
 class Dims(ctypes.Structure):
@@ -84,6 +85,7 @@ SIGNATURES = {
     "diffqkv_decode_from_host": ([_DIMS, _P, _P, _P, _P, _I32, _I32, _P, _P, _P, _P, _P, _P, _P, _SZ, _P], _I32),
     "diffqkv_decode_topv_workspace_size": ([_DIMS, _I32, _I32], _SZ),
     "diffqkv_decode_topv": ([_DIMS, _P, _P, _P, _P, _I32, _I32, _I32, _P, _P, _P, _SZ, _P], _I32),
+    "diffqkv_decode_topv_ex": ([_DIMS, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _P, _P, _P, _SZ, _P], _I32),
     "diffqkv_prefill_causal": ([_DIMS, _P, _P, _P, _I32, _P, _P], _I32),
     "diffqkv_get_device_status": ([_P, ctypes.POINTER(_I32)], _I32),
     "diffqkv_selftest_wait_timeout": ([_I64, _P], _I32),

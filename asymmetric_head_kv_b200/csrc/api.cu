@@ -275,6 +275,15 @@ diffqkv_status_t diffqkv_decode_topv(const diffqkv_dims_t *dims, const void *q, 
                                 workspace, workspace_bytes, (cudaStream_t)stream);
 }
 
+diffqkv_status_t diffqkv_decode_topv_ex(const diffqkv_dims_t *dims, const void *q, const void *k_cache,
+                                        const void *v_cache, const int32_t *seq_lens, int32_t t_max,
+                                        int32_t max_seq_len, int32_t topk, int32_t flags, void *out,
+                                        int32_t *idx_out, void *workspace, size_t workspace_bytes,
+                                        diffqkv_stream_t stream) {
+    return diffqkv::topv_launch(dims, q, k_cache, v_cache, seq_lens, t_max, max_seq_len, topk, out, idx_out,
+                                workspace, workspace_bytes, (cudaStream_t)stream, flags);
+}
+
 diffqkv_status_t diffqkv_prefill_causal(const diffqkv_dims_t *dims, const void *q, const void *k, const void *v,
                                         int32_t seq_len, void *out, diffqkv_stream_t stream) {
     return diffqkv::prefill_launch(dims, q, k, v, seq_len, out, (cudaStream_t)stream);

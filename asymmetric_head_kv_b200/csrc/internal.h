@@ -64,7 +64,7 @@ size_t topv_workspace_size(const diffqkv_dims_t *d, int32_t t_max, int32_t topk)
 diffqkv_status_t topv_launch(const diffqkv_dims_t *d, const void *q, const void *k_cache, const void *v_cache,
                              const int32_t *seq_lens, int32_t t_max, int32_t max_seq_len, int32_t topk,
                              void *out, int32_t *idx_out, void *workspace, size_t workspace_bytes,
-                             cudaStream_t stream);
+                             cudaStream_t stream, int32_t flags = 0);
 
 // prefill.cu
 diffqkv_status_t prefill_launch(const diffqkv_dims_t *d, const void *q, const void *k, const void *v,

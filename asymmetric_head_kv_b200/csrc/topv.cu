@@ -49,6 +49,8 @@ constexpr int kScoreTile = 128;         // positions per TMA tile (one per consu
 constexpr int kHistBuckets = 2048;      // first radix digit: top 11 bits of the order key
 constexpr int kHistWords = kHistBuckets / 2;  // score-kernel histogram: two 16-bit counters per word
 constexpr int kScoreMaxTilesPerCta = 511;     // keeps a CTA's positions (and any counter) below 2^16
+// Score CTAs per SM: three for d_k = 64; with d_k = 128 the q registers of four heads need two.
+constexpr int score_ctas_per_sm(int dk) { return dk == 64 ? 3 : 2; }
 constexpr int kRadixBuckets = 256;      // later radix digits: one byte
 constexpr int kFilterThreads = 256;
 constexpr int kFilterChunk = 8192;      // positions per filter CTA (32 per thread)
@@ -60,7 +62,8 @@ constexpr int kTopvHeader = 256;
 constexpr int kCandCap = 12288;         // candidates held in shared memory by the select kernel
 constexpr int kTopvMaxContext = 131072; // bitmap of kept positions: 16 KB of shared memory
 constexpr int kRowInfoWords = 8;       // per-row words handed from kernel to kernel
-enum RowInfo { kRiBucket = 0, kRiAbove = 1, kRiTwoDelta = 2, kRiMax = 3, kRiKept = 4 };
+enum RowInfo { kRiBucket = 0, kRiAbove = 1, kRiTwoDelta = 2, kRiMax = 3, kRiKept = 4, kRiFullSum = 5 };
+constexpr int kMaxFilterChunks = kTopvMaxContext / kFilterChunk;
 constexpr int kGatherThreads = 256;
 constexpr int kGatherWarps = kGatherThreads / 32;
 constexpr int kGatherRows = 128;        // kept V rows per gather CTA and round
@@ -87,6 +90,8 @@ struct TopvArgs {
     int32_t *status;
     int32_t batch, n_q, n_k, n_v, t_max, t_pad, topk, q_per_k, q_per_v;
     int32_t score_stages;
+    int32_t full_weights;  // 1: weight the kept rows by the full-softmax alpha_j (no renormalisation)
+    float2 *fpart;         // [B*n_q][kMaxFilterChunks] (max score, sum of 2^((s - max) scale log2 e)) per filter chunk
     float scale_log2;
     uint64_t wait_limit_ns;
 };
@@ -176,7 +181,7 @@ __device__ __forceinline__ int head_of_lane(int r) { return HG == 4 ? r : (HG ==
 // elements of q for up to four query heads in registers.  The four partial dot
 // products of each head are added across the group, and lane r writes head r.
 template <int DK, int QPK>
-__global__ void __launch_bounds__(kScoreThreads + 32, 3) topv_score_kernel(const __grid_constant__ CUtensorMap tm_k,
+__global__ void __launch_bounds__(kScoreThreads + 32, score_ctas_per_sm(DK)) topv_score_kernel(const __grid_constant__ CUtensorMap tm_k,
                                                                          const TopvArgs a) {
     constexpr int KB = DK / 64;  // 64-wide swizzle blocks per row
     constexpr int TILE_BYTES = kScoreTile * DK * 2;
@@ -557,6 +562,45 @@ __global__ void __launch_bounds__(kFilterThreads, 4) topv_filter_kernel(const To
     }
     const uint32_t kmax_bits = __ldcg(a.kmax + b * a.n_k + g);
 
+    if (a.full_weights) {
+        // this chunk's share of the full softmax denominator: its max and its sum of exponentials
+        float mx = -INFINITY;
+#pragma unroll
+        for (int u = 0; u < kVec; ++u) {
+            const int p = j_begin + (u * kFilterThreads + tid) * 4;
+            const float x[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                if (p + e < j_end) mx = fmaxf(mx, x[e]);
+        }
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        if (lane == 0) red[tid >> 5] = mx;
+        __syncthreads();
+        mx = red[0];
+        for (int w2 = 1; w2 < kFilterThreads / 32; ++w2) mx = fmaxf(mx, red[w2]);
+        __syncthreads();
+        float sum = 0.f;
+#pragma unroll
+        for (int u = 0; u < kVec; ++u) {
+            const int p = j_begin + (u * kFilterThreads + tid) * 4;
+            const float x[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                if (p + e < j_end) sum += fast_exp2((x[e] - mx) * a.scale_log2);
+        }
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+        if (lane == 0) red[tid >> 5] = sum;
+        __syncthreads();
+        if (tid == 0) {
+            float tot = 0.f;
+            for (int w2 = 0; w2 < kFilterThreads / 32; ++w2) tot += red[w2];
+            a.fpart[(size_t)row * kMaxFilterChunks + blockIdx.y] = make_float2(mx, tot);
+        }
+        __syncthreads();
+    }
+
     // bucket of the k-th largest score, and the lower end of the range that can be kept
     {
         const uint4 *src = reinterpret_cast<const uint4 *>(a.ghist + (size_t)row * kHistBuckets);
@@ -653,6 +697,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) topv_select_kernel(const TopvA
         if (tid == 0) {
             a.rowinfo[kRowInfoWords * row + kRiMax] = __float_as_uint(0.f);
             a.rowinfo[kRowInfoWords * row + kRiKept] = 0u;
+            a.rowinfo[kRowInfoWords * row + kRiFullSum] = 0u;
         }
         return;
     }
@@ -851,8 +896,21 @@ __global__ void __launch_bounds__(kSelThreads, 1) topv_select_kernel(const TopvA
     if (tid == 0) {
         float m = red_s[0];
         for (int w = 1; w < kSelWarps; ++w) m = fmaxf(m, red_s[w]);
+        float full_sum = 0.f;  // 0: renormalise over the kept set
+        if (a.full_weights && T > K) {
+            // the full softmax denominator from the filter's chunk partials, relative to the row max
+            const int nch = (T + kFilterChunk - 1) / kFilterChunk;
+            float M = -INFINITY;
+            for (int ch = 0; ch < nch; ++ch) M = fmaxf(M, __ldcg(&a.fpart[(size_t)row * kMaxFilterChunks + ch].x));
+            for (int ch = 0; ch < nch; ++ch) {
+                const float2 pc = __ldcg(&a.fpart[(size_t)row * kMaxFilterChunks + ch]);
+                full_sum += pc.y * fast_exp2((pc.x - M) * a.scale_log2);
+            }
+            m = M;
+        }
         a.rowinfo[kRowInfoWords * row + kRiMax] = __float_as_uint(m);
         a.rowinfo[kRowInfoWords * row + kRiKept] = (uint32_t)nsel;
+        a.rowinfo[kRowInfoWords * row + kRiFullSum] = __float_as_uint(full_sum);
     }
 }
 
@@ -943,6 +1001,9 @@ __global__ void __launch_bounds__(kGatherThreads) topv_gather_kernel(const TopvA
         const uint32_t base = smem_addr(part_s);
         float lt = 0.f;
         for (int p = 0; p < nparts; ++p) lt += ld_dsmem_f32(base + DV * 4u, (uint32_t)p);
+        // full-softmax weights: divide by the sum over every cached position instead
+        const float full_sum = __uint_as_float(__ldcg(a.rowinfo + kRowInfoWords * row + kRiFullSum));
+        if (full_sum > 0.f) lt = full_sum;
         for (int c = tid; c < DV; c += kGatherThreads) {
             float acc = 0.f;
             for (int p = 0; p < nparts; ++p) acc += ld_dsmem_f32(base + (uint32_t)c * 4u, (uint32_t)p);
@@ -1009,8 +1070,11 @@ size_t zeroed_bytes(const diffqkv_dims_t *d) {
 // Gather CTAs per row (one cluster): a round of kGatherRows kept rows each, at most kGatherMaxSplit.
 int gather_split(int32_t topk) { return std::max(1, std::min(kGatherMaxSplit, (topk + kGatherRows - 1) / kGatherRows)); }
 
-// rowinfo [rows][kRowInfoWords]
-size_t row_bytes(const diffqkv_dims_t *d) { return align_up((size_t)d->batch * d->n_q * kRowInfoWords * 4, 256); }
+// rowinfo [rows][kRowInfoWords], then the filter's softmax partials [rows][kMaxFilterChunks]
+size_t rowinfo_bytes(const diffqkv_dims_t *d) { return align_up((size_t)d->batch * d->n_q * kRowInfoWords * 4, 256); }
+size_t row_bytes(const diffqkv_dims_t *d) {
+    return rowinfo_bytes(d) + align_up((size_t)d->batch * d->n_q * kMaxFilterChunks * sizeof(float2), 256);
+}
 
 // Launch after the previous kernel of the stream with programmatic dependent launch;
 // cluster_y > 1 groups that many consecutive CTAs along y into one cluster.
@@ -1049,12 +1113,14 @@ size_t topv_workspace_size(const diffqkv_dims_t *d, int32_t t_max, int32_t topk)
 
 diffqkv_status_t topv_launch(const diffqkv_dims_t *d, const void *q, const void *k_cache, const void *v_cache,
                              const int32_t *seq_lens, int32_t t_max, int32_t max_seq_len, int32_t topk, void *out,
-                             int32_t *idx_out, void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+                             int32_t *idx_out, void *workspace, size_t workspace_bytes, cudaStream_t stream,
+                             int32_t flags) {
     diffqkv_status_t st = validate_dims(d);
     if (st != DIFFQKV_OK) return st;
     if (!q || !k_cache || !v_cache || !seq_lens || !out || !idx_out || t_max < 1 || topk < 1)
         return DIFFQKV_ERR_INVALID_ARG;
     if (t_max > kTopvMaxContext) return DIFFQKV_ERR_UNSUPPORTED;
+    if (flags & ~DIFFQKV_TOPV_FULL_SOFTMAX_WEIGHTS) return DIFFQKV_ERR_INVALID_ARG;
     const int qpk = d->n_q / d->n_k;
     ScoreFn score = pick_score(d->d_k, qpk);
     RowFn filter = pick_filter(d->d_k);
@@ -1080,6 +1146,8 @@ diffqkv_status_t topv_launch(const diffqkv_dims_t *d, const void *q, const void 
     a.ncand = a.ghist + rows * kHistBuckets;
     ws += align_up(zeroed_bytes(d), 256);
     a.rowinfo = reinterpret_cast<uint32_t *>(ws);
+    a.fpart = reinterpret_cast<float2 *>(ws + rowinfo_bytes(d));
+    a.full_weights = (flags & DIFFQKV_TOPV_FULL_SOFTMAX_WEIGHTS) ? 1 : 0;
     ws += row_bytes(d);
     a.scores = reinterpret_cast<float *>(ws);
     ws += align_up(rows * t_pad * 4, 256);
@@ -1123,13 +1191,14 @@ diffqkv_status_t topv_launch(const diffqkv_dims_t *d, const void *q, const void 
     if (st != DIFFQKV_OK) return st;
     const int tile_bytes = kScoreTile * d->d_k * 2;
     const int fixed = qpk * kHistWords * 4 + qpk * d->d_k * 4 + 16 * 8 + 16 + 1024;
-    // the deepest ring (2..8 tiles) that still lets three CTAs share an SM (228 KB, 1 KB reserved per
-    // CTA): occupancy hides more of the consumers' latency than a deeper ring does
+    // the deepest ring (2..8 tiles) that still lets score_ctas_per_sm CTAs share an SM (228 KB, 1 KB
+    // reserved per CTA): occupancy hides more of the consumers' latency than a deeper ring does
+    const int want = score_ctas_per_sm(d->d_k);
     int stages = 8;
-    while (stages > 2 && 3 * (stages * tile_bytes + fixed + 1024) > 228 * 1024) --stages;
+    while (stages > 2 && want * (stages * tile_bytes + fixed + 1024) > 228 * 1024) --stages;
     a.score_stages = stages;
     const int score_smem = stages * tile_bytes + fixed;
-    const int per_sm = std::max(1, std::min(3, (228 * 1024) / (score_smem + 1024)));
+    const int per_sm = std::max(1, std::min(want, (228 * 1024) / (score_smem + 1024)));
     const int units = d->batch * d->n_k;
     const int ntiles = (t_max + kScoreTile - 1) / kScoreTile;
     const int ygrid = std::max({1, (dev.num_sms * per_sm) / units,

@@ -425,6 +425,15 @@ def time_paths(ak, peaks, steps: int, warmup: int):
     res[w.name] = {"us": ms * 1e3, "algorithmic_bytes": nbytes, "gbs": nbytes / (ms * 1e-3) / 1e9,
                    "bound": "hbm", "peak_gbs": hbm, "frac": nbytes / (ms * 1e-3) / 1e9 / hbm,
                    "launches_per_call": 4}
+    # the same selection with the pages' full-softmax weights (no renormalisation over the kept set)
+    fn = lambda: ak.decode_topv(d["q"], d["k_cache"], d["v_cache"], d["seq_lens"], w.topk,  # noqa: E731
+                                scale=d["scale"], workspace=ws, full_weights=True)
+    for _ in range(max(3, warmup)):
+        fn()
+    ms = statistics.median(_timed_calls(fn, steps, flush))
+    res[w.name + "_full_weights"] = {"us": ms * 1e3, "algorithmic_bytes": nbytes,
+                                     "gbs": nbytes / (ms * 1e-3) / 1e9, "bound": "hbm", "peak_gbs": hbm,
+                                     "frac": nbytes / (ms * 1e-3) / 1e9 / hbm, "launches_per_call": 4}
     assert ak.device_status() == 0
     return res
 

@@ -218,6 +218,25 @@ diffqkv_status_t diffqkv_decode_topv(const diffqkv_dims_t *dims, const void *q, 
                                      int32_t *idx_out, void *workspace, size_t workspace_bytes,
                                      diffqkv_stream_t stream);
 
+/* Flags of diffqkv_decode_topv_ex. */
+#define DIFFQKV_TOPV_FULL_SOFTMAX_WEIGHTS 1 /* weight the kept V rows by the full-softmax
+                                               alpha_j of every cached position (the pages'
+                                               formula: the others count as zero) instead of
+                                               renormalising over the kept set */
+
+/*
+ * diffqkv_decode_topv with flags (0 = diffqkv_decode_topv).  With
+ * DIFFQKV_TOPV_FULL_SOFTMAX_WEIGHTS:
+ *   out[b,h] = sum_{j in S} e^{s_j - M} v[b,j,vh] / sum_{j < seq_lens[b]} e^{s_j - M},
+ *   M = max over every cached position; S and idx_out are unchanged.
+ * Other bits: DIFFQKV_ERR_INVALID_ARG.  Same workspace as diffqkv_decode_topv.
+ */
+diffqkv_status_t diffqkv_decode_topv_ex(const diffqkv_dims_t *dims, const void *q, const void *k_cache,
+                                        const void *v_cache, const int32_t *seq_lens, int32_t t_max,
+                                        int32_t max_seq_len, int32_t topk, int32_t flags, void *out,
+                                        int32_t *idx_out, void *workspace, size_t workspace_bytes,
+                                        diffqkv_stream_t stream);
+
 /* ------------------------------------------------------------------------ */
 /* Causal prefill (the "prefix" phase the paper's efficiency study times)    */
 /* ------------------------------------------------------------------------ */

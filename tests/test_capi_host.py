@@ -154,3 +154,10 @@ def test_decode_append_rejects_before_launch():
     assert call(vn=None) == _capi.INVALID_ARG
     assert call(kn=0x8008) == _capi.MISALIGNED
     assert call(q=None) == _capi.INVALID_ARG
+
+
+def test_topv_ex_rejects_unknown_flags():
+    d = dims()
+    st = _capi.lib().diffqkv_decode_topv_ex(ctypes.byref(d), 0x1000, 0x2000, 0x3000, 0x4000, 128, 128, 4, 2,
+                                             0x5000, 0x7000, 0x6000, 1 << 34, None)
+    assert st == _capi.INVALID_ARG

@@ -140,3 +140,19 @@ def test_workspace_reuse_is_bitwise_stable(cuda_device, topk):
     r_out, r_idx = oracle.decode_topv(d["q"], d["k_cache"], d["v_cache"], d["seq_lens"], topk, d["scale"])
     assert np.array_equal(runs[0][1].cpu().numpy(), r_idx)
     assert_parity(runs[0][0], r_out, f"reuse k={topk}")
+
+
+@pytest.mark.parametrize("name,shape,topk", [("diffqkv", wl.DIFFQKV, 100), ("diffqkv_k1", wl.DIFFQKV, 1),
+                                             ("gqa", wl.GQA_CONTROL, 64), ("mha64", Shape(8, 8, 8, 64, 64), 300)])
+def test_full_softmax_weights(cuda_device, name, shape, topk):
+    """The pages' formula: kept rows weighted by the full-softmax alpha_j of every cached position
+    (rows of 9000 positions span two filter chunks; a 200-position row keeps everything)."""
+    lens = [9000, 200, 0, 4100]
+    d = wl.random_decode_inputs(len(lens), 9000, shape, seed=309, seq_lens=lens)
+    out, idx = _gpu(d, topk, cuda_device, full_weights=True)
+    r_out, r_idx = oracle.decode_topv(d["q"], d["k_cache"], d["v_cache"], d["seq_lens"], topk, d["scale"],
+                                      full_weights=True)
+    assert np.array_equal(idx.cpu().numpy(), r_idx), f"{name}: index sets"
+    assert_parity(out, r_out, f"full weights {name}")
+    _, idx_renorm = _gpu(d, topk, cuda_device)
+    assert torch.equal(idx, idx_renorm)  # the selection does not depend on the weighting
