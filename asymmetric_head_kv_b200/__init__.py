@@ -221,6 +221,27 @@ def prefill_causal(q, k, v, *, scale: Optional[float] = None, out=None,
     return out
 
 
+def prefill_causal_prefix(q, k, v, prefix_len: int, *, scale: Optional[float] = None, out=None,
+                          stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Causal prefill over an existing prefix: q [B,S,n_q,d_k] for positions prefix_len..prefix_len+S-1,
+    k [B,P+S,n_k,d_k] and v [B,P+S,n_v,d_v] holding the prefix and the new rows -> out [B,S,n_q,d_v]."""
+    _bf16_dev(q, "q", 4)
+    _bf16_dev(k, "k", 4)
+    _bf16_dev(v, "v", 4)
+    B, S, n_q, d_k = q.shape
+    n_k, n_v, d_v = k.shape[2], v.shape[2], v.shape[3]
+    P = int(prefix_len)
+    if k.shape != (B, P + S, n_k, d_k) or v.shape[:2] != (B, P + S):
+        raise ValueError("k / v must hold prefix_len + S positions")
+    dims = make_dims(B, n_q, n_k, n_v, d_k, d_v, d_k ** -0.5 if scale is None else scale)
+    if out is None:
+        out = torch.empty((B, S, n_q, d_v), dtype=torch.bfloat16, device=q.device)
+    st = lib().diffqkv_prefill_causal_prefix(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), P, S, _ptr(out),
+                                             _stream_ptr(stream))
+    check(st, "diffqkv_prefill_causal_prefix")
+    return out
+
+
 def device_status(stream: Optional[torch.cuda.Stream] = None) -> int:
     """Synchronises the stream and returns (and clears) the device error word."""
     v = ctypes.c_int32(0)

@@ -289,6 +289,12 @@ diffqkv_status_t diffqkv_prefill_causal(const diffqkv_dims_t *dims, const void *
     return diffqkv::prefill_launch(dims, q, k, v, seq_len, out, (cudaStream_t)stream);
 }
 
+diffqkv_status_t diffqkv_prefill_causal_prefix(const diffqkv_dims_t *dims, const void *q, const void *k,
+                                               const void *v, int32_t prefix_len, int32_t seq_len, void *out,
+                                               diffqkv_stream_t stream) {
+    return diffqkv::prefill_launch(dims, q, k, v, seq_len, out, (cudaStream_t)stream, prefix_len);
+}
+
 diffqkv_status_t diffqkv_get_device_status(diffqkv_stream_t stream, int32_t *device_status) {
     if (!device_status) return DIFFQKV_ERR_INVALID_ARG;
     diffqkv::DeviceInfo dev;

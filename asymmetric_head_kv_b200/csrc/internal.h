@@ -68,7 +68,7 @@ diffqkv_status_t topv_launch(const diffqkv_dims_t *d, const void *q, const void 
 
 // prefill.cu
 diffqkv_status_t prefill_launch(const diffqkv_dims_t *d, const void *q, const void *k, const void *v,
-                                int32_t seq_len, void *out, cudaStream_t stream);
+                                int32_t seq_len, void *out, cudaStream_t stream, int32_t prefix_len = 0);
 
 // api.cu
 diffqkv_status_t wait_timeout_selftest_launch(int64_t timeout_ns, cudaStream_t stream);

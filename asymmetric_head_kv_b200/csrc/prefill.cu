@@ -38,6 +38,8 @@ struct PrefillArgs {
     __nv_bfloat16 *out;
     int32_t *status;
     int32_t batch, seq, n_q, n_k, n_v, q_per_k, q_per_v, n_ctas_per_head;
+    int32_t prefix;  // cached positions before the first query row (query row r sits at position prefix + r)
+    int32_t kv_len;  // prefix + seq: positions in K and V
     float scale_log2;
     uint64_t wait_limit_ns;
 };
@@ -100,9 +102,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int h = bh % a.n_q;
     const int kh = h / a.q_per_k;
     const int vh = h / a.q_per_v;
-    const int row0 = qt * BM;
-    const int kv_tiles_total = (a.seq + BN - 1) / BN;
-    const int n_kv = min(kv_tiles_total, (row0 + BM + BN - 1) / BN);
+    const int row0 = qt * BM;               // first query row of the tile (Q and out rows)
+    const int pos0 = a.prefix + row0;       // its position among the keys
+    const int kv_tiles_total = (a.kv_len + BN - 1) / BN;
+    const int n_kv = min(kv_tiles_total, (pos0 + BM + BN - 1) / BN);
 
     if (tid == 0) {
         for (int s = 0; s < C::STAGES; ++s) {
@@ -211,7 +214,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     } else {
         // ======================= softmax warps 0-3: thread tid owns query row row0 + tid
         const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-        const int i = row0 + tid;  // query position of this thread's row
+        const int i = pos0 + tid;     // key position of this thread's query row
+        const int qrow = row0 + tid;  // its row in q and out
         float m_used = -INFINITY;  // log2-domain maximum the stored O and l are relative to
         float l = 0.f;
         for (int n = 0; n < n_kv; ++n) {
@@ -234,7 +238,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 
             // causal mask on tiles that reach past this row
             const int j0 = n * BN;
-            if (j0 + BN - 1 > row0) {
+            if (j0 + BN - 1 > pos0) {
 #pragma unroll
                 for (int c = 0; c < BN; ++c)
                     if (j0 + c > i) s[c] = -INFINITY;
@@ -307,13 +311,13 @@ __global__ void __launch_bounds__(kThreads, 2)
         mbar_wait_bounded(pv_done, (uint32_t)((n_kv - 1) & 1), a.wait_limit_ns, abort_flag, a.status);
         tc_fence_after();
         const float inv_l = l > 0.f ? 1.f / l : 0.f;
-        __nv_bfloat16 *orow = a.out + (((size_t)b * a.seq + i) * a.n_q + h) * DV;
+        __nv_bfloat16 *orow = a.out + (((size_t)b * a.seq + qrow) * a.n_q + h) * DV;
 #pragma unroll 1
         for (int c = 0; c < DV; c += 32) {
             uint32_t r[32];
             tmem_ld32(t_o + lane_base + c, r);
             tmem_wait_ld();
-            if (i < a.seq) {
+            if (qrow < a.seq) {
 #pragma unroll
                 for (int e = 0; e < 32; e += 8) {
                     uint4 v;
@@ -402,11 +406,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int h = bh % a.n_q;
     const int kh = h / a.q_per_k;
     const int vh = h / a.q_per_v;
-    const int row0 = qp * QT * BM;
-    const int kv_tiles_total = (a.seq + BN - 1) / BN;
+    const int row0 = qp * QT * BM;          // first query row of the pair (Q and out rows)
+    const int pos0 = a.prefix + row0;       // its position among the keys
+    const int kv_tiles_total = (a.kv_len + BN - 1) / BN;
     int n_kv[QT];
 #pragma unroll
-    for (int t = 0; t < QT; ++t) n_kv[t] = min(kv_tiles_total, (row0 + (t + 1) * BM + BN - 1) / BN);
+    for (int t = 0; t < QT; ++t) n_kv[t] = min(kv_tiles_total, (pos0 + (t + 1) * BM + BN - 1) / BN);
     const int n_kv_all = n_kv[QT - 1];
 
     if (tid == 0) {
@@ -528,8 +533,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
         const uint32_t t_s = tmem + (uint32_t)(t * BN) + lane_base;
         const uint32_t t_o = tmem + C::T_O + (uint32_t)(t * DV) + lane_base;
-        const int tile_row0 = row0 + t * BM;
-        const int i = tile_row0 + r;  // query position of this thread's row
+        const int tile_row0 = pos0 + t * BM;  // key position of the tile's first query row
+        const int i = tile_row0 + r;          // key position of this thread's query row
+        const int qrow = row0 + t * BM + r;   // its row in q and out
         const int nk = n_kv[t];
         float m_used = -INFINITY;     // log2-domain maximum the stored O and l are relative to
         float l = 0.f;
@@ -625,13 +631,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_wait_bounded(&pv_done[t], (uint32_t)((nk - 1) & 1), a.wait_limit_ns, abort_flag, a.status);
             tc_fence_after();
             const float inv_l = l > 0.f ? 1.f / l : 0.f;
-            __nv_bfloat16 *orow = a.out + (((size_t)b * a.seq + i) * a.n_q + h) * DV;
+            __nv_bfloat16 *orow = a.out + (((size_t)b * a.seq + qrow) * a.n_q + h) * DV;
 #pragma unroll 1
             for (int c = 0; c < DV; c += 32) {
                 uint32_t rr[32];
                 tmem_ld32(t_o + (uint32_t)c, rr);
                 tmem_wait_ld();
-                if (i < a.seq) {
+                if (qrow < a.seq) {
 #pragma unroll
                     for (int e = 0; e < 32; e += 8) {
                         uint4 v;
@@ -686,10 +692,12 @@ bool pick(int dk, int dv, Plan *p) {
 }  // namespace
 
 diffqkv_status_t prefill_launch(const diffqkv_dims_t *d, const void *q, const void *k, const void *v, int32_t seq_len,
-                                void *out, cudaStream_t stream) {
+                                void *out, cudaStream_t stream, int32_t prefix_len) {
     diffqkv_status_t st = validate_dims(d);
     if (st != DIFFQKV_OK) return st;
-    if (!q || !k || !v || !out || seq_len < 1) return DIFFQKV_ERR_INVALID_ARG;
+    if (!q || !k || !v || !out || seq_len < 1 || prefix_len < 0) return DIFFQKV_ERR_INVALID_ARG;
+    if ((long long)prefix_len + seq_len > 0x7fffffffLL) return DIFFQKV_ERR_UNSUPPORTED;
+    const int32_t kv_len = prefix_len + seq_len;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return DIFFQKV_ERR_MISALIGNED;
     Plan plan;
     if (!pick(d->d_k, d->d_v, &plan)) return DIFFQKV_ERR_UNSUPPORTED;
@@ -701,10 +709,10 @@ diffqkv_status_t prefill_launch(const diffqkv_dims_t *d, const void *q, const vo
     st = make_tensor_map_4d(&tm_q, q, d->d_k, d->n_q, seq_len, d->batch, 64, 1, plan.q_box, 1,
                             CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != DIFFQKV_OK) return st;
-    st = make_tensor_map_4d(&tm_k, k, d->d_k, d->n_k, seq_len, d->batch, 64, 1, plan.kv_box, 1,
+    st = make_tensor_map_4d(&tm_k, k, d->d_k, d->n_k, kv_len, d->batch, 64, 1, plan.kv_box, 1,
                             CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != DIFFQKV_OK) return st;
-    st = make_tensor_map_4d(&tm_v, v, d->d_v, d->n_v, seq_len, d->batch, 64, 1, plan.kv_box, 1,
+    st = make_tensor_map_4d(&tm_v, v, d->d_v, d->n_v, kv_len, d->batch, 64, 1, plan.kv_box, 1,
                             CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != DIFFQKV_OK) return st;
 
@@ -713,6 +721,8 @@ diffqkv_status_t prefill_launch(const diffqkv_dims_t *d, const void *q, const vo
     a.status = dev.status_word;
     a.batch = d->batch;
     a.seq = seq_len;
+    a.prefix = prefix_len;
+    a.kv_len = kv_len;
     a.n_q = d->n_q;
     a.n_k = d->n_k;
     a.n_v = d->n_v;

@@ -372,6 +372,22 @@ def time_paths(ak, peaks, steps: int, warmup: int):
         res[w.name] = {"ms": ms, "causal_flops": flops, "tflops": tf, "bound": "tensor", "peak_tflops": bf16_peak,
                        "frac": tf / bf16_peak, "peak_source": "bf16_tflops (burst, cuBLAS bf16 GEMM)"}
         del d, out
+    # chunked prefill: 2048 new rows over an 8192-position prefix (batch 2, DiffQKV shape)
+    P, S, w = 8192, 2048, wl.PREFILL_8K
+    d = wl.random_prefill_inputs(w.batch, P + S, w.shape, seed=w.seed, device=dev)
+    qn = d["q"][:, P:].contiguous()
+    out = torch.empty((w.batch, S, w.shape.n_q, w.shape.d_v), dtype=torch.bfloat16, device=dev)
+    fn = lambda: ak.prefill_causal_prefix(qn, d["k"], d["v"], P, scale=d["scale"], out=out)  # noqa: E731
+    for _ in range(max(3, warmup)):
+        fn()
+    ms = statistics.median(_timed_calls(fn, steps, flush))
+    flops = 2 * w.batch * w.shape.n_q * (S * P + S * (S + 1) // 2) * (w.shape.d_k + w.shape.d_v)
+    tf = flops / (ms * 1e-3) / 1e12
+    res["prefill_prefix_b2_p8192_s2048"] = {"ms": ms, "causal_flops": flops, "tflops": tf, "bound": "tensor",
+                                            "peak_tflops": bf16_peak, "frac": tf / bf16_peak,
+                                            "peak_source": "bf16_tflops (burst, cuBLAS bf16 GEMM)"}
+    del d, qn, out
+
     # the small decode case (batch 1, 512 positions: 2.36 MB, launch/latency bound): microseconds
     # per call with L2 flushed before each call
     w = wl.DECODE_SMALL

@@ -252,6 +252,21 @@ diffqkv_status_t diffqkv_prefill_causal(const diffqkv_dims_t *dims, const void *
                                         const void *v, int32_t seq_len, void *out,
                                         diffqkv_stream_t stream);
 
+/*
+ * Causal prefill over an existing prefix (chunked prefill): the seq_len query
+ * rows sit at positions prefix_len .. prefix_len + seq_len - 1 of a sequence
+ * whose first prefix_len positions are already in k and v.
+ *   q   [B, seq_len, n_q, d_k]                 the new rows' queries
+ *   k   [B, prefix_len + seq_len, n_k, d_k]    prefix and new keys
+ *   v   [B, prefix_len + seq_len, n_v, d_v]
+ *   out [B, seq_len, n_q, d_v]
+ * out[b,r,h] = sum_{j <= prefix_len + r} softmax_j(scale q[b,r,h].k[b,j,kh]) v[b,j,vh].
+ * prefix_len >= 0 (0 is diffqkv_prefill_causal); other rules as there.
+ */
+diffqkv_status_t diffqkv_prefill_causal_prefix(const diffqkv_dims_t *dims, const void *q, const void *k,
+                                               const void *v, int32_t prefix_len, int32_t seq_len, void *out,
+                                               diffqkv_stream_t stream);
+
 /* ------------------------------------------------------------------------ */
 /* Device error word                                                        */
 /* ------------------------------------------------------------------------ */

@@ -161,3 +161,9 @@ def test_topv_ex_rejects_unknown_flags():
     st = _capi.lib().diffqkv_decode_topv_ex(ctypes.byref(d), 0x1000, 0x2000, 0x3000, 0x4000, 128, 128, 4, 2,
                                              0x5000, 0x7000, 0x6000, 1 << 34, None)
     assert st == _capi.INVALID_ARG
+
+
+def test_prefill_prefix_rejects_negative_prefix():
+    d = dims()
+    st = _capi.lib().diffqkv_prefill_causal_prefix(ctypes.byref(d), 0x1000, 0x2000, 0x3000, -1, 16, 0x5000, None)
+    assert st == _capi.INVALID_ARG

@@ -110,3 +110,43 @@ def test_full_prefill_sampled_rows(cuda_device, w):
     idx = torch.tensor(rows)
     got = out[idx[:, 0], idx[:, 1], idx[:, 2]]
     assert_parity(got, ref, w.name)
+
+
+def _prefix_expected(q, k, v, scale, P):
+    """Rows P.. of a causal prefill over the whole P+S sequence (rows are independent, so the
+    prefix rows' queries can be anything: zeros here)."""
+    B, S, n_q, d_k = q.shape
+    q_full = torch.cat([torch.zeros(B, P, n_q, d_k, dtype=q.dtype), q], dim=1)
+    return oracle.prefill_causal(q_full, k, v, scale)[:, P:]
+
+
+@pytest.mark.parametrize("shape_name", ["diffqkv", "gqa_control"])
+@pytest.mark.parametrize("P,S", [(1, 5), (64, 130), (100, 257), (128, 1), (300, 300)])
+def test_prefix_prefill(cuda_device, shape_name, P, S):
+    """Chunked prefill: S new rows at positions P.. attend over the P cached and the new keys
+    (both tilings; prefixes and lengths straddle the 64- and 128-position tile edges)."""
+    shape = SHAPES[shape_name]
+    d = wl.random_prefill_inputs(2, P + S, shape, seed=450 + P + S)
+    q = d["q"][:, P:].contiguous()
+    g = {k: d[k].to(cuda_device) for k in ("k", "v")}
+    out = ak.prefill_causal_prefix(q.to(cuda_device), g["k"], g["v"], P, scale=d["scale"])
+    torch.cuda.synchronize()
+    assert ak.device_status() == 0
+    assert_parity(out, _prefix_expected(q, d["k"], d["v"], d["scale"], P), f"{shape_name} P={P} S={S}")
+
+
+def test_prefix_zero_is_plain_prefill_and_chunks_compose(cuda_device):
+    s = wl.DIFFQKV
+    d = wl.random_prefill_inputs(1, 600, s, seed=460)
+    g = {k: d[k].to(cuda_device) for k in ("q", "k", "v")}
+    whole = ak.prefill_causal(g["q"], g["k"], g["v"], scale=d["scale"])
+    zero = ak.prefill_causal_prefix(g["q"], g["k"], g["v"], 0, scale=d["scale"])
+    torch.cuda.synchronize()
+    assert torch.equal(whole, zero)
+    # three chunks of 200 rows, each over its prefix, equal the whole prefill
+    parts = [ak.prefill_causal_prefix(g["q"][:, c:c + 200].contiguous(), g["k"][:, :c + 200].contiguous(),
+                                      g["v"][:, :c + 200].contiguous(), c, scale=d["scale"]) for c in (0, 200, 400)]
+    torch.cuda.synchronize()
+    assert ak.device_status() == 0
+    ref = oracle.prefill_causal(d["q"], d["k"], d["v"], d["scale"])
+    assert_parity(torch.cat(parts, dim=1), ref, "chunked prefill")
