@@ -21,7 +21,7 @@ from ._capi import DiffqkvError, Dims, DecodePlan, DecodeTuning, check, lib
 __all__ = [
     "decode", "decode_workspace", "decode_plan", "decode_from_host", "decode_topv", "decode_topv_workspace",
     "prefill_causal", "device_status", "selftest_wait_timeout", "DiffqkvError", "Dims", "library_path",
-    "decode_noalloc",
+    "decode_noalloc", "decode_append", "decode_paged", "prefill_causal_prefix",
 ]
 
 library_path = _capi.LIB_PATH
@@ -138,6 +138,50 @@ def decode_append(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor, k_c
                                      _ptr(v_cache), _ptr(seq_lens), t_max, msl, _ptr(out), _ptr(workspace),
                                      workspace.numel(), _stream_ptr(stream))
     check(st, "diffqkv_decode_append")
+    return out
+
+
+def decode_paged(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor, block_table: torch.Tensor,
+                 seq_lens: torch.Tensor, *, k_new: Optional[torch.Tensor] = None, v_new: Optional[torch.Tensor] = None,
+                 scale: Optional[float] = None, max_seq_len: Optional[int] = None, out: Optional[torch.Tensor] = None,
+                 workspace: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Decode over paged caches: k_pages [num_pages, page_size, n_k, d_k], v_pages [num_pages, page_size, n_v, d_v]
+    and block_table int32 [B, max_blocks]; position j of sequence b is row j % page_size of page
+    block_table[b, j // page_size].  With k_new / v_new given the step's token is appended at
+    position seq_lens[b] first (as in :func:`decode_append`).  Returns bf16 [B, n_q, d_v]."""
+    _bf16_dev(q, "q", 3)
+    _bf16_dev(k_pages, "k_pages", 4)
+    _bf16_dev(v_pages, "v_pages", 4)
+    for t, name in ((block_table, "block_table"), (seq_lens, "seq_lens")):
+        if t.dtype != torch.int32 or not t.is_cuda or not t.is_contiguous():
+            raise TypeError(f"{name} must be a contiguous int32 CUDA tensor")
+    B, n_q, d_k = q.shape
+    num_pages, page_size, n_k, d_k2 = k_pages.shape
+    num_pages2, page_size2, n_v, d_v = v_pages.shape
+    if d_k != d_k2 or num_pages != num_pages2 or page_size != page_size2:
+        raise ValueError("q / k_pages / v_pages shapes disagree")
+    if block_table.dim() != 2 or block_table.shape[0] != B:
+        raise ValueError("block_table must be [B, max_blocks]")
+    max_blocks = block_table.shape[1]
+    dims = make_dims(B, n_q, n_k, n_v, d_k, d_v, d_k ** -0.5 if scale is None else scale)
+    if (k_new is None) != (v_new is None):
+        raise ValueError("give both k_new and v_new, or neither")
+    if k_new is not None:
+        _bf16_dev(k_new, "k_new", 3)
+        _bf16_dev(v_new, "v_new", 3)
+        if tuple(k_new.shape) != (B, n_k, d_k) or tuple(v_new.shape) != (B, n_v, d_v):
+            raise ValueError("k_new must be [B, n_k, d_k] and v_new [B, n_v, d_v]")
+    if out is None:
+        out = torch.empty((B, n_q, d_v), dtype=torch.bfloat16, device=q.device)
+    if workspace is None:
+        workspace = decode_workspace(dims, device=q.device)
+    t_max = max_blocks * page_size
+    msl = t_max if max_seq_len is None else int(max_seq_len)
+    st = lib().diffqkv_decode_paged(ctypes.byref(dims), _ptr(q), _ptr(k_new),
+                                    _ptr(v_new), _ptr(k_pages), _ptr(v_pages),
+                                    _ptr(block_table), max_blocks, page_size, num_pages, _ptr(seq_lens), msl,
+                                    _ptr(out), _ptr(workspace), workspace.numel(), _stream_ptr(stream))
+    check(st, "diffqkv_decode_paged")
     return out
 
 

@@ -24,9 +24,10 @@ STATUS = {
     7: "DIFFQKV_ERR_DEVICE_SEQLEN",
     8: "DIFFQKV_ERR_NO_DEVICE",
     9: "DIFFQKV_ERR_SCRATCH_LIMIT",
+    10: "DIFFQKV_ERR_DEVICE_PAGE",
 }
 (OK, INVALID_ARG, UNSUPPORTED, MISALIGNED, WORKSPACE, CUDA_ERR, DEVICE_TIMEOUT, DEVICE_SEQLEN, NO_DEVICE,
- SCRATCH_LIMIT) = range(10)
+ SCRATCH_LIMIT, DEVICE_PAGE) = range(11)
 TOPV_FULL_SOFTMAX_WEIGHTS = 1  # flag of diffqkv_decode_topv_ex (include/diffqkv.h)
 
 
@@ -80,6 +81,7 @@ SIGNATURES = {
     "diffqkv_decode": ([_DIMS, _P, _P, _P, _P, _I32, _I32, _P, _P, _SZ, _P], _I32),
     "diffqkv_decode_ex": ([_DIMS, _P, _P, _P, _P, _I32, _I32, _P, _P, _SZ, ctypes.POINTER(DecodeTuning), _P], _I32),
     "diffqkv_decode_append": ([_DIMS, _P, _P, _P, _P, _P, _P, _I32, _I32, _P, _P, _SZ, _P], _I32),
+    "diffqkv_decode_paged": ([_DIMS, _P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _P, _I32, _P, _P, _SZ, _P], _I32),
     "diffqkv_decode_plan": ([_DIMS, _I32, _I32, _I32, ctypes.POINTER(DecodeTuning), ctypes.POINTER(DecodePlan)],
                             _I32),
     "diffqkv_decode_from_host": ([_DIMS, _P, _P, _P, _P, _I32, _I32, _P, _P, _P, _P, _P, _P, _P, _SZ, _P], _I32),

@@ -180,6 +180,7 @@ const char *diffqkv_status_string(int32_t status) {
         case DIFFQKV_ERR_DEVICE_SEQLEN: return "DIFFQKV_ERR_DEVICE_SEQLEN";
         case DIFFQKV_ERR_NO_DEVICE: return "DIFFQKV_ERR_NO_DEVICE";
         case DIFFQKV_ERR_SCRATCH_LIMIT: return "DIFFQKV_ERR_SCRATCH_LIMIT";
+        case DIFFQKV_ERR_DEVICE_PAGE: return "DIFFQKV_ERR_DEVICE_PAGE";
         default: return "DIFFQKV_ERR_UNKNOWN";
     }
 }
@@ -212,6 +213,20 @@ diffqkv_status_t diffqkv_decode_append(const diffqkv_dims_t *dims, const void *q
     if (!k_new || !v_new) return DIFFQKV_ERR_INVALID_ARG;
     return diffqkv::decode_launch(dims, q, k_cache, v_cache, seq_lens, t_max, max_seq_len, out, workspace,
                                   workspace_bytes, nullptr, (cudaStream_t)stream, k_new, v_new);
+}
+
+diffqkv_status_t diffqkv_decode_paged(const diffqkv_dims_t *dims, const void *q, const void *k_new,
+                                      const void *v_new, void *k_pages, void *v_pages,
+                                      const int32_t *block_table, int32_t max_blocks, int32_t page_size,
+                                      int32_t num_pages, const int32_t *seq_lens, int32_t max_seq_len,
+                                      void *out, void *workspace, size_t workspace_bytes,
+                                      diffqkv_stream_t stream) {
+    if ((k_new == nullptr) != (v_new == nullptr)) return DIFFQKV_ERR_INVALID_ARG;
+    if (max_blocks < 1 || page_size < 1 || (long long)max_blocks * page_size > 0x7fffffffLL)
+        return DIFFQKV_ERR_INVALID_ARG;
+    const diffqkv::PagedCache paged{block_table, max_blocks, page_size, num_pages};
+    return diffqkv::decode_launch(dims, q, k_pages, v_pages, seq_lens, max_blocks * page_size, max_seq_len, out,
+                                  workspace, workspace_bytes, nullptr, (cudaStream_t)stream, k_new, v_new, &paged);
 }
 
 diffqkv_status_t diffqkv_decode_ex(const diffqkv_dims_t *dims, const void *q, const void *k_cache,

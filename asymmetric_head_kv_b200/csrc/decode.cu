@@ -30,10 +30,18 @@
 //    tiles still cover the p cached positions only; the combining CTA adds the
 //    new token as one more partial (m = its score, l = 1, o = v_new) and writes
 //    k_new / v_new into the cache at p, which no CTA of this launch reads.
+//  * Paged caches (block table given): K and V live in two page pools
+//    [num_pages, page_size, heads, d] that share one block table [B, max_blocks]
+//    (position j of sequence b is row j % page_size of pool page
+//    table[b][j / page_size]).  The tiles, splits and combine are unchanged;
+//    the producer fills a tile with sub-boxes of gcd(tile, page_size)
+//    positions, each inside one page, so the consumers see the same shared
+//    memory layout as with contiguous caches.
 #include <math.h>
 
 #include <algorithm>
 #include <mutex>
+#include <numeric>
 
 #include "common.cuh"
 #include "internal.h"
@@ -67,7 +75,13 @@ struct DecodeArgs {
     uint32_t stage_stride;  // bytes between stages
     float scale_log2;       // scale * log2(e)
     uint64_t wait_limit_ns;
+    // paged caches; block_table == null means contiguous [B, t_max, heads, d] caches
+    const int32_t *block_table = nullptr;  // [B, max_blocks] pool page of each logical page
+    int32_t max_blocks = 0, page_size = 0, num_pages = 0;
+    int32_t sub_rows = 0;                  // positions per sub-box (divides the tile and the page)
+    uint32_t sub_k_bytes = 0, sub_v_bytes = 0;
 };
+
 
 // Position of the tile walk: unit (b, g), tile i of nt, first global tile P.
 struct Walker {
@@ -76,6 +90,32 @@ struct Walker {
 };
 
 __device__ __forceinline__ int clamp_len(int v, int t_max) { return v < 0 ? 0 : (v > t_max ? t_max : v); }
+
+// Block-table entry of logical page pi of sequence b, unchecked.
+__device__ __forceinline__ int page_entry(const DecodeArgs &a, int b, int pi) {
+    return __ldg(a.block_table + (size_t)b * a.max_blocks + pi);
+}
+
+// A block-table entry checked against the pool: an entry outside
+// [0, num_pages) is flagged DIFFQKV_ERR_DEVICE_PAGE and -1 returned.
+__device__ __forceinline__ int checked_page(const DecodeArgs &a, int page) {
+    if (page >= 0 && page < a.num_pages) return page;
+    record_error(a.status, DIFFQKV_ERR_DEVICE_PAGE);
+    return -1;
+}
+
+// Pool page holding logical page pi of sequence b (checked).
+__device__ __forceinline__ int paged_page(const DecodeArgs &a, int b, int pi) {
+    return checked_page(a, page_entry(a, b, pi));
+}
+
+// Storage row (one position's heads) of position p of sequence b, or -1 when
+// its page-table entry is out of range.
+__device__ __forceinline__ long long cache_row(const DecodeArgs &a, int b, int p) {
+    if (!a.block_table) return (long long)b * a.t_max + p;
+    const int page = paged_page(a, b, p / a.page_size);
+    return page < 0 ? -1 : (long long)page * a.page_size + p % a.page_size;
+}
 
 template <int TT>
 __device__ __forceinline__ void walker_advance(Walker &w, const DecodeArgs &a) {
@@ -96,6 +136,57 @@ __device__ __forceinline__ void walker_advance(Walker &w, const DecodeArgs &a) {
 // [floor(c N / G), floor((c+1) N / G)).
 __device__ __forceinline__ long long cta_of_tile(long long t, long long N, long long G) {
     return ((t + 1) * G - 1) / N;
+}
+
+// Sub-boxes holding the valid positions of the walker's current tile (paged caches).
+template <int TT>
+__device__ __forceinline__ int sub_boxes(const DecodeArgs &a, const Walker &w) {
+    return (min(TT, w.T - w.i * TT) + a.sub_rows - 1) / a.sub_rows;
+}
+
+// Block-table entry of sub-box f of the walker's current tile, 0 when f is past its sub-boxes.
+template <int TT>
+__device__ __forceinline__ int sub_box_entry(const DecodeArgs &a, const Walker &w, int f) {
+    return f < sub_boxes<TT>(a, w) ? page_entry(a, w.b, (w.i * TT + f * a.sub_rows) / a.page_size) : 0;
+}
+
+// Producer for paged caches, run by the whole producer warp.  Lane f issues the K and V loads of
+// sub-boxes f, f + 32, ... of a tile, so a tile's sub-boxes leave as one warp instruction each;
+// every lane reads its block-table entry for the next tile one full iteration ahead.  Returns the
+// number of tiles issued.
+template <int TT, int QPK>
+__device__ long long produce_paged(const CUtensorMap *tm_k, const CUtensorMap *tm_v, const DecodeArgs &a, Walker w,
+                                   long long t_begin, long long t_end, uint8_t *smem, uint64_t *full_bar,
+                                   uint64_t *empty_bar, volatile int *abort_flag, int lane) {
+    int cur = sub_box_entry<TT>(a, w, lane);
+    long long k = 0;
+    for (long long t = t_begin; t < t_end; ++t, ++k) {
+        const int stage = (int)(k % a.stages);
+        const int n_sub = sub_boxes<TT>(a, w);
+        Walker wn = w;
+        if (t + 1 < t_end) walker_advance<TT>(wn, a);
+        const int nxt = (t + 1 < t_end) ? sub_box_entry<TT>(a, wn, lane) : 0;
+        if (k >= a.stages) {
+            const uint32_t parity = (uint32_t)(((k / a.stages) - 1) & 1);
+            mbar_wait_bounded(&empty_bar[stage], parity, a.wait_limit_ns, abort_flag, a.status);
+        }
+        if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
+        uint8_t *sb = smem + (size_t)stage * a.stage_stride;
+        if (lane == 0) mbar_arrive_expect_tx(&full_bar[stage], (uint32_t)n_sub * (a.sub_k_bytes + a.sub_v_bytes));
+        __syncwarp();
+        const int v0 = (w.g * QPK) / a.q_per_v;
+        for (int f = lane; f < n_sub; f += 32) {
+            // a bad entry (flagged) loads pool page 0 instead: the loads stay in bounds
+            const int entry = f == lane ? cur : page_entry(a, w.b, (w.i * TT + f * a.sub_rows) / a.page_size);
+            const int page = max(checked_page(a, entry), 0);
+            const int row = (w.i * TT + f * a.sub_rows) % a.page_size;
+            tma_load_4d(sb + (size_t)f * a.sub_k_bytes, tm_k, &full_bar[stage], 0, w.g, row, page);
+            tma_load_4d(sb + a.k_tile_bytes + (size_t)f * a.sub_v_bytes, tm_v, &full_bar[stage], 0, v0, row, page);
+        }
+        cur = nxt;
+        w = wn;
+    }
+    return k;
 }
 
 template <int DK, int DV, int QPK, int TT, int NCW>
@@ -217,10 +308,13 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
                     const int h = e / DV;
                     o[e] = a.v_new[((size_t)b * a.n_v + h / a.q_per_v) * DV + e % DV];
                 }
-                for (int e = tid; e < a.n_k * DK; e += blockDim.x)
-                    a.k_store[(size_t)b * a.t_max * a.n_k * DK + e] = a.k_new[(size_t)b * a.n_k * DK + e];
-                for (int e = tid; e < a.n_v * DV; e += blockDim.x)
-                    a.v_store[(size_t)b * a.t_max * a.n_v * DV + e] = a.v_new[(size_t)b * a.n_v * DV + e];
+                const long long row0 = cache_row(a, b, 0);
+                if (row0 >= 0) {
+                    for (int e = tid; e < a.n_k * DK; e += blockDim.x)
+                        a.k_store[(size_t)row0 * a.n_k * DK + e] = a.k_new[(size_t)b * a.n_k * DK + e];
+                    for (int e = tid; e < a.n_v * DV; e += blockDim.x)
+                        a.v_store[(size_t)row0 * a.n_v * DV + e] = a.v_new[(size_t)b * a.n_v * DV + e];
+                }
             } else {
                 for (int e = tid; e < a.n_q * DV; e += blockDim.x) o[e] = __float2bfloat16(0.f);
             }
@@ -240,10 +334,14 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
     w0.nt = (w0.T + TT - 1) / TT;
 
     if (warp == NCW) {
-        // ================= producer: one elected lane issues all TMA loads
-        if (lane == 0) {
+        // ================= producer: one elected lane issues the TMA loads of contiguous caches;
+        // the whole warp runs the paged producer
+        long long k = 0;
+        if (a.block_table) {
+            k = produce_paged<TT, QPK>(&tm_k, &tm_v, a, w0, t_begin, t_end, smem, full_bar, empty_bar, abort_flag,
+                                       lane);
+        } else if (lane == 0) {
             Walker w = w0;
-            long long k = 0;
             for (long long t = t_begin; t < t_end; ++t, ++k) {
                 const int stage = (int)(k % a.stages);
                 if (k >= a.stages) {
@@ -258,6 +356,8 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
                 tma_load_4d(sb + a.k_tile_bytes, &tm_v, &full_bar[stage], 0, v0, w.i * TT, w.b);
                 walker_advance<TT>(w, a);
             }
+        }
+        if (lane == 0) {
             // drain: never leave the CTA with copies still landing in its shared memory
             const long long issued = k;
             for (long long j = (issued > a.stages ? issued - a.stages : 0); j < issued; ++j) {
@@ -466,15 +566,16 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
                         for (int off = 16; off >= 1; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
                         if (lane == 0) merge_s[warp] = dot * a.scale_log2;
                     }
-                    const size_t kdst = (((size_t)w.b * a.t_max + p) * a.n_k + w.g) * DK;
+                    const long long row = cache_row(a, w.b, p);  // -1: bad page entry, nothing written
+                    const size_t kdst = ((size_t)row * a.n_k + w.g) * DK;
                     const size_t ksrc = ((size_t)w.b * a.n_k + w.g) * DK;
-                    for (int e = tid; e < DK / 8; e += NCW * 32)
+                    for (int e = tid; e < DK / 8 && row >= 0; e += NCW * 32)
                         reinterpret_cast<uint4 *>(a.k_store + kdst)[e] = reinterpret_cast<const uint4 *>(a.k_new + ksrc)[e];
-                    for (int e = tid; e < QPK * (DV / 8); e += NCW * 32) {
+                    for (int e = tid; e < QPK * (DV / 8) && row >= 0; e += NCW * 32) {
                         const int h = w.g * QPK + e / (DV / 8);
                         if (h % a.q_per_v != 0) continue;  // one writer per V head: its first query head
                         const int vh = h / a.q_per_v;
-                        const size_t vdst = (((size_t)w.b * a.t_max + p) * a.n_v + vh) * DV;
+                        const size_t vdst = ((size_t)row * a.n_v + vh) * DV;
                         const size_t vsrc = ((size_t)w.b * a.n_v + vh) * DV;
                         reinterpret_cast<uint4 *>(a.v_store + vdst)[e % (DV / 8)] =
                             reinterpret_cast<const uint4 *>(a.v_new + vsrc)[e % (DV / 8)];
@@ -661,10 +762,16 @@ diffqkv_status_t decode_plan(const diffqkv_dims_t *d, int32_t t_max, int32_t max
 diffqkv_status_t decode_launch(const diffqkv_dims_t *d, const void *q, const void *k_cache, const void *v_cache,
                                const int32_t *seq_lens, int32_t t_max, int32_t max_seq_len, void *out,
                                void *workspace, size_t workspace_bytes, const diffqkv_decode_tuning_t *tuning,
-                               cudaStream_t stream, const void *k_new, const void *v_new) {
+                               cudaStream_t stream, const void *k_new, const void *v_new, const PagedCache *paged) {
     diffqkv_status_t st = validate_dims(d);
     if (st != DIFFQKV_OK) return st;
     if (!q || !k_cache || !v_cache || !seq_lens || !out || t_max < 1) return DIFFQKV_ERR_INVALID_ARG;
+    if (paged) {
+        if (!paged->block_table || paged->max_blocks < 1 || paged->page_size < 1 || paged->num_pages < 1 ||
+            (long long)paged->max_blocks * paged->page_size != t_max)
+            return DIFFQKV_ERR_INVALID_ARG;
+        if (reinterpret_cast<uintptr_t>(paged->block_table) & 3u) return DIFFQKV_ERR_MISALIGNED;
+    }
     if ((k_new == nullptr) != (v_new == nullptr)) return DIFFQKV_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
         (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
@@ -684,15 +791,29 @@ diffqkv_status_t decode_launch(const diffqkv_dims_t *d, const void *q, const voi
     KernelFn fn = pick_kernel(d->d_k, d->d_v, qpk);
     if (!fn) return DIFFQKV_ERR_UNSUPPORTED;
 
+    // contiguous caches: one box per tile over [B, t_max, heads, d]; paged: sub-boxes over
+    // [num_pages, page_size, heads, d], each gcd(tile, page_size) positions inside one page
+    const int sub_rows = paged ? std::gcd(plan.tile_tokens, paged->page_size) : plan.tile_tokens;
+    const uint64_t rows_dim = paged ? (uint64_t)paged->page_size : (uint64_t)t_max;
+    const uint64_t outer_dim = paged ? (uint64_t)paged->num_pages : (uint64_t)d->batch;
     CUtensorMap tm_k, tm_v;
-    st = make_tensor_map_4d(&tm_k, k_cache, d->d_k, d->n_k, t_max, d->batch, d->d_k, 1, plan.tile_tokens, 1,
+    st = make_tensor_map_4d(&tm_k, k_cache, d->d_k, d->n_k, rows_dim, outer_dim, d->d_k, 1, sub_rows, 1,
                             CU_TENSOR_MAP_SWIZZLE_NONE, k_promotion(d));
     if (st != DIFFQKV_OK) return st;
-    st = make_tensor_map_4d(&tm_v, v_cache, d->d_v, d->n_v, t_max, d->batch, d->d_v, plan.v_heads_per_tile,
-                            plan.tile_tokens, 1, CU_TENSOR_MAP_SWIZZLE_NONE);
+    st = make_tensor_map_4d(&tm_v, v_cache, d->d_v, d->n_v, rows_dim, outer_dim, d->d_v, plan.v_heads_per_tile,
+                            sub_rows, 1, CU_TENSOR_MAP_SWIZZLE_NONE);
     if (st != DIFFQKV_OK) return st;
 
     DecodeArgs a;
+    if (paged) {
+        a.block_table = paged->block_table;
+        a.max_blocks = paged->max_blocks;
+        a.page_size = paged->page_size;
+        a.num_pages = paged->num_pages;
+        a.sub_rows = sub_rows;
+        a.sub_k_bytes = (uint32_t)sub_rows * d->d_k * 2;
+        a.sub_v_bytes = (uint32_t)sub_rows * plan.v_heads_per_tile * d->d_v * 2;
+    }
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     const size_t units = (size_t)d->batch * d->n_k;
     a.q = static_cast<const __nv_bfloat16 *>(q);

@@ -45,15 +45,24 @@ diffqkv_status_t ensure_dynamic_smem(const void *kernel, int bytes);
 diffqkv_status_t validate_dims(const diffqkv_dims_t *d);
 
 // decode.cu
+// A paged K/V cache: pools [num_pages, page_size, heads, d] for K and for V and
+// one block table [batch, max_blocks] (device int32) of pool pages.
+struct PagedCache {
+    const int32_t *block_table;
+    int32_t max_blocks, page_size, num_pages;
+};
+
 diffqkv_status_t decode_plan(const diffqkv_dims_t *d, int32_t t_max, int32_t max_seq_len, int32_t num_sms,
                              const diffqkv_decode_tuning_t *tuning, diffqkv_decode_plan_t *plan);
 size_t decode_workspace_size(const diffqkv_dims_t *d);
 // k_new / v_new given (both or neither): append mode, the caches are written at seq_len.
+// paged given: k_cache / v_cache are page pools and t_max = max_blocks * page_size.
 diffqkv_status_t decode_launch(const diffqkv_dims_t *d, const void *q, const void *k_cache,
                                const void *v_cache, const int32_t *seq_lens, int32_t t_max,
                                int32_t max_seq_len, void *out, void *workspace, size_t workspace_bytes,
                                const diffqkv_decode_tuning_t *tuning, cudaStream_t stream,
-                               const void *k_new = nullptr, const void *v_new = nullptr);
+                               const void *k_new = nullptr, const void *v_new = nullptr,
+                               const PagedCache *paged = nullptr);
 
 diffqkv_status_t decode_noalloc_launch(const diffqkv_dims_t *d, const void *q, const void *k_cache,
                                        const void *v_cache, const int32_t *seq_lens, int32_t t_max,

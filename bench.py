@@ -51,6 +51,8 @@ PROFILE_CASES = {
     "prefill_b2_s8192": wl.PREFILL_8K,
     "prefill_gqa_b2_s8192": wl.PREFILL_8K_GQA,
     "topv_b4_t65536": wl.TOPV_64K,
+    "decode_paged_b4_t32768_p16": wl.DecodeWorkload("decode_paged_b4_t32768_p16", wl.DIFFQKV, 4, 32768, seed=1,
+                                                    page_size=16),
 }
 L2_FLUSH_BYTES = 256 << 20  # written between timed calls whose inputs fit in the 126 MB L2
 
@@ -315,6 +317,13 @@ def run_profile_case(name: str, launches: int = 4):
         for _ in range(launches):
             ak.prefill_causal(d["q"], d["k"], d["v"], scale=d["scale"], out=out)
         what = f"causal flops/launch {wl.prefill_causal_flops(w.shape, w.batch, w.seq)}"
+    elif w.page_size:
+        d = wl.random_paged_inputs(w.batch, w.t_max // w.page_size + 1, w.page_size, w.shape, seed=w.seed,
+                                   seq_lens=[w.t_max] * w.batch, device=dev)
+        for _ in range(launches):
+            ak.decode_paged(d["q"], d["k_pages"], d["v_pages"], d["block_table"], d["seq_lens"],
+                            scale=d["scale"], max_seq_len=w.t_max)
+        what = f"kv bytes/launch {wl.decode_kv_bytes(w.shape, d['seq_lens'].cpu())}"
     elif w.topk:
         d = wl.make_decode_inputs(w, dev)
         for _ in range(launches):
@@ -426,6 +435,27 @@ def time_paths(ak, peaks, steps: int, warmup: int):
                                        "frac": nbytes / (ms * 1e-3) / 1e9 / hbm, "launches_per_call": 1}
     assert ak.device_status() == 0
     del d, ws_d, out_d
+
+    # the same 16 x 32768 decode over paged caches: K and V page pools with one block table, pages
+    # dealt out to the sequences in random order
+    for page_size in (16, 64):
+        d = wl.random_paged_inputs(w.batch, w.t_max // page_size + 1, page_size, w.shape, seed=w.seed,
+                                   seq_lens=[w.t_max] * w.batch, device=dev)
+        ws_p = ak.decode_workspace(ak.make_dims(w.batch, w.shape.n_q, w.shape.n_k, w.shape.n_v, w.shape.d_k,
+                                                w.shape.d_v, w.shape.scale), device=dev)
+        out_p = torch.empty((w.batch, w.shape.n_q, w.shape.d_v), dtype=torch.bfloat16, device=dev)
+        fn = lambda: ak.decode_paged(d["q"], d["k_pages"], d["v_pages"], d["block_table"],  # noqa: E731
+                                     d["seq_lens"], scale=d["scale"], max_seq_len=w.t_max, out=out_p,
+                                     workspace=ws_p)
+        for _ in range(max(3, warmup)):
+            fn()
+        ms = statistics.median(_timed_calls(fn, steps, flush))
+        nbytes = wl.decode_kv_bytes(w.shape, d["seq_lens"].cpu())
+        res[f"decode_paged_b16_t32768_p{page_size}"] = {
+            "us": ms * 1e3, "kv_bytes": nbytes, "gbs": nbytes / (ms * 1e-3) / 1e9, "bound": "hbm",
+            "peak_gbs": hbm, "frac": nbytes / (ms * 1e-3) / 1e9 / hbm, "launches_per_call": 1}
+        assert ak.device_status() == 0
+        del d, ws_p, out_p
 
     w = wl.TOPV_64K
     d = wl.make_decode_inputs(w, dev)

@@ -64,7 +64,8 @@ typedef enum {
     DIFFQKV_ERR_DEVICE_TIMEOUT = 6, /* a bounded device-side wait ran out */
     DIFFQKV_ERR_DEVICE_SEQLEN = 7,  /* a device seq_len was < 0 or > t_max (clamped) */
     DIFFQKV_ERR_NO_DEVICE = 8,      /* no CUDA device / driver */
-    DIFFQKV_ERR_SCRATCH_LIMIT = 9   /* shape needs more than the built-in scratch of diffqkv_decode_noalloc */
+    DIFFQKV_ERR_SCRATCH_LIMIT = 9,  /* shape needs more than the built-in scratch of diffqkv_decode_noalloc */
+    DIFFQKV_ERR_DEVICE_PAGE = 10    /* a block-table entry a paged call used was outside [0, num_pages) */
 } diffqkv_status_t;
 
 /* Human-readable name of a status code (static storage; never NULL). */
@@ -135,6 +136,42 @@ diffqkv_status_t diffqkv_decode_append(const diffqkv_dims_t *dims, const void *q
                                        const int32_t *seq_lens, int32_t t_max, int32_t max_seq_len,
                                        void *out, void *workspace, size_t workspace_bytes,
                                        diffqkv_stream_t stream);
+
+/*
+ * Decode over PAGED K/V caches.  The pages compare DiffQKV with paged
+ * attention, which manages K and V as one interchangeable cache ("Where
+ * Existing Approaches Fall Short", system-level optimisations); here K and V
+ * keep separate pools whose rows differ in size (n_k*d_k against n_v*d_v)
+ * and share one block table:
+ *
+ *   k_pages     [num_pages, page_size, n_k, d_k]   K page pool (bf16, device)
+ *   v_pages     [num_pages, page_size, n_v, d_v]   V page pool
+ *   block_table [B, max_blocks] int32 (device)     pool page of each logical page
+ *
+ * Position j of sequence b is row j % page_size of pool page
+ * block_table[b, j / page_size].  The logical capacity per sequence is
+ * t_max = max_blocks * page_size (must fit in int32); seq_lens, q, out,
+ * max_seq_len and the workspace are those of diffqkv_decode with that t_max
+ * (the workspace size does not depend on t_max).  With k_new and v_new
+ * NULL the call is diffqkv_decode over the paged caches; with both given it
+ * is diffqkv_decode_append: position p_b = seq_lens[b] is written into its
+ * page (block_table[b, p_b / page_size] must then name a pool page).
+ * Only the entries of pages holding positions < seq_lens[b] (and p_b in
+ * append mode) are read; others may hold anything.  A read entry outside
+ * [0, num_pages) is flagged DIFFQKV_ERR_DEVICE_PAGE: pool page 0 is read in
+ * its place and an append into it writes nothing.  Any page_size >= 1 is
+ * accepted; a tile of the contiguous kernel is loaded as gcd(tile height,
+ * page_size)-position pieces, so page sizes sharing a factor of 8 or 16 with
+ * the tile height load fastest.  block_table must be 4-byte aligned, the
+ * other pointers 16-byte aligned.  Pages may be shared between sequences
+ * for reading; two sequences appending into one page row is a caller error.
+ */
+diffqkv_status_t diffqkv_decode_paged(const diffqkv_dims_t *dims, const void *q, const void *k_new,
+                                      const void *v_new, void *k_pages, void *v_pages,
+                                      const int32_t *block_table, int32_t max_blocks, int32_t page_size,
+                                      int32_t num_pages, const int32_t *seq_lens, int32_t max_seq_len,
+                                      void *out, void *workspace, size_t workspace_bytes,
+                                      diffqkv_stream_t stream);
 
 /* Optional launch controls for diffqkv_decode_ex (0 = library default). */
 typedef struct {

@@ -61,6 +61,8 @@ def _load():
         [c_i] * 6 + [c_d] + [c_p] * 4 + [c_i, c_i, c_i, c_p, c_i64, c_p, c_p, c_i]
     )
     lib.oracle_decode_topv_ex.restype = c_i
+    lib.oracle_gather_paged.argtypes = [c_i] * 6 + [c_p] * 4
+    lib.oracle_gather_paged.restype = c_i
     _lib = lib
     return lib
 
@@ -201,3 +203,30 @@ def decode_topv(q, k_cache, v_cache, seq_lens, topk: int, scale: float, *, rows=
     if rows is None:
         return out.reshape(B, n_q, d_v), idx.reshape(B, n_q, max(topk, 0))
     return out, idx
+
+
+def gather_paged(pool, block_table, seq_lens):
+    """Contiguous cache [B, max_blocks * page_size, heads, d] (bf16 bits as a torch bf16 tensor)
+    holding the first seq_lens[b] positions of each sequence of a paged pool
+    [num_pages, page_size, heads, d] under block_table [B, max_blocks]; zeros elsewhere."""
+    import torch
+
+    pb = _bits(pool)
+    num_pages, page_size, heads, d = pb.shape
+    bt = _i32(block_table)
+    B, max_blocks = bt.shape
+    sl = _i32(seq_lens)
+    assert sl.shape == (B,)
+    out = np.empty((B, max_blocks * page_size, heads, d), np.uint16)
+    rc = _load().oracle_gather_paged(B, heads, d, page_size, max_blocks, num_pages, _ptr(pb), _ptr(bt),
+                                     _ptr(sl), _ptr(out))
+    _check(rc, "gather_paged")
+    return torch.from_numpy(out.view(np.int16)).view(torch.bfloat16)
+
+
+def decode_paged(q, k_pages, v_pages, block_table, seq_lens, scale: float, *, rows=None,
+                 threads: int = 0) -> np.ndarray:
+    """fp64 decode over paged K/V pools: the pools gathered into contiguous caches, then :func:`decode`."""
+    k = gather_paged(k_pages, block_table, seq_lens)
+    v = gather_paged(v_pages, block_table, seq_lens)
+    return decode(q, k, v, seq_lens, scale, rows=rows, threads=threads)

@@ -19,6 +19,9 @@
  *                combine pass rescales each chunk by exp(m_c - M)   (FlexHeadFA)
  *   selective V  o_h  ~= sum over the top-k positions of the weights,
  *                renormalised over that set                         (Selective V)
+ *   paged cache  position j of sequence b is row j % P of pool page
+ *                table[b][j / P]; K and V keep separate pools  ("Where
+ *                Existing Approaches Fall Short", system-level optimisations)
  *
  * All arithmetic is fp64.  bf16 inputs arrive as raw 16-bit patterns and are
  * widened exactly.  The top-k selection ranks positions by the EXACT dot
@@ -517,4 +520,35 @@ int oracle_decode_topv(int batch, int n_q, int n_k, int n_v, int d_k, int d_v, d
                        int n_threads) {
     return oracle_decode_topv_ex(batch, n_q, n_k, n_v, d_k, d_v, scale, q, k_cache, v_cache, seq_lens, t_max,
                                  topk, 0, rows, n_rows, out, idx_out, n_threads);
+}
+
+/* ------------------------------------------------------------------ */
+/* Paged caches ("Where Existing Approaches Fall Short", item 4: paged */
+/* KV memory management; the per-position K and V caches of the       */
+/* deployment section kept as two pools of fixed-size pages)           */
+/* ------------------------------------------------------------------ */
+
+/* Copies the first seq_lens[b] positions of every sequence out of a page pool
+ * [num_pages, page_size, heads, d] into a contiguous cache
+ * [batch, max_blocks * page_size, heads, d]: position j of sequence b is row
+ * j % page_size of pool page table[b * max_blocks + j / page_size].  Positions
+ * at or past seq_lens[b] are zero.  Returns -1 on a bad argument, a seq_len
+ * outside [0, max_blocks * page_size] or a used table entry outside
+ * [0, num_pages). */
+int oracle_gather_paged(int batch, int heads, int d, int page_size, int max_blocks, int num_pages,
+                        const uint16_t *pool, const int32_t *table, const int32_t *seq_lens, uint16_t *out) {
+    if (batch < 0 || heads < 1 || d < 1 || page_size < 1 || max_blocks < 1 || num_pages < 1) return -1;
+    const int64_t t_max = (int64_t)max_blocks * page_size;
+    const int64_t row = (int64_t)heads * d; /* elements of one position */
+    memset(out, 0, sizeof(uint16_t) * (size_t)(batch * t_max * row));
+    for (int b = 0; b < batch; ++b) {
+        if (seq_lens[b] < 0 || seq_lens[b] > t_max) return -1;
+        for (int64_t j = 0; j < seq_lens[b]; ++j) {
+            const int32_t page = table[(int64_t)b * max_blocks + j / page_size];
+            if (page < 0 || page >= num_pages) return -1;
+            const uint16_t *src = pool + ((int64_t)page * page_size + j % page_size) * row;
+            memcpy(out + ((int64_t)b * t_max + j) * row, src, sizeof(uint16_t) * (size_t)row);
+        }
+    }
+    return 0;
 }

@@ -167,3 +167,20 @@ def test_prefill_prefix_rejects_negative_prefix():
     d = dims()
     st = _capi.lib().diffqkv_prefill_causal_prefix(ctypes.byref(d), 0x1000, 0x2000, 0x3000, -1, 16, 0x5000, None)
     assert st == _capi.INVALID_ARG
+
+
+def test_decode_paged_rejects_before_launch():
+    lib = _capi.lib()
+    d = dims()
+
+    def call(bt=0x7000, max_blocks=8, page_size=16, num_pages=10, kn=None, vn=None, q=0x1000):
+        return lib.diffqkv_decode_paged(ctypes.byref(d), q, kn, vn, 0x2000, 0x3000, bt, max_blocks, page_size,
+                                        num_pages, 0x4000, 128, 0x5000, 0x6000, 1 << 30, None)
+    assert call(bt=None) == _capi.INVALID_ARG
+    assert call(bt=0x7002) == _capi.MISALIGNED
+    assert call(page_size=0) == _capi.INVALID_ARG
+    assert call(max_blocks=0) == _capi.INVALID_ARG
+    assert call(num_pages=0) == _capi.INVALID_ARG
+    assert call(max_blocks=1 << 20, page_size=1 << 12) == _capi.INVALID_ARG  # capacity past int32
+    assert call(kn=0x8000) == _capi.INVALID_ARG                               # k_new without v_new
+    assert call(q=0x1008) == _capi.MISALIGNED

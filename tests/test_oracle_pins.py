@@ -352,3 +352,67 @@ def test_topv_full_weights_sum_to_the_kept_mass():
     assert np.all(out < 1.0) and np.all(out > 0.0)  # 5 of 60 positions: a strict part of the mass
     out, _ = oracle.decode_topv(d["q"], d["k_cache"], d["v_cache"], d["seq_lens"], 60, d["scale"], full_weights=True)
     np.testing.assert_allclose(out, 1.0, rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------- paged caches
+
+def _scatter_to_pages(cache, seq_lens, page_size, max_blocks, perm):
+    """Test-side inverse of the paged layout: cache [B, T, H, D] into a pool whose page for logical
+    page p of sequence b is perm[b * max_blocks + p], written position by position."""
+    B, T, H, D = cache.shape
+    pool = torch.zeros(B * max_blocks, page_size, H, D, dtype=cache.dtype)
+    table = torch.full((B, max_blocks), -1, dtype=torch.int32)
+    for b in range(B):
+        for j in range(int(seq_lens[b])):
+            page = int(perm[b * max_blocks + j // page_size])
+            table[b, j // page_size] = page
+            pool[page, j % page_size] = cache[b, j]
+    return pool, table
+
+
+@pytest.mark.parametrize("page_size", [1, 3, 16, 40])
+def test_gather_paged_inverts_a_scatter(page_size):
+    s = wl.DIFFQKV
+    t_max = 120
+    max_blocks = -(-t_max // page_size)
+    d = wl.random_decode_inputs(3, max_blocks * page_size, s, seed=61, seq_lens=[120, 0, 47])
+    perm = torch.randperm(3 * max_blocks, generator=torch.Generator().manual_seed(62))
+    for name in ("k_cache", "v_cache"):
+        pool, table = _scatter_to_pages(d[name], d["seq_lens"], page_size, max_blocks, perm)
+        got = oracle.gather_paged(pool, table, d["seq_lens"])
+        assert got.shape == d[name].shape
+        for b, T in enumerate(d["seq_lens"].tolist()):
+            assert torch.equal(got[b, :T], d[name][b, :T])
+            assert not got[b, T:].float().any()
+
+
+def test_gather_paged_one_page_per_sequence_is_the_pool():
+    """page_size = t_max with table[b] = [b]: the pool already is the contiguous cache."""
+    s = wl.DIFFQKV
+    d = wl.random_decode_inputs(2, 33, s, seed=63)
+    table = torch.arange(2, dtype=torch.int32)[:, None]
+    assert torch.equal(oracle.gather_paged(d["v_cache"], table, d["seq_lens"]), d["v_cache"])
+
+
+def test_gather_paged_rejects_a_bad_entry():
+    pool = torch.zeros(4, 8, 1, 8, dtype=torch.bfloat16)
+    with pytest.raises(RuntimeError):
+        oracle.gather_paged(pool, torch.tensor([[0, 4]], dtype=torch.int32), torch.tensor([9], dtype=torch.int32))
+    # an entry past the sequence's pages is never read
+    oracle.gather_paged(pool, torch.tensor([[0, -7]], dtype=torch.int32), torch.tensor([8], dtype=torch.int32))
+
+
+def test_decode_paged_matches_sdpa_over_the_pages():
+    """Paged decode against library SDPA on K/V rows looked up straight from the pools."""
+    s = wl.DIFFQKV
+    d = wl.random_paged_inputs(2, 5, 16, s, seed=64, seq_lens=[70, 33])
+    out = oracle.decode_paged(d["q"], d["k_pages"], d["v_pages"], d["block_table"], d["seq_lens"], d["scale"])
+    for b, T in enumerate(d["seq_lens"].tolist()):
+        pages = d["block_table"][b].long()
+        pos = torch.arange(T)
+        k = d["k_pages"][pages[pos // 16], pos % 16].double()   # [T, n_k, d_k]
+        v = d["v_pages"][pages[pos // 16], pos % 16].double()
+        k = k.repeat_interleave(s.n_q // s.n_k, dim=1).transpose(0, 1)[:, None]   # [n_q, 1, T, d_k]
+        v = v.repeat_interleave(s.n_q // s.n_v, dim=1).transpose(0, 1)[:, None]
+        ref = F.scaled_dot_product_attention(d["q"][b].double()[:, None, None], k, v, scale=d["scale"])
+        np.testing.assert_allclose(out[b], ref[:, 0, 0].numpy(), atol=1e-12, rtol=0)

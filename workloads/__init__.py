@@ -17,7 +17,12 @@ Recipe (per workload, ``seed`` fixed per workload):
   * q, then K, then V: ``torch.randn(..., dtype=float32)`` on a generator
     seeded ``seed`` on the chosen device, K and V drawn one batch element at a
     time ([t_max, heads, dim] per element), each rounded to bf16 (RNE);
-  * optional K scale (the ragged workload uses 0.5, exact in bf16).
+  * optional K scale (the ragged workload uses 0.5, exact in bf16);
+  * paged caches: q, then the K pool, then the V pool (one draw each, the
+    whole [num_pages, page_size, heads, dim] pool), then a random permutation of the pool pages
+    (``torch.randperm`` on the CPU generator seeded ``seed + 1``) dealt out
+    in sequence order, ceil((seq_len + 1) / page_size) pages per sequence
+    (one spare position for an append) and -1 in the unused table entries.
 The CPU and CUDA generators produce different streams; each run feeds the
 bytes it generated to both sides.
 """
@@ -64,6 +69,7 @@ class DecodeWorkload:
     ragged: Optional[tuple] = None  # (lo, hi) inclusive context lengths
     k_scale: float = 1.0
     topk: int = 0                    # >0: selective-V decode
+    page_size: int = 0               # >0: paged caches (random_paged_inputs)
 
     def seq_lens(self) -> torch.Tensor:
         if self.ragged is None:
@@ -146,6 +152,32 @@ def random_decode_inputs(batch, t_max, shape: Shape, seed: int, device="cpu", se
     if seq_lens is not None:
         d["seq_lens"] = torch.as_tensor(seq_lens, dtype=torch.int32).to(device)
     return d
+
+
+def random_paged_inputs(batch, max_blocks, page_size, shape: Shape, seed: int, seq_lens, device="cpu",
+                        spare_pages: int = 0):
+    """Paged decode inputs: dict(q, k_pages, v_pages, block_table, seq_lens, scale, num_pages).
+
+    k_pages [num_pages, page_size, n_k, d_k] and v_pages [num_pages, page_size, n_v, d_v] bf16;
+    block_table int32 [B, max_blocks] of distinct pool pages in random order, -1 where unused.
+    num_pages = the pages the sequences hold plus ``spare_pages`` never referenced."""
+    s = shape
+    lens = torch.as_tensor(seq_lens, dtype=torch.int32)
+    t_max = max_blocks * page_size
+    held = [min(max_blocks, (int(t) + 1 + page_size - 1) // page_size) for t in lens.clamp(0, t_max).tolist()]
+    num_pages = max(1, sum(held) + spare_pages)
+    g = torch.Generator(device=device).manual_seed(seed)
+    q = _randn_bf16((batch, s.n_q, s.d_k), g, device)
+    k = _randn_bf16((num_pages, page_size, s.n_k, s.d_k), g, device)
+    v = _randn_bf16((num_pages, page_size, s.n_v, s.d_v), g, device)
+    perm = torch.randperm(num_pages, generator=torch.Generator().manual_seed(seed + 1)).to(torch.int32)
+    table = torch.full((batch, max_blocks), -1, dtype=torch.int32)
+    at = 0
+    for b, n in enumerate(held):
+        table[b, :n] = perm[at:at + n]
+        at += n
+    return dict(q=q, k_pages=k, v_pages=v, block_table=table.to(device), seq_lens=lens.to(device),
+                scale=s.scale, num_pages=num_pages)
 
 
 def random_prefill_inputs(batch, seq, shape: Shape, seed: int, device="cpu"):
