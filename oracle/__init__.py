@@ -63,6 +63,10 @@ def _load():
     lib.oracle_decode_topv_ex.restype = c_i
     lib.oracle_gather_paged.argtypes = [c_i] * 6 + [c_p] * 4
     lib.oracle_gather_paged.restype = c_i
+    lib.oracle_decode_up_projected.argtypes = [c_i] * 8 + [c_d] + [c_p] * 5 + [c_i, c_p]
+    lib.oracle_decode_up_projected.restype = c_i
+    lib.oracle_fold_query.argtypes = [c_i] * 6 + [c_p] * 3
+    lib.oracle_fold_query.restype = c_i
     _lib = lib
     return lib
 
@@ -230,3 +234,32 @@ def decode_paged(q, k_pages, v_pages, block_table, seq_lens, scale: float, *, ro
     k = gather_paged(k_pages, block_table, seq_lens)
     v = gather_paged(v_pages, block_table, seq_lens)
     return decode(q, k, v, seq_lens, scale, rows=rows, threads=threads)
+
+
+def decode_up_projected(q_aug, w_up, k_cache, v_cache, seq_lens, scale: float) -> np.ndarray:
+    """fp64 decode whose keys are first projected up to the query width: q_aug [B, n_q, d_q],
+    w_up [w_heads, d_q, d_k] (w_heads 1 or n_k), caches as in :func:`decode`.  [B, n_q, d_v]."""
+    qb, wb, kb, vb = _bits(q_aug), _bits(w_up), _bits(k_cache), _bits(v_cache)
+    B, n_q, d_q = qb.shape
+    w_heads, d_q2, d_k = wb.shape
+    _, t_max, n_k, d_k2 = kb.shape
+    _, _, n_v, d_v = vb.shape
+    assert d_q == d_q2 and d_k == d_k2
+    sl = _i32(seq_lens)
+    out = np.empty((B, n_q, d_v), np.float64)
+    rc = _load().oracle_decode_up_projected(B, n_q, n_k, n_v, d_q, d_k, d_v, w_heads, float(scale), _ptr(qb),
+                                            _ptr(wb), _ptr(kb), _ptr(vb), _ptr(sl), t_max, _ptr(out))
+    _check(rc, "decode_up_projected")
+    return out
+
+
+def fold_query(q_aug, w_up, n_k: int) -> np.ndarray:
+    """fp64 W^T q for every query head (its K head's matrix): [B, n_q, d_k]."""
+    qb, wb = _bits(q_aug), _bits(w_up)
+    B, n_q, d_q = qb.shape
+    w_heads, d_q2, d_k = wb.shape
+    assert d_q == d_q2
+    out = np.empty((B, n_q, d_k), np.float64)
+    rc = _load().oracle_fold_query(B, n_q, n_k, d_q, d_k, w_heads, _ptr(qb), _ptr(wb), _ptr(out))
+    _check(rc, "fold_query")
+    return out

@@ -22,6 +22,8 @@
  *   paged cache  position j of sequence b is row j % P of pool page
  *                table[b][j / P]; K and V keep separate pools  ("Where
  *                Existing Approaches Fall Short", system-level optimisations)
+ *   d_q != d_k   each cached K row is projected up to the query width,
+ *                k_up = W k, before the dot product         (Step 4, Attend)
  *
  * All arithmetic is fp64.  bf16 inputs arrive as raw 16-bit patterns and are
  * widened exactly.  The top-k selection ranks positions by the EXACT dot
@@ -550,5 +552,87 @@ int oracle_gather_paged(int batch, int heads, int d, int page_size, int max_bloc
             memcpy(out + ((int64_t)b * t_max + j) * row, src, sizeof(uint16_t) * (size_t)row);
         }
     }
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* Query and key of different widths (section 3.4, Step 4: the Attend  */
+/* function; K is brought to the query's width by a feed-forward layer */
+/* before the dot product, read here as a linear map without bias)     */
+/* ------------------------------------------------------------------ */
+
+/* Decode with up-projected keys, in the pages' order: every cached K row of
+ * head g is mapped to the query width, k_up[r] = sum_c W[m][r][c] * K[j][g][c]
+ * (W [w_heads, d_q, d_k], m = g when w_heads == n_k, 0 when w_heads == 1), the
+ * score is s_j = scale * <q_aug[b][h], k_up>, and the output is the softmax-
+ * weighted sum of the V rows.  q_aug [B, n_q, d_q]; caches as in oracle_decode.
+ * out [B, n_q, d_v].  Single-threaded; meant for test sizes. */
+int oracle_decode_up_projected(int batch, int n_q, int n_k, int n_v, int d_q, int d_k, int d_v, int w_heads,
+                               double scale, const uint16_t *q_aug, const uint16_t *w_up,
+                               const uint16_t *k_cache, const uint16_t *v_cache, const int32_t *seq_lens,
+                               int t_max, double *out) {
+    if (check_dims(batch, n_q, n_k, n_v, d_k, d_v) || d_q < 1 || t_max < 0 || !(w_heads == 1 || w_heads == n_k))
+        return -1;
+    double *kup = (double *)malloc(sizeof(double) * (size_t)d_q);
+    double *s = (double *)malloc(sizeof(double) * (size_t)(t_max > 0 ? t_max : 1));
+    if (!kup || !s) { free(kup); free(s); return -3; }
+    for (int b = 0; b < batch; ++b) {
+        const int T = seq_lens[b];
+        if (T < 0 || T > t_max) { free(kup); free(s); return -1; }
+        for (int h = 0; h < n_q; ++h) {
+            const int g = oracle_head_map(n_q, n_k, h);
+            const int vh = oracle_head_map(n_q, n_v, h);
+            const uint16_t *W = w_up + (int64_t)(w_heads == 1 ? 0 : g) * d_q * d_k;
+            const uint16_t *qa = q_aug + ((int64_t)b * n_q + h) * d_q;
+            double *o = out + ((int64_t)b * n_q + h) * d_v;
+            for (int e = 0; e < d_v; ++e) o[e] = 0.0;
+            if (T == 0) continue;
+            double m = -INFINITY;
+            for (int j = 0; j < T; ++j) {
+                const uint16_t *kr = k_cache + (((int64_t)b * t_max + j) * n_k + g) * d_k;
+                for (int r = 0; r < d_q; ++r) {
+                    double acc = 0.0;
+                    for (int c = 0; c < d_k; ++c) acc += bf16_to_f64(W[(int64_t)r * d_k + c]) * bf16_to_f64(kr[c]);
+                    kup[r] = acc;
+                }
+                double dot = 0.0;
+                for (int r = 0; r < d_q; ++r) dot += bf16_to_f64(qa[r]) * kup[r];
+                s[j] = scale * dot;
+                if (s[j] > m) m = s[j];
+            }
+            double den = 0.0;
+            for (int j = 0; j < T; ++j) {
+                const double w = exp(s[j] - m);
+                den += w;
+                const uint16_t *vr = v_cache + (((int64_t)b * t_max + j) * n_v + vh) * d_v;
+                for (int e = 0; e < d_v; ++e) o[e] += w * bf16_to_f64(vr[e]);
+            }
+            for (int e = 0; e < d_v; ++e) o[e] /= den;
+        }
+    }
+    free(kup);
+    free(s);
+    return 0;
+}
+
+/* The same up-projection moved onto the query: <q, W k> = <W^T q, k>, so
+ * q_fold[b][h][c] = sum_r q_aug[b][h][r] * W[m][r][c] (m as above) is a query
+ * of width d_k for the ordinary decode.  out [B, n_q, d_k] in fp64. */
+int oracle_fold_query(int batch, int n_q, int n_k, int d_q, int d_k, int w_heads, const uint16_t *q_aug,
+                      const uint16_t *w_up, double *out) {
+    if (batch < 0 || n_q < 1 || n_k < 1 || n_q % n_k || d_q < 1 || d_k < 1 || !(w_heads == 1 || w_heads == n_k))
+        return -1;
+    for (int b = 0; b < batch; ++b)
+        for (int h = 0; h < n_q; ++h) {
+            const int g = oracle_head_map(n_q, n_k, h);
+            const uint16_t *W = w_up + (int64_t)(w_heads == 1 ? 0 : g) * d_q * d_k;
+            const uint16_t *qa = q_aug + ((int64_t)b * n_q + h) * d_q;
+            double *o = out + ((int64_t)b * n_q + h) * d_k;
+            for (int c = 0; c < d_k; ++c) {
+                double acc = 0.0;
+                for (int r = 0; r < d_q; ++r) acc += bf16_to_f64(qa[r]) * bf16_to_f64(W[(int64_t)r * d_k + c]);
+                o[c] = acc;
+            }
+        }
     return 0;
 }

@@ -416,3 +416,52 @@ def test_decode_paged_matches_sdpa_over_the_pages():
         v = v.repeat_interleave(s.n_q // s.n_v, dim=1).transpose(0, 1)[:, None]
         ref = F.scaled_dot_product_attention(d["q"][b].double()[:, None, None], k, v, scale=d["scale"])
         np.testing.assert_allclose(out[b], ref[:, 0, 0].numpy(), atol=1e-12, rtol=0)
+
+
+# ---------------------------------------------------------------- query and key of different widths
+
+def _up_inputs(seed, d_q, w_heads, shape=wl.DIFFQKV, T=40):
+    d = wl.random_decode_inputs(2, T, shape, seed=seed, seq_lens=[T, T // 2 + 1])
+    g = torch.Generator().manual_seed(seed + 1)
+    q_aug = torch.randn(2, shape.n_q, d_q, generator=g).to(torch.bfloat16)
+    w = (torch.randn(w_heads, d_q, shape.d_k, generator=g) / math.sqrt(shape.d_k)).to(torch.bfloat16)
+    return d, q_aug, w
+
+
+@pytest.mark.parametrize("w_heads", [1, 4])
+def test_up_projected_decode_matches_sdpa_on_projected_keys(w_heads):
+    """The pages' order: every K row projected up to d_q, then SDPA in fp64 (library routine)."""
+    s, d_q = wl.DIFFQKV, 96
+    d, q_aug, w = _up_inputs(71, d_q, w_heads)
+    scale = d_q ** -0.5
+    out = oracle.decode_up_projected(q_aug, w, d["k_cache"], d["v_cache"], d["seq_lens"], scale)
+    Wg = w.double().expand(s.n_k, -1, -1)                      # [n_k, d_q, d_k]
+    for b, T in enumerate(d["seq_lens"].tolist()):
+        kup = torch.einsum("grc,tgc->tgr", Wg, d["k_cache"][b, :T].double())          # [T, n_k, d_q]
+        kup = kup.repeat_interleave(s.n_q // s.n_k, dim=1).transpose(0, 1)[:, None]  # [n_q, 1, T, d_q]
+        v = d["v_cache"][b, :T].double().repeat_interleave(s.n_q // s.n_v, dim=1).transpose(0, 1)[:, None]
+        ref = F.scaled_dot_product_attention(q_aug[b].double()[:, None, None], kup, v, scale=scale)
+        np.testing.assert_allclose(out[b], ref[:, 0, 0].numpy(), atol=1e-12, rtol=0)
+
+
+def test_fold_query_moves_the_projection_onto_the_query():
+    """fold = einsum over each query head's K-head matrix, and <W^T q, k> = <q, W k> for every key."""
+    s, d_q = wl.DIFFQKV, 96
+    d, q_aug, w = _up_inputs(72, d_q, 4)
+    f = oracle.fold_query(q_aug, w, s.n_k)                     # [B, n_q, d_k]
+    Wh = w.double()[torch.arange(s.n_q) // (s.n_q // s.n_k)]  # [n_q, d_q, d_k]
+    np.testing.assert_allclose(f, torch.einsum("bhr,hrc->bhc", q_aug.double(), Wh).numpy(), atol=1e-12, rtol=0)
+    kk = d["k_cache"].double()[:, :, torch.arange(s.n_q) // (s.n_q // s.n_k)]   # [B, T, n_q, d_k]
+    folded = torch.einsum("bhc,bthc->bth", torch.from_numpy(f), kk)
+    projected = torch.einsum("bhr,bthr->bth", q_aug.double(), torch.einsum("hrc,bthc->bthr", Wh, kk))
+    np.testing.assert_allclose(folded.numpy(), projected.numpy(), atol=1e-10, rtol=0)
+
+
+def test_fold_query_identity_and_shared_matrix():
+    s = wl.DIFFQKV
+    q = wl.random_decode_inputs(2, 1, s, seed=73)["q"]
+    eye = torch.eye(s.d_k).to(torch.bfloat16)[None]
+    np.testing.assert_array_equal(oracle.fold_query(q, eye, s.n_k), q.double().numpy())
+    _, q_aug, w = _up_inputs(74, 40, 1)
+    shared = oracle.fold_query(q_aug, w, s.n_k)
+    np.testing.assert_array_equal(shared, oracle.fold_query(q_aug, w.expand(s.n_k, -1, -1).contiguous(), s.n_k))
