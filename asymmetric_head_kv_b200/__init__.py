@@ -21,7 +21,7 @@ from ._capi import DiffqkvError, Dims, DecodePlan, DecodeTuning, check, lib
 __all__ = [
     "decode", "decode_workspace", "decode_plan", "decode_from_host", "decode_topv", "decode_topv_workspace",
     "prefill_causal", "device_status", "selftest_wait_timeout", "DiffqkvError", "Dims", "library_path",
-    "decode_noalloc", "decode_append", "decode_paged", "prefill_causal_prefix",
+    "decode_noalloc", "decode_append", "decode_paged", "prefill_causal_prefix", "fold_query",
 ]
 
 library_path = _capi.LIB_PATH
@@ -182,6 +182,25 @@ def decode_paged(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor, 
                                     _ptr(block_table), max_blocks, page_size, num_pages, _ptr(seq_lens), msl,
                                     _ptr(out), _ptr(workspace), workspace.numel(), _stream_ptr(stream))
     check(st, "diffqkv_decode_paged")
+    return out
+
+
+def fold_query(q_aug: torch.Tensor, w_up: torch.Tensor, *, n_k: int, out: Optional[torch.Tensor] = None,
+               stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Folds the K up-projection into the query: q_aug [B, n_q, d_q] and w_up [w_heads, d_q, d_k]
+    (w_heads 1 or n_k) give the d_k-wide query W[h // (n_q // n_k)]^T q_aug[b, h], bf16 [B, n_q, d_k]."""
+    _bf16_dev(q_aug, "q_aug", 3)
+    _bf16_dev(w_up, "w_up", 3)
+    B, n_q, d_q = q_aug.shape
+    w_heads, d_q2, d_k = w_up.shape
+    if d_q != d_q2:
+        raise ValueError("q_aug and w_up disagree on d_q")
+    dims = make_dims(B, n_q, n_k, n_k, d_k, d_k, 1.0)
+    if out is None:
+        out = torch.empty((B, n_q, d_k), dtype=torch.bfloat16, device=q_aug.device)
+    st = lib().diffqkv_fold_query(ctypes.byref(dims), d_q, w_heads, _ptr(q_aug), _ptr(w_up), _ptr(out),
+                                  _stream_ptr(stream))
+    check(st, "diffqkv_fold_query")
     return out
 
 

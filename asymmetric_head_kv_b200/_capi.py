@@ -93,6 +93,7 @@ SIGNATURES = {
     "diffqkv_get_device_status": ([_P, ctypes.POINTER(_I32)], _I32),
     "diffqkv_selftest_wait_timeout": ([_I64, _P], _I32),
     "diffqkv_decode_noalloc": ([_DIMS, _P, _P, _P, _P, _I32, _I32, _P, _P], _I32),
+    "diffqkv_fold_query": ([_DIMS, _I32, _I32, _P, _P, _P, _P], _I32),
 }
 
 

@@ -457,6 +457,23 @@ def time_paths(ak, peaks, steps: int, warmup: int):
         assert ak.device_status() == 0
         del d, ws_p, out_p
 
+    # query fold for d_q != d_k (the K up-projection moved onto the query): 16 decode rows of 16 query
+    # heads, d_q = 192 (an augmented query of 3072 over 16 heads) onto d_k = 64; launch/latency bound
+    B, s_, d_q = 16, wl.DIFFQKV, 192
+    g = torch.Generator(device=dev).manual_seed(5)
+    q_aug = torch.randn(B, s_.n_q, d_q, generator=g, device=dev).to(torch.bfloat16)
+    w_up = (torch.randn(s_.n_k, d_q, s_.d_k, generator=g, device=dev) / 8).to(torch.bfloat16)
+    q_fold = torch.empty((B, s_.n_q, s_.d_k), dtype=torch.bfloat16, device=dev)
+    fn = lambda: ak.fold_query(q_aug, w_up, n_k=s_.n_k, out=q_fold)  # noqa: E731
+    for _ in range(max(3, warmup)):
+        fn()
+    ms = statistics.median(_timed_calls(fn, max(20, steps), flush))
+    nbytes = (q_aug.numel() + w_up.numel() + q_fold.numel()) * 2
+    res["fold_query_b16_dq192_dk64"] = {"us": ms * 1e3, "bytes": nbytes, "gbs": nbytes / (ms * 1e-3) / 1e9,
+                                        "bound": "launch/latency (L2 flushed between calls)",
+                                        "launches_per_call": 1}
+    del q_aug, w_up, q_fold
+
     w = wl.TOPV_64K
     d = wl.make_decode_inputs(w, dev)
     ws = ak.decode_topv_workspace(ak.make_dims(w.batch, w.shape.n_q, w.shape.n_k, w.shape.n_v, w.shape.d_k,

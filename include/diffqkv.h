@@ -173,6 +173,31 @@ diffqkv_status_t diffqkv_decode_paged(const diffqkv_dims_t *dims, const void *q,
                                       void *out, void *workspace, size_t workspace_bytes,
                                       diffqkv_stream_t stream);
 
+/*
+ * Query and key of different widths (section 3.4 Step 4, the Attend
+ * function): the pages bring each cached K row to the query width d_q with a
+ * feed-forward layer, k_up = W k, before the dot product.  For a linear layer
+ * without bias, <q, W k> = <W^T q, k>, so this call folds W into the query
+ * instead and the attention entry points run unchanged on the result:
+ *
+ *   q_aug [dims->batch, n_q, d_q]     augmented query (bf16, device)
+ *   w_up  [w_heads, d_q, d_k]         W of each K head (w_heads == n_k), or one
+ *                                     W shared by all K heads (w_heads == 1)
+ *   q_out [dims->batch, n_q, d_k]     q_out[b,h] = W[h/(n_q/n_k)]^T q_aug[b,h]
+ *
+ * Accumulation is fp32 and q_out is rounded to bf16 (nearest even).  Any
+ * number of query rows works (a prefill's [B, S] rows pass as B*S batch
+ * rows); the kernel runs on the CUDA cores and is sized for decode batches.
+ * dims->scale, n_v and d_v are not used (they must still be valid dims);
+ * the attention call that follows takes the scale of the d_q-wide dot product
+ * (1/sqrt(d_q) for the pages' formula).  d_k in {64, 128}, d_q >= 8 and a
+ * multiple of 8, w_heads in {1, n_k} (else DIFFQKV_ERR_INVALID_ARG /
+ * DIFFQKV_ERR_UNSUPPORTED); pointers 16-byte aligned.  Asynchronous on
+ * `stream`.
+ */
+diffqkv_status_t diffqkv_fold_query(const diffqkv_dims_t *dims, int32_t d_q, int32_t w_heads, const void *q_aug,
+                                    const void *w_up, void *q_out, diffqkv_stream_t stream);
+
 /* Optional launch controls for diffqkv_decode_ex (0 = library default). */
 typedef struct {
     int32_t grid_ctas;   /* CTAs of the split kernel (>= 1); changes the split points */

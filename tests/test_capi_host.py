@@ -184,3 +184,17 @@ def test_decode_paged_rejects_before_launch():
     assert call(max_blocks=1 << 20, page_size=1 << 12) == _capi.INVALID_ARG  # capacity past int32
     assert call(kn=0x8000) == _capi.INVALID_ARG                               # k_new without v_new
     assert call(q=0x1008) == _capi.MISALIGNED
+
+
+def test_fold_query_rejects_before_launch():
+    lib = _capi.lib()
+    d = dims()
+
+    def call(d_q=192, w_heads=4, q=0x1000, dd=d):
+        return lib.diffqkv_fold_query(ctypes.byref(dd), d_q, w_heads, q, 0x2000, 0x3000, None)
+    assert call(d_q=100) == _capi.INVALID_ARG     # not a multiple of 8
+    assert call(d_q=0) == _capi.INVALID_ARG
+    assert call(w_heads=2) == _capi.INVALID_ARG   # neither 1 nor n_k
+    assert call(q=None) == _capi.INVALID_ARG
+    assert call(q=0x1008) == _capi.MISALIGNED
+    assert call(dd=dims(d_k=96)) == _capi.UNSUPPORTED
