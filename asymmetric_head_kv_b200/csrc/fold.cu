@@ -15,8 +15,9 @@
 // at decode sizes, so it runs on the CUDA cores: one CTA per (row batch b,
 // K head g) covers the n_q/n_k query rows of the group.  Lane l of a warp owns
 // d_k/32 adjacent output columns, so a warp reads one W row (128 or 256 bytes)
-// per step; warps split the d_q sum into slices that are added in a fixed
-// order, so the result does not depend on timing.  Accumulation is fp32; the
+// per step; the 16 warps split the d_q sum into slices that are added in a
+// fixed order, so the result does not depend on timing, and each warp keeps
+// four steps of loads in flight (the kernel is load-latency bound).  Accumulation is fp32; the
 // folded query is rounded to bf16 (round to nearest even), the type of every
 // query the attention entry points take.
 #include <cuda_bf16.h>
@@ -29,7 +30,7 @@ namespace diffqkv {
 
 namespace {
 
-constexpr int kFoldThreads = 256;
+constexpr int kFoldThreads = 512;
 constexpr int kFoldWarps = kFoldThreads / 32;
 
 template <int DK>
@@ -61,6 +62,7 @@ __global__ void __launch_bounds__(kFoldThreads)
             const __nv_bfloat16 *qr = q_aug + ((size_t)b * n_q + g * qpk + j) * d_q;
             const int r0 = s * slice_len;
             const int r1 = min(d_q, r0 + slice_len);
+#pragma unroll 4
             for (int r = r0; r < r1; r += 8) {  // d_q and r0 are multiples of 8
                 const uint4 qv = __ldg(reinterpret_cast<const uint4 *>(qr + r));
                 const __nv_bfloat16 *qe = reinterpret_cast<const __nv_bfloat16 *>(&qv);
