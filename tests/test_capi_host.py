@@ -198,3 +198,35 @@ def test_fold_query_rejects_before_launch():
     assert call(q=None) == _capi.INVALID_ARG
     assert call(q=0x1008) == _capi.MISALIGNED
     assert call(dd=dims(d_k=96)) == _capi.UNSUPPORTED
+
+
+def test_paged_input_recipe_deals_distinct_pages():
+    """Each sequence holds ceil((seq_len + 1) / page_size) distinct pool pages, none shared, -1 elsewhere."""
+    import workloads as wl
+    d = wl.random_paged_inputs(4, 10, 16, wl.DIFFQKV, seed=5, seq_lens=[0, 15, 16, 150], spare_pages=2)
+    table = d["block_table"]
+    held = [(t + 1 + 15) // 16 for t in (0, 15, 16, 150)]
+    assert d["num_pages"] == sum(held) + 2
+    used = []
+    for b, n in enumerate(held):
+        assert (table[b, :n] >= 0).all() and (table[b, n:] == -1).all()
+        used += table[b, :n].tolist()
+    assert len(set(used)) == len(used) and max(used) < d["num_pages"]
+    assert d["k_pages"].shape == (d["num_pages"], 16, 4, 64) and d["v_pages"].shape == (d["num_pages"], 16, 16, 128)
+
+
+def test_python_bindings_reject_host_tensors_and_bad_shapes():
+    import torch
+    q = torch.zeros(2, 16, 64, dtype=torch.bfloat16)
+    kp = torch.zeros(8, 16, 4, 64, dtype=torch.bfloat16)
+    vp = torch.zeros(8, 16, 16, 128, dtype=torch.bfloat16)
+    bt = torch.zeros(2, 4, dtype=torch.int32)
+    lens = torch.zeros(2, dtype=torch.int32)
+    with pytest.raises(ValueError, match="CUDA"):
+        ak.decode_paged(q, kp, vp, bt, lens)
+    with pytest.raises(TypeError, match="bfloat16"):
+        ak.decode_paged(q.float(), kp, vp, bt, lens)
+    with pytest.raises(TypeError, match="bfloat16"):
+        ak.fold_query(q.float(), torch.zeros(4, 64, 64), n_k=4)
+    with pytest.raises(ValueError, match="CUDA"):
+        ak.fold_query(q, torch.zeros(4, 64, 64, dtype=torch.bfloat16), n_k=4)
