@@ -230,3 +230,26 @@ def test_python_bindings_reject_host_tensors_and_bad_shapes():
         ak.fold_query(q.float(), torch.zeros(4, 64, 64), n_k=4)
     with pytest.raises(ValueError, match="CUDA"):
         ak.fold_query(q, torch.zeros(4, 64, 64, dtype=torch.bfloat16), n_k=4)
+
+
+def test_header_is_plain_c_and_a_c_program_links(tmp_path):
+    """include/diffqkv.h compiles as strict C99 (no C++ in the ABI) and a C program links and calls the library."""
+    import os
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no gcc")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    src = tmp_path / "abi.c"
+    src.write_text('#include "diffqkv.h"\n#include <stdio.h>\n'
+                   'int main(void) { printf("%s %d\\n", diffqkv_status_string(DIFFQKV_ERR_DEVICE_PAGE), '
+                   'diffqkv_version() >= 10000); return 0; }\n')
+    pkg = os.path.dirname(_capi.LIB_PATH)
+    exe = tmp_path / "abi"
+    r = subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", os.path.join(root, "include"),
+                        str(src), "-L", pkg, "-ldiffqkv", "-Wl,-rpath," + pkg, "-o", str(exe)],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert out.returncode == 0 and out.stdout.strip() == "DIFFQKV_ERR_DEVICE_PAGE 1"
