@@ -269,7 +269,8 @@ size_t diffqkv_decode_topv_workspace_size(const diffqkv_dims_t *dims, int32_t t_
  * other buffers and the workspace 16-byte aligned (DIFFQKV_ERR_MISALIGNED).
  * max_seq_len is accepted for symmetry with diffqkv_decode and ignored: the
  * kernels read the lengths from seq_lens on the device.  Lengths outside
- * [0, t_max] are clamped to that range.  A row with length 0 gets a zero
+ * [0, t_max] are clamped to that range without touching the device error
+ * word (diffqkv_decode flags them).  A row with length 0 gets a zero
  * output and an all -1 index row.  Launches four kernels on `stream`
  * (chained with programmatic dependent launch);
  * returns once they are queued.
