@@ -21,7 +21,7 @@ from ._capi import DiffqkvError, Dims, DecodePlan, DecodeTuning, check, lib
 __all__ = [
     "decode", "decode_workspace", "decode_plan", "decode_from_host", "decode_topv", "decode_topv_workspace",
     "prefill_causal", "device_status", "selftest_wait_timeout", "DiffqkvError", "Dims", "library_path",
-    "decode_noalloc", "decode_append", "decode_paged", "prefill_causal_prefix", "fold_query",
+    "decode_noalloc", "decode_append", "decode_paged", "prefill_causal_prefix", "fold_query", "workspace_status",
 ]
 
 library_path = _capi.LIB_PATH
@@ -224,10 +224,11 @@ def decode_from_host(q_host, k_host, v_host, seq_lens_host, out_host, dev_buffer
 
 
 def decode_topv_workspace(dims: Dims, t_max: int, topk: int, device="cuda") -> torch.Tensor:
+    """Workspace for :func:`decode_topv`; zero-filled (its 256-byte header holds the error word)."""
     n = lib().diffqkv_decode_topv_workspace_size(ctypes.byref(dims), t_max, topk)
     if n == 0:
         raise DiffqkvError(_capi.INVALID_ARG, "decode_topv_workspace_size")
-    return torch.empty(n, dtype=torch.uint8, device=device)
+    return torch.zeros(n, dtype=torch.uint8, device=device)
 
 
 def decode_topv(q, k_cache, v_cache, seq_lens, topk: int, *, scale: Optional[float] = None,
@@ -265,9 +266,12 @@ def decode_topv(q, k_cache, v_cache, seq_lens, topk: int, *, scale: Optional[flo
     return out, idx_out
 
 
-def prefill_causal(q, k, v, *, scale: Optional[float] = None, out=None,
+def prefill_causal(q, k, v, *, scale: Optional[float] = None, out=None, status: Optional[torch.Tensor] = None,
                    stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
-    """Causal prefill: q [B,S,n_q,d_k], k [B,S,n_k,d_k], v [B,S,n_v,d_v] -> out [B,S,n_q,d_v] (bf16)."""
+    """Causal prefill: q [B,S,n_q,d_k], k [B,S,n_k,d_k], v [B,S,n_v,d_v] -> out [B,S,n_q,d_v] (bf16).
+
+    ``status``: an int32 CUDA tensor of one element, zero, that receives this call's device-side
+    error instead of the per-device word (``diffqkv_prefill_causal_ex``)."""
     _bf16_dev(q, "q", 4)
     _bf16_dev(k, "k", 4)
     _bf16_dev(v, "v", 4)
@@ -278,10 +282,20 @@ def prefill_causal(q, k, v, *, scale: Optional[float] = None, out=None,
     dims = make_dims(B, n_q, n_k, n_v, d_k, d_v, d_k ** -0.5 if scale is None else scale)
     if out is None:
         out = torch.empty((B, S, n_q, d_v), dtype=torch.bfloat16, device=q.device)
-    st = lib().diffqkv_prefill_causal(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), S, _ptr(out),
-                                      _stream_ptr(stream))
+    if status is not None:
+        _status_word(status)
+        st = lib().diffqkv_prefill_causal_ex(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), 0, S, _ptr(out),
+                                             _ptr(status), _stream_ptr(stream))
+    else:
+        st = lib().diffqkv_prefill_causal(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), S, _ptr(out),
+                                          _stream_ptr(stream))
     check(st, "diffqkv_prefill_causal")
     return out
+
+
+def _status_word(t: torch.Tensor):
+    if t.dtype != torch.int32 or not t.is_cuda or t.numel() < 1:
+        raise TypeError("status must be an int32 CUDA tensor with at least one element")
 
 
 def prefill_causal_prefix(q, k, v, prefix_len: int, *, scale: Optional[float] = None, out=None,
@@ -305,8 +319,20 @@ def prefill_causal_prefix(q, k, v, prefix_len: int, *, scale: Optional[float] = 
     return out
 
 
+def workspace_status(workspace: torch.Tensor, stream: Optional[torch.cuda.Stream] = None) -> int:
+    """Synchronises the stream and returns (and clears) the error word of a decode or top-v workspace:
+    the first device-side error of the calls that used it since the last read."""
+    if workspace.dtype != torch.uint8 or not workspace.is_cuda:
+        raise TypeError("workspace must be a uint8 CUDA tensor")
+    v = ctypes.c_int32(0)
+    check(lib().diffqkv_workspace_status(_ptr(workspace), workspace.numel(), _stream_ptr(stream), ctypes.byref(v)),
+          "diffqkv_workspace_status")
+    return v.value
+
+
 def device_status(stream: Optional[torch.cuda.Stream] = None) -> int:
-    """Synchronises the stream and returns (and clears) the device error word."""
+    """Synchronises the stream and returns (and clears) the per-device error word (the calls without a
+    word of their own: prefill without ``status``, the allocation-free decode, the wait self-test)."""
     v = ctypes.c_int32(0)
     check(lib().diffqkv_get_device_status(_stream_ptr(stream), ctypes.byref(v)), "diffqkv_get_device_status")
     return v.value

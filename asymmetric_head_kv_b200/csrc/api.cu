@@ -185,7 +185,7 @@ const char *diffqkv_status_string(int32_t status) {
     }
 }
 
-int32_t diffqkv_version(void) { return 10000; }
+int32_t diffqkv_version(void) { return 10100; }
 
 size_t diffqkv_decode_workspace_size(const diffqkv_dims_t *dims) { return diffqkv::decode_workspace_size(dims); }
 
@@ -248,34 +248,9 @@ diffqkv_status_t diffqkv_decode_from_host(const diffqkv_dims_t *dims, const void
                                           int32_t max_seq_len, void *out_host, void *q_dev, void *k_cache_dev,
                                           void *v_cache_dev, int32_t *seq_lens_dev, void *out_dev,
                                           void *workspace, size_t workspace_bytes, diffqkv_stream_t stream) {
-    diffqkv_status_t st = diffqkv::validate_dims(dims);
-    if (st != DIFFQKV_OK) return st;
-    if (!q_host || !k_cache_host || !v_cache_host || !seq_lens_host || !out_host || t_max < 1)
-        return DIFFQKV_ERR_INVALID_ARG;
-    const size_t B = dims->batch;
-    const size_t q_bytes = B * dims->n_q * dims->d_k * 2;
-    const size_t k_bytes = B * (size_t)t_max * dims->n_k * dims->d_k * 2;
-    const size_t v_bytes = B * (size_t)t_max * dims->n_v * dims->d_v * 2;
-    const size_t o_bytes = B * dims->n_q * dims->d_v * 2;
-    if (!q_dev || !k_cache_dev || !v_cache_dev || !seq_lens_dev || !out_dev) return DIFFQKV_ERR_INVALID_ARG;
-    cudaStream_t s = (cudaStream_t)stream;
-    // one plain async copy per buffer
-    if (cudaMemcpyAsync(q_dev, q_host, q_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-        cudaMemcpyAsync(k_cache_dev, k_cache_host, k_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-        cudaMemcpyAsync(v_cache_dev, v_cache_host, v_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-        cudaMemcpyAsync(seq_lens_dev, seq_lens_host, B * sizeof(int32_t), cudaMemcpyHostToDevice, s) !=
-            cudaSuccess) {
-        cudaGetLastError();
-        return DIFFQKV_ERR_CUDA;
-    }
-    st = diffqkv::decode_launch(dims, q_dev, k_cache_dev, v_cache_dev, seq_lens_dev, t_max, max_seq_len, out_dev,
-                                workspace, workspace_bytes, nullptr, s);
-    if (st != DIFFQKV_OK) return st;
-    if (cudaMemcpyAsync(out_host, out_dev, o_bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess) {
-        cudaGetLastError();
-        return DIFFQKV_ERR_CUDA;
-    }
-    return DIFFQKV_OK;
+    return diffqkv::decode_from_host_launch(dims, q_host, k_cache_host, v_cache_host, seq_lens_host, t_max,
+                                            max_seq_len, out_host, q_dev, k_cache_dev, v_cache_dev, seq_lens_dev,
+                                            out_dev, workspace, workspace_bytes, (cudaStream_t)stream);
 }
 
 size_t diffqkv_decode_topv_workspace_size(const diffqkv_dims_t *dims, int32_t t_max, int32_t topk) {
@@ -308,6 +283,29 @@ diffqkv_status_t diffqkv_prefill_causal_prefix(const diffqkv_dims_t *dims, const
                                                const void *v, int32_t prefix_len, int32_t seq_len, void *out,
                                                diffqkv_stream_t stream) {
     return diffqkv::prefill_launch(dims, q, k, v, seq_len, out, (cudaStream_t)stream, prefix_len);
+}
+
+diffqkv_status_t diffqkv_prefill_causal_ex(const diffqkv_dims_t *dims, const void *q, const void *k,
+                                           const void *v, int32_t prefix_len, int32_t seq_len, void *out,
+                                           int32_t *device_status_word, diffqkv_stream_t stream) {
+    return diffqkv::prefill_launch(dims, q, k, v, seq_len, out, (cudaStream_t)stream, prefix_len,
+                                   device_status_word);
+}
+
+diffqkv_status_t diffqkv_workspace_status(void *workspace, size_t workspace_bytes, diffqkv_stream_t stream,
+                                          int32_t *device_status) {
+    if (!device_status || !workspace || workspace_bytes < 256) return DIFFQKV_ERR_INVALID_ARG;
+    if (!diffqkv::aligned16(workspace)) return DIFFQKV_ERR_MISALIGNED;
+    cudaStream_t s = (cudaStream_t)stream;
+    int32_t v = 0;
+    if (cudaStreamSynchronize(s) != cudaSuccess ||
+        cudaMemcpyAsync(&v, workspace, sizeof v, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaMemsetAsync(workspace, 0, sizeof v, s) != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess) {
+        cudaGetLastError();
+        return DIFFQKV_ERR_CUDA;
+    }
+    *device_status = v;
+    return DIFFQKV_OK;
 }
 
 diffqkv_status_t diffqkv_get_device_status(diffqkv_stream_t stream, int32_t *device_status) {

@@ -759,13 +759,29 @@ diffqkv_status_t decode_plan(const diffqkv_dims_t *d, int32_t t_max, int32_t max
     return DIFFQKV_OK;
 }
 
-diffqkv_status_t decode_launch(const diffqkv_dims_t *d, const void *q, const void *k_cache, const void *v_cache,
-                               const int32_t *seq_lens, int32_t t_max, int32_t max_seq_len, void *out,
-                               void *workspace, size_t workspace_bytes, const diffqkv_decode_tuning_t *tuning,
-                               cudaStream_t stream, const void *k_new, const void *v_new, const PagedCache *paged) {
+namespace {
+
+// A checked, fully encoded decode launch: everything decode_launch needs except the stream.
+struct DecodeLaunch {
+    KernelFn fn = nullptr;
+    CUtensorMap tm_k, tm_v;
+    DecodeArgs a;
+    int grid = 0, threads = 0;
+    size_t smem = 0;
+};
+
+// Every host-side check of a decode call (dims, pointers, alignment, workspace, device, plan) and
+// the tensor-map encoding; nothing is enqueued.  The device status word is the workspace's first
+// 32-bit word (inside its 256-byte header), so every workspace reports its own calls' errors.
+diffqkv_status_t decode_prepare(const diffqkv_dims_t *d, const void *q, const void *k_cache, const void *v_cache,
+                                const int32_t *seq_lens, int32_t t_max, int32_t max_seq_len, void *out,
+                                void *workspace, size_t workspace_bytes, const diffqkv_decode_tuning_t *tuning,
+                                const void *k_new, const void *v_new, const PagedCache *paged, DecodeLaunch *L) {
     diffqkv_status_t st = validate_dims(d);
     if (st != DIFFQKV_OK) return st;
     if (!q || !k_cache || !v_cache || !seq_lens || !out || t_max < 1) return DIFFQKV_ERR_INVALID_ARG;
+    L->fn = pick_kernel(d->d_k, d->d_v, d->n_q / d->n_k);
+    if (!L->fn) return DIFFQKV_ERR_UNSUPPORTED;
     if (paged) {
         if (!paged->block_table || paged->max_blocks < 1 || paged->page_size < 1 || paged->num_pages < 1 ||
             (long long)paged->max_blocks * paged->page_size != t_max)
@@ -787,24 +803,20 @@ diffqkv_status_t decode_launch(const diffqkv_dims_t *d, const void *q, const voi
     diffqkv_decode_plan_t plan;
     st = decode_plan(d, t_max, max_seq_len, dev.num_sms, tuning, &plan);
     if (st != DIFFQKV_OK) return st;
-    const int qpk = d->n_q / d->n_k;
-    KernelFn fn = pick_kernel(d->d_k, d->d_v, qpk);
-    if (!fn) return DIFFQKV_ERR_UNSUPPORTED;
 
     // contiguous caches: one box per tile over [B, t_max, heads, d]; paged: sub-boxes over
     // [num_pages, page_size, heads, d], each gcd(tile, page_size) positions inside one page
     const int sub_rows = paged ? std::gcd(plan.tile_tokens, paged->page_size) : plan.tile_tokens;
     const uint64_t rows_dim = paged ? (uint64_t)paged->page_size : (uint64_t)t_max;
     const uint64_t outer_dim = paged ? (uint64_t)paged->num_pages : (uint64_t)d->batch;
-    CUtensorMap tm_k, tm_v;
-    st = make_tensor_map_4d(&tm_k, k_cache, d->d_k, d->n_k, rows_dim, outer_dim, d->d_k, 1, sub_rows, 1,
+    st = make_tensor_map_4d(&L->tm_k, k_cache, d->d_k, d->n_k, rows_dim, outer_dim, d->d_k, 1, sub_rows, 1,
                             CU_TENSOR_MAP_SWIZZLE_NONE, k_promotion(d));
     if (st != DIFFQKV_OK) return st;
-    st = make_tensor_map_4d(&tm_v, v_cache, d->d_v, d->n_v, rows_dim, outer_dim, d->d_v, plan.v_heads_per_tile,
+    st = make_tensor_map_4d(&L->tm_v, v_cache, d->d_v, d->n_v, rows_dim, outer_dim, d->d_v, plan.v_heads_per_tile,
                             sub_rows, 1, CU_TENSOR_MAP_SWIZZLE_NONE);
     if (st != DIFFQKV_OK) return st;
 
-    DecodeArgs a;
+    DecodeArgs &a = L->a;
     if (paged) {
         a.block_table = paged->block_table;
         a.max_blocks = paged->max_blocks;
@@ -827,7 +839,7 @@ diffqkv_status_t decode_launch(const diffqkv_dims_t *d, const void *q, const voi
     a.out = static_cast<__nv_bfloat16 *>(out);
     a.counters = reinterpret_cast<uint32_t *>(ws + kWorkspaceHeader);
     a.partials = reinterpret_cast<float *>(ws + kWorkspaceHeader + align_up(units * sizeof(uint32_t), 256));
-    a.status = dev.status_word;
+    a.status = reinterpret_cast<int32_t *>(ws);  // the workspace's own error word
     a.batch = d->batch;
     a.n_q = d->n_q;
     a.n_k = d->n_k;
@@ -842,10 +854,63 @@ diffqkv_status_t decode_launch(const diffqkv_dims_t *d, const void *q, const voi
     a.stage_stride = (uint32_t)align_up(a.stage_bytes, 1024);
     a.scale_log2 = (float)((double)d->scale * 1.4426950408889634);
     a.wait_limit_ns = kWaitLimitNs;
+    L->grid = plan.grid_ctas;
+    L->threads = plan.threads;
+    L->smem = (size_t)plan.smem_bytes;
+    if (ensure_dynamic_smem((const void *)L->fn, (int)plan.smem_bytes) != DIFFQKV_OK) return DIFFQKV_ERR_CUDA;
+    return DIFFQKV_OK;
+}
 
-    if (ensure_dynamic_smem((const void *)fn, (int)plan.smem_bytes) != DIFFQKV_OK) return DIFFQKV_ERR_CUDA;
-    fn<<<plan.grid_ctas, plan.threads, plan.smem_bytes, stream>>>(tm_k, tm_v, a);
+diffqkv_status_t decode_enqueue(const DecodeLaunch &L, cudaStream_t stream) {
+    L.fn<<<L.grid, L.threads, L.smem, stream>>>(L.tm_k, L.tm_v, L.a);
     if (cudaGetLastError() != cudaSuccess) return DIFFQKV_ERR_CUDA;
+    return DIFFQKV_OK;
+}
+
+}  // namespace
+
+diffqkv_status_t decode_launch(const diffqkv_dims_t *d, const void *q, const void *k_cache, const void *v_cache,
+                               const int32_t *seq_lens, int32_t t_max, int32_t max_seq_len, void *out,
+                               void *workspace, size_t workspace_bytes, const diffqkv_decode_tuning_t *tuning,
+                               cudaStream_t stream, const void *k_new, const void *v_new, const PagedCache *paged) {
+    DecodeLaunch L;
+    const diffqkv_status_t st = decode_prepare(d, q, k_cache, v_cache, seq_lens, t_max, max_seq_len, out, workspace,
+                                               workspace_bytes, tuning, k_new, v_new, paged, &L);
+    if (st != DIFFQKV_OK) return st;
+    return decode_enqueue(L, stream);
+}
+
+diffqkv_status_t decode_from_host_launch(const diffqkv_dims_t *d, const void *q_host, const void *k_host,
+                                         const void *v_host, const int32_t *seq_lens_host, int32_t t_max,
+                                         int32_t max_seq_len, void *out_host, void *q_dev, void *k_dev, void *v_dev,
+                                         int32_t *seq_lens_dev, void *out_dev, void *workspace,
+                                         size_t workspace_bytes, cudaStream_t stream) {
+    if (!q_host || !k_host || !v_host || !seq_lens_host || !out_host) return DIFFQKV_ERR_INVALID_ARG;
+    // every argument check of the decode runs before the first copy is enqueued
+    DecodeLaunch L;
+    diffqkv_status_t st = decode_prepare(d, q_dev, k_dev, v_dev, seq_lens_dev, t_max, max_seq_len, out_dev,
+                                         workspace, workspace_bytes, nullptr, nullptr, nullptr, nullptr, &L);
+    if (st != DIFFQKV_OK) return st;
+    const size_t B = d->batch;
+    const size_t q_bytes = B * d->n_q * d->d_k * 2;
+    const size_t k_bytes = B * (size_t)t_max * d->n_k * d->d_k * 2;
+    const size_t v_bytes = B * (size_t)t_max * d->n_v * d->d_v * 2;
+    const size_t o_bytes = B * d->n_q * d->d_v * 2;
+    // one plain async copy per buffer
+    if (cudaMemcpyAsync(q_dev, q_host, q_bytes, cudaMemcpyHostToDevice, stream) != cudaSuccess ||
+        cudaMemcpyAsync(k_dev, k_host, k_bytes, cudaMemcpyHostToDevice, stream) != cudaSuccess ||
+        cudaMemcpyAsync(v_dev, v_host, v_bytes, cudaMemcpyHostToDevice, stream) != cudaSuccess ||
+        cudaMemcpyAsync(seq_lens_dev, seq_lens_host, B * sizeof(int32_t), cudaMemcpyHostToDevice, stream) !=
+            cudaSuccess) {
+        cudaGetLastError();
+        return DIFFQKV_ERR_CUDA;
+    }
+    st = decode_enqueue(L, stream);
+    if (st != DIFFQKV_OK) return st;
+    if (cudaMemcpyAsync(out_host, out_dev, o_bytes, cudaMemcpyDeviceToHost, stream) != cudaSuccess) {
+        cudaGetLastError();
+        return DIFFQKV_ERR_CUDA;
+    }
     return DIFFQKV_OK;
 }
 

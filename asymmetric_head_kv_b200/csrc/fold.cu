@@ -50,15 +50,19 @@ __global__ void __launch_bounds__(kFoldThreads)
     const int slices = qpk >= kFoldWarps ? 1 : kFoldWarps / qpk;
     const int slice_len = ((d_q + slices - 1) / slices + 7) / 8 * 8;
 
-    // rows are handled in rounds of (kFoldWarps / slices) rows; partials of one round live in part[]
+    // rows are handled in rounds of (kFoldWarps / slices) rows; partials of one round live in part[].
+    // When slices does not divide kFoldWarps (n_q / n_k = 3, 5, ...), the last
+    // kFoldWarps - slices * rows_per_round warps get no (row, slice) pair: they
+    // neither compute nor write part[], whose slots all belong to other warps.
     const int rows_per_round = kFoldWarps / slices;
+    const bool has_slot = warp < slices * rows_per_round;
     for (int row0 = 0; row0 < qpk; row0 += rows_per_round) {
         const int j = row0 + warp / slices;  // query row of the group
         const int s = warp % slices;
         float acc[V];
 #pragma unroll
         for (int v = 0; v < V; ++v) acc[v] = 0.f;
-        if (j < qpk) {
+        if (has_slot && j < qpk) {
             const __nv_bfloat16 *qr = q_aug + ((size_t)b * n_q + g * qpk + j) * d_q;
             const int r0 = s * slice_len;
             const int r1 = min(d_q, r0 + slice_len);
@@ -87,9 +91,11 @@ __global__ void __launch_bounds__(kFoldThreads)
             }
         }
         // partial of (slice s, row warp / slices) -> part; then sum the slices in order
-        float *dst = part + ((size_t)s * rows_per_round + warp / slices) * DK + lane * V;
+        if (has_slot) {
+            float *dst = part + ((size_t)s * rows_per_round + warp / slices) * DK + lane * V;
 #pragma unroll
-        for (int v = 0; v < V; ++v) dst[v] = acc[v];
+            for (int v = 0; v < V; ++v) dst[v] = acc[v];
+        }
         __syncthreads();
         for (int t = threadIdx.x; t < rows_per_round * DK; t += kFoldThreads) {
             const int jj = row0 + t / DK;

@@ -64,6 +64,13 @@ diffqkv_status_t decode_launch(const diffqkv_dims_t *d, const void *q, const voi
                                const void *k_new = nullptr, const void *v_new = nullptr,
                                const PagedCache *paged = nullptr);
 
+// diffqkv_decode_from_host: all checks of the decode run before the first copy is enqueued.
+diffqkv_status_t decode_from_host_launch(const diffqkv_dims_t *d, const void *q_host, const void *k_host,
+                                         const void *v_host, const int32_t *seq_lens_host, int32_t t_max,
+                                         int32_t max_seq_len, void *out_host, void *q_dev, void *k_dev, void *v_dev,
+                                         int32_t *seq_lens_dev, void *out_dev, void *workspace,
+                                         size_t workspace_bytes, cudaStream_t stream);
+
 diffqkv_status_t decode_noalloc_launch(const diffqkv_dims_t *d, const void *q, const void *k_cache,
                                        const void *v_cache, const int32_t *seq_lens, int32_t t_max,
                                        int32_t max_seq_len, void *out, cudaStream_t stream);
@@ -76,8 +83,10 @@ diffqkv_status_t topv_launch(const diffqkv_dims_t *d, const void *q, const void 
                              cudaStream_t stream, int32_t flags = 0);
 
 // prefill.cu
+// status: device word the kernel reports into (NULL: the per-device word).
 diffqkv_status_t prefill_launch(const diffqkv_dims_t *d, const void *q, const void *k, const void *v,
-                                int32_t seq_len, void *out, cudaStream_t stream, int32_t prefix_len = 0);
+                                int32_t seq_len, void *out, cudaStream_t stream, int32_t prefix_len = 0,
+                                int32_t *status = nullptr);
 
 // api.cu
 diffqkv_status_t wait_timeout_selftest_launch(int64_t timeout_ns, cudaStream_t stream);

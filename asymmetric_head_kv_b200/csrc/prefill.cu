@@ -692,13 +692,15 @@ bool pick(int dk, int dv, Plan *p) {
 }  // namespace
 
 diffqkv_status_t prefill_launch(const diffqkv_dims_t *d, const void *q, const void *k, const void *v, int32_t seq_len,
-                                void *out, cudaStream_t stream, int32_t prefix_len) {
+                                void *out, cudaStream_t stream, int32_t prefix_len, int32_t *status) {
     diffqkv_status_t st = validate_dims(d);
     if (st != DIFFQKV_OK) return st;
     if (!q || !k || !v || !out || seq_len < 1 || prefix_len < 0) return DIFFQKV_ERR_INVALID_ARG;
     if ((long long)prefix_len + seq_len > 0x7fffffffLL) return DIFFQKV_ERR_UNSUPPORTED;
     const int32_t kv_len = prefix_len + seq_len;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return DIFFQKV_ERR_MISALIGNED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+        (reinterpret_cast<uintptr_t>(status) & 3u))
+        return DIFFQKV_ERR_MISALIGNED;
     Plan plan;
     if (!pick(d->d_k, d->d_v, &plan)) return DIFFQKV_ERR_UNSUPPORTED;
     DeviceInfo dev;
@@ -718,7 +720,7 @@ diffqkv_status_t prefill_launch(const diffqkv_dims_t *d, const void *q, const vo
 
     PrefillArgs a;
     a.out = static_cast<__nv_bfloat16 *>(out);
-    a.status = dev.status_word;
+    a.status = status ? status : dev.status_word;  // the caller's word, else the device's
     a.batch = d->batch;
     a.seq = seq_len;
     a.prefix = prefix_len;

@@ -2,7 +2,7 @@
 //
 // "Selective V Cache Fetching" (Sigma paper, structured summary page): after
 // the scores are computed from the full (thin) K cache, only the V rows of the
-// top-k scoring positions are read; the other positions are treated as zero.
+// top-k scoring positions are read; positions outside that set contribute nothing.
 // The softmax is renormalised over the kept positions, and the positions are
 // ranked by the EXACT dot product q.k (ties toward the lower position) so the
 // selected set is unique and reproducible.
@@ -197,8 +197,12 @@ __global__ void __launch_bounds__(kScoreThreads + 32, score_ctas_per_sm(DK)) top
     const int unit = blockIdx.x;
     const int b = unit / a.n_k;
     const int g = unit % a.n_k;
-    const int T = clamp_len(__ldg(a.seq_lens + b), a.t_max);
+    const int raw_len = __ldg(a.seq_lens + b);
+    const int T = clamp_len(raw_len, a.t_max);
     const int tid = threadIdx.x;
+    // a length outside [0, t_max] is clamped (every kernel of the call clamps it the same way) and
+    // flagged once per sequence
+    if (g == 0 && blockIdx.y == 0 && tid == 0 && raw_len != T) record_error(a.status, DIFFQKV_ERR_DEVICE_SEQLEN);
     const int warp = tid >> 5, lane = tid & 31;
     const int ntiles = (T + kScoreTile - 1) / kScoreTile;
     const int tb = (int)(((long long)ntiles * blockIdx.y) / gridDim.y);
@@ -1166,7 +1170,7 @@ diffqkv_status_t topv_launch(const diffqkv_dims_t *d, const void *q, const void 
     a.seq_lens = seq_lens;
     a.out = static_cast<__nv_bfloat16 *>(out);
     a.idx_out = idx_out;
-    a.status = dev.status_word;
+    a.status = reinterpret_cast<int32_t *>(workspace);  // the workspace's own error word (header word 0)
     a.batch = d->batch;
     a.n_q = d->n_q;
     a.n_k = d->n_k;

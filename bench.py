@@ -106,7 +106,10 @@ class ClockSampler:
         "hw_power_brake_slowdown": 0x80, "display_clock_setting": 0x100,
     }
 
-    def __init__(self, device_index: int):
+    def __init__(self, device_index: int, period_s: float = 0.0002):
+        # the headline's timed region can be a few milliseconds (20 steps of ~0.36 ms): sample
+        # every 0.2 ms so that it still holds ten or more readings
+        self.period_s = period_s
         self.samples, self.reasons, self.max_mhz = [], set(), None
         self._stop = threading.Event()
         try:
@@ -128,7 +131,7 @@ class ClockSampler:
                         self.reasons.add(name)
             except Exception:
                 pass
-            time.sleep(0.02)
+            time.sleep(self.period_s)
 
     def __enter__(self):
         if self.nv:
@@ -198,7 +201,7 @@ def time_decode(ak, w: wl.DecodeWorkload, steps: int, warmup: int, world: int, s
     for _ in range(max(warmup, 3)):
         step()
     torch.cuda.synchronize()
-    assert ak.device_status() == 0
+    assert ak.workspace_status(ws) == 0
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     barrier(world)
@@ -281,6 +284,16 @@ def oracle_sample_rate(w: wl.DecodeWorkload, d_cpu: dict, budget_s: float):
                       f"fp64 C oracle, {dt:.2f} s", "seconds": dt}
 
 
+def bench_config(world: int) -> dict:
+    """The workload both arms (the kernels and the oracle) measure, under the same keys."""
+    s = WORKLOAD.shape
+    return {"workload": WORKLOAD.name, "batch_per_gpu": WORKLOAD.batch, "context": WORKLOAD.t_max,
+            "n_q": s.n_q, "n_k": s.n_k, "n_v": s.n_v, "d_k": s.d_k, "d_v": s.d_v,
+            "parallelism": f"replicas x{world}",
+            "l2": "inputs (2.42 GB) larger than L2 (126 MB); no flush",
+            "kv_bytes_per_gpu_step": wl.decode_kv_bytes(s, WORKLOAD.seq_lens())}
+
+
 def run_reference(args, world, rank):
     if rank != 0:
         return
@@ -297,8 +310,7 @@ def run_reference(args, world, rank):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD.name, "batch": WORKLOAD.batch, "context": WORKLOAD.t_max,
-                   "n_q": 16, "n_k": 4, "n_v": 16, "d_k": 64, "d_v": 128},
+        "config": bench_config(world),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": info["cores"], "kind": "oracle",
                          "sample": info["sample"] + " per step"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -335,6 +347,7 @@ def run_profile_case(name: str, launches: int = 4):
         for _ in range(launches):
             ak.decode(d["q"], d["k_cache"], d["v_cache"], d["seq_lens"], scale=d["scale"], workspace=ws)
         what = f"kv bytes/launch {wl.decode_kv_bytes(w.shape, d['seq_lens'])}"
+        assert ak.workspace_status(ws) == 0
     torch.cuda.synchronize()
     assert ak.device_status() == 0
     print(f"profile case {name}: {launches} launches, {what}")
@@ -433,7 +446,7 @@ def time_paths(ak, peaks, steps: int, warmup: int):
     res["decode_append_b16_t32768"] = {"us": ms * 1e3, "algorithmic_bytes": nbytes,
                                        "gbs": nbytes / (ms * 1e-3) / 1e9, "bound": "hbm", "peak_gbs": hbm,
                                        "frac": nbytes / (ms * 1e-3) / 1e9 / hbm, "launches_per_call": 1}
-    assert ak.device_status() == 0
+    assert ak.workspace_status(ws_d) == 0 and ak.device_status() == 0
     del d, ws_d, out_d
 
     # the same 16 x 32768 decode over paged caches: K and V page pools with one block table, pages
@@ -454,7 +467,7 @@ def time_paths(ak, peaks, steps: int, warmup: int):
         res[f"decode_paged_b16_t32768_p{page_size}"] = {
             "us": ms * 1e3, "kv_bytes": nbytes, "gbs": nbytes / (ms * 1e-3) / 1e9, "bound": "hbm",
             "peak_gbs": hbm, "frac": nbytes / (ms * 1e-3) / 1e9 / hbm, "launches_per_call": 1}
-        assert ak.device_status() == 0
+        assert ak.workspace_status(ws_p) == 0
         del d, ws_p, out_p
 
     # query fold for d_q != d_k (the K up-projection moved onto the query): 16 decode rows of 16 query
@@ -497,7 +510,7 @@ def time_paths(ak, peaks, steps: int, warmup: int):
     res[w.name + "_full_weights"] = {"us": ms * 1e3, "algorithmic_bytes": nbytes,
                                      "gbs": nbytes / (ms * 1e-3) / 1e9, "bound": "hbm", "peak_gbs": hbm,
                                      "frac": nbytes / (ms * 1e-3) / 1e9 / hbm, "launches_per_call": 4}
-    assert ak.device_status() == 0
+    assert ak.workspace_status(ws) == 0
     return res
 
 
@@ -573,10 +586,7 @@ def main():
             "warmup": args.warmup, "ms_per_step": ms_per_step, "us_per_step": ms_per_step * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
-            "config": {"workload": WORKLOAD.name, "batch_per_gpu": WORKLOAD.batch, "context": WORKLOAD.t_max,
-                       "n_q": 16, "n_k": 4, "n_v": 16, "d_k": 64, "d_v": 128, "parallelism": f"replicas x{world}",
-                       "l2": "inputs (2.42 GB) larger than L2 (126 MB); no flush",
-                       "kv_bytes_per_gpu_step": main_res["kv_bytes"]},
+            "config": bench_config(world),
             "pct_of_hbm_peak": 100.0 * achieved / peak,
             "gqa_control": control,
             "long_context": long_ctx,

@@ -15,16 +15,26 @@
  *    pointers unless stated and must be 16-byte aligned.
  *  - The caller owns every buffer.  The library never allocates or frees
  *    device memory and keeps no per-call state; the only library-wide state is
- *    a per-device error word (see diffqkv_get_device_status) and cached device
- *    attributes.
+ *    cached device attributes, a per-device error word for the calls that have
+ *    no word of their own (see below), and the built-in scratch array of
+ *    diffqkv_decode_noalloc.
  *  - Every call is asynchronous on the caller's stream (NULL = legacy default
- *    stream) and never synchronises, except diffqkv_get_device_status and
- *    diffqkv_decode_from_host's callers' own syncs.
+ *    stream) and never synchronises, except the two status reads
+ *    (diffqkv_workspace_status, diffqkv_get_device_status).
  *  - Every call returns a diffqkv_status_t.  Argument errors are detected on
- *    the host before anything is launched; nothing crosses the ABI as an
- *    exception.  Conditions only the device can see (a seq_len outside
- *    [0, t_max], a bounded wait that ran out) are recorded in the device error
- *    word and reported by diffqkv_get_device_status.
+ *    the host before anything is launched or copied; nothing crosses the ABI
+ *    as an exception.  Conditions only the device can see (a seq_len outside
+ *    [0, t_max], a block-table entry outside the pool, a bounded wait that ran
+ *    out) are recorded, first error wins, in the call's device error word:
+ *      - calls that take a workspace (decode, its variants, top-v): the
+ *        workspace's first 32-bit word, read and cleared by
+ *        diffqkv_workspace_status;
+ *      - diffqkv_prefill_causal_ex: the word the caller passes;
+ *      - every other call (prefill without a word, diffqkv_decode_noalloc,
+ *        the wait self-test): the per-device word, read and cleared by
+ *        diffqkv_get_device_status.
+ *    So calls on different workspaces (different streams, different host
+ *    threads) report independently, and reading one word clears no other.
  *  - Supported shapes: n_q % n_k == 0, n_q % n_v == 0 (else INVALID_ARG);
  *    n_q / n_k in {1, 2, 4, 8, 16} and d_k, d_v in {64, 128} (else
  *    UNSUPPORTED).
@@ -83,8 +93,11 @@ int32_t diffqkv_version(void);
  * invalid).  Depends only on the dims, not on the device or the lengths.
  * The workspace must be zero-filled before its FIRST use (cudaMemset, or
  * diffqkv_workspace_init); every call that completes leaves it zero-filled
- * again, so it can be reused without clearing.  Two calls that may run
- * concurrently must not share a workspace. */
+ * again (its error word aside, which keeps the first device-side error until
+ * diffqkv_workspace_status reads it), so it can be reused without clearing.
+ * Two calls that may run concurrently must not share a workspace.  Layout: a
+ * 256-byte header whose first 32-bit word is the error word, then one counter
+ * per (batch, K head), then the split partials. */
 size_t diffqkv_decode_workspace_size(const diffqkv_dims_t *dims);
 
 /* Zero-fill a workspace on `stream` (cudaMemsetAsync). */
@@ -103,7 +116,8 @@ diffqkv_status_t diffqkv_workspace_init(void *workspace, size_t workspace_bytes,
  * out[b,h] = sum_j softmax_j(scale * q[b,h].k_cache[b,j,h/(n_q/n_k)])
  *                   * v_cache[b,j,h/(n_q/n_v)],  j < seq_lens[b].
  * A row with seq_lens[b] == 0 is written as zeros.  seq_lens[b] < 0 or
- * > t_max is clamped into [0, t_max] and flagged DIFFQKV_ERR_DEVICE_SEQLEN.
+ * > t_max is clamped into [0, t_max] and flagged DIFFQKV_ERR_DEVICE_SEQLEN in
+ * the workspace's error word.
  * max_seq_len is a host-side upper bound of seq_lens (used only to size the
  * grid; a wrong hint costs speed, never correctness); pass t_max if unknown.
  * Each KV chunk produces (running max, sum of exp, unnormalised output)
@@ -235,7 +249,9 @@ diffqkv_status_t diffqkv_decode_plan(const diffqkv_dims_t *dims, int32_t t_max, 
  * with one cudaMemcpyAsync each, runs diffqkv_decode, and copies the bf16
  * output back into out_host, all on `stream`.  The caller synchronises the
  * stream before reading out_host.  Device buffers follow diffqkv_decode's
- * layouts; host buffers the same layouts.
+ * layouts; host buffers the same layouts.  Every check of diffqkv_decode
+ * (dims, null or misaligned device pointers, the workspace) runs before the
+ * first copy is enqueued: an argument error returns with nothing queued.
  */
 diffqkv_status_t diffqkv_decode_from_host(const diffqkv_dims_t *dims, const void *q_host,
                                           const void *k_cache_host, const void *v_cache_host,
@@ -251,8 +267,10 @@ diffqkv_status_t diffqkv_decode_from_host(const diffqkv_dims_t *dims, const void
 /* over them).                                                              */
 /* ------------------------------------------------------------------------ */
 
-/* Workspace bytes for diffqkv_decode_topv (0 if invalid).  No zero-fill is
- * required. */
+/* Workspace bytes for diffqkv_decode_topv (0 if invalid).  Only the first
+ * 256 bytes (a header whose first 32-bit word is the error word) must be zero
+ * before the workspace's first use (diffqkv_workspace_init zero-fills the
+ * whole workspace); each call clears the rest it needs by itself. */
 size_t diffqkv_decode_topv_workspace_size(const diffqkv_dims_t *dims, int32_t t_max, int32_t topk);
 
 /*
@@ -269,9 +287,10 @@ size_t diffqkv_decode_topv_workspace_size(const diffqkv_dims_t *dims, int32_t t_
  * other buffers and the workspace 16-byte aligned (DIFFQKV_ERR_MISALIGNED).
  * max_seq_len is accepted for symmetry with diffqkv_decode and ignored: the
  * kernels read the lengths from seq_lens on the device.  Lengths outside
- * [0, t_max] are clamped to that range without touching the device error
- * word (diffqkv_decode flags them).  A row with length 0 gets a zero
- * output and an all -1 index row.  Launches four kernels on `stream`
+ * [0, t_max] are clamped to that range and flagged
+ * DIFFQKV_ERR_DEVICE_SEQLEN in the workspace's error word, as
+ * diffqkv_decode does.  A row with length 0 gets a zero output and an all -1
+ * index row.  Launches four kernels on `stream`
  * (chained with programmatic dependent launch);
  * returns once they are queued.
  */
@@ -330,13 +349,35 @@ diffqkv_status_t diffqkv_prefill_causal_prefix(const diffqkv_dims_t *dims, const
                                                const void *v, int32_t prefix_len, int32_t seq_len, void *out,
                                                diffqkv_stream_t stream);
 
+/*
+ * diffqkv_prefill_causal_prefix with the call's own device error word:
+ * device_status_word (int32, device memory, 4-byte aligned, zero before the
+ * call) receives the first device-side error of this call (a bounded wait
+ * that ran out) instead of the per-device word; NULL selects the per-device
+ * word.  The caller reads it like any device memory after synchronising.
+ */
+diffqkv_status_t diffqkv_prefill_causal_ex(const diffqkv_dims_t *dims, const void *q, const void *k,
+                                           const void *v, int32_t prefix_len, int32_t seq_len, void *out,
+                                           int32_t *device_status_word, diffqkv_stream_t stream);
+
 /* ------------------------------------------------------------------------ */
 /* Device error word                                                        */
 /* ------------------------------------------------------------------------ */
 
 /* Synchronises `stream`, returns (in *device_status) the first device-side
- * error recorded on the current device since the last read (DIFFQKV_OK if
- * none), and clears it.  The return value reports failures of the query. */
+ * error recorded in the workspace's error word since the last read
+ * (DIFFQKV_OK if none), and clears that word only.  For the workspaces of
+ * diffqkv_decode (and its variants) and diffqkv_decode_topv; workspace_bytes
+ * >= 256, 16-byte aligned.  The return value reports failures of the query. */
+diffqkv_status_t diffqkv_workspace_status(void *workspace, size_t workspace_bytes, diffqkv_stream_t stream,
+                                          int32_t *device_status);
+
+/* Synchronises `stream`, returns (in *device_status) the first device-side
+ * error recorded in the current device's word since the last read (DIFFQKV_OK
+ * if none), and clears it.  Only calls without a word of their own report
+ * there: diffqkv_prefill_causal / _prefix (and _ex given NULL),
+ * diffqkv_decode_noalloc and diffqkv_selftest_wait_timeout.  The return value
+ * reports failures of the query. */
 diffqkv_status_t diffqkv_get_device_status(diffqkv_stream_t stream, int32_t *device_status);
 
 /* Launches a kernel that waits on a barrier nothing ever signals, with a

@@ -253,3 +253,38 @@ def test_header_is_plain_c_and_a_c_program_links(tmp_path):
     assert r.returncode == 0, r.stderr
     out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
     assert out.returncode == 0 and out.stdout.strip() == "DIFFQKV_ERR_DEVICE_PAGE 1"
+
+
+def _from_host_raw(d, q_dev=0x11000, out_dev=0x15000, ws=0x16000, ws_bytes=1 << 30, t_max=128):
+    # host buffers are never touched when an argument is rejected
+    return _capi.lib().diffqkv_decode_from_host(ctypes.byref(d), 0x1000, 0x2000, 0x3000, 0x4000, t_max, t_max,
+                                                0x5000, q_dev, 0x12000, 0x13000, 0x14000, out_dev, ws, ws_bytes,
+                                                None)
+
+
+def test_from_host_checks_every_argument_before_any_copy():
+    """Without a GPU, an enqueued copy would fail with DIFFQKV_ERR_CUDA; these specific codes show
+    that the decode's checks ran before the first cudaMemcpyAsync."""
+    d = dims()
+    assert _from_host_raw(d, q_dev=0x11008) == _capi.MISALIGNED
+    assert _from_host_raw(d, out_dev=0x15004) == _capi.MISALIGNED
+    assert _from_host_raw(d, ws=None) == _capi.WORKSPACE
+    assert _from_host_raw(d, ws_bytes=64) == _capi.WORKSPACE
+    assert _from_host_raw(d, t_max=0) == _capi.INVALID_ARG
+    assert _from_host_raw(dims(n_k=3)) == _capi.INVALID_ARG
+    assert _from_host_raw(dims(d_k=96)) == _capi.UNSUPPORTED
+
+
+def test_workspace_status_and_prefill_word_reject_bad_args():
+    lib = _capi.lib()
+    v = ctypes.c_int32(0)
+    assert lib.diffqkv_workspace_status(None, 1 << 20, None, ctypes.byref(v)) == _capi.INVALID_ARG
+    assert lib.diffqkv_workspace_status(0x1000, 255, None, ctypes.byref(v)) == _capi.INVALID_ARG
+    assert lib.diffqkv_workspace_status(0x1000, 1 << 20, None, None) == _capi.INVALID_ARG
+    assert lib.diffqkv_workspace_status(0x1008, 1 << 20, None, ctypes.byref(v)) == _capi.MISALIGNED
+    d = dims()
+    # a misaligned status word is rejected before any device work
+    assert lib.diffqkv_prefill_causal_ex(ctypes.byref(d), 0x1000, 0x2000, 0x3000, 0, 16, 0x5000, 0x6002,
+                                         None) == _capi.MISALIGNED
+    assert lib.diffqkv_prefill_causal_ex(ctypes.byref(d), 0x1000, 0x2000, 0x3000, -1, 16, 0x5000, None,
+                                         None) == _capi.INVALID_ARG

@@ -22,10 +22,14 @@ SHAPES = {
 }
 
 
-def _run(d, dev, **kw):
+def _run(d, dev, expect=0, **kw):
+    """Decode through the C ABI; the call's workspace error word must read `expect`."""
     g = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
-    out = ak.decode(g["q"], g["k_cache"], g["v_cache"], g["seq_lens"], scale=d["scale"], **kw)
-    torch.cuda.synchronize()
+    ws = kw.pop("workspace", None)
+    if ws is None:
+        ws = ak.decode_workspace(g["q"], g["k_cache"], g["v_cache"])
+    out = ak.decode(g["q"], g["k_cache"], g["v_cache"], g["seq_lens"], scale=d["scale"], workspace=ws, **kw)
+    assert ak.workspace_status(ws) == expect
     return out
 
 
@@ -37,7 +41,6 @@ def test_small_workload_full(cuda_device):
     d = wl.make_decode_inputs(wl.DECODE_SMALL, "cpu")
     out = _run(d, cuda_device)
     assert_parity(out, _oracle(d), "decode B=1 T=512")
-    assert ak.device_status() == 0
 
 
 @pytest.mark.parametrize("name", list(SHAPES))
@@ -47,7 +50,6 @@ def test_shapes_ragged(cuda_device, name):
     d = wl.random_decode_inputs(len(lens), 1000, shape, seed=101, seq_lens=lens)
     out = _run(d, cuda_device)
     assert_parity(out, _oracle(d), name)
-    assert ak.device_status() == 0
 
 
 @pytest.mark.parametrize("grid", [1, 2, 3, 7, 64, 148, 333, 2048])
@@ -83,11 +85,9 @@ def test_empty_and_out_of_range_lengths(cuda_device):
     out = _run(d, cuda_device)
     assert torch.all(out[0] == 0) and torch.all(out[2] == 0)
     assert_parity(out, _oracle(d), "empty rows")
-    assert ak.device_status() == 0
-    # a negative or too-long length is clamped and flagged in the device error word
+    # a negative or too-long length is clamped and flagged in the workspace's error word
     bad = dict(d, seq_lens=torch.tensor([-3, 100, 150, 7], dtype=torch.int32))
-    out = _run(bad, cuda_device)
-    assert ak.device_status() == ak._capi.DEVICE_SEQLEN
+    out = _run(bad, cuda_device, expect=ak._capi.DEVICE_SEQLEN)
     clamped = dict(d, seq_lens=torch.tensor([0, 100, 100, 7], dtype=torch.int32))
     assert_parity(out, _oracle(clamped), "clamped lengths")
 
@@ -102,8 +102,9 @@ def test_workspace_reuse_across_shapes(cuda_device):
         d["seq_lens"] = torch.tensor(lens, dtype=torch.int32)
         out = _run(d, cuda_device, workspace=ws)
         assert_parity(out, _oracle(d), f"lens={lens[:3]}")
-    # the per-unit counters (after a 256-byte header, one uint32 per (batch, K head)) are zero again
-    assert torch.count_nonzero(ws[256:256 + 8 * 4 * 4]) == 0
+    # the per-unit counters (after a 256-byte header, one uint32 per (batch, K head)) are zero again,
+    # and so is the header (its first word is the error word, read and cleared by _run)
+    assert torch.count_nonzero(ws[:256 + 8 * 4 * 4]) == 0
 
 
 def test_bounded_wait_reports_timeout_and_context_survives(cuda_device):
@@ -118,9 +119,9 @@ def test_bounded_wait_reports_timeout_and_context_survives(cuda_device):
 @pytest.mark.parametrize("w", [wl.DECODE_32K, wl.DECODE_32K_GQA], ids=lambda w: w.name)
 def test_full_decode_32k(cuda_device, w):
     d = wl.make_decode_inputs(w, cuda_device)
-    out = ak.decode(d["q"], d["k_cache"], d["v_cache"], d["seq_lens"], scale=d["scale"])
-    torch.cuda.synchronize()
-    assert ak.device_status() == 0
+    ws = ak.decode_workspace(d["q"], d["k_cache"], d["v_cache"])
+    out = ak.decode(d["q"], d["k_cache"], d["v_cache"], d["seq_lens"], scale=d["scale"], workspace=ws)
+    assert ak.workspace_status(ws) == 0
     ref = oracle.decode(d["q"].cpu(), d["k_cache"].cpu(), d["v_cache"].cpu(), d["seq_lens"].cpu(), d["scale"])
     assert_parity(out, ref, w.name)
 
@@ -128,10 +129,10 @@ def test_full_decode_32k(cuda_device, w):
 @pytest.mark.parametrize("w", [wl.DECODE_RAGGED, wl.DECODE_RAGGED_GQA], ids=lambda w: w.name)
 def test_full_decode_ragged(cuda_device, w):
     d = wl.make_decode_inputs(w, cuda_device)
+    ws = ak.decode_workspace(d["q"], d["k_cache"], d["v_cache"])
     out = ak.decode(d["q"], d["k_cache"], d["v_cache"], d["seq_lens"], scale=d["scale"],
-                    max_seq_len=int(d["seq_lens"].max()))
-    torch.cuda.synchronize()
-    assert ak.device_status() == 0
+                    max_seq_len=int(d["seq_lens"].max()), workspace=ws)
+    assert ak.workspace_status(ws) == 0
     ref = oracle.decode(d["q"].cpu(), d["k_cache"].cpu(), d["v_cache"].cpu(), d["seq_lens"].cpu(), d["scale"])
     assert_parity(out, ref, w.name)
 
@@ -149,3 +150,44 @@ def test_decode_from_host_matches_device_path(cuda_device):
     ref_dev = _run(d, cuda_device)
     assert torch.equal(out_host, ref_dev.cpu())
     assert_parity(out_host, _oracle(d), "from host")
+
+
+def test_error_words_are_per_workspace(cuda_device):
+    """Two decodes on two streams, each with its own workspace: the one given out-of-range lengths
+    reports DIFFQKV_ERR_DEVICE_SEQLEN in its workspace, the other reports nothing, and reading one
+    word clears neither the other nor the per-device word."""
+    good = wl.random_decode_inputs(2, 500, wl.DIFFQKV, seed=107, seq_lens=[500, 3])
+    bad = dict(good, seq_lens=torch.tensor([600, -1], dtype=torch.int32))
+    gg = {k: (v.to(cuda_device) if isinstance(v, torch.Tensor) else v) for k, v in good.items()}
+    gb = {k: (v.to(cuda_device) if isinstance(v, torch.Tensor) else v) for k, v in bad.items()}
+    ws_good, ws_bad = (ak.decode_workspace(gg["q"], gg["k_cache"], gg["v_cache"]) for _ in range(2))
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    torch.cuda.synchronize()
+    out_b = ak.decode(gb["q"], gb["k_cache"], gb["v_cache"], gb["seq_lens"], scale=good["scale"],
+                      workspace=ws_bad, stream=s1)
+    out_g = ak.decode(gg["q"], gg["k_cache"], gg["v_cache"], gg["seq_lens"], scale=good["scale"],
+                      workspace=ws_good, stream=s2)
+    torch.cuda.synchronize()
+    assert ak.workspace_status(ws_good, stream=s2) == 0
+    assert ak.device_status() == 0
+    assert ak.workspace_status(ws_bad, stream=s1) == ak._capi.DEVICE_SEQLEN
+    assert ak.workspace_status(ws_bad, stream=s1) == 0     # read-and-clear of that word only
+    assert_parity(out_g, _oracle(good), "good stream")
+    clamped = dict(good, seq_lens=torch.tensor([500, 0], dtype=torch.int32))
+    assert_parity(out_b, _oracle(clamped), "bad stream, clamped")
+
+
+@pytest.mark.parametrize("grid", [0, 7, 2048])
+def test_poisoned_partials_are_never_read_before_written(cuda_device, grid):
+    """Every byte of the split-partial region starts as 0xFF (a NaN pattern): a combine that read a
+    partial no CTA of this call wrote would turn the output NaN or wrong."""
+    lens = [2000, 5, 1311, 0, 48, 49]
+    d = wl.random_decode_inputs(len(lens), 2000, wl.DIFFQKV, seed=108, seq_lens=lens)
+    g = {k: (v.to(cuda_device) if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
+    ws = ak.decode_workspace(g["q"], g["k_cache"], g["v_cache"])
+    counters_end = 256 + -(-len(lens) * wl.DIFFQKV.n_k * 4 // 256) * 256
+    ws[counters_end:] = 0xFF
+    tuning = {"grid_ctas": grid, "stages": 0, "ctas_per_sm": 0} if grid else None
+    out = _run(d, cuda_device, workspace=ws, tuning=tuning)
+    assert torch.isfinite(out.float()).all()
+    assert_parity(out, _oracle(d), f"poisoned partials, grid {grid}")

@@ -35,11 +35,14 @@ def _expected(d, k_new, v_new, t_max):
     return k_after, v_after, out
 
 
-def _run(d, k_new, v_new, dev):
+def _run(d, k_new, v_new, dev, expect=0):
+    """The fused append through the C ABI; the workspace's error word must read `expect`."""
     g = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
     kn, vn = k_new.to(dev), v_new.to(dev)
-    out = ak.decode_append(g["q"], kn, vn, g["k_cache"], g["v_cache"], g["seq_lens"], scale=d["scale"])
-    torch.cuda.synchronize()
+    ws = ak.decode_workspace(g["q"], g["k_cache"], g["v_cache"])
+    out = ak.decode_append(g["q"], kn, vn, g["k_cache"], g["v_cache"], g["seq_lens"], scale=d["scale"],
+                           workspace=ws)
+    assert ak.workspace_status(ws) == expect
     return out, g["k_cache"], g["v_cache"]
 
 
@@ -61,7 +64,6 @@ def test_append_matches_oracle(cuda_device, name):
     k_new, v_new = _new_rows(shape, len(lens), 502)
     k_after, v_after, ref = _expected(d, k_new, v_new, t_max)
     out, kc, vc = _run(d, k_new, v_new, cuda_device)
-    assert ak.device_status() == 0
     assert torch.equal(kc.cpu(), k_after) and torch.equal(vc.cpu(), v_after), f"{name}: cache contents"
     assert_parity(out, ref, f"append {name}")
     # an empty cache attends to the new token alone: exactly its V row
@@ -76,15 +78,15 @@ def test_append_consecutive_steps(cuda_device):
     d = wl.random_decode_inputs(len(lens), t_max, shape, seed=511, seq_lens=lens)
     g = {k: (v.to(cuda_device) if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
     k_cpu, v_cpu = d["k_cache"].clone(), d["v_cache"].clone()
+    ws = ak.decode_workspace(g["q"], g["k_cache"], g["v_cache"])
     for step in range(3):
         k_new, v_new = _new_rows(shape, len(lens), 520 + step)
         q = torch.randn(len(lens), shape.n_q, shape.d_k, generator=torch.Generator().manual_seed(530 + step))
         q = q.to(torch.bfloat16)
         cur = g["seq_lens"].cpu()
         out = ak.decode_append(q.to(cuda_device), k_new.to(cuda_device), v_new.to(cuda_device), g["k_cache"],
-                               g["v_cache"], g["seq_lens"], scale=d["scale"])
-        torch.cuda.synchronize()
-        assert ak.device_status() == 0
+                               g["v_cache"], g["seq_lens"], scale=d["scale"], workspace=ws)
+        assert ak.workspace_status(ws) == 0
         for b, p in enumerate(cur.tolist()):
             k_cpu[b, p] = k_new[b]
             v_cpu[b, p] = v_new[b]
@@ -96,15 +98,13 @@ def test_append_consecutive_steps(cuda_device):
 
 def test_append_full_cache_is_flagged(cuda_device):
     """No free slot (seq_len == t_max): nothing is written, the step attends over the cache, and the
-    device error word reports DIFFQKV_ERR_DEVICE_SEQLEN."""
+    workspace's error word reports DIFFQKV_ERR_DEVICE_SEQLEN."""
     shape, t_max = wl.DIFFQKV, 300
     lens = [300, 120]
     d = wl.random_decode_inputs(len(lens), t_max, shape, seed=541, seq_lens=lens)
     k_new, v_new = _new_rows(shape, len(lens), 542)
     k_after, v_after, ref = _expected(d, k_new, v_new, t_max)
-    out, kc, vc = _run(d, k_new, v_new, cuda_device)
-    assert ak.device_status() == ak._capi.DEVICE_SEQLEN
-    assert ak.device_status() == 0  # reading clears the word
+    out, kc, vc = _run(d, k_new, v_new, cuda_device, expect=ak._capi.DEVICE_SEQLEN)
     assert torch.equal(kc.cpu(), k_after) and torch.equal(vc.cpu(), v_after)
     assert torch.equal(kc.cpu()[0], d["k_cache"][0])  # the full row is untouched
     assert_parity(out, ref, "full cache")

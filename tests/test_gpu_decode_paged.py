@@ -19,6 +19,15 @@ def _to(d, dev):
     return {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
 
 
+def _paged(g, scale, expect=0, **kw):
+    """Paged decode through the C ABI; the workspace's error word must read `expect`."""
+    ws = ak.decode_workspace(g["q"], g["k_pages"], g["v_pages"])
+    out = ak.decode_paged(g["q"], g["k_pages"], g["v_pages"], g["block_table"], g["seq_lens"], scale=scale,
+                          workspace=ws, **kw)
+    assert ak.workspace_status(ws) == expect
+    return out
+
+
 def _gathered(d):
     return (oracle.gather_paged(d["k_pages"], d["block_table"], d["seq_lens"]),
             oracle.gather_paged(d["v_pages"], d["block_table"], d["seq_lens"]))
@@ -41,9 +50,7 @@ def test_paged_matches_oracle(cuda_device, name, page_size):
     d = wl.random_paged_inputs(len(lens), max_blocks, page_size, shape, seed=601, seq_lens=lens, spare_pages=3)
     ref = oracle.decode_paged(d["q"], d["k_pages"], d["v_pages"], d["block_table"], d["seq_lens"], d["scale"])
     g = _to(d, cuda_device)
-    out = ak.decode_paged(g["q"], g["k_pages"], g["v_pages"], g["block_table"], g["seq_lens"], scale=d["scale"])
-    torch.cuda.synchronize()
-    assert ak.device_status() == 0
+    out = _paged(g, d["scale"])
     assert_parity(out, ref, f"paged {name} P={page_size}")
     kc, vc = _gathered(d)
     flat = ak.decode(g["q"], kc.to(cuda_device), vc.to(cuda_device), g["seq_lens"], scale=d["scale"])
@@ -56,11 +63,10 @@ def test_paged_mid_size_against_contiguous(cuda_device):
     shape, page_size, T = wl.DIFFQKV, 16, 8192
     d = wl.random_paged_inputs(4, T // page_size + 1, page_size, shape, seed=611, seq_lens=[T, T - 5, 4097, 16])
     g = _to(d, cuda_device)
-    out = ak.decode_paged(g["q"], g["k_pages"], g["v_pages"], g["block_table"], g["seq_lens"], scale=d["scale"])
+    out = _paged(g, d["scale"])
     kc, vc = _gathered(d)
     flat = ak.decode(g["q"], kc.to(cuda_device), vc.to(cuda_device), g["seq_lens"], scale=d["scale"])
     torch.cuda.synchronize()
-    assert ak.device_status() == 0
     assert torch.equal(out, flat)
     rows = [(0, 0), (0, 15), (1, 7), (2, 3), (3, 12)]
     ref = oracle.decode(d["q"], kc, vc, d["seq_lens"], d["scale"], rows=rows)
@@ -85,10 +91,7 @@ def test_paged_append(cuda_device, page_size):
     new_lens = d["seq_lens"] + 1
     ref = oracle.decode_paged(d["q"], k_after, v_after, d["block_table"], new_lens, d["scale"])
     g = _to(d, cuda_device)
-    out = ak.decode_paged(g["q"], g["k_pages"], g["v_pages"], g["block_table"], g["seq_lens"],
-                          k_new=k_new.to(cuda_device), v_new=v_new.to(cuda_device), scale=d["scale"])
-    torch.cuda.synchronize()
-    assert ak.device_status() == 0
+    out = _paged(g, d["scale"], k_new=k_new.to(cuda_device), v_new=v_new.to(cuda_device))
     assert torch.equal(g["k_pages"].cpu(), k_after) and torch.equal(g["v_pages"].cpu(), v_after)
     assert_parity(out, ref, f"paged append P={page_size}")
 
@@ -102,10 +105,7 @@ def test_bad_page_entry_is_flagged(cuda_device):
     ref = oracle.decode_paged(d["q"], d["k_pages"], d["v_pages"], d["block_table"], d["seq_lens"], d["scale"])
     d["block_table"][0, 1] = d["num_pages"] + 5
     g = _to(d, cuda_device)
-    out = ak.decode_paged(g["q"], g["k_pages"], g["v_pages"], g["block_table"], g["seq_lens"], scale=d["scale"])
-    torch.cuda.synchronize()
-    assert ak.device_status() == ak._capi.DEVICE_PAGE
-    assert ak.device_status() == 0
+    out = _paged(g, d["scale"], expect=ak._capi.DEVICE_PAGE)
     assert_parity(out[1:], ref[1:], "paged, other sequence")
     # append into a position whose page entry is bad: nothing written anywhere
     d["block_table"][0, 1] = -3
@@ -114,10 +114,7 @@ def test_bad_page_entry_is_flagged(cuda_device):
     vn = torch.ones(2, shape.n_v, shape.d_v, dtype=torch.bfloat16, device=cuda_device)
     g["seq_lens"][0] = 20  # position 20 lives in logical page 1
     before = g["k_pages"].clone()
-    ak.decode_paged(g["q"], g["k_pages"], g["v_pages"], g["block_table"], g["seq_lens"], k_new=kn, v_new=vn,
-                    scale=d["scale"])
-    torch.cuda.synchronize()
-    assert ak.device_status() == ak._capi.DEVICE_PAGE
+    _paged(g, d["scale"], expect=ak._capi.DEVICE_PAGE, k_new=kn, v_new=vn)
     page1 = int(d["block_table"][1, 40 // page_size])
     changed = (g["k_pages"] != before).flatten(1).any(1).nonzero().flatten().tolist()
     assert changed == [page1]  # only sequence 1's append

@@ -33,6 +33,8 @@ CASES = [
     ("diffqkv_dq96_shared", wl.DIFFQKV, 96, 1),
     ("gqa_dk128_dq256", wl.GQA_CONTROL, 256, 16),
     ("qpk3_dq40", Shape(12, 4, 4, 64, 64), 40, 4),
+    # 16 warps over 5 rows: 3 slices x 5 rows leave one warp without a (row, slice) slot
+    ("qpk5_dq72", Shape(20, 4, 4, 64, 64), 72, 4),
     ("mha_dq8", Shape(8, 8, 8, 128, 64), 8, 8),
 ]
 
@@ -59,9 +61,9 @@ def test_fold_then_decode_matches_up_projected_attention(cuda_device, name, shap
     ref = oracle.decode_up_projected(q_aug, w, d["k_cache"], d["v_cache"], d["seq_lens"], scale)
     g = {k: (v.to(cuda_device) if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
     q = ak.fold_query(q_aug.to(cuda_device), w.to(cuda_device), n_k=shape.n_k)
-    out = ak.decode(q, g["k_cache"], g["v_cache"], g["seq_lens"], scale=scale)
-    torch.cuda.synchronize()
-    assert ak.device_status() == 0
+    ws = ak.decode_workspace(q, g["k_cache"], g["v_cache"])
+    out = ak.decode(q, g["k_cache"], g["v_cache"], g["seq_lens"], scale=scale, workspace=ws)
+    assert ak.workspace_status(ws) == 0
     assert_parity(out, ref, f"fold + decode {name}")
 
 

@@ -7,7 +7,7 @@ import asymmetric_head_kv_b200 as ak
 import oracle
 import workloads as wl
 from workloads import Shape
-from parity import assert_parity
+from parity import assert_parity, assert_parity_prefill
 
 pytestmark = pytest.mark.gpu
 
@@ -33,7 +33,7 @@ def _gpu(d, dev):
 def test_lengths_diffqkv(cuda_device, seq):
     d = wl.random_prefill_inputs(2, seq, wl.DIFFQKV, seed=400 + seq)
     out = _gpu(d, cuda_device)
-    assert_parity(out, oracle.prefill_causal(d["q"], d["k"], d["v"], d["scale"]), f"S={seq}")
+    assert_parity_prefill(out, oracle.prefill_causal(d["q"], d["k"], d["v"], d["scale"]), f"S={seq}")
     # row 0 attends to position 0 only: exactly V_0 (weight 2^0 = 1)
     assert torch.equal(out[:, 0].cpu(), d["v"][:, 0].repeat_interleave(wl.DIFFQKV.n_q // wl.DIFFQKV.n_v, dim=1))
 
@@ -42,7 +42,7 @@ def test_lengths_diffqkv(cuda_device, seq):
 def test_shapes(cuda_device, name):
     d = wl.random_prefill_inputs(2, 333, SHAPES[name], seed=410)
     out = _gpu(d, cuda_device)
-    assert_parity(out, oracle.prefill_causal(d["q"], d["k"], d["v"], d["scale"]), name)
+    assert_parity_prefill(out, oracle.prefill_causal(d["q"], d["k"], d["v"], d["scale"]), name)
 
 
 @pytest.mark.parametrize("seq", [1, 5, 127, 128, 129, 255, 256, 257, 300, 600])
@@ -53,7 +53,7 @@ def test_lengths_dk128(cuda_device, seq):
     s = wl.GQA_CONTROL
     d = wl.random_prefill_inputs(1, seq, s, seed=440 + seq)
     out = _gpu(d, cuda_device)
-    assert_parity(out, oracle.prefill_causal(d["q"], d["k"], d["v"], d["scale"]), f"d_k 128, S={seq}")
+    assert_parity_prefill(out, oracle.prefill_causal(d["q"], d["k"], d["v"], d["scale"]), f"d_k 128, S={seq}")
     assert torch.equal(out[:, 0].cpu(), d["v"][:, 0].repeat_interleave(s.n_q // s.n_v, dim=1))
 
 
@@ -63,7 +63,7 @@ def test_sharp_softmax_rescaling(cuda_device):
     ramp = torch.linspace(0.1, 6.0, 700).to(torch.bfloat16)
     d["k"] = (d["k"].float() * ramp[None, :, None, None].float()).to(torch.bfloat16)
     out = _gpu(d, cuda_device)
-    assert_parity(out, oracle.prefill_causal(d["q"], d["k"], d["v"], d["scale"]), "rescale")
+    assert_parity_prefill(out, oracle.prefill_causal(d["q"], d["k"], d["v"], d["scale"]), "rescale")
 
 
 def test_sharp_softmax_rescaling_dk128(cuda_device):
@@ -72,7 +72,7 @@ def test_sharp_softmax_rescaling_dk128(cuda_device):
     ramp = torch.linspace(0.1, 6.0, 700).to(torch.bfloat16)
     d["k"] = (d["k"].float() * ramp[None, :, None, None].float()).to(torch.bfloat16)
     out = _gpu(d, cuda_device)
-    assert_parity(out, oracle.prefill_causal(d["q"], d["k"], d["v"], d["scale"]), "rescale d_k 128")
+    assert_parity_prefill(out, oracle.prefill_causal(d["q"], d["k"], d["v"], d["scale"]), "rescale d_k 128")
 
 
 def test_prefill_rows_match_gpu_decode(cuda_device):
@@ -87,29 +87,44 @@ def test_prefill_rows_match_gpu_decode(cuda_device):
         dec = ak.decode(q, k, v, torch.tensor([i + 1], dtype=torch.int32, device=cuda_device), scale=d["scale"])
         ref = oracle.decode(d["q"][:, i].contiguous(), d["k"], d["v"], torch.tensor([i + 1], dtype=torch.int32),
                             d["scale"])
-        assert_parity(out[:, i], ref, f"row {i}")
+        assert_parity_prefill(out[:, i], ref, f"row {i}")
         assert_parity(dec, ref, f"decode {i}")
 
 
-def _sample_rows(B, S, n_q, seed):
-    rng = np.random.default_rng(seed)
-    pos = sorted(set([0, 1, 2, 63, 64, 65, 127, 128, 129, 1000, S // 2 - 1, S // 2, S - 2, S - 1] +
-                     rng.integers(0, S, 16).tolist()))
-    return [(b, i, h) for b in range(B) for i in pos for h in range(n_q)]
+def _full_check_rows(w, n_heads_full):
+    """Every query position of one (batch, head) per covered K head, plus every head of both
+    sequences on every 64th position (and the last one).  The covered heads are spread over the K
+    heads (and so over the tile scheduler's (batch, head) order) and alternate between sequences."""
+    s = w.shape
+    qpk = s.n_q // s.n_k
+    stride = max(1, s.n_k // n_heads_full)
+    full = []
+    for i, g in enumerate(range(0, s.n_k, stride)):
+        h = g * qpk + (i % qpk)          # a different member of each group, so V heads vary too
+        full.append((i % w.batch, h))
+    rows = [(b, pos, h) for b, h in full for pos in range(w.seq)]
+    strided = sorted(set(list(range(0, w.seq, 64)) + [w.seq - 1]))
+    rows += [(b, pos, h) for b in range(w.batch) for pos in strided for h in range(s.n_q)
+             if (b, h) not in full]
+    return full, rows
 
 
-@pytest.mark.parametrize("w", [wl.PREFILL_8K, wl.PREFILL_8K_GQA], ids=lambda w: w.name)
-def test_full_prefill_sampled_rows(cuda_device, w):
+@pytest.mark.parametrize("w,n_heads_full", [(wl.PREFILL_8K, 4), (wl.PREFILL_8K_GQA, 4)], ids=lambda x: getattr(x, "name", str(x)))
+def test_full_prefill_every_row_of_covered_heads(cuda_device, w, n_heads_full):
+    """The full 2 x 8192 causal prefill: all 8192 query positions of one (batch, head) per K head
+    (for the DiffQKV shape; four spread K heads of the 16 of the GQA control), and every head on
+    every 64th position, against the fp64 oracle."""
     d = wl.make_prefill_inputs(w, cuda_device)
     out = ak.prefill_causal(d["q"], d["k"], d["v"], scale=d["scale"])
     torch.cuda.synchronize()
     assert ak.device_status() == 0
     assert torch.isfinite(out.float()).all()
-    rows = _sample_rows(w.batch, w.seq, w.shape.n_q, 440)
+    full, rows = _full_check_rows(w, n_heads_full)
+    assert len(full) == n_heads_full
     ref = oracle.prefill_causal(d["q"].cpu(), d["k"].cpu(), d["v"].cpu(), d["scale"], rows=rows)
     idx = torch.tensor(rows)
     got = out[idx[:, 0], idx[:, 1], idx[:, 2]]
-    assert_parity(got, ref, w.name)
+    assert_parity_prefill(got, ref, w.name)
 
 
 def _prefix_expected(q, k, v, scale, P):
@@ -132,7 +147,7 @@ def test_prefix_prefill(cuda_device, shape_name, P, S):
     out = ak.prefill_causal_prefix(q.to(cuda_device), g["k"], g["v"], P, scale=d["scale"])
     torch.cuda.synchronize()
     assert ak.device_status() == 0
-    assert_parity(out, _prefix_expected(q, d["k"], d["v"], d["scale"], P), f"{shape_name} P={P} S={S}")
+    assert_parity_prefill(out, _prefix_expected(q, d["k"], d["v"], d["scale"], P), f"{shape_name} P={P} S={S}")
 
 
 def test_prefix_zero_is_plain_prefill_and_chunks_compose(cuda_device):
@@ -149,4 +164,18 @@ def test_prefix_zero_is_plain_prefill_and_chunks_compose(cuda_device):
     torch.cuda.synchronize()
     assert ak.device_status() == 0
     ref = oracle.prefill_causal(d["q"], d["k"], d["v"], d["scale"])
-    assert_parity(torch.cat(parts, dim=1), ref, "chunked prefill")
+    assert_parity_prefill(torch.cat(parts, dim=1), ref, "chunked prefill")
+
+
+def test_prefill_reports_into_the_callers_status_word(cuda_device):
+    """diffqkv_prefill_causal_ex: the call's device-side errors go to the word the caller passes,
+    not to the per-device word (a clean call leaves both at zero and computes the same bits)."""
+    d = wl.random_prefill_inputs(1, 200, wl.DIFFQKV, seed=470)
+    g = {k: d[k].to(cuda_device) for k in ("q", "k", "v")}
+    word = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    out = ak.prefill_causal(g["q"], g["k"], g["v"], scale=d["scale"], status=word)
+    plain = ak.prefill_causal(g["q"], g["k"], g["v"], scale=d["scale"])
+    torch.cuda.synchronize()
+    assert int(word.item()) == 0 and ak.device_status() == 0
+    assert torch.equal(out, plain)
+    assert_parity_prefill(out, oracle.prefill_causal(d["q"], d["k"], d["v"], d["scale"]), "prefill with status word")

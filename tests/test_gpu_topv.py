@@ -15,11 +15,15 @@ from parity import assert_parity
 pytestmark = pytest.mark.gpu
 
 
-def _gpu(d, topk, dev, **kw):
+def _gpu(d, topk, dev, expect=0, **kw):
+    """Selective-V decode through the C ABI; the workspace's error word must read `expect`."""
     g = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
-    out, idx = ak.decode_topv(g["q"], g["k_cache"], g["v_cache"], g["seq_lens"], topk, scale=d["scale"], **kw)
-    torch.cuda.synchronize()
-    assert ak.device_status() == 0
+    dims = ak.make_dims(*g["q"].shape[:2], g["k_cache"].shape[2], g["v_cache"].shape[2], g["q"].shape[2],
+                        g["v_cache"].shape[3], d["scale"])
+    ws = ak.decode_topv_workspace(dims, g["k_cache"].shape[1], topk, dev)
+    out, idx = ak.decode_topv(g["q"], g["k_cache"], g["v_cache"], g["seq_lens"], topk, scale=d["scale"],
+                              workspace=ws, **kw)
+    assert ak.workspace_status(ws) == expect
     return out, idx
 
 
@@ -112,9 +116,11 @@ def test_workspace_too_small_is_rejected(cuda_device):
 def test_full_topv_workload(cuda_device):
     w = wl.TOPV_64K
     d = wl.make_decode_inputs(w, cuda_device)
-    out, idx = ak.decode_topv(d["q"], d["k_cache"], d["v_cache"], d["seq_lens"], w.topk, scale=d["scale"])
-    torch.cuda.synchronize()
-    assert ak.device_status() == 0
+    dims = ak.make_dims(w.batch, w.shape.n_q, w.shape.n_k, w.shape.n_v, w.shape.d_k, w.shape.d_v, d["scale"])
+    ws = ak.decode_topv_workspace(dims, w.t_max, w.topk, cuda_device)
+    out, idx = ak.decode_topv(d["q"], d["k_cache"], d["v_cache"], d["seq_lens"], w.topk, scale=d["scale"],
+                              workspace=ws)
+    assert ak.workspace_status(ws) == 0
     cpu = {k: (v.cpu() if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
     r_out, r_idx = oracle.decode_topv(cpu["q"], cpu["k_cache"], cpu["v_cache"], cpu["seq_lens"], w.topk, d["scale"])
     assert np.array_equal(idx.cpu().numpy(), r_idx)
@@ -133,8 +139,7 @@ def test_workspace_reuse_is_bitwise_stable(cuda_device, topk):
     for _ in range(2):
         out, idx = ak.decode_topv(g["q"], g["k_cache"], g["v_cache"], g["seq_lens"], topk, scale=d["scale"],
                                   workspace=ws)
-        torch.cuda.synchronize()
-        assert ak.device_status() == 0
+        assert ak.workspace_status(ws) == 0
         runs.append((out.clone(), idx.clone()))
     assert torch.equal(runs[0][0], runs[1][0]) and torch.equal(runs[0][1], runs[1][1])
     r_out, r_idx = oracle.decode_topv(d["q"], d["k_cache"], d["v_cache"], d["seq_lens"], topk, d["scale"])
@@ -156,3 +161,36 @@ def test_full_softmax_weights(cuda_device, name, shape, topk):
     assert_parity(out, r_out, f"full weights {name}")
     _, idx_renorm = _gpu(d, topk, cuda_device)
     assert torch.equal(idx, idx_renorm)  # the selection does not depend on the weighting
+
+
+def test_out_of_range_lengths_are_clamped_and_flagged(cuda_device):
+    """Lengths outside [0, t_max] are clamped, as in the decode, and flagged
+    DIFFQKV_ERR_DEVICE_SEQLEN in the workspace's error word."""
+    d = wl.random_decode_inputs(3, 800, wl.DIFFQKV, seed=310, seq_lens=[800, 300, 800])
+    bad = dict(d, seq_lens=torch.tensor([900, 300, -4], dtype=torch.int32))
+    out, idx = _gpu(bad, 50, cuda_device, expect=ak._capi.DEVICE_SEQLEN)
+    clamped = dict(d, seq_lens=torch.tensor([800, 300, 0], dtype=torch.int32))
+    r_out, r_idx = oracle.decode_topv(d["q"], d["k_cache"], d["v_cache"], clamped["seq_lens"], 50, d["scale"])
+    assert np.array_equal(idx.cpu().numpy(), r_idx)
+    assert_parity(out, r_out, "clamped lengths")
+    _gpu(d, 50, cuda_device)   # in-range lengths: nothing flagged
+
+
+@pytest.mark.parametrize("topk", [1, 100, 1024])
+def test_poisoned_workspace_is_never_read_before_written(cuda_device, topk):
+    """Every byte after the workspace header (scores, candidate lists, ambiguous lists, per-row
+    words) starts as 0xFF: a kernel that read scratch this call did not write would change the
+    index sets or the output."""
+    lens = [5000, 1, 2047, 0, 3000]
+    d = wl.random_decode_inputs(len(lens), 5000, wl.DIFFQKV, seed=311, seq_lens=lens)
+    g = {k: (v.to(cuda_device) if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
+    dims = ak.make_dims(len(lens), 16, 4, 16, 64, 128, d["scale"])
+    ws = ak.decode_topv_workspace(dims, 5000, topk, cuda_device)
+    ws[256:] = 0xFF
+    out, idx = ak.decode_topv(g["q"], g["k_cache"], g["v_cache"], g["seq_lens"], topk, scale=d["scale"],
+                              workspace=ws)
+    assert ak.workspace_status(ws) == 0
+    r_out, r_idx = oracle.decode_topv(d["q"], d["k_cache"], d["v_cache"], d["seq_lens"], topk, d["scale"])
+    assert np.array_equal(idx.cpu().numpy(), r_idx)
+    assert torch.isfinite(out.float()).all()
+    assert_parity(out, r_out, f"poisoned workspace k={topk}")
