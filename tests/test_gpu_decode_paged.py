@@ -21,7 +21,9 @@ def _to(d, dev):
 
 def _paged(g, scale, expect=0, **kw):
     """Paged decode through the C ABI; the workspace's error word must read `expect`."""
-    ws = ak.decode_workspace(g["q"], g["k_pages"], g["v_pages"])
+    B, n_q, d_k = g["q"].shape
+    dims = ak.make_dims(B, n_q, g["k_pages"].shape[2], g["v_pages"].shape[2], d_k, g["v_pages"].shape[3], scale)
+    ws = ak.decode_workspace(dims, device=g["q"].device)
     out = ak.decode_paged(g["q"], g["k_pages"], g["v_pages"], g["block_table"], g["seq_lens"], scale=scale,
                           workspace=ws, **kw)
     assert ak.workspace_status(ws) == expect

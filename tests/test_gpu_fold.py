@@ -15,7 +15,7 @@ import asymmetric_head_kv_b200 as ak
 import oracle
 import workloads as wl
 from workloads import Shape
-from parity import assert_parity
+from parity import assert_parity, assert_parity_prefill
 
 pytestmark = pytest.mark.gpu
 
@@ -64,7 +64,13 @@ def test_fold_then_decode_matches_up_projected_attention(cuda_device, name, shap
     ws = ak.decode_workspace(q, g["k_cache"], g["v_cache"])
     out = ak.decode(q, g["k_cache"], g["v_cache"], g["seq_lens"], scale=scale, workspace=ws)
     assert ak.workspace_status(ws) == 0
-    assert_parity(out, ref, f"fold + decode {name}")
+    # the decode on the folded (bf16) query: element-wise against the oracle on that same query
+    q_bf16 = q.cpu()
+    assert_parity(out, oracle.decode(q_bf16, d["k_cache"], d["v_cache"], d["seq_lens"], scale), f"decode {name}")
+    # end to end against the pages' order (keys projected up in fp64): the folded query is rounded
+    # to bf16 (2^-9 relative), which perturbs every score of a row together, like the bf16 weights
+    # of the tensor-core prefill, so this comparison takes the per-vector rule
+    assert_parity_prefill(out, ref, f"fold + decode {name}")
 
 
 def test_fold_is_deterministic(cuda_device):
