@@ -35,6 +35,14 @@ __device__ __forceinline__ uint32_t smem_addr(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// The first 1024-byte aligned byte of a dynamic shared-memory array, reached by
+// pointer arithmetic on the array itself: pointers derived from it keep the
+// shared address space, so the compiler emits shared loads, stores and atomics
+// (an integer round trip would leave them generic).
+__device__ __forceinline__ uint8_t *align_smem_1024(uint8_t *raw) {
+    return raw + ((1024u - (smem_addr(raw) & 1023u)) & 1023u);
+}
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

@@ -160,16 +160,14 @@ __device__ long long produce_paged(const CUtensorMap *tm_k, const CUtensorMap *t
                                    uint64_t *empty_bar, volatile int *abort_flag, int lane) {
     int cur = sub_box_entry<TT>(a, w, lane);
     long long k = 0;
+    int stage = 0;        // k mod stages, kept incrementally
+    uint32_t par = 0;     // parity of k / stages
     for (long long t = t_begin; t < t_end; ++t, ++k) {
-        const int stage = (int)(k % a.stages);
         const int n_sub = sub_boxes<TT>(a, w);
         Walker wn = w;
         if (t + 1 < t_end) walker_advance<TT>(wn, a);
         const int nxt = (t + 1 < t_end) ? sub_box_entry<TT>(a, wn, lane) : 0;
-        if (k >= a.stages) {
-            const uint32_t parity = (uint32_t)(((k / a.stages) - 1) & 1);
-            mbar_wait_bounded(&empty_bar[stage], parity, a.wait_limit_ns, abort_flag, a.status);
-        }
+        if (k >= a.stages) mbar_wait_bounded(&empty_bar[stage], par ^ 1u, a.wait_limit_ns, abort_flag, a.status);
         if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
         uint8_t *sb = smem + (size_t)stage * a.stage_stride;
         if (lane == 0) mbar_arrive_expect_tx(&full_bar[stage], (uint32_t)n_sub * (a.sub_k_bytes + a.sub_v_bytes));
@@ -185,6 +183,10 @@ __device__ long long produce_paged(const CUtensorMap *tm_k, const CUtensorMap *t
         }
         cur = nxt;
         w = wn;
+        if (++stage == a.stages) {
+            stage = 0;
+            par ^= 1u;
+        }
     }
     return k;
 }
@@ -342,12 +344,10 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
                                        lane);
         } else if (lane == 0) {
             Walker w = w0;
+            int stage = 0;     // k mod stages, kept incrementally
+            uint32_t par = 0;  // parity of k / stages
             for (long long t = t_begin; t < t_end; ++t, ++k) {
-                const int stage = (int)(k % a.stages);
-                if (k >= a.stages) {
-                    const uint32_t parity = (uint32_t)(((k / a.stages) - 1) & 1);
-                    mbar_wait_bounded(&empty_bar[stage], parity, a.wait_limit_ns, abort_flag, a.status);
-                }
+                if (k >= a.stages) mbar_wait_bounded(&empty_bar[stage], par ^ 1u, a.wait_limit_ns, abort_flag, a.status);
                 if (*abort_flag) break;
                 uint8_t *sb = smem + (size_t)stage * a.stage_stride;
                 mbar_arrive_expect_tx(&full_bar[stage], a.stage_bytes);
@@ -355,6 +355,10 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
                 tma_load_4d(sb, &tm_k, &full_bar[stage], 0, w.g, w.i * TT, w.b);
                 tma_load_4d(sb + a.k_tile_bytes, &tm_v, &full_bar[stage], 0, v0, w.i * TT, w.b);
                 walker_advance<TT>(w, a);
+                if (++stage == a.stages) {
+                    stage = 0;
+                    par ^= 1u;
+                }
             }
         }
         if (lane == 0) {
@@ -385,8 +389,9 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
     int v_local = 0;
 
     Walker w = w0;
-    long long k = 0;
-    for (long long t = t_begin; t < t_end; ++t, ++k) {
+    int stage = 0;     // tile index mod stages, kept incrementally
+    uint32_t par = 0;  // parity of tile index / stages
+    for (long long t = t_begin; t < t_end; ++t) {
         const int h = w.g * QPK + hs;
         if (t == t_begin || w.i == 0) {
             // new split: this warp's query chunk, pre-scaled into the log2 domain
@@ -402,8 +407,7 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
             l_run = 0.f;
             v_local = h / a.q_per_v - (w.g * QPK) / a.q_per_v;
         }
-        const int stage = (int)(k % a.stages);
-        mbar_wait_bounded(&full_bar[stage], (uint32_t)((k / a.stages) & 1), a.wait_limit_ns, abort_flag, a.status);
+        mbar_wait_bounded(&full_bar[stage], par, a.wait_limit_ns, abort_flag, a.status);
         const uint8_t *sb = smem + (size_t)stage * a.stage_stride;
         const __nv_bfloat16 *Ks = reinterpret_cast<const __nv_bfloat16 *>(sb);
         const __nv_bfloat16 *Vs = reinterpret_cast<const __nv_bfloat16 *>(sb + a.k_tile_bytes);
@@ -483,6 +487,10 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty_bar[stage]);
+        if (++stage == a.stages) {
+            stage = 0;
+            par ^= 1u;
+        }
 
         // ---- end of this CTA's piece of the unit: write the split partial, maybe combine
         if (w.i == w.nt - 1 || t == t_end - 1) {

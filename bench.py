@@ -500,7 +500,7 @@ def time_paths(ak, peaks, steps: int, warmup: int):
     hbm = float(peaks["hbm_gbs"])
     res[w.name] = {"us": ms * 1e3, "algorithmic_bytes": nbytes, "gbs": nbytes / (ms * 1e-3) / 1e9,
                    "bound": "hbm", "peak_gbs": hbm, "frac": nbytes / (ms * 1e-3) / 1e9 / hbm,
-                   "launches_per_call": 4}
+                   "launches_per_call": 1}
     # the same selection with the pages' full-softmax weights (no renormalisation over the kept set)
     fn = lambda: ak.decode_topv(d["q"], d["k_cache"], d["v_cache"], d["seq_lens"], w.topk,  # noqa: E731
                                 scale=d["scale"], workspace=ws, full_weights=True)
@@ -509,7 +509,7 @@ def time_paths(ak, peaks, steps: int, warmup: int):
     ms = statistics.median(_timed_calls(fn, steps, flush))
     res[w.name + "_full_weights"] = {"us": ms * 1e3, "algorithmic_bytes": nbytes,
                                      "gbs": nbytes / (ms * 1e-3) / 1e9, "bound": "hbm", "peak_gbs": hbm,
-                                     "frac": nbytes / (ms * 1e-3) / 1e9 / hbm, "launches_per_call": 4}
+                                     "frac": nbytes / (ms * 1e-3) / 1e9 / hbm, "launches_per_call": 1}
     assert ak.workspace_status(ws) == 0
     return res
 

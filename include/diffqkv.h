@@ -267,10 +267,18 @@ diffqkv_status_t diffqkv_decode_from_host(const diffqkv_dims_t *dims, const void
 /* over them).                                                              */
 /* ------------------------------------------------------------------------ */
 
-/* Workspace bytes for diffqkv_decode_topv (0 if invalid).  Only the first
- * 256 bytes (a header whose first 32-bit word is the error word) must be zero
- * before the workspace's first use (diffqkv_workspace_init zero-fills the
- * whole workspace); each call clears the rest it needs by itself. */
+/* Workspace bytes for diffqkv_decode_topv (0 if invalid).  Zero-fill it
+ * before its first use (diffqkv_workspace_init); every call that completes
+ * leaves it reusable without clearing (its error word aside, which keeps the
+ * first device-side error until diffqkv_workspace_status reads it).  After a
+ * call that reported DIFFQKV_ERR_DEVICE_TIMEOUT, zero-fill it again.  Layout,
+ * with R = batch * n_q rows and U = batch * n_k (batch, K head) units, each
+ * region starting on a 256-byte boundary:
+ *   - a 256-byte header whose first 32-bit word is the error word;
+ *   - the counters, kept zero between calls: U x 4 uint32, R x 4 uint32, and
+ *     an R x 2048 uint32 histogram;
+ *   - scratch written before it is read within a call.
+ * Two calls that may run concurrently must not share a workspace. */
 size_t diffqkv_decode_topv_workspace_size(const diffqkv_dims_t *dims, int32_t t_max, int32_t topk);
 
 /*
@@ -290,9 +298,9 @@ size_t diffqkv_decode_topv_workspace_size(const diffqkv_dims_t *dims, int32_t t_
  * [0, t_max] are clamped to that range and flagged
  * DIFFQKV_ERR_DEVICE_SEQLEN in the workspace's error word, as
  * diffqkv_decode does.  A row with length 0 gets a zero output and an all -1
- * index row.  Launches four kernels on `stream`
- * (chained with programmatic dependent launch);
- * returns once they are queued.
+ * index row.  One cooperative kernel launch on `stream` (its CTAs wait on
+ * one another, with bounded waits, so the grid is sized to be resident at
+ * once: one CTA per SM); returns once it is queued.
  */
 diffqkv_status_t diffqkv_decode_topv(const diffqkv_dims_t *dims, const void *q, const void *k_cache,
                                      const void *v_cache, const int32_t *seq_lens, int32_t t_max,

@@ -137,10 +137,10 @@ def test_topv_rejects_before_launch():
     assert _topv_raw(d, idx=0x7002) == _capi.MISALIGNED
     assert _topv_raw(d, ws_bytes=16) == _capi.WORKSPACE
     assert _capi.lib().diffqkv_decode_topv_workspace_size(ctypes.byref(d), 131072, 1024) > 0
-    # 18 bytes per (row, position) plus the zeroed histograms
+    # 14 bytes per (row, position): candidate position and score, ambiguous position, two state bytes
     small = _capi.lib().diffqkv_decode_topv_workspace_size(ctypes.byref(d), 1024, 8)
     large = _capi.lib().diffqkv_decode_topv_workspace_size(ctypes.byref(d), 2048, 8)
-    assert large - small == d.batch * d.n_q * 1024 * 18
+    assert large - small == d.batch * d.n_q * 1024 * 14
 
 
 def test_decode_append_rejects_before_launch():

@@ -15,6 +15,16 @@ from parity import assert_parity
 pytestmark = pytest.mark.gpu
 
 
+def _a256(x):
+    return -(-x // 256) * 256
+
+
+def _counter_region(batch, n_q, n_k):
+    """Byte range of the counters that every completed call leaves zero (the header's layout)."""
+    rows, units = batch * n_q, batch * n_k
+    return 256, 256 + _a256(_a256(units * 16) + _a256(rows * 16) + rows * 2048 * 4)
+
+
 def _gpu(d, topk, dev, expect=0, **kw):
     """Selective-V decode through the C ABI; the workspace's error word must read `expect`."""
     g = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
@@ -129,8 +139,8 @@ def test_full_topv_workload(cuda_device):
 
 @pytest.mark.parametrize("topk", [64, 1024, 4000])
 def test_workspace_reuse_is_bitwise_stable(cuda_device, topk):
-    """Two calls on one workspace (the gather's per-row counters must come back to
-    zero) give identical bits: the parts of a row are added in a fixed order."""
+    """Two calls on one workspace (every counter must come back to zero) give identical bits:
+    the parts of a row are added in a fixed order."""
     d = wl.random_decode_inputs(3, 6000, wl.DIFFQKV, seed=308, seq_lens=[6000, 2500, 4100])
     g = {k: (v.to(cuda_device) if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
     dims = ak.make_dims(3, 16, 4, 16, 64, 128, d["scale"])
@@ -142,6 +152,8 @@ def test_workspace_reuse_is_bitwise_stable(cuda_device, topk):
         assert ak.workspace_status(ws) == 0
         runs.append((out.clone(), idx.clone()))
     assert torch.equal(runs[0][0], runs[1][0]) and torch.equal(runs[0][1], runs[1][1])
+    c0, c1 = _counter_region(3, 16, 4)
+    assert torch.count_nonzero(ws[c0:c1]) == 0, "counters not returned to zero"
     r_out, r_idx = oracle.decode_topv(d["q"], d["k_cache"], d["v_cache"], d["seq_lens"], topk, d["scale"])
     assert np.array_equal(runs[0][1].cpu().numpy(), r_idx)
     assert_parity(runs[0][0], r_out, f"reuse k={topk}")
@@ -178,15 +190,16 @@ def test_out_of_range_lengths_are_clamped_and_flagged(cuda_device):
 
 @pytest.mark.parametrize("topk", [1, 100, 1024])
 def test_poisoned_workspace_is_never_read_before_written(cuda_device, topk):
-    """Every byte after the workspace header (scores, candidate lists, ambiguous lists, per-row
-    words) starts as 0xFF: a kernel that read scratch this call did not write would change the
-    index sets or the output."""
+    """Every byte of the scratch after the counters (candidate lists, ambiguous lists, kept scores,
+    per-row words, per-part sums) starts as 0xFF: a kernel that read scratch this call did not
+    write would change the index sets or the output.  The counters are zero again afterwards."""
     lens = [5000, 1, 2047, 0, 3000]
     d = wl.random_decode_inputs(len(lens), 5000, wl.DIFFQKV, seed=311, seq_lens=lens)
     g = {k: (v.to(cuda_device) if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
     dims = ak.make_dims(len(lens), 16, 4, 16, 64, 128, d["scale"])
     ws = ak.decode_topv_workspace(dims, 5000, topk, cuda_device)
-    ws[256:] = 0xFF
+    c0, c1 = _counter_region(len(lens), 16, 4)
+    ws[c1:] = 0xFF
     out, idx = ak.decode_topv(g["q"], g["k_cache"], g["v_cache"], g["seq_lens"], topk, scale=d["scale"],
                               workspace=ws)
     assert ak.workspace_status(ws) == 0
@@ -194,3 +207,4 @@ def test_poisoned_workspace_is_never_read_before_written(cuda_device, topk):
     assert np.array_equal(idx.cpu().numpy(), r_idx)
     assert torch.isfinite(out.float()).all()
     assert_parity(out, r_out, f"poisoned workspace k={topk}")
+    assert torch.count_nonzero(ws[c0:c1]) == 0, "counters not returned to zero"
