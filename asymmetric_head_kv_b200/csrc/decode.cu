@@ -591,26 +591,50 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
                     named_barrier(1, NCW * 32);
                 }
                 constexpr int ITEMS = QPK * (DV / 4);
+                constexpr int kBatch = QPK >= 16 ? 1 : 4;  // partials loaded together (one L2 round trip per batch)
                 for (int it = tid; it < ITEMS; it += NCW * 32) {
                     const int h2 = it / (DV / 4);
                     const int d4 = it % (DV / 4);
+                    constexpr int kBatchM = QPK >= 16 ? 4 : 16;  // maxima only: wider batches
                     float M = -INFINITY;
-                    for (long long cc = first; cc <= last; ++cc)
-                        M = fmaxf(M, __ldcg(a.partials + ((size_t)(u + cc) * QPK + h2) * (DV + kPartialPad) + DV));
+                    for (long long c0 = first; c0 <= last; c0 += kBatchM) {
+                        float mv[kBatchM];
+#pragma unroll
+                        for (int e = 0; e < kBatchM; ++e)
+                            mv[e] = c0 + e <= last
+                                        ? __ldcg(a.partials + ((size_t)(u + c0 + e) * QPK + h2) * (DV + kPartialPad) + DV)
+                                        : -INFINITY;
+#pragma unroll
+                        for (int e = 0; e < kBatchM; ++e) M = fmaxf(M, mv[e]);
+                    }
                     const float s_new = append ? merge_s[h2] : -INFINITY;
                     M = fmaxf(M, s_new);
                     const float Mu = (M == -INFINITY) ? 0.f : M;
                     float L = 0.f;
                     float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
-                    for (long long cc = first; cc <= last; ++cc) {
-                        const float *src = a.partials + ((size_t)(u + cc) * QPK + h2) * (DV + kPartialPad);
-                        const float f = fast_exp2(__ldcg(src + DV) - Mu);
-                        L = fmaf(f, __ldcg(src + DV + 1), L);
-                        const float4 x = __ldcg(reinterpret_cast<const float4 *>(src) + d4);
-                        O.x = fmaf(f, x.x, O.x);
-                        O.y = fmaf(f, x.y, O.y);
-                        O.z = fmaf(f, x.z, O.z);
-                        O.w = fmaf(f, x.w, O.w);
+                    for (long long c0 = first; c0 <= last; c0 += kBatch) {
+                        float mv[kBatch], lv[kBatch];
+                        float4 xv[kBatch];
+#pragma unroll
+                        for (int e = 0; e < kBatch; ++e) {
+                            if (c0 + e <= last) {
+                                const float *src = a.partials + ((size_t)(u + c0 + e) * QPK + h2) * (DV + kPartialPad);
+                                mv[e] = __ldcg(src + DV);
+                                lv[e] = __ldcg(src + DV + 1);
+                                xv[e] = __ldcg(reinterpret_cast<const float4 *>(src) + d4);
+                            }
+                        }
+                        // the same fixed order over the partials as one at a time
+#pragma unroll
+                        for (int e = 0; e < kBatch; ++e) {
+                            if (c0 + e > last) break;
+                            const float f = fast_exp2(mv[e] - Mu);
+                            L = fmaf(f, lv[e], L);
+                            O.x = fmaf(f, xv[e].x, O.x);
+                            O.y = fmaf(f, xv[e].y, O.y);
+                            O.z = fmaf(f, xv[e].z, O.z);
+                            O.w = fmaf(f, xv[e].w, O.w);
+                        }
                     }
                     if (append) {  // the new token: m = s_new, l = 1, o = v_new
                         const float f = fast_exp2(s_new - Mu);

@@ -75,7 +75,7 @@ constexpr int kMaxStages = 6;
 constexpr int kEmitIters = 8;            // float4 vectors per thread and emission chunk (32 mask bits)
 constexpr int kRowInfoWords = 8;
 enum RowInfo { kRiBucket = 0, kRiAbove = 1, kRiTwoDelta = 2, kRiMax = 3, kRiKept = 4, kRiFullSum = 5 };
-enum UnitSync { kUsHist = 0, kUsCand = 1, kUsSelDone = 2, kUsKmax = 3 };
+enum UnitSync { kUsHist = 0, kUsCand = 1, kUsKmax = 3 };
 enum RowSync { kRsSelected = 0, kRsGathered = 1, kRsCand = 2 };
 constexpr int kDynSmemCap = 219 * 1024;  // dynamic shared memory (the static part needs the rest of 227 KB)
 
@@ -88,7 +88,7 @@ struct TopvArgs {
     int32_t *idx_out;
     int32_t *status;
     // zero before the first call, left zero by every call that completes
-    uint32_t *unit_sync;  // [units][4]: H arrivals, C arrivals, rows selected, max |k| (bf16 bits)
+    uint32_t *unit_sync;  // [units][4]: H arrivals, C arrivals, -, max |k| (bf16 bits)
     uint32_t *row_sync;   // [rows][4]: selected flag, parts gathered, candidate count, -
     uint32_t *hist1;      // [rows][2048]: top 11 key bits of every score
     // written and read within a call
@@ -148,6 +148,23 @@ __device__ __forceinline__ uint32_t ld_acquire(const uint32_t *p) {
     return v;
 }
 
+// Release operations at GPU scope.  After a __syncthreads, one of them by thread 0
+// publishes every write the CTA made before it (release is cumulative over the
+// writes the barrier ordered before it); a reader's ld.acquire of the value, a
+// __syncthreads, and L2 loads see them all.
+__device__ __forceinline__ void red_release_add(uint32_t *p, uint32_t v) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ void st_release(uint32_t *p, uint32_t v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// Add with acquire and release semantics; returns the old value.
+__device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t *p, uint32_t v) {
+    uint32_t old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+
 // Thread 0 waits, for at most limit_ns, until *ctr >= target; false when the wait ran out
 // (DIFFQKV_ERR_DEVICE_TIMEOUT recorded).
 __device__ bool wait_at_least(const uint32_t *ctr, uint32_t target, const TopvArgs &a) {
@@ -168,11 +185,7 @@ __device__ bool wait_at_least(const uint32_t *ctr, uint32_t target, const TopvAr
 // afterwards with L2 loads (__ldcg).
 __device__ bool cta_wait_at_least(const uint32_t *ctr, uint32_t target, const TopvArgs &a, volatile int *flag) {
     __syncthreads();
-    if (threadIdx.x == 0) {
-        const bool ok = wait_at_least(ctr, target, a);
-        __threadfence();
-        *flag = ok ? 1 : 0;
-    }
+    if (threadIdx.x == 0) *flag = wait_at_least(ctr, target, a) ? 1 : 0;
     __syncthreads();
     const bool ok = *flag != 0;
     __syncthreads();
@@ -182,10 +195,7 @@ __device__ bool cta_wait_at_least(const uint32_t *ctr, uint32_t target, const To
 // Every thread calls this after its global writes: they become visible before *ctr grows by one.
 __device__ __forceinline__ void cta_arrive(uint32_t *ctr) {
     __syncthreads();
-    if (threadIdx.x == 0) {
-        __threadfence();
-        atomicAdd(ctr, 1u);
-    }
+    if (threadIdx.x == 0) red_release_add(ctr, 1u);
 }
 
 // ------------------------------------------------------------------ block helpers
@@ -1019,16 +1029,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 a.rowinfo[kRowInfoWords * row + kRiKept] = (uint32_t)nsel;
                 a.rowinfo[kRowInfoWords * row + kRiFullSum] = __float_as_uint(full_sum);
                 a.row_sync[(size_t)row * 4 + kRsCand] = 0u;
-                __threadfence();
-                atomicExch(a.row_sync + (size_t)row * 4 + kRsSelected, 1u);
-                // the unit's last selected row resets the unit's counters: every part of the unit has
-                // passed its waits on H and C by now
-                if (atomicAdd(usync + kUsSelDone, 1u) == (uint32_t)QPK - 1) {
-                    usync[kUsHist] = 0u;
-                    usync[kUsCand] = 0u;
-                    usync[kUsSelDone] = 0u;
-                    usync[kUsKmax] = 0u;
-                }
+                st_release(a.row_sync + (size_t)row * 4 + kRsSelected, 1u);  // after the idx / score writes
             }
             __syncthreads();
         }
@@ -1038,7 +1039,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (tid == 0) {
             bool ok = true;
             for (int hh = 0; hh < QPK && ok; ++hh) ok = wait_at_least(a.row_sync + (size_t)(row0 + hh) * 4 + kRsSelected, 1u, a);
-            __threadfence();
             *flag = ok ? 1 : 0;
         }
         __syncthreads();
@@ -1054,7 +1054,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             constexpr int WPR = kWarps / QPK;          // warps per row (every warp gathers)
             constexpr int CPV = DV / 8;                // lanes per V row
             constexpr int RPW = 32 / CPV;              // V rows per warp step
-            constexpr int GU = 8;                      // V rows in flight per lane
+            constexpr int GU = 16;                     // V rows in flight per lane
             float *o_s = reinterpret_cast<float *>(overlay);  // [kWarps][DV + 4]
             const int vc = lane % CPV, vs = lane / CPV;
             {
@@ -1119,11 +1119,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             __syncthreads();
             if (tid == 0) {
-                __threadfence();
+                // release this part's sums; the last part also acquires every other part's
                 for (int hh = 0; hh < QPK; ++hh)
                     sh.combine[hh] =
-                        atomicAdd(a.row_sync + (size_t)(row0 + hh) * 4 + kRsGathered, 1u) == (uint32_t)Y - 1;
-                __threadfence();
+                        atom_add_acq_rel(a.row_sync + (size_t)(row0 + hh) * 4 + kRsGathered, 1u) == (uint32_t)Y - 1;
             }
             __syncthreads();
             // the last part of a row adds the Y parts in part order and writes the output
@@ -1140,9 +1139,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     a.out[(size_t)row * DV + c] = __float2bfloat16(lt > 0.f ? acc / lt : 0.f);
                 }
                 if (tid == 0) {
-                    // every part of the row has passed its wait on the flag
+                    // every part of the row has passed its wait on the flag; and since every part of the
+                    // unit waited for every row of the group to be selected, every wait on the unit's
+                    // counters (H by all parts, C by the select CTAs) is over: reset them too
                     a.row_sync[(size_t)row * 4 + kRsGathered] = 0u;
                     a.row_sync[(size_t)row * 4 + kRsSelected] = 0u;
+                    usync[kUsHist] = 0u;
+                    usync[kUsCand] = 0u;
+                    usync[kUsKmax] = 0u;
                 }
             }
             __syncthreads();

@@ -212,6 +212,10 @@ def time_decode(ak, w: wl.DecodeWorkload, steps: int, warmup: int, world: int, s
             starts[i].record(stream)
             step()
             ends[i].record(stream)
+        # let the clock sampler thread run while the GPU works: torch.cuda.synchronize() would hold
+        # the interpreter lock for the whole wait
+        while not ends[-1].query():
+            time.sleep(0.0001)
         torch.cuda.synchronize()
     barrier(world)
     region_ms = starts[0].elapsed_time(ends[-1])
