@@ -22,6 +22,7 @@ __all__ = [
     "decode", "decode_workspace", "decode_plan", "decode_from_host", "decode_topv", "decode_topv_workspace",
     "prefill_causal", "device_status", "selftest_wait_timeout", "DiffqkvError", "Dims", "library_path",
     "decode_noalloc", "decode_append", "decode_paged", "prefill_causal_prefix", "fold_query", "workspace_status",
+    "decode_topv_paged",
 ]
 
 library_path = _capi.LIB_PATH
@@ -263,6 +264,41 @@ def decode_topv(q, k_cache, v_cache, seq_lens, topk: int, *, scale: Optional[flo
                                        t_max, msl, topk, _ptr(out), _ptr(idx_out), _ptr(workspace),
                                        workspace.numel(), _stream_ptr(stream))
     check(st, "diffqkv_decode_topv")
+    return out, idx_out
+
+
+def decode_topv_paged(q, k_pages, v_pages, block_table, seq_lens, topk: int, *, scale: Optional[float] = None,
+                      max_seq_len: Optional[int] = None, out=None, idx_out=None, workspace=None,
+                      full_weights: bool = False, stream: Optional[torch.cuda.Stream] = None):
+    """:func:`decode_topv` over paged caches: K and V page pools [num_pages, page_size, heads, d] and an
+    int32 block table [B, max_blocks] of pool pages (position j of sequence b is row j % page_size of pool
+    page block_table[b, j // page_size]).  Returns (out, idx) as :func:`decode_topv`."""
+    _bf16_dev(q, "q", 3)
+    _bf16_dev(k_pages, "k_pages", 4)
+    _bf16_dev(v_pages, "v_pages", 4)
+    for t, name in ((seq_lens, "seq_lens"), (block_table, "block_table")):
+        if t.dtype != torch.int32 or not t.is_cuda:
+            raise TypeError(f"{name} must be an int32 CUDA tensor")
+    if block_table.dim() != 2 or not block_table.is_contiguous():
+        raise ValueError("block_table must be a contiguous [B, max_blocks] tensor")
+    B, n_q, d_k = q.shape
+    num_pages, page_size, n_k, _ = k_pages.shape
+    n_v, d_v = v_pages.shape[2], v_pages.shape[3]
+    max_blocks = block_table.shape[1]
+    t_max = max_blocks * page_size
+    dims = make_dims(B, n_q, n_k, n_v, d_k, d_v, d_k ** -0.5 if scale is None else scale)
+    if out is None:
+        out = torch.empty((B, n_q, d_v), dtype=torch.bfloat16, device=q.device)
+    if idx_out is None:
+        idx_out = torch.empty((B, n_q, topk), dtype=torch.int32, device=q.device)
+    if workspace is None:
+        workspace = decode_topv_workspace(dims, t_max, topk, q.device)
+    msl = t_max if max_seq_len is None else int(max_seq_len)
+    flags = _capi.TOPV_FULL_SOFTMAX_WEIGHTS if full_weights else 0
+    st = lib().diffqkv_decode_topv_paged(ctypes.byref(dims), _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table),
+                                         max_blocks, page_size, num_pages, _ptr(seq_lens), msl, topk, flags, _ptr(out),
+                                         _ptr(idx_out), _ptr(workspace), workspace.numel(), _stream_ptr(stream))
+    check(st, "diffqkv_decode_topv_paged")
     return out, idx_out
 
 

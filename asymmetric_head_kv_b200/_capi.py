@@ -88,6 +88,8 @@ SIGNATURES = {
     "diffqkv_decode_topv_workspace_size": ([_DIMS, _I32, _I32], _SZ),
     "diffqkv_decode_topv": ([_DIMS, _P, _P, _P, _P, _I32, _I32, _I32, _P, _P, _P, _SZ, _P], _I32),
     "diffqkv_decode_topv_ex": ([_DIMS, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _P, _P, _P, _SZ, _P], _I32),
+    "diffqkv_decode_topv_paged": ([_DIMS, _P, _P, _P, _P, _I32, _I32, _I32, _P, _I32, _I32, _I32, _P, _P, _P, _SZ,
+                                   _P], _I32),
     "diffqkv_prefill_causal": ([_DIMS, _P, _P, _P, _I32, _P, _P], _I32),
     "diffqkv_prefill_causal_prefix": ([_DIMS, _P, _P, _P, _I32, _I32, _P, _P], _I32),
     "diffqkv_prefill_causal_ex": ([_DIMS, _P, _P, _P, _I32, _I32, _P, _P, _P], _I32),

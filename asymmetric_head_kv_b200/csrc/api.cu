@@ -274,6 +274,19 @@ diffqkv_status_t diffqkv_decode_topv_ex(const diffqkv_dims_t *dims, const void *
                                 workspace, workspace_bytes, (cudaStream_t)stream, flags);
 }
 
+diffqkv_status_t diffqkv_decode_topv_paged(const diffqkv_dims_t *dims, const void *q, const void *k_pages,
+                                           const void *v_pages, const int32_t *block_table, int32_t max_blocks,
+                                           int32_t page_size, int32_t num_pages, const int32_t *seq_lens,
+                                           int32_t max_seq_len, int32_t topk, int32_t flags, void *out,
+                                           int32_t *idx_out, void *workspace, size_t workspace_bytes,
+                                           diffqkv_stream_t stream) {
+    if (max_blocks < 1 || page_size < 1 || (long long)max_blocks * page_size > 0x7fffffffLL)
+        return DIFFQKV_ERR_INVALID_ARG;
+    const diffqkv::PagedCache paged{block_table, max_blocks, page_size, num_pages};
+    return diffqkv::topv_launch(dims, q, k_pages, v_pages, seq_lens, max_blocks * page_size, max_seq_len, topk, out,
+                                idx_out, workspace, workspace_bytes, (cudaStream_t)stream, flags, &paged);
+}
+
 diffqkv_status_t diffqkv_prefill_causal(const diffqkv_dims_t *dims, const void *q, const void *k, const void *v,
                                         int32_t seq_len, void *out, diffqkv_stream_t stream) {
     return diffqkv::prefill_launch(dims, q, k, v, seq_len, out, (cudaStream_t)stream);

@@ -77,10 +77,11 @@ diffqkv_status_t decode_noalloc_launch(const diffqkv_dims_t *d, const void *q, c
 
 // topv.cu
 size_t topv_workspace_size(const diffqkv_dims_t *d, int32_t t_max, int32_t topk);
+// paged given: k_cache / v_cache are page pools and t_max = max_blocks * page_size.
 diffqkv_status_t topv_launch(const diffqkv_dims_t *d, const void *q, const void *k_cache, const void *v_cache,
                              const int32_t *seq_lens, int32_t t_max, int32_t max_seq_len, int32_t topk,
                              void *out, int32_t *idx_out, void *workspace, size_t workspace_bytes,
-                             cudaStream_t stream, int32_t flags = 0);
+                             cudaStream_t stream, int32_t flags = 0, const PagedCache *paged = nullptr);
 
 // prefill.cu
 // status: device word the kernel reports into (NULL: the per-device word).

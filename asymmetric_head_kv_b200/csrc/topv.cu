@@ -47,6 +47,7 @@
 #include <math.h>
 
 #include <algorithm>
+#include <numeric>
 
 #include "common.cuh"
 #include "internal.h"
@@ -98,6 +99,8 @@ struct TopvArgs {
     int32_t *cand_j;      // [rows][t_pad]
     float *cand_s;        // [rows][t_pad]
     float *kept_s;        // [rows][k_pad]: scores of the kept positions, in idx_out order
+    int32_t *kept_row;    // [rows][k_pad]: their cache rows (sequence b position j: b t_max + j, or the
+                          // pool row of a paged cache)
     int32_t *alist;       // [rows][t_pad]: ambiguous positions
     uint8_t *astate;      // [rows][t_pad]
     uint8_t *adigit;      // [rows][t_pad]
@@ -107,11 +110,32 @@ struct TopvArgs {
     int32_t score_stride; // floats between two rows' score arrays in shared memory
     int32_t cand_cap;     // candidates the select keeps in shared memory
     int32_t full_weights;
+    // paged caches: block_table == null means contiguous [B, t_max, heads, d] caches; else K and V
+    // are pools [num_pages, page_size, heads, d] and position j of sequence b is row j % page_size
+    // of pool page block_table[b][j / page_size]
+    const int32_t *block_table;
+    int32_t max_blocks, page_size, num_pages;
+    int32_t sub_rows;     // positions per TMA sub-box of a paged tile (divides kTile and page_size)
     float scale_log2;
     uint64_t wait_limit_ns;
 };
 
 __device__ __forceinline__ int clamp_len(int v, int t_max) { return v < 0 ? 0 : (v > t_max ? t_max : v); }
+
+// Pool page of logical page pi of sequence b; an entry outside [0, num_pages) is flagged
+// DIFFQKV_ERR_DEVICE_PAGE and page 0 used in its place, so no access leaves the pools.
+__device__ __forceinline__ int paged_page(const TopvArgs &a, int b, int pi) {
+    const int e = __ldg(a.block_table + (size_t)b * a.max_blocks + pi);
+    if (e >= 0 && e < a.num_pages) return e;
+    record_error(a.status, DIFFQKV_ERR_DEVICE_PAGE);
+    return 0;
+}
+
+// Cache row of position j of sequence b: [row][heads][d] indexing of the K and V caches or pools.
+__device__ __forceinline__ long long cache_row(const TopvArgs &a, int b, int j) {
+    if (!a.block_table) return (long long)b * a.t_max + j;
+    return (long long)paged_page(a, b, j / a.page_size) * a.page_size + j % a.page_size;
+}
 
 // max(a, b, c) in one instruction (three-input form of max.f32, sm_100).
 __device__ __forceinline__ float fmax3f(float a, float b, float c) {
@@ -529,7 +553,55 @@ __global__ void __launch_bounds__(kThreads, 1)
             q_s[i] = __bfloat162float(a.q[((size_t)row0 + hh) * DK + c]);
         }
         __syncthreads();
-        if (warp == kConsumerWarps) {
+        if (warp == kConsumerWarps && a.block_table) {
+            // ---- producer, paged caches: the whole warp; lane f issues sub-box f (sub_rows positions
+            //      inside one page) of each tile, so a tile's sub-boxes leave as one warp instruction,
+            //      and loads its block-table entry a tile ahead.  Only sub-boxes holding cached
+            //      positions are loaded (later table entries may hold anything).
+            if (te > tb) {
+                if (lane == 0) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                __syncwarp();
+                const long long k0 = ring_k;
+                const int per_tile = kTile / a.sub_rows;
+                auto n_sub = [&](int t) { return (min(kTile, T - t * kTile) + a.sub_rows - 1) / a.sub_rows; };
+                auto entry = [&](int t, int f) {
+                    return f < n_sub(t) ? paged_page(a, b, (t * kTile + f * a.sub_rows) / a.page_size) : 0;
+                };
+                int cur = lane < per_tile ? entry(tb, lane) : 0;
+                int st = (int)(k0 % a.stages);
+                uint32_t par = (uint32_t)((k0 / a.stages) & 1);
+                bool wrapped = k0 >= a.stages;
+                long long issued_end = k0;
+                for (int t = tb; t < te; ++t) {
+                    const int ns = n_sub(t);
+                    const int nxt = (t + 1 < te && lane < per_tile) ? entry(t + 1, lane) : 0;
+                    if (wrapped) mbar_wait_bounded(&empty_bar[st], par ^ 1u, a.wait_limit_ns, abort_flag, a.status);
+                    if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
+                    uint8_t *dst = ring + (size_t)st * TILE_BYTES;
+                    if (lane == 0) mbar_arrive_expect_tx(&full_bar[st], (uint32_t)(ns * a.sub_rows * DK * 2));
+                    __syncwarp();
+                    for (int f = lane; f < ns; f += 32) {
+                        const int page = f == lane ? cur : entry(t, f);
+                        const int row = (t * kTile + f * a.sub_rows) % a.page_size;
+#pragma unroll
+                        for (int kb = 0; kb < DK / 64; ++kb)
+                            tma_load_4d(dst + kb * (kTile * 128) + f * a.sub_rows * 128, &tm_k, &full_bar[st],
+                                        kb * 64, g, row, page);
+                    }
+                    cur = nxt;
+                    issued_end = k0 + (t - tb) + 1;
+                    if (++st == a.stages) {
+                        st = 0;
+                        par ^= 1u;
+                        wrapped = true;
+                    }
+                }
+                if (lane == 0)
+                    for (long long kk = (issued_end - a.stages > k0 ? issued_end - a.stages : k0); kk < issued_end; ++kk)
+                        mbar_wait_bounded(&full_bar[kk % a.stages], (uint32_t)((kk / a.stages) & 1), a.wait_limit_ns,
+                                          nullptr, a.status);
+            }
+        } else if (warp == kConsumerWarps) {
             // ---- producer: one lane issues the TMA loads of this part's tiles into the ring
             if (lane == 0 && te > tb) {
                 // the ring may hold the previous round's select and gather data, written by the generic proxy
@@ -816,6 +888,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int row = row0 + hh;
             int32_t *idx = a.idx_out + (size_t)row * K;
             float *ks = a.kept_s + (size_t)row * a.k_pad;
+            int32_t *kr = a.kept_row + (size_t)row * a.k_pad;
             const uint32_t nc = min(__ldcg(a.row_sync + (size_t)row * 4 + kRsCand), (uint32_t)T);
             const int nwords = (T + 31) / 32;
             // overlay: bitmap | word prefixes | histogram | candidate positions | candidate scores
@@ -848,6 +921,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int jj = cj[i];
                     idx[jj] = jj;
                     ks[jj] = cs[i];
+                    kr[jj] = (int32_t)cache_row(a, b, jj);
                     mx = fmaxf(mx, cs[i]);
                 }
                 for (int i = T + tid; i < K; i += kThreads) idx[i] = -1;
@@ -909,8 +983,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncthreads();
                 const int na = sh.sh_na;
                 const int need = K - sh.sh_cnt_in;  // 1 <= need <= na when the bound holds
-                const __nv_bfloat16 *krow0 = a.k + ((size_t)b * a.t_max * a.n_k + g) * DK;
-                const size_t kstride = (size_t)a.n_k * DK;
+                // K row of position jj (exact keys of the ambiguous positions)
+                auto krow = [&](int jj) {
+                    return reinterpret_cast<const uint16_t *>(a.k + ((size_t)cache_row(a, b, jj) * a.n_k + g) * DK);
+                };
                 auto keep = [&](int jj) { atomicOr(bitmap + (jj >> 5), 1u << (jj & 31)); };
                 if (need <= 0) {
                     // nothing left to choose (cannot happen when the bound holds)
@@ -920,8 +996,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // rank the few ambiguous positions pairwise by exact key (a warp per key)
                     for (int rr = warp; rr < na; rr += kWarps) {
                         const int jj = sh.alist[rr];
-                        exact_key_warp<DK>(sh.qbits, reinterpret_cast<const uint16_t *>(krow0 + (size_t)jj * kstride),
-                                           jj, sh.keys[rr], lane);
+                        exact_key_warp<DK>(sh.qbits, krow(jj), jj, sh.keys[rr], lane);
                     }
                     __syncthreads();
                     if (tid < na) {
@@ -946,8 +1021,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             if (i < na && ast[i] == 0) {
                                 uint32_t key[kKeyWords];
                                 const int jj = alist[i];
-                                exact_key<DK>(sh.qbits, reinterpret_cast<const uint16_t *>(krow0 + (size_t)jj * kstride),
-                                              jj, key);
+                                exact_key<DK>(sh.qbits, krow(jj), jj, key);
                                 bkt = (int)((key[p >> 2] >> (24 - 8 * (p & 3))) & 0xffu);
                                 adg[i] = (uint8_t)bkt;
                             }
@@ -994,6 +1068,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (slot < (uint32_t)K) {  // more than K kept only if the bound failed (flagged below)
                             idx[slot] = jj;
                             ks[slot] = cs[i];
+                            kr[slot] = (int32_t)cache_row(a, b, jj);
                             mx = fmaxf(mx, cs[i]);
                         }
                     }
@@ -1064,9 +1139,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int nsel = sh.row_nsel[hh];
                 const float m = sh.row_m[hh];
                 const int i_begin = (int)(((long long)nsel * j) / Y), i_end = (int)(((long long)nsel * (j + 1)) / Y);
-                const int32_t *idx = a.idx_out + (size_t)row * K;
                 const float *ks = a.kept_s + (size_t)row * a.k_pad;
-                const __nv_bfloat16 *vbase = a.v + ((size_t)b * a.t_max * a.n_v + vh) * DV + vc * 8;
+                const int32_t *kr = a.kept_row + (size_t)row * a.k_pad;
+                const __nv_bfloat16 *vbase = a.v + (size_t)vh * DV + vc * 8;
                 const size_t vstride = (size_t)a.n_v * DV;
                 float o[8];
 #pragma unroll
@@ -1078,7 +1153,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int uu = 0; uu < GU; ++uu) {
                         const int i = i0 + uu * WPR * RPW;
-                        jj[uu] = i < i_end ? __ldcg(idx + i) : -1;
+                        jj[uu] = i < i_end ? __ldcg(kr + i) : -1;  // the kept position's cache row
                         sx[uu] = i < i_end ? __ldcg(ks + i) : -INFINITY;
                     }
                     uint4 vv[GU];
@@ -1248,20 +1323,34 @@ size_t topv_workspace_size(const diffqkv_dims_t *d, int32_t t_max, int32_t topk)
     const size_t per = padded_len(t_max);
     return kTopvHeader + align_up(zeroed_bytes(d), 256) + align_up(rows * kRowInfoWords * 4, 256) +
            align_up(rows * kMaxParts * sizeof(float2), 256) + align_up(rows * kMaxParts * (d->d_v + 4) * 4, 256) +
-           align_up(rows * per * 4, 256) * 3 + align_up(rows * padded_k(topk) * 4, 256) +
+           align_up(rows * per * 4, 256) * 3 + align_up(rows * padded_k(topk) * 4, 256) * 2 +
            align_up(rows * per, 256) * 2;
 }
 
 diffqkv_status_t topv_launch(const diffqkv_dims_t *d, const void *q, const void *k_cache, const void *v_cache,
                              const int32_t *seq_lens, int32_t t_max, int32_t max_seq_len, int32_t topk, void *out,
                              int32_t *idx_out, void *workspace, size_t workspace_bytes, cudaStream_t stream,
-                             int32_t flags) {
+                             int32_t flags, const PagedCache *paged) {
     diffqkv_status_t st = validate_dims(d);
     if (st != DIFFQKV_OK) return st;
     if (!q || !k_cache || !v_cache || !seq_lens || !out || !idx_out || t_max < 1 || topk < 1)
         return DIFFQKV_ERR_INVALID_ARG;
     if (t_max > kTopvMaxContext) return DIFFQKV_ERR_UNSUPPORTED;
     if (flags & ~DIFFQKV_TOPV_FULL_SOFTMAX_WEIGHTS) return DIFFQKV_ERR_INVALID_ARG;
+    int sub_rows = kTile;
+    if (paged) {
+        if (!paged->block_table || paged->max_blocks < 1 || paged->page_size < 1 || paged->num_pages < 1 ||
+            (long long)paged->max_blocks * paged->page_size != t_max)
+            return DIFFQKV_ERR_INVALID_ARG;
+        if (reinterpret_cast<uintptr_t>(paged->block_table) & 3u) return DIFFQKV_ERR_MISALIGNED;
+        // a tile is loaded as sub-boxes of gcd(tile, page) positions, each inside one page; with the
+        // 128-byte swizzle every sub-box must start on an 8-row boundary
+        sub_rows = std::gcd(kTile, (int)paged->page_size);
+        if (sub_rows % 8 != 0) return DIFFQKV_ERR_UNSUPPORTED;
+        if ((long long)paged->num_pages * paged->page_size > 0x7fffffffLL) return DIFFQKV_ERR_UNSUPPORTED;
+    } else if ((long long)d->batch * t_max > 0x7fffffffLL) {
+        return DIFFQKV_ERR_UNSUPPORTED;  // kept positions' cache rows are int32
+    }
     const int qpk = d->n_q / d->n_k;
     TopvFn fn = pick_kernel(d->d_k, d->d_v, qpk);
     if (!fn) return DIFFQKV_ERR_UNSUPPORTED;
@@ -1301,6 +1390,8 @@ diffqkv_status_t topv_launch(const diffqkv_dims_t *d, const void *q, const void 
     ws += align_up(rows * t_pad * 4, 256);
     a.kept_s = reinterpret_cast<float *>(ws);
     ws += align_up(rows * padded_k(topk) * 4, 256);
+    a.kept_row = reinterpret_cast<int32_t *>(ws);
+    ws += align_up(rows * padded_k(topk) * 4, 256);
     a.astate = ws;
     ws += align_up(rows * t_pad, 256);
     a.adigit = ws;
@@ -1326,14 +1417,22 @@ diffqkv_status_t topv_launch(const diffqkv_dims_t *d, const void *q, const void 
     a.score_stride = plan.score_stride;
     a.cand_cap = plan.cand_cap;
     a.full_weights = (flags & DIFFQKV_TOPV_FULL_SOFTMAX_WEIGHTS) ? 1 : 0;
+    a.block_table = paged ? paged->block_table : nullptr;
+    a.max_blocks = paged ? paged->max_blocks : 0;
+    a.page_size = paged ? paged->page_size : 0;
+    a.num_pages = paged ? paged->num_pages : 0;
+    a.sub_rows = sub_rows;
     a.scale_log2 = (float)((double)d->scale * 1.4426950408889634);
     a.wait_limit_ns = kWaitLimitNs;
     (void)max_seq_len;  // the parts adapt to the device lengths by themselves
 
-    // K tiles {64 elements, 1 head, kTile positions, 1 sequence} of [B, t_max, n_k, d_k], 128-byte swizzle
+    // K tiles {64 elements, 1 head, kTile positions, 1 sequence} of [B, t_max, n_k, d_k], or sub-boxes
+    // {64, 1, sub_rows, 1} of the pool [num_pages, page_size, n_k, d_k]; 128-byte swizzle
     CUtensorMap tm_k;
-    st = make_tensor_map_4d(&tm_k, k_cache, d->d_k, d->n_k, t_max, d->batch, 64, 1, kTile, 1,
-                            CU_TENSOR_MAP_SWIZZLE_128B);
+    st = paged ? make_tensor_map_4d(&tm_k, k_cache, d->d_k, d->n_k, paged->page_size, paged->num_pages, 64, 1,
+                                    sub_rows, 1, CU_TENSOR_MAP_SWIZZLE_128B)
+               : make_tensor_map_4d(&tm_k, k_cache, d->d_k, d->n_k, t_max, d->batch, 64, 1, kTile, 1,
+                                    CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != DIFFQKV_OK) return st;
     if (ensure_dynamic_smem((const void *)fn, (int)plan.smem) != DIFFQKV_OK) return DIFFQKV_ERR_CUDA;
     // parts of a unit wait on one another: the whole grid must be resident at once (cooperative launch)

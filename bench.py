@@ -505,6 +505,23 @@ def time_paths(ak, peaks, steps: int, warmup: int):
     res[w.name] = {"us": ms * 1e3, "algorithmic_bytes": nbytes, "gbs": nbytes / (ms * 1e-3) / 1e9,
                    "bound": "hbm", "peak_gbs": hbm, "frac": nbytes / (ms * 1e-3) / 1e9 / hbm,
                    "launches_per_call": 1}
+    # the same selection over paged caches (16-position pages dealt out in random order)
+    del d
+    dp = wl.random_paged_inputs(w.batch, w.t_max // 16 + 1, 16, w.shape, seed=w.seed, seq_lens=[w.t_max] * w.batch,
+                                device=dev)
+    ws_pg = ak.decode_topv_workspace(ak.make_dims(w.batch, w.shape.n_q, w.shape.n_k, w.shape.n_v, w.shape.d_k,
+                                                  w.shape.d_v, w.shape.scale), (w.t_max // 16 + 1) * 16, w.topk, dev)
+    fn = lambda: ak.decode_topv_paged(dp["q"], dp["k_pages"], dp["v_pages"], dp["block_table"],  # noqa: E731
+                                      dp["seq_lens"], w.topk, scale=dp["scale"], workspace=ws_pg)
+    for _ in range(max(3, warmup)):
+        fn()
+    ms = statistics.median(_timed_calls(fn, steps, flush))
+    res[w.name + "_paged_p16"] = {"us": ms * 1e3, "algorithmic_bytes": nbytes, "gbs": nbytes / (ms * 1e-3) / 1e9,
+                                  "bound": "hbm", "peak_gbs": hbm, "frac": nbytes / (ms * 1e-3) / 1e9 / hbm,
+                                  "launches_per_call": 1}
+    assert ak.workspace_status(ws_pg) == 0
+    del dp, ws_pg
+    d = wl.make_decode_inputs(w, dev)
     # the same selection with the pages' full-softmax weights (no renormalisation over the kept set)
     fn = lambda: ak.decode_topv(d["q"], d["k_cache"], d["v_cache"], d["seq_lens"], w.topk,  # noqa: E731
                                 scale=d["scale"], workspace=ws, full_weights=True)

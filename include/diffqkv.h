@@ -327,6 +327,35 @@ diffqkv_status_t diffqkv_decode_topv_ex(const diffqkv_dims_t *dims, const void *
                                         int32_t *idx_out, void *workspace, size_t workspace_bytes,
                                         diffqkv_stream_t stream);
 
+/*
+ * Selective V fetch over PAGED K/V caches: diffqkv_decode_topv_ex with the
+ * K and V page pools and block table of diffqkv_decode_paged
+ * ("Selective V Cache Fetching" over the separate per-position K and V
+ * caches of section 3.4 Step 2, kept in pages):
+ *
+ *   k_pages     [num_pages, page_size, n_k, d_k]   K page pool (bf16, device)
+ *   v_pages     [num_pages, page_size, n_v, d_v]   V page pool
+ *   block_table [B, max_blocks] int32 (device)     pool page of each logical page
+ *
+ * Position j of sequence b is row j % page_size of pool page
+ * block_table[b, j / page_size]; t_max = max_blocks * page_size <= 131072.
+ * Selection, index output, weights (flags), lengths and the workspace
+ * (diffqkv_decode_topv_workspace_size with that t_max) are those of
+ * diffqkv_decode_topv_ex; for the same cached rows the results are those
+ * of the contiguous call, bit for bit.  page_size must be a multiple of 8
+ * (a K tile is loaded as gcd(120, page_size)-position pieces, each inside one
+ * page, into 8-row swizzle atoms), else DIFFQKV_ERR_UNSUPPORTED.  Only the
+ * entries of pages holding positions < seq_lens[b] are read; a read entry
+ * outside [0, num_pages) is flagged DIFFQKV_ERR_DEVICE_PAGE and pool page 0
+ * read in its place.  block_table must be 4-byte aligned.
+ */
+diffqkv_status_t diffqkv_decode_topv_paged(const diffqkv_dims_t *dims, const void *q, const void *k_pages,
+                                           const void *v_pages, const int32_t *block_table, int32_t max_blocks,
+                                           int32_t page_size, int32_t num_pages, const int32_t *seq_lens,
+                                           int32_t max_seq_len, int32_t topk, int32_t flags, void *out,
+                                           int32_t *idx_out, void *workspace, size_t workspace_bytes,
+                                           diffqkv_stream_t stream);
+
 /* ------------------------------------------------------------------------ */
 /* Causal prefill (the "prefix" phase the paper's efficiency study times)    */
 /* ------------------------------------------------------------------------ */

@@ -288,3 +288,20 @@ def test_workspace_status_and_prefill_word_reject_bad_args():
                                          None) == _capi.MISALIGNED
     assert lib.diffqkv_prefill_causal_ex(ctypes.byref(d), 0x1000, 0x2000, 0x3000, -1, 16, 0x5000, None,
                                          None) == _capi.INVALID_ARG
+
+
+def test_decode_topv_paged_rejects_before_launch():
+    lib = _capi.lib()
+    d = dims()
+
+    def call(bt=0x7000, max_blocks=8, page_size=16, num_pages=10, q=0x1000, flags=0):
+        return lib.diffqkv_decode_topv_paged(ctypes.byref(d), q, 0x2000, 0x3000, bt, max_blocks, page_size, num_pages,
+                                             0x4000, 128, 4, flags, 0x5000, 0x7000, 0x6000, 1 << 34, None)
+    assert call(bt=None) == _capi.INVALID_ARG
+    assert call(bt=0x7002) == _capi.MISALIGNED
+    assert call(page_size=0) == _capi.INVALID_ARG
+    assert call(num_pages=0) == _capi.INVALID_ARG
+    assert call(page_size=12) == _capi.UNSUPPORTED          # not a multiple of 8
+    assert call(max_blocks=2048, page_size=128) == _capi.UNSUPPORTED  # capacity past 131072
+    assert call(flags=2) == _capi.INVALID_ARG
+    assert call(q=0x1008) == _capi.MISALIGNED
