@@ -10,7 +10,10 @@ import os
 import re
 
 PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(PKG, "libdiffqkv.so")
+# DIFFQKV_BOUNDS_CHECK=1 selects the checked build (device-side index checks that skip an out-of-range
+# access and report DIFFQKV_ERR_DEVICE_BOUNDS); both are built in-tree by asymmetric_head_kv_b200.build
+CHECKED = os.environ.get("DIFFQKV_BOUNDS_CHECK", "") not in ("", "0")
+LIB_PATH = os.path.join(PKG, "libdiffqkv_checked.so" if CHECKED else "libdiffqkv.so")
 HEADER = os.path.join(os.path.dirname(PKG), "include", "diffqkv.h")
 
 STATUS = {
@@ -25,9 +28,10 @@ STATUS = {
     8: "DIFFQKV_ERR_NO_DEVICE",
     9: "DIFFQKV_ERR_SCRATCH_LIMIT",
     10: "DIFFQKV_ERR_DEVICE_PAGE",
+    11: "DIFFQKV_ERR_DEVICE_BOUNDS",
 }
 (OK, INVALID_ARG, UNSUPPORTED, MISALIGNED, WORKSPACE, CUDA_ERR, DEVICE_TIMEOUT, DEVICE_SEQLEN, NO_DEVICE,
- SCRATCH_LIMIT, DEVICE_PAGE) = range(11)
+ SCRATCH_LIMIT, DEVICE_PAGE, DEVICE_BOUNDS) = range(12)
 TOPV_FULL_SOFTMAX_WEIGHTS = 1  # flag of diffqkv_decode_topv_ex (include/diffqkv.h)
 
 

@@ -19,6 +19,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libdiffqkv.so")
+LIB_CHECKED = os.path.join(PKG, "libdiffqkv_checked.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ARCH + [
@@ -47,14 +48,14 @@ def _compile(src: str, obj: str, extra) -> str:
     return r.stderr
 
 
-def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
-    os.makedirs(BUILD, exist_ok=True)
+def _build_one(lib: str, objdir: str, force: bool, verbose: bool, extra_flags) -> str:
+    os.makedirs(objdir, exist_ok=True)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     hdr_mtime = max([os.path.getmtime(h) for h in _headers()] + [os.path.getmtime(__file__)])
     jobs = []
     objs = []
     for s in srcs:
-        o = os.path.join(BUILD, os.path.basename(s)[:-3] + ".o")
+        o = os.path.join(objdir, os.path.basename(s)[:-3] + ".o")
         objs.append(o)
         if force or not os.path.exists(o) or os.path.getmtime(o) < max(os.path.getmtime(s), hdr_mtime):
             jobs.append((s, o))
@@ -63,14 +64,23 @@ def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
             for (s, _), log in zip(jobs, ex.map(lambda j: _compile(j[0], j[1], extra_flags), jobs)):
                 if verbose and log.strip():
                     print(f"[{os.path.basename(s)}]\n{log}", file=sys.stderr)
-    if jobs or not os.path.exists(LIB):
-        tmp = LIB + f".tmp{os.getpid()}"
+    if jobs or not os.path.exists(lib):
+        tmp = lib + f".tmp{os.getpid()}"
         cmd = [_nvcc()] + ARCH + ["-shared", "-o", tmp] + objs + ["-lcudart"]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-        os.replace(tmp, LIB)
-    return LIB
+        os.replace(tmp, lib)
+    return lib
+
+
+def build(force: bool = False, verbose: bool = False, extra_flags=(), checked: bool = True) -> str:
+    """Builds libdiffqkv.so and, unless checked=False, libdiffqkv_checked.so: the same sources with
+    -DDIFFQKV_BOUNDS_CHECK (device-side index checks; selected at run time by DIFFQKV_BOUNDS_CHECK=1)."""
+    lib = _build_one(LIB, BUILD, force, verbose, extra_flags)
+    if checked:
+        _build_one(LIB_CHECKED, BUILD + "_checked", force, verbose, tuple(extra_flags) + ("-DDIFFQKV_BOUNDS_CHECK",))
+    return lib
 
 
 if __name__ == "__main__":

@@ -5,7 +5,9 @@
 // topv.cu, prefill.cu).
 #include <cudaTypedefs.h>
 #include <math.h>
+#include <nvtx3/nvToolsExt.h>
 #include <stdio.h>
+#include <stdlib.h>
 
 #include <mutex>
 
@@ -154,6 +156,16 @@ diffqkv_status_t validate_dims(const diffqkv_dims_t *d) {
     return DIFFQKV_OK;
 }
 
+bool nvtx_enabled() {
+    static const bool on = [] {
+        const char *e = getenv("DIFFQKV_NVTX");
+        return e != nullptr && e[0] != '\0' && !(e[0] == '0' && e[1] == '\0');
+    }();
+    return on;
+}
+void nvtx_push(const char *name) { nvtxRangePushA(name); }
+void nvtx_pop() { nvtxRangePop(); }
+
 diffqkv_status_t wait_timeout_selftest_launch(int64_t timeout_ns, cudaStream_t stream) {
     if (timeout_ns < 1000 || timeout_ns > 5000000000LL) return DIFFQKV_ERR_INVALID_ARG;
     DeviceInfo dev;
@@ -181,6 +193,7 @@ const char *diffqkv_status_string(int32_t status) {
         case DIFFQKV_ERR_NO_DEVICE: return "DIFFQKV_ERR_NO_DEVICE";
         case DIFFQKV_ERR_SCRATCH_LIMIT: return "DIFFQKV_ERR_SCRATCH_LIMIT";
         case DIFFQKV_ERR_DEVICE_PAGE: return "DIFFQKV_ERR_DEVICE_PAGE";
+        case DIFFQKV_ERR_DEVICE_BOUNDS: return "DIFFQKV_ERR_DEVICE_BOUNDS";
         default: return "DIFFQKV_ERR_UNKNOWN";
     }
 }
@@ -190,6 +203,7 @@ int32_t diffqkv_version(void) { return 10100; }
 size_t diffqkv_decode_workspace_size(const diffqkv_dims_t *dims) { return diffqkv::decode_workspace_size(dims); }
 
 diffqkv_status_t diffqkv_workspace_init(void *workspace, size_t workspace_bytes, diffqkv_stream_t stream) {
+    diffqkv::ApiRange nvtx_range("diffqkv_workspace_init");
     if (!workspace || workspace_bytes == 0) return DIFFQKV_ERR_INVALID_ARG;
     if (cudaMemsetAsync(workspace, 0, workspace_bytes, (cudaStream_t)stream) != cudaSuccess) {
         cudaGetLastError();
@@ -201,6 +215,7 @@ diffqkv_status_t diffqkv_workspace_init(void *workspace, size_t workspace_bytes,
 diffqkv_status_t diffqkv_decode(const diffqkv_dims_t *dims, const void *q, const void *k_cache, const void *v_cache,
                                 const int32_t *seq_lens, int32_t t_max, int32_t max_seq_len, void *out,
                                 void *workspace, size_t workspace_bytes, diffqkv_stream_t stream) {
+    diffqkv::ApiRange nvtx_range("diffqkv_decode");
     return diffqkv::decode_launch(dims, q, k_cache, v_cache, seq_lens, t_max, max_seq_len, out, workspace,
                                   workspace_bytes, nullptr, (cudaStream_t)stream);
 }
@@ -210,6 +225,7 @@ diffqkv_status_t diffqkv_decode_append(const diffqkv_dims_t *dims, const void *q
                                        const int32_t *seq_lens, int32_t t_max, int32_t max_seq_len,
                                        void *out, void *workspace, size_t workspace_bytes,
                                        diffqkv_stream_t stream) {
+    diffqkv::ApiRange nvtx_range("diffqkv_decode_append");
     if (!k_new || !v_new) return DIFFQKV_ERR_INVALID_ARG;
     return diffqkv::decode_launch(dims, q, k_cache, v_cache, seq_lens, t_max, max_seq_len, out, workspace,
                                   workspace_bytes, nullptr, (cudaStream_t)stream, k_new, v_new);
@@ -221,6 +237,7 @@ diffqkv_status_t diffqkv_decode_paged(const diffqkv_dims_t *dims, const void *q,
                                       int32_t num_pages, const int32_t *seq_lens, int32_t max_seq_len,
                                       void *out, void *workspace, size_t workspace_bytes,
                                       diffqkv_stream_t stream) {
+    diffqkv::ApiRange nvtx_range("diffqkv_decode_paged");
     if ((k_new == nullptr) != (v_new == nullptr)) return DIFFQKV_ERR_INVALID_ARG;
     if (max_blocks < 1 || page_size < 1 || (long long)max_blocks * page_size > 0x7fffffffLL)
         return DIFFQKV_ERR_INVALID_ARG;
@@ -233,6 +250,7 @@ diffqkv_status_t diffqkv_decode_ex(const diffqkv_dims_t *dims, const void *q, co
                                    const void *v_cache, const int32_t *seq_lens, int32_t t_max, int32_t max_seq_len,
                                    void *out, void *workspace, size_t workspace_bytes,
                                    const diffqkv_decode_tuning_t *tuning, diffqkv_stream_t stream) {
+    diffqkv::ApiRange nvtx_range("diffqkv_decode_ex");
     return diffqkv::decode_launch(dims, q, k_cache, v_cache, seq_lens, t_max, max_seq_len, out, workspace,
                                   workspace_bytes, tuning, (cudaStream_t)stream);
 }
@@ -240,6 +258,7 @@ diffqkv_status_t diffqkv_decode_ex(const diffqkv_dims_t *dims, const void *q, co
 diffqkv_status_t diffqkv_decode_plan(const diffqkv_dims_t *dims, int32_t t_max, int32_t max_seq_len,
                                      int32_t num_sms, const diffqkv_decode_tuning_t *tuning,
                                      diffqkv_decode_plan_t *plan) {
+    diffqkv::ApiRange nvtx_range("diffqkv_decode_plan");
     return diffqkv::decode_plan(dims, t_max, max_seq_len, num_sms, tuning, plan);
 }
 
@@ -248,6 +267,7 @@ diffqkv_status_t diffqkv_decode_from_host(const diffqkv_dims_t *dims, const void
                                           int32_t max_seq_len, void *out_host, void *q_dev, void *k_cache_dev,
                                           void *v_cache_dev, int32_t *seq_lens_dev, void *out_dev,
                                           void *workspace, size_t workspace_bytes, diffqkv_stream_t stream) {
+    diffqkv::ApiRange nvtx_range("diffqkv_decode_from_host");
     return diffqkv::decode_from_host_launch(dims, q_host, k_cache_host, v_cache_host, seq_lens_host, t_max,
                                             max_seq_len, out_host, q_dev, k_cache_dev, v_cache_dev, seq_lens_dev,
                                             out_dev, workspace, workspace_bytes, (cudaStream_t)stream);
@@ -261,6 +281,7 @@ diffqkv_status_t diffqkv_decode_topv(const diffqkv_dims_t *dims, const void *q, 
                                      const void *v_cache, const int32_t *seq_lens, int32_t t_max,
                                      int32_t max_seq_len, int32_t topk, void *out, int32_t *idx_out,
                                      void *workspace, size_t workspace_bytes, diffqkv_stream_t stream) {
+    diffqkv::ApiRange nvtx_range("diffqkv_decode_topv");
     return diffqkv::topv_launch(dims, q, k_cache, v_cache, seq_lens, t_max, max_seq_len, topk, out, idx_out,
                                 workspace, workspace_bytes, (cudaStream_t)stream);
 }
@@ -270,6 +291,7 @@ diffqkv_status_t diffqkv_decode_topv_ex(const diffqkv_dims_t *dims, const void *
                                         int32_t max_seq_len, int32_t topk, int32_t flags, void *out,
                                         int32_t *idx_out, void *workspace, size_t workspace_bytes,
                                         diffqkv_stream_t stream) {
+    diffqkv::ApiRange nvtx_range("diffqkv_decode_topv_ex");
     return diffqkv::topv_launch(dims, q, k_cache, v_cache, seq_lens, t_max, max_seq_len, topk, out, idx_out,
                                 workspace, workspace_bytes, (cudaStream_t)stream, flags);
 }
@@ -280,6 +302,7 @@ diffqkv_status_t diffqkv_decode_topv_paged(const diffqkv_dims_t *dims, const voi
                                            int32_t max_seq_len, int32_t topk, int32_t flags, void *out,
                                            int32_t *idx_out, void *workspace, size_t workspace_bytes,
                                            diffqkv_stream_t stream) {
+    diffqkv::ApiRange nvtx_range("diffqkv_decode_topv_paged");
     if (max_blocks < 1 || page_size < 1 || (long long)max_blocks * page_size > 0x7fffffffLL)
         return DIFFQKV_ERR_INVALID_ARG;
     const diffqkv::PagedCache paged{block_table, max_blocks, page_size, num_pages};
@@ -289,24 +312,28 @@ diffqkv_status_t diffqkv_decode_topv_paged(const diffqkv_dims_t *dims, const voi
 
 diffqkv_status_t diffqkv_prefill_causal(const diffqkv_dims_t *dims, const void *q, const void *k, const void *v,
                                         int32_t seq_len, void *out, diffqkv_stream_t stream) {
+    diffqkv::ApiRange nvtx_range("diffqkv_prefill_causal");
     return diffqkv::prefill_launch(dims, q, k, v, seq_len, out, (cudaStream_t)stream);
 }
 
 diffqkv_status_t diffqkv_prefill_causal_prefix(const diffqkv_dims_t *dims, const void *q, const void *k,
                                                const void *v, int32_t prefix_len, int32_t seq_len, void *out,
                                                diffqkv_stream_t stream) {
+    diffqkv::ApiRange nvtx_range("diffqkv_prefill_causal_prefix");
     return diffqkv::prefill_launch(dims, q, k, v, seq_len, out, (cudaStream_t)stream, prefix_len);
 }
 
 diffqkv_status_t diffqkv_prefill_causal_ex(const diffqkv_dims_t *dims, const void *q, const void *k,
                                            const void *v, int32_t prefix_len, int32_t seq_len, void *out,
                                            int32_t *device_status_word, diffqkv_stream_t stream) {
+    diffqkv::ApiRange nvtx_range("diffqkv_prefill_causal_ex");
     return diffqkv::prefill_launch(dims, q, k, v, seq_len, out, (cudaStream_t)stream, prefix_len,
                                    device_status_word);
 }
 
 diffqkv_status_t diffqkv_workspace_status(void *workspace, size_t workspace_bytes, diffqkv_stream_t stream,
                                           int32_t *device_status) {
+    diffqkv::ApiRange nvtx_range("diffqkv_workspace_status");
     if (!device_status || !workspace || workspace_bytes < 256) return DIFFQKV_ERR_INVALID_ARG;
     if (!diffqkv::aligned16(workspace)) return DIFFQKV_ERR_MISALIGNED;
     cudaStream_t s = (cudaStream_t)stream;
@@ -322,6 +349,7 @@ diffqkv_status_t diffqkv_workspace_status(void *workspace, size_t workspace_byte
 }
 
 diffqkv_status_t diffqkv_get_device_status(diffqkv_stream_t stream, int32_t *device_status) {
+    diffqkv::ApiRange nvtx_range("diffqkv_get_device_status");
     if (!device_status) return DIFFQKV_ERR_INVALID_ARG;
     diffqkv::DeviceInfo dev;
     diffqkv_status_t st = diffqkv::current_device_info(&dev);
@@ -339,12 +367,14 @@ diffqkv_status_t diffqkv_get_device_status(diffqkv_stream_t stream, int32_t *dev
 }
 
 diffqkv_status_t diffqkv_selftest_wait_timeout(int64_t timeout_ns, diffqkv_stream_t stream) {
+    diffqkv::ApiRange nvtx_range("diffqkv_selftest_wait_timeout");
     return diffqkv::wait_timeout_selftest_launch(timeout_ns, (cudaStream_t)stream);
 }
 
 diffqkv_status_t diffqkv_decode_noalloc(const diffqkv_dims_t *dims, const void *q, const void *k_cache,
                                         const void *v_cache, const int32_t *seq_lens, int32_t t_max,
                                         int32_t max_seq_len, void *out, diffqkv_stream_t stream) {
+    diffqkv::ApiRange nvtx_range("diffqkv_decode_noalloc");
     return diffqkv::decode_noalloc_launch(dims, q, k_cache, v_cache, seq_lens, t_max, max_seq_len, out,
                                           (cudaStream_t)stream);
 }

@@ -30,6 +30,21 @@ __device__ __forceinline__ void record_error(int32_t *status, int32_t code) {
     if (status) atomicCAS(reinterpret_cast<int *>(status), 0, code);
 }
 
+// ----------------------------------------------------------------- bounds checks
+// The checked build (-DDIFFQKV_BOUNDS_CHECK) tests the index of the kernels'
+// global accesses against the extent of their buffer: an index outside is
+// recorded as DIFFQKV_ERR_DEVICE_BOUNDS in the call's status word and the
+// access is skipped (never a trap).  In the normal build the test is `true`.
+#ifdef DIFFQKV_BOUNDS_CHECK
+__device__ __forceinline__ bool in_bounds(long long i, long long n, int32_t *status) {
+    if (i >= 0 && i < n) return true;
+    record_error(status, DIFFQKV_ERR_DEVICE_BOUNDS);
+    return false;
+}
+#else
+__device__ __forceinline__ bool in_bounds(long long, long long, int32_t *) { return true; }
+#endif
+
 // ----------------------------------------------------------------- addressing
 __device__ __forceinline__ uint32_t smem_addr(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));

@@ -79,6 +79,8 @@ struct DecodeArgs {
     const int32_t *block_table = nullptr;  // [B, max_blocks] pool page of each logical page
     int32_t max_blocks = 0, page_size = 0, num_pages = 0;
     int32_t sub_rows = 0;                  // positions per sub-box (divides the tile and the page)
+    long long partial_slots = 0;           // split-partial records the scratch holds
+    long long store_rows = 0;              // rows of the K / V caches or pools (append stores)
     uint32_t sub_k_bytes = 0, sub_v_bytes = 0;
 };
 
@@ -395,7 +397,9 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
         const int h = w.g * QPK + hs;
         if (t == t_begin || w.i == 0) {
             // new split: this warp's query chunk, pre-scaled into the log2 domain
-            const uint4 qv = __ldg(reinterpret_cast<const uint4 *>(a.q + ((size_t)w.b * a.n_q + h) * DK) + kc);
+            const uint4 qv = in_bounds((long long)w.b * a.n_q + h, (long long)a.batch * a.n_q, a.status)
+                                 ? __ldg(reinterpret_cast<const uint4 *>(a.q + ((size_t)w.b * a.n_q + h) * DK) + kc)
+                                 : make_uint4(0, 0, 0, 0);
             const f32x2_t sc2 = f2_pack(a.scale_log2, a.scale_log2);
             q2[0] = f2_mul(bf16x2_to_f2(qv.x), sc2);
             q2[1] = f2_mul(bf16x2_to_f2(qv.y), sc2);
@@ -539,7 +543,7 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
                     }
                 }
                 float *dst = a.partials + ((size_t)(u + c) * QPK + hs) * (DV + kPartialPad);
-                if (vs == 0) {
+                if (vs == 0 && in_bounds(u + c, a.partial_slots, a.status)) {
                     __stcg(reinterpret_cast<float4 *>(dst + vc * 8), make_float4(O[0], O[1], O[2], O[3]));
                     __stcg(reinterpret_cast<float4 *>(dst + vc * 8 + 4), make_float4(O[4], O[5], O[6], O[7]));
                 }
@@ -551,7 +555,8 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
             __threadfence();
             named_barrier(1, NCW * 32);
             if (tid == 0) {
-                const unsigned old = atomicAdd(a.counters + u, 1u);
+                const unsigned old =
+                    in_bounds(u, (long long)a.batch * a.n_k, a.status) ? atomicAdd(a.counters + u, 1u) : 0u;
                 *last_flag = (old == (unsigned)(last - first)) ? 1 : 0;
             }
             named_barrier(1, NCW * 32);
@@ -574,7 +579,8 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
                         for (int off = 16; off >= 1; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
                         if (lane == 0) merge_s[warp] = dot * a.scale_log2;
                     }
-                    const long long row = cache_row(a, w.b, p);  // -1: bad page entry, nothing written
+                    long long row = cache_row(a, w.b, p);  // -1: bad page entry, nothing written
+                    if (row >= 0 && !in_bounds(row, a.store_rows, a.status)) row = -1;
                     const size_t kdst = ((size_t)row * a.n_k + w.g) * DK;
                     const size_t ksrc = ((size_t)w.b * a.n_k + w.g) * DK;
                     for (int e = tid; e < DK / 8 && row >= 0; e += NCW * 32)
@@ -592,7 +598,9 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
                 }
                 constexpr int ITEMS = QPK * (DV / 4);
                 constexpr int kBatch = QPK >= 16 ? 1 : 4;  // partials loaded together (one L2 round trip per batch)
-                for (int it = tid; it < ITEMS; it += NCW * 32) {
+                // (checked build: a combine whose partial records would fall outside the scratch is skipped)
+                const bool parts_ok = in_bounds(u + last, a.partial_slots, a.status);
+                for (int it = tid; it < ITEMS && parts_ok; it += NCW * 32) {
                     const int h2 = it / (DV / 4);
                     const int d4 = it % (DV / 4);
                     constexpr int kBatchM = QPK >= 16 ? 4 : 16;  // maxima only: wider batches
@@ -652,7 +660,8 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
                     uint2 packed;
                     packed.x = *reinterpret_cast<uint32_t *>(&lo);
                     packed.y = *reinterpret_cast<uint32_t *>(&hi);
-                    *reinterpret_cast<uint2 *>(a.out + ((size_t)w.b * a.n_q + w.g * QPK + h2) * DV + d4 * 4) = packed;
+                    if (in_bounds((long long)w.b * a.n_q + w.g * QPK + h2, (long long)a.batch * a.n_q, a.status))
+                        *reinterpret_cast<uint2 *>(a.out + ((size_t)w.b * a.n_q + w.g * QPK + h2) * DV + d4 * 4) = packed;
                 }
                 if (tid == 0) a.counters[u] = 0u;
             }
@@ -872,6 +881,8 @@ diffqkv_status_t decode_prepare(const diffqkv_dims_t *d, const void *q, const vo
     a.counters = reinterpret_cast<uint32_t *>(ws + kWorkspaceHeader);
     a.partials = reinterpret_cast<float *>(ws + kWorkspaceHeader + align_up(units * sizeof(uint32_t), 256));
     a.status = reinterpret_cast<int32_t *>(ws);  // the workspace's own error word
+    a.partial_slots = (long long)units + kGridMax;
+    a.store_rows = paged ? (long long)paged->num_pages * paged->page_size : (long long)d->batch * t_max;
     a.batch = d->batch;
     a.n_q = d->n_q;
     a.n_k = d->n_k;
@@ -1020,6 +1031,8 @@ diffqkv_status_t decode_noalloc_launch(const diffqkv_dims_t *d, const void *q, c
     a.seq_lens = seq_lens;
     a.out = static_cast<__nv_bfloat16 *>(out);
     a.counters = reinterpret_cast<uint32_t *>(scratch + kWorkspaceHeader);
+    a.partial_slots = (long long)units + plan.grid_ctas;
+    a.store_rows = (long long)d->batch * t_max;
     a.partials = reinterpret_cast<float *>(scratch + kWorkspaceHeader + counter_bytes);
     a.status = dev.status_word;
     a.batch = d->batch;

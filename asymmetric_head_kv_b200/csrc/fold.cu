@@ -135,5 +135,6 @@ diffqkv_status_t fold_query_launch(const diffqkv_dims_t *d, int32_t d_q, int32_t
 extern "C" diffqkv_status_t diffqkv_fold_query(const diffqkv_dims_t *dims, int32_t d_q, int32_t w_heads,
                                                const void *q_aug, const void *w_up, void *q_out,
                                                diffqkv_stream_t stream) {
+    diffqkv::ApiRange nvtx_range("diffqkv_fold_query");
     return diffqkv::fold_query_launch(dims, d_q, w_heads, q_aug, w_up, q_out, (cudaStream_t)stream);
 }

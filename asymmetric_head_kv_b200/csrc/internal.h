@@ -92,4 +92,22 @@ diffqkv_status_t prefill_launch(const diffqkv_dims_t *d, const void *q, const vo
 // api.cu
 diffqkv_status_t wait_timeout_selftest_launch(int64_t timeout_ns, cudaStream_t stream);
 
+// An NVTX range around one C-ABI call, named after it, when the environment variable
+// DIFFQKV_NVTX is set (read once); otherwise nothing.  Profilers show each call's
+// host-side span next to the kernels it launched.
+bool nvtx_enabled();
+void nvtx_push(const char *name);
+void nvtx_pop();
+struct ApiRange {
+    const bool on;
+    explicit ApiRange(const char *name) : on(nvtx_enabled()) {
+        if (on) nvtx_push(name);
+    }
+    ~ApiRange() {
+        if (on) nvtx_pop();
+    }
+    ApiRange(const ApiRange &) = delete;
+    ApiRange &operator=(const ApiRange &) = delete;
+};
+
 }  // namespace diffqkv

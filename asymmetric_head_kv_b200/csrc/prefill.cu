@@ -317,7 +317,8 @@ __global__ void __launch_bounds__(kThreads, 2)
             uint32_t r[32];
             tmem_ld32(t_o + lane_base + c, r);
             tmem_wait_ld();
-            if (qrow < a.seq) {
+            if (qrow < a.seq &&
+                in_bounds(((long long)b * a.seq + qrow) * a.n_q + h, (long long)a.batch * a.seq * a.n_q, a.status)) {
 #pragma unroll
                 for (int e = 0; e < 32; e += 8) {
                     uint4 v;
@@ -637,7 +638,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 uint32_t rr[32];
                 tmem_ld32(t_o + (uint32_t)c, rr);
                 tmem_wait_ld();
-                if (qrow < a.seq) {
+                if (qrow < a.seq &&
+                    in_bounds(((long long)b * a.seq + qrow) * a.n_q + h, (long long)a.batch * a.seq * a.n_q, a.status)) {
 #pragma unroll
                     for (int e = 0; e < 32; e += 8) {
                         uint4 v;

@@ -116,6 +116,7 @@ struct TopvArgs {
     const int32_t *block_table;
     int32_t max_blocks, page_size, num_pages;
     int32_t sub_rows;     // positions per TMA sub-box of a paged tile (divides kTile and page_size)
+    long long cache_rows; // rows of the K / V caches or pools
     float scale_log2;
     uint64_t wait_limit_ns;
 };
@@ -720,7 +721,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const float score = reduce_heads<HG>(part, r);
                     if (lane_writes<HG>(r) && valid) {
                         const int hh = pass * HG + head_of_lane<HG>(r);
-                        scores[(size_t)hh * a.score_stride + lp] = score;
+                        if (in_bounds(lp, a.score_stride, a.status)) scores[(size_t)hh * a.score_stride + lp] = score;
                         const uint32_t bk = float_key(score) >> 21;
                         atomicAdd(hist_s + hh * kHistWords + (bk >> 1), 1u << ((bk & 1u) << 4));
                     }
@@ -919,6 +920,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // every cached position is kept: the candidate list holds them all
                 for (uint32_t i = tid; i < nc; i += kThreads) {
                     const int jj = cj[i];
+                    if (!in_bounds(jj, K, a.status)) continue;
                     idx[jj] = jj;
                     ks[jj] = cs[i];
                     kr[jj] = (int32_t)cache_row(a, b, jj);
@@ -985,7 +987,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int need = K - sh.sh_cnt_in;  // 1 <= need <= na when the bound holds
                 // K row of position jj (exact keys of the ambiguous positions)
                 auto krow = [&](int jj) {
-                    return reinterpret_cast<const uint16_t *>(a.k + ((size_t)cache_row(a, b, jj) * a.n_k + g) * DK);
+                    long long r = cache_row(a, b, jj);
+                    if (!in_bounds(r, a.cache_rows, a.status)) r = 0;
+                    return reinterpret_cast<const uint16_t *>(a.k + ((size_t)r * a.n_k + g) * DK);
                 };
                 auto keep = [&](int jj) { atomicOr(bitmap + (jj >> 5), 1u << (jj & 31)); };
                 if (need <= 0) {
@@ -1154,6 +1158,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int uu = 0; uu < GU; ++uu) {
                         const int i = i0 + uu * WPR * RPW;
                         jj[uu] = i < i_end ? __ldcg(kr + i) : -1;  // the kept position's cache row
+                        if (jj[uu] >= 0 && !in_bounds(jj[uu], a.cache_rows, a.status)) jj[uu] = -1;
                         sx[uu] = i < i_end ? __ldcg(ks + i) : -INFINITY;
                     }
                     uint4 vv[GU];
@@ -1211,7 +1216,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int c = tid; c < DV; c += kThreads) {
                     float acc = 0.f;
                     for (int p = 0; p < Y; ++p) acc += __ldcg(gp + (size_t)p * (DV + 4) + c);
-                    a.out[(size_t)row * DV + c] = __float2bfloat16(lt > 0.f ? acc / lt : 0.f);
+                    if (in_bounds(row, (long long)a.batch * a.n_q, a.status))
+                        a.out[(size_t)row * DV + c] = __float2bfloat16(lt > 0.f ? acc / lt : 0.f);
                 }
                 if (tid == 0) {
                     // every part of the row has passed its wait on the flag; and since every part of the
@@ -1422,6 +1428,7 @@ diffqkv_status_t topv_launch(const diffqkv_dims_t *d, const void *q, const void 
     a.page_size = paged ? paged->page_size : 0;
     a.num_pages = paged ? paged->num_pages : 0;
     a.sub_rows = sub_rows;
+    a.cache_rows = paged ? (long long)paged->num_pages * paged->page_size : (long long)d->batch * t_max;
     a.scale_log2 = (float)((double)d->scale * 1.4426950408889634);
     a.wait_limit_ns = kWaitLimitNs;
     (void)max_seq_len;  // the parts adapt to the device lengths by themselves

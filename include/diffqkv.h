@@ -75,7 +75,9 @@ typedef enum {
     DIFFQKV_ERR_DEVICE_SEQLEN = 7,  /* a device seq_len was < 0 or > t_max (clamped) */
     DIFFQKV_ERR_NO_DEVICE = 8,      /* no CUDA device / driver */
     DIFFQKV_ERR_SCRATCH_LIMIT = 9,  /* shape needs more than the built-in scratch of diffqkv_decode_noalloc */
-    DIFFQKV_ERR_DEVICE_PAGE = 10    /* a block-table entry a paged call used was outside [0, num_pages) */
+    DIFFQKV_ERR_DEVICE_PAGE = 10,   /* a block-table entry a paged call used was outside [0, num_pages) */
+    DIFFQKV_ERR_DEVICE_BOUNDS = 11  /* a device-side index check failed (checked build only; the access
+                                       was skipped) */
 } diffqkv_status_t;
 
 /* Human-readable name of a status code (static storage; never NULL). */

@@ -305,3 +305,26 @@ def test_decode_topv_paged_rejects_before_launch():
     assert call(max_blocks=2048, page_size=128) == _capi.UNSUPPORTED  # capacity past 131072
     assert call(flags=2) == _capi.INVALID_ARG
     assert call(q=0x1008) == _capi.MISALIGNED
+
+
+def test_checked_build_exports_every_declared_symbol_and_nvtx_switch_is_harmless():
+    """The checked library exports the same C ABI; with DIFFQKV_NVTX set, calls still return their
+    status (here without a GPU) through the NVTX-ranged entry points."""
+    import subprocess
+    import sys
+    code = (
+        "import ctypes, asymmetric_head_kv_b200 as ak\n"
+        "from asymmetric_head_kv_b200 import _capi\n"
+        "lib = _capi.lib()\n"
+        "assert _capi.LIB_PATH.endswith('libdiffqkv_checked.so')\n"
+        "for n in _capi.header_symbols(): getattr(lib, n)\n"
+        "d = ak.make_dims(1, 16, 4, 16, 64, 128, 0.125)\n"
+        "st = lib.diffqkv_decode(ctypes.byref(d), None, 0, 0, 0, 16, 16, 0, 0, 0, None)\n"
+        "assert st == _capi.INVALID_ARG, st\n"
+        "assert lib.diffqkv_status_string(11).decode() == 'DIFFQKV_ERR_DEVICE_BOUNDS'\n"
+        "print('ok')\n")
+    import os
+    env = dict(os.environ, DIFFQKV_BOUNDS_CHECK="1", DIFFQKV_NVTX="1")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-c", code], env=env, cwd=root, capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0 and "ok" in r.stdout, r.stdout + r.stderr
