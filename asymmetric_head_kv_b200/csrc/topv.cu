@@ -46,8 +46,9 @@
 // workspace needs zero-filling only before its first use.
 #include <math.h>
 
+#include <string.h>
+
 #include <algorithm>
-#include <numeric>
 
 #include "common.cuh"
 #include "internal.h"
@@ -74,6 +75,8 @@ constexpr int kTopvMaxContext = 131072;  // bitmap of kept positions
 constexpr int kMaxParts = 256;           // CTAs per unit (sizes the per-part records)
 constexpr int kMaxStages = 6;
 constexpr int kEmitIters = 8;            // float4 vectors per thread and emission chunk (32 mask bits)
+constexpr int kTableAhead = 4;           // paged producer: tiles whose block-table entries are in flight
+constexpr int kTableRing = 8;            // rows of the entry ring (> kTableAhead)
 constexpr int kRowInfoWords = 8;
 enum RowInfo { kRiBucket = 0, kRiAbove = 1, kRiTwoDelta = 2, kRiMax = 3, kRiKept = 4, kRiFullSum = 5 };
 enum UnitSync { kUsHist = 0, kUsCand = 1, kUsKmax = 3 };
@@ -115,7 +118,8 @@ struct TopvArgs {
     // of pool page block_table[b][j / page_size]
     const int32_t *block_table;
     int32_t max_blocks, page_size, num_pages;
-    int32_t sub_rows;     // positions per TMA sub-box of a paged tile (divides kTile and page_size)
+    int32_t max_box_log;  // paged: boxes of 8 << i rows, i <= max_box_log, divide the page size
+    int32_t tile_box;     // paged, page size a multiple of kTile: one kTile-row box per tile (m[0])
     long long cache_rows; // rows of the K / V caches or pools
     float scale_log2;
     uint64_t wait_limit_ns;
@@ -481,14 +485,21 @@ struct Shared {
     int combine[16];        // rows whose output this CTA writes after the gather
     uint32_t emit_total[16];
     uint32_t emit_base[16];
+    int32_t table[kTableRing][32];  // paged producer: block-table entries of tile t in row t % kTableRing
     float row_m[16];
     int row_nsel[16];
     float row_full[16];
 };
 
+// K tensor maps: m[0] has kTile-row boxes over a contiguous cache; over a paged pool m[i] has
+// (8 << i)-row boxes, for the heights that divide the page size (i <= TopvArgs::max_box_log).
+struct KMaps {
+    CUtensorMap m[4];
+};
+
 template <int DK, int DV, int QPK>
 __global__ void __launch_bounds__(kThreads, 1)
-    topv_fused_kernel(const __grid_constant__ CUtensorMap tm_k, const TopvArgs a) {
+    topv_fused_kernel(const __grid_constant__ KMaps maps, const TopvArgs a) {
     // rows per consumer pass (their q in registers: 4 rows x d_k / 4 values per lane)
     constexpr int HG = QPK < (DK == 64 ? 4 : 2) ? QPK : (DK == 64 ? 4 : 2);
     constexpr int NPASS = QPK / HG;
@@ -527,7 +538,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         sh.abort_flag = 0;
         fence_barrier_init();
     }
-    if (warp == kConsumerWarps && lane == 0) prefetch_tensormap(&tm_k);
+    if (warp == kConsumerWarps && lane == 0) {
+        prefetch_tensormap(&maps.m[0]);
+        if (a.block_table) {
+            prefetch_tensormap(&maps.m[1]);
+            prefetch_tensormap(&maps.m[2]);
+            prefetch_tensormap(&maps.m[3]);
+        }
+    }
     __syncthreads();
 
     long long ring_k = 0;  // tiles this CTA has put through its ring (all rounds): barrier phases
@@ -555,41 +573,78 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncthreads();
         if (warp == kConsumerWarps && a.block_table) {
-            // ---- producer, paged caches: the whole warp; lane f issues sub-box f (sub_rows positions
-            //      inside one page) of each tile, so a tile's sub-boxes leave as one warp instruction,
-            //      and loads its block-table entry a tile ahead.  Only sub-boxes holding cached
-            //      positions are loaded (later table entries may hold anything).
+            // ---- producer, paged caches (the whole warp).  A tile's rows are covered greedily by
+            //      aligned boxes of 8, 16, 32 or 64 rows (heights that divide the page, so a box never
+            //      leaves its page), or by one whole-tile box when the page size is a multiple of the
+            //      tile; lane f issues box f, so a tile's boxes leave as one warp instruction (one lane
+            //      issuing them all measured slower).  The tile's block-table entries (one page per
+            //      lane) reach shared memory by asynchronous copies issued kTableAhead tiles ahead (a
+            //      register copy of a pending load would wait for it at once); an entry is checked when
+            //      a box uses it.  Only pages holding cached positions are read (later entries may hold
+            //      anything); rows past the sequence inside a loaded box are harmless.
             if (te > tb) {
                 if (lane == 0) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 __syncwarp();
                 const long long k0 = ring_k;
-                const int per_tile = kTile / a.sub_rows;
-                auto n_sub = [&](int t) { return (min(kTile, T - t * kTile) + a.sub_rows - 1) / a.sub_rows; };
-                auto entry = [&](int t, int f) {
-                    return f < n_sub(t) ? paged_page(a, b, (t * kTile + f * a.sub_rows) / a.page_size) : 0;
+                auto covered = [&](int t) { return (min(kTile, T - t * kTile) + 7) & ~7; };  // rows loaded
+                auto first_page = [&](int t) { return (t * kTile) / a.page_size; };
+                auto fetch = [&](int t) {
+                    if (t < te) {
+                        const int np = (t * kTile + covered(t) - 1) / a.page_size - first_page(t) + 1;
+                        if (lane < np) {
+                            const int32_t *src = a.block_table + (size_t)b * a.max_blocks + first_page(t) + lane;
+                            asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(
+                                             smem_addr(&sh.table[t % kTableRing][lane])),
+                                         "l"(src)
+                                         : "memory");
+                        }
+                    }
+                    asm volatile("cp.async.commit_group;" ::: "memory");
                 };
-                int cur = lane < per_tile ? entry(tb, lane) : 0;
+                for (int i = 0; i < kTableAhead; ++i) fetch(tb + i);
                 int st = (int)(k0 % a.stages);
                 uint32_t par = (uint32_t)((k0 / a.stages) & 1);
                 bool wrapped = k0 >= a.stages;
                 long long issued_end = k0;
                 for (int t = tb; t < te; ++t) {
-                    const int ns = n_sub(t);
-                    const int nxt = (t + 1 < te && lane < per_tile) ? entry(t + 1, lane) : 0;
+                    fetch(t + kTableAhead);
                     if (wrapped) mbar_wait_bounded(&empty_bar[st], par ^ 1u, a.wait_limit_ns, abort_flag, a.status);
                     if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
+                    asm volatile("cp.async.wait_group %0;" ::"n"(kTableAhead) : "memory");  // tile t's entries
+                    const int cur_e = sh.table[t % kTableRing][lane];  // this lane's own copy
+                    // every lane walks the same decomposition and keeps box `lane`
+                    const int start = t * kTile, end = start + (a.tile_box ? kTile : covered(t));
+                    int cur = a.tile_box ? end : start, f = 0, my_cur = -1, my_hi = 0;
+                    if (a.tile_box && lane == 0) my_cur = start;
+                    while (cur < end) {
+                        int hi = a.max_box_log;
+                        while (hi > 0 && ((cur & ((8 << hi) - 1)) != 0 || cur + (8 << hi) > end)) --hi;
+                        if (f == lane) {
+                            my_cur = cur;
+                            my_hi = hi;
+                        }
+                        cur += 8 << hi;
+                        ++f;
+                    }
                     uint8_t *dst = ring + (size_t)st * TILE_BYTES;
-                    if (lane == 0) mbar_arrive_expect_tx(&full_bar[st], (uint32_t)(ns * a.sub_rows * DK * 2));
+                    if (lane == 0) mbar_arrive_expect_tx(&full_bar[st], (uint32_t)((end - start) * DK * 2));
                     __syncwarp();
-                    for (int f = lane; f < ns; f += 32) {
-                        const int page = f == lane ? cur : entry(t, f);
-                        const int row = (t * kTile + f * a.sub_rows) % a.page_size;
+                    int page = __shfl_sync(0xffffffffu, cur_e, my_cur >= 0 ? my_cur / a.page_size - first_page(t) : 0);
+                    if (my_cur >= 0) {
+                        if (page < 0 || page >= a.num_pages) {  // flagged; pool page 0 read in its place
+                            record_error(a.status, DIFFQKV_ERR_DEVICE_PAGE);
+                            page = 0;
+                        }
+                        // constant indices keep the descriptors in the kernel's parameter space
+                        const CUtensorMap *tm = my_hi == 0 ? &maps.m[0]
+                                                : my_hi == 1 ? &maps.m[1]
+                                                : my_hi == 2 ? &maps.m[2]
+                                                             : &maps.m[3];
 #pragma unroll
                         for (int kb = 0; kb < DK / 64; ++kb)
-                            tma_load_4d(dst + kb * (kTile * 128) + f * a.sub_rows * 128, &tm_k, &full_bar[st],
-                                        kb * 64, g, row, page);
+                            tma_load_4d(dst + kb * (kTile * 128) + (my_cur - start) * 128, tm, &full_bar[st], kb * 64,
+                                        g, my_cur % a.page_size, page);
                     }
-                    cur = nxt;
                     issued_end = k0 + (t - tb) + 1;
                     if (++st == a.stages) {
                         st = 0;
@@ -597,6 +652,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         wrapped = true;
                     }
                 }
+                asm volatile("cp.async.wait_all;" ::: "memory");  // no entry copy outlives the loop
                 if (lane == 0)
                     for (long long kk = (issued_end - a.stages > k0 ? issued_end - a.stages : k0); kk < issued_end; ++kk)
                         mbar_wait_bounded(&full_bar[kk % a.stages], (uint32_t)((kk / a.stages) & 1), a.wait_limit_ns,
@@ -624,7 +680,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mbar_arrive_expect_tx(&full_bar[st], TILE_BYTES);
 #pragma unroll
                     for (int kb = 0; kb < DK / 64; ++kb)
-                        tma_load_4d(dst + kb * (kTile * 128), &tm_k, &full_bar[st], kb * 64, g, t * kTile, b);
+                        tma_load_4d(dst + kb * (kTile * 128), &maps.m[0], &full_bar[st], kb * 64, g, t * kTile, b);
                     issued_end = kk + 1;
                     if (++st == a.stages) {
                         st = 0;
@@ -1239,7 +1295,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 size_t align_up(size_t x, size_t al) { return (x + al - 1) / al * al; }
 
-using TopvFn = void (*)(CUtensorMap, TopvArgs);
+using TopvFn = void (*)(KMaps, TopvArgs);
 
 template <int DK, int DV>
 TopvFn pick_qpk(int qpk) {
@@ -1343,16 +1399,16 @@ diffqkv_status_t topv_launch(const diffqkv_dims_t *d, const void *q, const void 
         return DIFFQKV_ERR_INVALID_ARG;
     if (t_max > kTopvMaxContext) return DIFFQKV_ERR_UNSUPPORTED;
     if (flags & ~DIFFQKV_TOPV_FULL_SOFTMAX_WEIGHTS) return DIFFQKV_ERR_INVALID_ARG;
-    int sub_rows = kTile;
+    int max_box_log = 0;
     if (paged) {
         if (!paged->block_table || paged->max_blocks < 1 || paged->page_size < 1 || paged->num_pages < 1 ||
             (long long)paged->max_blocks * paged->page_size != t_max)
             return DIFFQKV_ERR_INVALID_ARG;
         if (reinterpret_cast<uintptr_t>(paged->block_table) & 3u) return DIFFQKV_ERR_MISALIGNED;
-        // a tile is loaded as sub-boxes of gcd(tile, page) positions, each inside one page; with the
-        // 128-byte swizzle every sub-box must start on an 8-row boundary
-        sub_rows = std::gcd(kTile, (int)paged->page_size);
-        if (sub_rows % 8 != 0) return DIFFQKV_ERR_UNSUPPORTED;
+        // a tile is loaded as boxes of 8, 16, 32 or 64 rows that divide the page (so each lies in one
+        // page); with the 128-byte swizzle every box must start on an 8-row boundary
+        if (paged->page_size % 8 != 0) return DIFFQKV_ERR_UNSUPPORTED;
+        while (max_box_log < 3 && paged->page_size % (16 << max_box_log) == 0) ++max_box_log;
         if ((long long)paged->num_pages * paged->page_size > 0x7fffffffLL) return DIFFQKV_ERR_UNSUPPORTED;
     } else if ((long long)d->batch * t_max > 0x7fffffffLL) {
         return DIFFQKV_ERR_UNSUPPORTED;  // kept positions' cache rows are int32
@@ -1427,19 +1483,32 @@ diffqkv_status_t topv_launch(const diffqkv_dims_t *d, const void *q, const void 
     a.max_blocks = paged ? paged->max_blocks : 0;
     a.page_size = paged ? paged->page_size : 0;
     a.num_pages = paged ? paged->num_pages : 0;
-    a.sub_rows = sub_rows;
+    a.max_box_log = max_box_log;
     a.cache_rows = paged ? (long long)paged->num_pages * paged->page_size : (long long)d->batch * t_max;
     a.scale_log2 = (float)((double)d->scale * 1.4426950408889634);
     a.wait_limit_ns = kWaitLimitNs;
     (void)max_seq_len;  // the parts adapt to the device lengths by themselves
 
-    // K tiles {64 elements, 1 head, kTile positions, 1 sequence} of [B, t_max, n_k, d_k], or sub-boxes
-    // {64, 1, sub_rows, 1} of the pool [num_pages, page_size, n_k, d_k]; 128-byte swizzle
-    CUtensorMap tm_k;
-    st = paged ? make_tensor_map_4d(&tm_k, k_cache, d->d_k, d->n_k, paged->page_size, paged->num_pages, 64, 1,
-                                    sub_rows, 1, CU_TENSOR_MAP_SWIZZLE_128B)
-               : make_tensor_map_4d(&tm_k, k_cache, d->d_k, d->n_k, t_max, d->batch, 64, 1, kTile, 1,
-                                    CU_TENSOR_MAP_SWIZZLE_128B);
+    // K tiles {64 elements, 1 head, kTile positions, 1 sequence} of [B, t_max, n_k, d_k], or boxes
+    // {64, 1, 8 << i, 1} of the pool [num_pages, page_size, n_k, d_k]; 128-byte swizzle
+    KMaps maps;
+    memset(&maps, 0, sizeof maps);
+    const bool tile_box = paged && paged->page_size % kTile == 0;
+    a.tile_box = tile_box ? 1 : 0;
+    if (tile_box) {
+        st = make_tensor_map_4d(&maps.m[0], k_cache, d->d_k, d->n_k, paged->page_size, paged->num_pages, 64, 1,
+                                kTile, 1, CU_TENSOR_MAP_SWIZZLE_128B);
+        for (int i = 1; i < 4; ++i) maps.m[i] = maps.m[0];
+    } else if (paged) {
+        for (int i = 0; i <= max_box_log && st == DIFFQKV_OK; ++i)
+            st = make_tensor_map_4d(&maps.m[i], k_cache, d->d_k, d->n_k, paged->page_size, paged->num_pages, 64, 1,
+                                    8u << i, 1, CU_TENSOR_MAP_SWIZZLE_128B);
+        for (int i = max_box_log + 1; i < 4; ++i) maps.m[i] = maps.m[0];
+    } else {
+        st = make_tensor_map_4d(&maps.m[0], k_cache, d->d_k, d->n_k, t_max, d->batch, 64, 1, kTile, 1,
+                                CU_TENSOR_MAP_SWIZZLE_128B);
+        for (int i = 1; i < 4; ++i) maps.m[i] = maps.m[0];
+    }
     if (st != DIFFQKV_OK) return st;
     if (ensure_dynamic_smem((const void *)fn, (int)plan.smem) != DIFFQKV_OK) return DIFFQKV_ERR_CUDA;
     // parts of a unit wait on one another: the whole grid must be resident at once (cooperative launch)
@@ -1459,7 +1528,7 @@ diffqkv_status_t topv_launch(const diffqkv_dims_t *d, const void *q, const void 
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, fn, tm_k, a) != cudaSuccess) {
+    if (cudaLaunchKernelEx(&cfg, fn, maps, a) != cudaSuccess) {
         cudaGetLastError();
         return DIFFQKV_ERR_CUDA;
     }

@@ -97,8 +97,35 @@ def profiled_traffic():
     return float(m_tr.group(1))
 
 
+def _clock_sampler_proc(device_index: int, conn, period_s: float):
+    """Child process: samples the SM clock and the clock-event reasons through NVML (read-only) until
+    told to stop, then sends back (timestamp, MHz, reason mask) samples.  A separate process, so the
+    samples keep coming while the parent waits on the GPU."""
+    try:
+        import pynvml
+        pynvml.nvmlInit()
+        h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+        max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+    except Exception:  # no NVML: no samples
+        conn.send((None, []))
+        return
+    conn.send(("ready", max_mhz))
+    samples = []
+    while not conn.poll():
+        try:
+            samples.append((time.monotonic(), pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM),
+                            pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)))
+        except Exception:
+            pass
+        time.sleep(period_s)
+    conn.recv()
+    conn.send((max_mhz, samples))
+
+
 class ClockSampler:
-    """Samples SM clock and clock-event reasons through NVML while the timed region runs (read-only)."""
+    """SM clock and clock-event reasons sampled through NVML during the timed region, in a child
+    process started before the warm-up; only the samples taken between entering and leaving the
+    context count."""
 
     REASONS = {
         "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4, "hw_slowdown": 0x8,
@@ -107,42 +134,36 @@ class ClockSampler:
     }
 
     def __init__(self, device_index: int, period_s: float = 0.0002):
-        # the headline's timed region can be a few milliseconds (20 steps of ~0.36 ms): sample
-        # every 0.2 ms so that it still holds ten or more readings
-        self.period_s = period_s
-        self.samples, self.reasons, self.max_mhz = [], set(), None
-        self._stop = threading.Event()
-        try:
-            import pynvml
-            pynvml.nvmlInit()
-            self.nv = pynvml
-            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
-            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
-        except Exception:  # no NVML: report no samples
-            self.nv = None
-
-    def _run(self):
-        while not self._stop.is_set():
-            try:
-                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
-                mask = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
-                for name, bit in self.REASONS.items():
-                    if mask & bit and name != "gpu_idle":
-                        self.reasons.add(name)
-            except Exception:
-                pass
-            time.sleep(self.period_s)
+        import multiprocessing as mp
+        ctx = mp.get_context("spawn")
+        self.conn, child = ctx.Pipe()
+        self.proc = ctx.Process(target=_clock_sampler_proc, args=(device_index, child, period_s), daemon=True)
+        self.proc.start()
+        first = self.conn.recv()
+        self.ok = first[0] == "ready"
+        self.max_mhz = first[1] if self.ok else None
+        self.samples, self.reasons = [], set()
+        self.t0 = self.t1 = None
 
     def __enter__(self):
-        if self.nv:
-            self.t = threading.Thread(target=self._run, daemon=True)
-            self.t.start()
+        self.t0 = time.monotonic()
         return self
 
     def __exit__(self, *a):
-        self._stop.set()
-        if self.nv:
-            self.t.join()
+        self.t1 = time.monotonic()
+        return False
+
+    def close(self):
+        if self.ok:
+            self.conn.send("stop")
+            _, samples = self.conn.recv()
+            for t, mhz, mask in samples:
+                if self.t0 is not None and self.t0 <= t <= self.t1:
+                    self.samples.append(mhz)
+                    for name, bit in self.REASONS.items():
+                        if mask & bit and name != "gpu_idle":
+                            self.reasons.add(name)
+        self.proc.join(timeout=10)
 
     def summary(self):
         return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
@@ -212,8 +233,7 @@ def time_decode(ak, w: wl.DecodeWorkload, steps: int, warmup: int, world: int, s
             starts[i].record(stream)
             step()
             ends[i].record(stream)
-        # let the clock sampler thread run while the GPU works: torch.cuda.synchronize() would hold
-        # the interpreter lock for the whole wait
+        # wait for the last step without holding the interpreter lock the whole time
         while not ends[-1].query():
             time.sleep(0.0001)
         torch.cuda.synchronize()
@@ -548,7 +568,7 @@ def main():
 
     torch.cuda.set_device(local)
     peaks, peak_src = load_peaks()
-    sampler = ClockSampler(local)
+    sampler = ClockSampler(local)  # started before the first GPU work (a spawned process)
     main_res = time_decode(ak, WORKLOAD, args.steps, args.warmup, world, sampler)
     region_ms = max_over_ranks(main_res["region_ms"], world)
     ms_per_step = region_ms / args.steps
@@ -592,6 +612,7 @@ def main():
            "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": args.e2e_steps,
            "api": "diffqkv_decode_from_host (pinned host buffers)"}
 
+    sampler.close()
     paths = time_paths(ak, peaks, max(10, min(50, args.steps // 10)), args.warmup)
 
     cpu = None
