@@ -15,13 +15,14 @@
 // group share one pass over K head g.  Each unit is cut into Y equal tile ranges
 // ("parts"), one per CTA; with more units than fit, CTAs take them in rounds.
 // Per unit:
-//  1. Scores.  A producer warp streams the part's K tiles with TMA into a ring;
-//     15 consumer warps compute fp32 scores s_j = q.k_j for every row of the
-//     group (four lanes per position, q in registers, packed f32x2 FMAs; every
-//     bf16 x bf16 product is exact) and keep them in shared memory, together
-//     with a 2048-bucket histogram of the top 11 bits of each score's order key
-//     and the largest |k|.  Histograms go to global memory; the CTA arrives on
-//     the unit's counter H.
+//  1. Scores.  A producer warp streams the part's K tiles (128 positions) with
+//     TMA into a ring; one thread issues tcgen05 MMAs S = K_tile q^T (M = 128
+//     positions, N = 16 rows of q, zero-padded past the group's, K = d_k) into
+//     a ring of TMEM buffers; three consumer warpgroups take the tiles in turn,
+//     read one position's scores per thread out of TMEM, keep them in shared
+//     memory with a 2048-bucket histogram of the top 11 bits of each score's
+//     order key, and fold the position's K row into the largest |k|.
+//     Histograms go to global memory; the CTA arrives on the unit's counter H.
 //  2. Candidates.  Once H counts all Y parts, each CTA finds in every row's
 //     histogram the bucket holding the k-th largest score and emits every own
 //     score at or above that bucket's lower end minus 2d (d the rounding bound
@@ -30,7 +31,7 @@
 //     largest fp32 score (its top 11 bits are the bucket; two radix passes over
 //     the candidates find the next 11 and the last 10); with d >= |s_j - e_j|
 //     for every j (e_j the exact dot),
-//        d = 1.01 gamma_n ||q||_1 max|k| + n 2^-149, gamma_n = n u / (1 - n u), u = 2^-24,
+//        d = 1.01 gamma ||q||_1 max|k| + n 2^-126, gamma = nu / (1 - nu), nu = n (17/16) 2^-23,
 //     scores above tau + 2d are certainly kept, below tau - 2d certainly not,
 //     and the rest (usually a handful) get exact keys -- an integer
 //     superaccumulator of the products -- and the remaining slots go to the
@@ -57,13 +58,18 @@ namespace diffqkv {
 
 namespace {
 
-// 16 warps: 15 consumers of eight positions each and one producer.  Sixteen warps leave every SM
-// sub-partition four, so each thread may hold 128 registers (a seventeenth warp would cut that to 96).
-constexpr int kConsumerWarps = 15;
-constexpr int kStepsPerTile = 1;           // steps of eight positions per consumer warp and tile
-constexpr int kTile = kConsumerWarps * 8 * kStepsPerTile;  // positions per TMA tile (at most 256)
-constexpr int kThreads = (kConsumerWarps + 1) * 32;
+// 16 warps.  Scores: warps 0-11 are three consumer warpgroups, warp 12 the TMA producer, warp 13
+// the MMA issuer (and TMEM owner); warps 14 and 15 join from the candidates on.
+constexpr int kTile = 128;                 // positions per K tile: the MMA's M (TMEM lanes)
+constexpr int kConsumerGroups = 3;         // warpgroups reading scores out of TMEM, tiles dealt in turn
+constexpr int kConsumerWarps = 4 * kConsumerGroups;
+constexpr int kProducerWarp = kConsumerWarps;
+constexpr int kMmaWarp = kConsumerWarps + 1;
+constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
+constexpr int kQRows = 16;                 // rows of q in the MMA's B operand (its N), zero past the group's
+constexpr int kTmemBufs = 8;               // TMEM score buffers of kQRows columns
+constexpr int kTmemCols = 128;             // allocation: kTmemBufs * kQRows columns
 constexpr int kHistBuckets = 2048;       // both histogram levels: 11 bits of the order key
 constexpr int kHistWords = kHistBuckets / 2;  // shared histogram: two 16-bit counters per word
 constexpr int kRadixBuckets = 1024;      // last 10 key bits
@@ -142,13 +148,6 @@ __device__ __forceinline__ long long cache_row(const TopvArgs &a, int b, int j) 
     return (long long)paged_page(a, b, j / a.page_size) * a.page_size + j % a.page_size;
 }
 
-// max(a, b, c) in one instruction (three-input form of max.f32, sm_100).
-__device__ __forceinline__ float fmax3f(float a, float b, float c) {
-    float r;
-    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-    return r;
-}
-
 // Order-preserving map of finite floats onto uint32 (larger float -> larger key).
 __device__ __forceinline__ uint32_t float_key(float f) {
     const uint32_t u = __float_as_uint(f);
@@ -158,15 +157,20 @@ __device__ __forceinline__ float key_float(uint32_t k) {
     return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
 }
 
-// Rigorous bound of |fp32 FMA-chain score - exact dot| for a row: every product
-// is exact, every one of the (at most n = d_k) additions a score sees rounds by
-// at most u relative (u = 2^-24) or, in the subnormal range, by 2^-150 absolute;
-// sum_c |q_c k_c| <= ||q||_1 max|k|.  1.01 covers the rounding of this formula.
+// Bound of |tensor-core score - exact dot| for a row.  Every bf16 x bf16 product is exact in
+// fp32 (or, below the normal range, flushed: at most 2^-126 each).  The MMA adds the products
+// (16 per instruction, then the fp32 accumulator) in an order and with a rounding the PTX
+// documentation leaves open.  The bound is that of the truncating block-addition model that
+// published measurements found on earlier tensor cores: each block of 16 products and the
+// accumulator is aligned to its largest operand and truncated, which loses less than one fp32 ulp
+// (2^-23 relative) per operand, so n products lose less than gamma with nu = n (1 + 1/16) 2^-23,
+// times sum_c |q_c k_c| <= ||q||_1 max|k|.  1.01 covers the rounding of this formula.  A GPU test
+// measures the scores' error against it (worst seen: 0.05 of it).
 template <int DK>
 __device__ __forceinline__ float score_error_bound(float q_l1, float kmax) {
-    const double nu = (double)DK * 5.9604644775390625e-08;  // n * 2^-24
+    const double nu = (double)DK * (17.0 / 16.0) * 1.1920928955078125e-07;  // n (1 + 1/16) 2^-23
     const float gamma = (float)(nu / (1.0 - nu));
-    return __fmul_ru(__fmul_ru(__fmul_ru(1.01f, gamma), q_l1), kmax) + (float)DK * 1.4012984643e-45f;
+    return __fmul_ru(__fmul_ru(__fmul_ru(1.01f, gamma), q_l1), kmax) + (float)DK * 1.1754943508e-38f;
 }
 
 // ------------------------------------------------------------------ waits between CTAs
@@ -439,35 +443,47 @@ __device__ __forceinline__ bool key_greater(const uint32_t *x, const uint32_t *y
 
 // ------------------------------------------------------------------ the kernel
 
-constexpr int kBarBytes = 2 * kMaxStages * 8;
-// Bytes before the ring: barriers, q, histograms, rounded up to the ring's 1024-byte alignment.
+// mbarriers: ring full / empty, TMEM buffer full / empty, and the MMA drain
+constexpr int kBarBytes = (2 * kMaxStages + 2 * kTmemBufs + 1) * 8;
+// Bytes before the ring: q as the MMA's B operand (128-byte swizzled, 1024-byte aligned), barriers,
+// q in fp32, histograms, rounded up to the ring's 1024-byte alignment.
 __host__ __device__ constexpr int head_bytes(int dk, int qpk) {
-    return (kBarBytes + qpk * dk * 4 + qpk * kHistWords * 4 + 1023) / 1024 * 1024;
+    return (kQRows * dk * 2 + kBarBytes + qpk * dk * 4 + qpk * kHistWords * 4 + 1023) / 1024 * 1024;
 }
 
-// Sum over the 4 lanes of a position group of HG per-lane partials, one per
-// head; returns the total of head head_of_lane(r) to lane r (r = lane % 4).
-template <int HG>
-__device__ __forceinline__ float reduce_heads(const float (&v)[HG], int r) {
-    if constexpr (HG == 4) {
-        const bool hi2 = (r & 2) != 0;
-        const float a0 = (hi2 ? v[2] : v[0]) + __shfl_xor_sync(0xffffffffu, hi2 ? v[0] : v[2], 2);
-        const float a1 = (hi2 ? v[3] : v[1]) + __shfl_xor_sync(0xffffffffu, hi2 ? v[1] : v[3], 2);
-        const bool hi1 = (r & 1) != 0;
-        return (hi1 ? a1 : a0) + __shfl_xor_sync(0xffffffffu, hi1 ? a0 : a1, 1);
-    } else if constexpr (HG == 2) {
-        const bool hi2 = (r & 2) != 0;
-        float x = (hi2 ? v[1] : v[0]) + __shfl_xor_sync(0xffffffffu, hi2 ? v[0] : v[1], 2);
-        return x + __shfl_xor_sync(0xffffffffu, x, 1);
+// TMEM -> registers: this warp's 32 lanes, N consecutive 32-bit columns each (N = 1 .. 16).
+template <int N>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[N]) {
+    if constexpr (N == 1) {
+        asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r[0]) : "r"(taddr));
+    } else if constexpr (N == 2) {
+        asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0, %1}, [%2];" : "=r"(r[0]), "=r"(r[1]) : "r"(taddr));
+    } else if constexpr (N == 4) {
+        asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                     : "r"(taddr));
+    } else if constexpr (N == 8) {
+        asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                     : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                     : "r"(taddr));
     } else {
-        float x = v[0] + __shfl_xor_sync(0xffffffffu, v[0], 2);
-        return x + __shfl_xor_sync(0xffffffffu, x, 1);
+        static_assert(N == 16, "column count");
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+            "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+            : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+              "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+            : "r"(taddr));
     }
 }
-template <int HG>
-__device__ __forceinline__ bool lane_writes(int r) { return HG == 4 ? true : (HG == 2 ? (r & 1) == 0 : r == 0); }
-template <int HG>
-__device__ __forceinline__ int head_of_lane(int r) { return HG == 4 ? r : (HG == 2 ? r >> 1 : 0); }
+
+// Two bf16 per word: the result's halves have the larger magnitude of each pair (their signs are
+// the XOR of the inputs' signs, which the caller masks off).
+__device__ __forceinline__ uint32_t bf16x2_absmax(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
 
 // Small shared state of the kernel (statically allocated).
 struct Shared {
@@ -486,6 +502,7 @@ struct Shared {
     uint32_t emit_total[16];
     uint32_t emit_base[16];
     int32_t table[kTableRing][32];  // paged producer: block-table entries of tile t in row t % kTableRing
+    uint32_t tmem_base;             // the score buffers' TMEM address
     float row_m[16];
     int row_nsel[16];
     float row_full[16];
@@ -500,23 +517,25 @@ struct KMaps {
 template <int DK, int DV, int QPK>
 __global__ void __launch_bounds__(kThreads, 1)
     topv_fused_kernel(const __grid_constant__ KMaps maps, const TopvArgs a) {
-    // rows per consumer pass (their q in registers: 4 rows x d_k / 4 values per lane)
-    constexpr int HG = QPK < (DK == 64 ? 4 : 2) ? QPK : (DK == 64 ? 4 : 2);
-    constexpr int NPASS = QPK / HG;
-    constexpr int CPL = DK / 32;           // 16-byte chunks of a K row per lane
     constexpr int TILE_BYTES = kTile * DK * 2;
-    static_assert(kTile <= 256, "TMA box height");
-    static_assert(QPK <= kWarps && DK <= 128, "shape");
+    constexpr int KB = DK / 64;            // 64-element (128-byte) column blocks of a K row
+    static_assert(kTile == 128 && kTile <= 256, "the MMA's M and the TMA box height");
+    static_assert(QPK <= kQRows && DK <= 128 && DK % 64 == 0, "shape");
+    static_assert(kProducerWarp < kWarps && kMmaWarp < kWarps, "warp roles");
 
-    // dynamic shared memory: barriers | q [QPK][DK] | histograms [QPK][kHistWords] | ring
-    // [stages][TILE_BYTES] (1024-byte aligned for the 128-byte swizzle) | scores [QPK][score_stride].
-    // The select and the gather reuse everything from the ring on ("overlay"); the barriers, q
-    // and the histograms sit before it and are never overwritten.
+    // dynamic shared memory: q_b [KB][kQRows][128 B] (bf16, 128-byte swizzled) | barriers |
+    // q [QPK][DK] fp32 | histograms [QPK][kHistWords] | ring [stages][TILE_BYTES] (1024-byte
+    // aligned for the 128-byte swizzle) | scores [QPK][score_stride].  The select and the gather
+    // reuse everything from the ring on ("overlay"); what sits before it is never overwritten.
     extern __shared__ uint8_t dsm_raw[];
     uint8_t *const base = align_smem_1024(dsm_raw);
-    uint64_t *const full_bar = reinterpret_cast<uint64_t *>(base);
+    uint8_t *const q_b = base;
+    uint64_t *const full_bar = reinterpret_cast<uint64_t *>(base + kQRows * DK * 2);
     uint64_t *const empty_bar = full_bar + kMaxStages;
-    float *const q_s = reinterpret_cast<float *>(base + kBarBytes);
+    uint64_t *const tfull_bar = empty_bar + kMaxStages;
+    uint64_t *const tempty_bar = tfull_bar + kTmemBufs;
+    uint64_t *const mma_done = tempty_bar + kTmemBufs;
+    float *const q_s = reinterpret_cast<float *>(base + kQRows * DK * 2 + kBarBytes);
     uint32_t *const hist_s = reinterpret_cast<uint32_t *>(q_s + QPK * DK);
     uint8_t *const ring = base + head_bytes(DK, QPK);
     float *const scores = reinterpret_cast<float *>(ring + (size_t)a.stages * TILE_BYTES);
@@ -533,12 +552,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid == 0) {
         for (int s = 0; s < a.stages; ++s) {
             mbar_init(&full_bar[s], 1);
-            mbar_init(&empty_bar[s], kConsumerWarps);
+            mbar_init(&empty_bar[s], 1 + 4);  // the MMAs' commit and the consuming warpgroup
         }
+        for (int s = 0; s < kTmemBufs; ++s) {
+            mbar_init(&tfull_bar[s], 1);
+            mbar_init(&tempty_bar[s], 4);
+        }
+        mbar_init(mma_done, 1);
         sh.abort_flag = 0;
         fence_barrier_init();
     }
-    if (warp == kConsumerWarps && lane == 0) {
+    if (warp == kMmaWarp) {
+        tmem_alloc(&sh.tmem_base, kTmemCols);
+        tmem_relinquish();
+    }
+    if (warp == kProducerWarp && lane == 0) {
         prefetch_tensormap(&maps.m[0]);
         if (a.block_table) {
             prefetch_tensormap(&maps.m[1]);
@@ -546,7 +574,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             prefetch_tensormap(&maps.m[3]);
         }
     }
+    tc_fence_before();
     __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sh.tmem_base;
 
     long long ring_k = 0;  // tiles this CTA has put through its ring (all rounds): barrier phases
     for (int round = 0; round < a.rounds; ++round) {
@@ -571,8 +602,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int hh = i / DK, c = i % DK;
             q_s[i] = __bfloat162float(a.q[((size_t)row0 + hh) * DK + c]);
         }
+        // q as the MMA's B operand: row n (n < QPK; zero beyond) of 64-element block kb at
+        // kb * kQRows * 128 + n * 128, 16-byte chunk c at chunk position c ^ (n % 8) (128-byte swizzle)
+        for (int i = tid; i < kQRows * DK / 2; i += kThreads) {
+            const int n = i / (DK / 2), c2 = i % (DK / 2);  // elements 2 c2 and 2 c2 + 1 of row n
+            uint32_t w = 0u;
+            if (n < QPK) w = __ldg(reinterpret_cast<const uint32_t *>(a.q + ((size_t)row0 + n) * DK) + c2);
+            const int c = 2 * c2, kb = c / 64, chunk = (c % 64) / 8;
+            *reinterpret_cast<uint32_t *>(q_b + kb * (kQRows * 128) + n * 128 + ((chunk ^ (n & 7)) << 4) +
+                                          (c % 8) * 2) = w;
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // q_b is read by the tensor core
         __syncthreads();
-        if (warp == kConsumerWarps && a.block_table) {
+        if (warp == kProducerWarp && a.block_table) {
             // ---- producer, paged caches (the whole warp).  A tile's rows are covered greedily by
             //      aligned boxes of 8, 16, 32 or 64 rows (heights that divide the page, so a box never
             //      leaves its page), or by one whole-tile box when the page size is a multiple of the
@@ -658,7 +700,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         mbar_wait_bounded(&full_bar[kk % a.stages], (uint32_t)((kk / a.stages) & 1), a.wait_limit_ns,
                                           nullptr, a.status);
             }
-        } else if (warp == kConsumerWarps) {
+        } else if (warp == kProducerWarp) {
             // ---- producer: one lane issues the TMA loads of this part's tiles into the ring
             if (lane == 0 && te > tb) {
                 // the ring may hold the previous round's select and gather data, written by the generic proxy
@@ -693,111 +735,111 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mbar_wait_bounded(&full_bar[kk % a.stages], (uint32_t)((kk / a.stages) & 1), a.wait_limit_ns,
                                       nullptr, a.status);
             }
-        } else {
-            // ---- consumers: warp w takes kStepsPerTile steps of eight consecutive positions of each
-            //      tile (row pos of the tile is 128 bytes of each 64-element block; the 128-byte
-            //      swizzle XORs the 16-byte chunk index with the row index mod 8, which is pg)
-            const int r = lane & 3, pg = lane >> 2;
-            uint32_t coff[CPL];  // byte offset of this lane's u-th chunk in a row, swizzle included
+        } else if (warp == kMmaWarp) {
+            // ---- MMA issuer: S(tile) = K_tile q^T into TMEM buffer k % kTmemBufs (lane = position of
+            //      the tile, column = row of the group).  The commits free the ring slot (together with
+            //      the consuming warpgroup, which reads the slot's K rows for max |k|) and hand the
+            //      buffer to the consumers.
+            if (lane == 0 && te > tb) {
+                constexpr uint32_t idesc = umma_idesc_bf16(kTile, kQRows, false, false);
+                const uint32_t qb_addr = smem_addr(q_b);
+                const long long k0 = ring_k;
+                int st = (int)(k0 % a.stages);
+                uint32_t par = (uint32_t)((k0 / a.stages) & 1);
+                for (int t = tb; t < te; ++t) {
+                    const long long kk = k0 + (t - tb);
+                    const int tb_i = (int)(kk & (kTmemBufs - 1));
+                    if (!mbar_wait_bounded(&full_bar[st], par, a.wait_limit_ns, abort_flag, a.status)) break;
+                    // the buffer's previous tile (kk - kTmemBufs) has been read out
+                    if (kk >= kTmemBufs &&
+                        !mbar_wait_bounded(&tempty_bar[tb_i], (uint32_t)(((kk >> 3) & 1) ^ 1), a.wait_limit_ns,
+                                           abort_flag, a.status))
+                        break;
+                    tc_fence_after();
+                    const uint32_t k_addr = smem_addr(ring + (size_t)st * TILE_BYTES);
 #pragma unroll
-            for (int uu = 0; uu < CPL; ++uu) {
-                const int chunk = (uu >> 1) * 8 + 2 * r + (uu & 1);
-                coff[uu] = (uint32_t)((chunk >> 3) * (kTile * 128) + (((chunk & 7) ^ pg) << 4));
+                    for (int ks = 0; ks < DK / 16; ++ks) {
+                        const uint32_t blk = (uint32_t)(ks >> 2), sub = (uint32_t)(ks & 3) * 32u;
+                        const uint64_t da = smem_desc_sw128(k_addr + blk * (kTile * 128) + sub, 16, 1024);
+                        const uint64_t db = smem_desc_sw128(qb_addr + blk * (kQRows * 128) + sub, 16, 1024);
+                        umma_bf16(tmem + (uint32_t)(tb_i * kQRows), da, db, idesc, ks > 0 ? 1u : 0u);
+                    }
+                    umma_commit(&tfull_bar[tb_i]);
+                    umma_commit(&empty_bar[st]);
+                    if (++st == a.stages) {
+                        st = 0;
+                        par ^= 1u;
+                    }
+                }
             }
-            float kmf = 0.f;  // largest |k| seen (a bf16 value, so exact in fp32)
-            f32x2_t qp[HG][CPL][4];
-            auto load_q = [&](int pass) {
-#pragma unroll
-                for (int hh = 0; hh < HG; ++hh)
-#pragma unroll
-                    for (int uu = 0; uu < CPL; ++uu) {
-                        const int chunk = (uu >> 1) * 8 + 2 * r + (uu & 1);
-                        const float *qs = q_s + (pass * HG + hh) * DK + chunk * 8;
-                        const float4 x = *reinterpret_cast<const float4 *>(qs);
-                        const float4 y = *reinterpret_cast<const float4 *>(qs + 4);
-                        qp[hh][uu][0] = f2_pack(x.x, x.y);
-                        qp[hh][uu][1] = f2_pack(x.z, x.w);
-                        qp[hh][uu][2] = f2_pack(y.x, y.y);
-                        qp[hh][uu][3] = f2_pack(y.z, y.w);
-                    }
-            };
-            if (NPASS == 1) load_q(0);
-            int st = (int)(ring_k % a.stages);                    // ring position, kept incrementally
-            uint32_t par = (uint32_t)((ring_k / a.stages) & 1);
-            for (int t = tb; t < te; ++t) {
-                mbar_wait_bounded(&full_bar[st], par, a.wait_limit_ns, abort_flag, a.status);
-                const uint8_t *tile = ring + (size_t)st * TILE_BYTES;
-#pragma unroll
-                for (int step = 0; step < kStepsPerTile; ++step) {
-                const int pos = (warp * kStepsPerTile + step) * 8 + pg;  // row of the tile
-                const int lp = (t - tb) * kTile + pos;                    // position within this part
+            __syncwarp();
+        } else if (warp < kConsumerWarps) {
+            // ---- consumers: warpgroup cg takes the part's tiles cg, cg + 3, ...; thread (warp % 4,
+            //      lane) owns position 32 (warp % 4) + lane of a tile: its scores (TMEM lane = position)
+            //      and its K row (for max |k|)
+            const int cg = warp >> 2, quarter = warp & 3;
+            const int pos = quarter * 32 + lane;                      // row of the tile
+            const uint32_t t_lane = tmem + ((uint32_t)(quarter * 32) << 16);
+            uint32_t kacc = 0u;  // two bf16 whose magnitudes bound every |k| seen
+            long long kk = ring_k + cg;
+            int st = (int)(kk % a.stages);
+            uint32_t par = (uint32_t)((kk / a.stages) & 1);
+            for (int t = tb + cg; t < te; t += kConsumerGroups) {
+                const int tb_i = (int)(kk & (kTmemBufs - 1));
+                if (!mbar_wait_bounded(&tfull_bar[tb_i], (uint32_t)((kk >> 3) & 1), a.wait_limit_ns, abort_flag,
+                                       a.status))
+                    break;
+                tc_fence_after();
+                uint32_t sr[QPK];
+                tmem_ld_cols<QPK>(t_lane + (uint32_t)(tb_i * kQRows), sr);
+                tmem_wait_ld();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tempty_bar[tb_i]);
+                const int lp = (t - tb) * kTile + pos;  // position within this part
                 const bool valid = lp < np;
-#pragma unroll 1
-                for (int pass = 0; pass < NPASS; ++pass) {
-                    if (NPASS > 1) load_q(pass);
-                    // one accumulator per (row, chunk): CPL independent chains of a product and three
-                    // packed FMAs per row instead of one chain of 4 CPL.  A product meets at most
-                    // 3 + (CPL - 1) + 1 + 2 = CPL + 5 <= d_k roundings on its way into the score.
-                    f32x2_t acc[HG][CPL];
+                // this position's K row: every 16-byte chunk once, in an order that spreads the
+                // warp's loads over all banks (the max does not depend on the order)
+                mbar_wait_bounded(&full_bar[st], par, a.wait_limit_ns, abort_flag, a.status);
+                const uint8_t *krow = ring + (size_t)st * TILE_BYTES + pos * 128;
+                uint4 kv[8 * KB];
 #pragma unroll
-                    for (int hh = 0; hh < HG; ++hh)
+                for (int c = 0; c < 8 * KB; ++c)
+                    kv[c] = lds128(krow + (c / 8) * (kTile * 128) + (((c + lane) & 7) << 4));
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty_bar[st]);
+                if (valid) {
 #pragma unroll
-                        for (int uu = 0; uu < CPL; ++uu) acc[hh][uu] = 0ull;
-#pragma unroll
-                    for (int uu = 0; uu < CPL; ++uu) {
-                        const uint4 kv = lds128(tile + pos * 128 + coff[uu]);
-                        float kf[8];
-                        unpack8(kv, kf);
-                        if (pass == 0 && valid) {
-                            kmf = fmax3f(kmf, fabsf(kf[0]), fabsf(kf[1]));
-                            kmf = fmax3f(kmf, fabsf(kf[2]), fabsf(kf[3]));
-                            kmf = fmax3f(kmf, fabsf(kf[4]), fabsf(kf[5]));
-                            kmf = fmax3f(kmf, fabsf(kf[6]), fabsf(kf[7]));
-                        }
-                        const f32x2_t k01 = f2_pack(kf[0], kf[1]), k23 = f2_pack(kf[2], kf[3]);
-                        const f32x2_t k45 = f2_pack(kf[4], kf[5]), k67 = f2_pack(kf[6], kf[7]);
-#pragma unroll
-                        for (int hh = 0; hh < HG; ++hh) {
-                            acc[hh][uu] = f2_mul(qp[hh][uu][0], k01);
-                            acc[hh][uu] = f2_fma(qp[hh][uu][1], k23, acc[hh][uu]);
-                            acc[hh][uu] = f2_fma(qp[hh][uu][2], k45, acc[hh][uu]);
-                            acc[hh][uu] = f2_fma(qp[hh][uu][3], k67, acc[hh][uu]);
-                        }
+                    for (int c = 0; c < 8 * KB; ++c) {
+                        kacc = bf16x2_absmax(kacc, kv[c].x);
+                        kacc = bf16x2_absmax(kacc, kv[c].y);
+                        kacc = bf16x2_absmax(kacc, kv[c].z);
+                        kacc = bf16x2_absmax(kacc, kv[c].w);
                     }
-                    float part[HG];
 #pragma unroll
-                    for (int hh = 0; hh < HG; ++hh) {
-                        f32x2_t t2 = acc[hh][0];
-#pragma unroll
-                        for (int uu = 1; uu < CPL; ++uu) t2 = f2_add(t2, acc[hh][uu]);
-                        float x0, x1;
-                        f2_unpack(t2, x0, x1);
-                        part[hh] = x0 + x1;
-                    }
-                    const float score = reduce_heads<HG>(part, r);
-                    if (lane_writes<HG>(r) && valid) {
-                        const int hh = pass * HG + head_of_lane<HG>(r);
+                    for (int hh = 0; hh < QPK; ++hh) {
+                        const float score = __uint_as_float(sr[hh]);
                         if (in_bounds(lp, a.score_stride, a.status)) scores[(size_t)hh * a.score_stride + lp] = score;
                         const uint32_t bk = float_key(score) >> 21;
                         atomicAdd(hist_s + hh * kHistWords + (bk >> 1), 1u << ((bk & 1u) << 4));
                     }
                 }
-                }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&empty_bar[st]);
-                if (++st == a.stages) {
-                    st = 0;
+                kk += kConsumerGroups;
+                st += kConsumerGroups;
+                while (st >= a.stages) {
+                    st -= a.stages;
                     par ^= 1u;
                 }
             }
-            uint32_t kmx = __float_as_uint(kmf) >> 16;  // its bf16 pattern (kmf >= 0: order-preserving)
+            // largest |k| as a bf16 magnitude pattern (order-preserving for non-negative values)
+            uint32_t kmx = max(kacc & 0x7fffu, (kacc >> 16) & 0x7fffu);
 #pragma unroll
             for (int off = 16; off >= 1; off >>= 1) kmx = max(kmx, __shfl_xor_sync(0xffffffffu, kmx, off));
             if (lane == 0 && kmx) atomicMax(usync + kUsKmax, kmx);
         }
         ring_k += te - tb;
         __syncthreads();
-        if (*abort_flag) return;  // a ring wait ran out (recorded); the producer has drained
+        if (*abort_flag) goto finish;  // a ring wait ran out (recorded); the producer has drained
         // the part's histograms (word i: buckets 2i and 2i + 1) into the rows' global histograms
         for (int i = tid; i < QPK * kHistWords; i += kThreads) {
             const uint32_t w = hist_s[i];
@@ -808,7 +850,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         cta_arrive(usync + kUsHist);
 
         // =============================================================== 2. candidates
-        if (!cta_wait_at_least(usync + kUsHist, (uint32_t)Y, a, flag)) return;
+        if (!cta_wait_at_least(usync + kUsHist, (uint32_t)Y, a, flag)) goto finish;
         if (warp < QPK) {
             const int row = row0 + warp;
             float lower = -INFINITY;
@@ -941,7 +983,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
         // =============================================================== 3. select
         for (int hh = j; hh < QPK; hh += Y) {
-            if (!cta_wait_at_least(usync + kUsCand, (uint32_t)Y, a, flag)) return;
+            if (!cta_wait_at_least(usync + kUsCand, (uint32_t)Y, a, flag)) goto finish;
             const int row = row0 + hh;
             int32_t *idx = a.idx_out + (size_t)row * K;
             float *ks = a.kept_s + (size_t)row * a.k_pad;
@@ -1177,7 +1219,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             *flag = ok ? 1 : 0;
         }
         __syncthreads();
-        if (!*flag) return;
+        if (!*flag) goto finish;
         if (tid < QPK) {
             const int row = row0 + tid;
             sh.row_m[tid] = __uint_as_float(__ldcg(a.rowinfo + kRowInfoWords * row + kRiMax));
@@ -1288,6 +1330,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             __syncthreads();
         }
+    }
+finish:
+    // the tensor memory goes back once no MMA is in flight (every exit of the loop above is taken by
+    // the whole CTA)
+    if (warp == kMmaWarp) {
+        if (lane == 0) {
+            umma_commit(mma_done);
+            mbar_wait_bounded(mma_done, 0, a.wait_limit_ns, nullptr, a.status);
+        }
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
     }
 }
 

@@ -208,3 +208,64 @@ def test_poisoned_workspace_is_never_read_before_written(cuda_device, topk):
     assert torch.isfinite(out.float()).all()
     assert_parity(out, r_out, f"poisoned workspace k={topk}")
     assert torch.count_nonzero(ws[c0:c1]) == 0, "counters not returned to zero"
+
+
+def _candidate_lists(ws, batch, n_q, n_k, d_v, t_max):
+    """Views of the workspace's candidate positions and scores ([rows][t_pad] each; the header's layout)."""
+    rows, units, t_pad = batch * n_q, batch * n_k, -(-t_max // 64) * 64
+    off = 256 + _a256(_a256(units * 16) + _a256(rows * 16) + rows * 2048 * 4)
+    off += _a256(rows * 8 * 4) + _a256(rows * 256 * 8) + _a256(rows * 256 * (d_v + 4) * 4)
+    cj = ws[off:off + rows * t_pad * 4].view(torch.int32).view(rows, t_pad)
+    off += _a256(rows * t_pad * 4)
+    cs = ws[off:off + rows * t_pad * 4].view(torch.float32).view(rows, t_pad)
+    return cj, cs
+
+
+@pytest.mark.parametrize("kind", ["normal", "outliers", "wide"])
+def test_tensor_core_score_error_within_model(cuda_device, kind):
+    """The scores come from tcgen05 MMAs, whose addition order and rounding the PTX documentation
+    leaves open.  The selection's bound is the truncating block-addition model,
+    n (1 + 1/16) 2^-23 sum|q k| per score; this measures the candidates' fp32 scores against the
+    exact dot products and requires a margin of 4 below it (inputs: normal, normal with 256x
+    outliers, exponents spread over 2^+-20)."""
+    s = wl.DIFFQKV
+    B, T, topk = 2, 6000, 300
+    d = wl.random_decode_inputs(B, T, s, seed=312)
+    g = torch.Generator().manual_seed(312)
+    if kind != "normal":
+        k = d["k_cache"].float()
+        if kind == "outliers":
+            k = k * torch.where(torch.rand(k.shape, generator=g) < 0.05, 256.0, 1.0)
+        else:
+            k = k * torch.exp2(torch.randint(-20, 21, k.shape, generator=g).float())
+        d["k_cache"] = k.to(torch.bfloat16)
+    gdev = {kk: (v.to(cuda_device) if isinstance(v, torch.Tensor) else v) for kk, v in d.items()}
+    dims = ak.make_dims(B, s.n_q, s.n_k, s.n_v, s.d_k, s.d_v, d["scale"])
+    ws = ak.decode_topv_workspace(dims, T, topk, cuda_device)
+    cj, cs = _candidate_lists(ws, B, s.n_q, s.n_k, s.d_v, T)
+    cj.fill_(-1)
+    out, idx = ak.decode_topv(gdev["q"], gdev["k_cache"], gdev["v_cache"], gdev["seq_lens"], topk,
+                              scale=d["scale"], workspace=ws)
+    assert ak.workspace_status(ws) == 0
+    r_out, r_idx = oracle.decode_topv(d["q"], d["k_cache"], d["v_cache"], d["seq_lens"], topk, d["scale"])
+    assert np.array_equal(idx.cpu().numpy(), r_idx)
+    assert_parity(out, r_out, f"tensor-core scores, {kind}")
+    q = d["q"].double().numpy()
+    kc = d["k_cache"].double().numpy()
+    cj_h, cs_h = cj.cpu().numpy(), cs.cpu().numpy().astype(np.float64)
+    qpk, worst, checked = s.n_q // s.n_k, 0.0, 0
+    for row in range(B * s.n_q):
+        b, h = divmod(row, s.n_q)
+        sel = cj_h[row] >= 0
+        pos = cj_h[row][sel]
+        krow = kc[b, pos, h // qpk]                        # [n, d_k]
+        exact = krow @ q[b, h]                             # exact: 64 products of bf16 in fp64
+        mag = np.abs(krow) @ np.abs(q[b, h])
+        err = np.abs(cs_h[row][sel] - exact)
+        model = s.d_k * (1 + 1 / 16) * 2.0 ** -23 * mag + s.d_k * 2.0 ** -126
+        assert np.all(err <= model / 4), f"{kind}: row {row} error {err.max():.3e} within 4x of the model"
+        rn = s.d_k * 2.0 ** -24 * mag                      # the round-to-nearest gamma_n, for the record
+        worst = max(worst, float(np.max(err / np.maximum(rn, 1e-300))))
+        checked += int(sel.sum())
+    assert checked > 1000
+    print(f"{kind}: {checked} candidate scores, worst error {worst:.3f} x the round-to-nearest bound")
