@@ -8,8 +8,9 @@ executes anything here, and this package imports nothing from it.
 The arithmetic lives in ``oracle.c`` (plain C, fp64) and follows "Sigma:
 Differential Rescaling of Query, Key and Value for Efficient Language Models"
 (structured summary page), section 3.4 "DiffQKV Attention: Generalized
-Formulation" Steps 2-5, "Selective V Cache Fetching", and "FlexHeadFA Kernel
-and Deployment Infrastructure".  This module only marshals arrays.
+Formulation" Steps 2-5, "Selective V Cache Fetching", "FlexHeadFA Kernel
+and Deployment Infrastructure", and section 3.2 "Big-Picture Architecture"
+item 4 (augmented Q with SwiGLU gating).  This module only marshals arrays.
 
 Inputs are bf16 tensors (torch) or uint16 arrays holding bf16 bit patterns.
 """
@@ -67,6 +68,10 @@ def _load():
     lib.oracle_decode_up_projected.restype = c_i
     lib.oracle_fold_query.argtypes = [c_i] * 6 + [c_p] * 3
     lib.oracle_fold_query.restype = c_i
+    lib.oracle_augq_hidden.argtypes = [c_i] * 3 + [c_p] * 4 + [c_i, c_p, c_i]
+    lib.oracle_augq_hidden.restype = c_i
+    lib.oracle_augq_down.argtypes = [c_i] * 3 + [c_p] * 3 + [c_i]
+    lib.oracle_augq_down.restype = c_i
     _lib = lib
     return lib
 
@@ -263,3 +268,40 @@ def fold_query(q_aug, w_up, n_k: int) -> np.ndarray:
     rc = _load().oracle_fold_query(B, n_q, n_k, d_q, d_k, w_heads, _ptr(qb), _ptr(wb), _ptr(out))
     _check(rc, "fold_query")
     return out
+
+
+def augq_hidden(x, w_gate, w_up, *, rows=None, threads: int = 0) -> np.ndarray:
+    """fp64 gated hidden state of the augmented query projection, SiLU(x W_gate^T) * (x W_up^T):
+    x [tokens, d_model], w_gate / w_up [d_inter, d_model] (bf16).  ``rows``: token indices to
+    evaluate (all when None).  [n_rows, d_inter]."""
+    xb, gb, ub = _bits(x), _bits(w_gate), _bits(w_up)
+    tokens, d_model = xb.shape
+    d_inter, d_model2 = gb.shape
+    assert ub.shape == gb.shape and d_model == d_model2
+    r = None if rows is None else np.ascontiguousarray(np.asarray(rows, np.int32))
+    n = tokens if r is None else len(r)
+    out = np.empty((n, d_inter), np.float64)
+    rc = _load().oracle_augq_hidden(tokens, d_model, d_inter, _ptr(xb), _ptr(gb), _ptr(ub),
+                                    None if r is None else _ptr(r), n, _ptr(out), threads)
+    _check(rc, "augq_hidden")
+    return out
+
+
+def augq_down(h, w_down, *, threads: int = 0) -> np.ndarray:
+    """fp64 down projection h W_down^T: h [n_rows, d_inter] (any float array, e.g. a rounded
+    hidden state), w_down [d_out, d_inter] (bf16).  [n_rows, d_out]."""
+    hd = np.ascontiguousarray(np.asarray(h, np.float64))
+    wb = _bits(w_down)
+    n, d_inter = hd.shape
+    d_out, d_inter2 = wb.shape
+    assert d_inter == d_inter2
+    out = np.empty((n, d_out), np.float64)
+    rc = _load().oracle_augq_down(n, d_inter, d_out, _ptr(hd), _ptr(wb), _ptr(out), threads)
+    _check(rc, "augq_down")
+    return out
+
+
+def augq_project(x, w_gate, w_up, w_down, *, rows=None, threads: int = 0) -> np.ndarray:
+    """fp64 augmented query q = q_down(SiLU(q_gate(x)) * q_up(x)) for the token rows ``rows``
+    (all when None): [n_rows, d_out]."""
+    return augq_down(augq_hidden(x, w_gate, w_up, rows=rows, threads=threads), w_down, threads=threads)

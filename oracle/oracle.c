@@ -24,6 +24,9 @@
  *                Existing Approaches Fall Short", system-level optimisations)
  *   d_q != d_k   each cached K row is projected up to the query width,
  *                k_up = W k, before the dot product         (Step 4, Attend)
+ *   augmented Q  q = q_down( SiLU(q_gate(x)) * q_up(x) ), SiLU(g) = g / (1 + e^-g),
+ *                three bias-free linear maps (section 3.2 "Big-Picture
+ *                Architecture", item 4: augmented Q with SwiGLU gating)
  *
  * All arithmetic is fp64.  bf16 inputs arrive as raw 16-bit patterns and are
  * widened exactly.  The top-k selection ranks positions by the EXACT dot
@@ -634,5 +637,77 @@ int oracle_fold_query(int batch, int n_q, int n_k, int d_q, int d_k, int w_heads
                 o[c] = acc;
             }
         }
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* Augmented query projection (section 3.2, item 4)                     */
+/* ------------------------------------------------------------------ */
+/* The hidden state x passes through two parallel bias-free linear maps, q_gate
+ * and q_up; the gate's output goes through SiLU (the Swish of SwiGLU) and
+ * multiplies the up branch element by element; q_down maps the product to the
+ * query width.  Weights follow the linear-layer layout: W[o][i] is the weight
+ * of input feature i in output feature o.
+ *
+ * oracle_augq_hidden: h[r][o] = SiLU(sum_i x[t][i] Wg[o][i]) * sum_i x[t][i] Wu[o][i]
+ *   for the token rows t = rows[r] (all tokens when rows is NULL; n_rows of them).
+ *   x [tokens, d_model], Wg and Wu [d_inter, d_model] bf16; h [n_rows, d_inter] fp64.
+ * oracle_augq_down: q[r][o] = sum_i h[r][i] Wd[o][i]; h [n_rows, d_inter] fp64 (any
+ *   source, e.g. the GPU's rounded hidden state), Wd [d_out, d_inter] bf16, q fp64. */
+
+typedef struct {
+    int d_in, d_out;
+    const uint16_t *x;      /* bf16 rows of width d_in (hidden stage) */
+    const double *xd;       /* fp64 rows of width d_in (down stage)   */
+    const uint16_t *w0, *w1;
+    const int32_t *rows;
+    double *out;
+} augq_ctx;
+
+static double silu(double g) { return g / (1.0 + exp(-g)); }
+
+static void augq_hidden_row(void *vctx, int64_t r) {
+    const augq_ctx *c = (const augq_ctx *)vctx;
+    const int64_t t = c->rows ? c->rows[r] : r;
+    const uint16_t *xr = c->x + t * c->d_in;
+    for (int o = 0; o < c->d_out; ++o) {
+        const uint16_t *wg = c->w0 + (int64_t)o * c->d_in, *wu = c->w1 + (int64_t)o * c->d_in;
+        double g = 0.0, u = 0.0;
+        for (int i = 0; i < c->d_in; ++i) {
+            const double xi = bf16_to_f64(xr[i]);
+            g += xi * bf16_to_f64(wg[i]);
+            u += xi * bf16_to_f64(wu[i]);
+        }
+        c->out[r * c->d_out + o] = silu(g) * u;
+    }
+}
+
+static void augq_down_row(void *vctx, int64_t r) {
+    const augq_ctx *c = (const augq_ctx *)vctx;
+    const double *hr = c->xd + r * c->d_in;
+    for (int o = 0; o < c->d_out; ++o) {
+        const uint16_t *wd = c->w0 + (int64_t)o * c->d_in;
+        double acc = 0.0;
+        for (int i = 0; i < c->d_in; ++i) acc += hr[i] * bf16_to_f64(wd[i]);
+        c->out[r * c->d_out + o] = acc;
+    }
+}
+
+int oracle_augq_hidden(int tokens, int d_model, int d_inter, const uint16_t *x, const uint16_t *w_gate,
+                       const uint16_t *w_up, const int32_t *rows, int n_rows, double *h, int n_threads) {
+    if (tokens < 0 || d_model < 1 || d_inter < 1 || n_rows < 0 || !x || !w_gate || !w_up || !h) return -1;
+    if (!rows && n_rows != tokens) return -1;
+    for (int r = 0; rows && r < n_rows; ++r)
+        if (rows[r] < 0 || rows[r] >= tokens) return -1;
+    augq_ctx c = {d_model, d_inter, x, NULL, w_gate, w_up, rows, h};
+    run_rows(augq_hidden_row, &c, n_rows, n_threads);
+    return 0;
+}
+
+int oracle_augq_down(int n_rows, int d_inter, int d_out, const double *h, const uint16_t *w_down, double *q,
+                     int n_threads) {
+    if (n_rows < 0 || d_inter < 1 || d_out < 1 || !h || !w_down || !q) return -1;
+    augq_ctx c = {d_inter, d_out, NULL, h, w_down, NULL, NULL, q};
+    run_rows(augq_down_row, &c, n_rows, n_threads);
     return 0;
 }
