@@ -22,7 +22,7 @@ __all__ = [
     "decode", "decode_workspace", "decode_plan", "decode_from_host", "decode_topv", "decode_topv_workspace",
     "prefill_causal", "device_status", "selftest_wait_timeout", "DiffqkvError", "Dims", "library_path",
     "decode_noalloc", "decode_append", "decode_paged", "prefill_causal_prefix", "fold_query", "workspace_status",
-    "decode_topv_paged",
+    "decode_topv_paged", "augq_project",
 ]
 
 library_path = _capi.LIB_PATH
@@ -203,6 +203,41 @@ def fold_query(q_aug: torch.Tensor, w_up: torch.Tensor, *, n_k: int, out: Option
                                   _stream_ptr(stream))
     check(st, "diffqkv_fold_query")
     return out
+
+
+def augq_project(x: torch.Tensor, w_gate: torch.Tensor, w_up: torch.Tensor, w_down: torch.Tensor, *,
+                 h_out: Optional[torch.Tensor] = None, q_out: Optional[torch.Tensor] = None,
+                 status: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None):
+    """Augmented query projection q = (SiLU(x W_gate^T) * (x W_up^T)) W_down^T.
+
+    x [tokens, d_model]; w_gate, w_up [d_inter, d_model]; w_down [d_out, d_inter] (bf16, CUDA).
+    Returns (q [tokens, d_out], h [tokens, d_inter]), h being the gated hidden state the second
+    GEMM read.  ``status``: an int32 CUDA tensor of one element, zero, for this call's device-side
+    error (else the per-device word)."""
+    _bf16_dev(x, "x", 2)
+    _bf16_dev(w_gate, "w_gate", 2)
+    _bf16_dev(w_up, "w_up", 2)
+    _bf16_dev(w_down, "w_down", 2)
+    tokens, d_model = x.shape
+    d_inter = w_gate.shape[0]
+    d_out = w_down.shape[0]
+    if w_gate.shape != (d_inter, d_model) or w_up.shape != (d_inter, d_model) or w_down.shape != (d_out, d_inter):
+        raise ValueError("x / w_gate / w_up / w_down shapes disagree")
+    if h_out is None:
+        h_out = torch.empty((tokens, d_inter), dtype=torch.bfloat16, device=x.device)
+    if q_out is None:
+        q_out = torch.empty((tokens, d_out), dtype=torch.bfloat16, device=x.device)
+    _bf16_dev(h_out, "h_out", 2)
+    _bf16_dev(q_out, "q_out", 2)
+    if h_out.shape != (tokens, d_inter) or q_out.shape != (tokens, d_out):
+        raise ValueError("h_out / q_out shapes disagree")
+    if status is not None:
+        _status_word(status)
+    st = lib().diffqkv_augq_project(_ptr(x), _ptr(w_gate), _ptr(w_up), _ptr(w_down), tokens, d_model, d_inter,
+                                    d_out, _ptr(h_out), _ptr(q_out), None if status is None else _ptr(status),
+                                    _stream_ptr(stream))
+    check(st, "diffqkv_augq_project")
+    return q_out, h_out
 
 
 def decode_from_host(q_host, k_host, v_host, seq_lens_host, out_host, dev_buffers: dict, *,

@@ -331,6 +331,15 @@ diffqkv_status_t diffqkv_prefill_causal_ex(const diffqkv_dims_t *dims, const voi
                                    device_status_word);
 }
 
+diffqkv_status_t diffqkv_augq_project(const void *x, const void *w_gate, const void *w_up, const void *w_down,
+                                      int32_t tokens, int32_t d_model, int32_t d_inter, int32_t d_out,
+                                      void *h_out, void *q_out, int32_t *device_status_word,
+                                      diffqkv_stream_t stream) {
+    diffqkv::ApiRange nvtx_range("diffqkv_augq_project");
+    return diffqkv::augq_launch(x, w_gate, w_up, w_down, tokens, d_model, d_inter, d_out, h_out, q_out,
+                                device_status_word, (cudaStream_t)stream);
+}
+
 diffqkv_status_t diffqkv_workspace_status(void *workspace, size_t workspace_bytes, diffqkv_stream_t stream,
                                           int32_t *device_status) {
     diffqkv::ApiRange nvtx_range("diffqkv_workspace_status");

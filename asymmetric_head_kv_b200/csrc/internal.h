@@ -89,6 +89,12 @@ diffqkv_status_t prefill_launch(const diffqkv_dims_t *d, const void *q, const vo
                                 int32_t seq_len, void *out, cudaStream_t stream, int32_t prefix_len = 0,
                                 int32_t *status = nullptr);
 
+// augq.cu
+// status: device word the kernels report into (NULL: the per-device word).
+diffqkv_status_t augq_launch(const void *x, const void *w_gate, const void *w_up, const void *w_down, int32_t tokens,
+                             int32_t d_model, int32_t d_inter, int32_t d_out, void *h_out, void *q_out,
+                             int32_t *status, cudaStream_t stream);
+
 // api.cu
 diffqkv_status_t wait_timeout_selftest_launch(int64_t timeout_ns, cudaStream_t stream);
 

@@ -29,7 +29,8 @@
  *      - calls that take a workspace (decode, its variants, top-v): the
  *        workspace's first 32-bit word, read and cleared by
  *        diffqkv_workspace_status;
- *      - diffqkv_prefill_causal_ex: the word the caller passes;
+ *      - diffqkv_prefill_causal_ex, diffqkv_augq_project: the word the caller
+ *        passes (NULL: the per-device word);
  *      - every other call (prefill without a word, diffqkv_decode_noalloc,
  *        the wait self-test): the per-device word, read and cleared by
  *        diffqkv_get_device_status.
@@ -213,6 +214,39 @@ diffqkv_status_t diffqkv_decode_paged(const diffqkv_dims_t *dims, const void *q,
  */
 diffqkv_status_t diffqkv_fold_query(const diffqkv_dims_t *dims, int32_t d_q, int32_t w_heads, const void *q_aug,
                                     const void *w_up, void *q_out, diffqkv_stream_t stream);
+
+/*
+ * Augmented query projection (section 3.2 "Big-Picture Architecture", item 4:
+ * augmented Q with SwiGLU gating).  The query comes from a gated projection of
+ * the hidden state whose parameters are never cached:
+ *
+ *   h = SiLU(x W_gate^T) * (x W_up^T)     SiLU(g) = g / (1 + e^-g), elementwise product
+ *   q = h W_down^T
+ *
+ *   x      [tokens, d_model]     hidden states (bf16, device)
+ *   w_gate [d_inter, d_model]    q_gate weights, one row per output feature
+ *   w_up   [d_inter, d_model]    q_up weights
+ *   w_down [d_out, d_inter]      q_down weights
+ *   h_out  [tokens, d_inter]     the gated hidden state (written; bf16)
+ *   q_out  [tokens, d_out]       the query (written; bf16), e.g. [tokens, n_q, d_q]
+ *
+ * Two tcgen05 GEMM launches on `stream`, fp32 accumulation; h is rounded to
+ * bf16 (nearest even) before the second, q once at the end.  When the
+ * attention uses query heads wider than the keys (diffqkv_fold_query), the
+ * fold is linear and composes with q_down offline: per head, W_down's rows for
+ * that head multiplied by W^T give a W_down of d_k-wide heads, and this call
+ * then yields the folded query directly.
+ * d_model a multiple of 64, d_inter a multiple of 128, d_out a multiple of 32
+ * (else DIFFQKV_ERR_UNSUPPORTED); tokens >= 0 (0: nothing is launched, and
+ * x, h_out and q_out may be NULL);
+ * tokens * max(d_model, d_inter, d_out) < 2^31.  Pointers 16-byte aligned.
+ * device_status_word as in diffqkv_prefill_causal_ex (NULL: the per-device
+ * word); it receives DIFFQKV_ERR_DEVICE_TIMEOUT if a bounded wait runs out.
+ */
+diffqkv_status_t diffqkv_augq_project(const void *x, const void *w_gate, const void *w_up, const void *w_down,
+                                      int32_t tokens, int32_t d_model, int32_t d_inter, int32_t d_out,
+                                      void *h_out, void *q_out, int32_t *device_status_word,
+                                      diffqkv_stream_t stream);
 
 /* Optional launch controls for diffqkv_decode_ex (0 = library default). */
 typedef struct {

@@ -102,3 +102,25 @@ def assert_parity_prefill(got, ref, what=""):
     mx, row_rel, _, _ = errs
     assert mx <= ATOL and row_rel <= RTOL, _msg(what, errs)
     return errs
+
+
+def assert_parity_gemm(got, ref, what=""):
+    """Element-wise rule for outputs of unbounded scale (GEMM results): |g - r| <= 1e-2 max(|r|, 1e-2)
+    for every element.  The attention rules' 2e-2 absolute cap would reject the bf16 rounding of
+    values above ~10 (2^-9 of them is over 2e-2); below the floor the bound is 1e-4 absolute."""
+    g = _np(got)
+    assert np.all(np.isfinite(g)), f"{what}: non-finite output"
+    errs = errors(got, ref)
+    _log("gemm-element", what, errs)
+    assert errs[2] <= RTOL, _msg(what, errs)
+    return errs
+
+
+def assert_parity_gemm_vector(got, ref, what=""):
+    """Per-vector rule for GEMM results: max over output rows of ||g - r|| / ||r|| <= 1e-2."""
+    g = _np(got)
+    assert np.all(np.isfinite(g)), f"{what}: non-finite output"
+    errs = errors(got, ref)
+    _log("gemm-vector", what, errs)
+    assert errs[1] <= RTOL, _msg(what, errs)
+    return errs

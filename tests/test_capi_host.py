@@ -328,3 +328,26 @@ def test_checked_build_exports_every_declared_symbol_and_nvtx_switch_is_harmless
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
     r = subprocess.run([sys.executable, "-c", code], env=env, cwd=root, capture_output=True, text=True, timeout=120)
     assert r.returncode == 0 and "ok" in r.stdout, r.stdout + r.stderr
+
+
+def test_augq_project_rejects_before_launch():
+    """The augmented query projection checks pointers, alignment and tile multiples on the host;
+    zero tokens launch nothing (no device needed for any of these)."""
+    lib = _capi.lib()
+
+    def call(x=0x1000, wg=0x2000, wu=0x3000, wd=0x4000, tokens=300, d_model=2048, d_inter=3072, d_out=2048,
+             h=0x5000, q=0x6000, status=None):
+        return lib.diffqkv_augq_project(x, wg, wu, wd, tokens, d_model, d_inter, d_out, h, q, status, None)
+    assert call(x=None) == _capi.INVALID_ARG
+    assert call(h=None) == _capi.INVALID_ARG
+    assert call(tokens=-1) == _capi.INVALID_ARG
+    assert call(d_model=32) == _capi.INVALID_ARG
+    assert call(d_model=2048 + 32) == _capi.UNSUPPORTED   # reduction in whole 64-element steps
+    assert call(d_inter=3072 + 64) == _capi.UNSUPPORTED   # gate/up tiles of 128 features
+    assert call(d_out=2048 + 16) == _capi.UNSUPPORTED     # 32-column epilogue chunks
+    assert call(wd=0x4008) == _capi.MISALIGNED
+    assert call(status=0x7002) == _capi.MISALIGNED
+    assert call(tokens=1 << 20) == _capi.UNSUPPORTED      # tokens * 3072 >= 2^31
+    assert call(tokens=0) == _capi.OK                     # nothing to do
+    assert call(tokens=0, x=None, h=None, q=None) == _capi.OK  # empty tensors have no storage
+    assert call(tokens=0, wg=None) == _capi.INVALID_ARG

@@ -7,7 +7,7 @@ import torch
 
 import oracle
 import workloads as wl
-from parity import assert_parity, assert_parity_prefill, errors
+from parity import assert_parity, assert_parity_gemm, assert_parity_gemm_vector, assert_parity_prefill, errors
 
 
 def _long_context_ref():
@@ -57,3 +57,25 @@ def test_vector_rule_zero_reference_rows_must_be_exact():
     assert errors(np.zeros_like(ref), ref)[1] == 0.0
     with pytest.raises(AssertionError):
         assert_parity_prefill(np.full_like(ref, 1e-6), ref, "nonzero where zero")
+
+
+def test_gemm_rules_scale_free():
+    """GEMM rules: the bf16 rounding of values up to 100 passes (the attention rules' absolute cap
+    would not), a 3% scale error or one element 3% off fails the element rule, and the vector rule
+    rejects a swapped pair of rows."""
+    rng = np.random.default_rng(3)
+    ref = rng.standard_normal((40, 64)) * 30.0
+    got = torch.from_numpy(ref).to(torch.bfloat16)
+    assert errors(got, ref)[0] > 2e-2
+    assert_parity_gemm(got, ref, "bf16 of large values")
+    assert_parity_gemm_vector(got, ref, "bf16 of large values")
+    with pytest.raises(AssertionError):
+        assert_parity(got, ref, "attention rule caps the absolute error")
+    with pytest.raises(AssertionError):
+        assert_parity_gemm(ref * 1.03, ref, "3% scale")
+    bad = ref.copy()
+    bad[5, 7] *= 1.03
+    with pytest.raises(AssertionError):
+        assert_parity_gemm(bad, ref, "one element")
+    with pytest.raises(AssertionError):
+        assert_parity_gemm_vector(ref[[1, 0] + list(range(2, 40))], ref, "rows swapped")

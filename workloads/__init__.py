@@ -23,6 +23,11 @@ Recipe (per workload, ``seed`` fixed per workload):
     (``torch.randperm`` on the CPU generator seeded ``seed + 1``) dealt out
     in sequence order, ceil((seq_len + 1) / page_size) pages per sequence
     (one spare position for an append) and -1 in the unused table entries.
+  * augmented query projection: x [tokens, d_model] ~ N(0, 1) (hidden states
+    after the layer's RMSNorm have unit scale), then W_gate, W_up
+    [d_inter, d_model] and W_down [d_out, d_inter] ~ N(0, 1 / fan_in) (the usual
+    initialisation scale, so the gate and up sums are ~ N(0, 1)), drawn in that
+    order on a generator seeded ``seed``, each rounded to bf16.
 The CPU and CUDA generators produce different streams; each run feeds the
 bytes it generated to both sides.
 """
@@ -182,6 +187,43 @@ def random_paged_inputs(batch, max_blocks, page_size, shape: Shape, seed: int, s
 
 def random_prefill_inputs(batch, seq, shape: Shape, seed: int, device="cpu"):
     return make_prefill_inputs(PrefillWorkload("adhoc", shape, batch, seq, seed), device)
+
+
+@dataclasses.dataclass(frozen=True)
+class AugQWorkload:
+    """Augmented query projection of ``tokens`` hidden states (section 3.2, item 4)."""
+    name: str
+    tokens: int
+    d_model: int
+    d_inter: int
+    d_out: int
+    seed: int
+
+
+# Sigma-1.5B's attention block: hidden 2048, Q intermediate 3072 (1.5x the hidden size), 32 query heads
+# of 64 = 2048 outputs; 16384 tokens = the 2 x 8192 prefill rows.
+AUGQ_16K = AugQWorkload("augq_proj_t16384_d2048_i3072_o2048", 16384, 2048, 3072, 2048, seed=5)
+
+
+def make_augq_inputs(w: AugQWorkload, device="cpu"):
+    """Returns dict(x, w_gate, w_up, w_down) on ``device`` (bf16)."""
+    g = torch.Generator(device=device).manual_seed(w.seed)
+    x = _randn_bf16((w.tokens, w.d_model), g, device)
+    out = {"x": x}
+    for name, rows, fan_in in (("w_gate", w.d_inter, w.d_model), ("w_up", w.d_inter, w.d_model),
+                               ("w_down", w.d_out, w.d_inter)):
+        v = torch.randn((rows, fan_in), generator=g, dtype=torch.float32, device=device) * fan_in ** -0.5
+        out[name] = v.to(torch.bfloat16)
+    return out
+
+
+def random_augq_inputs(tokens, d_model, d_inter, d_out, seed: int, device="cpu"):
+    return make_augq_inputs(AugQWorkload("adhoc", tokens, d_model, d_inter, d_out, seed), device)
+
+
+def augq_flops(w: AugQWorkload) -> int:
+    """FLOPs of the two GEMMs: 2 T d_model (2 d_inter) + 2 T d_inter d_out."""
+    return 2 * w.tokens * w.d_model * 2 * w.d_inter + 2 * w.tokens * w.d_inter * w.d_out
 
 
 # Measurement units (algorithmic traffic/work per step), used by the benchmark.
