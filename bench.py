@@ -416,7 +416,8 @@ def time_paths(ak, peaks, steps: int, warmup: int):
         flops = wl.prefill_causal_flops(w.shape, w.batch, w.seq)
         tf = flops / (ms * 1e-3) / 1e12
         res[w.name] = {"ms": ms, "causal_flops": flops, "tflops": tf, "bound": "tensor", "peak_tflops": bf16_peak,
-                       "frac": tf / bf16_peak, "peak_source": "bf16_tflops (burst, cuBLAS bf16 GEMM)"}
+                       "frac": tf / bf16_peak, "frac_kind": "FLOP-derived tensor fraction (causal FLOPs / event "
+                       "time / peak)", "peak_source": "bf16_tflops (burst, cuBLAS bf16 GEMM)"}
         del d, out
     # chunked prefill: 2048 new rows over an 8192-position prefix (batch 2, DiffQKV shape)
     P, S, w = 8192, 2048, wl.PREFILL_8K
@@ -510,6 +511,24 @@ def time_paths(ak, peaks, steps: int, warmup: int):
                                         "bound": "launch/latency (L2 flushed between calls)",
                                         "launches_per_call": 1}
     del q_aug, w_up, q_fold
+
+    # augmented query projection of Sigma-1.5B's attention (hidden 2048 -> gated 3072 -> 2048 query
+    # features) for the 16384 rows of the 2 x 8192 prefill: two tcgen05 GEMMs, TFLOP/s
+    w = wl.AUGQ_16K
+    d = wl.make_augq_inputs(w, dev)
+    h_a = torch.empty((w.tokens, w.d_inter), dtype=torch.bfloat16, device=dev)
+    q_a = torch.empty((w.tokens, w.d_out), dtype=torch.bfloat16, device=dev)
+    fn = lambda: ak.augq_project(d["x"], d["w_gate"], d["w_up"], d["w_down"], h_out=h_a, q_out=q_a)  # noqa: E731
+    for _ in range(max(3, warmup)):
+        fn()
+    ms = statistics.median(_timed_calls(fn, steps, flush))
+    flops = wl.augq_flops(w)
+    tf = flops / (ms * 1e-3) / 1e12
+    res[w.name] = {"us": ms * 1e3, "flops": flops, "tflops": tf, "bound": "tensor", "peak_tflops": bf16_peak,
+                   "frac": tf / bf16_peak, "frac_kind": "FLOP-derived (2 GEMMs' FLOPs / event time / peak)",
+                   "peak_source": "bf16_tflops (burst, cuBLAS bf16 GEMM)", "launches_per_call": 2}
+    assert ak.device_status() == 0
+    del d, h_a, q_a
 
     w = wl.TOPV_64K
     d = wl.make_decode_inputs(w, dev)
