@@ -53,6 +53,8 @@ PROFILE_CASES = {
     "topv_b4_t65536": wl.TOPV_64K,
     "decode_paged_b4_t32768_p16": wl.DecodeWorkload("decode_paged_b4_t32768_p16", wl.DIFFQKV, 4, 32768, seed=1,
                                                     page_size=16),
+    "decode_b1_t512": wl.DECODE_SMALL,
+    "augq_t16384": wl.AUGQ_16K,
 }
 L2_FLUSH_BYTES = 256 << 20  # written between timed calls whose inputs fit in the 126 MB L2
 
@@ -347,7 +349,12 @@ def run_profile_case(name: str, launches: int = 4):
 
     w = PROFILE_CASES[name]
     dev = torch.device("cuda", 0)
-    if isinstance(w, wl.PrefillWorkload):
+    if isinstance(w, wl.AugQWorkload):
+        d = wl.make_augq_inputs(w, dev)
+        for _ in range(launches):
+            ak.augq_project(d["x"], d["w_gate"], d["w_up"], d["w_down"])
+        what = f"flops/call {wl.augq_flops(w)} (two launches per call)"
+    elif isinstance(w, wl.PrefillWorkload):
         d = wl.make_prefill_inputs(w, dev)
         out = torch.empty((w.batch, w.seq, w.shape.n_q, w.shape.d_v), dtype=torch.bfloat16, device=dev)
         for _ in range(launches):
