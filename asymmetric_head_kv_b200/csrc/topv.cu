@@ -19,9 +19,10 @@
 //     TMA into a ring; one thread issues tcgen05 MMAs S = K_tile q^T (M = 128
 //     positions, N = 16 rows of q, zero-padded past the group's, K = d_k) into
 //     a ring of TMEM buffers; three consumer warpgroups take the tiles in turn,
-//     read one position's scores per thread out of TMEM, keep them in shared
-//     memory with a 2048-bucket histogram of the top 11 bits of each score's
-//     order key, and fold the position's K row into the largest |k|.
+//     read one position's scores per thread out of TMEM, keep the group's rows
+//     of them in TMEM (the whole part's scores stay there, so shared memory is
+//     all ring), add them to a 2048-bucket histogram of the top 11 bits of each
+//     score's order key, and fold the position's K row into the largest |k|.
 //     Histograms go to global memory; the CTA arrives on the unit's counter H.
 //  2. Candidates.  Once H counts all Y parts, each CTA finds in every row's
 //     histogram the bucket holding the k-th largest score and emits every own
@@ -68,8 +69,10 @@ constexpr int kMmaWarp = kConsumerWarps + 1;
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
 constexpr int kQRows = 16;                 // rows of q in the MMA's B operand (its N), zero past the group's
-constexpr int kTmemBufs = 8;               // TMEM score buffers of kQRows columns
-constexpr int kTmemCols = 128;             // allocation: kTmemBufs * kQRows columns
+constexpr int kTmemBufs = 8;               // TMEM buffers of kQRows columns the MMAs write
+constexpr int kTmemCols = 512;             // allocation: the MMA buffers, then the part's scores
+constexpr int kScoreCol0 = kTmemBufs * kQRows;      // first column of the part's scores
+constexpr int kScoreCols = kTmemCols - kScoreCol0;  // tile i's row hh at column kScoreCol0 + i QPK + hh
 constexpr int kHistBuckets = 2048;       // both histogram levels: 11 bits of the order key
 constexpr int kHistWords = kHistBuckets / 2;  // shared histogram: two 16-bit counters per word
 constexpr int kRadixBuckets = 1024;      // last 10 key bits
@@ -79,8 +82,7 @@ constexpr int kKeyWords = 19;            // 18 superaccumulator digits + inverte
 constexpr int kTopvHeader = 256;
 constexpr int kTopvMaxContext = 131072;  // bitmap of kept positions
 constexpr int kMaxParts = 256;           // CTAs per unit (sizes the per-part records)
-constexpr int kMaxStages = 6;
-constexpr int kEmitIters = 8;            // float4 vectors per thread and emission chunk (32 mask bits)
+constexpr int kMaxStages = 12;
 constexpr int kTableAhead = 4;           // paged producer: tiles whose block-table entries are in flight
 constexpr int kTableRing = 8;            // rows of the entry ring (> kTableAhead)
 constexpr int kRowInfoWords = 8;
@@ -116,7 +118,6 @@ struct TopvArgs {
     int32_t batch, n_q, n_k, n_v, t_max, t_pad, topk, k_pad, q_per_v;
     int32_t parts;        // Y: CTAs per unit
     int32_t units_per_round, rounds, stages;
-    int32_t score_stride; // floats between two rows' score arrays in shared memory
     int32_t cand_cap;     // candidates the select keeps in shared memory
     int32_t full_weights;
     // paged caches: block_table == null means contiguous [B, t_max, heads, d] caches; else K and V
@@ -477,6 +478,33 @@ __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[N]) {
     }
 }
 
+// registers -> TMEM: this warp's 32 lanes, N consecutive 32-bit columns each (N = 1 .. 16).
+template <int N>
+__device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t (&r)[N]) {
+    if constexpr (N == 1) {
+        asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(r[0]) : "memory");
+    } else if constexpr (N == 2) {
+        asm volatile("tcgen05.st.sync.aligned.32x32b.x2.b32 [%0], {%1, %2};" ::"r"(taddr), "r"(r[0]), "r"(r[1])
+                     : "memory");
+    } else if constexpr (N == 4) {
+        asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(r[0]),
+                     "r"(r[1]), "r"(r[2]), "r"(r[3])
+                     : "memory");
+    } else if constexpr (N == 8) {
+        asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+                     "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+                     : "memory");
+    } else {
+        static_assert(N == 16, "column count");
+        asm volatile(
+            "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+            "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+            "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+            "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+            : "memory");
+    }
+}
+
 // Two bf16 per word: the result's halves have the larger magnitude of each pair (their signs are
 // the XOR of the inputs' signs, which the caller masks off).
 __device__ __forceinline__ uint32_t bf16x2_absmax(uint32_t a, uint32_t b) {
@@ -525,8 +553,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // dynamic shared memory: q_b [KB][kQRows][128 B] (bf16, 128-byte swizzled) | barriers |
     // q [QPK][DK] fp32 | histograms [QPK][kHistWords] | ring [stages][TILE_BYTES] (1024-byte
-    // aligned for the 128-byte swizzle) | scores [QPK][score_stride].  The select and the gather
-    // reuse everything from the ring on ("overlay"); what sits before it is never overwritten.
+    // aligned for the 128-byte swizzle).  The select and the gather reuse the ring ("overlay");
+    // what sits before it is never overwritten.  The part's scores live in TMEM.
     extern __shared__ uint8_t dsm_raw[];
     uint8_t *const base = align_smem_1024(dsm_raw);
     uint8_t *const q_b = base;
@@ -538,7 +566,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     float *const q_s = reinterpret_cast<float *>(base + kQRows * DK * 2 + kBarBytes);
     uint32_t *const hist_s = reinterpret_cast<uint32_t *>(q_s + QPK * DK);
     uint8_t *const ring = base + head_bytes(DK, QPK);
-    float *const scores = reinterpret_cast<float *>(ring + (size_t)a.stages * TILE_BYTES);
     uint8_t *const overlay = ring;
     __shared__ Shared sh;
     volatile int *const abort_flag = &sh.abort_flag;
@@ -818,12 +845,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
 #pragma unroll
                     for (int hh = 0; hh < QPK; ++hh) {
-                        const float score = __uint_as_float(sr[hh]);
-                        if (in_bounds(lp, a.score_stride, a.status)) scores[(size_t)hh * a.score_stride + lp] = score;
-                        const uint32_t bk = float_key(score) >> 21;
+                        const uint32_t bk = float_key(__uint_as_float(sr[hh])) >> 21;
                         atomicAdd(hist_s + hh * kHistWords + (bk >> 1), 1u << ((bk & 1u) << 4));
                     }
                 }
+                // the part keeps its scores in TMEM: tile t's rows at columns kScoreCol0 + (t - tb) QPK
+                const int col = kScoreCol0 + (t - tb) * QPK;
+                if (in_bounds(col + QPK - 1, kTmemCols, a.status))
+                    tmem_st_cols<QPK>(t_lane + (uint32_t)col, sr);
                 kk += kConsumerGroups;
                 st += kConsumerGroups;
                 while (st >= a.stages) {
@@ -831,6 +860,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     par ^= 1u;
                 }
             }
+            tmem_wait_st();
+            tc_fence_before();  // the scores' stores, before the barrier that ends the phase
             // largest |k| as a bf16 magnitude pattern (order-preserving for non-negative values)
             uint32_t kmx = max(kacc & 0x7fffu, (kacc >> 16) & 0x7fffu);
 #pragma unroll
@@ -878,107 +909,111 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         __syncthreads();
+        tc_fence_after();  // the scores the consumers stored to TMEM in phase 1
+        // The part's scores, read back out of TMEM: warp w reads TMEM lanes 32 (w % 4) .. + 31 (the
+        // positions 32 (w % 4) + lane of a tile) of the tiles w / 4, w / 4 + 4, ...; f(lp, valid, s)
+        // sees position lp of the part and its QPK scores.
+        auto for_each_score = [&](auto &&f) {
+            const uint32_t t_lane = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+            for (int i = warp >> 2; i < te - tb; i += kWarps / 4) {
+                uint32_t sr[QPK];
+                tmem_ld_cols<QPK>(t_lane + (uint32_t)(kScoreCol0 + i * QPK), sr);
+                tmem_wait_ld();
+                const int lp = i * kTile + (warp & 3) * 32 + lane;
+                f(lp, lp < np, sr);
+            }
+        };
         if (a.full_weights && T > K) {
             // this part's share of each row's full softmax denominator: its max and its sum of exponentials
+            float mx[QPK], sum[QPK];
+#pragma unroll
+            for (int hh = 0; hh < QPK; ++hh) mx[hh] = -INFINITY, sum[hh] = 0.f;
+            for_each_score([&](int, bool valid, const uint32_t(&sr)[QPK]) {
+                if (valid)
+#pragma unroll
+                    for (int hh = 0; hh < QPK; ++hh) mx[hh] = fmaxf(mx[hh], __uint_as_float(sr[hh]));
+            });
             for (int hh = 0; hh < QPK; ++hh) {
-                const float *s = scores + (size_t)hh * a.score_stride;
-                float mx = -INFINITY;
-                for (int p = tid; p < np; p += kThreads) mx = fmaxf(mx, s[p]);
+                float m = mx[hh];
 #pragma unroll
-                for (int off = 16; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-                if (lane == 0) sh.red[warp] = mx;
+                for (int off = 16; off >= 1; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+                if (lane == 0) sh.red[warp] = m;
                 __syncthreads();
-                mx = sh.red[0];
-                for (int w = 1; w < kWarps; ++w) mx = fmaxf(mx, sh.red[w]);
+                m = sh.red[0];
+                for (int w = 1; w < kWarps; ++w) m = fmaxf(m, sh.red[w]);
                 __syncthreads();
-                float sum = 0.f;
-                if (mx != -INFINITY)
-                    for (int p = tid; p < np; p += kThreads) sum += fast_exp2((s[p] - mx) * a.scale_log2);
+                mx[hh] = m;
+            }
+            for_each_score([&](int, bool valid, const uint32_t(&sr)[QPK]) {
+                if (valid)
 #pragma unroll
-                for (int off = 16; off >= 1; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-                if (lane == 0) sh.red[warp] = sum;
+                    for (int hh = 0; hh < QPK; ++hh)
+                        if (mx[hh] != -INFINITY)
+                            sum[hh] += fast_exp2((__uint_as_float(sr[hh]) - mx[hh]) * a.scale_log2);
+            });
+            for (int hh = 0; hh < QPK; ++hh) {
+                float v = sum[hh];
+#pragma unroll
+                for (int off = 16; off >= 1; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+                if (lane == 0) sh.red[warp] = v;
                 __syncthreads();
                 if (tid == 0) {
                     float tot = 0.f;
                     for (int w = 0; w < kWarps; ++w) tot += sh.red[w];
-                    a.chunk_part[(size_t)(row0 + hh) * kMaxParts + j] = make_float2(mx, tot);
+                    a.chunk_part[(size_t)(row0 + hh) * kMaxParts + j] = make_float2(mx[hh], tot);
                 }
                 __syncthreads();
             }
         }
-        // emit candidates.  Thread t tests the float4 vectors t, t + kThreads, ... of a chunk of
-        // kEmitIters * kThreads vectors for every row of the group (all loads independent), keeps a
-        // hit mask per row, and one block scan of the per-thread hit counts plus one atomic per
-        // (CTA, row) gives every hit its slot in the row's candidate list.
+        // emit candidates: each thread counts its hits per row (first pass over its scores), one
+        // block scan of the counts plus one atomic per (CTA, row) gives every hit its slot in the
+        // row's candidate list, and the second pass writes them
         {
-            const int nv = (np + 3) / 4;
-            for (int v0 = 0; v0 < nv; v0 += kThreads * kEmitIters) {
-                uint32_t mask[QPK];  // bit 4i + e: position 4 (v0 + tid + kThreads i) + e is a candidate
+            uint32_t cnt[QPK];
 #pragma unroll
-                for (int hh = 0; hh < QPK; ++hh) mask[hh] = 0u;
+            for (int hh = 0; hh < QPK; ++hh) cnt[hh] = 0u;
+            for_each_score([&](int, bool valid, const uint32_t(&sr)[QPK]) {
 #pragma unroll
-                for (int i = 0; i < kEmitIters; ++i) {
-                    const int v = v0 + tid + kThreads * i;
-                    if (v < nv) {
+                for (int hh = 0; hh < QPK; ++hh) cnt[hh] += (valid && __uint_as_float(sr[hh]) >= sh.lower[hh]) ? 1u : 0u;
+            });
+            // exclusive prefix of every row's hit count, two rows per scan (16-bit fields: a part holds
+            // at most kScoreCols / QPK * kTile <= 49152 positions)
+            uint32_t slot[QPK];
 #pragma unroll
-                        for (int hh = 0; hh < QPK; ++hh) {
-                            const float4 x = *reinterpret_cast<const float4 *>(scores + (size_t)hh * a.score_stride + 4 * v);
-                            const float lower = sh.lower[hh];
-                            const int pp = 4 * v;
-                            uint32_t m = 0;
-                            m |= (pp + 0 < np && x.x >= lower) ? 1u : 0u;
-                            m |= (pp + 1 < np && x.y >= lower) ? 2u : 0u;
-                            m |= (pp + 2 < np && x.z >= lower) ? 4u : 0u;
-                            m |= (pp + 3 < np && x.w >= lower) ? 8u : 0u;
-                            mask[hh] |= m << (4 * i);
-                        }
-                    }
+            for (int hh = 0; hh < QPK; hh += 2) {
+                const uint32_t packed = cnt[hh] | (hh + 1 < QPK ? cnt[hh + 1 < QPK ? hh + 1 : hh] << 16 : 0u);
+                uint32_t total;
+                const uint32_t ex = block_exclusive_scan(packed, sh.warp_sums, &total);
+                slot[hh] = ex & 0xffffu;
+                if (hh + 1 < QPK) slot[hh + 1 < QPK ? hh + 1 : hh] = ex >> 16;
+                if (tid == 0) {
+                    sh.emit_total[hh] = total & 0xffffu;
+                    if (hh + 1 < QPK) sh.emit_total[hh + 1] = total >> 16;
                 }
-                // exclusive prefix of every row's hit count, two rows per scan (16-bit fields: a chunk
-                // holds at most kEmitIters * kThreads * 4 = 16384 positions)
-                uint32_t pre[QPK];
+            }
+            __syncthreads();
+            if (tid < QPK)
+                sh.emit_base[tid] = sh.emit_total[tid]
+                                        ? atomicAdd(a.row_sync + (size_t)(row0 + tid) * 4 + kRsCand, sh.emit_total[tid])
+                                        : 0u;
+            __syncthreads();
 #pragma unroll
-                for (int hh = 0; hh < QPK; hh += 2) {
-                    const uint32_t packed = (uint32_t)__popc(mask[hh]) |
-                                            (hh + 1 < QPK ? (uint32_t)__popc(mask[hh + 1 < QPK ? hh + 1 : hh]) << 16 : 0u);
-                    uint32_t total;
-                    const uint32_t ex = block_exclusive_scan(packed, sh.warp_sums, &total);
-                    pre[hh] = ex & 0xffffu;
-                    if (hh + 1 < QPK) pre[hh + 1 < QPK ? hh + 1 : hh] = ex >> 16;
-                    if (tid == 0) {
-                        sh.emit_total[hh] = total & 0xffffu;
-                        if (hh + 1 < QPK) sh.emit_total[hh + 1] = total >> 16;
-                    }
-                }
-                __syncthreads();
-                if (tid < QPK)
-                    sh.emit_base[tid] = sh.emit_total[tid]
-                                            ? atomicAdd(a.row_sync + (size_t)(row0 + tid) * 4 + kRsCand, sh.emit_total[tid])
-                                            : 0u;
-                __syncthreads();
+            for (int hh = 0; hh < QPK; ++hh) slot[hh] += sh.emit_base[hh];
+            for_each_score([&](int lp, bool valid, const uint32_t(&sr)[QPK]) {
 #pragma unroll
                 for (int hh = 0; hh < QPK; ++hh) {
-                    uint32_t m = mask[hh];
-                    if (!m) continue;
-                    const int row = row0 + hh;
-                    int32_t *cj = a.cand_j + (size_t)row * a.t_pad;
-                    float *cs = a.cand_s + (size_t)row * a.t_pad;
-                    const float *srow = scores + (size_t)hh * a.score_stride;
-                    uint32_t slot = sh.emit_base[hh] + pre[hh];
-                    while (m) {
-                        const int bit = __ffs(m) - 1;
-                        m &= m - 1u;
-                        const int p = 4 * (v0 + tid + kThreads * (bit >> 2)) + (bit & 3);
-                        if (slot < (uint32_t)a.t_pad) {  // (a count left over by an aborted call stays in bounds)
-                            cj[slot] = p0 + p;
-                            cs[slot] = srow[p];
+                    const float x = __uint_as_float(sr[hh]);
+                    if (valid && x >= sh.lower[hh]) {
+                        if (slot[hh] < (uint32_t)a.t_pad) {  // (a count left over by an aborted call stays in bounds)
+                            a.cand_j[(size_t)(row0 + hh) * a.t_pad + slot[hh]] = p0 + lp;
+                            a.cand_s[(size_t)(row0 + hh) * a.t_pad + slot[hh]] = x;
                         }
-                        ++slot;
+                        ++slot[hh];
                     }
                 }
-                __syncthreads();  // emit_base is reused by the next chunk
-            }
+            });
         }
+        tc_fence_before();  // the score loads, before the barriers that let the next round's MMAs in
         cta_arrive(usync + kUsCand);
 
         // =============================================================== 3. select
@@ -1383,13 +1418,12 @@ size_t zeroed_bytes(const diffqkv_dims_t *d) {
 
 // Launch plan: parts per unit (Y), rounds, ring depth, shared memory.
 struct Plan {
-    int parts, units_per_round, rounds, stages, score_stride, cand_cap, grid;
+    int parts, units_per_round, rounds, stages, cand_cap, grid;
     size_t smem;
 };
 
-
-// The largest Y that is still useful is one tile per part; the smallest is the one whose
-// part's scores fit next to a two-stage ring.  Y = G / units when that fits (one round).
+// Y = G / units (one round) unless a part's scores would not fit in TMEM; the ring takes as many
+// stages as shared memory holds.
 bool make_plan(const diffqkv_dims_t *d, int32_t t_max, int num_sms, Plan *p) {
     const int qpk = d->n_q / d->n_k;
     const int units = d->batch * d->n_k;
@@ -1399,33 +1433,31 @@ bool make_plan(const diffqkv_dims_t *d, int32_t t_max, int num_sms, Plan *p) {
     // the select's overlay: bitmap and word prefixes, a histogram, then candidates (at least 1024)
     const size_t sel_fixed = 2 * (t_pad / 8) + (size_t)kHistBuckets * 4;
     const size_t gather_bytes = (size_t)kWarps * (d->d_v + 4) * 4;
-    // dynamic bytes: 1 KB of alignment slack, the head, then the overlay (ring + scores, at least
-    // what the select and the gather need)
-    auto layout = [&](int Y, int stages, int *stride, size_t *smem, int *cap) {
-        const int tiles = (nt_max + Y - 1) / Y;
-        // a row's scores start 8 banks after the previous row's: one warp's stores of 8 positions x 4
-        // rows touch 32 distinct banks
-        *stride = (tiles * kTile + 31) / 32 * 32 + 8;
-        const size_t ring_scores = (size_t)stages * kTile * d->d_k * 2 + (size_t)qpk * (*stride) * 4;
-        const size_t overlay = std::max({ring_scores, sel_fixed + 8 * 1024, gather_bytes});
+    // a part's scores stay in TMEM: at most kScoreCols / qpk tiles per part
+    const int max_tiles = kScoreCols / qpk;
+    int Y = std::max(1, std::min(G / std::max(1, units), nt_max));
+    Y = std::max(Y, (nt_max + max_tiles - 1) / max_tiles);
+    if (Y > G) return false;
+    // dynamic bytes: 1 KB of alignment slack, the head, then the overlay (the ring, at least what the
+    // select and the gather need)
+    auto layout = [&](int stages, size_t *smem, int *cap) {
+        const size_t ring = (size_t)stages * kTile * d->d_k * 2;
+        const size_t overlay = std::max({ring, sel_fixed + 8 * 1024, gather_bytes});
         *smem = 1024 + head_bytes(d->d_k, qpk) + overlay;
         *cap = (int)std::min<size_t>((overlay - sel_fixed) / 8, t_pad);
         return *smem <= (size_t)kDynSmemCap;
     };
-    int Y = std::max(1, std::min(G / std::max(1, units), nt_max));
-    int stride = 0, cap = 0;
     size_t smem = 0;
-    while (Y <= G && !layout(Y, 2, &stride, &smem, &cap)) ++Y;
-    if (Y > G) return false;
+    int cap = 0;
     int stages = 2;
-    while (stages < kMaxStages && layout(Y, stages + 1, &stride, &smem, &cap)) ++stages;
-    layout(Y, stages, &stride, &smem, &cap);
+    if (!layout(stages, &smem, &cap)) return false;
+    while (stages < kMaxStages && layout(stages + 1, &smem, &cap)) ++stages;
+    layout(stages, &smem, &cap);
     p->parts = Y;
     p->units_per_round = std::max(1, G / Y);
     p->rounds = (units + p->units_per_round - 1) / p->units_per_round;
     p->grid = std::min(units, p->units_per_round) * Y;
     p->stages = stages;
-    p->score_stride = stride;
     p->cand_cap = cap;
     p->smem = smem;
     return true;
@@ -1530,7 +1562,6 @@ diffqkv_status_t topv_launch(const diffqkv_dims_t *d, const void *q, const void 
     a.units_per_round = plan.units_per_round;
     a.rounds = plan.rounds;
     a.stages = plan.stages;
-    a.score_stride = plan.score_stride;
     a.cand_cap = plan.cand_cap;
     a.full_weights = (flags & DIFFQKV_TOPV_FULL_SOFTMAX_WEIGHTS) ? 1 : 0;
     a.block_table = paged ? paged->block_table : nullptr;
