@@ -569,28 +569,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                                    fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
             const float m_new = mx * a.scale_log2;
-            bool waited_pv = false;
+            // the lazy O rescale is decided here and done after P is stored (the row's 128 scores are
+            // dead by then; loading O next to them overran the 168 registers ten warps leave a thread)
+            bool rescale = false;
+            float alpha = 1.f;
             if (n == 0) {
                 m_used = m_new;
             } else {
                 const bool need = m_new > m_used + kRescaleLog2;
                 if (__any_sync(0xffffffffu, need)) {
-                    // O must be final for tile n-1 before it is rescaled in TMEM
-                    mbar_wait_bounded(&pv_done[t], (uint32_t)((n - 1) & 1), a.wait_limit_ns, abort_flag, a.status);
-                    waited_pv = true;
-                    tc_fence_after();
-                    const float alpha = need ? fast_exp2(m_used - m_new) : 1.f;
-#pragma unroll 1
-                    for (int c = 0; c < DV; c += 32) {
-                        uint32_t rr[32];
-                        tmem_ld32(t_o + (uint32_t)c, rr);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) rr[e] = __float_as_uint(__uint_as_float(rr[e]) * alpha);
-                        tmem_st32(t_o + (uint32_t)c, rr);
-                    }
-                    tmem_wait_st();
+                    rescale = true;
                     if (need) {
+                        alpha = fast_exp2(m_used - m_new);
                         l *= alpha;
                         m_used = m_new;
                     }
@@ -602,10 +592,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             const f32x2_t nm2 = f2_pack(-m_used, -m_used);
             f32x2_t l2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-            for (int c0 = 0; c0 < BN; c0 += 64) {
-                uint32_t pk[32];
+            for (int c0 = 0; c0 < BN; c0 += 32) {  // 32 keys (16 packed columns) per store
+                uint32_t pk[16];
 #pragma unroll
-                for (int c = 0; c < 64; c += 2) {
+                for (int c = 0; c < 32; c += 2) {
                     float t0, t1;
                     f2_unpack(f2_fma(f2_pack(s[c0 + c], s[c0 + c + 1]), sc2, nm2), t0, t1);
                     const float p0 = fast_exp2(t0);
@@ -613,15 +603,29 @@ __global__ void __launch_bounds__(kThreads, 1)
                     l2[(c >> 1) & 3] = f2_add(l2[(c >> 1) & 3], f2_pack(p0, p1));
                     pk[c >> 1] = pack_bf16x2(p0, p1);
                 }
-                tmem_st32(t_s + (uint32_t)(c0 / 2), pk);
+                tmem_st_cols<16>(t_s + (uint32_t)(c0 / 2), pk);
             }
             float la, lb;
             f2_unpack(f2_add(f2_add(l2[0], l2[1]), f2_add(l2[2], l2[3])), la, lb);
             l += la + lb;
             tmem_wait_st();
-            if (n >= 1 && !waited_pv) {
-                // keeps this group at most one P.V behind, so every pv_done phase is waited in turn
+            if (n >= 1) {
+                // O is final for tile n-1 (and this group stays at most one P.V behind, so every pv_done
+                // phase is waited in turn); then the rescale, before P(n) is handed to the MMA
                 mbar_wait_bounded(&pv_done[t], (uint32_t)((n - 1) & 1), a.wait_limit_ns, abort_flag, a.status);
+                if (rescale) {
+                    tc_fence_after();
+#pragma unroll 1
+                    for (int c = 0; c < DV; c += 32) {
+                        uint32_t rr[32];
+                        tmem_ld32(t_o + (uint32_t)c, rr);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) rr[e] = __float_as_uint(__uint_as_float(rr[e]) * alpha);
+                        tmem_st32(t_o + (uint32_t)c, rr);
+                    }
+                    tmem_wait_st();
+                }
             }
             tc_fence_before();
             __syncwarp();

@@ -392,12 +392,20 @@ def topv_bytes(w: wl.DecodeWorkload, seq_lens) -> int:
     return k_bytes + v_rows * w.shape.d_v * 2
 
 
+PATHS_TIMING = ("per-call CUDA events on the launch stream, median of the steps; before each call (untimed) a "
+                "256 MB buffer is written (L2 flush) and then read, so the call finds none of its inputs in L2 and "
+                "does not pay for the write-back of the flush's dirty lines")
+
+
 def _timed_calls(fn, steps: int, flush: torch.Tensor):
-    """Per-call CUDA-event times (ms) on the current stream, L2 flushed before every call."""
+    """Per-call CUDA-event times (ms) on the current stream.  Before every call, untimed: the flush
+    buffer (larger than L2) is written, which evicts the call's inputs, then read, so the dirty lines
+    the write left behind are written back before the call starts instead of during it."""
     stream = torch.cuda.current_stream()
     times = []
     for _ in range(steps):
         flush.add_(1)
+        flush.sum()
         s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         s.record(stream)
         fn()
@@ -659,6 +667,7 @@ def main():
             "gqa_control": control,
             "long_context": long_ctx,
             "paths": paths,
+            "paths_timing": PATHS_TIMING,
             "roofline": roofline,
             "cpu_baseline": cpu,
             "e2e": e2e,
