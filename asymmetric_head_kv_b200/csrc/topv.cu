@@ -858,16 +858,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncthreads();
         tc_fence_after();  // the scores the consumers stored to TMEM in phase 1
         // The part's scores, read back out of TMEM: warp w reads TMEM lanes 32 (w % 4) .. + 31 (the
-        // positions 32 (w % 4) + lane of a tile) of the tiles w / 4, w / 4 + 4, ...; f(lp, valid, s)
-        // sees position lp of the part and its QPK scores.
+        // positions 32 (w % 4) + lane of a tile), 16 columns = TPL consecutive tiles per load, the
+        // blocks of TPL tiles dealt to the four warps of a lane quarter in turn; f(lp, valid, s)
+        // sees position lp of the part and its QPK scores s[0 .. QPK).  (A part has at most
+        // kScoreCols / QPK tiles, a multiple of TPL, so no load reaches past the allocation.)
+        constexpr int TPL = 16 / QPK;
         auto for_each_score = [&](auto &&f) {
             const uint32_t t_lane = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-            for (int i = warp >> 2; i < te - tb; i += kWarps / 4) {
-                uint32_t sr[QPK];
-                tmem_ld_cols<QPK>(t_lane + (uint32_t)(kScoreCol0 + i * QPK), sr);
+            const int ntl = te - tb;
+            for (int i0 = (warp >> 2) * TPL; i0 < ntl; i0 += (kWarps / 4) * TPL) {
+                uint32_t sr[16];
+                tmem_ld_cols<16>(t_lane + (uint32_t)(kScoreCol0 + i0 * QPK), sr);
                 tmem_wait_ld();
-                const int lp = i * kTile + (warp & 3) * 32 + lane;
-                f(lp, lp < np, sr);
+#pragma unroll
+                for (int k = 0; k < TPL; ++k) {
+                    const int lp = (i0 + k) * kTile + (warp & 3) * 32 + lane;
+                    f(lp, i0 + k < ntl && lp < np, sr + k * QPK);
+                }
             }
         };
         if (a.full_weights && T > K) {
@@ -875,7 +882,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             float mx[QPK], sum[QPK];
 #pragma unroll
             for (int hh = 0; hh < QPK; ++hh) mx[hh] = -INFINITY, sum[hh] = 0.f;
-            for_each_score([&](int, bool valid, const uint32_t(&sr)[QPK]) {
+            for_each_score([&](int, bool valid, const uint32_t *sr) {
                 if (valid)
 #pragma unroll
                     for (int hh = 0; hh < QPK; ++hh) mx[hh] = fmaxf(mx[hh], __uint_as_float(sr[hh]));
@@ -891,7 +898,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncthreads();
                 mx[hh] = m;
             }
-            for_each_score([&](int, bool valid, const uint32_t(&sr)[QPK]) {
+            for_each_score([&](int, bool valid, const uint32_t *sr) {
                 if (valid)
 #pragma unroll
                     for (int hh = 0; hh < QPK; ++hh)
@@ -919,7 +926,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t cnt[QPK];
 #pragma unroll
             for (int hh = 0; hh < QPK; ++hh) cnt[hh] = 0u;
-            for_each_score([&](int, bool valid, const uint32_t(&sr)[QPK]) {
+            for_each_score([&](int, bool valid, const uint32_t *sr) {
 #pragma unroll
                 for (int hh = 0; hh < QPK; ++hh) cnt[hh] += (valid && __uint_as_float(sr[hh]) >= sh.lower[hh]) ? 1u : 0u;
             });
@@ -946,7 +953,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncthreads();
 #pragma unroll
             for (int hh = 0; hh < QPK; ++hh) slot[hh] += sh.emit_base[hh];
-            for_each_score([&](int lp, bool valid, const uint32_t(&sr)[QPK]) {
+            for_each_score([&](int lp, bool valid, const uint32_t *sr) {
 #pragma unroll
                 for (int hh = 0; hh < QPK; ++hh) {
                     const float x = __uint_as_float(sr[hh]);
@@ -1194,21 +1201,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
 
         // =============================================================== 4. gather
+        if (tid == 0) *flag = 1;
         __syncthreads();
-        if (tid == 0) {
-            bool ok = true;
-            for (int hh = 0; hh < QPK && ok; ++hh) ok = wait_at_least(a.row_sync + (size_t)(row0 + hh) * 4 + kRsSelected, 1u, a);
-            *flag = ok ? 1 : 0;
+        // thread hh waits for row hh's selection (the rows in parallel) and reads what the select wrote
+        if (tid < QPK) {
+            const int row = row0 + tid;
+            if (wait_at_least(a.row_sync + (size_t)row * 4 + kRsSelected, 1u, a)) {
+                sh.row_m[tid] = __uint_as_float(__ldcg(a.rowinfo + kRowInfoWords * row + kRiMax));
+                sh.row_nsel[tid] = (int)__ldcg(a.rowinfo + kRowInfoWords * row + kRiKept);
+                sh.row_full[tid] = __uint_as_float(__ldcg(a.rowinfo + kRowInfoWords * row + kRiFullSum));
+            } else {
+                *flag = 0;
+            }
         }
         __syncthreads();
         if (!*flag) goto finish;
-        if (tid < QPK) {
-            const int row = row0 + tid;
-            sh.row_m[tid] = __uint_as_float(__ldcg(a.rowinfo + kRowInfoWords * row + kRiMax));
-            sh.row_nsel[tid] = (int)__ldcg(a.rowinfo + kRowInfoWords * row + kRiKept);
-            sh.row_full[tid] = __uint_as_float(__ldcg(a.rowinfo + kRowInfoWords * row + kRiFullSum));
-        }
-        __syncthreads();
         {
             constexpr int WPR = kWarps / QPK;          // warps per row (every warp gathers)
             constexpr int CPV = DV / 8;                // lanes per V row
@@ -1278,11 +1285,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __stcg(a.gpart + ((size_t)(row0 + hh) * kMaxParts + j) * (DV + 4) + e, acc);
             }
             __syncthreads();
-            if (tid == 0) {
-                // release this part's sums; the last part also acquires every other part's
-                for (int hh = 0; hh < QPK; ++hh)
-                    sh.combine[hh] =
-                        atom_add_acq_rel(a.row_sync + (size_t)(row0 + hh) * 4 + kRsGathered, 1u) == (uint32_t)Y - 1;
+            if (tid < QPK) {
+                // thread hh releases this part's sums of row hh (release is cumulative over the whole
+                // CTA's writes the barrier ordered before it); the last part also acquires every other's
+                sh.combine[tid] =
+                    atom_add_acq_rel(a.row_sync + (size_t)(row0 + tid) * 4 + kRsGathered, 1u) == (uint32_t)Y - 1;
             }
             __syncthreads();
             // the last part of a row adds the Y parts in part order and writes the output
@@ -1380,7 +1387,8 @@ bool make_plan(const diffqkv_dims_t *d, int32_t t_max, int num_sms, Plan *p) {
     // the select's overlay: bitmap and word prefixes, a histogram, then candidates (at least 1024)
     const size_t sel_fixed = 2 * (t_pad / 8) + (size_t)kHistBuckets * 4;
     const size_t gather_bytes = (size_t)kWarps * (d->d_v + 4) * 4;
-    // a part's scores stay in TMEM: at most kScoreCols / qpk tiles per part
+    // a part's scores stay in TMEM: at most kScoreCols / qpk tiles per part (a multiple of the
+    // 16 / qpk tiles one phase-2 load reads)
     const int max_tiles = kScoreCols / qpk;
     int Y = std::max(1, std::min(G / std::max(1, units), nt_max));
     Y = std::max(Y, (nt_max + max_tiles - 1) / max_tiles);
