@@ -64,6 +64,13 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
     return t;
 }
 
+// max(a, b, c) in one instruction (the three-input form of max.f32, sm_100).
+__device__ __forceinline__ float fmax3f(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
 // 2^x on the SFU (ex2.approx, flush-to-zero; 2^-inf = +0).
 __device__ __forceinline__ float fast_exp2(float x) {
     float y;

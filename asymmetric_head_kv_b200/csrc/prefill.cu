@@ -243,14 +243,17 @@ __global__ void __launch_bounds__(kThreads, 2)
                 for (int c = 0; c < BN; ++c)
                     if (j0 + c > i) s[c] = -INFINITY;
             }
-            // row max as 8 independent chains (a single 64-long chain is latency-bound)
+            // row max as 8 independent chains of three-input maxima (a single 64-long chain is
+            // latency-bound; the three-input form halves the instructions)
             float mx8[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) mx8[e] = s[e];
+            for (int e = 0; e < 8; ++e) mx8[e] = fmaxf(s[e], s[8 + e]);
 #pragma unroll
-            for (int c = 8; c < BN; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
-            const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                   fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+            for (int c = 16; c < BN; c += 16)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) mx8[e] = fmax3f(mx8[e], s[c + e], s[c + 8 + e]);
+            const float mx = fmax3f(fmax3f(mx8[0], mx8[1], mx8[2]), fmax3f(mx8[3], mx8[4], mx8[5]),
+                                    fmaxf(mx8[6], mx8[7]));
             const float m_new = mx * a.scale_log2;
             bool waited_pv = false;
             if (n == 0) {
@@ -561,13 +564,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (j0 + c > i) s[c] = -INFINITY;
             }
             // row max as 8 independent chains
-            float mx8[8];
+            float mx8[8];  // three-input maxima, as in the d_k = 64 tiling
 #pragma unroll
-            for (int e = 0; e < 8; ++e) mx8[e] = s[e];
+            for (int e = 0; e < 8; ++e) mx8[e] = fmaxf(s[e], s[8 + e]);
 #pragma unroll
-            for (int c = 8; c < BN; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
-            const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                   fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+            for (int c = 16; c < BN; c += 16)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) mx8[e] = fmax3f(mx8[e], s[c + e], s[c + 8 + e]);
+            const float mx = fmax3f(fmax3f(mx8[0], mx8[1], mx8[2]), fmax3f(mx8[3], mx8[4], mx8[5]),
+                                    fmaxf(mx8[6], mx8[7]));
             const float m_new = mx * a.scale_log2;
             // the lazy O rescale is decided here and done after P is stored (the row's 128 scores are
             // dead by then; loading O next to them overran the 168 registers ten warps leave a thread)
