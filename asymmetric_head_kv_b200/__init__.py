@@ -22,7 +22,7 @@ __all__ = [
     "decode", "decode_workspace", "decode_plan", "decode_from_host", "decode_topv", "decode_topv_workspace",
     "prefill_causal", "device_status", "selftest_wait_timeout", "DiffqkvError", "Dims", "library_path",
     "decode_noalloc", "decode_append", "decode_paged", "prefill_causal_prefix", "fold_query", "workspace_status",
-    "decode_topv_paged", "augq_project",
+    "decode_topv_paged", "augq_project", "prefill_causal_paged",
 ]
 
 library_path = _capi.LIB_PATH
@@ -361,6 +361,35 @@ def prefill_causal(q, k, v, *, scale: Optional[float] = None, out=None, status: 
         st = lib().diffqkv_prefill_causal(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), S, _ptr(out),
                                           _stream_ptr(stream))
     check(st, "diffqkv_prefill_causal")
+    return out
+
+
+def prefill_causal_paged(q, k_pages, v_pages, block_table, prefix_len: int, *, scale: Optional[float] = None,
+                         out=None, status: Optional[torch.Tensor] = None,
+                         stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Causal prefill over paged K/V pools: q [B,S,n_q,d_k] for positions prefix_len..prefix_len+S-1;
+    k_pages [num_pages, page_size, n_k, d_k], v_pages [num_pages, page_size, n_v, d_v] holding every
+    sequence's prefix_len + S positions through block_table [B, max_blocks] (int32) -> [B,S,n_q,d_v]."""
+    _bf16_dev(q, "q", 4)
+    _bf16_dev(k_pages, "k_pages", 4)
+    _bf16_dev(v_pages, "v_pages", 4)
+    if block_table.dtype != torch.int32 or not block_table.is_cuda or block_table.dim() != 2 \
+            or not block_table.is_contiguous():
+        raise ValueError("block_table must be a contiguous int32 CUDA tensor [B, max_blocks]")
+    B, S, n_q, d_k = q.shape
+    num_pages, page_size, n_k, d_k2 = k_pages.shape
+    n_v, d_v = v_pages.shape[2], v_pages.shape[3]
+    if d_k2 != d_k or v_pages.shape[:2] != (num_pages, page_size) or block_table.shape[0] != B:
+        raise ValueError("q / k_pages / v_pages / block_table shapes disagree")
+    dims = make_dims(B, n_q, n_k, n_v, d_k, d_v, d_k ** -0.5 if scale is None else scale)
+    if out is None:
+        out = torch.empty((B, S, n_q, d_v), dtype=torch.bfloat16, device=q.device)
+    if status is not None:
+        _status_word(status)
+    st = lib().diffqkv_prefill_causal_paged(ctypes.byref(dims), _ptr(q), _ptr(k_pages), _ptr(v_pages),
+                                            _ptr(block_table), block_table.shape[1], page_size, num_pages,
+                                            int(prefix_len), S, _ptr(out), _ptr(status), _stream_ptr(stream))
+    check(st, "diffqkv_prefill_causal_paged")
     return out
 
 

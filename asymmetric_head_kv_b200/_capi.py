@@ -97,6 +97,7 @@ SIGNATURES = {
     "diffqkv_prefill_causal": ([_DIMS, _P, _P, _P, _I32, _P, _P], _I32),
     "diffqkv_prefill_causal_prefix": ([_DIMS, _P, _P, _P, _I32, _I32, _P, _P], _I32),
     "diffqkv_prefill_causal_ex": ([_DIMS, _P, _P, _P, _I32, _I32, _P, _P, _P], _I32),
+    "diffqkv_prefill_causal_paged": ([_DIMS, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _P, _P, _P], _I32),
     "diffqkv_augq_project": ([_P, _P, _P, _P, _I32, _I32, _I32, _I32, _P, _P, _P, _P], _I32),
     "diffqkv_workspace_status": ([_P, _SZ, _P, ctypes.POINTER(_I32)], _I32),
     "diffqkv_get_device_status": ([_P, ctypes.POINTER(_I32)], _I32),

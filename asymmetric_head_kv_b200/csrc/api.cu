@@ -99,6 +99,21 @@ diffqkv_status_t make_tensor_map_4d(CUtensorMap *map, const void *base, uint64_t
     return r == CUDA_SUCCESS ? DIFFQKV_OK : DIFFQKV_ERR_INVALID_ARG;
 }
 
+diffqkv_status_t make_tensor_map_4d_strided(CUtensorMap *map, const void *base, const uint64_t dims[4],
+                                            const uint64_t strides_bytes[3], const uint32_t box[4],
+                                            CUtensorMapSwizzle swizzle) {
+    auto fn = encode_fn();
+    if (!fn) return DIFFQKV_ERR_CUDA;
+    const cuuint64_t d[4] = {dims[0], dims[1], dims[2], dims[3]};
+    const cuuint64_t st[3] = {strides_bytes[0], strides_bytes[1], strides_bytes[2]};
+    const cuuint32_t bx[4] = {box[0], box[1], box[2], box[3]};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), d, st, bx, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? DIFFQKV_OK : DIFFQKV_ERR_INVALID_ARG;
+}
+
 diffqkv_status_t make_tensor_map_3d(CUtensorMap *map, const void *base, uint64_t dim0, uint64_t dim1,
                                     uint64_t dim2, uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box0,
                                     uint32_t box1, uint32_t box2, CUtensorMapSwizzle swizzle) {
@@ -329,6 +344,17 @@ diffqkv_status_t diffqkv_prefill_causal_ex(const diffqkv_dims_t *dims, const voi
     diffqkv::ApiRange nvtx_range("diffqkv_prefill_causal_ex");
     return diffqkv::prefill_launch(dims, q, k, v, seq_len, out, (cudaStream_t)stream, prefix_len,
                                    device_status_word);
+}
+
+diffqkv_status_t diffqkv_prefill_causal_paged(const diffqkv_dims_t *dims, const void *q, const void *k_pages,
+                                              const void *v_pages, const int32_t *block_table, int32_t max_blocks,
+                                              int32_t page_size, int32_t num_pages, int32_t prefix_len,
+                                              int32_t seq_len, void *out, int32_t *device_status_word,
+                                              diffqkv_stream_t stream) {
+    diffqkv::ApiRange nvtx_range("diffqkv_prefill_causal_paged");
+    const diffqkv::PagedCache paged{block_table, max_blocks, page_size, num_pages};
+    return diffqkv::prefill_launch(dims, q, k_pages, v_pages, seq_len, out, (cudaStream_t)stream, prefix_len,
+                                   device_status_word, &paged);
 }
 
 diffqkv_status_t diffqkv_augq_project(const void *x, const void *w_gate, const void *w_up, const void *w_down,

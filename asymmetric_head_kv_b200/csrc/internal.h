@@ -30,6 +30,11 @@ diffqkv_status_t make_tensor_map_4d(CUtensorMap *map, const void *base, uint64_t
                                     uint32_t box2, uint32_t box3, CUtensorMapSwizzle swizzle,
                                     CUtensorMapL2promotion promotion = CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
 
+// Rank-4 tiled tensor map with explicit byte strides of dims 1..3 (a view that need not be dense).
+diffqkv_status_t make_tensor_map_4d_strided(CUtensorMap *map, const void *base, const uint64_t dims[4],
+                                            const uint64_t strides_bytes[3], const uint32_t box[4],
+                                            CUtensorMapSwizzle swizzle);
+
 // Encodes a rank-3 tiled tensor map ([dim2][dim1][dim0], dim0 contiguous).
 diffqkv_status_t make_tensor_map_3d(CUtensorMap *map, const void *base, uint64_t dim0, uint64_t dim1,
                                     uint64_t dim2, uint64_t stride1_bytes, uint64_t stride2_bytes,
@@ -85,9 +90,11 @@ diffqkv_status_t topv_launch(const diffqkv_dims_t *d, const void *q, const void 
 
 // prefill.cu
 // status: device word the kernel reports into (NULL: the per-device word).
+// paged given: k / v are page pools [num_pages, page_size, heads, d] and position j of sequence b
+// is row j % page_size of pool page block_table[b][j / page_size].
 diffqkv_status_t prefill_launch(const diffqkv_dims_t *d, const void *q, const void *k, const void *v,
                                 int32_t seq_len, void *out, cudaStream_t stream, int32_t prefix_len = 0,
-                                int32_t *status = nullptr);
+                                int32_t *status = nullptr, const PagedCache *paged = nullptr);
 
 // augq.cu
 // status: device word the kernels report into (NULL: the per-device word).

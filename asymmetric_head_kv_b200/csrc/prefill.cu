@@ -23,7 +23,12 @@
 // by more than 2^8 (the stale maximum is used consistently for O and the row
 // sum, so the result is exact up to rounding).  Every mbarrier wait is bounded;
 // CTAs are ordered heaviest (most K/V tiles) first.
+//
+// K and V may also come from page pools [num_pages, page_size, heads, d] with a
+// block table (position j of sequence b is row j % page_size of pool page
+// table[b][j / page_size]); only the producer differs (paged_kv_producer).
 #include <math.h>
+#include <string.h>
 
 #include "common.cuh"
 #include "internal.h"
@@ -42,7 +47,118 @@ struct PrefillArgs {
     int32_t kv_len;  // prefix + seq: positions in K and V
     float scale_log2;
     uint64_t wait_limit_ns;
+    // paged pools (block_table NULL: contiguous [B, kv_len, heads, d] caches)
+    const int32_t *block_table;  // [batch][max_blocks]
+    int32_t max_blocks, page_size, num_pages;
+    int32_t n_pages;      // pages a sequence uses: ceil(kv_len / page_size)
+    int32_t max_box_log;  // paged boxes are 8 << i rows, i <= max_box_log (heights that divide the page)
 };
+
+constexpr int kPgTableAhead = 4;  // paged producer: tiles whose block-table entries are in flight
+constexpr int kPgTableRing = 8;   // rows of the entry ring (> kPgTableAhead)
+
+// K and V tensor maps of paged pools: k[i] / v[i] have (8 << i)-row boxes over the whole pool;
+// k_tail[i] / v_tail[i] the same boxes over a view of the pool whose pages hold only the rows of
+// a sequence's last page that carry positions, so that rows past the sequence read as zeros, as
+// the contiguous maps' rows past kv_len do (the P.V MMA multiplies them by P = 0, and 0 times a
+// stale NaN would not be 0).
+struct PagedMaps {
+    CUtensorMap k[4], v[4], k_tail[4], v_tail[4];
+};
+
+// Paged K/V producer of both tilings (all 32 lanes of the producer warp).  Tile n holds positions
+// [n BN, n BN + BN) of sequence b in stage n % STAGES of the ring (K: KB 64-column blocks of BN
+// rows, then V: VB blocks).  The tile's rows are covered greedily by aligned boxes of 8 << i rows
+// that stay inside one page; lane f issues box f.  Boxes in the sequence's last page use the tail
+// maps; boxes past it use a tail map at a row past its extent (all zeros).  The block-table
+// entries of a tile reach shared memory by asynchronous copies kPgTableAhead tiles ahead; an
+// entry outside [0, num_pages) is flagged DIFFQKV_ERR_DEVICE_PAGE and pool page 0 read instead.
+template <int BN, int KB, int VB, int STAGES, int STAGE_BYTES, int K_BYTES>
+__device__ __noinline__ void paged_kv_producer(const PagedMaps &pm, const PrefillArgs &a, int b, int kh, int vh, int n_kv,
+                                  uint8_t *kv_base, uint64_t *kv_full, uint64_t *kv_empty,
+                                  int32_t (*table)[32], volatile int *abort_flag, int lane) {
+    const int P = a.page_size;
+    const int pend = a.n_pages * P;  // positions the sequence's pages hold
+    auto first_page = [&](int t) { return (t * BN) / P; };
+    auto fetch = [&](int t) {
+        if (t < n_kv) {
+            const int last = min(a.n_pages - 1, (t * BN + BN - 1) / P);
+            if (lane <= last - first_page(t)) {
+                const int32_t *src = a.block_table + (size_t)b * a.max_blocks + first_page(t) + lane;
+                asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_addr(&table[t % kPgTableRing][lane])),
+                             "l"(src)
+                             : "memory");
+            }
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    for (int i = 0; i < kPgTableAhead; ++i) fetch(i);
+    int issued = 0;
+    for (int n = 0; n < n_kv; ++n) {
+        fetch(n + kPgTableAhead);
+        const int st = n % STAGES;
+        if (n >= STAGES)
+            mbar_wait_bounded(&kv_empty[st], (uint32_t)(((n / STAGES) - 1) & 1), a.wait_limit_ns, abort_flag, a.status);
+        if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
+        asm volatile("cp.async.wait_group %0;" ::"n"(kPgTableAhead) : "memory");  // tile n's entries
+        const int my_e = table[n % kPgTableRing][lane];
+        // every lane walks the same decomposition and keeps box `lane`
+        const int start = n * BN, end = start + BN;
+        int cur = start, f = 0, my_cur = -1, my_hi = 0;
+        while (cur < end) {
+            const int seg_end = cur < pend ? min(end, (cur / P + 1) * P) : end;
+            int hi = a.max_box_log;
+            while (hi > 0 && ((cur & ((8 << hi) - 1)) != 0 || cur + (8 << hi) > seg_end)) --hi;
+            if (f == lane) {
+                my_cur = cur;
+                my_hi = hi;
+            }
+            cur += 8 << hi;
+            ++f;
+        }
+        uint8_t *kdst = kv_base + st * STAGE_BYTES;
+        uint8_t *vdst = kdst + K_BYTES;
+        if (lane == 0) mbar_arrive_expect_tx(&kv_full[st], STAGE_BYTES);
+        __syncwarp();
+        const bool in_seq = my_cur >= 0 && my_cur < pend;
+        const int pidx = in_seq ? my_cur / P : 0;
+        int page = __shfl_sync(0xffffffffu, my_e, in_seq ? pidx - first_page(n) : 0);
+        if (my_cur >= 0) {
+            int row = P;        // past the sequence's pages: a row past the tail view's extent
+            bool tail = true;
+            if (in_seq) {
+                if (page < 0 || page >= a.num_pages) {
+                    record_error(a.status, DIFFQKV_ERR_DEVICE_PAGE);
+                    page = 0;
+                }
+                row = my_cur % P;
+                tail = pidx == a.n_pages - 1;
+            } else {
+                page = 0;
+            }
+            // constant indices keep the descriptors in the kernel's parameter space
+            const CUtensorMap *km, *vm;
+            if (tail) {
+                km = my_hi == 0 ? &pm.k_tail[0] : my_hi == 1 ? &pm.k_tail[1] : my_hi == 2 ? &pm.k_tail[2] : &pm.k_tail[3];
+                vm = my_hi == 0 ? &pm.v_tail[0] : my_hi == 1 ? &pm.v_tail[1] : my_hi == 2 ? &pm.v_tail[2] : &pm.v_tail[3];
+            } else {
+                km = my_hi == 0 ? &pm.k[0] : my_hi == 1 ? &pm.k[1] : my_hi == 2 ? &pm.k[2] : &pm.k[3];
+                vm = my_hi == 0 ? &pm.v[0] : my_hi == 1 ? &pm.v[1] : my_hi == 2 ? &pm.v[2] : &pm.v[3];
+            }
+            const int off = (my_cur - start) * 128;
+#pragma unroll
+            for (int kb = 0; kb < KB; ++kb) tma_load_4d(kdst + kb * (BN * 128) + off, km, &kv_full[st], kb * 64, kh, row, page);
+#pragma unroll
+            for (int vb = 0; vb < VB; ++vb) tma_load_4d(vdst + vb * (BN * 128) + off, vm, &kv_full[st], vb * 64, vh, row, page);
+        }
+        issued = n + 1;
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");  // no entry copy outlives the loop
+    // drain: no copy may still be landing when the CTA exits
+    if (lane == 0)
+        for (int n = (issued > STAGES ? issued - STAGES : 0); n < issued; ++n)
+            mbar_wait_bounded(&kv_full[n % STAGES], (uint32_t)((n / STAGES) & 1), a.wait_limit_ns, nullptr, a.status);
+}
 
 // ---------------------------------------------------------------- d_k = 64
 // warps 0-3 softmax (thread t owns query row t = TMEM lane t), warp 4 TMA
@@ -75,7 +191,8 @@ struct Cfg {
 template <int DK, int DV>
 __global__ void __launch_bounds__(kThreads, 2)
     prefill_causal_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                          const __grid_constant__ CUtensorMap tm_v, const PrefillArgs a) {
+                          const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ PagedMaps pm,
+                          const PrefillArgs a) {
     using C = Cfg<DK, DV>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -133,14 +250,22 @@ __global__ void __launch_bounds__(kThreads, 2)
 
     if (warp == kProducerWarp) {
         // ======================= TMA producer
+        __shared__ int32_t pg_table[kPgTableRing][32];  // paged: block-table entries of the tiles ahead
         if (lane == 0) {
             prefetch_tensormap(&tm_q);
-            prefetch_tensormap(&tm_k);
-            prefetch_tensormap(&tm_v);
             mbar_arrive_expect_tx(q_full, C::Q_BYTES);
 #pragma unroll
             for (int kb = 0; kb < C::KB; ++kb)
                 tma_load_4d(smem + C::OFF_Q + kb * (BM * 128), &tm_q, q_full, kb * 64, h, row0, b);
+        }
+        if (a.block_table) {
+            __syncwarp();
+            paged_kv_producer<BN, C::KB, C::VB, C::STAGES, C::STAGE_BYTES, C::K_BYTES>(
+                pm, a, b, kh, vh, n_kv, smem + C::OFF_KV, kv_full, kv_empty, pg_table, abort_flag, lane);
+            if (lane == 0) mbar_wait_bounded(q_full, 0, a.wait_limit_ns, nullptr, a.status);
+        } else if (lane == 0) {
+            prefetch_tensormap(&tm_k);
+            prefetch_tensormap(&tm_v);
             for (int n = 0; n < n_kv; ++n) {
                 const int st = n % C::STAGES;
                 if (n >= C::STAGES)
@@ -383,7 +508,8 @@ struct Cfg {
 template <int DK, int DV>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_causal_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                          const __grid_constant__ CUtensorMap tm_v, const PrefillArgs a) {
+                          const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ PagedMaps pm,
+                          const PrefillArgs a) {
     using C = Cfg<DK, DV>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -444,10 +570,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp == kProducerWarp) {
         // ======================= TMA producer
+        __shared__ int32_t pg_table[kPgTableRing][32];  // paged: block-table entries of the tiles ahead
         if (lane == 0) {
             prefetch_tensormap(&tm_q);
-            prefetch_tensormap(&tm_k);
-            prefetch_tensormap(&tm_v);
             mbar_arrive_expect_tx(q_full, QT * C::Q_BYTES);
 #pragma unroll
             for (int t = 0; t < QT; ++t)
@@ -455,6 +580,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int kb = 0; kb < C::KB; ++kb)
                     tma_load_4d(smem + C::OFF_Q + t * C::Q_BYTES + kb * (BM * 128), &tm_q, q_full, kb * 64, h,
                                 row0 + t * BM, b);
+        }
+        if (a.block_table) {
+            __syncwarp();
+            paged_kv_producer<BN, C::KB, C::VB, C::STAGES, C::STAGE_BYTES, C::K_BYTES>(
+                pm, a, b, kh, vh, n_kv_all, smem + C::OFF_KV, kv_full, kv_empty, pg_table, abort_flag, lane);
+            if (lane == 0) mbar_wait_bounded(q_full, 0, a.wait_limit_ns, nullptr, a.status);
+        } else if (lane == 0) {
+            prefetch_tensormap(&tm_k);
+            prefetch_tensormap(&tm_v);
             for (int n = 0; n < n_kv_all; ++n) {
                 const int st = n % C::STAGES;
                 if (n >= C::STAGES)
@@ -672,7 +806,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace pair128
 
-using PrefillFn = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, PrefillArgs);
+using PrefillFn = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, PagedMaps, PrefillArgs);
 
 struct Plan {
     PrefillFn fn;
@@ -703,7 +837,8 @@ bool pick(int dk, int dv, Plan *p) {
 }  // namespace
 
 diffqkv_status_t prefill_launch(const diffqkv_dims_t *d, const void *q, const void *k, const void *v, int32_t seq_len,
-                                void *out, cudaStream_t stream, int32_t prefix_len, int32_t *status) {
+                                void *out, cudaStream_t stream, int32_t prefix_len, int32_t *status,
+                                const PagedCache *paged) {
     diffqkv_status_t st = validate_dims(d);
     if (st != DIFFQKV_OK) return st;
     if (!q || !k || !v || !out || seq_len < 1 || prefix_len < 0) return DIFFQKV_ERR_INVALID_ARG;
@@ -714,20 +849,64 @@ diffqkv_status_t prefill_launch(const diffqkv_dims_t *d, const void *q, const vo
         return DIFFQKV_ERR_MISALIGNED;
     Plan plan;
     if (!pick(d->d_k, d->d_v, &plan)) return DIFFQKV_ERR_UNSUPPORTED;
+    int32_t n_pages = 0, max_box_log = 0;
+    if (paged) {
+        const long long P = paged->page_size;
+        if (!paged->block_table || paged->max_blocks < 1 || P < 1 || paged->num_pages < 1)
+            return DIFFQKV_ERR_INVALID_ARG;
+        if (reinterpret_cast<uintptr_t>(paged->block_table) & 3u) return DIFFQKV_ERR_MISALIGNED;
+        // boxes of at least 8 rows keep every box on a 1024-byte swizzle atom of the tile
+        if (P % 8 != 0) return DIFFQKV_ERR_UNSUPPORTED;
+        n_pages = (int32_t)((kv_len + P - 1) / P);
+        if (n_pages > paged->max_blocks) return DIFFQKV_ERR_INVALID_ARG;
+        if ((long long)paged->num_pages * P > 0x7fffffffLL ||
+            (long long)d->batch * paged->max_blocks > 0x7fffffffLL)
+            return DIFFQKV_ERR_UNSUPPORTED;
+        while (max_box_log < 3 && P % (8 << (max_box_log + 1)) == 0 && (8 << (max_box_log + 1)) <= plan.kv_box)
+            ++max_box_log;
+    }
     DeviceInfo dev;
     st = current_device_info(&dev);
     if (st != DIFFQKV_OK) return st;
 
     CUtensorMap tm_q, tm_k, tm_v;
+    PagedMaps pm;
+    memset(&pm, 0, sizeof(pm));
     st = make_tensor_map_4d(&tm_q, q, d->d_k, d->n_q, seq_len, d->batch, 64, 1, plan.q_box, 1,
                             CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != DIFFQKV_OK) return st;
-    st = make_tensor_map_4d(&tm_k, k, d->d_k, d->n_k, kv_len, d->batch, 64, 1, plan.kv_box, 1,
-                            CU_TENSOR_MAP_SWIZZLE_128B);
-    if (st != DIFFQKV_OK) return st;
-    st = make_tensor_map_4d(&tm_v, v, d->d_v, d->n_v, kv_len, d->batch, 64, 1, plan.kv_box, 1,
-                            CU_TENSOR_MAP_SWIZZLE_128B);
-    if (st != DIFFQKV_OK) return st;
+    if (!paged) {
+        st = make_tensor_map_4d(&tm_k, k, d->d_k, d->n_k, kv_len, d->batch, 64, 1, plan.kv_box, 1,
+                                CU_TENSOR_MAP_SWIZZLE_128B);
+        if (st != DIFFQKV_OK) return st;
+        st = make_tensor_map_4d(&tm_v, v, d->d_v, d->n_v, kv_len, d->batch, 64, 1, plan.kv_box, 1,
+                                CU_TENSOR_MAP_SWIZZLE_128B);
+        if (st != DIFFQKV_OK) return st;
+    } else {
+        // whole-pool maps with boxes of 8 << i rows, and the tail views: the same pages with only the
+        // rows of the last page that hold positions (the rest of a box there reads as zeros)
+        const uint64_t P = (uint64_t)paged->page_size;
+        const uint64_t last_rows = (uint64_t)kv_len - (uint64_t)(n_pages - 1) * P;
+        for (int i = 0; i < 4; ++i) {
+            const int hi = i <= max_box_log ? i : 0;
+            const uint32_t rows = 8u << hi;
+            st = make_tensor_map_4d(&pm.k[i], k, d->d_k, d->n_k, P, paged->num_pages, 64, 1, rows, 1,
+                                    CU_TENSOR_MAP_SWIZZLE_128B);
+            if (st == DIFFQKV_OK)
+                st = make_tensor_map_4d(&pm.v[i], v, d->d_v, d->n_v, P, paged->num_pages, 64, 1, rows, 1,
+                                        CU_TENSOR_MAP_SWIZZLE_128B);
+            const uint64_t kd[4] = {(uint64_t)d->d_k, (uint64_t)d->n_k, last_rows, (uint64_t)paged->num_pages};
+            const uint64_t ks[3] = {(uint64_t)d->d_k * 2, (uint64_t)d->d_k * d->n_k * 2, (uint64_t)d->d_k * d->n_k * P * 2};
+            const uint64_t vd[4] = {(uint64_t)d->d_v, (uint64_t)d->n_v, last_rows, (uint64_t)paged->num_pages};
+            const uint64_t vs[3] = {(uint64_t)d->d_v * 2, (uint64_t)d->d_v * d->n_v * 2, (uint64_t)d->d_v * d->n_v * P * 2};
+            const uint32_t box[4] = {64, 1, rows, 1};
+            if (st == DIFFQKV_OK) st = make_tensor_map_4d_strided(&pm.k_tail[i], k, kd, ks, box, CU_TENSOR_MAP_SWIZZLE_128B);
+            if (st == DIFFQKV_OK) st = make_tensor_map_4d_strided(&pm.v_tail[i], v, vd, vs, box, CU_TENSOR_MAP_SWIZZLE_128B);
+            if (st != DIFFQKV_OK) return st;
+        }
+        tm_k = pm.k[0];
+        tm_v = pm.v[0];
+    }
 
     PrefillArgs a;
     a.out = static_cast<__nv_bfloat16 *>(out);
@@ -744,10 +923,16 @@ diffqkv_status_t prefill_launch(const diffqkv_dims_t *d, const void *q, const vo
     a.n_ctas_per_head = (seq_len + plan.rows_per_cta - 1) / plan.rows_per_cta;
     a.scale_log2 = (float)((double)d->scale * 1.4426950408889634);
     a.wait_limit_ns = kWaitLimitNs;
+    a.block_table = paged ? paged->block_table : nullptr;
+    a.max_blocks = paged ? paged->max_blocks : 0;
+    a.page_size = paged ? paged->page_size : 0;
+    a.num_pages = paged ? paged->num_pages : 0;
+    a.n_pages = n_pages;
+    a.max_box_log = max_box_log;
     const long long grid = (long long)a.n_ctas_per_head * d->batch * d->n_q;
     if (grid > 0x7fffffffLL) return DIFFQKV_ERR_UNSUPPORTED;
     if (ensure_dynamic_smem((const void *)plan.fn, plan.smem) != DIFFQKV_OK) return DIFFQKV_ERR_CUDA;
-    plan.fn<<<(unsigned)grid, plan.threads, plan.smem, stream>>>(tm_q, tm_k, tm_v, a);
+    plan.fn<<<(unsigned)grid, plan.threads, plan.smem, stream>>>(tm_q, tm_k, tm_v, pm, a);
     if (cudaGetLastError() != cudaSuccess) return DIFFQKV_ERR_CUDA;
     return DIFFQKV_OK;
 }

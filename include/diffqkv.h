@@ -29,8 +29,9 @@
  *      - calls that take a workspace (decode, its variants, top-v): the
  *        workspace's first 32-bit word, read and cleared by
  *        diffqkv_workspace_status;
- *      - diffqkv_prefill_causal_ex, diffqkv_augq_project: the word the caller
- *        passes (NULL: the per-device word);
+ *      - diffqkv_prefill_causal_ex, diffqkv_prefill_causal_paged,
+ *        diffqkv_augq_project: the word the caller passes (NULL: the
+ *        per-device word);
  *      - every other call (prefill without a word, diffqkv_decode_noalloc,
  *        the wait self-test): the per-device word, read and cleared by
  *        diffqkv_get_device_status.
@@ -432,6 +433,32 @@ diffqkv_status_t diffqkv_prefill_causal_prefix(const diffqkv_dims_t *dims, const
 diffqkv_status_t diffqkv_prefill_causal_ex(const diffqkv_dims_t *dims, const void *q, const void *k,
                                            const void *v, int32_t prefix_len, int32_t seq_len, void *out,
                                            int32_t *device_status_word, diffqkv_stream_t stream);
+
+/*
+ * diffqkv_prefill_causal_ex over paged K/V pools (chunked prefill whose prefix
+ * sits in a paged cache, the layout of diffqkv_decode_paged):
+ *   q        [B, seq_len, n_q, d_k]                  the new rows' queries
+ *   k_pages  [num_pages, page_size, n_k, d_k]        K pool
+ *   v_pages  [num_pages, page_size, n_v, d_v]        V pool
+ *   block_table [B, max_blocks] int32 (device): position j of sequence b is
+ *            row j % page_size of pool page block_table[b][j / page_size]
+ *   out      [B, seq_len, n_q, d_v]
+ * Every sequence holds prefix_len + seq_len positions, the new rows' k and v
+ * included (written into their pages by the caller beforehand); query row r
+ * sits at position prefix_len + r and attends to positions 0 .. prefix_len + r.
+ * Only the first ceil((prefix_len + seq_len) / page_size) table entries of a
+ * sequence are read; an entry outside [0, num_pages) is flagged
+ * DIFFQKV_ERR_DEVICE_PAGE in the call's word and pool page 0 is read instead.
+ * page_size a multiple of 8 (else DIFFQKV_ERR_UNSUPPORTED); max_blocks *
+ * page_size >= prefix_len + seq_len (else DIFFQKV_ERR_INVALID_ARG); the table
+ * 4-byte aligned.  The result equals diffqkv_prefill_causal_ex on contiguous
+ * caches holding the same rows, bit for bit.  device_status_word as there.
+ */
+diffqkv_status_t diffqkv_prefill_causal_paged(const diffqkv_dims_t *dims, const void *q, const void *k_pages,
+                                              const void *v_pages, const int32_t *block_table, int32_t max_blocks,
+                                              int32_t page_size, int32_t num_pages, int32_t prefix_len,
+                                              int32_t seq_len, void *out, int32_t *device_status_word,
+                                              diffqkv_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
 /* Device error word                                                        */

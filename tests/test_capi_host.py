@@ -351,3 +351,20 @@ def test_augq_project_rejects_before_launch():
     assert call(tokens=0) == _capi.OK                     # nothing to do
     assert call(tokens=0, x=None, h=None, q=None) == _capi.OK  # empty tensors have no storage
     assert call(tokens=0, wg=None) == _capi.INVALID_ARG
+
+
+def test_prefill_causal_paged_rejects_before_launch():
+    lib = _capi.lib()
+    d = dims(batch=2)
+
+    def call(bt=0x7000, max_blocks=8, page_size=16, num_pages=10, prefix=64, seq=64, status=None):
+        return lib.diffqkv_prefill_causal_paged(ctypes.byref(d), 0x1000, 0x2000, 0x3000, bt, max_blocks, page_size,
+                                                num_pages, prefix, seq, 0x5000, status, None)
+    assert call(bt=None) == _capi.INVALID_ARG
+    assert call(bt=0x7002) == _capi.MISALIGNED
+    assert call(page_size=12) == _capi.UNSUPPORTED        # boxes need whole 8-row swizzle atoms
+    assert call(max_blocks=7) == _capi.INVALID_ARG        # 128 positions need 8 pages of 16
+    assert call(num_pages=0) == _capi.INVALID_ARG
+    assert call(seq=0) == _capi.INVALID_ARG
+    assert call(prefix=-1) == _capi.INVALID_ARG
+    assert call(status=0x6002) == _capi.MISALIGNED
