@@ -213,7 +213,7 @@ const char *diffqkv_status_string(int32_t status) {
     }
 }
 
-int32_t diffqkv_version(void) { return 10100; }
+int32_t diffqkv_version(void) { return 10200; }
 
 size_t diffqkv_decode_workspace_size(const diffqkv_dims_t *dims) { return diffqkv::decode_workspace_size(dims); }
 

@@ -448,7 +448,26 @@ def time_paths(ak, peaks, steps: int, warmup: int):
     res["prefill_prefix_b2_p8192_s2048"] = {"ms": ms, "causal_flops": flops, "tflops": tf, "bound": "tensor",
                                             "peak_tflops": bf16_peak, "frac": tf / bf16_peak,
                                             "peak_source": "bf16_tflops (burst, cuBLAS bf16 GEMM)"}
-    del d, qn, out
+    # the same chunked prefill with K and V in 16-position pages dealt out in random order
+    page = 16
+    per_seq = (P + S + page - 1) // page
+    g = torch.Generator().manual_seed(w.seed + 7)
+    perm = torch.randperm(w.batch * per_seq, generator=g).to(torch.int32).view(w.batch, per_seq)
+    table = perm.to(dev).contiguous()
+    kp = torch.empty((w.batch * per_seq, page, w.shape.n_k, w.shape.d_k), dtype=torch.bfloat16, device=dev)
+    vp = torch.empty((w.batch * per_seq, page, w.shape.n_v, w.shape.d_v), dtype=torch.bfloat16, device=dev)
+    kp[table.long().view(-1)] = d["k"].view(w.batch * per_seq, page, w.shape.n_k, w.shape.d_k)
+    vp[table.long().view(-1)] = d["v"].view(w.batch * per_seq, page, w.shape.n_v, w.shape.d_v)
+    fn = lambda: ak.prefill_causal_paged(qn, kp, vp, table, P, scale=d["scale"], out=out)  # noqa: E731
+    for _ in range(max(3, warmup)):
+        fn()
+    ms = statistics.median(_timed_calls(fn, steps, flush))
+    tf = flops / (ms * 1e-3) / 1e12
+    res["prefill_prefix_paged_b2_p8192_s2048_page16"] = {
+        "ms": ms, "causal_flops": flops, "tflops": tf, "bound": "tensor", "peak_tflops": bf16_peak,
+        "frac": tf / bf16_peak, "peak_source": "bf16_tflops (burst, cuBLAS bf16 GEMM)"}
+    assert ak.device_status() == 0
+    del d, qn, out, kp, vp, table
 
     # the small decode case (batch 1, 512 positions: 2.36 MB, launch/latency bound): microseconds
     # per call with L2 flushed before each call
