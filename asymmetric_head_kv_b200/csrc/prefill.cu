@@ -52,6 +52,7 @@ struct PrefillArgs {
     int32_t max_blocks, page_size, num_pages;
     int32_t n_pages;      // pages a sequence uses: ceil(kv_len / page_size)
     int32_t max_box_log;  // paged boxes are 8 << i rows, i <= max_box_log (heights that divide the page)
+    int32_t page_shift;   // log2(page_size) when it is a power of two, else -1
 };
 
 constexpr int kPgTableAhead = 4;  // paged producer: tiles whose block-table entries are in flight
@@ -79,10 +80,15 @@ __device__ __noinline__ void paged_kv_producer(const PagedMaps &pm, const Prefil
                                   int32_t (*table)[32], volatile int *abort_flag, int lane) {
     const int P = a.page_size;
     const int pend = a.n_pages * P;  // positions the sequence's pages hold
-    auto first_page = [&](int t) { return (t * BN) / P; };
+    // position -> page and row in page: shifts for power-of-two pages (a runtime division is dozens
+    // of instructions, and this warp shares its sub-partition with softmax warps)
+    const int ps = a.page_shift;
+    auto pdiv = [&](int x) { return ps >= 0 ? x >> ps : x / P; };
+    auto pmod = [&](int x) { return ps >= 0 ? x & (P - 1) : x % P; };
+    auto first_page = [&](int t) { return pdiv(t * BN); };
     auto fetch = [&](int t) {
         if (t < n_kv) {
-            const int last = min(a.n_pages - 1, (t * BN + BN - 1) / P);
+            const int last = min(a.n_pages - 1, pdiv(t * BN + BN - 1));
             if (lane <= last - first_page(t)) {
                 const int32_t *src = a.block_table + (size_t)b * a.max_blocks + first_page(t) + lane;
                 asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_addr(&table[t % kPgTableRing][lane])),
@@ -102,26 +108,33 @@ __device__ __noinline__ void paged_kv_producer(const PagedMaps &pm, const Prefil
         if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
         asm volatile("cp.async.wait_group %0;" ::"n"(kPgTableAhead) : "memory");  // tile n's entries
         const int my_e = table[n % kPgTableRing][lane];
-        // every lane walks the same decomposition and keeps box `lane`
         const int start = n * BN, end = start + BN;
-        int cur = start, f = 0, my_cur = -1, my_hi = 0;
-        while (cur < end) {
-            const int seg_end = cur < pend ? min(end, (cur / P + 1) * P) : end;
-            int hi = a.max_box_log;
-            while (hi > 0 && ((cur & ((8 << hi) - 1)) != 0 || cur + (8 << hi) > seg_end)) --hi;
-            if (f == lane) {
-                my_cur = cur;
-                my_hi = hi;
+        int my_cur = -1, my_hi = a.max_box_log;
+        if (ps >= 0) {
+            // power-of-two pages: every box is 8 << max_box_log rows (the page, or 64 rows of it)
+            const int rows = 8 << a.max_box_log;
+            if (lane < BN / rows) my_cur = start + lane * rows;
+        } else {
+            // every lane walks the same greedy decomposition and keeps box `lane`
+            int cur = start, f = 0;
+            while (cur < end) {
+                const int seg_end = cur < pend ? min(end, (pdiv(cur) + 1) * P) : end;
+                int hi = a.max_box_log;
+                while (hi > 0 && ((cur & ((8 << hi) - 1)) != 0 || cur + (8 << hi) > seg_end)) --hi;
+                if (f == lane) {
+                    my_cur = cur;
+                    my_hi = hi;
+                }
+                cur += 8 << hi;
+                ++f;
             }
-            cur += 8 << hi;
-            ++f;
         }
         uint8_t *kdst = kv_base + st * STAGE_BYTES;
         uint8_t *vdst = kdst + K_BYTES;
         if (lane == 0) mbar_arrive_expect_tx(&kv_full[st], STAGE_BYTES);
         __syncwarp();
         const bool in_seq = my_cur >= 0 && my_cur < pend;
-        const int pidx = in_seq ? my_cur / P : 0;
+        const int pidx = in_seq ? pdiv(my_cur) : 0;
         int page = __shfl_sync(0xffffffffu, my_e, in_seq ? pidx - first_page(n) : 0);
         if (my_cur >= 0) {
             int row = P;        // past the sequence's pages: a row past the tail view's extent
@@ -131,7 +144,7 @@ __device__ __noinline__ void paged_kv_producer(const PagedMaps &pm, const Prefil
                     record_error(a.status, DIFFQKV_ERR_DEVICE_PAGE);
                     page = 0;
                 }
-                row = my_cur % P;
+                row = pmod(my_cur);
                 tail = pidx == a.n_pages - 1;
             } else {
                 page = 0;
@@ -929,6 +942,11 @@ diffqkv_status_t prefill_launch(const diffqkv_dims_t *d, const void *q, const vo
     a.num_pages = paged ? paged->num_pages : 0;
     a.n_pages = n_pages;
     a.max_box_log = max_box_log;
+    a.page_shift = -1;
+    if (paged && (paged->page_size & (paged->page_size - 1)) == 0) {
+        a.page_shift = 0;
+        while ((1 << a.page_shift) < paged->page_size) ++a.page_shift;
+    }
     const long long grid = (long long)a.n_ctas_per_head * d->batch * d->n_q;
     if (grid > 0x7fffffffLL) return DIFFQKV_ERR_UNSUPPORTED;
     if (ensure_dynamic_smem((const void *)plan.fn, plan.smem) != DIFFQKV_OK) return DIFFQKV_ERR_CUDA;

@@ -127,6 +127,7 @@ struct TopvArgs {
     int32_t max_blocks, page_size, num_pages;
     int32_t max_box_log;  // paged: boxes of 8 << i rows, i <= max_box_log, divide the page size
     int32_t tile_box;     // paged, page size a multiple of kTile: one kTile-row box per tile (m[0])
+    int32_t page_shift;   // paged: log2(page_size) when it is a power of two, else -1
     long long cache_rows; // rows of the K / V caches or pools
     float scale_log2;
     uint64_t wait_limit_ns;
@@ -603,10 +604,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncwarp();
                 const long long k0 = ring_k;
                 auto covered = [&](int t) { return (min(kTile, T - t * kTile) + 7) & ~7; };  // rows loaded
-                auto first_page = [&](int t) { return (t * kTile) / a.page_size; };
+                // position -> page and row: shifts for power-of-two pages (a runtime division is dozens
+                // of instructions, and this warp shares its sub-partition with consumer warps)
+                const int ps = a.page_shift;
+                auto pdiv = [&](int x) { return ps >= 0 ? x >> ps : x / a.page_size; };
+                auto pmod = [&](int x) { return ps >= 0 ? x & (a.page_size - 1) : x % a.page_size; };
+                auto first_page = [&](int t) { return pdiv(t * kTile); };
                 auto fetch = [&](int t) {
                     if (t < te) {
-                        const int np = (t * kTile + covered(t) - 1) / a.page_size - first_page(t) + 1;
+                        const int np = pdiv(t * kTile + covered(t) - 1) - first_page(t) + 1;
                         if (lane < np) {
                             const int32_t *src = a.block_table + (size_t)b * a.max_blocks + first_page(t) + lane;
                             asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(
@@ -628,10 +634,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
                     asm volatile("cp.async.wait_group %0;" ::"n"(kTableAhead) : "memory");  // tile t's entries
                     const int cur_e = sh.table[t % kTableRing][lane];  // this lane's own copy
-                    // every lane walks the same decomposition and keeps box `lane`
                     const int start = t * kTile, end = start + (a.tile_box ? kTile : covered(t));
                     int cur = a.tile_box ? end : start, f = 0, my_cur = -1, my_hi = 0;
                     if (a.tile_box && lane == 0) my_cur = start;
+                    if (!a.tile_box && ps >= 0 && end - start == kTile) {
+                        // a full tile over power-of-two pages: every box is 8 << max_box_log rows
+                        const int rows = 8 << a.max_box_log;
+                        if (lane < kTile / rows) {
+                            my_cur = start + lane * rows;
+                            my_hi = a.max_box_log;
+                        }
+                        cur = end;
+                    }
+                    // otherwise every lane walks the same greedy decomposition and keeps box `lane`
                     while (cur < end) {
                         int hi = a.max_box_log;
                         while (hi > 0 && ((cur & ((8 << hi) - 1)) != 0 || cur + (8 << hi) > end)) --hi;
@@ -645,7 +660,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     uint8_t *dst = ring + (size_t)st * TILE_BYTES;
                     if (lane == 0) mbar_arrive_expect_tx(&full_bar[st], (uint32_t)((end - start) * DK * 2));
                     __syncwarp();
-                    int page = __shfl_sync(0xffffffffu, cur_e, my_cur >= 0 ? my_cur / a.page_size - first_page(t) : 0);
+                    int page = __shfl_sync(0xffffffffu, cur_e, my_cur >= 0 ? pdiv(my_cur) - first_page(t) : 0);
                     if (my_cur >= 0) {
                         if (page < 0 || page >= a.num_pages) {  // flagged; pool page 0 read in its place
                             record_error(a.status, DIFFQKV_ERR_DEVICE_PAGE);
@@ -659,7 +674,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int kb = 0; kb < DK / 64; ++kb)
                             tma_load_4d(dst + kb * (kTile * 128) + (my_cur - start) * 128, tm, &full_bar[st], kb * 64,
-                                        g, my_cur % a.page_size, page);
+                                        g, pmod(my_cur), page);
                     }
                     issued_end = k0 + (t - tb) + 1;
                     if (++st == a.stages) {
@@ -1535,6 +1550,11 @@ diffqkv_status_t topv_launch(const diffqkv_dims_t *d, const void *q, const void 
     memset(&maps, 0, sizeof maps);
     const bool tile_box = paged && paged->page_size % kTile == 0;
     a.tile_box = tile_box ? 1 : 0;
+    a.page_shift = -1;
+    if (paged && (paged->page_size & (paged->page_size - 1)) == 0) {
+        a.page_shift = 0;
+        while ((1 << a.page_shift) < paged->page_size) ++a.page_shift;
+    }
     if (tile_box) {
         st = make_tensor_map_4d(&maps.m[0], k_cache, d->d_k, d->n_k, paged->page_size, paged->num_pages, 64, 1,
                                 kTile, 1, CU_TENSOR_MAP_SWIZZLE_128B);
