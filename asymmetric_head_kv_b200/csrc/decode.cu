@@ -79,6 +79,7 @@ struct DecodeArgs {
     const int32_t *block_table = nullptr;  // [B, max_blocks] pool page of each logical page
     int32_t max_blocks = 0, page_size = 0, num_pages = 0;
     int32_t sub_rows = 0;                  // positions per sub-box (divides the tile and the page)
+    int32_t sub_shift = -1, page_shift = -1;  // log2 of sub_rows / page_size when powers of two, else -1
     long long partial_slots = 0;           // split-partial records the scratch holds
     long long store_rows = 0;              // rows of the K / V caches or pools (append stores)
     uint32_t sub_k_bytes = 0, sub_v_bytes = 0;
@@ -140,16 +141,28 @@ __device__ __forceinline__ long long cta_of_tile(long long t, long long N, long 
     return ((t + 1) * G - 1) / N;
 }
 
+// x / sub_rows, x / page_size and x % page_size: shifts when they are powers of two (the producer
+// warp shares its sub-partition with consumers, and a runtime division is dozens of instructions).
+__device__ __forceinline__ int div_sub(const DecodeArgs &a, int x) {
+    return a.sub_shift >= 0 ? x >> a.sub_shift : x / a.sub_rows;
+}
+__device__ __forceinline__ int div_page(const DecodeArgs &a, int x) {
+    return a.page_shift >= 0 ? x >> a.page_shift : x / a.page_size;
+}
+__device__ __forceinline__ int mod_page(const DecodeArgs &a, int x) {
+    return a.page_shift >= 0 ? x & (a.page_size - 1) : x % a.page_size;
+}
+
 // Sub-boxes holding the valid positions of the walker's current tile (paged caches).
 template <int TT>
 __device__ __forceinline__ int sub_boxes(const DecodeArgs &a, const Walker &w) {
-    return (min(TT, w.T - w.i * TT) + a.sub_rows - 1) / a.sub_rows;
+    return div_sub(a, min(TT, w.T - w.i * TT) + a.sub_rows - 1);
 }
 
 // Block-table entry of sub-box f of the walker's current tile, 0 when f is past its sub-boxes.
 template <int TT>
 __device__ __forceinline__ int sub_box_entry(const DecodeArgs &a, const Walker &w, int f) {
-    return f < sub_boxes<TT>(a, w) ? page_entry(a, w.b, (w.i * TT + f * a.sub_rows) / a.page_size) : 0;
+    return f < sub_boxes<TT>(a, w) ? page_entry(a, w.b, div_page(a, w.i * TT + f * a.sub_rows)) : 0;
 }
 
 // Producer for paged caches, run by the whole producer warp.  Lane f issues the K and V loads of
@@ -177,9 +190,9 @@ __device__ long long produce_paged(const CUtensorMap *tm_k, const CUtensorMap *t
         const int v0 = (w.g * QPK) / a.q_per_v;
         for (int f = lane; f < n_sub; f += 32) {
             // a bad entry (flagged) loads pool page 0 instead: the loads stay in bounds
-            const int entry = f == lane ? cur : page_entry(a, w.b, (w.i * TT + f * a.sub_rows) / a.page_size);
+            const int entry = f == lane ? cur : page_entry(a, w.b, div_page(a, w.i * TT + f * a.sub_rows));
             const int page = max(checked_page(a, entry), 0);
-            const int row = (w.i * TT + f * a.sub_rows) % a.page_size;
+            const int row = mod_page(a, w.i * TT + f * a.sub_rows);
             tma_load_4d(sb + (size_t)f * a.sub_k_bytes, tm_k, &full_bar[stage], 0, w.g, row, page);
             tma_load_4d(sb + a.k_tile_bytes + (size_t)f * a.sub_v_bytes, tm_v, &full_bar[stage], 0, v0, row, page);
         }
@@ -864,6 +877,14 @@ diffqkv_status_t decode_prepare(const diffqkv_dims_t *d, const void *q, const vo
         a.page_size = paged->page_size;
         a.num_pages = paged->num_pages;
         a.sub_rows = sub_rows;
+        auto log2_or = [](int v) {
+            if (v <= 0 || (v & (v - 1))) return -1;
+            int l = 0;
+            while ((1 << l) < v) ++l;
+            return l;
+        };
+        a.sub_shift = log2_or(sub_rows);
+        a.page_shift = log2_or(paged->page_size);
         a.sub_k_bytes = (uint32_t)sub_rows * d->d_k * 2;
         a.sub_v_bytes = (uint32_t)sub_rows * plan.v_heads_per_tile * d->d_v * 2;
     }
