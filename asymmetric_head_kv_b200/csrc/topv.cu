@@ -37,11 +37,10 @@
 //     and the rest (usually a handful) get exact keys -- an integer
 //     superaccumulator of the products -- and the remaining slots go to the
 //     largest exact keys, the lower position first.  Kept positions are written
-//     in ascending order with their scores; a flag S marks the row done.
-//  4. Gather.  Every CTA of the unit takes an equal share of every row's kept
-//     list, once the rows' flags are set: the weighted sum of those V rows and
-//     of the weights.  The last part to arrive (a counter) adds the parts in
-//     part order and writes the output, so the result does not depend on timing.
+//     in ascending order with their scores.
+//  4. Gather, by the same CTA: the weighted sum of the row's kept V rows and of
+//     the weights, the warps' sums added in warp order (so the result does not
+//     depend on timing), and the output.
 // Every wait on another CTA is bounded (globaltimer): a wait that runs out
 // records DIFFQKV_ERR_DEVICE_TIMEOUT and the CTA returns.  The counters and
 // histograms clean themselves up (the last user of each resets it), so the
@@ -86,9 +85,9 @@ constexpr int kMaxStages = 12;
 constexpr int kTableAhead = 4;           // paged producer: tiles whose block-table entries are in flight
 constexpr int kTableRing = 8;            // rows of the entry ring (> kTableAhead)
 constexpr int kRowInfoWords = 8;
-enum RowInfo { kRiBucket = 0, kRiAbove = 1, kRiTwoDelta = 2, kRiMax = 3, kRiKept = 4, kRiFullSum = 5 };
-enum UnitSync { kUsHist = 0, kUsCand = 1, kUsKmax = 3 };
-enum RowSync { kRsSelected = 0, kRsGathered = 1, kRsCand = 2 };
+enum RowInfo { kRiBucket = 0, kRiAbove = 1, kRiTwoDelta = 2 };
+enum UnitSync { kUsHist = 0, kUsCand = 1, kUsDone = 2, kUsKmax = 3 };
+enum RowSync { kRsCand = 2 };  // (words 0, 1 and 3 of a row's four are unused)
 constexpr int kDynSmemCap = 219 * 1024;  // dynamic shared memory (the static part needs the rest of 227 KB)
 
 struct TopvArgs {
@@ -106,7 +105,6 @@ struct TopvArgs {
     // written and read within a call
     uint32_t *rowinfo;    // [rows][8]
     float2 *chunk_part;   // [rows][kMaxParts]: (max score, sum of 2^((s - max) scale log2 e)) of a part
-    float *gpart;         // [rows][kMaxParts][d_v + 4]: gathered sums of a part, weight sum at d_v
     int32_t *cand_j;      // [rows][t_pad]
     float *cand_s;        // [rows][t_pad]
     float *kept_s;        // [rows][k_pad]: scores of the kept positions, in idx_out order
@@ -183,21 +181,11 @@ __device__ __forceinline__ uint32_t ld_acquire(const uint32_t *p) {
     return v;
 }
 
-// Release operations at GPU scope.  After a __syncthreads, one of them by thread 0
-// publishes every write the CTA made before it (release is cumulative over the
-// writes the barrier ordered before it); a reader's ld.acquire of the value, a
-// __syncthreads, and L2 loads see them all.
+// Release add at GPU scope.  After a __syncthreads, one by thread 0 publishes every write the CTA
+// made before it (release is cumulative over the writes the barrier ordered before it); a
+// reader's ld.acquire of the value, a __syncthreads, and L2 loads see them all.
 __device__ __forceinline__ void red_release_add(uint32_t *p, uint32_t v) {
     asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-__device__ __forceinline__ void st_release(uint32_t *p, uint32_t v) {
-    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-// Add with acquire and release semantics; returns the old value.
-__device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t *p, uint32_t v) {
-    uint32_t old;
-    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
-    return old;
 }
 
 // Thread 0 waits, for at most limit_ns, until *ctr >= target; false when the wait ran out
@@ -474,14 +462,12 @@ struct Shared {
     uint16_t qbits[128];
     uint32_t keys[kPairwiseMax][kKeyWords];
     int32_t alist[kPairwiseMax];
-    int combine[16];        // rows whose output this CTA writes after the gather
     uint32_t emit_total[16];
     uint32_t emit_base[16];
     int32_t table[kTableRing][32];  // paged producer: block-table entries of tile t in row t % kTableRing
+    float sel_m, sel_full;          // the selected row's weight maximum and full softmax sum (0: renormalise)
+    int sel_n;                      // its kept positions
     uint32_t tmem_base;             // the score buffers' TMEM address
-    float row_m[16];
-    int row_nsel[16];
-    float row_full[16];
 };
 
 // K tensor maps: m[0] has kTile-row boxes over a contiguous cache; over a paged pool m[i] has
@@ -1206,62 +1192,55 @@ __global__ void __launch_bounds__(kThreads, 1)
                     m = M;
                 }
                 if (T == 0) m = 0.f;
-                a.rowinfo[kRowInfoWords * row + kRiMax] = __float_as_uint(m);
-                a.rowinfo[kRowInfoWords * row + kRiKept] = (uint32_t)nsel;
-                a.rowinfo[kRowInfoWords * row + kRiFullSum] = __float_as_uint(full_sum);
+                sh.sel_m = m;
+                sh.sel_n = nsel;
+                sh.sel_full = full_sum;
                 a.row_sync[(size_t)row * 4 + kRsCand] = 0u;
-                st_release(a.row_sync + (size_t)row * 4 + kRsSelected, 1u);  // after the idx / score writes
             }
             __syncthreads();
-        }
 
-        // =============================================================== 4. gather
-        if (tid == 0) *flag = 1;
-        __syncthreads();
-        // thread hh waits for row hh's selection (the rows in parallel) and reads what the select wrote
-        if (tid < QPK) {
-            const int row = row0 + tid;
-            if (wait_at_least(a.row_sync + (size_t)row * 4 + kRsSelected, 1u, a)) {
-                sh.row_m[tid] = __uint_as_float(__ldcg(a.rowinfo + kRowInfoWords * row + kRiMax));
-                sh.row_nsel[tid] = (int)__ldcg(a.rowinfo + kRowInfoWords * row + kRiKept);
-                sh.row_full[tid] = __uint_as_float(__ldcg(a.rowinfo + kRowInfoWords * row + kRiFullSum));
-            } else {
-                *flag = 0;
-            }
-        }
-        __syncthreads();
-        if (!*flag) goto finish;
-        {
-            constexpr int WPR = kWarps / QPK;          // warps per row (every warp gathers)
-            constexpr int CPV = DV / 8;                // lanes per V row
-            constexpr int RPW = 32 / CPV;              // V rows per warp step
-            constexpr int GU = 16;                     // V rows in flight per lane
-            float *o_s = reinterpret_cast<float *>(overlay);  // [kWarps][DV + 4]
-            const int vc = lane % CPV, vs = lane / CPV;
+            // ---- e. gather: this CTA sums the row's kept V rows itself (16 in flight per lane), the
+            //         weights 2^((s_j - m) scale log2 e), and writes the output.  The warps' sums are
+            //         added in warp order, so the result does not depend on timing.
             {
-                const int hh = warp / WPR, wi = warp % WPR;
-                const int row = row0 + hh;
+                constexpr int CPV = DV / 8;  // lanes per V row
+                constexpr int RPW = 32 / CPV;  // V rows per warp step
+                constexpr int GU = 16;         // V rows in flight per lane
+                const int vc = lane % CPV, vs = lane / CPV;
                 const int vh = (g * QPK + hh) / a.q_per_v;
-                const int nsel = sh.row_nsel[hh];
-                const float m = sh.row_m[hh];
-                const int i_begin = (int)(((long long)nsel * j) / Y), i_end = (int)(((long long)nsel * (j + 1)) / Y);
-                const float *ks = a.kept_s + (size_t)row * a.k_pad;
-                const int32_t *kr = a.kept_row + (size_t)row * a.k_pad;
+                const float m = sh.sel_m;
+                const int ns = sh.sel_n;
                 const __nv_bfloat16 *vbase = a.v + (size_t)vh * DV + vc * 8;
+                // the kept list (cache rows, scores) into shared memory in one round trip, past the
+                // warps' partial sums, when it fits (the V loads below then wait on nothing else)
+                float *o_s = reinterpret_cast<float *>(overlay);  // [kWarps][DV + 4] (the select is done with it)
+                int32_t *kr_s = reinterpret_cast<int32_t *>(o_s + kWarps * (DV + 4));
+                float *ks_s = reinterpret_cast<float *>(kr_s + ns);
+                const bool kept_in_smem =
+                    (size_t)kWarps * (DV + 4) * 4 + (size_t)ns * 8 <= (size_t)a.stages * kTile * DK * 2;
+                if (kept_in_smem) {
+                    for (int i = tid; i < ns; i += kThreads) {
+                        kr_s[i] = __ldcg(kr + i);
+                        ks_s[i] = __ldcg(ks + i);
+                    }
+                    __syncthreads();
+                }
+                const int32_t *krp = kept_in_smem ? kr_s : kr;
+                const float *ksp = kept_in_smem ? ks_s : ks;
                 const size_t vstride = (size_t)a.n_v * DV;
                 float o[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) o[e] = 0.f;
                 float l = 0.f;
-                for (int i0 = i_begin + wi * RPW + vs; i0 < i_end; i0 += WPR * RPW * GU) {
+                for (int i0 = warp * RPW + vs; i0 < ns; i0 += kWarps * RPW * GU) {
                     int jj[GU];
                     float sx[GU];
 #pragma unroll
                     for (int uu = 0; uu < GU; ++uu) {
-                        const int i = i0 + uu * WPR * RPW;
-                        jj[uu] = i < i_end ? __ldcg(kr + i) : -1;  // the kept position's cache row
+                        const int i = i0 + uu * kWarps * RPW;
+                        jj[uu] = i < ns ? (kept_in_smem ? krp[i] : __ldcg(krp + i)) : -1;  // the cache row
                         if (jj[uu] >= 0 && !in_bounds(jj[uu], a.cache_rows, a.status)) jj[uu] = -1;
-                        sx[uu] = i < i_end ? __ldcg(ks + i) : -INFINITY;
+                        sx[uu] = i < ns ? (kept_in_smem ? ksp[i] : __ldcg(ksp + i)) : -INFINITY;
                     }
                     uint4 vv[GU];
 #pragma unroll
@@ -1290,50 +1269,32 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int e = 0; e < 8; ++e) dst[vc * 8 + e] = o[e];
                 }
                 if (lane == 0) dst[DV] = l;
-            }
-            __syncthreads();
-            // this part's sums of every row, the warps of a row added in order
-            for (int c = tid; c < QPK * (DV + 1); c += kThreads) {
-                const int hh = c / (DV + 1), e = c % (DV + 1);
-                float acc = 0.f;
-                for (int w = 0; w < WPR; ++w) acc += o_s[(hh * WPR + w) * (DV + 4) + e];
-                __stcg(a.gpart + ((size_t)(row0 + hh) * kMaxParts + j) * (DV + 4) + e, acc);
-            }
-            __syncthreads();
-            if (tid < QPK) {
-                // thread hh releases this part's sums of row hh (release is cumulative over the whole
-                // CTA's writes the barrier ordered before it); the last part also acquires every other's
-                sh.combine[tid] =
-                    atom_add_acq_rel(a.row_sync + (size_t)(row0 + tid) * 4 + kRsGathered, 1u) == (uint32_t)Y - 1;
-            }
-            __syncthreads();
-            // the last part of a row adds the Y parts in part order and writes the output
-            for (int hh = 0; hh < QPK; ++hh) {
-                if (!sh.combine[hh]) continue;
-                const int row = row0 + hh;
-                const float *gp = a.gpart + (size_t)row * kMaxParts * (DV + 4);
-                float lt = 0.f;
-                for (int p = 0; p < Y; ++p) lt += __ldcg(gp + (size_t)p * (DV + 4) + DV);
-                if (sh.row_full[hh] > 0.f) lt = sh.row_full[hh];
+                __syncthreads();
                 for (int c = tid; c < DV; c += kThreads) {
-                    float acc = 0.f;
-                    for (int p = 0; p < Y; ++p) acc += __ldcg(gp + (size_t)p * (DV + 4) + c);
+                    float acc = 0.f, lt = 0.f;
+                    for (int w = 0; w < kWarps; ++w) {
+                        acc += o_s[w * (DV + 4) + c];
+                        lt += o_s[w * (DV + 4) + DV];
+                    }
+                    if (sh.sel_full > 0.f) lt = sh.sel_full;
                     if (in_bounds(row, (long long)a.batch * a.n_q, a.status))
                         a.out[(size_t)row * DV + c] = __float2bfloat16(lt > 0.f ? acc / lt : 0.f);
                 }
                 if (tid == 0) {
-                    // every part of the row has passed its wait on the flag; and since every part of the
-                    // unit waited for every row of the group to be selected, every wait on the unit's
-                    // counters (H by all parts, C by the select CTAs) is over: reset them too
-                    a.row_sync[(size_t)row * 4 + kRsGathered] = 0u;
-                    a.row_sync[(size_t)row * 4 + kRsSelected] = 0u;
-                    usync[kUsHist] = 0u;
-                    usync[kUsCand] = 0u;
-                    usync[kUsKmax] = 0u;
+                    // every select of the unit has passed its wait on C once all of them counted
+                    // themselves here, and every part read H and max |k| before it arrived on C: the
+                    // last one resets the unit's counters for the next call
+                    if (atomicAdd(usync + kUsDone, 1u) == (uint32_t)QPK - 1) {
+                        usync[kUsHist] = 0u;
+                        usync[kUsCand] = 0u;
+                        usync[kUsKmax] = 0u;
+                        usync[kUsDone] = 0u;
+                    }
                 }
+                __syncthreads();  // o_s and the smem state are reused by the next row
             }
-            __syncthreads();
         }
+
     }
 finish:
     // the tensor memory goes back once no MMA is in flight (every exit of the loop above is taken by
@@ -1440,7 +1401,7 @@ size_t topv_workspace_size(const diffqkv_dims_t *d, int32_t t_max, int32_t topk)
     const size_t rows = (size_t)d->batch * d->n_q;
     const size_t per = padded_len(t_max);
     return kTopvHeader + align_up(zeroed_bytes(d), 256) + align_up(rows * kRowInfoWords * 4, 256) +
-           align_up(rows * kMaxParts * sizeof(float2), 256) + align_up(rows * kMaxParts * (d->d_v + 4) * 4, 256) +
+           align_up(rows * kMaxParts * sizeof(float2), 256) +
            align_up(rows * per * 4, 256) * 3 + align_up(rows * padded_k(topk) * 4, 256) * 2 +
            align_up(rows * per, 256) * 2;
 }
@@ -1498,8 +1459,6 @@ diffqkv_status_t topv_launch(const diffqkv_dims_t *d, const void *q, const void 
     ws += align_up(rows * kRowInfoWords * 4, 256);
     a.chunk_part = reinterpret_cast<float2 *>(ws);
     ws += align_up(rows * kMaxParts * sizeof(float2), 256);
-    a.gpart = reinterpret_cast<float *>(ws);
-    ws += align_up(rows * kMaxParts * (d->d_v + 4) * 4, 256);
     a.cand_j = reinterpret_cast<int32_t *>(ws);
     ws += align_up(rows * t_pad * 4, 256);
     a.cand_s = reinterpret_cast<float *>(ws);

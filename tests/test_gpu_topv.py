@@ -214,7 +214,7 @@ def _candidate_lists(ws, batch, n_q, n_k, d_v, t_max):
     """Views of the workspace's candidate positions and scores ([rows][t_pad] each; the header's layout)."""
     rows, units, t_pad = batch * n_q, batch * n_k, -(-t_max // 64) * 64
     off = 256 + _a256(_a256(units * 16) + _a256(rows * 16) + rows * 2048 * 4)
-    off += _a256(rows * 8 * 4) + _a256(rows * 256 * 8) + _a256(rows * 256 * (d_v + 4) * 4)
+    off += _a256(rows * 8 * 4) + _a256(rows * 256 * 8)
     cj = ws[off:off + rows * t_pad * 4].view(torch.int32).view(rows, t_pad)
     off += _a256(rows * t_pad * 4)
     cs = ws[off:off + rows * t_pad * 4].view(torch.float32).view(rows, t_pad)
