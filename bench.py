@@ -447,6 +447,7 @@ def time_paths(ak, peaks, steps: int, warmup: int):
     tf = flops / (ms * 1e-3) / 1e12
     res["prefill_prefix_b2_p8192_s2048"] = {"ms": ms, "causal_flops": flops, "tflops": tf, "bound": "tensor",
                                             "peak_tflops": bf16_peak, "frac": tf / bf16_peak,
+                                            "frac_kind": "FLOP-derived tensor fraction",
                                             "peak_source": "bf16_tflops (burst, cuBLAS bf16 GEMM)"}
     # the same chunked prefill with K and V in 16-position pages dealt out in random order
     page = 16
@@ -465,7 +466,8 @@ def time_paths(ak, peaks, steps: int, warmup: int):
     tf = flops / (ms * 1e-3) / 1e12
     res["prefill_prefix_paged_b2_p8192_s2048_page16"] = {
         "ms": ms, "causal_flops": flops, "tflops": tf, "bound": "tensor", "peak_tflops": bf16_peak,
-        "frac": tf / bf16_peak, "peak_source": "bf16_tflops (burst, cuBLAS bf16 GEMM)"}
+        "frac": tf / bf16_peak, "frac_kind": "FLOP-derived tensor fraction",
+        "peak_source": "bf16_tflops (burst, cuBLAS bf16 GEMM)"}
     assert ak.device_status() == 0
     del d, qn, out, kp, vp, table
 
