@@ -466,6 +466,8 @@ struct Shared {
     uint32_t emit_base[16];
     int32_t table[kTableRing][32];  // paged producer: block-table entries of tile t in row t % kTableRing
     float sel_m, sel_full;          // the selected row's weight maximum and full softmax sum (0: renormalise)
+    int small_n;                    // select: candidates left after the first radix pass (when few)
+    uint32_t small_keys[32], small_tau;
     int sel_n;                      // its kept positions
     uint32_t tmem_base;             // the score buffers' TMEM address
 };
@@ -1025,6 +1027,36 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int pass = 0; pass < 2; ++pass) {
                     const int shift = pass == 0 ? 10 : 0;
                     const int nb = pass == 0 ? kHistBuckets : kRadixBuckets;
+                    if (pass == 1 && hist[sh.sh_d] <= 32u) {
+                        // at most 32 candidates share the first 22 key bits: warp 0 ranks their keys
+                        // directly (the kk-th largest, ties counted in slot order) instead of a
+                        // block-wide histogram pass over the last 10 bits
+                        if (tid == 0) sh.small_n = 0;
+                        __syncthreads();
+                        for (uint32_t i = tid; i < nc; i += kThreads) {
+                            const uint32_t key = float_key(cs[i]);
+                            if ((key & pmask) == prefix) {
+                                const int sl = atomicAdd(&sh.small_n, 1);
+                                if (sl < 32) sh.small_keys[sl] = key;
+                            }
+                        }
+                        __syncthreads();
+                        if (warp == 0) {
+                            const int n = min(sh.small_n, 32);
+                            const uint32_t my = lane < n ? sh.small_keys[lane] : 0u;
+                            int greater = 0;
+                            for (int jl = 0; jl < n; ++jl) {
+                                const uint32_t kj = __shfl_sync(0xffffffffu, my, jl);
+                                greater += (kj > my || (kj == my && jl < lane)) ? 1 : 0;
+                            }
+                            const unsigned hit = __ballot_sync(0xffffffffu, lane < n && greater == (int)kk - 1);
+                            const uint32_t tkey = __shfl_sync(0xffffffffu, my, hit ? __ffs(hit) - 1 : 0);
+                            if (lane == 0) sh.small_tau = hit ? tkey : prefix;
+                        }
+                        __syncthreads();
+                        prefix = sh.small_tau;
+                        break;
+                    }
                     for (int i = tid; i < nb; i += kThreads) hist[i] = 0;
                     __syncthreads();
                     for (uint32_t base_i = 0; base_i < nc; base_i += kThreads) {
