@@ -89,7 +89,7 @@ __device__ __noinline__ void paged_kv_producer(const PagedMaps &pm, const Prefil
     auto fetch = [&](int t) {
         if (t < n_kv) {
             const int last = min(a.n_pages - 1, pdiv(t * BN + BN - 1));
-            if (lane <= last - first_page(t)) {
+            if (lane <= last - first_page(t) && in_bounds(first_page(t) + lane, a.max_blocks, a.status)) {
                 const int32_t *src = a.block_table + (size_t)b * a.max_blocks + first_page(t) + lane;
                 asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_addr(&table[t % kPgTableRing][lane])),
                              "l"(src)

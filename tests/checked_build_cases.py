@@ -17,7 +17,7 @@ import asymmetric_head_kv_b200 as ak  # noqa: E402
 from asymmetric_head_kv_b200 import _capi  # noqa: E402
 import oracle  # noqa: E402
 import workloads as wl  # noqa: E402
-from parity import assert_parity, assert_parity_prefill  # noqa: E402
+from parity import assert_parity, assert_parity_gemm, assert_parity_prefill  # noqa: E402
 
 
 def to(d, dev):
@@ -66,10 +66,10 @@ def main():
     assert np.array_equal(idx.cpu().numpy(), r_idx)
     assert_parity(out, r_out, "checked paged top-v")
     print("paged decode and paged selective V ok")
-    # selective V: lengths around the 120-position tile
-    t = wl.random_decode_inputs(4, 250, s, seed=75, seq_lens=[119, 120, 121, 250])
+    # selective V: lengths around the 128-position tile
+    t = wl.random_decode_inputs(4, 300, s, seed=75, seq_lens=[127, 128, 129, 300])
     gt = to(t, dev)
-    tws = ak.decode_topv_workspace(ak.make_dims(4, 16, 4, 16, 64, 128, t["scale"]), 250, 100, dev)
+    tws = ak.decode_topv_workspace(ak.make_dims(4, 16, 4, 16, 64, 128, t["scale"]), 300, 100, dev)
     out, idx = ak.decode_topv(gt["q"], gt["k_cache"], gt["v_cache"], gt["seq_lens"], 100, scale=t["scale"],
                               workspace=tws)
     assert ak.workspace_status(tws) == 0
@@ -87,6 +87,34 @@ def main():
         assert int(word.item()) == 0
         assert_parity_prefill(out, oracle.prefill_causal(pr["q"], pr["k"], pr["v"], pr["scale"]), "checked prefill")
     print("prefill ok")
+    # prefill over paged pools (16-position pages) and a prefix
+    pr = wl.random_prefill_inputs(2, 300, wl.DIFFQKV, seed=77)
+    per = -(-300 // 16)
+    perm = torch.randperm(2 * per, generator=torch.Generator().manual_seed(78)).to(torch.int32).view(2, per)
+    kp = torch.zeros((2 * per, 16, s.n_k, s.d_k), dtype=torch.bfloat16)
+    vp = torch.zeros((2 * per, 16, s.n_v, s.d_v), dtype=torch.bfloat16)
+    for b in range(2):
+        for pg in range(per):
+            n = min(16, 300 - pg * 16)
+            kp[perm[b, pg], :n] = pr["k"][b, pg * 16:pg * 16 + n]
+            vp[perm[b, pg], :n] = pr["v"][b, pg * 16:pg * 16 + n]
+    word = torch.zeros(1, dtype=torch.int32, device=dev)
+    out = ak.prefill_causal_paged(pr["q"][:, 100:].contiguous().to(dev), kp.to(dev), vp.to(dev), perm.to(dev), 100,
+                                  scale=pr["scale"], status=word)
+    torch.cuda.synchronize()
+    assert int(word.item()) == 0
+    assert_parity_prefill(out, oracle.prefill_causal(pr["q"], pr["k"], pr["v"], pr["scale"])[:, 100:],
+                          "checked paged prefill")
+    print("paged prefill ok")
+    # augmented query projection: a token tail and a partial output tile
+    a = wl.random_augq_inputs(300, 256, 384, 160, seed=79)
+    word = torch.zeros(1, dtype=torch.int32, device=dev)
+    q, h = ak.augq_project(*(a[k].to(dev) for k in ("x", "w_gate", "w_up", "w_down")), status=word)
+    torch.cuda.synchronize()
+    assert int(word.item()) == 0
+    assert_parity_gemm(h, oracle.augq_hidden(a["x"], a["w_gate"], a["w_up"]), "checked augmented Q: h")
+    assert_parity_gemm(q, oracle.augq_down(h.cpu().double().numpy(), a["w_down"]), "checked augmented Q: q")
+    print("augmented query projection ok")
     print("all cases ok")
 
 
