@@ -82,13 +82,12 @@ constexpr int kTopvHeader = 256;
 constexpr int kTopvMaxContext = 131072;  // bitmap of kept positions
 constexpr int kMaxParts = 256;           // CTAs per unit (sizes the per-part records)
 constexpr int kMaxStages = 12;
-constexpr int kTableAhead = 4;           // paged producer: tiles whose block-table entries are in flight
-constexpr int kTableRing = 8;            // rows of the entry ring (> kTableAhead)
+constexpr int kTableWin = 512;           // paged producer: block-table entries held in shared memory
 constexpr int kRowInfoWords = 8;
 enum RowInfo { kRiBucket = 0, kRiAbove = 1, kRiTwoDelta = 2 };
 enum UnitSync { kUsHist = 0, kUsCand = 1, kUsDone = 2, kUsKmax = 3 };
 enum RowSync { kRsCand = 2 };  // (words 0, 1 and 3 of a row's four are unused)
-constexpr int kDynSmemCap = 219 * 1024;  // dynamic shared memory (the static part needs the rest of 227 KB)
+constexpr int kDynSmemCap = 218 * 1024;  // dynamic shared memory (the static part needs the rest of 227 KB)
 
 struct TopvArgs {
     const __nv_bfloat16 *q;
@@ -464,7 +463,7 @@ struct Shared {
     int32_t alist[kPairwiseMax];
     uint32_t emit_total[16];
     uint32_t emit_base[16];
-    int32_t table[kTableRing][32];  // paged producer: block-table entries of tile t in row t % kTableRing
+    int32_t table[kTableWin];       // paged producer: block-table entries of pages tbl0 .. tbl0 + kTableWin - 1
     float sel_m, sel_full;          // the selected row's weight maximum and full softmax sum (0: renormalise)
     int small_n;                    // select: candidates left after the first radix pass (when few)
     uint32_t small_keys[32], small_tau;
@@ -582,11 +581,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             //      aligned boxes of 8, 16, 32 or 64 rows (heights that divide the page, so a box never
             //      leaves its page), or by one whole-tile box when the page size is a multiple of the
             //      tile; lane f issues box f, so a tile's boxes leave as one warp instruction (one lane
-            //      issuing them all measured slower).  The tile's block-table entries (one page per
-            //      lane) reach shared memory by asynchronous copies issued kTableAhead tiles ahead (a
-            //      register copy of a pending load would wait for it at once); an entry is checked when
-            //      a box uses it.  Only pages holding cached positions are read (later entries may hold
-            //      anything); rows past the sequence inside a loaded box are harmless.
+            //      issuing them all measured slower).  The block-table entries sit in shared memory, a
+            //      window of kTableWin pages loaded at once; an entry is checked when a box uses it.
+            //      Only pages holding cached positions are read (later entries may hold anything);
+            //      rows past the sequence inside a loaded box are harmless.
             if (te > tb) {
                 if (lane == 0) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 __syncwarp();
@@ -598,30 +596,28 @@ __global__ void __launch_bounds__(kThreads, 1)
                 auto pdiv = [&](int x) { return ps >= 0 ? x >> ps : x / a.page_size; };
                 auto pmod = [&](int x) { return ps >= 0 ? x & (a.page_size - 1) : x % a.page_size; };
                 auto first_page = [&](int t) { return pdiv(t * kTile); };
-                auto fetch = [&](int t) {
-                    if (t < te) {
-                        const int np = pdiv(t * kTile + covered(t) - 1) - first_page(t) + 1;
-                        if (lane < np) {
-                            const int32_t *src = a.block_table + (size_t)b * a.max_blocks + first_page(t) + lane;
-                            asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(
-                                             smem_addr(&sh.table[t % kTableRing][lane])),
-                                         "l"(src)
-                                         : "memory");
-                        }
-                    }
-                    asm volatile("cp.async.commit_group;" ::: "memory");
-                };
-                for (int i = 0; i < kTableAhead; ++i) fetch(tb + i);
+                // the part's block-table entries, a window of kTableWin pages at a time, loaded into
+                // shared memory by the whole warp in one round trip (per-tile copies of a few entries
+                // cost this warp more than they saved); entries for pages past the sequence's are
+                // never loaded
+                const int pages_seq = T > 0 ? pdiv(((T + 7) & ~7) - 1) + 1 : 0;
+                int tbl0 = -kTableWin;
                 int st = (int)(k0 % a.stages);
                 uint32_t par = (uint32_t)((k0 / a.stages) & 1);
                 bool wrapped = k0 >= a.stages;
                 long long issued_end = k0;
                 for (int t = tb; t < te; ++t) {
-                    fetch(t + kTableAhead);
+                    const int last_page = pdiv(t * kTile + covered(t) - 1);
+                    if (last_page >= tbl0 + kTableWin) {  // (the same decision in every lane)
+                        tbl0 = first_page(t);
+                        const int cnt = min(kTableWin, pages_seq - tbl0);
+                        __syncwarp();
+                        for (int i = lane; i < cnt; i += 32)
+                            sh.table[i] = __ldg(a.block_table + (size_t)b * a.max_blocks + tbl0 + i);
+                        __syncwarp();
+                    }
                     if (wrapped) mbar_wait_bounded(&empty_bar[st], par ^ 1u, a.wait_limit_ns, abort_flag, a.status);
                     if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
-                    asm volatile("cp.async.wait_group %0;" ::"n"(kTableAhead) : "memory");  // tile t's entries
-                    const int cur_e = sh.table[t % kTableRing][lane];  // this lane's own copy
                     const int start = t * kTile, end = start + (a.tile_box ? kTile : covered(t));
                     int cur = a.tile_box ? end : start, f = 0, my_cur = -1, my_hi = 0;
                     if (a.tile_box && lane == 0) my_cur = start;
@@ -648,8 +644,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     uint8_t *dst = ring + (size_t)st * TILE_BYTES;
                     if (lane == 0) mbar_arrive_expect_tx(&full_bar[st], (uint32_t)((end - start) * DK * 2));
                     __syncwarp();
-                    int page = __shfl_sync(0xffffffffu, cur_e, my_cur >= 0 ? pdiv(my_cur) - first_page(t) : 0);
                     if (my_cur >= 0) {
+                        int page = sh.table[pdiv(my_cur) - tbl0];
                         if (page < 0 || page >= a.num_pages) {  // flagged; pool page 0 read in its place
                             record_error(a.status, DIFFQKV_ERR_DEVICE_PAGE);
                             page = 0;
@@ -671,7 +667,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                         wrapped = true;
                     }
                 }
-                asm volatile("cp.async.wait_all;" ::: "memory");  // no entry copy outlives the loop
                 if (lane == 0)
                     for (long long kk = (issued_end - a.stages > k0 ? issued_end - a.stages : k0); kk < issued_end; ++kk)
                         mbar_wait_bounded(&full_bar[kk % a.stages], (uint32_t)((kk / a.stages) & 1), a.wait_limit_ns,
