@@ -55,8 +55,7 @@ struct PrefillArgs {
     int32_t page_shift;   // log2(page_size) when it is a power of two, else -1
 };
 
-constexpr int kPgTableAhead = 4;  // paged producer: tiles whose block-table entries are in flight
-constexpr int kPgTableRing = 8;   // rows of the entry ring (> kPgTableAhead)
+constexpr int kPgTableWin = 512;  // paged producer: block-table entries held in shared memory
 
 // K and V tensor maps of paged pools: k[i] / v[i] have (8 << i)-row boxes over the whole pool;
 // k_tail[i] / v_tail[i] the same boxes over a view of the pool whose pages hold only the rows of
@@ -72,12 +71,13 @@ struct PagedMaps {
 // rows, then V: VB blocks).  The tile's rows are covered greedily by aligned boxes of 8 << i rows
 // that stay inside one page; lane f issues box f.  Boxes in the sequence's last page use the tail
 // maps; boxes past it use a tail map at a row past its extent (all zeros).  The block-table
-// entries of a tile reach shared memory by asynchronous copies kPgTableAhead tiles ahead; an
-// entry outside [0, num_pages) is flagged DIFFQKV_ERR_DEVICE_PAGE and pool page 0 read instead.
+// entries sit in shared memory, a window of kPgTableWin pages loaded by the warp in one round
+// trip; an entry outside [0, num_pages) is flagged DIFFQKV_ERR_DEVICE_PAGE and pool page 0 read
+// instead.
 template <int BN, int KB, int VB, int STAGES, int STAGE_BYTES, int K_BYTES>
 __device__ __noinline__ void paged_kv_producer(const PagedMaps &pm, const PrefillArgs &a, int b, int kh, int vh, int n_kv,
                                   uint8_t *kv_base, uint64_t *kv_full, uint64_t *kv_empty,
-                                  int32_t (*table)[32], volatile int *abort_flag, int lane) {
+                                  int32_t *table, volatile int *abort_flag, int lane) {
     const int P = a.page_size;
     const int pend = a.n_pages * P;  // positions the sequence's pages hold
     // position -> page and row in page: shifts for power-of-two pages (a runtime division is dozens
@@ -86,28 +86,23 @@ __device__ __noinline__ void paged_kv_producer(const PagedMaps &pm, const Prefil
     auto pdiv = [&](int x) { return ps >= 0 ? x >> ps : x / P; };
     auto pmod = [&](int x) { return ps >= 0 ? x & (P - 1) : x % P; };
     auto first_page = [&](int t) { return pdiv(t * BN); };
-    auto fetch = [&](int t) {
-        if (t < n_kv) {
-            const int last = min(a.n_pages - 1, pdiv(t * BN + BN - 1));
-            if (lane <= last - first_page(t) && in_bounds(first_page(t) + lane, a.max_blocks, a.status)) {
-                const int32_t *src = a.block_table + (size_t)b * a.max_blocks + first_page(t) + lane;
-                asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_addr(&table[t % kPgTableRing][lane])),
-                             "l"(src)
-                             : "memory");
-            }
-        }
-        asm volatile("cp.async.commit_group;" ::: "memory");
-    };
-    for (int i = 0; i < kPgTableAhead; ++i) fetch(i);
+    int tbl0 = -kPgTableWin;  // pages tbl0 .. tbl0 + kPgTableWin - 1 are in `table`
     int issued = 0;
     for (int n = 0; n < n_kv; ++n) {
-        fetch(n + kPgTableAhead);
+        const int last = min(a.n_pages - 1, pdiv(n * BN + BN - 1));
+        if (last >= tbl0 + kPgTableWin) {  // (the same decision in every lane)
+            tbl0 = first_page(n);
+            const int cnt = min(kPgTableWin, a.n_pages - tbl0);
+            __syncwarp();
+            for (int i = lane; i < cnt; i += 32)
+                if (in_bounds(tbl0 + i, a.max_blocks, a.status))
+                    table[i] = __ldg(a.block_table + (size_t)b * a.max_blocks + tbl0 + i);
+            __syncwarp();
+        }
         const int st = n % STAGES;
         if (n >= STAGES)
             mbar_wait_bounded(&kv_empty[st], (uint32_t)(((n / STAGES) - 1) & 1), a.wait_limit_ns, abort_flag, a.status);
         if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
-        asm volatile("cp.async.wait_group %0;" ::"n"(kPgTableAhead) : "memory");  // tile n's entries
-        const int my_e = table[n % kPgTableRing][lane];
         const int start = n * BN, end = start + BN;
         int my_cur = -1, my_hi = a.max_box_log;
         if (ps >= 0) {
@@ -135,8 +130,8 @@ __device__ __noinline__ void paged_kv_producer(const PagedMaps &pm, const Prefil
         __syncwarp();
         const bool in_seq = my_cur >= 0 && my_cur < pend;
         const int pidx = in_seq ? pdiv(my_cur) : 0;
-        int page = __shfl_sync(0xffffffffu, my_e, in_seq ? pidx - first_page(n) : 0);
         if (my_cur >= 0) {
+            int page = in_seq ? table[pidx - tbl0] : 0;
             int row = P;        // past the sequence's pages: a row past the tail view's extent
             bool tail = true;
             if (in_seq) {
@@ -166,7 +161,6 @@ __device__ __noinline__ void paged_kv_producer(const PagedMaps &pm, const Prefil
         }
         issued = n + 1;
     }
-    asm volatile("cp.async.wait_all;" ::: "memory");  // no entry copy outlives the loop
     // drain: no copy may still be landing when the CTA exits
     if (lane == 0)
         for (int n = (issued > STAGES ? issued - STAGES : 0); n < issued; ++n)
@@ -263,7 +257,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 
     if (warp == kProducerWarp) {
         // ======================= TMA producer
-        __shared__ int32_t pg_table[kPgTableRing][32];  // paged: block-table entries of the tiles ahead
+        __shared__ int32_t pg_table[kPgTableWin];  // paged: a window of block-table entries
         if (lane == 0) {
             prefetch_tensormap(&tm_q);
             mbar_arrive_expect_tx(q_full, C::Q_BYTES);
@@ -583,7 +577,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp == kProducerWarp) {
         // ======================= TMA producer
-        __shared__ int32_t pg_table[kPgTableRing][32];  // paged: block-table entries of the tiles ahead
+        __shared__ int32_t pg_table[kPgTableWin];  // paged: a window of block-table entries
         if (lane == 0) {
             prefetch_tensormap(&tm_q);
             mbar_arrive_expect_tx(q_full, QT * C::Q_BYTES);
