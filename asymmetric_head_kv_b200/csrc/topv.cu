@@ -380,9 +380,10 @@ __device__ void exact_key(const uint16_t *qbits, const uint16_t *kbits, int j, u
 // exact_key computed by a whole warp: lane l takes products l, l + 32, ...; the
 // per-lane digit slots are integers, so summing them across the warp is exact
 // in any order (|slot| < d_k 2^47 <= 2^54).  Only the slots some lane used are
-// summed (the range is warp-uniform); lane 0 normalises and writes.
+// summed (the range is warp-uniform); lane 0 normalises and writes.  Out of line, so that the one
+// copy of its code can be fetched ahead of the select (see the warm-up in phase 1).
 template <int DK>
-__device__ void exact_key_warp(const uint16_t *qbits, const uint16_t *kbits, int j, uint32_t *out, int lane) {
+__device__ __noinline__ void exact_key_warp(const uint16_t *qbits, const uint16_t *kbits, int j, uint32_t *out, int lane) {
     long long acc[18];
 #pragma unroll
     for (int i = 0; i < 18; ++i) acc[i] = 0;
@@ -812,6 +813,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int off = 16; off >= 1; off >>= 1) kmx = max(kmx, __shfl_xor_sync(0xffffffffu, kmx, off));
             if (lane == 0 && kmx) atomicMax(usync + kUsKmax, kmx);
+        } else if (warp == kWarps - 1 && j < QPK && T > K) {
+            // idle in phase 1: run the exact-key code once on a scratch key, so that a select CTA
+            // finds it in the instruction caches instead of fetching it on the critical path
+            exact_key_warp<DK>(sh.qbits, reinterpret_cast<const uint16_t *>(a.k), 0, sh.keys[kPairwiseMax - 1], lane);
         }
         ring_k += te - tb;
         __syncthreads();
