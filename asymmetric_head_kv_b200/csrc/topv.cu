@@ -814,9 +814,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int off = 16; off >= 1; off >>= 1) kmx = max(kmx, __shfl_xor_sync(0xffffffffu, kmx, off));
             if (lane == 0 && kmx) atomicMax(usync + kUsKmax, kmx);
         } else if (warp == kWarps - 1 && j < QPK && T > K) {
-            // idle in phase 1: run the exact-key code once on a scratch key, so that a select CTA
-            // finds it in the instruction caches instead of fetching it on the critical path
-            exact_key_warp<DK>(sh.qbits, reinterpret_cast<const uint16_t *>(a.k), 0, sh.keys[kPairwiseMax - 1], lane);
+            // idle in phase 1: run the exact-key code once on a scratch key (the cache's first K row
+            // against itself), so that a select CTA finds it in the instruction caches instead of
+            // fetching it on the critical path
+            const uint16_t *k0 = reinterpret_cast<const uint16_t *>(a.k);
+            exact_key_warp<DK>(k0, k0, 0, sh.keys[kPairwiseMax - 1], lane);
         }
         ring_k += te - tb;
         __syncthreads();
