@@ -56,6 +56,15 @@ def test_ragged_shapes(cuda_device, name, shape):
     _check(d, 100, cuda_device, name)
 
 
+def test_more_units_than_ctas_run_in_rounds(cuda_device):
+    """40 sequences x 4 K heads = 160 (batch, K head) units: more than one CTA per SM can hold, so one
+    part per unit, each CTA selecting all four rows of its unit, units taken in two rounds (ragged
+    lengths, some at or below k)."""
+    lens = [600, 37, 600, 1, 420, 50, 599, 64] * 5
+    d = wl.random_decode_inputs(len(lens), 600, wl.DIFFQKV, seed=313, seq_lens=lens)
+    _check(d, 50, cuda_device, "160 units in rounds")
+
+
 @pytest.mark.parametrize("topk", [1, 2, 7, 64, 1024, 2999, 3000, 5000])
 def test_topk_sizes(cuda_device, topk):
     d = wl.random_decode_inputs(2, 3000, wl.DIFFQKV, seed=302, seq_lens=[3000, 1500])
