@@ -70,6 +70,26 @@ def test_paged_topv_full_weights_and_large_k(cuda_device):
         assert_parity(out, r_out, f"paged top-v k={topk} full={full}")
 
 
+def test_paged_topv_units_in_rounds(cuda_device):
+    """160 (batch, K head) units over 16-position pages: one part per unit, two rounds; index sets and
+    outputs bit for bit those of the contiguous call over the gathered caches."""
+    shape, page_size = wl.DIFFQKV, 16
+    lens = [600, 37, 600, 1, 420, 50, 599, 64] * 5
+    max_blocks = -(-600 // page_size)
+    d = wl.random_paged_inputs(len(lens), max_blocks, page_size, shape, seed=931, seq_lens=lens)
+    kc = oracle.gather_paged(d["k_pages"], d["block_table"], d["seq_lens"])
+    vc = oracle.gather_paged(d["v_pages"], d["block_table"], d["seq_lens"])
+    r_out, r_idx = oracle.decode_topv(d["q"], kc, vc, d["seq_lens"], 50, d["scale"])
+    g = _to(d, cuda_device)
+    out, idx = _paged(g, d, shape, 50)
+    assert np.array_equal(idx.cpu().numpy(), r_idx), "index sets"
+    assert_parity(out, r_out, "paged top-v in rounds")
+    flat_out, flat_idx = ak.decode_topv(g["q"], kc.to(cuda_device), vc.to(cuda_device), g["seq_lens"], 50,
+                                        scale=d["scale"])
+    torch.cuda.synchronize()
+    assert torch.equal(idx, flat_idx) and torch.equal(out, flat_out), "paged and contiguous top-v differ"
+
+
 def test_paged_topv_bad_entry_is_flagged(cuda_device):
     """A used block-table entry past the pool: flagged DIFFQKV_ERR_DEVICE_PAGE, pool page 0 read in its
     place (every load stays in the pools); the other sequence is unaffected."""
