@@ -52,6 +52,17 @@ def test_shapes_ragged(cuda_device, name):
     assert_parity(out, _oracle(d), name)
 
 
+def test_many_short_sequences(cuda_device):
+    """96 sequences x 4 K heads = 384 (batch, K head) units, more than the CTAs, with ragged lengths
+    from 0 to 700 (empty rows, single positions, tile edges)."""
+    g = torch.Generator().manual_seed(109)
+    lens = torch.randint(0, 701, (96,), generator=g).tolist()
+    lens[:6] = [0, 1, 47, 48, 49, 700]
+    d = wl.random_decode_inputs(len(lens), 700, wl.DIFFQKV, seed=109, seq_lens=lens)
+    out = _run(d, cuda_device)
+    assert_parity(out, _oracle(d), "decode 96 short sequences")
+
+
 @pytest.mark.parametrize("grid", [1, 2, 3, 7, 64, 148, 333, 2048])
 def test_split_points_do_not_change_result(cuda_device, grid):
     """Forcing the split-kernel grid moves every split boundary; the combined result must not move."""

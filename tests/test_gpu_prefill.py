@@ -38,6 +38,16 @@ def test_lengths_diffqkv(cuda_device, seq):
     assert torch.equal(out[:, 0].cpu(), d["v"][:, 0].repeat_interleave(wl.DIFFQKV.n_q // wl.DIFFQKV.n_v, dim=1))
 
 
+@pytest.mark.parametrize("shape_name", ["diffqkv", "gqa"])
+def test_many_sequences(cuda_device, shape_name):
+    """33 sequences of 191 positions: more CTAs than the GPU holds at once in both tilings, each
+    with a ragged last query tile."""
+    s = wl.DIFFQKV if shape_name == "diffqkv" else wl.GQA_CONTROL
+    d = wl.random_prefill_inputs(33, 191, s, seed=480)
+    out = _gpu(d, cuda_device)
+    assert_parity_prefill(out, oracle.prefill_causal(d["q"], d["k"], d["v"], d["scale"]), f"33 x 191 {shape_name}")
+
+
 @pytest.mark.parametrize("name", list(SHAPES))
 def test_shapes(cuda_device, name):
     d = wl.random_prefill_inputs(2, 333, SHAPES[name], seed=410)
